@@ -1,0 +1,26 @@
+"""Plain, slow fp64 CPU oracle of one 4-bit-Muon-GRASP optimizer step.
+
+TEST INFRASTRUCTURE ONLY. Nothing in the product path imports this package:
+only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may use it. It shares no code with the CUDA library; the only
+module both sides use is the seeded input generator
+(``bit_muon_optimizer_b200.workloads``), which holds none of the method's
+arithmetic.
+
+Sources (cited in each function by page and section):
+
+* [GRASP]  "Achieving low-bit Muon through subspace preservation and grid
+  quantization" (ICLR 2026 paper note) -- the step itself.
+* [LiMuon] "LiMuon: Light and Fast Muon Optimizer for Large Models" (paper
+  note) -- the constant quintic Newton-Schulz coefficients.
+* [GramNS] "优化器 (3)（Gram Newton-Schulz）" (blog post on Gram
+  Newton-Schulz) -- standard NS, Algorithms 1 and 2, Proposition 1,
+  Theorem 1.
+
+Every function here is pinned by a ``-m "not gpu"`` test against something
+other than itself (closed forms, brute force, library routines, the pages'
+printed numbers). The end-to-end training quality the pages report needs
+datasets and is "parity unpinned".
+"""
+
+from .grasp import *  # noqa: F401,F403

@@ -1,0 +1,416 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these tests compares the oracle with itself: each checks it against a
+closed form, a theorem of the pages, brute force, a library routine or a
+printed value (fixtures under tests/golden, each with its citation).
+"""
+
+import math
+import os
+
+import pytest
+import torch
+
+import oracle as O
+from bit_muon_optimizer_b200 import flops as F
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+DT = torch.float64
+
+
+def _orthogonal(n, gen):
+    q, r = torch.linalg.qr(torch.randn(n, n, generator=gen, dtype=DT))
+    return q * torch.sign(torch.diagonal(r))
+
+
+def _read_sections(path):
+    sec, out = None, {}
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        if line.startswith("["):
+            sec = line.strip("[]")
+            out[sec] = []
+            continue
+        out[sec].append(line.split())
+    return out
+
+
+# ---------------------------------------------------------------- generator
+
+def test_splitmix64_published_stream():
+    vals = []
+    for line in open(os.path.join(GOLDEN, "splitmix64_seed0.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        i, v = line.split()
+        vals.append((int(i), int(v, 16)))
+    golden = 0x9E3779B97F4A7C15
+    for i, v in vals:
+        # splitmix64(x) adds the increment itself: counter (i-1)*golden gives output i
+        assert O.splitmix64(((i - 1) * golden) & ((1 << 64) - 1)) == v
+
+
+def test_rademacher_column_is_pm_one_over_sqrt_n_and_balanced():
+    col = O.rademacher_column(1234, 3, 4096, 5)
+    assert torch.all(torch.isclose(col.abs(), torch.full_like(col, 1 / 64.0)))
+    frac_pos = float((col > 0).double().mean())
+    assert 0.45 < frac_pos < 0.55
+    assert float(col @ col) == pytest.approx(1.0, abs=1e-12)
+    other = O.rademacher_column(1234, 3, 4096, 6)
+    assert abs(float(col @ other)) < 0.1       # different counters -> different signs
+
+
+# ---------------------------------------------------------- NS coefficients
+
+def test_quintic_coefficients_match_printed_values():
+    d = {}
+    for line in open(os.path.join(GOLDEN, "ns_coefficients.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        k, v = line.split()
+        d[k] = float(v)
+    assert O.QUINTIC_ABC == (d["a"], d["b"], d["c"])
+
+
+# ------------------------------------------------------ Proposition 1 (NS)
+
+@pytest.mark.parametrize("m,n", [(6, 10), (24, 40), (40, 24), (32, 32)])
+def test_ns_standard_proposition1_singular_vectors_kept(m, n):
+    """NS(U S V^T) = U f(S) V^T, f the scalar composition [GramNS Prop. 1]."""
+    gen = torch.Generator().manual_seed(7 + m * n)
+    r = min(m, n)
+    U = _orthogonal(m, gen)[:, :r]
+    V = _orthogonal(n, gen)[:, :r]
+    # sigma in [2e-3, 1] with |X|_F = 1: the top value absorbs the remaining norm
+    rest = torch.logspace(math.log10(2e-3), math.log10(0.15), r - 1, dtype=DT)
+    s = torch.cat([torch.sqrt(1 - (rest * rest).sum()).reshape(1), rest.flip(0)])
+    X = U @ torch.diag(s) @ V.T
+    out = O.ns_standard(X)
+    scale = 1.0 / (1.0 + O.NS_EPS)
+    fs = torch.tensor([O.quintic_scalar(float(v) * scale) for v in s], dtype=DT)
+    expect = U @ torch.diag(fs) @ V.T
+    assert torch.allclose(out, expect, atol=1e-10, rtol=0)
+    sv = torch.linalg.svdvals(out)
+    assert float(sv.min()) >= 0.6818 - 1e-4
+    assert float(sv.max()) <= 1.2024 + 1e-4
+
+
+def test_quintic_band_closed_form():
+    """Scalar composition over [2e-3, 1] stays inside [0.6818, 1.2024]; f(1) = 0.6964."""
+    xs = torch.linspace(2e-3, 1.0, 200001, dtype=DT)
+    y = xs.clone()
+    for a, b, c in [O.QUINTIC_ABC] * 5:
+        y = a * y + b * y ** 3 + c * y ** 5
+    assert 0.6818 <= float(y.min()) < 0.6819
+    assert 1.2023 < float(y.max()) <= 1.2024
+    assert O.quintic_scalar(1.0) == pytest.approx(0.6964, abs=1e-4)
+
+
+def test_ns_standard_transpose_rule():
+    gen = torch.Generator().manual_seed(3)
+    X = torch.randn(12, 30, generator=gen, dtype=DT)
+    assert torch.allclose(O.ns_standard(X.T), O.ns_standard(X).T, atol=1e-13)
+
+
+# -------------------------------------------------------- Theorem 1 (Gram NS)
+
+@pytest.mark.parametrize("m,n", [(4, 9), (16, 40), (64, 256), (40, 16)])
+@pytest.mark.parametrize("restart", [(), (2,), (1, 3), (1, 2, 3, 4)])
+def test_gram_ns_equals_standard_ns_in_fp64(m, n, restart):
+    """Gram NS equals standard NS in exact arithmetic [GramNS Theorem 1]; a
+    restart only regroups the same products [GramNS §3.2]."""
+    gen = torch.Generator().manual_seed(m * 1000 + n)
+    X = torch.randn(m, n, generator=gen, dtype=DT)
+    a = O.ns_standard(X)
+    g = O.gram_ns(X, restart_after=restart)
+    assert float(torch.linalg.matrix_norm(g - a) / torch.linalg.matrix_norm(a)) < 1e-10
+
+
+def test_gram_ns_polar_express_table_equivalence():
+    """Theorem 1 holds for any per-step coefficients, e.g. the Polar Express
+    table printed in [GramNS §3.2]."""
+    pe = [(8.123737, -22.232240, 16.373715), (4.026529, -2.776323, 0.514551),
+          (3.870284, -2.739120, 0.520999), (3.253351, -2.343223, 0.481420),
+          (2.300652, -1.668904, 0.418807)]
+    gen = torch.Generator().manual_seed(11)
+    X = torch.randn(8, 20, generator=gen, dtype=DT) * 1e-3
+    a = O.ns_standard(X, abc=pe)
+    for restart in [(), (2,)]:
+        g = O.gram_ns(X, abc=pe, restart_after=restart)
+        assert float(torch.linalg.matrix_norm(g - a) / torch.linalg.matrix_norm(a)) < 1e-9
+
+
+def test_gram_ns_negative_eigenvalue_grows():
+    """[GramNS Prop. 2]: a negative eigenvalue of R grows under r <- r h(r)^2
+    with h(x) = 15/8 - 10/8 x + 3/8 x^2. Checked on the oracle's R update by
+    running it on a diagonal R with one negative entry."""
+    abc = [(15 / 8, -10 / 8, 3 / 8)] * 5
+    R = torch.diag(torch.tensor([0.5, 0.1, -1e-5], dtype=DT))
+    # run the oracle's R recursion: Z = bR + cR^2; RZ = RZ + aR; R = Z RZ + a RZ
+    mags = []
+    for a, b, c in abc:
+        Z = b * R + c * (R @ R)
+        RZ = R @ Z + a * R
+        R = Z @ RZ + a * RZ
+        mags.append(abs(float(R[2, 2])))
+    assert all(mags[i + 1] > 3.0 * mags[i] for i in range(4))
+    # and the positive eigenvalues converge towards 1 (r_t = x_t^2)
+    assert abs(float(R[0, 0]) - 1.0) < 0.05
+
+
+# ------------------------------------------------------------ FLOP counters
+
+def test_flop_counters_match_printed_savings():
+    rows = []
+    for line in open(os.path.join(GOLDEN, "gram_ns_flop_savings.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        v, a, s1, s2 = line.split()
+        rows.append((v, int(a), int(s1), int(s2)))
+    N = 64
+    for v, alpha, s_sym, s_typ in rows:
+        restart = () if v == "naive" else (2,)
+        g = F.gram_ns_flops(N, alpha * N, 5, restart)
+        std_sym = F.ns_standard_flops(N, alpha * N, 5, symmetric=True)
+        std_typ = F.ns_standard_flops(N, alpha * N, 5, symmetric=False)
+        assert round(100 * (1 - g / std_sym)) == s_sym
+        assert round(100 * (1 - g / std_typ)) == s_typ
+
+
+def test_flop_counter_closed_forms_and_gemm_counts():
+    N = 32
+    for alpha in [1, 2, 4, 8]:
+        assert F.gram_ns_flops(N, alpha * N, 5, ()) == (17 + 3 * alpha) * N ** 3
+        assert F.gram_ns_flops(N, alpha * N, 5, (2,)) == (14 + 6 * alpha) * N ** 3
+        assert F.ns_standard_flops(N, alpha * N) == 5 * (3 * alpha + 1) * N ** 3
+        assert F.ns_standard_flops(N, alpha * N, symmetric=False) == (20 * alpha + 10) * N ** 3
+    assert F.gram_ns_gemm_count(5, ()) == 19
+    # alpha = 1: Gram NS gives no saving over symmetric standard NS [GramNS §5.2]
+    assert F.gram_ns_flops(N, N, 5, (2,)) == F.ns_standard_flops(N, N)
+    # T-1 restarts regroup Gram NS into standard NS, product count aside [GramNS §3.4]
+    assert F.ns_standard_flops(N, 4 * N) <= F.gram_ns_flops(N, 4 * N, 5, (1, 2, 3, 4))
+
+
+# ------------------------------------------------------- power iteration + QR
+
+def test_orth_positive_matches_library_qr_full_rank():
+    gen = torch.Generator().manual_seed(5)
+    A = torch.randn(200, 12, generator=gen, dtype=DT) * torch.logspace(0, -3, 12, dtype=DT)
+    P, live = O.orth_positive(A)
+    q, r = torch.linalg.qr(A)
+    q = q * torch.sign(torch.diagonal(r))
+    assert all(live)
+    assert torch.allclose(P, q, atol=1e-11)
+    Rqr = P.T @ A
+    assert torch.all(torch.diagonal(Rqr) > 0)
+    assert torch.allclose(torch.triu(Rqr), Rqr, atol=1e-11)   # upper triangular
+
+
+def test_orth_positive_dead_columns():
+    gen = torch.Generator().manual_seed(6)
+    A = torch.randn(50, 4, generator=gen, dtype=DT)
+    A[:, 2] = 2.0 * A[:, 0] - A[:, 1]          # exactly dependent
+    A = torch.cat([A, torch.zeros(50, 1, dtype=DT)], dim=1)
+    P, live = O.orth_positive(A)
+    assert live == [True, True, False, True, False]
+    assert torch.all(P[:, 2] == 0) and torch.all(P[:, 4] == 0)
+    Pl = P[:, [0, 1, 3]]
+    assert torch.allclose(Pl.T @ Pl, torch.eye(3, dtype=DT), atol=1e-13)
+    # the live columns still span the input
+    assert torch.allclose(Pl @ (Pl.T @ A), A, atol=1e-12)
+    P0, live0 = O.orth_positive(torch.zeros(10, 3, dtype=DT))
+    assert live0 == [False] * 3 and torch.all(P0 == 0)
+
+
+def test_power_iteration_invariants():
+    gen = torch.Generator().manual_seed(8)
+    M = torch.randn(120, 90, generator=gen, dtype=DT)
+    Q = O.warm_start(torch.zeros(90, 6), 99, 0)
+    P, R, Ptil, live = O.power_iteration(M, Q)
+    assert torch.allclose(P.T @ P, torch.eye(6, dtype=DT), atol=1e-13)
+    assert torch.allclose(P @ (P.T @ Ptil), Ptil, atol=1e-11)       # P R_qr = P~
+    res = M - P @ R.T
+    assert float(torch.linalg.matrix_norm(P.T @ res)) < 1e-11       # P^T M_res = 0
+
+
+def test_power_iteration_exact_rank_k_is_lossless():
+    gen = torch.Generator().manual_seed(9)
+    k = 5
+    U = _orthogonal(80, gen)[:, :k]
+    V = _orthogonal(60, gen)[:, :k]
+    M = U @ torch.diag(torch.tensor([5.0, 4, 3, 2, 1], dtype=DT)) @ V.T
+    Qs = V + 0.3 * torch.randn(60, k, generator=gen, dtype=DT)      # spans V_k generically
+    P, R, _, live = O.power_iteration(M, Qs)
+    assert all(live)
+    assert float(torch.linalg.matrix_norm(M - P @ R.T)) < 1e-12
+
+
+def test_power_iteration_subspace_bound():
+    """One step of subspace iteration: tan(theta_1) <= (s_{k+1}/s_k) tan(theta_0)
+    (textbook bound), and with s_k/s_{k+1} >= 20 from a warm start the relative
+    error of the rank-k part is <= 0.01 (the 1-step figure of [GRASP, ablation])."""
+    gen = torch.Generator().manual_seed(10)
+    m, n, k = 300, 200, 8
+    U = _orthogonal(m, gen)
+    V = _orthogonal(n, gen)
+    s = torch.cat([torch.linspace(40, 20, k, dtype=DT), torch.linspace(1.0, 0.01, n - k, dtype=DT)])
+    M = U[:, :n] @ torch.diag(s) @ V.T
+    Vk = V[:, :k]
+    Mk = U[:, :k] @ torch.diag(s[:k]) @ Vk.T
+
+    def tan_theta(B, target):
+        B, _ = torch.linalg.qr(B)
+        c = torch.linalg.svdvals(target.T @ B).min()
+        return math.sqrt(max(0.0, 1 - float(c) ** 2)) / float(c)
+
+    for noise in [0.05, 0.01]:
+        Q0 = Vk + noise * torch.randn(n, k, generator=gen, dtype=DT)   # warm start near V_k
+        Q0 = Q0 / torch.linalg.vector_norm(Q0, dim=0)
+        P, R, _, _ = O.power_iteration(M, Q0)
+        t0 = tan_theta(Q0, Vk)
+        t1 = tan_theta(P, U[:, :k])
+        assert t1 <= float(s[k] / s[k - 1]) * t0 + 1e-12
+        # P P^T M - M_k = -(I - PP^T) U_k S_k V_k^T + PP^T U_perp S_perp V_perp^T, so
+        # |.|_F <= sin(theta_1) (|S_k|_F + sqrt(k) s_{k+1})
+        rel = float(torch.linalg.matrix_norm(P @ R.T - Mk) / torch.linalg.matrix_norm(Mk))
+        sin1 = t1 / math.sqrt(1 + t1 * t1)
+        skf = float(torch.linalg.vector_norm(s[:k]))
+        assert rel <= sin1 * (1 + math.sqrt(k) * float(s[k]) / skf) + 1e-12
+        if t0 <= 0.19:       # then tan(theta_1) <= 0.0095 and the 1-step error is <= 0.01
+            assert rel <= 0.01
+
+
+def test_warm_start_normalises_columns_and_uses_rademacher_for_zero_columns():
+    Rh = torch.zeros(40, 3, dtype=DT)
+    Rh[:, 0] = torch.arange(40, dtype=DT) - 20.0
+    Q = O.warm_start(Rh, 5, 2)
+    assert float(torch.linalg.vector_norm(Q[:, 0])) == pytest.approx(1.0, abs=1e-14)
+    assert torch.allclose(Q[:, 0] * torch.linalg.vector_norm(Rh[:, 0]), Rh[:, 0])
+    assert torch.equal(Q[:, 1], O.rademacher_column(5, 2, 40, 1))
+    assert torch.equal(Q[:, 2], O.rademacher_column(5, 2, 40, 2))
+
+
+# ------------------------------------------------------------- 4-bit grid
+
+def test_grid_quant4_handworked_example():
+    g = _read_sections(os.path.join(GOLDEN, "grid_quant4_handworked.txt"))
+    bits = torch.tensor([[int(v, 16) for v in row] for row in g["X_bits_hex"]], dtype=torch.int64)
+    X = bits.to(torch.int32).view(torch.float32)
+    codes, rs, cs = O.grid_quant4(X, block=2)
+    assert codes.tolist() == [[int(v) for v in row] for row in g["codes"]]
+    assert torch.equal(rs, torch.tensor([[float(v) for v in r] for r in g["rscale"]], dtype=torch.float32))
+    assert torch.equal(cs, torch.tensor([[float(v) for v in r] for r in g["cscale"]], dtype=torch.float32))
+    packed = O.pack_nibbles(codes)
+    assert packed.tolist() == [[int(v, 16) for v in row] for row in g["packed_hex"]]
+    assert torch.equal(O.unpack_nibbles(packed), codes)
+
+
+def test_grid_quant4_brute_force_codes():
+    """q is the code minimising |x - (q/7) s| over all 16 nibble values; ties
+    (equal distance) go to the even code."""
+    gen = torch.Generator().manual_seed(12)
+    for (m, n, blk) in [(8, 8, 4), (13, 22, 8), (130, 260, 128)]:
+        X = (torch.randn(m, n, generator=gen) * torch.rand(m, 1, generator=gen) * 3).to(torch.float32)
+        X[0, :] *= 50.0
+        codes, rs, cs = O.grid_quant4(X, block=blk)
+        s = O.grid_scale_matrix(rs, cs, m, n, blk)
+        r = (X / torch.where(s > 0, s, torch.ones_like(s))) * torch.tensor(7.0)   # fp32 ratio
+        cand = torch.arange(-8, 8, dtype=torch.float32)
+        dist = (r.unsqueeze(-1) - cand).abs()
+        best = dist.min(dim=-1).values
+        chosen = dist.gather(-1, (codes.to(torch.int64) + 8).unsqueeze(-1)).squeeze(-1)
+        assert torch.all(chosen[s > 0] == best[s > 0])
+        ties = (dist == best.unsqueeze(-1)).sum(-1) > 1
+        assert torch.all(codes[ties & (s > 0)] % 2 == 0)
+        # half-step error bound |x - x^| <= s/14 (plus fp32 rounding)
+        xh = O.grid_dequant4(codes, rs, cs, blk)
+        err = (X.double() - xh).abs()
+        assert torch.all(err <= s.double() / 14 * (1 + 1e-6) + 1e-30)
+
+
+def test_grid_quant4_invariants():
+    gen = torch.Generator().manual_seed(13)
+    m, n, blk = 256, 384, 128
+    X = torch.randn(m, n, generator=gen).to(torch.float32)
+    X[128:256, 0:128] = 0.0                         # one zero block
+    codes, rs, cs = O.grid_quant4(X, block=blk)
+    assert torch.all(codes[128:256, 0:128] == 0)
+    assert codes.abs().max() <= 7
+    for bi in range(2):
+        for bj in range(3):
+            blkc = codes[bi * blk:(bi + 1) * blk, bj * blk:(bj + 1) * blk]
+            blkx = X[bi * blk:(bi + 1) * blk, bj * blk:(bj + 1) * blk]
+            nz_rows = blkx.abs().amax(dim=1) > 0
+            nz_cols = blkx.abs().amax(dim=0) > 0
+            # each nonzero row and column of a block holds a +-7 code (its absmax)
+            assert torch.all((blkc.abs() == 7).any(dim=1)[nz_rows])
+            assert torch.all((blkc.abs() == 7).any(dim=0)[nz_cols])
+
+
+# ------------------------------------------------------------ 8-bit factors
+
+def test_quant8_brute_force_and_bounds():
+    gen = torch.Generator().manual_seed(14)
+    X = (torch.randn(333, 7, generator=gen) * torch.logspace(-4, 1, 7)).to(torch.float32)
+    X[:, 3] = 0.0
+    codes, s = O.quant8(X)
+    assert s[3] == 0 and torch.all(codes[:, 3] == 0)
+    for l in [0, 1, 2, 4, 5, 6]:
+        i = int(X[:, l].abs().argmax())
+        assert abs(int(codes[i, l])) == 127
+    safe = torch.where(s > 0, s, torch.ones_like(s))
+    r = (X / safe) * torch.tensor(127.0)
+    cand = torch.arange(-128, 128, dtype=torch.float32)
+    for l in [0, 5]:
+        dist = (r[:, l].unsqueeze(-1) - cand).abs()
+        best = dist.min(dim=-1).values
+        chosen = dist.gather(-1, (codes[:, l].to(torch.int64) + 128).unsqueeze(-1)).squeeze(-1)
+        assert torch.all(chosen == best)
+    err = (X.double() - O.dequant8(codes, s)).abs()
+    assert torch.all(err <= s.double() / 254 * (1 + 1e-6))
+
+
+# ------------------------------------------------------------ the full step
+
+def test_step_zero_gradient_zero_state_stays_zero():
+    st = O.zero_state(64, 96, 4, block=32)
+    W = torch.zeros(64, 96)
+    r = O.grasp_step(st, W, torch.zeros(64, 96), mu=0.95, eta=0.02, block=32)
+    assert torch.all(r.M == 0) and torch.all(r.P == 0) and torch.all(r.R == 0)
+    assert torch.all(r.state.codes4 == 0) and torch.all(r.state.P8 == 0)
+    assert torch.all(r.O == 0) and torch.all(r.W == 0)
+
+
+def test_step_mu_zero_momentum_is_gradient_and_k_full_is_lossless():
+    gen = torch.Generator().manual_seed(15)
+    m, n = 48, 80
+    G = torch.randn(m, n, generator=gen) * 1e-3
+    st = O.zero_state(m, n, 4, block=16)
+    st.codes4 = torch.randint(0, 255, (m, n // 2), generator=gen, dtype=torch.uint8)
+    st.rscale = torch.rand(st.rscale.shape, generator=gen)
+    st.cscale = torch.rand(st.cscale.shape, generator=gen)
+    r = O.grasp_step(st, torch.zeros(m, n), G, mu=0.0, eta=0.0, block=16)
+    assert torch.equal(r.M, G.double())
+    st2 = O.zero_state(m, n, m, block=16)
+    r2 = O.grasp_step(st2, torch.zeros(m, n), G, mu=0.9, eta=0.0, block=16)
+    assert float(torch.linalg.matrix_norm(r2.residual)) < 1e-12 * float(torch.linalg.matrix_norm(r2.M))
+
+
+def test_step_rebuild_roundtrip():
+    """After a step, rebuilding from the new state reproduces M_t up to the
+    codes' half-step bounds: |M - M^| <= s/14 + 8-bit factor error."""
+    gen = torch.Generator().manual_seed(16)
+    m, n, k = 64, 128, 4
+    G = torch.randn(m, n, generator=gen) * 1e-3
+    G[3, :] *= 10
+    G[:, 7] *= 10
+    st = O.zero_state(m, n, k, block=32)
+    r = O.grasp_step(st, torch.zeros(m, n), G, mu=0.95, eta=0.02, block=32)
+    Mh = O.rebuild_momentum(r.state, block=32)
+    rel = float(torch.linalg.matrix_norm(Mh - r.M) / torch.linalg.matrix_norm(r.M))
+    assert rel < 0.1
+    top = O.dequant8(r.state.P8, r.state.Pscale) @ O.dequant8(r.state.R8, r.state.Rscale).T
+    rel_top = float(torch.linalg.matrix_norm(top - r.P @ r.R.T) / torch.linalg.matrix_norm(r.P @ r.R.T))
+    assert rel_top < 0.02
