@@ -1,0 +1,55 @@
+// Internal helpers shared by the libgmuon translation units (not installed).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gmuon.h"
+
+namespace gm {
+
+constexpr int kGrid = GM_GRID_BLOCK;   // 128 x 128 grid-quant blocks
+constexpr int kMaxK = GM_MAX_K;
+
+__host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ inline long long cdivll(long long a, long long b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------- dtypes
+__device__ __forceinline__ float load_as_float(const void* p, long long idx, int dt) {
+  if (dt == GM_F32) return static_cast<const float*>(p)[idx];
+  if (dt == GM_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[idx]);
+  return __half2float(static_cast<const __half*>(p)[idx]);
+}
+
+// 16-bit float bits <-> float, for operands stored as raw uint16 (bf16 or f16)
+__device__ __forceinline__ float h16_to_float(uint16_t v, bool f16) {
+  if (f16) return __half2float(__ushort_as_half(v));
+  return __bfloat162float(__ushort_as_bfloat16(v));
+}
+__device__ __forceinline__ uint16_t float_to_h16(float v, bool f16) {
+  if (f16) return __half_as_ushort(__float2half_rn(v));
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+__device__ __forceinline__ void store_from_float(void* p, long long idx, int dt, float v) {
+  if (dt == GM_F32) static_cast<float*>(p)[idx] = v;
+  else if (dt == GM_BF16) static_cast<__nv_bfloat16*>(p)[idx] = __float2bfloat16_rn(v);
+  else static_cast<__half*>(p)[idx] = __float2half_rn(v);
+}
+
+// ----------------------------------------------------- splitmix64 (Steele et al.)
+__host__ __device__ inline uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// --------------------------------------------------------------- errors
+// Host-side error bookkeeping lives in gm_api.cu.
+gm_status set_error(gm_status s, const char* fmt, ...);
+
+}  // namespace gm

@@ -1,0 +1,664 @@
+// Tensor-core Newton-Schulz chains for sm_100a: tcgen05.mma with the
+// accumulator in TMEM, operands staged in shared memory by TMA.
+//
+// Standard NS ("优化器 (3)（Gram Newton-Schulz）", §1.2 eq. (2)) and the
+// stabilized Gram NS (same page, Algorithm 2) reduce to three product shapes
+// on the wide-form iterate X (N x M', row-major, 16-bit):
+//   XX^T      : C = X X^T                     (both operands K-major rows of X)
+//   sym       : C = S1 S2 for symmetric N x N S1, S2 (both operands K-major rows)
+//   left      : C = S X (S symmetric N x N)   (B operand MN-major: rows of X are K)
+// The first two produce symmetric results: only the lower-triangle tiles are
+// computed and each off-diagonal tile is stored twice (the triangular
+// scheduler of the page's §4). Epilogues apply C = alpha acc + beta Cin +
+// gamma I in fp32 (a_t enters here, never as an explicit identity).
+//
+// Kernel anatomy (one 128 x BN output tile per CTA, 6 warps):
+//   warp 0 lane 0 : TMA producer over a STAGES-deep shared-memory ring
+//   warp 1        : allocates TMEM; lane 0 issues tcgen05.mma (M=128, N=BN, K=16)
+//   warps 2..5    : epilogue, tcgen05.ld 32 lanes x 32 columns at a time
+// Every mbarrier wait is bounded (~2 s of %globaltimer); on timeout the
+// kernel records GM_E_TIMEOUT in an error word and unwinds.
+
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "gm_common.cuh"
+#include "gm_internal.h"
+
+namespace gm {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                 // 64 x 16-bit = 128 B = one swizzle row
+constexpr int kStages = 3;
+constexpr int kGemmThreads = 192;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ int32_t g_device_error = 0;
+
+enum EpiMode : int { EPI_STORE = 0, EPI_OUT = 1, EPI_WUPDATE = 2 };
+
+struct GemmParams {
+  int M, N, K;                 // output M x N; reduction K
+  int tiles_m, tiles_n;
+  int sym;                     // lower-triangle schedule + mirrored store
+  int f16;                     // operand / 16-bit output type: 1 fp16, 0 bf16
+  float alpha, beta, gamma;    // v = alpha acc + beta Cin + gamma [r == c]
+  const uint16_t* C; long long c_bs; int ldc;
+  uint16_t* D; long long d_bs; int ldd;
+  uint16_t* D2; float gamma2;  // optional D2 = v + gamma2 [r == c]
+  int mode;
+  int transpose_out;           // EPI_OUT / EPI_WUPDATE: natural = transpose of the tile
+  void* O; int odt; long long o_bs; int ldo;
+  float* W; long long w_bs; int ldw; float eta, wd;
+  const int32_t* skip;
+  int32_t* err;
+};
+
+// ------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false (and the error word set) once ~2 s have passed.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0 && globaltimer() - t0 > kWaitLimitNs) {
+      if (err) atomicExch(err, (int32_t)GM_E_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// UMMA shared-memory descriptor: SWIZZLE_128B, version 1 (sm_100).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+// Instruction descriptor, kind::f16: D f32, A/B bf16 or f16, A K-major.
+__host__ __device__ constexpr uint32_t idesc_f16(bool f16, bool b_mn_major, int n) {
+  return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) |
+         ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                     uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tri_tile(int x, int& ti, int& tj) {
+  int i = (int)((sqrtf(8.0f * (float)x + 1.0f) - 1.0f) * 0.5f);
+  while ((i + 1) * (i + 2) / 2 <= x) ++i;
+  while (i * (i + 1) / 2 > x) --i;
+  ti = i;
+  tj = x - i * (i + 1) / 2;
+}
+
+// ------------------------------------------------------------------ kernel
+template <int BN, bool B_MN>
+__global__ void __launch_bounds__(kGemmThreads, 2)
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+           const GemmParams p) {
+  if (p.skip && *p.skip) return;
+  constexpr uint32_t kABytes = BM * BK * 2;
+  constexpr uint32_t kBBytes = BN * BK * 2;
+  constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  constexpr uint32_t kTmemCols = BN;   // fp32 accumulator columns (power of 2 >= 32)
+
+  extern __shared__ __align__(1024) uint8_t dsm[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* accum = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* consumed = abort_flag + 1;   // k-blocks whose full barrier the MMA warp waited on
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bz = blockIdx.y;
+  int ti, tj;
+  if (p.sym) tri_tile(blockIdx.x, ti, tj);
+  else { ti = blockIdx.x % p.tiles_m; tj = blockIdx.x / p.tiles_m; }
+  const int nk = cdiv(p.K, BK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    mbar_init(smem_u32(accum), 1);
+    *abort_flag = 0;
+    *consumed = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    prefetch_map(&tmA);
+    prefetch_map(&tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  int issued = 0;   // producer only
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kStages;
+      const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+      if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err)) { *abort_flag = 1; break; }
+      const uint32_t a_dst = smem_u32(base + s * kStageBytes);
+      const uint32_t b_dst = a_dst + kABytes;
+      const uint32_t bar = smem_u32(&full[s]);
+      mbar_expect_tx(bar, kStageBytes);
+      tma_load_3d(a_dst, &tmA, bar, kb * BK, ti * BM, bz);
+      if (!B_MN) {
+        tma_load_3d(b_dst, &tmB, bar, kb * BK, tj * BN, bz);
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c)
+          tma_load_3d(b_dst + c * (BK * 128), &tmB, bar, tj * BN + c * 64, kb * BK, bz);
+      }
+      issued = kb + 1;
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idesc = idesc_f16(false, B_MN, BN);
+    const uint32_t idesc_rt = p.f16 ? idesc_f16(true, B_MN, BN) : idesc;
+    bool ok = true;
+    int kb = 0;
+    for (; kb < nk; ++kb) {
+      const int s = kb % kStages;
+      const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+      if (!mbar_wait(smem_u32(&full[s]), ph, p.err)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t a_base = smem_u32(base + s * kStageBytes);
+      const uint32_t b_base = a_base + kABytes;
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk) {
+        const uint64_t ad = sdesc(a_base + kk * 32, 16, 1024);
+        const uint64_t bd = B_MN ? sdesc(b_base + kk * 2048, BK * 128, 1024)
+                                 : sdesc(b_base + kk * 32, 16, 1024);
+        umma(tmem, ad, bd, idesc_rt, (kb | kk) ? 1u : 0u);
+      }
+      umma_commit(smem_u32(&empty[s]));   // frees the stage once these MMAs finish
+    }
+    *consumed = kb;
+    if (!ok) *abort_flag = 1;
+    // Arrives once every MMA issued above has completed, abort or not.
+    umma_commit(smem_u32(accum));
+  } else if (warp >= 2) {
+    // ---------------- epilogue
+    const bool ok = mbar_wait(smem_u32(accum), 0, p.err);
+    tc_fence_after();
+    if (ok) {
+      const int q = warp & 3;               // TMEM lane quarter this warp may access
+      const int r = ti * BM + q * 32 + lane;  // output row of this thread
+      const bool rvalid = r < p.M;
+      const float alpha = p.alpha, beta = p.beta;
+      const bool store = !*abort_flag;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        float v[32];
+        __syncwarp();
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+        const int cb = tj * BN + c0;
+        if (!store || !rvalid || cb >= p.N) continue;
+        // N is a multiple of 16: a 32-column chunk is full or half full.
+        const int ncols = min(32, p.N - cb);
+        if (p.mode == EPI_STORE) {
+          const long long cin_off = (long long)bz * p.c_bs + (long long)r * p.ldc + cb;
+          float cin[32];
+          if (p.C && beta != 0.f) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              if (g * 8 < ncols) {
+                const uint4 raw = *reinterpret_cast<const uint4*>(p.C + cin_off + g * 8);
+                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  cin[g * 8 + 2 * e] = h16_to_float(w[e] & 0xFFFF, p.f16);
+                  cin[g * 8 + 2 * e + 1] = h16_to_float(w[e] >> 16, p.f16);
+                }
+              }
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) cin[e] = 0.f;
+          }
+          uint16_t outv[32];
+          uint16_t out2[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float x = alpha * v[e] + beta * cin[e];
+            if (r == cb + e) x += p.gamma;
+            outv[e] = float_to_h16(x, p.f16);
+            if (p.D2) out2[e] = float_to_h16(x + ((r == cb + e) ? p.gamma2 : 0.f), p.f16);
+          }
+          uint16_t* drow = p.D + (long long)bz * p.d_bs + (long long)r * p.ldd + cb;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            if (g * 8 < ncols) {
+              uint4 w;
+              w.x = outv[g * 8 + 0] | ((uint32_t)outv[g * 8 + 1] << 16);
+              w.y = outv[g * 8 + 2] | ((uint32_t)outv[g * 8 + 3] << 16);
+              w.z = outv[g * 8 + 4] | ((uint32_t)outv[g * 8 + 5] << 16);
+              w.w = outv[g * 8 + 6] | ((uint32_t)outv[g * 8 + 7] << 16);
+              *reinterpret_cast<uint4*>(drow + g * 8) = w;
+            }
+          }
+          if (p.D2) {
+            uint16_t* d2row = p.D2 + (long long)bz * p.d_bs + (long long)r * p.ldd + cb;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              if (g * 8 < ncols) {
+                uint4 w;
+                w.x = out2[g * 8 + 0] | ((uint32_t)out2[g * 8 + 1] << 16);
+                w.y = out2[g * 8 + 2] | ((uint32_t)out2[g * 8 + 3] << 16);
+                w.z = out2[g * 8 + 4] | ((uint32_t)out2[g * 8 + 5] << 16);
+                w.w = out2[g * 8 + 6] | ((uint32_t)out2[g * 8 + 7] << 16);
+                *reinterpret_cast<uint4*>(d2row + g * 8) = w;
+              }
+            }
+          }
+          if (p.sym && ti != tj) {
+            // mirrored tile: D[c][r]; consecutive lanes write consecutive r
+            uint16_t* dcol = p.D + (long long)bz * p.d_bs + r;
+            uint16_t* d2col = p.D2 ? p.D2 + (long long)bz * p.d_bs + r : nullptr;
+#pragma unroll 8
+            for (int e = 0; e < ncols; ++e) {
+              dcol[(long long)(cb + e) * p.ldd] = outv[e];
+              if (d2col) d2col[(long long)(cb + e) * p.ldd] = out2[e];
+            }
+          }
+        } else {
+          // natural-orientation output O = alpha acc + beta Cin, or the W update
+          const long long cin_off = (long long)bz * p.c_bs + (long long)r * p.ldc + cb;
+          float val[32];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            if (g * 8 < ncols) {
+              uint4 raw = make_uint4(0, 0, 0, 0);
+              if (p.C && beta != 0.f) raw = *reinterpret_cast<const uint4*>(p.C + cin_off + g * 8);
+              const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                val[g * 8 + 2 * e] = alpha * v[g * 8 + 2 * e] + beta * h16_to_float(w[e] & 0xFFFF, p.f16);
+                val[g * 8 + 2 * e + 1] = alpha * v[g * 8 + 2 * e + 1] + beta * h16_to_float(w[e] >> 16, p.f16);
+              }
+            }
+          }
+          for (int e = 0; e < ncols; ++e) {
+            const int c = cb + e;
+            long long idx;
+            if (p.transpose_out) idx = (long long)c * (p.mode == EPI_OUT ? p.ldo : p.ldw) + r;
+            else idx = (long long)r * (p.mode == EPI_OUT ? p.ldo : p.ldw) + c;
+            if (p.mode == EPI_OUT) {
+              store_from_float(p.O, (long long)bz * p.o_bs + idx, p.odt, val[e]);
+            } else {
+              float* w = p.W + (long long)bz * p.w_bs + idx;
+              const float wv = *w;
+              *w = wv - p.eta * (val[e] + p.wd * wv);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0 && lane == 0) {
+    // After an abort, let the copies still in flight land before the CTA exits.
+    for (int kb = *consumed; kb < issued; ++kb)
+      mbar_wait(smem_u32(&full[kb % kStages]), (uint32_t)(kb / kStages) & 1u, p.err);
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 3-D map over [batch][rows][cols] of 16-bit elements with a {64, box_rows, 1}
+// box and the 128-byte swizzle the UMMA descriptors above expect.
+bool make_map(CUtensorMap* map, const void* base, bool f16, int rows, int cols, int ld,
+              int batch, long long batch_stride, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)batch_stride * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, bool B_MN>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int batch,
+                        cudaStream_t s) {
+  constexpr int smem = kStages * (BM * BK * 2 + BN * BK * 2) + 1024 + 256;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm<BN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int tiles = p.sym ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
+  dim3 grid(tiles, batch);
+  k_gemm<BN, B_MN><<<grid, kGemmThreads, smem, s>>>(a, b, p);
+  return cudaGetLastError();
+}
+
+GemmParams base_params(int M, int N, int K, bool f16, const int32_t* skip, int32_t* err) {
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = M; p.N = N; p.K = K;
+  p.f16 = f16 ? 1 : 0;
+  p.alpha = 1.f;
+  p.skip = skip;
+  p.err = err;
+  return p;
+}
+
+struct Ns {
+  int B, N, Mp;     // wide form N x M'
+  bool f16;
+  bool tall;        // natural = transpose of the wide form
+  const int32_t* skip;
+  int32_t* err;
+  cudaStream_t s;
+};
+
+// C (N x N, symmetric) = X X^T (+ epilogue), X: N x M'.
+cudaError_t xxt(const Ns& c, const uint16_t* X, uint16_t* D) {
+  CUtensorMap ma;
+  if (!make_map(&ma, X, c.f16, c.N, c.Mp, c.Mp, c.B, (long long)c.N * c.Mp, BM)) return cudaErrorInvalidValue;
+  GemmParams p = base_params(c.N, c.N, c.Mp, c.f16, c.skip, c.err);
+  p.tiles_m = p.tiles_n = cdiv(c.N, BM);
+  p.sym = 1;
+  p.D = D; p.d_bs = (long long)c.N * c.N; p.ldd = c.N;
+  return launch_gemm<128, false>(ma, ma, p, c.B, c.s);
+}
+
+// D = alpha S1 S2 + beta Cin + gamma I (symmetric N x N operands); D2 optional.
+cudaError_t symmul(const Ns& c, const uint16_t* S1, const uint16_t* S2, float alpha, float beta,
+                   const uint16_t* Cin, float gamma, uint16_t* D, uint16_t* D2 = nullptr,
+                   float gamma2 = 0.f) {
+  CUtensorMap ma, mb;
+  const long long bs = (long long)c.N * c.N;
+  if (!make_map(&ma, S1, c.f16, c.N, c.N, c.N, c.B, bs, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&mb, S2, c.f16, c.N, c.N, c.N, c.B, bs, 128)) return cudaErrorInvalidValue;
+  GemmParams p = base_params(c.N, c.N, c.N, c.f16, c.skip, c.err);
+  p.tiles_m = p.tiles_n = cdiv(c.N, BM);
+  p.sym = 1;
+  p.alpha = alpha; p.beta = beta; p.gamma = gamma;
+  p.C = Cin; p.c_bs = bs; p.ldc = c.N;
+  p.D = D; p.d_bs = bs; p.ldd = c.N;
+  p.D2 = D2; p.gamma2 = gamma2;
+  return launch_gemm<128, false>(ma, mb, p, c.B, c.s);
+}
+
+// Y = alpha S X + beta X  (S symmetric N x N, X N x M'); either stored as a new
+// iterate (D) or written out in natural orientation (final step).
+cudaError_t leftmul(const Ns& c, const uint16_t* S, const uint16_t* X, float alpha, float beta,
+                    uint16_t* D, const NsOutput* out) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, S, c.f16, c.N, c.N, c.N, c.B, (long long)c.N * c.N, BM)) return cudaErrorInvalidValue;
+  // MN-major B operand: rows of X are the K index, columns the N index.
+  if (!make_map(&mb, X, c.f16, c.N, c.Mp, c.Mp, c.B, (long long)c.N * c.Mp, BK)) return cudaErrorInvalidValue;
+  GemmParams p = base_params(c.N, c.Mp, c.N, c.f16, c.skip, c.err);
+  p.tiles_m = cdiv(c.N, BM);
+  p.tiles_n = cdiv(c.Mp, 128);
+  p.alpha = alpha; p.beta = beta;
+  p.C = X; p.c_bs = (long long)c.N * c.Mp; p.ldc = c.Mp;
+  if (!out) {
+    p.mode = EPI_STORE;
+    p.D = D; p.d_bs = (long long)c.N * c.Mp; p.ldd = c.Mp;
+  } else {
+    p.transpose_out = c.tall ? 1 : 0;
+    const int ld = c.tall ? c.N : c.Mp;   // natural row length
+    if (out->mode == 0) {
+      p.mode = EPI_OUT;
+      p.O = out->O; p.odt = out->odt; p.o_bs = (long long)c.N * c.Mp; p.ldo = ld;
+    } else {
+      p.mode = EPI_WUPDATE;
+      p.W = out->W; p.w_bs = (long long)c.N * c.Mp; p.ldw = ld;
+      p.eta = out->eta; p.wd = out->wd;
+    }
+  }
+  return launch_gemm<128, true>(ma, mb, p, c.B, c.s);
+}
+
+#define GM_TRY(x)                          \
+  do {                                     \
+    cudaError_t e_ = (x);                  \
+    if (e_ != cudaSuccess) return e_;      \
+  } while (0)
+
+uint8_t* carve(uint8_t*& cur, size_t bytes) {
+  uint8_t* p = cur;
+  cur += (bytes + 255) & ~size_t(255);
+  return p;
+}
+
+}  // namespace
+
+size_t ns_standard_ws_bytes(int B, int m, int n) {
+  const size_t N = (size_t)(m < n ? m : n), Mp = (size_t)(m < n ? n : m);
+  auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
+  return al(B * N * Mp * 2) + 2 * al(B * N * N * 2);
+}
+size_t ns_gram_ws_bytes(int B, int m, int n) {
+  const size_t N = (size_t)(m < n ? m : n), Mp = (size_t)(m < n ? n : m);
+  auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
+  return al(B * N * Mp * 2) + 6 * al(B * N * N * 2);
+}
+
+cudaError_t run_ns_standard(int B, int m, int n, uint16_t* X16, const float* abc, int T,
+                            const NsOutput& out, void* ws, const int32_t* skip, int32_t* err,
+                            cudaStream_t s) {
+  Ns c{B, m < n ? m : n, m < n ? n : m, false, m > n, skip, err ? err : device_error_word(), s};
+  uint8_t* cur = static_cast<uint8_t*>(ws);
+  uint16_t* Xb = reinterpret_cast<uint16_t*>(carve(cur, (size_t)B * c.N * c.Mp * 2));
+  uint16_t* A = reinterpret_cast<uint16_t*>(carve(cur, (size_t)B * c.N * c.N * 2));
+  uint16_t* Bm = reinterpret_cast<uint16_t*>(carve(cur, (size_t)B * c.N * c.N * 2));
+  uint16_t* X = X16;
+  uint16_t* Xn = Xb;
+  for (int t = 0; t < T; ++t) {
+    const float a = abc[3 * t], b = abc[3 * t + 1], cc = abc[3 * t + 2];
+    GM_TRY(xxt(c, X, A));                                  // A = X X^T
+    GM_TRY(symmul(c, A, A, cc, b, A, 0.f, Bm));            // B = c A^2 + b A
+    const bool last = (t == T - 1);
+    GM_TRY(leftmul(c, Bm, X, 1.f, a, Xn, last ? &out : nullptr));   // X = B X + a X
+    uint16_t* tmp = X; X = Xn; Xn = tmp;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t run_ns_gram(int B, int m, int n, uint16_t* X16, const float* abc, int T,
+                        const int* restart_after, int n_restart, const NsOutput& out, void* ws,
+                        const int32_t* skip, int32_t* err, cudaStream_t s) {
+  Ns c{B, m < n ? m : n, m < n ? n : m, true, m > n, skip, err ? err : device_error_word(), s};
+  uint8_t* cur = static_cast<uint8_t*>(ws);
+  const size_t nn = (size_t)B * c.N * c.N * 2;
+  uint16_t* Xb = reinterpret_cast<uint16_t*>(carve(cur, (size_t)B * c.N * c.Mp * 2));
+  uint16_t* R = reinterpret_cast<uint16_t*>(carve(cur, nn));
+  uint16_t* Rn = reinterpret_cast<uint16_t*>(carve(cur, nn));
+  uint16_t* Z = reinterpret_cast<uint16_t*>(carve(cur, nn));
+  uint16_t* Q = reinterpret_cast<uint16_t*>(carve(cur, nn));
+  uint16_t* Qn = reinterpret_cast<uint16_t*>(carve(cur, nn));
+  uint16_t* RZ = reinterpret_cast<uint16_t*>(carve(cur, nn));
+  bool restart_at[GM_MAX_T + 1] = {false};
+  for (int i = 0; i < n_restart; ++i)
+    if (restart_after[i] >= 1 && restart_after[i] < T) restart_at[restart_after[i]] = true;
+  uint16_t* X = X16;
+  uint16_t* Xn = Xb;
+  GM_TRY(xxt(c, X, R));                                    // R = X X^T
+  bool q_is_identity = true;
+  for (int t = 1; t <= T; ++t) {
+    const float a = abc[3 * (t - 1)], b = abc[3 * (t - 1) + 1], cc = abc[3 * (t - 1) + 2];
+    const bool block_end = restart_at[t] || t == T;
+    if (q_is_identity) {
+      // Z = c R^2 + b R, and Q = Z + a I from the same epilogue
+      GM_TRY(symmul(c, R, R, cc, b, R, 0.f, Z, Q, a));
+      q_is_identity = false;
+    } else {
+      GM_TRY(symmul(c, R, R, cc, b, R, 0.f, Z));
+      GM_TRY(symmul(c, Q, Z, 1.f, a, Q, 0.f, Qn));          // Q = Q Z + a Q
+      uint16_t* tq = Q; Q = Qn; Qn = tq;
+    }
+    if (!block_end) {
+      GM_TRY(symmul(c, R, Z, 1.f, a, R, 0.f, RZ));          // RZ = R Z + a R
+      GM_TRY(symmul(c, Z, RZ, 1.f, a, RZ, 0.f, Rn));        // R = Z RZ + a RZ
+      uint16_t* tr = R; R = Rn; Rn = tr;
+    } else if (t < T) {
+      GM_TRY(leftmul(c, Q, X, 1.f, 0.f, Xn, nullptr));      // restart: X = Q X
+      uint16_t* tx = X; X = Xn; Xn = tx;
+      GM_TRY(xxt(c, X, R));
+      q_is_identity = true;
+    } else {
+      GM_TRY(leftmul(c, Q, X, 1.f, 0.f, nullptr, &out));    // O = Q X
+    }
+  }
+  return cudaSuccess;
+}
+
+void ns_schedule_flops(int ns_mode, int m, int n, int T, const int* restart_after, int n_restart,
+                       double* flops, int* products) {
+  const double N = (double)(m < n ? m : n), Mp = (double)(m < n ? n : m);
+  const double xxt_f = Mp * N * N, sym_f = N * N * N, left_f = 2.0 * Mp * N * N;
+  double f = 0.0;
+  int cnt = 0;
+  if (ns_mode == GM_NS_STANDARD) {
+    f = T * (xxt_f + sym_f + left_f);
+    cnt = 3 * T;
+  } else {
+    bool restart_at[GM_MAX_T + 1] = {false};
+    for (int i = 0; i < n_restart; ++i)
+      if (restart_after[i] >= 1 && restart_after[i] < T) restart_at[restart_after[i]] = true;
+    f += xxt_f; cnt += 1;
+    bool qi = true;
+    for (int t = 1; t <= T; ++t) {
+      const bool block_end = restart_at[t] || t == T;
+      f += sym_f; cnt += 1;                  // R^2 (Q = Z + aI rides in its epilogue)
+      if (!qi) { f += sym_f; cnt += 1; }     // Q Z
+      qi = false;
+      if (!block_end) { f += 2 * sym_f; cnt += 2; }
+      else {
+        f += left_f; cnt += 1;
+        if (t < T) { f += xxt_f; cnt += 1; qi = true; }
+      }
+    }
+  }
+  if (flops) *flops = f;
+  if (products) *products = cnt;
+}
+
+int32_t* device_error_word() {
+  static int32_t* ptr = nullptr;
+  if (!ptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) ptr = static_cast<int32_t*>(p);
+  }
+  return ptr;
+}
+
+}  // namespace gm

@@ -1,0 +1,80 @@
+// Internal launcher interface between the libgmuon translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gm {
+
+// Column / row split counts of the power-iteration reductions. They depend
+// only on the problem shape, so the workspace layout is a pure function of it.
+int project_col_splits(int B, int m, int n);
+int backproject_row_splits(int B, int m, int n);
+int gram_row_splits(int B, int m);
+
+// ---- codec / power-iteration kernels (gm_codec.cu) ------------------------
+cudaError_t launch_warm_start(int B, int n, int k, const int8_t* R8, const float* Rscale,
+                              const float* Rprev, uint64_t seed, float* Q,
+                              const int32_t* skip, cudaStream_t s);
+
+// M = mu * Mprev + G where Mprev is either the rebuilt state (codes4 != NULL)
+// or a dense fp32 matrix (Mprev32 != NULL) or zero. norm2_part gets one fp64
+// partial |M|^2 per 128x128 tile; status (nullable) gets GM_E_NONFINITE.
+cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4,
+                           const float* rscale, const float* cscale, const int8_t* P8,
+                           const float* Pscale, const int8_t* R8, const float* Rscale,
+                           const float* Mprev32, float mu, const void* G, int gdt, float* M,
+                           double* norm2_part, int32_t* status, cudaStream_t s);
+
+cudaError_t launch_project(int B, int m, int n, int k, const float* M, const float* Q,
+                           double* Ppart, const int32_t* skip, cudaStream_t s);
+
+cudaError_t launch_orth(int B, int m, int k, int csplit, const double* Ppart, double* Ptil,
+                        double* gram_part, double* Tmat, const double* norm2_part, int ntiles,
+                        float eps, float* scale, float* P, const int32_t* skip, cudaStream_t s);
+
+cudaError_t launch_backproject(int B, int m, int n, int k, const float* M, const float* P,
+                               const float* scale, void* X16, bool f16, double* Rpart,
+                               float* R, const int32_t* skip, cudaStream_t s);
+
+cudaError_t launch_residual_quant4(int B, int m, int n, int k, const float* X, const float* P,
+                                   const float* R, uint8_t* codes4, float* rscale,
+                                   float* cscale, const int32_t* skip, cudaStream_t s);
+
+cudaError_t launch_quant8(int B, int rows0, int rows1, int k, const float* X0, int8_t* c0,
+                          float* s0, const float* X1, int8_t* c1, float* s1,
+                          int64_t* step, const int32_t* skip, cudaStream_t s);
+
+// Standalone NS input: scale = 1/(|X|_F + eps) per matrix, then the wide
+// 16-bit copy Y = round(scale * X) (transposed when m > n).
+cudaError_t launch_ns_prep(int B, int m, int n, const void* X, int xdt, float eps,
+                           double* norm2_part, int nparts, float* scale, void* Y16, bool f16,
+                           cudaStream_t s);
+int ns_prep_parts(int m, int n);
+
+// ---- tensor-core Newton-Schulz chains (gm_gemm.cu) --------------------------
+struct NsOutput {
+  int mode;            // 0: write O (dtype odt), 1: W -= eta (O + wd W)
+  void* O;
+  int odt;
+  float* W;
+  float eta, wd;
+};
+
+size_t ns_standard_ws_bytes(int B, int m, int n);
+size_t ns_gram_ws_bytes(int B, int m, int n);
+
+// X16: wide-form normalised input [B][N][M'] (bf16 for standard, fp16 for
+// Gram); it is overwritten. ws: scratch of the sizes above.
+cudaError_t run_ns_standard(int B, int m, int n, uint16_t* X16, const float* abc, int T,
+                            const NsOutput& out, void* ws, const int32_t* skip, int32_t* err,
+                            cudaStream_t s);
+cudaError_t run_ns_gram(int B, int m, int n, uint16_t* X16, const float* abc, int T,
+                        const int* restart_after, int n_restart, const NsOutput& out, void* ws,
+                        const int32_t* skip, int32_t* err, cudaStream_t s);
+
+void ns_schedule_flops(int ns_mode, int m, int n, int T, const int* restart_after,
+                       int n_restart, double* flops, int* products);
+int32_t* device_error_word();
+
+}  // namespace gm

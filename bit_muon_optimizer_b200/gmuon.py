@@ -1,0 +1,327 @@
+"""Thin ctypes binding of libgmuon (include/gmuon.h).
+
+Argument marshalling only: every step of the optimizer runs in the library's
+CUDA kernels. Tensors are torch CUDA tensors, contiguous, batch-first
+([B, rows, cols]); work is enqueued on torch's current CUDA stream. Importing
+this module fails loudly when the library has not been built.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgmuon.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "gmuon.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m bit_muon_optimizer_b200.build`")
+lib = ctypes.CDLL(LIB_PATH)
+
+GM_OK, GM_E_ARG, GM_E_CUDA, GM_E_NONFINITE, GM_E_WORKSPACE, GM_E_UNSUPPORTED, GM_E_TIMEOUT = (
+    0, -1, -2, -3, -4, -5, -6)
+GM_F32, GM_BF16, GM_F16 = 0, 1, 2
+GM_NS_STANDARD, GM_NS_GRAM = 0, 1
+GM_OP_MOMENTUM_POWERIT, GM_OP_NEWTON_SCHULZ, GM_OP_GRAM_NS, GM_OP_GRASP_STEP = 1, 2, 3, 4
+GRID_BLOCK = 128
+
+_DT = {torch.float32: GM_F32, torch.bfloat16: GM_BF16, torch.float16: GM_F16}
+
+c_int, c_float, c_size_t, c_uint64, vp = (ctypes.c_int, ctypes.c_float, ctypes.c_size_t,
+                                          ctypes.c_uint64, ctypes.c_void_p)
+
+
+class GraspParams(ctypes.Structure):
+    _fields_ = [("mu", c_float), ("eta", c_float), ("wd", c_float), ("k", c_int), ("T", c_int),
+                ("ns", c_int), ("abc", ctypes.POINTER(c_float)),
+                ("restart_after", ctypes.POINTER(c_int)), ("n_restart", c_int),
+                ("eps", c_float), ("seed", c_uint64)]
+
+
+class GraspStateC(ctypes.Structure):
+    _fields_ = [("codes4", vp), ("rscale", vp), ("cscale", vp), ("P8", vp), ("Pscale", vp),
+                ("R8", vp), ("Rscale", vp), ("step", vp), ("dev_status", vp)]
+
+
+class GraspWsLayout(ctypes.Structure):
+    _fields_ = [("M", c_size_t), ("Q", c_size_t), ("P", c_size_t), ("R", c_size_t),
+                ("X", c_size_t), ("scale", c_size_t), ("total", c_size_t)]
+
+
+def _sig(name, res, args):
+    f = getattr(lib, name)
+    f.restype = res
+    f.argtypes = args
+    return f
+
+
+_sig("gm_status_string", ctypes.c_char_p, [c_int])
+_sig("gm_last_error", ctypes.c_char_p, [])
+_sig("gm_version", c_int, [])
+_sig("gm_workspace_bytes", c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int])
+_sig("gm_dequant_rebuild", c_int, [c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp])
+_sig("gm_momentum_powerit", c_int, [c_int, c_int, c_int, c_int, c_float, vp, vp, c_int, vp,
+                                    c_uint64, vp, vp, vp, vp, c_size_t, vp])
+_sig("gm_grid_quant4", c_int, [c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, vp])
+_sig("gm_quant8", c_int, [c_int, c_int, c_int, vp, vp, vp, vp])
+_sig("gm_newton_schulz", c_int, [c_int, c_int, c_int, vp, c_int, vp, c_int, c_float, vp, c_int,
+                                 vp, c_size_t, vp])
+_sig("gm_gram_ns", c_int, [c_int, c_int, c_int, vp, c_int, vp, c_int, vp, c_int, c_float, vp,
+                           c_int, vp, c_size_t, vp])
+_sig("gm_grasp_step", c_int, [c_int, c_int, c_int, ctypes.POINTER(GraspParams),
+                              ctypes.POINTER(GraspStateC), vp, vp, c_int, vp, c_size_t, vp])
+_sig("gm_grasp_workspace_layout", c_int, [c_int, c_int, c_int, c_int, c_int,
+                                          ctypes.POINTER(GraspWsLayout)])
+_sig("gm_ns_flops", c_int, [c_int, c_int, c_int, c_int, vp, c_int,
+                            ctypes.POINTER(ctypes.c_double), ctypes.POINTER(c_int)])
+_sig("gm_device_errors", c_int, [vp])
+
+
+class GmuonError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.gm_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {lib.gm_status_string(status).decode()} ({msg})")
+
+
+def _check(status: int, where: str):
+    if status != GM_OK:
+        raise GmuonError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _bmn(X):
+    if X.dim() == 2:
+        return 1, X.shape[0], X.shape[1]
+    if X.dim() != 3:
+        raise ValueError("expected [B, m, n] or [m, n]")
+    return X.shape[0], X.shape[1], X.shape[2]
+
+
+def _floats(vals):
+    if vals is None:
+        return None
+    arr = (c_float * len(vals))(*vals)
+    return arr
+
+
+def abc_table(abc, T):
+    """Flatten a list of (a, b, c) triples (or None: constant quintic)."""
+    if abc is None:
+        return None
+    flat = [float(v) for tri in abc for v in tri]
+    if len(flat) != 3 * T:
+        raise ValueError("abc must hold T triples")
+    return _floats(flat)
+
+
+_WS = {}
+
+
+def workspace(nbytes: int, device=None, tag="default") -> torch.Tensor:
+    """A cached 256-byte-aligned device scratch buffer of at least nbytes."""
+    device = torch.device(device or torch.cuda.current_device())
+    key = (tag, device)
+    buf = _WS.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _WS[key] = buf
+    return buf
+
+
+def workspace_bytes(op, B, m, n, k=0, ns=GM_NS_STANDARD) -> int:
+    return int(lib.gm_workspace_bytes(op, B, m, n, k, ns))
+
+
+# ----------------------------------------------------------------- entry points
+
+def dequant_rebuild(codes4, rscale, cscale, P8=None, Pscale=None, R8=None, Rscale=None, out=None):
+    B, m, n2 = _bmn(codes4)
+    n = 2 * n2
+    k = 0 if P8 is None else P8.shape[-1]
+    if out is None:
+        out = torch.empty((B, m, n), dtype=torch.float32, device=codes4.device)
+    _check(lib.gm_dequant_rebuild(B, m, n, k, _ptr(codes4), _ptr(rscale), _ptr(cscale), _ptr(P8),
+                                  _ptr(Pscale), _ptr(R8), _ptr(Rscale), _ptr(out), _stream()),
+           "gm_dequant_rebuild")
+    return out
+
+
+def momentum_powerit(G, k, mu=0.95, M_prev=None, R_prev=None, seed=0):
+    B, m, n = _bmn(G)
+    dev = G.device
+    M = torch.empty((B, m, n), dtype=torch.float32, device=dev)
+    P = torch.empty((B, m, k), dtype=torch.float32, device=dev)
+    R = torch.empty((B, n, k), dtype=torch.float32, device=dev)
+    nb = workspace_bytes(GM_OP_MOMENTUM_POWERIT, B, m, n, k)
+    ws = workspace(nb, dev)
+    _check(lib.gm_momentum_powerit(B, m, n, k, mu, _ptr(M_prev), _ptr(G), _DT[G.dtype],
+                                   _ptr(R_prev), seed, _ptr(M), _ptr(P), _ptr(R), _ptr(ws), nb,
+                                   _stream()), "gm_momentum_powerit")
+    return M, P, R
+
+
+def grid_quant4(X, P=None, R=None):
+    B, m, n = _bmn(X)
+    dev = X.device
+    k = 0 if P is None else P.shape[-1]
+    codes = torch.empty((B, m, n // 2), dtype=torch.uint8, device=dev)
+    rs = torch.empty((B, m, -(-n // GRID_BLOCK)), dtype=torch.float32, device=dev)
+    cs = torch.empty((B, -(-m // GRID_BLOCK), n), dtype=torch.float32, device=dev)
+    _check(lib.gm_grid_quant4(B, m, n, k, _ptr(X), _ptr(P), _ptr(R), _ptr(codes), _ptr(rs),
+                              _ptr(cs), _stream()), "gm_grid_quant4")
+    return codes, rs, cs
+
+
+def quant8(X):
+    B, rows, k = _bmn(X)
+    codes = torch.empty((B, rows, k), dtype=torch.int8, device=X.device)
+    scale = torch.empty((B, k), dtype=torch.float32, device=X.device)
+    _check(lib.gm_quant8(B, rows, k, _ptr(X), _ptr(codes), _ptr(scale), _stream()), "gm_quant8")
+    return codes, scale
+
+
+def newton_schulz(X, abc=None, T=5, eps=1e-7, out_dtype=torch.float32):
+    B, m, n = _bmn(X)
+    O = torch.empty((B, m, n), dtype=out_dtype, device=X.device)
+    nb = workspace_bytes(GM_OP_NEWTON_SCHULZ, B, m, n)
+    ws = workspace(nb, X.device)
+    _check(lib.gm_newton_schulz(B, m, n, _ptr(X), _DT[X.dtype], abc_table(abc, T), T, eps,
+                                _ptr(O), _DT[out_dtype], _ptr(ws), nb, _stream()),
+           "gm_newton_schulz")
+    return O
+
+
+def gram_ns(X, abc=None, T=5, restart_after=(2,), eps=1e-7, out_dtype=torch.float32):
+    B, m, n = _bmn(X)
+    O = torch.empty((B, m, n), dtype=out_dtype, device=X.device)
+    nb = workspace_bytes(GM_OP_GRAM_NS, B, m, n)
+    ws = workspace(nb, X.device)
+    rl = list(restart_after)
+    rarr = (c_int * max(1, len(rl)))(*rl) if rl else None
+    _check(lib.gm_gram_ns(B, m, n, _ptr(X), _DT[X.dtype], abc_table(abc, T), T, rarr, len(rl),
+                          eps, _ptr(O), _DT[out_dtype], _ptr(ws), nb, _stream()), "gm_gram_ns")
+    return O
+
+
+def ns_flops(ns, m, n, T=5, restart_after=(2,)):
+    rl = list(restart_after) if ns == GM_NS_GRAM else []
+    rarr = (c_int * max(1, len(rl)))(*rl) if rl else None
+    f = ctypes.c_double()
+    cnt = c_int()
+    _check(lib.gm_ns_flops(ns, m, n, T, rarr, len(rl), ctypes.byref(f), ctypes.byref(cnt)),
+           "gm_ns_flops")
+    return f.value, cnt.value
+
+
+def device_errors():
+    _check(lib.gm_device_errors(_stream()), "gm_device_errors")
+
+
+@dataclass
+class GraspState:
+    """Device tensors of the quantized momentum of B same-shape matrices."""
+    codes4: torch.Tensor
+    rscale: torch.Tensor
+    cscale: torch.Tensor
+    P8: torch.Tensor
+    Pscale: torch.Tensor
+    R8: torch.Tensor
+    Rscale: torch.Tensor
+    step: torch.Tensor
+    dev_status: torch.Tensor
+
+    @staticmethod
+    def zeros(B, m, n, k, device=None):
+        d = device or torch.device("cuda")
+        mb, nb = -(-m // GRID_BLOCK), -(-n // GRID_BLOCK)
+        z = lambda shape, dt: torch.zeros(shape, dtype=dt, device=d)   # noqa: E731
+        return GraspState(z((B, m, n // 2), torch.uint8), z((B, m, nb), torch.float32),
+                          z((B, mb, n), torch.float32), z((B, m, k), torch.int8),
+                          z((B, k), torch.float32), z((B, n, k), torch.int8),
+                          z((B, k), torch.float32), z((1,), torch.int64), z((1,), torch.int32))
+
+    def tensors(self):
+        return [self.codes4, self.rscale, self.cscale, self.P8, self.Pscale, self.R8,
+                self.Rscale, self.step, self.dev_status]
+
+    def c_struct(self):
+        return GraspStateC(*[t.data_ptr() for t in self.tensors()])
+
+    def clone(self):
+        return GraspState(*[t.clone() for t in self.tensors()])
+
+
+class GraspStep:
+    """Marshals one gm_grasp_step call for a fixed shape batch."""
+
+    def __init__(self, B, m, n, k, mu=0.95, eta=0.02, wd=0.0, T=5, ns=GM_NS_STANDARD, abc=None,
+                 restart_after=(2,), eps=1e-7, seed=0, device=None, ws=None):
+        self.B, self.m, self.n, self.k = B, m, n, k
+        self._abc = abc_table(abc, T)
+        rl = list(restart_after) if ns == GM_NS_GRAM else []
+        self._rarr = (c_int * max(1, len(rl)))(*rl)
+        self.params = GraspParams(mu, eta, wd, k, T, ns,
+                                  ctypes.cast(self._abc, ctypes.POINTER(c_float)) if self._abc else None,
+                                  ctypes.cast(self._rarr, ctypes.POINTER(c_int)) if rl else None,
+                                  len(rl), eps, seed)
+        self.ws_bytes = workspace_bytes(GM_OP_GRASP_STEP, B, m, n, k, ns)
+        if ws is None:
+            ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device or torch.device("cuda"))
+        self.ws = ws
+        lay = GraspWsLayout()
+        _check(lib.gm_grasp_workspace_layout(B, m, n, k, ns, ctypes.byref(lay)),
+               "gm_grasp_workspace_layout")
+        self.layout = lay
+        self.ns = ns
+
+    def __call__(self, state: GraspState, W, G):
+        st = state.c_struct()
+        _check(lib.gm_grasp_step(self.B, self.m, self.n, ctypes.byref(self.params), ctypes.byref(st),
+                                 _ptr(W), _ptr(G), _DT[G.dtype], _ptr(self.ws), self.ws_bytes,
+                                 _stream()), "gm_grasp_step")
+
+    # stage buffers inside the workspace (views; valid after the step ran)
+    def _view(self, off, shape, dtype):
+        nbytes = 1
+        for s in shape:
+            nbytes *= s
+        nbytes *= torch.empty((), dtype=dtype).element_size()
+        return self.ws[off:off + nbytes].view(dtype).view(shape)
+
+    def stage_M(self):
+        return self._view(self.layout.M, (self.B, self.m, self.n), torch.float32)
+
+    def stage_Q(self):
+        return self._view(self.layout.Q, (self.B, self.n, self.k), torch.float32)
+
+    def stage_P(self):
+        return self._view(self.layout.P, (self.B, self.m, self.k), torch.float32)
+
+    def stage_R(self):
+        return self._view(self.layout.R, (self.B, self.n, self.k), torch.float32)
+
+    def stage_scale(self):
+        return self._view(self.layout.scale, (self.B,), torch.float32)
+
+    def stage_X(self):
+        N, Mp = min(self.m, self.n), max(self.m, self.n)
+        dt = torch.float16 if self.ns == GM_NS_GRAM else torch.bfloat16
+        return self._view(self.layout.X, (self.B, N, Mp), dt)

@@ -1,0 +1,234 @@
+/*
+ * libgmuon -- one 4-bit-Muon-GRASP optimizer step on an NVIDIA B200 (sm_100a).
+ *
+ * C ABI. Every pointer argument is a DEVICE pointer unless marked "host".
+ * All matrices are row-major and batch-contiguous: a call operates on B
+ * same-shape matrices stored back to back (batch stride = rows * cols).
+ * Shapes: m, n multiples of 16, 16 <= m, n <= 65536; top rank 1 <= k <= 32.
+ * The 4-bit grid uses fixed 128 x 128 blocks (ragged edge blocks allowed).
+ *
+ * Ownership: the caller allocates every buffer (typically torch tensors) and
+ * keeps it alive until the stream work completes. The library never
+ * allocates or frees device memory and keeps no per-call device state.
+ *
+ * Execution: every call enqueues work on `stream` and returns without
+ * synchronising. Argument errors are detected on the host before any launch
+ * and return GM_E_ARG (nothing is enqueued). A CUDA launch error returns
+ * GM_E_CUDA. Device-side conditions (non-finite input, a bounded wait that
+ * ran out) are reported through `dev_status` words or gm_device_errors().
+ *
+ * Sources (cited per entry point):
+ *  [GRASP]  "Achieving low-bit Muon through subspace preservation and grid
+ *           quantization" (ICLR 2026 paper note)
+ *  [LiMuon] "LiMuon: Light and Fast Muon Optimizer for Large Models" (note)
+ *  [GramNS] "优化器 (3)（Gram Newton-Schulz）" (blog post on Gram NS)
+ */
+#ifndef GMUON_H
+#define GMUON_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GMUON_VERSION 1
+#define GM_GRID_BLOCK 128
+#define GM_MAX_K 32
+#define GM_MAX_T 16
+
+/* Same underlying type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* gm_stream_t;
+
+typedef int gm_status;
+enum {
+  GM_OK = 0,
+  GM_E_ARG = -1,          /* bad shape, pointer, dtype or parameter */
+  GM_E_CUDA = -2,         /* a CUDA runtime call or launch failed */
+  GM_E_NONFINITE = -3,    /* NaN/Inf in G or in the rebuilt momentum (device) */
+  GM_E_WORKSPACE = -4,    /* workspace pointer NULL or smaller than required */
+  GM_E_UNSUPPORTED = -5,  /* device is not sm_100 */
+  GM_E_TIMEOUT = -6       /* a kernel's bounded wait ran out (device) */
+};
+
+typedef enum { GM_F32 = 0, GM_BF16 = 1, GM_F16 = 2 } gm_dtype;
+typedef enum { GM_NS_STANDARD = 0, GM_NS_GRAM = 1 } gm_ns_mode;
+typedef enum {
+  GM_OP_MOMENTUM_POWERIT = 1,
+  GM_OP_NEWTON_SCHULZ = 2,
+  GM_OP_GRAM_NS = 3,
+  GM_OP_GRASP_STEP = 4
+} gm_op;
+
+/* Human-readable name of a status code (static string). */
+const char* gm_status_string(gm_status s);
+/* Detail of the last host-side error on the calling thread (static per thread). */
+const char* gm_last_error(void);
+int gm_version(void);
+
+/*
+ * Workspace bytes needed by `op` for B matrices of m x n with top rank k.
+ * `ns_mode` matters for GM_OP_GRASP_STEP only. Returns 0 on bad arguments.
+ * The workspace must be 256-byte aligned.
+ */
+size_t gm_workspace_bytes(int op, int B, int m, int n, int k, int ns_mode);
+
+/*
+ * Rebuild the previous momentum from the stored low-bit state
+ * [GRASP, worked step, step 1]:
+ *   M[i][j] = (q4_ij / 7) * s_ij + sum_l (p_il / 127 * Pscale_l)(r_jl / 127 * Rscale_l)
+ * with s_ij = min(rscale[i][j/128], cscale[i/128][j]).
+ *   codes4  uint8 [B][m][n/2]  two's-complement nibbles, low nibble = even col
+ *   rscale  f32   [B][m][ceil(n/128)]   cscale f32 [B][ceil(m/128)][n]
+ *   P8 int8 [B][m][k], Pscale f32 [B][k], R8 int8 [B][n][k], Rscale f32 [B][k]
+ *   M_out   f32   [B][m][n]
+ * k = 0 rebuilds the residual only (P8..Rscale may be NULL).
+ */
+gm_status gm_dequant_rebuild(int B, int m, int n, int k,
+                             const uint8_t* codes4, const float* rscale, const float* cscale,
+                             const int8_t* P8, const float* Pscale,
+                             const int8_t* R8, const float* Rscale,
+                             float* M_out, gm_stream_t stream);
+
+/*
+ * Momentum update and one warm-started power iteration
+ * [GRASP, key design 1; worked step, steps 2-4]:
+ *   M = mu * M_prev + G
+ *   Q[:, l] = R_prev[:, l] / |R_prev[:, l]|   (Rademacher +-1/sqrt(n) column when
+ *             R_prev is NULL or the column is zero; sign = top bit of
+ *             splitmix64(seed ^ b<<48 ^ j<<16 ^ l), b = index in the batch)
+ *   P = orth(M Q)  (thin QR, positive diagonal; a column whose residual is
+ *                   <= 1e-6 * max column norm of M Q is zero)
+ *   R = M^T P
+ *   M_prev f32 [B][m][n] (NULL: zero), G [B][m][n] of dtype gdt (f32/bf16/f16),
+ *   R_prev f32 [B][n][k] or NULL, M_out f32 [B][m][n], P_out f32 [B][m][k],
+ *   R_out f32 [B][n][k]; ws >= gm_workspace_bytes(GM_OP_MOMENTUM_POWERIT, ...).
+ */
+gm_status gm_momentum_powerit(int B, int m, int n, int k, float mu,
+                              const float* M_prev, const void* G, gm_dtype gdt,
+                              const float* R_prev, uint64_t seed,
+                              float* M_out, float* P_out, float* R_out,
+                              void* ws, size_t ws_bytes, gm_stream_t stream);
+
+/*
+ * 4-bit grid quantization of X - P R^T [GRASP, key design 2, N_grid;
+ * worked step 5]. Per 128 x 128 block: r_i = max_j |x_ij|, c_j = max_i |x_ij|,
+ * s_ij = min(r_i, c_j), q = clamp(rint(fp32(x / s) * 7), -7, 7) (IEEE fp32
+ * division, ties to even), s = 0 -> q = 0.
+ *   X f32 [B][m][n]; P f32 [B][m][k] and R f32 [B][n][k] both NULL (quantize X)
+ *   or both non-NULL (quantize the residual, fp32 FMA); codes4/rscale/cscale as
+ *   in gm_dequant_rebuild (outputs).
+ */
+gm_status gm_grid_quant4(int B, int m, int n, int k, const float* X,
+                         const float* P, const float* R,
+                         uint8_t* codes4, float* rscale, float* cscale, gm_stream_t stream);
+
+/*
+ * 8-bit per-column absmax quantization of P or R [GRASP, worked step 5;
+ * training strategy: INT8 factors]:
+ *   s_l = max_i |x_il|; q = clamp(rint(fp32(x / s_l) * 127), -127, 127); s = 0 -> 0.
+ *   X f32 [B][rows][k] -> codes int8 [B][rows][k], colscale f32 [B][k].
+ */
+gm_status gm_quant8(int B, int rows, int k, const float* X,
+                    int8_t* codes, float* colscale, gm_stream_t stream);
+
+/*
+ * Standard quintic Newton-Schulz [GramNS §1.2, eq. (2); Algorithm 1 first
+ * line for the normalisation; LiMuon key design 3 for the coefficients]:
+ *   wide form Y = X (m <= n) or X^T (m > n); Y <- Y / (|Y|_F + eps);
+ *   T times: A = Y Y^T; B = b A + c A^2; Y <- a Y + B Y;  O = Y (or Y^T).
+ * Operands are bf16 with fp32 accumulation on the tensor cores; X^T-products
+ * that produce a symmetric matrix compute one triangle and mirror it.
+ *   X [B][m][n] of dtype xdt (f32/bf16/f16); abc host f32 [3T] (a_t, b_t, c_t)
+ *   per step, NULL = the constant quintic (3.4445, -4.7750, 2.0315);
+ *   1 <= T <= 16; O [B][m][n] of dtype odt.
+ */
+gm_status gm_newton_schulz(int B, int m, int n, const void* X, gm_dtype xdt,
+                           const float* abc, int T, float eps,
+                           void* O, gm_dtype odt,
+                           void* ws, size_t ws_bytes, gm_stream_t stream);
+
+/*
+ * Stabilized Gram Newton-Schulz [GramNS Algorithm 2; Algorithm 1 with
+ * n_restart = 0]: fp16 operands, fp32 accumulation, a_t added in fp32
+ * epilogues:
+ *   Y <- fp16(Y / (|Y|_F + eps)); R = Y Y^T; Q = I;
+ *   per step: Z = b R + c R^2; Q <- Q Z + a Q; RZ = R Z + a R; R <- Z RZ + a RZ;
+ *   after each step listed in restart_after (host int[n_restart], 1-based,
+ *   < T): Y <- Q Y, R <- Y Y^T, Q <- I.  O = Q Y (transposed back if tall).
+ * Products whose result is not used again are skipped (Q_1 = Z + a I; no R
+ * update on the last step of a block).
+ */
+gm_status gm_gram_ns(int B, int m, int n, const void* X, gm_dtype xdt,
+                     const float* abc, int T, const int* restart_after, int n_restart,
+                     float eps, void* O, gm_dtype odt,
+                     void* ws, size_t ws_bytes, gm_stream_t stream);
+
+/* Hyper-parameters of one GRASP step (host struct). */
+typedef struct {
+  float mu;                  /* momentum coefficient */
+  float eta;                 /* learning rate */
+  float wd;                  /* decoupled weight decay lambda */
+  int k;                     /* top rank, 1..32 */
+  int T;                     /* NS steps, 1..16 */
+  gm_ns_mode ns;             /* standard (bf16) or Gram (fp16) NS */
+  const float* abc;          /* host f32 [3T] or NULL for the constant quintic */
+  const int* restart_after;  /* host, Gram NS only (NULL with n_restart = 0) */
+  int n_restart;
+  float eps;                 /* Frobenius normalisation epsilon (1e-7) */
+  uint64_t seed;             /* Rademacher start vectors */
+} gm_grasp_params;
+
+/* The quantized momentum state [GRASP, worked step, last paragraph];
+ * all device pointers, layouts as in gm_dequant_rebuild. A zero state (all
+ * codes and scales 0, *step = 0) is the state before the first step. */
+typedef struct {
+  uint8_t* codes4;
+  float* rscale;
+  float* cscale;
+  int8_t* P8;
+  float* Pscale;
+  int8_t* R8;
+  float* Rscale;
+  int64_t* step;        /* [1] incremented on device by every completed step */
+  int32_t* dev_status;  /* [1] written by every step: GM_OK, GM_E_NONFINITE or GM_E_TIMEOUT */
+} gm_grasp_state;
+
+/*
+ * One full GRASP step for B same-shape matrices [GRASP, overall framework;
+ * worked step 1-6]:
+ *   rebuild M_{t-1}; warm start Q; M_t = mu M_{t-1} + G; P, R = PowerIter(M_t, Q);
+ *   residual M_t - P R^T -> 4-bit grid codes; P, R -> 8-bit codes (state updated
+ *   in place); O = NS(M_t) (standard or Gram); W <- W - eta (O + wd W).
+ *   W f32 [B][m][n] (in place), G [B][m][n] of dtype gdt.
+ * If G or M_t holds a NaN/Inf, *dev_status = GM_E_NONFINITE and W and the
+ * state are left unchanged (the step counter too).
+ */
+gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* params,
+                        const gm_grasp_state* state, float* W, const void* G, gm_dtype gdt,
+                        void* ws, size_t ws_bytes, gm_stream_t stream);
+
+/* Byte offsets of the stage buffers inside the gm_grasp_step workspace, for
+ * inspection by tests: M f32 [B][m][n]; Q f32 [B][n][k]; P, R f32; X the NS
+ * input (bf16 or fp16, wide form); scale f32 [B] = 1/(|M|_F + eps). */
+typedef struct {
+  size_t M, Q, P, R, X, scale, total;
+} gm_grasp_ws_layout;
+gm_status gm_grasp_workspace_layout(int B, int m, int n, int k, int ns_mode,
+                                    gm_grasp_ws_layout* out);
+
+/* Algorithmic FLOPs (symmetric products counted once) and product count of
+ * the NS schedule this library issues for one matrix [GramNS §1.2, §2.4, §3.4]. */
+gm_status gm_ns_flops(int ns_mode, int m, int n, int T, const int* restart_after,
+                      int n_restart, double* flops, int* products);
+
+/* Synchronises `stream`, then reads and clears the library's device error
+ * word (set when a kernel's bounded wait ran out). Returns GM_OK or
+ * GM_E_TIMEOUT (or GM_E_CUDA). */
+gm_status gm_device_errors(gm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GMUON_H */

@@ -1,0 +1,78 @@
+"""The C-ABI library loads, exports every symbol include/gmuon.h declares, and
+its host-only logic works without a GPU (no compute call is made here)."""
+
+import ctypes
+import re
+
+import pytest
+
+from bit_muon_optimizer_b200 import flops as F
+from bit_muon_optimizer_b200 import gmuon as gm
+
+
+def _declared_functions():
+    src = open(gm.HEADER_PATH).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gm_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared_functions()
+    assert len(names) >= 14
+    for name in names:
+        assert hasattr(gm.lib, name), name
+
+
+def test_version_and_status_strings():
+    assert gm.lib.gm_version() == 1
+    assert gm.lib.gm_status_string(gm.GM_E_NONFINITE) == b"GM_E_NONFINITE"
+    assert gm.lib.gm_status_string(0) == b"GM_OK"
+
+
+def test_workspace_sizes_are_host_only_and_consistent():
+    b1 = gm.workspace_bytes(gm.GM_OP_GRASP_STEP, 1, 256, 512, 8, gm.GM_NS_STANDARD)
+    b2 = gm.workspace_bytes(gm.GM_OP_GRASP_STEP, 2, 256, 512, 8, gm.GM_NS_STANDARD)
+    bg = gm.workspace_bytes(gm.GM_OP_GRASP_STEP, 1, 256, 512, 8, gm.GM_NS_GRAM)
+    assert 0 < b1 < b2 and bg > b1
+    assert gm.workspace_bytes(gm.GM_OP_GRASP_STEP, 1, 250, 512, 8, 0) == 0    # m % 16 != 0
+    assert gm.workspace_bytes(gm.GM_OP_GRASP_STEP, 1, 256, 512, 33, 0) == 0   # k > 32
+    lay = gm.GraspWsLayout()
+    assert gm.lib.gm_grasp_workspace_layout(1, 256, 512, 8, 0, ctypes.byref(lay)) == 0
+    assert lay.total == b1
+    offs = [lay.M, lay.Q, lay.P, lay.R, lay.X, lay.scale]
+    assert all(o % 256 == 0 for o in offs) and len(set(offs)) == len(offs)
+    assert lay.M + 256 * 512 * 4 <= lay.Q
+
+
+@pytest.mark.parametrize("m,n", [(256, 512), (768, 2048), (2048, 768), (4096, 16384)])
+def test_library_ns_schedule_matches_flop_counter(m, n):
+    f, cnt = gm.ns_flops(gm.GM_NS_STANDARD, m, n, 5)
+    assert f == F.ns_standard_flops(m, n, 5) and cnt == 15
+    for restart in [(), (2,), (1, 3)]:
+        f, cnt = gm.ns_flops(gm.GM_NS_GRAM, m, n, 5, restart)
+        assert f == F.gram_ns_flops(m, n, 5, restart)
+        assert cnt == F.gram_ns_gemm_count(5, restart)
+
+
+def test_argument_errors_are_reported_before_any_launch():
+    st = gm.GraspStateC()
+    prm = gm.GraspParams(0.95, 0.02, 0.0, 8, 5, 0, None, None, 0, 1e-7, 0)
+    # NULL state pointers
+    r = gm.lib.gm_grasp_step(1, 256, 512, ctypes.byref(prm), ctypes.byref(st), None, None, 0,
+                             None, 0, None)
+    assert r == gm.GM_E_ARG
+    assert b"NULL" in gm.lib.gm_last_error()
+    # bad shape
+    r = gm.lib.gm_grid_quant4(1, 250, 512, 0, ctypes.c_void_p(256), None, None, ctypes.c_void_p(256),
+                              ctypes.c_void_p(256), ctypes.c_void_p(256), None)
+    assert r == gm.GM_E_ARG
+    # k out of range
+    r = gm.lib.gm_quant8(1, 100, 33, ctypes.c_void_p(256), ctypes.c_void_p(256),
+                         ctypes.c_void_p(256), None)
+    assert r == gm.GM_E_ARG
+    # workspace too small
+    prm2 = gm.GraspParams(0.95, 0.02, 0.0, 8, 5, 0, None, None, 0, 1e-7, 0)
+    p = ctypes.c_void_p(256)
+    st2 = gm.GraspStateC(256, 256, 256, 256, 256, 256, 256, 256, 256)
+    r = gm.lib.gm_grasp_step(1, 256, 512, ctypes.byref(prm2), ctypes.byref(st2), p, p, 0, p, 16, None)
+    assert r == gm.GM_E_WORKSPACE

@@ -1,0 +1,325 @@
+"""CUDA path vs the fp64 oracle, element by element, on seeded inputs.
+
+Tolerances (from the acceptance bar of the method's fixed reading):
+* codes: bit-exact when both sides see identical fp32 inputs; when the GPU
+  forms the residual itself (fp32 FMA vs the oracle's fp64), codes may differ
+  by one step in at most 1e-4 of the elements (rounding-boundary ties);
+* dequantized M, P, R: relative Frobenius error <= 1e-5;
+* NS output: relative Frobenius error <= 2e-2 vs fp64 NS (bf16 standard NS,
+  fp16 Gram NS).
+Sizes span several 128-tiles and a ragged tail (144 = 128 + 16, 272 = 2*128 + 16).
+"""
+
+import pytest
+import torch
+
+import oracle as O
+from bit_muon_optimizer_b200 import workloads as WL
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def rel(a, b):
+    a, b = a.double().cpu(), b.double().cpu()
+    return float((a - b).norm() / b.norm())
+
+
+def _outlier_matrix(B, m, n, seed, std=1e-3, dtype=torch.float32):
+    X = WL.random_matrix((B, m, n), seed, std=std)
+    g = torch.Generator().manual_seed(seed + 1)
+    for b in range(B):
+        rows = torch.randperm(m, generator=g)[:2]
+        cols = torch.randperm(n, generator=g)[:2]
+        X[b, rows, :] *= 10
+        X[b, :, cols] *= 10
+    return X.to(dtype)
+
+
+# ------------------------------------------------------------------ codec
+
+@pytest.mark.parametrize("B,m,n", [(1, 256, 512), (3, 144, 272), (2, 128, 128), (1, 16, 48)])
+def test_grid_quant4_bit_exact(cuda_lib, B, m, n):
+    gm = cuda_lib
+    X = _outlier_matrix(B, m, n, 100 + m)
+    if m >= 144:
+        X[0, 128:, :128] = 0.0                          # an all-zero ragged block
+    codes, rs, cs = gm.grid_quant4(X.to(DEV))
+    torch.cuda.synchronize()
+    for b in range(B):
+        q, r, c = O.grid_quant4(X[b])
+        assert torch.equal(codes[b].cpu(), O.pack_nibbles(q)), f"codes differ in matrix {b}"
+        assert torch.equal(rs[b].cpu(), r)
+        assert torch.equal(cs[b].cpu(), c)
+
+
+def test_grid_quant4_handworked_layout(cuda_lib):
+    """A 16 x 16 matrix quantized in one block: zero block scales -> zero codes,
+    and the packed byte layout (low nibble = even column)."""
+    gm = cuda_lib
+    X = torch.zeros(1, 16, 16)
+    X[0, 0, 0], X[0, 0, 1], X[0, 1, 0] = 1.0, -0.5, 0.25
+    codes, rs, cs = gm.grid_quant4(X.to(DEV))
+    q, r, c = O.grid_quant4(X[0])
+    assert torch.equal(codes[0].cpu(), O.pack_nibbles(q))
+    assert int(codes[0, 0, 0]) == (7 & 0xF) | ((-7 & 0xF) << 4)
+
+
+@pytest.mark.parametrize("k", [8, 32])
+def test_grid_quant4_fused_residual(cuda_lib, k):
+    gm = cuda_lib
+    B, m, n = 2, 272, 400
+    X = _outlier_matrix(B, m, n, 7)
+    P = WL.random_matrix((B, m, k), 8) * 0.05
+    R = WL.random_matrix((B, n, k), 9) * 0.05
+    codes, rs, cs = gm.grid_quant4(X.to(DEV), P.to(DEV), R.to(DEV))
+    torch.cuda.synchronize()
+    for b in range(B):
+        res = (X[b].double() - P[b].double() @ R[b].double().T).float()
+        q, r, c = O.grid_quant4(res)
+        got = O.unpack_nibbles(codes[b].cpu())
+        diff = (got.int() - q.int()).abs()
+        assert int(diff.max()) <= 1
+        assert float((diff > 0).double().mean()) <= 1e-4
+        assert rel(rs[b], r) < 1e-6 and rel(cs[b], c) < 1e-6
+
+
+@pytest.mark.parametrize("rows,k", [(256, 8), (2048, 16), (777, 3), (18944, 32)])
+def test_quant8_bit_exact(cuda_lib, rows, k):
+    gm = cuda_lib
+    X = WL.random_matrix((2, rows, k), rows + k) * torch.logspace(-3, 0, k)
+    X[1, :, 0] = 0.0
+    codes, scale = gm.quant8(X.to(DEV))
+    for b in range(2):
+        q, s = O.quant8(X[b])
+        assert torch.equal(codes[b].cpu(), q)
+        assert torch.equal(scale[b].cpu(), s)
+
+
+def _random_state(B, m, n, k, seed):
+    g = torch.Generator().manual_seed(seed)
+    mb, nb = -(-m // 128), -(-n // 128)
+    return dict(
+        codes4=torch.randint(0, 256, (B, m, n // 2), generator=g, dtype=torch.uint8),
+        rscale=torch.rand((B, m, nb), generator=g) * 1e-2,
+        cscale=torch.rand((B, mb, n), generator=g) * 1e-2,
+        P8=torch.randint(-127, 128, (B, m, k), generator=g, dtype=torch.int8),
+        Pscale=torch.rand((B, k), generator=g),
+        R8=torch.randint(-127, 128, (B, n, k), generator=g, dtype=torch.int8),
+        Rscale=torch.rand((B, k), generator=g) * 1e-2,
+    )
+
+
+@pytest.mark.parametrize("B,m,n,k", [(2, 256, 512, 8), (1, 144, 272, 32), (3, 128, 384, 16)])
+def test_dequant_rebuild(cuda_lib, B, m, n, k):
+    gm = cuda_lib
+    s = _random_state(B, m, n, k, 11)
+    d = {key: v.to(DEV) for key, v in s.items()}
+    M = gm.dequant_rebuild(d["codes4"], d["rscale"], d["cscale"], d["P8"], d["Pscale"], d["R8"],
+                           d["Rscale"])
+    for b in range(B):
+        st = O.GraspState(s["codes4"][b], s["rscale"][b], s["cscale"][b], s["P8"][b],
+                          s["Pscale"][b], s["R8"][b], s["Rscale"][b])
+        assert rel(M[b], O.rebuild_momentum(st)) <= 1e-6
+
+
+# ------------------------------------------------------------ power iteration
+
+@pytest.mark.parametrize("B,m,n,k,warm", [(2, 256, 512, 8, False), (2, 512, 256, 8, True),
+                                          (1, 144, 272, 32, True), (1, 768, 2048, 16, True)])
+def test_momentum_powerit(cuda_lib, B, m, n, k, warm):
+    gm = cuda_lib
+    G = _outlier_matrix(B, m, n, 21, dtype=torch.bfloat16)
+    Mp = _outlier_matrix(B, m, n, 22)
+    Rp = WL.random_matrix((B, n, k), 23) if warm else None
+    M, P, R = gm.momentum_powerit(G.to(DEV), k, mu=0.95, M_prev=Mp.to(DEV),
+                                  R_prev=Rp.to(DEV) if warm else None, seed=1234)
+    torch.cuda.synchronize()
+    for b in range(B):
+        Mo = 0.95 * Mp[b].double() + G[b].double()
+        Rh = Rp[b].double() if warm else torch.zeros(n, k, dtype=torch.float64)
+        Q = O.warm_start(Rh, 1234, b)
+        Po, Ro, _, live = O.power_iteration(Mo, Q)
+        assert all(live)
+        assert rel(M[b], Mo) <= 1e-6
+        assert rel(P[b], Po) <= 1e-5
+        assert rel(R[b], Ro) <= 1e-5
+
+
+def test_powerit_dead_columns(cuda_lib):
+    """Rank-deficient M Q: dead columns are zero in P and R on both sides."""
+    gm = cuda_lib
+    m, n, k = 256, 384, 8
+    U = WL.random_matrix((m, 3), 31, dtype=torch.float64)
+    V = WL.random_matrix((n, 3), 32, dtype=torch.float64)
+    Mo = (U @ V.T) * 1e-3                                   # exact rank 3
+    G = Mo.float().unsqueeze(0)
+    M, P, R = gm.momentum_powerit(G.to(DEV), k, mu=0.0, seed=5)
+    Q = O.warm_start(torch.zeros(n, k, dtype=torch.float64), 5, 0)
+    Po, Ro, _, live = O.power_iteration(G[0].double(), Q)
+    assert sum(live) == 3
+    for l in range(k):
+        if not live[l]:
+            assert float(P[0, :, l].abs().max()) == 0.0
+    assert rel(P[0], Po) <= 1e-5 and rel(R[0], Ro) <= 1e-5
+
+
+# --------------------------------------------------------------- Newton-Schulz
+
+NS_SHAPES = [(2, 256, 512), (2, 512, 256), (1, 384, 384), (2, 144, 400), (1, 768, 2048)]
+
+
+@pytest.mark.parametrize("B,m,n", NS_SHAPES)
+def test_newton_schulz_vs_oracle(cuda_lib, B, m, n):
+    gm = cuda_lib
+    X = _outlier_matrix(B, m, n, 41)
+    Og = gm.newton_schulz(X.to(DEV))
+    for b in range(B):
+        assert rel(Og[b], O.ns_standard(X[b].double())) <= 2e-2
+
+
+@pytest.mark.parametrize("abc", [[(1.0, 0.0, 0.0)], [(0.0, 1.0, 0.0)], [(0.0, 0.0, 1.0)],
+                                 [(0.5, -0.25, 0.125)]])
+@pytest.mark.parametrize("B,m,n", [(2, 256, 512), (1, 400, 144)])
+def test_newton_schulz_single_terms(cuda_lib, abc, B, m, n):
+    """One NS step with one term at a time isolates the three products:
+    a X (epilogue), b X X^T X (X X^T and the MN-major left product), c (XX^T)^2 X."""
+    gm = cuda_lib
+    X = WL.random_matrix((B, m, n), 43)
+    Og = gm.newton_schulz(X.to(DEV), abc=abc, T=1)
+    for b in range(B):
+        assert rel(Og[b], O.ns_standard(X[b].double(), abc=abc, T=1)) <= 1e-2
+
+
+@pytest.mark.parametrize("restart", [(2,), (), (1, 3)])
+@pytest.mark.parametrize("B,m,n", NS_SHAPES)
+def test_gram_ns_vs_oracle(cuda_lib, B, m, n, restart):
+    gm = cuda_lib
+    X = _outlier_matrix(B, m, n, 51)
+    Og = gm.gram_ns(X.to(DEV), restart_after=restart)
+    for b in range(B):
+        ref = O.ns_standard(X[b].double())          # Gram NS equals NS in exact arithmetic
+        assert rel(Og[b], ref) <= 2e-2
+
+
+# ----------------------------------------------------------------- full step
+
+def _to_oracle_state(st, b):
+    return O.GraspState(st.codes4[b].cpu(), st.rscale[b].cpu(), st.cscale[b].cpu(),
+                        st.P8[b].cpu(), st.Pscale[b].cpu(), st.R8[b].cpu(), st.Rscale[b].cpu(),
+                        int(st.step.item()))
+
+
+def _run_teacher_forced(gm, cid, group, B, steps, ns):
+    w = WL.WORKLOADS[cid]
+    g = w.groups[group]
+    m, n, k = g.m, g.n, w.k
+    base = w.group_base(group)
+    nsmode = gm.GM_NS_GRAM if ns == "gram" else gm.GM_NS_STANDARD
+    step = gm.GraspStep(B, m, n, k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=nsmode,
+                        seed=w.seed, device=DEV)
+    st = gm.GraspState.zeros(B, m, n, k, DEV)
+    W = torch.stack([WL.initial_weight(w, base + b, m, n) for b in range(B)]).to(DEV)
+    for t in range(1, steps + 1):
+        G = torch.stack([WL.gradient(w, base + b, t, m, n) for b in range(B)]).to(DEV)
+        before = [_to_oracle_state(st, b) for b in range(B)]
+        W0 = W.clone()
+        step(st, W, G)
+        torch.cuda.synchronize()
+        assert int(st.dev_status.item()) == 0
+        assert int(st.step.item()) == t
+        for b in range(B):
+            r = O.grasp_step(before[b], W0[b].cpu(), G[b].cpu(), mu=w.mu, eta=w.eta, wd=w.wd,
+                             seed=w.seed, b=b, ns=ns, T=w.T)
+            assert rel(step.stage_M()[b], r.M) <= 1e-5
+            assert rel(step.stage_P()[b], r.P) <= 1e-5
+            assert rel(step.stage_R()[b], r.R) <= 1e-5
+            # 8-bit codes: bit-exact on the GPU's own fp32 P and R
+            q, s = O.quant8(step.stage_P()[b].cpu())
+            assert torch.equal(st.P8[b].cpu(), q) and torch.equal(st.Pscale[b].cpu(), s)
+            q, s = O.quant8(step.stage_R()[b].cpu())
+            assert torch.equal(st.R8[b].cpu(), q) and torch.equal(st.Rscale[b].cpu(), s)
+            # 4-bit codes: the GPU forms the residual in fp32
+            got = O.unpack_nibbles(st.codes4[b].cpu())
+            want = O.unpack_nibbles(r.state.codes4)
+            diff = (got.int() - want.int()).abs()
+            assert int(diff.max()) <= 1
+            assert float((diff > 0).double().mean()) <= 1e-4
+            # update direction recovered from W (wd = 0)
+            Og = (W0[b].double() - W[b].double()).cpu() / w.eta
+            assert rel(Og, r.O) <= 2e-2
+
+
+def test_grasp_step_single_fp32_matrix(cuda_lib):
+    """256 x 512 fp32 gradients, k = 8, 3 steps from a zero state."""
+    _run_teacher_forced(cuda_lib, 1, 0, 1, 3, "standard")
+
+
+@pytest.mark.parametrize("ns", ["standard", "gram"])
+def test_grasp_step_llama130m_shapes(cuda_lib, ns):
+    """2048 x 768 (tall) and 768 x 2048 gradients in bf16, k = 16."""
+    _run_teacher_forced(cuda_lib, 2, 1, 2, 2, ns)
+    _run_teacher_forced(cuda_lib, 2, 2, 1, 2, ns)
+
+
+def test_grasp_step_nonfinite_leaves_state_and_weights(cuda_lib):
+    gm = cuda_lib
+    B, m, n, k = 2, 256, 512, 8
+    step = gm.GraspStep(B, m, n, k, device=DEV)
+    st = gm.GraspState.zeros(B, m, n, k, DEV)
+    W = WL.random_matrix((B, m, n), 3).to(DEV)
+    G = WL.random_matrix((B, m, n), 4, std=1e-3).to(DEV)
+    step(st, W, G)
+    torch.cuda.synchronize()
+    snap = st.clone()
+    W1 = W.clone()
+    G[1, 5, 7] = float("nan")
+    step(st, W, G)
+    torch.cuda.synchronize()
+    assert int(st.dev_status.item()) == gm.GM_E_NONFINITE
+    assert torch.equal(W, W1)
+    for a, b in zip(st.tensors(), snap.tensors()):
+        if a is not st.dev_status:
+            assert torch.equal(a, b)
+    # the next finite step proceeds
+    G[1, 5, 7] = 0.0
+    step(st, W, G)
+    torch.cuda.synchronize()
+    assert int(st.dev_status.item()) == 0 and int(st.step.item()) == 2
+
+
+def test_grasp_step_checkpoint_and_batch_consistency(cuda_lib):
+    """5 steps straight == 2 steps, save/load, 3 steps (bit-exact); a batch of 3
+    matrices == each matrix alone (bit-exact)."""
+    gm = cuda_lib
+    w = WL.WORKLOADS[2]
+    m, n, k, B = 768, 768, 16, 3
+    grads = [torch.stack([WL.gradient(w, b, t, m, n) for b in range(B)]).to(DEV) for t in range(1, 6)]
+    W0 = torch.stack([WL.initial_weight(w, b, m, n) for b in range(B)]).to(DEV)
+
+    def run(Bs, idx, st, W, ts):
+        step = gm.GraspStep(Bs, m, n, k, seed=w.seed, device=DEV)
+        for t in ts:
+            step(st, W, grads[t][idx].contiguous())
+        torch.cuda.synchronize()
+
+    stA = gm.GraspState.zeros(B, m, n, k, DEV)
+    WA = W0.clone()
+    run(B, slice(0, B), stA, WA, range(5))
+    stB = gm.GraspState.zeros(B, m, n, k, DEV)
+    WB = W0.clone()
+    run(B, slice(0, B), stB, WB, range(2))
+    saved = {f: t.cpu() for f, t in zip("abcdefghi", stB.tensors())}
+    stC = gm.GraspState(*[saved[f].to(DEV) for f in "abcdefghi"])
+    WC = WB.cpu().to(DEV)
+    run(B, slice(0, B), stC, WC, range(2, 5))
+    assert torch.equal(WA, WC)
+    for a, c in zip(stA.tensors(), stC.tensors()):
+        assert torch.equal(a, c)
+    # one matrix alone (its seed-index b differs, so compare the W of matrix 0 only)
+    st1 = gm.GraspState.zeros(1, m, n, k, DEV)
+    W1 = W0[0:1].clone()
+    run(1, slice(0, 1), st1, W1, range(5))
+    assert torch.equal(W1[0], WA[0])
+    assert torch.equal(st1.codes4[0], stA.codes4[0])
