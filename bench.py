@@ -1,0 +1,431 @@
+"""Benchmark of one GRASP optimizer step over a parameter set, on B200s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--ns standard|gram]
+                    [--impl ours|reference]
+
+A "step" is one full GRASP step (rebuild, momentum, power iteration, 4/8-bit
+re-quantization, Newton-Schulz, weight update) over every matrix of the
+parameter set, with that step's synthetic gradients already resident in HBM.
+Each shape group is one batched gm_grasp_step call; the three calls of a step
+run on three streams and are replayed from a CUDA graph (one graph per step,
+since each step has its own gradient buffer). N > 1 (torchrun): every rank
+steps its own parameter set (weak scaling, no collective on the data path);
+the time is the max over ranks.
+
+Printed (rank 0): one JSON line with value = ms per parameter set for the
+whole job, the NS chain's tensor-core roofline, the codec passes' HBM rate,
+an end-to-end number through host buffers, and the fp64 CPU oracle timed on a
+bounded sample as the CPU baseline.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
+
+from bit_muon_optimizer_b200 import flops as FL  # noqa: E402
+from bit_muon_optimizer_b200 import workloads as WL  # noqa: E402
+
+METRIC = "GRASP-Muon step ms per param set; NS TFLOP/s; (de)quant HBM GB/s vs peak"
+UNIT = "ms/param_set"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.file is None:
+            return None
+        try:
+            with open(self.file.name) as f:
+                rows = [r.split(",") for r in f.read().strip().splitlines() if r.strip()]
+            os.unlink(self.file.name)
+        except Exception:
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def init_dist(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    if world != n_gpus and rank == 0:
+        print(f"warning: --gpus {n_gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_sample_seconds(w: WL.Workload, ns: str, budget_s: float):
+    """Time the fp64 oracle on one matrix of every shape group, step 1 and 2,
+    repeated until ~budget_s; returns (ms per parameter set, sample text, cores)."""
+    import oracle as O
+    per_shape = []
+    t_all = time.perf_counter()
+    for gi, g in enumerate(w.groups):
+        m, n, k = g.m, g.n, w.k
+        b = w.group_base(gi)
+        st = O.zero_state(m, n, k)
+        W = WL.initial_weight(w, b, m, n)
+        times = []
+        t = 1
+        while True:
+            G = WL.gradient(w, b, t, m, n)
+            t0 = time.perf_counter()
+            r = O.grasp_step(st, W, G, mu=w.mu, eta=w.eta, wd=w.wd, seed=w.seed, b=0, ns=ns, T=w.T)
+            times.append(time.perf_counter() - t0)
+            st, W = r.state, r.W.float()
+            t += 1
+            if t > 2 and (time.perf_counter() - t_all) > budget_s * (gi + 1) / len(w.groups):
+                break
+            if t > 6:
+                break
+        per_shape.append((g, statistics.median(times[1:] if len(times) > 1 else times)))
+    ms = 1e3 * sum(g.count * s for g, s in per_shape)
+    sample = ("fp64 oracle, one matrix per shape group ("
+              + ", ".join(f"{g.m}x{g.n}" for g, _ in per_shape)
+              + "), median of its steps 2+, extrapolated by the group counts")
+    return ms, sample, torch.get_num_threads()
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = WL.WORKLOADS[args.config]
+    budget = max(3.0, 90.0 / max(1, args.steps + args.warmup))
+    vals = []
+    sample = ""
+    cores = torch.get_num_threads()
+    for i in range(args.warmup + args.steps):
+        ms, sample, cores = oracle_sample_seconds(w, args.ns, budget)
+        if i >= args.warmup:
+            vals.append(ms)
+    v = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "ns": args.ns, "k": w.k, "matrices": sum(g.count for g in w.groups)},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def build_set(gm, w: WL.Workload, ns_mode: int, rank: int, steps_total: int, dev):
+    groups = []
+    rank_offset = rank * sum(g.count for g in w.groups)
+    for gi, g in enumerate(w.groups):
+        B, m, n = g.count, g.m, g.n
+        base = rank_offset + w.group_base(gi)
+        step = gm.GraspStep(B, m, n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=ns_mode,
+                            seed=w.seed + rank, device=dev)
+        st = gm.GraspState.zeros(B, m, n, w.k, dev)
+        W = torch.empty((B, m, n), dtype=torch.float32, device=dev)
+        for b in range(B):
+            W[b] = WL.initial_weight(w, base + b, m, n, device=dev)
+        grads = []
+        for t in range(1, steps_total + 1):
+            G = torch.empty((B, m, n), dtype=w.gdtype, device=dev)
+            for b in range(B):
+                WL.gradient(w, base + b, t, m, n, device=dev, out=G[b])
+            grads.append(G)
+        groups.append(dict(step=step, st=st, W=W, grads=grads, B=B, m=m, n=n))
+    return groups
+
+
+def run_ours(args, world, rank, local):
+    from bit_muon_optimizer_b200 import gmuon as gm
+    dev = torch.device("cuda", local)
+    w = WL.WORKLOADS[args.config]
+    ns_mode = gm.GM_NS_GRAM if args.ns == "gram" else gm.GM_NS_STANDARD
+    hbm, bf16, bf16_sus, peak_kind = _peaks()
+    total = args.warmup + args.steps
+    groups = build_set(gm, w, ns_mode, rank, total, dev)
+    streams = [torch.cuda.Stream(device=dev) for _ in groups]
+    main = torch.cuda.Stream(device=dev)        # graphs are captured on a side stream
+
+    def one_step(t):
+        ev = torch.cuda.Event()
+        ev.record(main)
+        done = []
+        for g, s in zip(groups, streams):
+            s.wait_event(ev)
+            with torch.cuda.stream(s):
+                g["step"](g["st"], g["W"], g["grads"][t])
+            e = torch.cuda.Event()
+            e.record(s)
+            done.append(e)
+        for e in done:
+            main.wait_event(e)
+
+    # eager warm-up (also sets kernel attributes), then one graph per step
+    main.wait_stream(torch.cuda.current_stream(dev))
+    one_step(0)
+    torch.cuda.synchronize()
+    graphs = []
+    for t in range(1, total):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=main):
+            one_step(t)
+        graphs.append(gr)
+    torch.cuda.synchronize()
+    for t in range(0, args.warmup - 1):
+        graphs[t].replay()
+    torch.cuda.synchronize()
+    barrier(world)
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        barrier(world)
+        start.record(main)
+        for t in range(args.warmup - 1, args.warmup - 1 + args.steps):
+            graphs[t].replay()
+        end.record(main)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms_step = start.elapsed_time(end) / args.steps
+    ms_step = max_over_ranks(ms_step, world)
+    clocks = clk.summary()
+    status = [int(g["st"].dev_status.item()) for g in groups]
+    if any(status):
+        raise RuntimeError(f"device status {status}")
+
+    # ---- NS chain alone (tensor-core roofline): gm_newton_schulz / gm_gram_ns per group
+    ns_ms, ns_flops = 0.0, 0.0
+    for g in groups:
+        Mx = g["step"].stage_M().clone()
+        out = torch.empty_like(Mx)
+        f, _ = gm.ns_flops(ns_mode, g["m"], g["n"], w.T)
+        fn = (lambda: gm.gram_ns(Mx, T=w.T)) if ns_mode == gm.GM_NS_GRAM else (lambda: gm.newton_schulz(Mx, T=w.T))
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        reps = 10
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(reps):
+            fn()
+        s1.record()
+        torch.cuda.synchronize()
+        ns_ms += s0.elapsed_time(s1) / reps
+        ns_flops += f * g["B"]
+        del out
+    ns_tflops = ns_flops / (ns_ms * 1e-3) / 1e12
+
+    # ---- codec HBM passes alone: dequant-rebuild (codes -> fp32 M), grid-quant4 (M - P R^T -> codes)
+    cod_ms, cod_bytes = 0.0, 0.0
+    for g in groups:
+        st, B, m, n, k = g["st"], g["B"], g["m"], g["n"], w.k
+        Mx = g["step"].stage_M()
+        P, R = g["step"].stage_P(), g["step"].stage_R()
+        Mout = torch.empty((B, m, n), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            gm.dequant_rebuild(st.codes4, st.rscale, st.cscale, st.P8, st.Pscale, st.R8, st.Rscale, out=Mout)
+            gm.grid_quant4(Mx, P, R)
+        torch.cuda.synchronize()
+        reps = 10
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(reps):
+            gm.dequant_rebuild(st.codes4, st.rscale, st.cscale, st.P8, st.Pscale, st.R8, st.Rscale, out=Mout)
+            gm.grid_quant4(Mx, P, R)
+        s1.record()
+        torch.cuda.synchronize()
+        cod_ms += s0.elapsed_time(s1) / reps
+        # algorithmic bytes: rebuild reads codes + scales, writes fp32 M; quant reads fp32 M,
+        # writes codes + scales (k(m+n) factor bytes ignored)
+        cod_bytes += 2 * B * m * n * (4 + 0.5 + 0.0625)
+        del Mout
+    codec_gbs = cod_bytes / (cod_ms * 1e-3) / 1e9
+
+    # ---- end to end through host buffers: H2D W and G, the step, D2H W
+    e2e = None
+    if not args.no_e2e:
+        host = []
+        for g in groups:
+            host.append(dict(W=g["W"].cpu().pin_memory(), G=g["grads"][-1].cpu().pin_memory()))
+        h2d = sum(h["W"].numel() * 4 + h["G"].numel() * h["G"].element_size() for h in host)
+        d2h = sum(h["W"].numel() * 4 for h in host)
+        Wd = [torch.empty_like(g["W"]) for g in groups]
+        Gd = [torch.empty_like(g["grads"][-1]) for g in groups]
+        e_steps = max(2, min(args.steps, 5))
+        torch.cuda.synchronize()
+        barrier(world)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(e_steps):
+            for g, h, wd_, gd_ in zip(groups, host, Wd, Gd):
+                wd_.copy_(h["W"], non_blocking=True)
+                gd_.copy_(h["G"], non_blocking=True)
+                g["step"](g["st"], wd_, gd_)
+                h["W"].copy_(wd_, non_blocking=True)
+        s1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        e_ms = max_over_ranks(s0.elapsed_time(s1) / e_steps, world)
+        e2e = {"value": e_ms / world, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
+
+    # ---- kernel count inside the timed region
+    per_call = 10 + gm.ns_flops(ns_mode, 768, 768, w.T)[1]
+    launches = per_call * len(groups) * args.steps
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        ms_cpu, sample, cores = oracle_sample_seconds(w, args.ns, 20.0)
+        cpu = {"value": ms_cpu, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+
+    elements = sum(g["B"] * g["m"] * g["n"] for g in groups)
+    step_flops = sum(gm.ns_flops(ns_mode, g["m"], g["n"], w.T)[0] * g["B"] for g in groups)
+    step_bytes = elements * FL.step_bytes_per_element(2 if w.gdtype != torch.float32 else 4)
+    t_roof = max(step_flops / (bf16 * 1e12), step_bytes / (hbm * 1e9)) * 1e3
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": ms_step / world, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if ns_mode == gm.GM_NS_STANDARD else "f16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "ns": args.ns, "k": w.k,
+                       "shapes": [[g["m"], g["n"], g["B"]] for g in groups],
+                       "elements": elements, "grad_dtype": str(w.gdtype).replace("torch.", ""),
+                       "l2": "per-step working set (G, W, state, fp32 M) > L2; no flush",
+                       "parallelism": f"weak x{world}, one parameter set per rank",
+                       "graph": "one CUDA graph per step, 3 streams"},
+            "roofline": {"bound": "tensor", "achieved": ns_tflops, "peak": bf16, "unit": "TFLOP/s",
+                         "frac": ns_tflops / bf16, "traffic": None,
+                         "kernel": "NS chain (k_gemm tcgen05 products), gm_newton_schulz alone",
+                         "peak_kind": f"{peak_kind} bf16 dense burst"},
+            "ns": {"tflops": ns_tflops, "ms": ns_ms, "flops": ns_flops},
+            "codec": {"gbs": codec_gbs, "peak_gbs": hbm, "frac": codec_gbs / hbm,
+                      "ms": cod_ms, "kernels": "k_rebuild + k_residual_quant4"},
+            "step_roofline": {"ms": t_roof, "frac": t_roof / ms_step, "flops": step_flops,
+                              "bytes": step_bytes},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    # graphs hold no NCCL work; release them before the process group goes
+    del graphs
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=8)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--ns", choices=["standard", "gram"], default="standard")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = init_dist(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -316,40 +316,49 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
             outv[e] = float_to_h16(x, p.f16);
             if (p.D2) out2[e] = float_to_h16(x + ((r == cb + e) ? p.gamma2 : 0.f), p.f16);
           }
+          // Symmetric products: the lower triangle is computed, the upper is its
+          // mirror -- on diagonal tiles too, so the stored result is exactly symmetric.
+          const bool diag = p.sym && ti == tj;
           uint16_t* drow = p.D + (long long)bz * p.d_bs + (long long)r * p.ldd + cb;
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (g * 8 < ncols) {
-              uint4 w;
-              w.x = outv[g * 8 + 0] | ((uint32_t)outv[g * 8 + 1] << 16);
-              w.y = outv[g * 8 + 2] | ((uint32_t)outv[g * 8 + 3] << 16);
-              w.z = outv[g * 8 + 4] | ((uint32_t)outv[g * 8 + 5] << 16);
-              w.w = outv[g * 8 + 6] | ((uint32_t)outv[g * 8 + 7] << 16);
-              *reinterpret_cast<uint4*>(drow + g * 8) = w;
-            }
-          }
-          if (p.D2) {
-            uint16_t* d2row = p.D2 + (long long)bz * p.d_bs + (long long)r * p.ldd + cb;
+          uint16_t* d2row = p.D2 ? p.D2 + (long long)bz * p.d_bs + (long long)r * p.ldd + cb : nullptr;
+          if (!diag) {
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
               if (g * 8 < ncols) {
                 uint4 w;
-                w.x = out2[g * 8 + 0] | ((uint32_t)out2[g * 8 + 1] << 16);
-                w.y = out2[g * 8 + 2] | ((uint32_t)out2[g * 8 + 3] << 16);
-                w.z = out2[g * 8 + 4] | ((uint32_t)out2[g * 8 + 5] << 16);
-                w.w = out2[g * 8 + 6] | ((uint32_t)out2[g * 8 + 7] << 16);
-                *reinterpret_cast<uint4*>(d2row + g * 8) = w;
+                w.x = outv[g * 8 + 0] | ((uint32_t)outv[g * 8 + 1] << 16);
+                w.y = outv[g * 8 + 2] | ((uint32_t)outv[g * 8 + 3] << 16);
+                w.z = outv[g * 8 + 4] | ((uint32_t)outv[g * 8 + 5] << 16);
+                w.w = outv[g * 8 + 6] | ((uint32_t)outv[g * 8 + 7] << 16);
+                *reinterpret_cast<uint4*>(drow + g * 8) = w;
+                if (d2row) {
+                  uint4 w2;
+                  w2.x = out2[g * 8 + 0] | ((uint32_t)out2[g * 8 + 1] << 16);
+                  w2.y = out2[g * 8 + 2] | ((uint32_t)out2[g * 8 + 3] << 16);
+                  w2.z = out2[g * 8 + 4] | ((uint32_t)out2[g * 8 + 5] << 16);
+                  w2.w = out2[g * 8 + 6] | ((uint32_t)out2[g * 8 + 7] << 16);
+                  *reinterpret_cast<uint4*>(d2row + g * 8) = w2;
+                }
+              }
+            }
+          } else {
+            for (int e = 0; e < ncols; ++e) {
+              if (cb + e <= r) {
+                drow[e] = outv[e];
+                if (d2row) d2row[e] = out2[e];
               }
             }
           }
-          if (p.sym && ti != tj) {
-            // mirrored tile: D[c][r]; consecutive lanes write consecutive r
+          if (p.sym) {
+            // mirrored entries D[c][r] (c < r on diagonal tiles); consecutive lanes
+            // write consecutive r
             uint16_t* dcol = p.D + (long long)bz * p.d_bs + r;
             uint16_t* d2col = p.D2 ? p.D2 + (long long)bz * p.d_bs + r : nullptr;
-#pragma unroll 8
             for (int e = 0; e < ncols; ++e) {
-              dcol[(long long)(cb + e) * p.ldd] = outv[e];
-              if (d2col) d2col[(long long)(cb + e) * p.ldd] = out2[e];
+              if (!diag || cb + e < r) {
+                dcol[(long long)(cb + e) * p.ldd] = outv[e];
+                if (d2col) d2col[(long long)(cb + e) * p.ldd] = out2[e];
+              }
             }
           }
         } else {
