@@ -202,6 +202,9 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ GPU arm
 
+GRAD_POOL = 6   # distinct gradient buffers per group, used cyclically step after step
+
+
 def build_set(gm, w: WL.Workload, ns_mode: int, rank: int, steps_total: int, dev):
     groups = []
     rank_offset = rank * sum(g.count for g in w.groups)
@@ -215,7 +218,7 @@ def build_set(gm, w: WL.Workload, ns_mode: int, rank: int, steps_total: int, dev
         for b in range(B):
             W[b] = WL.initial_weight(w, base + b, m, n, device=dev)
         grads = []
-        for t in range(1, steps_total + 1):
+        for t in range(1, min(steps_total, GRAD_POOL) + 1):
             G = torch.empty((B, m, n), dtype=w.gdtype, device=dev)
             for b in range(B):
                 WL.gradient(w, base + b, t, m, n, device=dev, out=G[b])
@@ -249,30 +252,34 @@ def run_ours(args, world, rank, local):
         for e in done:
             main.wait_event(e)
 
-    # eager warm-up (also sets kernel attributes), then one graph per step
+    # eager warm-up (also sets kernel attributes), then one graph per gradient slot
     main.wait_stream(torch.cuda.current_stream(dev))
+    npool = len(groups[0]["grads"])
     one_step(0)
     torch.cuda.synchronize()
     graphs = []
-    for t in range(1, total):
+    for t in range(npool):
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=main):
             one_step(t)
         graphs.append(gr)
     torch.cuda.synchronize()
-    for t in range(0, args.warmup - 1):
-        graphs[t].replay()
+    with torch.cuda.stream(main):
+        for t in range(1, args.warmup):
+            graphs[t % npool].replay()
     torch.cuda.synchronize()
     barrier(world)
 
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
+        time.sleep(0.3)
         torch.cuda.synchronize()
         barrier(world)
-        start.record(main)
-        for t in range(args.warmup - 1, args.warmup - 1 + args.steps):
-            graphs[t].replay()
-        end.record(main)
+        with torch.cuda.stream(main):
+            start.record(main)
+            for t in range(args.warmup, args.warmup + args.steps):
+                graphs[t % npool].replay()
+            end.record(main)
         torch.cuda.synchronize()
         barrier(world)
     ms_step = start.elapsed_time(end) / args.steps
@@ -282,52 +289,68 @@ def run_ours(args, world, rank, local):
     if any(status):
         raise RuntimeError(f"device status {status}")
 
-    # ---- NS chain alone (tensor-core roofline): gm_newton_schulz / gm_gram_ns per group
-    ns_ms, ns_flops = 0.0, 0.0
-    for g in groups:
-        Mx = g["step"].stage_M().clone()
-        out = torch.empty_like(Mx)
-        f, _ = gm.ns_flops(ns_mode, g["m"], g["n"], w.T)
-        fn = (lambda: gm.gram_ns(Mx, T=w.T)) if ns_mode == gm.GM_NS_GRAM else (lambda: gm.newton_schulz(Mx, T=w.T))
-        for _ in range(3):
-            fn()
+    # ---- NS chain alone (tensor-core roofline) and codec passes alone (HBM), each
+    # replayed from a graph with the three groups on their own streams, as in the step
+    def graph_ms(enqueue, reps):
+        def fork():
+            ev = torch.cuda.Event()
+            ev.record(main)
+            done = []
+            for g, s in zip(groups, streams):
+                s.wait_event(ev)
+                with torch.cuda.stream(s):
+                    enqueue(g)
+                e = torch.cuda.Event()
+                e.record(s)
+                done.append(e)
+            for e in done:
+                main.wait_event(e)
+        fork()                                   # eager once (attributes, workspaces)
         torch.cuda.synchronize()
-        reps = 10
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=main):
+            fork()
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record()
-        for _ in range(reps):
-            fn()
-        s1.record()
+        with torch.cuda.stream(main):       # replay on the stream the events are recorded on
+            for _ in range(3):
+                gr.replay()
+            torch.cuda.synchronize()
+            s0.record(main)
+            for _ in range(reps):
+                gr.replay()
+            s1.record(main)
         torch.cuda.synchronize()
-        ns_ms += s0.elapsed_time(s1) / reps
-        ns_flops += f * g["B"]
-        del out
-    ns_tflops = ns_flops / (ns_ms * 1e-3) / 1e12
+        return s0.elapsed_time(s1) / reps
 
-    # ---- codec HBM passes alone: dequant-rebuild (codes -> fp32 M), grid-quant4 (M - P R^T -> codes)
-    cod_ms, cod_bytes = 0.0, 0.0
     for g in groups:
-        st, B, m, n, k = g["st"], g["B"], g["m"], g["n"], w.k
-        Mx = g["step"].stage_M()
-        P, R = g["step"].stage_P(), g["step"].stage_R()
-        Mout = torch.empty((B, m, n), dtype=torch.float32, device=dev)
-        for _ in range(3):
-            gm.dequant_rebuild(st.codes4, st.rscale, st.cscale, st.P8, st.Pscale, st.R8, st.Rscale, out=Mout)
-            gm.grid_quant4(Mx, P, R)
-        torch.cuda.synchronize()
-        reps = 10
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record()
-        for _ in range(reps):
-            gm.dequant_rebuild(st.codes4, st.rscale, st.cscale, st.P8, st.Pscale, st.R8, st.Rscale, out=Mout)
-            gm.grid_quant4(Mx, P, R)
-        s1.record()
-        torch.cuda.synchronize()
-        cod_ms += s0.elapsed_time(s1) / reps
-        # algorithmic bytes: rebuild reads codes + scales, writes fp32 M; quant reads fp32 M,
-        # writes codes + scales (k(m+n) factor bytes ignored)
-        cod_bytes += 2 * B * m * n * (4 + 0.5 + 0.0625)
-        del Mout
+        g["Mx"] = g["step"].stage_M().clone()
+        g["Mout"] = torch.empty_like(g["Mx"])
+        g["O"] = torch.empty_like(g["Mx"])
+        g["ws_ns"] = torch.empty(gm.workspace_bytes(gm.GM_OP_GRAM_NS if ns_mode == gm.GM_NS_GRAM
+                                                    else gm.GM_OP_NEWTON_SCHULZ, g["B"], g["m"], g["n"]),
+                                 dtype=torch.uint8, device=dev)
+        g["codes"] = (torch.empty_like(g["st"].codes4), torch.empty_like(g["st"].rscale),
+                      torch.empty_like(g["st"].cscale))
+
+    def ns_enqueue(g):
+        if ns_mode == gm.GM_NS_GRAM:
+            gm.gram_ns(g["Mx"], T=w.T, out=g["O"], ws=g["ws_ns"])
+        else:
+            gm.newton_schulz(g["Mx"], T=w.T, out=g["O"], ws=g["ws_ns"])
+
+    def codec_enqueue(g):
+        st = g["st"]
+        gm.dequant_rebuild(st.codes4, st.rscale, st.cscale, st.P8, st.Pscale, st.R8, st.Rscale,
+                           out=g["Mout"])
+        gm.grid_quant4(g["Mx"], g["step"].stage_P(), g["step"].stage_R(), out=g["codes"])
+
+    ns_ms = graph_ms(ns_enqueue, 20)
+    ns_flops = sum(gm.ns_flops(ns_mode, g["m"], g["n"], w.T)[0] * g["B"] for g in groups)
+    ns_tflops = ns_flops / (ns_ms * 1e-3) / 1e12
+    cod_ms = graph_ms(codec_enqueue, 20)
+    # algorithmic bytes: rebuild reads codes + scales and writes fp32 M; quant reads fp32 M
+    # and writes codes + scales (the k (m + n) factor bytes are ignored)
+    cod_bytes = sum(2 * g["B"] * g["m"] * g["n"] * (4 + 0.5 + 0.0625) for g in groups)
     codec_gbs = cod_bytes / (cod_ms * 1e-3) / 1e9
 
     # ---- end to end through host buffers: H2D W and G, the step, D2H W
@@ -383,10 +406,11 @@ def run_ours(args, world, rank, local):
                        "elements": elements, "grad_dtype": str(w.gdtype).replace("torch.", ""),
                        "l2": "per-step working set (G, W, state, fp32 M) > L2; no flush",
                        "parallelism": f"weak x{world}, one parameter set per rank",
-                       "graph": "one CUDA graph per step, 3 streams"},
+                       "graph": "one CUDA graph per gradient slot, 3 streams",
+                       "grad_pool": GRAD_POOL},
             "roofline": {"bound": "tensor", "achieved": ns_tflops, "peak": bf16, "unit": "TFLOP/s",
                          "frac": ns_tflops / bf16, "traffic": None,
-                         "kernel": "NS chain (k_gemm tcgen05 products), gm_newton_schulz alone",
+                         "kernel": "NS chain (k_gemm tcgen05 products) of all groups, graph-replayed alone",
                          "peak_kind": f"{peak_kind} bf16 dense burst"},
             "ns": {"tflops": ns_tflops, "ms": ns_ms, "flops": ns_flops},
             "codec": {"gbs": codec_gbs, "peak_gbs": hbm, "frac": codec_gbs / hbm,
@@ -406,8 +430,8 @@ def run_ours(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=8)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", type=int, default=2)
     ap.add_argument("--ns", choices=["standard", "gram"], default="standard")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")

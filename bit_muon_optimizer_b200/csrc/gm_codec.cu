@@ -72,19 +72,19 @@ __global__ void __launch_bounds__(kThreads) k_warm_start(int n, int k, const int
   if (t < k) {
     double s = 0.0;
     for (int g = 0; g < groups; ++g) s += red[g * k + t];
-    nrm2[t] = s;
+    nrm2[t] = s > 0.0 ? 1.0 / sqrt(s) : 0.0;   // inverse column norm; 0 marks a zero column
   }
   __syncthreads();
   const float rad = (float)(1.0 / sqrt((double)n));
   for (long long e = t; e < (long long)n * k; e += kThreads) {
     const int j = (int)(e / k), l = (int)(e % k);
-    const double s2 = nrm2[l];
+    const double inv = nrm2[l];
     float q;
-    if (s2 == 0.0) {
+    if (inv == 0.0) {
       const uint64_t ctr = seed ^ ((uint64_t)b << 48) ^ ((uint64_t)j << 16) ^ (uint64_t)l;
       q = (splitmix64(ctr) >> 63) ? -rad : rad;
     } else {
-      q = (float)((double)rhat(j, l) / sqrt(s2));
+      q = (float)((double)rhat(j, l) * inv);
     }
     Q[off + e] = q;
   }

@@ -168,6 +168,219 @@ __device__ __forceinline__ void tri_tile(int x, int& ti, int& tj) {
   tj = x - i * (i + 1) / 2;
 }
 
+// ------------------------------------------------------------------ epilogue
+// Staging layout in the (then idle) pipeline shared memory:
+//   EPI_STORE : sC [BM][BN + 8] 16-bit (C tile in, output tile out, in place)
+//               sT [BN][BM + 8] 16-bit (transposed output, for mirrored stores)
+//   otherwise : sF [BM][BN + 4] fp32 output values, then sC as above for C.
+template <int BN>
+__host__ __device__ constexpr uint32_t smem_data_bytes() {
+  constexpr uint32_t ring = kStages * (BM * BK * 2 + BN * BK * 2);
+  constexpr uint32_t st = BM * (BN + 8) * 2 + BN * (BM + 8) * 2;
+  constexpr uint32_t out = BM * (BN + 4) * 4 + BM * (BN + 8) * 2;
+  constexpr uint32_t epi = st > out ? st : out;
+  return ring > epi ? ring : epi;
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ void unpack8(const uint4 w, bool f16, float (&o)[8]) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    o[2 * e] = h16_to_float(u[e] & 0xFFFF, f16);
+    o[2 * e + 1] = h16_to_float(u[e] >> 16, f16);
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float (&v)[8], bool f16) {
+  uint32_t u[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    u[e] = (uint32_t)float_to_h16(v[2 * e], f16) | ((uint32_t)float_to_h16(v[2 * e + 1], f16) << 16);
+  return make_uint4(u[0], u[1], u[2], u[3]);
+}
+
+template <int BN>
+__device__ __forceinline__ void epilogue(const GemmParams& p, uint8_t* base, uint32_t tmem,
+                                         bool ok, int ti, int tj, int bz, int warp, int lane,
+                                         uint16_t* d2diag) {
+  constexpr int SP = BN + 8;          // 16-bit row stride of sC (16-byte multiple)
+  constexpr int TP = BM + 8;          // 16-bit row stride of sT
+  constexpr int FP = BN + 4;          // fp32 row stride of sF
+  const int et = threadIdx.x - 64;    // 0..127 over the four epilogue warps
+  const int q = warp & 3;             // TMEM lane quarter this warp may access
+  const int rr = q * 32 + lane;       // tile row owned by this thread
+  const int r0 = ti * BM, c0 = tj * BN;
+  const int r = r0 + rr;
+  const bool f16 = p.f16 != 0;
+  const bool store_mode = p.mode == EPI_STORE;
+  float* sF = reinterpret_cast<float*>(base);
+  uint16_t* sC = reinterpret_cast<uint16_t*>(store_mode ? base : base + BM * FP * 4);
+  uint16_t* sT = reinterpret_cast<uint16_t*>(base) + BM * SP;
+  const int rows_valid = min(BM, p.M - r0);
+  const int cols_valid = min(BN, p.N - c0);   // multiple of 16
+  const bool use_c = ok && p.C && p.beta != 0.f;
+
+  // 1. C tile -> sC (coalesced 16-byte loads)
+  if (use_c) {
+    const uint16_t* cbase = p.C + (long long)bz * p.c_bs + (long long)r0 * p.ldc + c0;
+    constexpr int CPR = BN / 8;   // 16-byte chunks per row
+    for (int idx = et; idx < BM * CPR; idx += 128) {
+      const int row = idx / CPR, cc = idx % CPR;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (row < rows_valid && cc * 8 < cols_valid)
+        v = *reinterpret_cast<const uint4*>(cbase + (long long)row * p.ldc + cc * 8);
+      *reinterpret_cast<uint4*>(sC + row * SP + cc * 8) = v;
+    }
+  }
+  epi_bar();
+
+  // 2. TMEM -> registers -> epilogue math -> staging
+  if (ok) {
+#pragma unroll 1
+    for (int cb = 0; cb < BN; cb += 32) {
+      float v[32];
+      __syncwarp();
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)cb, v);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        float cin[8];
+        if (use_c) unpack8(*reinterpret_cast<const uint4*>(sC + rr * SP + cb + g * 8), f16, cin);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float x = p.alpha * v[g * 8 + e];
+          if (use_c) x = fmaf(p.beta, cin[e], x);
+          v[g * 8 + e] = x;
+        }
+      }
+      if (store_mode) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            x[e] = v[g * 8 + e];
+            const int c = c0 + cb + g * 8 + e;
+            if (c == r) {
+              x[e] += p.gamma;
+              if (p.D2) d2diag[rr] = float_to_h16(x[e] + p.gamma2, f16);
+            }
+          }
+          *reinterpret_cast<uint4*>(sC + rr * SP + cb + g * 8) = pack8(x, f16);
+          if (p.sym) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sT[(cb + g * 8 + e) * TP + rr] = float_to_h16(x[e], f16);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          *reinterpret_cast<float4*>(sF + rr * FP + cb + g * 4) =
+              make_float4(v[g * 4], v[g * 4 + 1], v[g * 4 + 2], v[g * 4 + 3]);
+      }
+    }
+  }
+  epi_bar();
+  if (!ok) return;
+  (void)r;
+
+  // 3. staging -> global (coalesced)
+  if (store_mode) {
+    constexpr int CPR = BN / 8;
+    const bool diag = p.sym && ti == tj;
+    uint16_t* dbase = p.D + (long long)bz * p.d_bs;
+    uint16_t* d2base = p.D2 ? p.D2 + (long long)bz * p.d_bs : nullptr;
+    // direct tile (on diagonal tiles: lower triangle from sC, upper from sT)
+    for (int idx = et; idx < BM * CPR; idx += 128) {
+      const int row = idx / CPR, cc = idx % CPR;
+      if (row >= rows_valid || cc * 8 >= cols_valid) continue;
+      uint4 w = *reinterpret_cast<const uint4*>(sC + row * SP + cc * 8);
+      if (diag && cc * 8 + 7 > row) {
+        if (cc * 8 > row) {
+          w = *reinterpret_cast<const uint4*>(sT + row * TP + cc * 8);
+        } else {
+          uint16_t hv[8];
+          *reinterpret_cast<uint4*>(hv) = w;
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if (cc * 8 + e > row) hv[e] = sT[row * TP + cc * 8 + e];
+          w = *reinterpret_cast<const uint4*>(hv);
+        }
+      }
+      const long long goff = (long long)(r0 + row) * p.ldd + c0 + cc * 8;
+      *reinterpret_cast<uint4*>(dbase + goff) = w;
+      if (d2base) {
+        if (diag && cc * 8 <= row && row < cc * 8 + 8) {
+          uint16_t hv[8];
+          *reinterpret_cast<uint4*>(hv) = w;
+          hv[row - cc * 8] = d2diag[row];
+          w = *reinterpret_cast<const uint4*>(hv);
+        }
+        *reinterpret_cast<uint4*>(d2base + goff) = w;
+      }
+    }
+    // mirrored tile D[c0 + j][r0 + i] = sT[j][i] (off-diagonal tiles)
+    if (p.sym && !diag) {
+      constexpr int TPR = BM / 8;
+      for (int idx = et; idx < BN * TPR; idx += 128) {
+        const int row = idx / TPR, cc = idx % TPR;   // row: tile column j; cc: chunk of tile rows
+        if (row >= cols_valid || cc * 8 >= rows_valid) continue;
+        const uint4 w = *reinterpret_cast<const uint4*>(sT + row * TP + cc * 8);
+        const long long goff = (long long)(c0 + row) * p.ldd + r0 + cc * 8;
+        *reinterpret_cast<uint4*>(dbase + goff) = w;
+        if (d2base) *reinterpret_cast<uint4*>(d2base + goff) = w;
+      }
+    }
+  } else {
+    const int ld = p.mode == EPI_OUT ? p.ldo : p.ldw;
+    if (!p.transpose_out) {
+      constexpr int QPR = BN / 4;   // float4 per tile row
+      for (int idx = et; idx < BM * QPR; idx += 128) {
+        const int row = idx / QPR, qq = idx % QPR;
+        if (row >= rows_valid || qq * 4 >= cols_valid) continue;
+        const float4 val = *reinterpret_cast<const float4*>(sF + row * FP + qq * 4);
+        const long long off = (long long)(r0 + row) * ld + c0 + qq * 4;
+        if (p.mode == EPI_OUT) {
+          const float vv[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) store_from_float(p.O, (long long)bz * p.o_bs + off + e, p.odt, vv[e]);
+        } else {
+          float4* wp = reinterpret_cast<float4*>(p.W + (long long)bz * p.w_bs + off);
+          float4 w = *wp;
+          w.x -= p.eta * (val.x + p.wd * w.x);
+          w.y -= p.eta * (val.y + p.wd * w.y);
+          w.z -= p.eta * (val.z + p.wd * w.z);
+          w.w -= p.eta * (val.w + p.wd * w.w);
+          *wp = w;
+        }
+      }
+    } else {
+      // natural row = tile column j, natural columns = tile rows i..i+3
+      constexpr int QPR = BM / 4;
+      for (int idx = et; idx < BN * QPR; idx += 128) {
+        const int j = idx / QPR, qq = idx % QPR;
+        if (j >= cols_valid || qq * 4 >= rows_valid) continue;
+        float vv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) vv[e] = sF[(qq * 4 + e) * FP + j];
+        const long long off = (long long)(c0 + j) * ld + r0 + qq * 4;
+        if (p.mode == EPI_OUT) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) store_from_float(p.O, (long long)bz * p.o_bs + off + e, p.odt, vv[e]);
+        } else {
+          float4* wp = reinterpret_cast<float4*>(p.W + (long long)bz * p.w_bs + off);
+          float4 w = *wp;
+          w.x -= p.eta * (vv[0] + p.wd * w.x);
+          w.y -= p.eta * (vv[1] + p.wd * w.y);
+          w.z -= p.eta * (vv[2] + p.wd * w.z);
+          w.w -= p.eta * (vv[3] + p.wd * w.w);
+          *wp = w;
+        }
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 template <int BN, bool B_MN>
 __global__ void __launch_bounds__(kGemmThreads, 2)
@@ -182,12 +395,13 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   extern __shared__ __align__(1024) uint8_t dsm[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + smem_data_bytes<BN>());
   uint64_t* empty = full + kStages;
   uint64_t* accum = empty + kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* consumed = abort_flag + 1;   // k-blocks whose full barrier the MMA warp waited on
+  uint16_t* d2diag = reinterpret_cast<uint16_t*>(consumed + 2);   // [BM] second-output diagonal
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bz = blockIdx.y;
@@ -272,128 +486,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     // ---------------- epilogue
     const bool ok = mbar_wait(smem_u32(accum), 0, p.err);
     tc_fence_after();
-    if (ok) {
-      const int q = warp & 3;               // TMEM lane quarter this warp may access
-      const int r = ti * BM + q * 32 + lane;  // output row of this thread
-      const bool rvalid = r < p.M;
-      const float alpha = p.alpha, beta = p.beta;
-      const bool store = !*abort_flag;
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        float v[32];
-        __syncwarp();
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
-        const int cb = tj * BN + c0;
-        if (!store || !rvalid || cb >= p.N) continue;
-        // N is a multiple of 16: a 32-column chunk is full or half full.
-        const int ncols = min(32, p.N - cb);
-        if (p.mode == EPI_STORE) {
-          const long long cin_off = (long long)bz * p.c_bs + (long long)r * p.ldc + cb;
-          float cin[32];
-          if (p.C && beta != 0.f) {
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              if (g * 8 < ncols) {
-                const uint4 raw = *reinterpret_cast<const uint4*>(p.C + cin_off + g * 8);
-                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  cin[g * 8 + 2 * e] = h16_to_float(w[e] & 0xFFFF, p.f16);
-                  cin[g * 8 + 2 * e + 1] = h16_to_float(w[e] >> 16, p.f16);
-                }
-              }
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) cin[e] = 0.f;
-          }
-          uint16_t outv[32];
-          uint16_t out2[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float x = alpha * v[e] + beta * cin[e];
-            if (r == cb + e) x += p.gamma;
-            outv[e] = float_to_h16(x, p.f16);
-            if (p.D2) out2[e] = float_to_h16(x + ((r == cb + e) ? p.gamma2 : 0.f), p.f16);
-          }
-          // Symmetric products: the lower triangle is computed, the upper is its
-          // mirror -- on diagonal tiles too, so the stored result is exactly symmetric.
-          const bool diag = p.sym && ti == tj;
-          uint16_t* drow = p.D + (long long)bz * p.d_bs + (long long)r * p.ldd + cb;
-          uint16_t* d2row = p.D2 ? p.D2 + (long long)bz * p.d_bs + (long long)r * p.ldd + cb : nullptr;
-          if (!diag) {
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              if (g * 8 < ncols) {
-                uint4 w;
-                w.x = outv[g * 8 + 0] | ((uint32_t)outv[g * 8 + 1] << 16);
-                w.y = outv[g * 8 + 2] | ((uint32_t)outv[g * 8 + 3] << 16);
-                w.z = outv[g * 8 + 4] | ((uint32_t)outv[g * 8 + 5] << 16);
-                w.w = outv[g * 8 + 6] | ((uint32_t)outv[g * 8 + 7] << 16);
-                *reinterpret_cast<uint4*>(drow + g * 8) = w;
-                if (d2row) {
-                  uint4 w2;
-                  w2.x = out2[g * 8 + 0] | ((uint32_t)out2[g * 8 + 1] << 16);
-                  w2.y = out2[g * 8 + 2] | ((uint32_t)out2[g * 8 + 3] << 16);
-                  w2.z = out2[g * 8 + 4] | ((uint32_t)out2[g * 8 + 5] << 16);
-                  w2.w = out2[g * 8 + 6] | ((uint32_t)out2[g * 8 + 7] << 16);
-                  *reinterpret_cast<uint4*>(d2row + g * 8) = w2;
-                }
-              }
-            }
-          } else {
-            for (int e = 0; e < ncols; ++e) {
-              if (cb + e <= r) {
-                drow[e] = outv[e];
-                if (d2row) d2row[e] = out2[e];
-              }
-            }
-          }
-          if (p.sym) {
-            // mirrored entries D[c][r] (c < r on diagonal tiles); consecutive lanes
-            // write consecutive r
-            uint16_t* dcol = p.D + (long long)bz * p.d_bs + r;
-            uint16_t* d2col = p.D2 ? p.D2 + (long long)bz * p.d_bs + r : nullptr;
-            for (int e = 0; e < ncols; ++e) {
-              if (!diag || cb + e < r) {
-                dcol[(long long)(cb + e) * p.ldd] = outv[e];
-                if (d2col) d2col[(long long)(cb + e) * p.ldd] = out2[e];
-              }
-            }
-          }
-        } else {
-          // natural-orientation output O = alpha acc + beta Cin, or the W update
-          const long long cin_off = (long long)bz * p.c_bs + (long long)r * p.ldc + cb;
-          float val[32];
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (g * 8 < ncols) {
-              uint4 raw = make_uint4(0, 0, 0, 0);
-              if (p.C && beta != 0.f) raw = *reinterpret_cast<const uint4*>(p.C + cin_off + g * 8);
-              const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                val[g * 8 + 2 * e] = alpha * v[g * 8 + 2 * e] + beta * h16_to_float(w[e] & 0xFFFF, p.f16);
-                val[g * 8 + 2 * e + 1] = alpha * v[g * 8 + 2 * e + 1] + beta * h16_to_float(w[e] >> 16, p.f16);
-              }
-            }
-          }
-          for (int e = 0; e < ncols; ++e) {
-            const int c = cb + e;
-            long long idx;
-            if (p.transpose_out) idx = (long long)c * (p.mode == EPI_OUT ? p.ldo : p.ldw) + r;
-            else idx = (long long)r * (p.mode == EPI_OUT ? p.ldo : p.ldw) + c;
-            if (p.mode == EPI_OUT) {
-              store_from_float(p.O, (long long)bz * p.o_bs + idx, p.odt, val[e]);
-            } else {
-              float* w = p.W + (long long)bz * p.w_bs + idx;
-              const float wv = *w;
-              *w = wv - p.eta * (val[e] + p.wd * wv);
-            }
-          }
-        }
-      }
-    }
+    epilogue<BN>(p, base, tmem, ok && !*abort_flag, ti, tj, bz, warp, lane, d2diag);
   }
   tc_fence_before();
   __syncthreads();
@@ -443,7 +536,7 @@ bool make_map(CUtensorMap* map, const void* base, bool f16, int rows, int cols, 
 template <int BN, bool B_MN>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int batch,
                         cudaStream_t s) {
-  constexpr int smem = kStages * (BM * BK * 2 + BN * BK * 2) + 1024 + 256;
+  constexpr int smem = smem_data_bytes<BN>() + 1024 + 512;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(k_gemm<BN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -178,13 +178,16 @@ def momentum_powerit(G, k, mu=0.95, M_prev=None, R_prev=None, seed=0):
     return M, P, R
 
 
-def grid_quant4(X, P=None, R=None):
+def grid_quant4(X, P=None, R=None, out=None):
     B, m, n = _bmn(X)
     dev = X.device
     k = 0 if P is None else P.shape[-1]
-    codes = torch.empty((B, m, n // 2), dtype=torch.uint8, device=dev)
-    rs = torch.empty((B, m, -(-n // GRID_BLOCK)), dtype=torch.float32, device=dev)
-    cs = torch.empty((B, -(-m // GRID_BLOCK), n), dtype=torch.float32, device=dev)
+    if out is not None:
+        codes, rs, cs = out
+    else:
+        codes = torch.empty((B, m, n // 2), dtype=torch.uint8, device=dev)
+        rs = torch.empty((B, m, -(-n // GRID_BLOCK)), dtype=torch.float32, device=dev)
+        cs = torch.empty((B, -(-m // GRID_BLOCK), n), dtype=torch.float32, device=dev)
     _check(lib.gm_grid_quant4(B, m, n, k, _ptr(X), _ptr(P), _ptr(R), _ptr(codes), _ptr(rs),
                               _ptr(cs), _stream()), "gm_grid_quant4")
     return codes, rs, cs
@@ -198,22 +201,25 @@ def quant8(X):
     return codes, scale
 
 
-def newton_schulz(X, abc=None, T=5, eps=1e-7, out_dtype=torch.float32):
+def newton_schulz(X, abc=None, T=5, eps=1e-7, out_dtype=torch.float32, out=None, ws=None):
     B, m, n = _bmn(X)
-    O = torch.empty((B, m, n), dtype=out_dtype, device=X.device)
+    O = out if out is not None else torch.empty((B, m, n), dtype=out_dtype, device=X.device)
+    out_dtype = O.dtype
     nb = workspace_bytes(GM_OP_NEWTON_SCHULZ, B, m, n)
-    ws = workspace(nb, X.device)
+    ws = ws if ws is not None else workspace(nb, X.device)
     _check(lib.gm_newton_schulz(B, m, n, _ptr(X), _DT[X.dtype], abc_table(abc, T), T, eps,
                                 _ptr(O), _DT[out_dtype], _ptr(ws), nb, _stream()),
            "gm_newton_schulz")
     return O
 
 
-def gram_ns(X, abc=None, T=5, restart_after=(2,), eps=1e-7, out_dtype=torch.float32):
+def gram_ns(X, abc=None, T=5, restart_after=(2,), eps=1e-7, out_dtype=torch.float32, out=None,
+            ws=None):
     B, m, n = _bmn(X)
-    O = torch.empty((B, m, n), dtype=out_dtype, device=X.device)
+    O = out if out is not None else torch.empty((B, m, n), dtype=out_dtype, device=X.device)
+    out_dtype = O.dtype
     nb = workspace_bytes(GM_OP_GRAM_NS, B, m, n)
-    ws = workspace(nb, X.device)
+    ws = ws if ws is not None else workspace(nb, X.device)
     rl = list(restart_after)
     rarr = (c_int * max(1, len(rl)))(*rl) if rl else None
     _check(lib.gm_gram_ns(B, m, n, _ptr(X), _DT[X.dtype], abc_table(abc, T), T, rarr, len(rl),
