@@ -382,7 +382,7 @@ def run_ours(args, world, rank, local):
                "d2h_bytes_per_step": int(d2h)}
 
     # ---- kernel count inside the timed region
-    per_call = 10 + gm.ns_flops(ns_mode, 768, 768, w.T)[1]
+    per_call = 11 + gm.ns_flops(ns_mode, 768, 768, w.T)[1]   # 11 codec kernels + NS products
     launches = per_call * len(groups) * args.steps
 
     cpu = None

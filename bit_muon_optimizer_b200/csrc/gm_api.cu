@@ -45,7 +45,7 @@ void expand_abc(const float* abc, int T, float* out) {
 }
 
 struct StepLayout {
-  size_t M, Q, P, R, X, scale, norm2, Ppart, Ptil, gram, Tm, Rpart, ns, total;
+  size_t M, Q, P, R, X, scale, norm2, Ppart, Ptil, gram, Tm, Rpart, qnorm, ns, total;
   int csplit, rsplit_b, rsplit_g, ntiles;
 };
 
@@ -71,6 +71,7 @@ StepLayout step_layout(int B, int m, int n, int k, int ns_mode, bool with_ns) {
   L.gram = take(Bz * L.rsplit_g * kz * kz * 8);
   L.Tm = take(Bz * kz * kz * 8);
   L.Rpart = take(Bz * L.rsplit_b * nz * kz * 8);
+  L.qnorm = take(Bz * kz * 4);
   if (with_ns)
     L.ns = take(ns_mode == GM_NS_GRAM ? ns_gram_ws_bytes(B, m, n) : ns_standard_ws_bytes(B, m, n));
   L.total = off;
@@ -232,7 +233,7 @@ gm_status gm_momentum_powerit(int B, int m, int n, int k, float mu, const float*
   double* Tm = reinterpret_cast<double*>(w + L.Tm);
   double* Rpart = reinterpret_cast<double*>(w + L.Rpart);
   float* scale = reinterpret_cast<float*>(w + L.scale);
-  GM_CUDA(launch_warm_start(B, n, k, nullptr, nullptr, R_prev, seed, Q, nullptr, s));
+  GM_CUDA(launch_warm_start(B, n, k, nullptr, nullptr, R_prev, seed, Q, nullptr, nullptr, s));
   GM_CUDA(launch_rebuild(B, m, n, 0, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                          M_prev, mu, G, gdt, M_out, norm2, nullptr, s));
   GM_CUDA(launch_project(B, m, n, k, M_out, Q, Ppart, nullptr, s));
@@ -353,7 +354,8 @@ gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* prm, const g
 
   GM_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
   // worked step 2: warm start from the stored R (read before it is overwritten)
-  GM_CUDA(launch_warm_start(B, n, k, st->R8, st->Rscale, nullptr, prm->seed, Q, status, s));
+  GM_CUDA(launch_warm_start(B, n, k, st->R8, st->Rscale, nullptr, prm->seed, Q,
+                            reinterpret_cast<int*>(w + L.qnorm), status, s));
   // worked steps 1 and 3: rebuild M_{t-1}, M_t = mu M_{t-1} + G
   GM_CUDA(launch_rebuild(B, m, n, k, st->codes4, st->rscale, st->cscale, st->P8, st->Pscale,
                          st->R8, st->Rscale, nullptr, prm->mu, G, gdt, M, norm2, status, s));

@@ -90,6 +90,69 @@ __global__ void __launch_bounds__(kThreads) k_warm_start(int n, int k, const int
   }
 }
 
+// S2 on the stored 8-bit state. Q[:, l] = R^[:, l] / |R^[:, l]| with
+// R^[:, l] = (r8[:, l] / 127) s_l equals sign(s_l) r8[:, l] / |r8[:, l]|, so the
+// column norms are exact integer sums of squared codes. Integer atomics make the
+// sum independent of the order the CTAs arrive in. A zero code column or a zero
+// scale gives the Rademacher column.
+__global__ void __launch_bounds__(kThreads) k_colnorm_int(int n, int k, const int8_t* __restrict__ R8,
+                                                           int* __restrict__ norm2,
+                                                           const int32_t* skip) {
+  if (skip && *skip) return;
+  const int b = blockIdx.y, t = threadIdx.x;
+  __shared__ int red[kThreads];
+  const int groups = kThreads / k;
+  const int j0 = blockIdx.x * kThreads;
+  const int j1 = min(n, j0 + kThreads);
+  int acc = 0;
+  if (t < groups * k) {
+    const int l = t % k, g = t / k;
+    for (int j = j0 + g; j < j1; j += groups) {
+      const int v = R8[((long long)b * n + j) * k + l];
+      acc += v * v;
+    }
+  }
+  red[t] = acc;
+  __syncthreads();
+  if (t < k) {
+    int s = 0;
+    for (int g = 0; g < groups; ++g) s += red[g * k + t];
+    if (s) atomicAdd(&norm2[b * k + t], s);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) k_warm_q(int n, int k, const int8_t* __restrict__ R8,
+                                                      const float* __restrict__ Rscale,
+                                                      const int* __restrict__ norm2, uint64_t seed,
+                                                      float* __restrict__ Q, const int32_t* skip) {
+  if (skip && *skip) return;
+  const int b = blockIdx.y, t = threadIdx.x;
+  __shared__ double inv[kMaxK];
+  if (t < k) {
+    const int s2 = norm2[b * k + t];
+    const float sc = Rscale[b * k + t];
+    inv[t] = (s2 > 0 && sc != 0.f) ? (sc > 0.f ? 1.0 : -1.0) / sqrt((double)s2) : 0.0;
+  }
+  __syncthreads();
+  const float rad = (float)(1.0 / sqrt((double)n));
+  const long long base = (long long)blockIdx.x * kThreads * 4;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const long long e = base + u * kThreads + t;
+    if (e >= (long long)n * k) break;
+    const int j = (int)(e / k), l = (int)(e % k);
+    const double iv = inv[l];
+    float q;
+    if (iv == 0.0) {
+      const uint64_t ctr = seed ^ ((uint64_t)b << 48) ^ ((uint64_t)j << 16) ^ (uint64_t)l;
+      q = (splitmix64(ctr) >> 63) ? -rad : rad;
+    } else {
+      q = (float)((double)R8[(long long)b * n * k + e] * iv);
+    }
+    Q[(long long)b * n * k + e] = q;
+  }
+}
+
 // ------------------------------------------------------------------ S1
 // One 128 x 128 grid block per CTA; thread (ty, tx) owns rows ty + 16 i and
 // columns 4 tx + {0..3}, 64 + 4 tx + {0..3}.
@@ -829,9 +892,19 @@ int ns_prep_parts(int m, int n) { return (int)cdivll((long long)m * n, kPrepChun
 
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_warm_start(int B, int n, int k, const int8_t* R8, const float* Rscale,
-                              const float* Rprev, uint64_t seed, float* Q, const int32_t* skip,
-                              cudaStream_t s) {
-  k_warm_start<<<B, kThreads, 0, s>>>(n, k, R8, Rscale, Rprev, seed, Q, skip);
+                              const float* Rprev, uint64_t seed, float* Q, int* norm2_int,
+                              const int32_t* skip, cudaStream_t s) {
+  if (Rprev || !R8 || !norm2_int) {
+    k_warm_start<<<B, kThreads, 0, s>>>(n, k, R8, Rscale, Rprev, seed, Q, skip);
+    return cudaGetLastError();
+  }
+  cudaError_t e = cudaMemsetAsync(norm2_int, 0, sizeof(int) * (size_t)B * k, s);
+  if (e != cudaSuccess) return e;
+  k_colnorm_int<<<dim3(cdiv(n, kThreads), B), kThreads, 0, s>>>(n, k, R8, norm2_int, skip);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_warm_q<<<dim3((int)cdivll((long long)n * k, kThreads * 4), B), kThreads, 0, s>>>(
+      n, k, R8, Rscale, norm2_int, seed, Q, skip);
   return cudaGetLastError();
 }
 

@@ -40,6 +40,19 @@ __device__ __forceinline__ void store_from_float(void* p, long long idx, int dt,
   else static_cast<__half*>(p)[idx] = __float2half_rn(v);
 }
 
+// Four consecutive elements from fp32 values (idx a multiple of 4, aligned).
+__device__ __forceinline__ void store4_from_float(void* p, long long idx, int dt, float4 v) {
+  if (dt == GM_F32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(p) + idx) = v;
+  } else {
+    const bool f16 = dt == GM_F16;
+    uint2 w;
+    w.x = (uint32_t)float_to_h16(v.x, f16) | ((uint32_t)float_to_h16(v.y, f16) << 16);
+    w.y = (uint32_t)float_to_h16(v.z, f16) | ((uint32_t)float_to_h16(v.w, f16) << 16);
+    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p) + idx) = w;
+  }
+}
+
 // ----------------------------------------------------- splitmix64 (Steele et al.)
 __host__ __device__ inline uint64_t splitmix64(uint64_t x) {
   uint64_t z = x + 0x9E3779B97F4A7C15ull;

@@ -332,49 +332,50 @@ __device__ __forceinline__ void epilogue(const GemmParams& p, uint8_t* base, uin
       }
     }
   } else {
+    // fp32 values -> O (any dtype) or W -= eta (O + wd W), natural orientation.
+    // Eight 16-byte accesses per thread are issued before any is consumed.
     const int ld = p.mode == EPI_OUT ? p.ldo : p.ldw;
-    if (!p.transpose_out) {
-      constexpr int QPR = BN / 4;   // float4 per tile row
-      for (int idx = et; idx < BM * QPR; idx += 128) {
-        const int row = idx / QPR, qq = idx % QPR;
-        if (row >= rows_valid || qq * 4 >= cols_valid) continue;
-        const float4 val = *reinterpret_cast<const float4*>(sF + row * FP + qq * 4);
-        const long long off = (long long)(r0 + row) * ld + c0 + qq * 4;
-        if (p.mode == EPI_OUT) {
-          const float vv[4] = {val.x, val.y, val.z, val.w};
+    constexpr int NB = 8;
+    constexpr int kChunks = BM * BN / 4;
+    const bool tr = p.transpose_out != 0;
+    for (int b0 = 0; b0 < kChunks; b0 += 128 * NB) {
+      float4 val[NB], wv[NB];
+      long long off[NB];
+      bool okc[NB];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) store_from_float(p.O, (long long)bz * p.o_bs + off + e, p.odt, vv[e]);
+      for (int u = 0; u < NB; ++u) {
+        const int idx = b0 + u * 128 + et;
+        int row, col;   // tile coordinates of the first of four consecutive natural elements
+        if (!tr) {
+          row = idx / (BN / 4);
+          col = (idx % (BN / 4)) * 4;
+          okc[u] = row < rows_valid && col < cols_valid;
+          off[u] = (long long)(r0 + row) * ld + c0 + col;
+          if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + row * FP + col);
         } else {
-          float4* wp = reinterpret_cast<float4*>(p.W + (long long)bz * p.w_bs + off);
-          float4 w = *wp;
-          w.x -= p.eta * (val.x + p.wd * w.x);
-          w.y -= p.eta * (val.y + p.wd * w.y);
-          w.z -= p.eta * (val.z + p.wd * w.z);
-          w.w -= p.eta * (val.w + p.wd * w.w);
-          *wp = w;
+          col = idx / (BM / 4);            // tile column = natural row
+          row = (idx % (BM / 4)) * 4;      // tile rows = natural columns
+          okc[u] = col < cols_valid && row < rows_valid;
+          off[u] = (long long)(c0 + col) * ld + r0 + row;
+          if (okc[u])
+            val[u] = make_float4(sF[row * FP + col], sF[(row + 1) * FP + col],
+                                 sF[(row + 2) * FP + col], sF[(row + 3) * FP + col]);
         }
+        if (p.mode == EPI_WUPDATE && okc[u])
+          wv[u] = *reinterpret_cast<const float4*>(p.W + (long long)bz * p.w_bs + off[u]);
       }
-    } else {
-      // natural row = tile column j, natural columns = tile rows i..i+3
-      constexpr int QPR = BM / 4;
-      for (int idx = et; idx < BN * QPR; idx += 128) {
-        const int j = idx / QPR, qq = idx % QPR;
-        if (j >= cols_valid || qq * 4 >= rows_valid) continue;
-        float vv[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) vv[e] = sF[(qq * 4 + e) * FP + j];
-        const long long off = (long long)(c0 + j) * ld + r0 + qq * 4;
+      for (int u = 0; u < NB; ++u) {
+        if (!okc[u]) continue;
         if (p.mode == EPI_OUT) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) store_from_float(p.O, (long long)bz * p.o_bs + off + e, p.odt, vv[e]);
+          store4_from_float(p.O, (long long)bz * p.o_bs + off[u], p.odt, val[u]);
         } else {
-          float4* wp = reinterpret_cast<float4*>(p.W + (long long)bz * p.w_bs + off);
-          float4 w = *wp;
-          w.x -= p.eta * (vv[0] + p.wd * w.x);
-          w.y -= p.eta * (vv[1] + p.wd * w.y);
-          w.z -= p.eta * (vv[2] + p.wd * w.z);
-          w.w -= p.eta * (vv[3] + p.wd * w.w);
-          *wp = w;
+          float4 w = wv[u];
+          w.x -= p.eta * (val[u].x + p.wd * w.x);
+          w.y -= p.eta * (val[u].y + p.wd * w.y);
+          w.z -= p.eta * (val[u].z + p.wd * w.z);
+          w.w -= p.eta * (val[u].w + p.wd * w.w);
+          *reinterpret_cast<float4*>(p.W + (long long)bz * p.w_bs + off[u]) = w;
         }
       }
     }

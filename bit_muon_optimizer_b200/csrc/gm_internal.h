@@ -13,8 +13,9 @@ int backproject_row_splits(int B, int m, int n);
 int gram_row_splits(int B, int m);
 
 // ---- codec / power-iteration kernels (gm_codec.cu) ------------------------
+// Q from the stored 8-bit R (norm2_int: scratch int [B][k]) or from fp32 Rprev.
 cudaError_t launch_warm_start(int B, int n, int k, const int8_t* R8, const float* Rscale,
-                              const float* Rprev, uint64_t seed, float* Q,
+                              const float* Rprev, uint64_t seed, float* Q, int* norm2_int,
                               const int32_t* skip, cudaStream_t s);
 
 // M = mu * Mprev + G where Mprev is either the rebuilt state (codes4 != NULL)
