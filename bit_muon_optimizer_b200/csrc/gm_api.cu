@@ -52,10 +52,10 @@ struct StepLayout {
 StepLayout step_layout(int B, int m, int n, int k, int ns_mode, bool with_ns) {
   StepLayout L;
   memset(&L, 0, sizeof(L));
-  L.csplit = project_col_splits(B, m, n);
+  L.csplit = cdiv(n, kGrid);                        // projection partials: one per column block
   L.rsplit_b = backproject_row_splits(B, m, n);
   L.rsplit_g = gram_row_splits(B, m);
-  L.ntiles = cdiv(m, kGrid) * cdiv(n, kGrid);
+  L.ntiles = rebuild_row_blocks(m) * cdiv(n, kGrid);  // |M|^2 partials
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off += al256(bytes); return o; };
   const size_t Bz = (size_t)B, mz = (size_t)m, nz = (size_t)n, kz = (size_t)k;
@@ -66,7 +66,7 @@ StepLayout step_layout(int B, int m, int n, int k, int ns_mode, bool with_ns) {
   L.X = with_ns ? take(Bz * mz * nz * 2) : 0;
   L.scale = take(Bz * 4);
   L.norm2 = take(Bz * L.ntiles * 8);
-  L.Ppart = take(Bz * L.csplit * mz * kz * 8);
+  L.Ppart = take(Bz * L.csplit * mz * kz * 4);
   L.Ptil = take(Bz * mz * kz * 8);
   L.gram = take(Bz * L.rsplit_g * kz * kz * 8);
   L.Tm = take(Bz * kz * kz * 8);
@@ -207,7 +207,7 @@ gm_status gm_dequant_rebuild(int B, int m, int n, int k, const uint8_t* codes4,
   GM_DEVICE();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   GM_CUDA(launch_rebuild(B, m, n, k, codes4, rscale, cscale, P8, Pscale, R8, Rscale, nullptr, 1.0f,
-                         nullptr, GM_F32, M_out, nullptr, nullptr, s));
+                         nullptr, GM_F32, nullptr, M_out, nullptr, nullptr, nullptr, s));
   return GM_OK;
 }
 
@@ -227,16 +227,15 @@ gm_status gm_momentum_powerit(int B, int m, int n, int k, float mu, const float*
   uint8_t* w = static_cast<uint8_t*>(ws);
   float* Q = reinterpret_cast<float*>(w + L.Q);
   double* norm2 = reinterpret_cast<double*>(w + L.norm2);
-  double* Ppart = reinterpret_cast<double*>(w + L.Ppart);
+  float* Ppart = reinterpret_cast<float*>(w + L.Ppart);
   double* Ptil = reinterpret_cast<double*>(w + L.Ptil);
   double* gram = reinterpret_cast<double*>(w + L.gram);
   double* Tm = reinterpret_cast<double*>(w + L.Tm);
   double* Rpart = reinterpret_cast<double*>(w + L.Rpart);
   float* scale = reinterpret_cast<float*>(w + L.scale);
   GM_CUDA(launch_warm_start(B, n, k, nullptr, nullptr, R_prev, seed, Q, nullptr, nullptr, s));
-  GM_CUDA(launch_rebuild(B, m, n, 0, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-                         M_prev, mu, G, gdt, M_out, norm2, nullptr, s));
-  GM_CUDA(launch_project(B, m, n, k, M_out, Q, Ppart, nullptr, s));
+  GM_CUDA(launch_rebuild(B, m, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                         M_prev, mu, G, gdt, Q, M_out, norm2, Ppart, nullptr, s));
   GM_CUDA(launch_orth(B, m, k, L.csplit, Ppart, Ptil, gram, Tm, norm2, L.ntiles, 1e-7f, scale,
                       P_out, nullptr, s));
   GM_CUDA(launch_backproject(B, m, n, k, M_out, P_out, nullptr, nullptr, false, Rpart, R_out,
@@ -342,7 +341,7 @@ gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* prm, const g
   uint16_t* X = reinterpret_cast<uint16_t*>(w + L.X);
   float* scale = reinterpret_cast<float*>(w + L.scale);
   double* norm2 = reinterpret_cast<double*>(w + L.norm2);
-  double* Ppart = reinterpret_cast<double*>(w + L.Ppart);
+  float* Ppart = reinterpret_cast<float*>(w + L.Ppart);
   double* Ptil = reinterpret_cast<double*>(w + L.Ptil);
   double* gram = reinterpret_cast<double*>(w + L.gram);
   double* Tm = reinterpret_cast<double*>(w + L.Tm);
@@ -357,10 +356,10 @@ gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* prm, const g
   GM_CUDA(launch_warm_start(B, n, k, st->R8, st->Rscale, nullptr, prm->seed, Q,
                             reinterpret_cast<int*>(w + L.qnorm), status, s));
   // worked steps 1 and 3: rebuild M_{t-1}, M_t = mu M_{t-1} + G
+  // (with the projection P~ = M Q of worked step 4 fused in)
   GM_CUDA(launch_rebuild(B, m, n, k, st->codes4, st->rscale, st->cscale, st->P8, st->Pscale,
-                         st->R8, st->Rscale, nullptr, prm->mu, G, gdt, M, norm2, status, s));
-  // worked step 4: P = orth(M Q), R = M^T P
-  GM_CUDA(launch_project(B, m, n, k, M, Q, Ppart, status, s));
+                         st->R8, st->Rscale, nullptr, prm->mu, G, gdt, Q, M, norm2, Ppart, status, s));
+  // worked step 4: P = orth(P~), R = M^T P
   GM_CUDA(launch_orth(B, m, k, L.csplit, Ppart, Ptil, gram, Tm, norm2, L.ntiles, prm->eps, scale,
                       P, status, s));
   GM_CUDA(launch_backproject(B, m, n, k, M, P, scale, X, gramns, Rpart, R, status, s));

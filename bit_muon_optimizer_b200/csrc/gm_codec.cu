@@ -153,216 +153,202 @@ __global__ void __launch_bounds__(kThreads) k_warm_q(int n, int k, const int8_t*
   }
 }
 
-// ------------------------------------------------------------------ S1
-// One 128 x 128 grid block per CTA; thread (ty, tx) owns rows ty + 16 i and
-// columns 4 tx + {0..3}, 64 + 4 tx + {0..3}.
-__global__ void __launch_bounds__(kThreads) k_rebuild(
+// ------------------------------------------------------------------ S1 + S3
+// Rebuild + momentum, fused with the projection P~ = M Q.
+// CTA: 64 rows x 128 columns (half a grid block); thread (ty, tx) owns rows
+// ty + 16 i (i < 4) and columns 4 tx + {0..3}, 64 + 4 tx + {0..3}.
+// Global loads of the tile are issued before the rank-k product. The decoded
+// nibble value q / 7 comes from a 16-entry table filled with IEEE divisions, so it
+// is bit-identical to (float)q / 7.0f. P~ partials of the tile (sum over its 128
+// columns, fp32) go to Ppart[b][bj][row][l]; the orthonormalisation sums the
+// column blocks in fp64 in a fixed order.
+constexpr int kRB = 64;   // rows per rebuild CTA
+
+__device__ __forceinline__ void reduce_scatter16(float (&v)[16], int tx) {
+  // After the four steps lane tx (of a 16-lane group) holds the group sum of v[tx].
+#pragma unroll
+  for (int s = 8; s >= 1; s >>= 1) {
+    const bool up = (tx & s) != 0;
+#pragma unroll
+    for (int j = 0; j < s; ++j) {
+      const float send = up ? v[j] : v[j + s];
+      const float keep = up ? v[j + s] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+}
+
+enum RebuildSrc { SRC_STATE = 0, SRC_DENSE = 1, SRC_ZERO = 2 };
+
+template <int SRC, bool G32>
+__global__ void __launch_bounds__(kThreads, 2) k_rebuild_proj(
     int m, int n, int k, const uint8_t* __restrict__ codes4, const float* __restrict__ rscale,
     const float* __restrict__ cscale, const int8_t* __restrict__ P8,
     const float* __restrict__ Pscale, const int8_t* __restrict__ R8,
     const float* __restrict__ Rscale, const float* __restrict__ Mprev, float mu,
-    const void* __restrict__ G, int gdt, float* __restrict__ M, double* __restrict__ norm2_part,
-    int32_t* status) {
-  const int bj = blockIdx.x, bi = blockIdx.y, b = blockIdx.z;
-  const int nb = gridDim.x, mb = gridDim.y;
-  const int r0 = bi * kGrid, c0 = bj * kGrid;
+    const void* __restrict__ G, int gdt, const float* __restrict__ Q, float* __restrict__ M,
+    double* __restrict__ norm2_part, float* __restrict__ Ppart, int32_t* status) {
+  const int bj = blockIdx.x, bh = blockIdx.y, b = blockIdx.z;
+  const int nb = gridDim.x;
+  const int mb = cdiv(m, kGrid);
+  const int r0 = bh * kRB, c0 = bj * kGrid, bi = r0 / kGrid;
   const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
-  __shared__ __align__(16) float Ps[kMaxK][kGrid];
-  __shared__ __align__(16) float Rs[kMaxK][kGrid];
+  const int kk = SRC == SRC_STATE ? k : 0;
+  const int kq = Q ? ((k + 3) & ~3) : 0;
+  extern __shared__ __align__(16) float sm[];
+  float* Ps = sm;                  // [kk][64]
+  float* Rs = Ps + kk * kRB;       // [kk][128]
+  float* Qs = Rs + kk * kGrid;     // [kq][128]
+  __shared__ float deq4[16];
   __shared__ double red[kThreads / 32];
   const long long mn = (long long)m * n;
-  const bool use_state = (codes4 != nullptr);
-  const int kk = use_state ? k : 0;
+  const bool f16 = gdt == GM_F16;
 
-  for (int e = t; e < kGrid * kk; e += kThreads) {
-    const int rr = e / kk, l = e % kk;
-    const int gi = r0 + rr, gj = c0 + rr;
-    Ps[l][rr] = (gi < m) ? deq8(P8[((long long)b * m + gi) * kk + l], Pscale[b * kk + l]) : 0.f;
-    Rs[l][rr] = (gj < n) ? deq8(R8[((long long)b * n + gj) * kk + l], Rscale[b * kk + l]) : 0.f;
-  }
-  __syncthreads();
-
-  float acc[8][8];
+  // 1. global loads of this thread's 32 elements, all issued up front
+  uint32_t cw[4][2];      // four nibbles per (row, half)
+  float4 mpv[4][2];       // dense M_prev
+  uint2 gw[4][2];         // 16-bit gradient
+  float4 gf[4][2];        // fp32 gradient
+  float rsc[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  for (int l = 0; l < kk; ++l) {
-    const float4 ra = *reinterpret_cast<const float4*>(&Rs[l][4 * tx]);
-    const float4 rb = *reinterpret_cast<const float4*>(&Rs[l][64 + 4 * tx]);
-    const float rv[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float p = Ps[l][ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(p, rv[j], acc[i][j]);
-    }
-  }
-
-  float cs[8];
-#pragma unroll
-  for (int h = 0; h < 2; ++h)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int gj = c0 + 64 * h + 4 * tx + e;
-      cs[4 * h + e] = (use_state && gj < n) ? cscale[((long long)b * mb + bi) * n + gj] : 0.f;
-    }
-
-  float nsq = 0.f;
-  bool bad = false;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < 4; ++i) {
     const int gi = r0 + ty + 16 * i;
-    if (gi >= m) continue;
-    const float rsc = use_state ? rscale[((long long)b * m + gi) * nb + bj] : 0.f;
+    if (SRC == SRC_STATE) rsc[i] = gi < m ? rscale[((long long)b * m + gi) * nb + bj] : 0.f;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int cb = c0 + 64 * h + 4 * tx;
-      if (cb >= n) continue;
+      const bool ok = gi < m && cb < n;
       const long long base = (long long)b * mn + (long long)gi * n + cb;
-      float mp[4];
-      if (use_state) {
-        const uint16_t two = *reinterpret_cast<const uint16_t*>(
-            codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2);
+      if (SRC == SRC_STATE)
+        cw[i][h] = ok ? *reinterpret_cast<const uint16_t*>(codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2) : 0u;
+      if (SRC == SRC_DENSE)
+        mpv[i][h] = ok ? *reinterpret_cast<const float4*>(Mprev + base) : make_float4(0.f, 0.f, 0.f, 0.f);
+      if (G32) gf[i][h] = (ok && G) ? *reinterpret_cast<const float4*>(static_cast<const float*>(G) + base)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      else gw[i][h] = (ok && G) ? *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(G) + base)
+                                : make_uint2(0u, 0u);
+    }
+  }
+  float cs[8];
+  if (SRC == SRC_STATE) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int gj = c0 + 64 * h + 4 * tx + e;
+        cs[4 * h + e] = gj < n ? cscale[((long long)b * mb + bi) * n + gj] : 0.f;
+      }
+  }
+
+  // 2. factors of the tile into shared memory
+  if (t < 16) deq4[t] = __fdiv_rn((float)((t & 8) ? t - 16 : t), 7.0f);
+  for (int e = t; e < kRB * kk; e += kThreads) {
+    const int rr = e / kk, l = e % kk, gi = r0 + rr;
+    Ps[l * kRB + rr] = (gi < m) ? deq8(P8[((long long)b * m + gi) * kk + l], Pscale[b * kk + l]) : 0.f;
+  }
+  for (int e = t; e < kGrid * kk; e += kThreads) {
+    const int cc = e / kk, l = e % kk, gj = c0 + cc;
+    Rs[l * kGrid + cc] = (gj < n) ? deq8(R8[((long long)b * n + gj) * kk + l], Rscale[b * kk + l]) : 0.f;
+  }
+  for (int e = t; e < kGrid * kq; e += kThreads) {
+    const int cc = e / kq, l = e % kq, gj = c0 + cc;
+    Qs[l * kGrid + cc] = (gj < n && l < k) ? Q[((long long)b * n + gj) * k + l] : 0.f;
+  }
+  __syncthreads();
+
+  // 3. rank-k rebuild P^ R^T
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  for (int l = 0; l < kk; ++l) {
+    const float4 ra = *reinterpret_cast<const float4*>(Rs + l * kGrid + 4 * tx);
+    const float4 rb = *reinterpret_cast<const float4*>(Rs + l * kGrid + 64 + 4 * tx);
+    const float rv[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float pv = Ps[l * kRB + ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(pv, rv[j], acc[i][j]);
+    }
+  }
+
+  // 4. M = mu M_prev + G, with M_prev = deq4 + P^R^T (state) or dense
+  float nsq = 0.f;
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int gi = r0 + ty + 16 * i;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int cb = c0 + 64 * h + 4 * tx;
+      const bool ok = gi < m && cb < n;
+      float g[4], mp[4];
+      if (G32) {
+        g[0] = gf[i][h].x; g[1] = gf[i][h].y; g[2] = gf[i][h].z; g[3] = gf[i][h].w;
+      } else {
+        g[0] = h16_to_float(gw[i][h].x & 0xFFFF, f16);
+        g[1] = h16_to_float(gw[i][h].x >> 16, f16);
+        g[2] = h16_to_float(gw[i][h].y & 0xFFFF, f16);
+        g[3] = h16_to_float(gw[i][h].y >> 16, f16);
+      }
+      if (SRC == SRC_STATE) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int q = sext4((two >> (4 * e)) & 0xF);
-          const float s = fminf(rsc, cs[4 * h + e]);
-          mp[e] = __fmul_rn(__fdiv_rn((float)q, 7.0f), s) + acc[i][4 * h + e];
+          const float sc = fminf(rsc[i], cs[4 * h + e]);
+          mp[e] = __fmul_rn(deq4[(cw[i][h] >> (4 * e)) & 0xF], sc) + acc[i][4 * h + e];
         }
-      } else if (Mprev) {
-        const float4 v = *reinterpret_cast<const float4*>(Mprev + base);
-        mp[0] = v.x; mp[1] = v.y; mp[2] = v.z; mp[3] = v.w;
+      } else if (SRC == SRC_DENSE) {
+        mp[0] = mpv[i][h].x; mp[1] = mpv[i][h].y; mp[2] = mpv[i][h].z; mp[3] = mpv[i][h].w;
       } else {
         mp[0] = mp[1] = mp[2] = mp[3] = 0.f;
       }
-      float g[4] = {0.f, 0.f, 0.f, 0.f};
-      if (G) {
-        if (gdt == GM_F32) {
-          const float4 v = *reinterpret_cast<const float4*>(static_cast<const float*>(G) + base);
-          g[0] = v.x; g[1] = v.y; g[2] = v.z; g[3] = v.w;
-        } else {
-          const uint2 raw = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(G) + base);
-          const bool f16 = (gdt == GM_F16);
-          g[0] = h16_to_float(raw.x & 0xFFFF, f16);
-          g[1] = h16_to_float(raw.x >> 16, f16);
-          g[2] = h16_to_float(raw.y & 0xFFFF, f16);
-          g[3] = h16_to_float(raw.y >> 16, f16);
-        }
-      }
-      float4 o;
-      float* ov = &o.x;
+      float o[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float v = __fadd_rn(__fmul_rn(mu, mp[e]), g[e]);
-        ov[e] = v;
-        bad |= !isfinite(v);
-        nsq = fmaf(v, v, nsq);
+        o[e] = ok ? __fadd_rn(__fmul_rn(mu, mp[e]), g[e]) : 0.f;
+        acc[i][4 * h + e] = o[e];        // keep M for the projection
+        bad |= !isfinite(o[e]);
+        nsq = fmaf(o[e], o[e], nsq);
       }
-      *reinterpret_cast<float4*>(M + base) = o;
+      if (ok)
+        *reinterpret_cast<float4*>(M + (long long)b * mn + (long long)gi * n + cb) =
+            make_float4(o[0], o[1], o[2], o[3]);
     }
   }
   const double tot = block_sum_d((double)nsq, red);
-  if (t == 0 && norm2_part) norm2_part[((long long)b * mb + bi) * nb + bj] = tot;
+  if (t == 0 && norm2_part) norm2_part[((long long)b * cdiv(m, kRB) + bh) * nb + bj] = tot;
   if (bad && status) atomicExch(status, GM_E_NONFINITE);
-}
 
-// ------------------------------------------------------------------ S3
-// P~ = M Q. CTA: 64 rows x a contiguous range of 128-column chunks. Thread
-// (rg, lg, jg) owns rows rg + 16 r (r < 4), columns l = 8 lg + {0..7} of P~
-// and the j-slice jg of every chunk; fp32 within a chunk, fp64 across chunks.
-template <int KP>
-__global__ void __launch_bounds__(kThreads) k_project(int m, int n, int k, int csplit,
-                                                       const float* __restrict__ M,
-                                                       const float* __restrict__ Q,
-                                                       double* __restrict__ Ppart,
-                                                       const int32_t* skip) {
-  if (skip && *skip) return;
-  constexpr int RB = 64, CH = 128, LG = KP / 8, JG = kThreads / (16 * LG), JPER = CH / JG;
-  constexpr int MS = CH + 1;   // odd row stride: conflict-free column reads
-  extern __shared__ __align__(16) float smem[];   // RB * MS + CH * KP floats
-  float* Ms = smem;
-  float* Qs = smem + RB * MS;
-  const int rb = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
-  const int t = threadIdx.x, rg = t & 15, lg = (t >> 4) % LG, jg = t / (16 * LG);
-  const int r0 = rb * RB;
-  const int nchunks = cdiv(n, CH);
-  const int per = cdiv(nchunks, csplit);
-  const int ch0 = split * per, ch1 = min(nchunks, ch0 + per);
-  const float* Mb = M + (long long)b * m * n;
-  const float* Qb = Q + (long long)b * n * k;
-
-  double accd[4][8];
+  // 5. projection partials: this tile's share of M Q, four columns of Q at a time
+  if (Q) {
+    for (int l0 = 0; l0 < kq; l0 += 4) {
+      float v[16];
 #pragma unroll
-  for (int r = 0; r < 4; ++r)
+      for (int j = 0; j < 4; ++j) {
+        const float4 qa = *reinterpret_cast<const float4*>(Qs + (l0 + j) * kGrid + 4 * tx);
+        const float4 qb = *reinterpret_cast<const float4*>(Qs + (l0 + j) * kGrid + 64 + 4 * tx);
+        const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-    for (int l = 0; l < 8; ++l) accd[r][l] = 0.0;
-
-  for (int ch = ch0; ch < ch1; ++ch) {
-    const int c0 = ch * CH;
-    for (int e = t; e < RB * (CH / 4); e += kThreads) {
-      const int rr = e / (CH / 4), q4 = e % (CH / 4);
-      const int gi = r0 + rr, gj = c0 + 4 * q4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (gi < m && gj < n) v = *reinterpret_cast<const float4*>(Mb + (long long)gi * n + gj);
-      float* d = Ms + rr * MS + 4 * q4;
-      d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
-    }
-    for (int e = t; e < CH * KP; e += kThreads) {
-      const int jj = e / KP, l = e % KP;
-      const int gj = c0 + jj;
-      Qs[e] = (gj < n && l < k) ? Qb[(long long)gj * k + l] : 0.f;
-    }
-    __syncthreads();
-    float accf[4][8];
+        for (int i = 0; i < 4; ++i) {
+          float sacc = 0.f;
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int l = 0; l < 8; ++l) accf[r][l] = 0.f;
-#pragma unroll 4
-    for (int jj = 0; jj < JPER; ++jj) {
-      const int j = jg * JPER + jj;
-      const float4 qa = *reinterpret_cast<const float4*>(Qs + j * KP + 8 * lg);
-      const float4 qb = *reinterpret_cast<const float4*>(Qs + j * KP + 8 * lg + 4);
-      const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float mv = Ms[(rg + 16 * r) * MS + j];
-#pragma unroll
-        for (int l = 0; l < 8; ++l) accf[r][l] = fmaf(mv, qv[l], accf[r][l]);
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int l = 0; l < 8; ++l) accd[r][l] += (double)accf[r][l];
-    __syncthreads();
-  }
-  // Ordered reduction over the j-groups, reusing the tile buffer.
-  double* red = reinterpret_cast<double*>(smem);   // RB * KP doubles <= smem size
-  for (int g = JG - 1; g >= 0; --g) {
-    if (jg == g) {
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int l = 0; l < 8; ++l) {
-          double* slot = red + (rg + 16 * r) * KP + 8 * lg + l;
-          *slot = (g == JG - 1) ? accd[r][l] : (*slot + accd[r][l]);
+          for (int e = 0; e < 8; ++e) sacc = fmaf(acc[i][e], qv[e], sacc);
+          v[i * 4 + j] = sacc;
         }
+      }
+      reduce_scatter16(v, tx);
+      const int row = r0 + ty + 16 * (tx >> 2), l = l0 + (tx & 3);
+      if (row < m && l < k) Ppart[(((long long)b * nb + bj) * m + row) * k + l] = v[0];
     }
-    __syncthreads();
-  }
-  double* out = Ppart + ((long long)b * csplit + split) * m * k;
-  for (int e = t; e < RB * k; e += kThreads) {
-    const int rr = e / k, l = e % k;
-    if (r0 + rr < m) out[(long long)(r0 + rr) * k + l] = red[rr * KP + l];
   }
 }
 
 // ------------------------------------------------------------------ S4
 // (a) P~ = sum of column-split partials (fixed order); partial Gram P~^T P~.
 __global__ void __launch_bounds__(kThreads) k_orth_gram(int m, int k, int csplit, int rsplit,
-                                                         const double* __restrict__ Ppart,
+                                                         const float* __restrict__ Ppart,
                                                          double* __restrict__ Ptil,
                                                          double* __restrict__ gram_part,
                                                          const int32_t* skip) {
@@ -387,7 +373,7 @@ __global__ void __launch_bounds__(kThreads) k_orth_gram(int m, int k, int csplit
       const int rr = e / k, l = e % k, gi = c + rr;
       double v = 0.0;
       if (gi < i1) {
-        for (int s = 0; s < csplit; ++s) v += Ppart[(((long long)b * csplit + s) * m + gi) * k + l];
+        for (int s = 0; s < csplit; ++s) v += (double)Ppart[(((long long)b * csplit + s) * m + gi) * k + l];
         Ptil[((long long)b * m + gi) * k + l] = v;
       }
       Ps[rr][l] = v;
@@ -498,105 +484,111 @@ __global__ void __launch_bounds__(kThreads) k_orth_apply(int m, int k, const dou
 }
 
 // ------------------------------------------------------------------ S5
-// R = M^T P over row splits (fp64 partials), and the normalised wide-form NS
-// input X = round16(scale * M) (X = M^T when m > n).
+// R = M^T P over row splits, and the normalised wide-form NS input
+// X = round16(scale * M) (X = M^T when m > n).
+// CTA: 64 columns x the rows of its split, in chunks of 128 rows. Warp w owns
+// rows 16 w .. 16 w + 15 of a chunk, lane c the columns 2c, 2c + 1, so every
+// warp reads whole 256-byte row segments of M straight into registers; P rows
+// are broadcast from shared memory. fp32 sums over at most 1024 rows per split,
+// fp64 across splits.
 template <int KP>
-__global__ void __launch_bounds__(kThreads) k_backproject(int m, int n, int k, int rsplit,
-                                                           const float* __restrict__ M,
-                                                           const float* __restrict__ P,
-                                                           const float* __restrict__ scale,
-                                                           uint16_t* __restrict__ X16, int f16,
-                                                           double* __restrict__ Rpart,
-                                                           const int32_t* skip) {
+__global__ void __launch_bounds__(kThreads, 2) k_backproject(int m, int n, int k, int rsplit,
+                                                              const float* __restrict__ M,
+                                                              const float* __restrict__ P,
+                                                              const float* __restrict__ scale,
+                                                              uint16_t* __restrict__ X16, int f16,
+                                                              double* __restrict__ Rpart,
+                                                              const int32_t* skip) {
   if (skip && *skip) return;
-  constexpr int CB = 64, CH = 128, LG = KP / 8, IG = kThreads / (16 * LG), IPER = CH / IG;
-  constexpr int MS = CB + 1;
-  extern __shared__ __align__(16) float smem[];   // CH * MS + CH * KP floats
-  float* Ms = smem;
-  float* Ps = smem + CH * MS;
+  constexpr int CB = 64, CH = 128, RPW = 16, XS = CH + 2;
+  extern __shared__ __align__(16) float smb[];
+  float* Ps = smb;                                             // [CH][KP]
+  uint16_t* Xt = reinterpret_cast<uint16_t*>(Ps + CH * KP);     // [CB][XS], tall staging
   const int cbk = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
-  const int t = threadIdx.x, cg = t & 15, lg = (t >> 4) % LG, ig = t / (16 * LG);
+  const int t = threadIdx.x, cq = t & 31, rg = t >> 5;
   const int c0 = cbk * CB;
+  const int col = c0 + 2 * cq;
   const int nchunks = cdiv(m, CH);
   const int per = cdiv(nchunks, rsplit);
   const int ch0 = split * per, ch1 = min(nchunks, ch0 + per);
   const float* Mb = M + (long long)b * m * n;
   const float* Pb = P + (long long)b * m * k;
-  const float sc = X16 ? scale[b] : 0.f;
   const bool tall = m > n;
+  const float sc = X16 ? scale[b] : 0.f;
   uint16_t* Xb = X16 ? X16 + (long long)b * m * n : nullptr;
 
-  double accd[4][8];
+  float acc[2][KP];
 #pragma unroll
-  for (int c = 0; c < 4; ++c)
+  for (int c = 0; c < 2; ++c)
 #pragma unroll
-    for (int l = 0; l < 8; ++l) accd[c][l] = 0.0;
+    for (int l = 0; l < KP; ++l) acc[c][l] = 0.f;
 
   for (int ch = ch0; ch < ch1; ++ch) {
     const int i0 = ch * CH;
-    for (int e = t; e < CH * (CB / 4); e += kThreads) {
-      const int ii = e / (CB / 4), q4 = e % (CB / 4);
-      const int gi = i0 + ii, gj = c0 + 4 * q4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      const bool ok = gi < m && gj < n;
-      if (ok) v = *reinterpret_cast<const float4*>(Mb + (long long)gi * n + gj);
-      float* d = Ms + ii * MS + 4 * q4;
-      d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
-      if (Xb && ok && !tall) {
-        const float xv[4] = {v.x * sc, v.y * sc, v.z * sc, v.w * sc};
-        uint2 pk;
-        pk.x = (uint32_t)float_to_h16(xv[0], f16) | ((uint32_t)float_to_h16(xv[1], f16) << 16);
-        pk.y = (uint32_t)float_to_h16(xv[2], f16) | ((uint32_t)float_to_h16(xv[3], f16) << 16);
-        *reinterpret_cast<uint2*>(Xb + (long long)gi * n + gj) = pk;
-      }
+    float2 mv[RPW];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const int gi = i0 + rg * RPW + r;
+      mv[r] = (gi < m && col < n) ? *reinterpret_cast<const float2*>(Mb + (long long)gi * n + col)
+                                  : make_float2(0.f, 0.f);
     }
     for (int e = t; e < CH * KP; e += kThreads) {
       const int ii = e / KP, l = e % KP, gi = i0 + ii;
       Ps[e] = (gi < m && l < k) ? Pb[(long long)gi * k + l] : 0.f;
     }
+    if (Xb) {
+#pragma unroll
+      for (int r = 0; r < RPW; ++r) {
+        const int gi = i0 + rg * RPW + r;
+        const uint16_t x0 = float_to_h16(mv[r].x * sc, f16), x1 = float_to_h16(mv[r].y * sc, f16);
+        if (!tall) {
+          if (gi < m && col < n)
+            *reinterpret_cast<uint32_t*>(Xb + (long long)gi * n + col) = (uint32_t)x0 | ((uint32_t)x1 << 16);
+        } else {
+          Xt[(2 * cq) * XS + rg * RPW + r] = x0;
+          Xt[(2 * cq + 1) * XS + rg * RPW + r] = x1;
+        }
+      }
+    }
     __syncthreads();
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const float* prow = Ps + (rg * RPW + r) * KP;
+#pragma unroll
+      for (int l = 0; l < KP; l += 4) {
+        const float4 pv = *reinterpret_cast<const float4*>(prow + l);
+        acc[0][l] = fmaf(mv[r].x, pv.x, acc[0][l]);
+        acc[0][l + 1] = fmaf(mv[r].x, pv.y, acc[0][l + 1]);
+        acc[0][l + 2] = fmaf(mv[r].x, pv.z, acc[0][l + 2]);
+        acc[0][l + 3] = fmaf(mv[r].x, pv.w, acc[0][l + 3]);
+        acc[1][l] = fmaf(mv[r].y, pv.x, acc[1][l]);
+        acc[1][l + 1] = fmaf(mv[r].y, pv.y, acc[1][l + 1]);
+        acc[1][l + 2] = fmaf(mv[r].y, pv.z, acc[1][l + 2]);
+        acc[1][l + 3] = fmaf(mv[r].y, pv.w, acc[1][l + 3]);
+      }
+    }
     if (Xb && tall) {
-      // X[j][i] = M[i][j]: consecutive threads take consecutive i.
-      for (int e = t; e < CH * CB; e += kThreads) {
-        const int ii = e % CH, jj = e / CH;
-        const int gi = i0 + ii, gj = c0 + jj;
-        if (gi < m && gj < n)
-          Xb[(long long)gj * m + gi] = float_to_h16(Ms[ii * MS + jj] * sc, f16);
+      // X[j][i] = M[i][j]: rows of X are 256-byte runs of this chunk
+      for (int idx = t; idx < CB * (CH / 2); idx += kThreads) {
+        const int j = idx / (CH / 2), i2 = idx % (CH / 2);
+        const int gj = c0 + j, gi = i0 + 2 * i2;
+        if (gj < n && gi < m)
+          *reinterpret_cast<uint32_t*>(Xb + (long long)gj * m + gi) =
+              *reinterpret_cast<const uint32_t*>(Xt + j * XS + 2 * i2);
       }
     }
-    float accf[4][8];
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-#pragma unroll
-      for (int l = 0; l < 8; ++l) accf[c][l] = 0.f;
-#pragma unroll 4
-    for (int ii = 0; ii < IPER; ++ii) {
-      const int i = ig * IPER + ii;
-      const float4 pa = *reinterpret_cast<const float4*>(Ps + i * KP + 8 * lg);
-      const float4 pb = *reinterpret_cast<const float4*>(Ps + i * KP + 8 * lg + 4);
-      const float pv[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float mv = Ms[i * MS + cg + 16 * c];
-#pragma unroll
-        for (int l = 0; l < 8; ++l) accf[c][l] = fmaf(mv, pv[l], accf[c][l]);
-      }
-    }
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-#pragma unroll
-      for (int l = 0; l < 8; ++l) accd[c][l] += (double)accf[c][l];
     __syncthreads();
   }
-  double* red = reinterpret_cast<double*>(smem);   // CB * KP doubles
-  for (int g = IG - 1; g >= 0; --g) {
-    if (ig == g) {
+  // ordered reduction over the eight warps
+  float* red = smb;   // [CB][KP]
+  for (int w = (kThreads / 32) - 1; w >= 0; --w) {
+    if (rg == w) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int l = 0; l < 8; ++l) {
-          double* slot = red + (cg + 16 * c) * KP + 8 * lg + l;
-          *slot = (g == IG - 1) ? accd[c][l] : (*slot + accd[c][l]);
+        for (int l = 0; l < KP; ++l) {
+          float* slot = red + (2 * cq + c) * KP + l;
+          *slot = (w == (kThreads / 32) - 1) ? acc[c][l] : (*slot + acc[c][l]);
         }
     }
     __syncthreads();
@@ -604,7 +596,7 @@ __global__ void __launch_bounds__(kThreads) k_backproject(int m, int n, int k, i
   double* out = Rpart + ((long long)b * rsplit + split) * n * k;
   for (int e = t; e < CB * k; e += kThreads) {
     const int cc = e / k, l = e % k;
-    if (c0 + cc < n) out[(long long)(c0 + cc) * k + l] = red[cc * KP + l];
+    if (c0 + cc < n) out[(long long)(c0 + cc) * k + l] = (double)red[cc * KP + l];
   }
 }
 
@@ -622,7 +614,11 @@ __global__ void __launch_bounds__(kThreads) k_finalize_r(int n, int k, int rspli
 }
 
 // ------------------------------------------------------------------ S7
-__global__ void __launch_bounds__(kThreads) k_residual_quant4(
+// One 128 x 128 grid block per CTA of 512 threads; thread (ty, tx) owns rows
+// ty + 32 i (i < 4) and columns 4 tx + {0..3}, 64 + 4 tx + {0..3}. The residual
+// x = M - sum_l P_il R_jl is formed in place (fp32 FMA), then the block's row and
+// column absolute maxima, then the codes q = rint(fp32(x / s) * 7).
+__global__ void __launch_bounds__(512, 2) k_residual_quant4(
     int m, int n, int k, const float* __restrict__ X, const float* __restrict__ P,
     const float* __restrict__ R, uint8_t* __restrict__ codes4, float* __restrict__ rscale,
     float* __restrict__ cscale, const int32_t* skip) {
@@ -631,57 +627,52 @@ __global__ void __launch_bounds__(kThreads) k_residual_quant4(
   const int nb = gridDim.x, mb = gridDim.y;
   const int r0 = bi * kGrid, c0 = bj * kGrid;
   const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
-  __shared__ __align__(16) float Ps[kMaxK][kGrid];
-  __shared__ __align__(16) float Rs[kMaxK][kGrid];
-  __shared__ float cm[16][kGrid];
-  __shared__ float cmax[kGrid];
   const int kk = (P && R) ? k : 0;
-  for (int e = t; e < kGrid * kk; e += kThreads) {
-    const int rr = e / kk, l = e % kk;
-    const int gi = r0 + rr, gj = c0 + rr;
-    Ps[l][rr] = (gi < m) ? P[((long long)b * m + gi) * kk + l] : 0.f;
-    Rs[l][rr] = (gj < n) ? R[((long long)b * n + gj) * kk + l] : 0.f;
-  }
-  __syncthreads();
-  float acc[8][8];
+  extern __shared__ __align__(16) float smq[];
+  float* Ps = smq;                 // [kk][128]
+  float* Rs = Ps + kk * kGrid;     // [kk][128]
+  __shared__ float cm[32][kGrid];
+  __shared__ float cmax[kGrid];
+
+  float x[4][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  for (int l = 0; l < kk; ++l) {
-    const float4 ra = *reinterpret_cast<const float4*>(&Rs[l][4 * tx]);
-    const float4 rb = *reinterpret_cast<const float4*>(&Rs[l][64 + 4 * tx]);
-    const float rv[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float p = Ps[l][ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(p, rv[j], acc[i][j]);
-    }
-  }
-  // x = M - P R^T in registers (zero outside the matrix).
-  float x[8][8];
-  float cmx[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) cmx[j] = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int gi = r0 + ty + 16 * i;
+  for (int i = 0; i < 4; ++i) {
+    const int gi = r0 + ty + 32 * i;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int cb = c0 + 64 * h + 4 * tx;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (gi < m && cb < n) v = *reinterpret_cast<const float4*>(X + ((long long)b * m + gi) * n + cb);
-      const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float r = (gi < m && cb < n) ? __fsub_rn(vv[e], acc[i][4 * h + e]) : 0.f;
-        x[i][4 * h + e] = r;
-        cmx[4 * h + e] = fmaxf(cmx[4 * h + e], fabsf(r));
-      }
+      x[i][4 * h] = v.x; x[i][4 * h + 1] = v.y; x[i][4 * h + 2] = v.z; x[i][4 * h + 3] = v.w;
     }
   }
-  // column absmax: per-thread over its 8 rows, then over the 16 row groups
+  for (int e = t; e < kGrid * kk; e += 512) {
+    const int rr = e / kk, l = e % kk;
+    const int gi = r0 + rr, gj = c0 + rr;
+    Ps[l * kGrid + rr] = (gi < m) ? P[((long long)b * m + gi) * kk + l] : 0.f;
+    Rs[l * kGrid + rr] = (gj < n) ? R[((long long)b * n + gj) * kk + l] : 0.f;
+  }
+  __syncthreads();
+  for (int l = 0; l < kk; ++l) {
+    const float4 ra = *reinterpret_cast<const float4*>(Rs + l * kGrid + 4 * tx);
+    const float4 rb = *reinterpret_cast<const float4*>(Rs + l * kGrid + 64 + 4 * tx);
+    const float rv[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float pv = -Ps[l * kGrid + ty + 32 * i];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[i][j] = fmaf(pv, rv[j], x[i][j]);
+    }
+  }
+  // rows and columns outside the matrix are 0 (loaded as 0; their P, R rows are 0)
+  float cmx[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    float v = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v = fmaxf(v, fabsf(x[i][j]));
+    cmx[j] = v;
+  }
 #pragma unroll
   for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -689,7 +680,8 @@ __global__ void __launch_bounds__(kThreads) k_residual_quant4(
   __syncthreads();
   if (t < kGrid) {
     float v = 0.f;
-    for (int g = 0; g < 16; ++g) v = fmaxf(v, cm[g][t]);
+#pragma unroll 8
+    for (int g = 0; g < 32; ++g) v = fmaxf(v, cm[g][t]);
     cmax[t] = v;
     if (c0 + t < n) cscale[((long long)b * mb + bi) * n + c0 + t] = v;
   }
@@ -700,12 +692,11 @@ __global__ void __launch_bounds__(kThreads) k_residual_quant4(
 #pragma unroll
     for (int e = 0; e < 4; ++e) cs[4 * h + e] = cmax[64 * h + 4 * tx + e];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int gi = r0 + ty + 16 * i;
+  for (int i = 0; i < 4; ++i) {
+    const int gi = r0 + ty + 32 * i;
     float rmx = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) rmx = fmaxf(rmx, fabsf(x[i][j]));
-    // the 16 threads of a row are lanes 16*(ty&1) .. +15 of one warp
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) rmx = fmaxf(rmx, __shfl_xor_sync(0xffffffffu, rmx, o));
     if (gi >= m) continue;
@@ -717,17 +708,15 @@ __global__ void __launch_bounds__(kThreads) k_residual_quant4(
       uint32_t packed = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float s = fminf(rmx, cs[4 * h + e]);
+        const float sv = fminf(rmx, cs[4 * h + e]);
         int q = 0;
-        if (s > 0.f) {
-          const float r = __fmul_rn(__fdiv_rn(x[i][4 * h + e], s), 7.0f);
-          q = (int)rintf(r);
+        if (sv > 0.f) {
+          q = (int)rintf(__fmul_rn(__fdiv_rn(x[i][4 * h + e], sv), 7.0f));
           q = max(-7, min(7, q));
         }
         packed |= (uint32_t)(q & 0xF) << (4 * e);
       }
-      *reinterpret_cast<uint16_t*>(codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2) =
-          (uint16_t)packed;
+      *reinterpret_cast<uint16_t*>(codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2) = (uint16_t)packed;
     }
   }
 }
@@ -829,28 +818,11 @@ __global__ void __launch_bounds__(kThreads) k_cast_wide(int m, int n, const void
 }
 
 template <int KP>
-cudaError_t launch_project_t(int B, int m, int n, int k, const float* M, const float* Q,
-                             double* Ppart, const int32_t* skip, cudaStream_t s) {
-  const int cs = project_col_splits(B, m, n);
-  const size_t smem = (size_t)(64 * 129 + 128 * KP) * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_project<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  dim3 grid(cdiv(m, 64), cs, B);
-  k_project<KP><<<grid, kThreads, smem, s>>>(m, n, k, cs, M, Q, Ppart, skip);
-  return cudaGetLastError();
-}
-
-template <int KP>
 cudaError_t launch_backproject_t(int B, int m, int n, int k, const float* M, const float* P,
                                  const float* scale, void* X16, bool f16, double* Rpart,
                                  float* R, const int32_t* skip, cudaStream_t s) {
   const int rs = backproject_row_splits(B, m, n);
-  const size_t smem = (size_t)(128 * 65 + 128 * KP) * sizeof(float);
+  const size_t smem = (size_t)128 * KP * sizeof(float) + (size_t)64 * 130 * sizeof(uint16_t);
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(k_backproject<KP>,
@@ -872,16 +844,12 @@ cudaError_t launch_backproject_t(int B, int m, int n, int k, const float* M, con
 }  // namespace
 
 // ------------------------------------------------------------------ splits
-int project_col_splits(int B, int m, int n) {
-  const int ctas = cdiv(m, 64) * B;
-  const int nchunks = cdiv(n, 128);
-  int cs = cdiv(kTargetCtas, ctas);
-  return max(1, min(cs, nchunks));
-}
+int rebuild_row_blocks(int m) { return cdiv(m, kRB); }
 int backproject_row_splits(int B, int m, int n) {
   const int ctas = cdiv(n, 64) * B;
   const int nchunks = cdiv(m, 128);
-  int rs = cdiv(kTargetCtas, ctas);
+  const int need = cdiv(m, 1024);            // at most 1024 rows summed in fp32
+  const int rs = max(need, cdiv(kTargetCtas, ctas));
   return max(1, min(rs, nchunks));
 }
 int gram_row_splits(int B, int m) {
@@ -908,25 +876,47 @@ cudaError_t launch_warm_start(int B, int n, int k, const int8_t* R8, const float
   return cudaGetLastError();
 }
 
-cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4, const float* rscale,
-                           const float* cscale, const int8_t* P8, const float* Pscale,
-                           const int8_t* R8, const float* Rscale, const float* Mprev32, float mu,
-                           const void* G, int gdt, float* M, double* norm2_part, int32_t* status,
-                           cudaStream_t s) {
-  dim3 grid(cdiv(n, kGrid), cdiv(m, kGrid), B);
-  k_rebuild<<<grid, kThreads, 0, s>>>(m, n, k, codes4, rscale, cscale, P8, Pscale, R8, Rscale,
-                                      Mprev32, mu, G, gdt, M, norm2_part, status);
+template <int SRC, bool G32>
+cudaError_t launch_rebuild_t(dim3 grid, size_t smem, cudaStream_t s, int m, int n, int k,
+                             const uint8_t* codes4, const float* rscale, const float* cscale,
+                             const int8_t* P8, const float* Pscale, const int8_t* R8,
+                             const float* Rscale, const float* Mprev32, float mu, const void* G,
+                             int gdt, const float* Q, float* M, double* norm2_part, float* Ppart,
+                             int32_t* status) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_rebuild_proj<SRC, G32>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)((2 * kMaxK * kGrid + kMaxK * kRB) * sizeof(float)));
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  k_rebuild_proj<SRC, G32><<<grid, kThreads, smem, s>>>(m, n, k, codes4, rscale, cscale, P8, Pscale,
+                                                        R8, Rscale, Mprev32, mu, G, gdt, Q, M,
+                                                        norm2_part, Ppart, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_project(int B, int m, int n, int k, const float* M, const float* Q,
-                           double* Ppart, const int32_t* skip, cudaStream_t s) {
-  if (k <= 8) return launch_project_t<8>(B, m, n, k, M, Q, Ppart, skip, s);
-  if (k <= 16) return launch_project_t<16>(B, m, n, k, M, Q, Ppart, skip, s);
-  return launch_project_t<32>(B, m, n, k, M, Q, Ppart, skip, s);
+cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4, const float* rscale,
+                           const float* cscale, const int8_t* P8, const float* Pscale,
+                           const int8_t* R8, const float* Rscale, const float* Mprev32, float mu,
+                           const void* G, int gdt, const float* Q, float* M, double* norm2_part,
+                           float* Ppart, int32_t* status, cudaStream_t s) {
+  dim3 grid(cdiv(n, kGrid), cdiv(m, kRB), B);
+  const int kk = codes4 ? k : 0;
+  const int kq = Q ? ((k + 3) & ~3) : 0;
+  const size_t smem = (size_t)(kk * kRB + kk * kGrid + kq * kGrid) * sizeof(float);
+  const bool g32 = (G == nullptr) || gdt == GM_F32;
+  const int src = codes4 ? SRC_STATE : (Mprev32 ? SRC_DENSE : SRC_ZERO);
+#define GM_RB(S, W) launch_rebuild_t<S, W>(grid, smem, s, m, n, k, codes4, rscale, cscale, P8, Pscale, \
+                                           R8, Rscale, Mprev32, mu, G, gdt, Q, M, norm2_part, Ppart, status)
+  if (src == SRC_STATE) return g32 ? GM_RB(SRC_STATE, true) : GM_RB(SRC_STATE, false);
+  if (src == SRC_DENSE) return g32 ? GM_RB(SRC_DENSE, true) : GM_RB(SRC_DENSE, false);
+  return g32 ? GM_RB(SRC_ZERO, true) : GM_RB(SRC_ZERO, false);
+#undef GM_RB
 }
 
-cudaError_t launch_orth(int B, int m, int k, int csplit, const double* Ppart, double* Ptil,
+cudaError_t launch_orth(int B, int m, int k, int csplit, const float* Ppart, double* Ptil,
                         double* gram_part, double* Tmat, const double* norm2_part, int ntiles,
                         float eps, float* scale, float* P, const int32_t* skip, cudaStream_t s) {
   const int rs = gram_row_splits(B, m);
@@ -953,7 +943,15 @@ cudaError_t launch_residual_quant4(int B, int m, int n, int k, const float* X, c
                                    const float* R, uint8_t* codes4, float* rscale, float* cscale,
                                    const int32_t* skip, cudaStream_t s) {
   dim3 grid(cdiv(n, kGrid), cdiv(m, kGrid), B);
-  k_residual_quant4<<<grid, kThreads, 0, s>>>(m, n, k, X, P, R, codes4, rscale, cscale, skip);
+  const size_t smem = (size_t)2 * k * kGrid * sizeof(float);
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_residual_quant4, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(2 * kMaxK * kGrid * sizeof(float)));
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  k_residual_quant4<<<grid, 512, smem, s>>>(m, n, k, X, P, R, codes4, rscale, cscale, skip);
   return cudaGetLastError();
 }
 

@@ -8,7 +8,7 @@ namespace gm {
 
 // Column / row split counts of the power-iteration reductions. They depend
 // only on the problem shape, so the workspace layout is a pure function of it.
-int project_col_splits(int B, int m, int n);
+int rebuild_row_blocks(int m);   // 64-row blocks of the fused rebuild / projection
 int backproject_row_splits(int B, int m, int n);
 int gram_row_splits(int B, int m);
 
@@ -19,18 +19,18 @@ cudaError_t launch_warm_start(int B, int n, int k, const int8_t* R8, const float
                               const int32_t* skip, cudaStream_t s);
 
 // M = mu * Mprev + G where Mprev is either the rebuilt state (codes4 != NULL)
-// or a dense fp32 matrix (Mprev32 != NULL) or zero. norm2_part gets one fp64
-// partial |M|^2 per 128x128 tile; status (nullable) gets GM_E_NONFINITE.
+// or a dense fp32 matrix (Mprev32 != NULL) or zero; with Q != NULL also the
+// projection partials Ppart f32 [B][ceil(n/128)][m][k] (sum over one column
+// block each). norm2_part gets one fp64 partial |M|^2 per 64 x 128 tile
+// ([B][ceil(m/64)][ceil(n/128)]); status (nullable) gets GM_E_NONFINITE.
 cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4,
                            const float* rscale, const float* cscale, const int8_t* P8,
                            const float* Pscale, const int8_t* R8, const float* Rscale,
-                           const float* Mprev32, float mu, const void* G, int gdt, float* M,
-                           double* norm2_part, int32_t* status, cudaStream_t s);
+                           const float* Mprev32, float mu, const void* G, int gdt, const float* Q,
+                           float* M, double* norm2_part, float* Ppart, int32_t* status,
+                           cudaStream_t s);
 
-cudaError_t launch_project(int B, int m, int n, int k, const float* M, const float* Q,
-                           double* Ppart, const int32_t* skip, cudaStream_t s);
-
-cudaError_t launch_orth(int B, int m, int k, int csplit, const double* Ppart, double* Ptil,
+cudaError_t launch_orth(int B, int m, int k, int csplit, const float* Ppart, double* Ptil,
                         double* gram_part, double* Tmat, const double* norm2_part, int ntiles,
                         float eps, float* scale, float* P, const int32_t* skip, cudaStream_t s);
 
