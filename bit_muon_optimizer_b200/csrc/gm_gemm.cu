@@ -33,8 +33,6 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;                 // 64 x 16-bit = 128 B = one swizzle row
-constexpr int kStages = 3;
-constexpr int kGemmThreads = 192;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ int32_t g_device_error = 0;
@@ -43,6 +41,7 @@ enum EpiMode : int { EPI_STORE = 0, EPI_OUT = 1, EPI_WUPDATE = 2 };
 
 struct GemmParams {
   int M, N, K;                 // output M x N; reduction K
+  int batch;
   int tiles_m, tiles_n;
   int sym;                     // lower-triangle schedule + mirrored store
   int f16;                     // operand / 16-bit output type: 1 fp16, 0 bf16
@@ -169,20 +168,45 @@ __device__ __forceinline__ void tri_tile(int x, int& ti, int& tj) {
 }
 
 // ------------------------------------------------------------------ epilogue
-// Staging layout in the (then idle) pipeline shared memory:
-//   EPI_STORE : sC [BM][BN + 8] 16-bit (C tile in, output tile out, in place)
-//               sT [BN][BM + 8] 16-bit (transposed output, for mirrored stores)
-//   otherwise : sF [BM][BN + 4] fp32 output values, then sC as above for C.
-template <int BN>
-__host__ __device__ constexpr uint32_t smem_data_bytes() {
-  constexpr uint32_t ring = kStages * (BM * BK * 2 + BN * BK * 2);
-  constexpr uint32_t st = BM * (BN + 8) * 2 + BN * (BM + 8) * 2;
-  constexpr uint32_t out = BM * (BN + 4) * 4 + BM * (BN + 8) * 2;
-  constexpr uint32_t epi = st > out ? st : out;
-  return ring > epi ? ring : epi;
+// Staging buffers (separate from the operand ring, which keeps streaming the
+// next tile while this one is written out), one 128-column slab at a time:
+//   EPI_STORE : sC [BM][SP] 16-bit (C tile in, output out, in place)
+//               sT [128][TP] 16-bit (transposed output, for mirrored stores)
+//   otherwise : sF [BM][FP] fp32 output values
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kGemmThreadsP = 64 + kEpiThreads;
+constexpr int SP = 128 + 8;
+constexpr int TP = BM + 8;
+constexpr int FP = 128 + 4;
+constexpr uint32_t kStagingBytes =
+    (uint32_t)(BM * SP * 2 + 128 * TP * 2) > (uint32_t)(BM * FP * 4) ? (uint32_t)(BM * SP * 2 + 128 * TP * 2)
+                                                                     : (uint32_t)(BM * FP * 4);
+
+template <int BN, int STAGES>
+__host__ __device__ constexpr uint32_t gemm_smem_bytes() {
+  return STAGES * (BM * BK * 2 + BN * BK * 2) + kStagingBytes + 256 /* barriers etc. */ +
+         BM * 2 /* second-output diagonal */ + 1024 /* alignment slack */;
 }
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ bool epi_any(bool pred) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(res)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return res != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 
 __device__ __forceinline__ void unpack8(const uint4 w, bool f16, float (&o)[8]) {
   const uint32_t u[4] = {w.x, w.y, w.z, w.w};
@@ -200,33 +224,47 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8], bool f16) {
   return make_uint4(u[0], u[1], u[2], u[3]);
 }
 
+struct TileCoord {
+  int bz, ti, tj;
+};
+__device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int T, int tiles_per) {
+  TileCoord c;
+  c.bz = T / tiles_per;
+  const int x = T - c.bz * tiles_per;
+  if (p.sym) tri_tile(x, c.ti, c.tj);
+  else { c.ti = x % p.tiles_m; c.tj = x / p.tiles_m; }
+  return c;
+}
+
+// One output slab (128 columns of the tile) from TMEM through staging to global.
+// Returns false if the tile's accumulator could not be waited for.
 template <int BN>
-__device__ __forceinline__ void epilogue(const GemmParams& p, uint8_t* base, uint32_t tmem,
-                                         bool ok, int ti, int tj, int bz, int warp, int lane,
-                                         uint16_t* d2diag) {
-  constexpr int SP = BN + 8;          // 16-bit row stride of sC (16-byte multiple)
-  constexpr int TP = BM + 8;          // 16-bit row stride of sT
-  constexpr int FP = BN + 4;          // fp32 row stride of sF
-  const int et = threadIdx.x - 64;    // 0..127 over the four epilogue warps
-  const int q = warp & 3;             // TMEM lane quarter this warp may access
-  const int rr = q * 32 + lane;       // tile row owned by this thread
-  const int r0 = ti * BM, c0 = tj * BN;
+__device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg, uint32_t tacc,
+                                              const TileCoord& tc, int slab, int warp, int lane,
+                                              uint16_t* d2diag, bool last_slab, uint32_t acc_empty_bar) {
+  const int et = threadIdx.x - 64;          // 0..255
+  const int q = warp & 3;                   // TMEM lane quarter of this warp
+  const int half = (warp - 2) >> 2;         // 64-column half of the slab
+  const int rr = q * 32 + lane;             // tile row owned by this thread
+  const int r0 = tc.ti * BM;
+  const int cs0 = slab * 128;               // slab column offset inside the tile
+  const int c0 = tc.tj * BN + cs0;          // global column of the slab
   const int r = r0 + rr;
   const bool f16 = p.f16 != 0;
   const bool store_mode = p.mode == EPI_STORE;
-  float* sF = reinterpret_cast<float*>(base);
-  uint16_t* sC = reinterpret_cast<uint16_t*>(store_mode ? base : base + BM * FP * 4);
-  uint16_t* sT = reinterpret_cast<uint16_t*>(base) + BM * SP;
+  uint16_t* sC = reinterpret_cast<uint16_t*>(stg);
+  uint16_t* sT = sC + BM * SP;
+  float* sF = reinterpret_cast<float*>(stg);
   const int rows_valid = min(BM, p.M - r0);
-  const int cols_valid = min(BN, p.N - c0);   // multiple of 16
-  const bool use_c = ok && p.C && p.beta != 0.f;
+  const int cols_valid = min(128, p.N - c0);   // may be <= 0 for a ragged last slab
+  const bool use_c = p.C && p.beta != 0.f;
+  const long long cbs = (long long)tc.bz * p.c_bs;
 
-  // 1. C tile -> sC (coalesced 16-byte loads)
-  if (use_c) {
-    const uint16_t* cbase = p.C + (long long)bz * p.c_bs + (long long)r0 * p.ldc + c0;
-    constexpr int CPR = BN / 8;   // 16-byte chunks per row
-    for (int idx = et; idx < BM * CPR; idx += 128) {
-      const int row = idx / CPR, cc = idx % CPR;
+  // 1. C slab -> sC (store mode; coalesced 16-byte loads)
+  if (store_mode && use_c) {
+    const uint16_t* cbase = p.C + cbs + (long long)r0 * p.ldc + c0;
+    for (int idx = et; idx < BM * 16; idx += kEpiThreads) {
+      const int row = idx >> 4, cc = idx & 15;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (row < rows_valid && cc * 8 < cols_valid)
         v = *reinterpret_cast<const uint4*>(cbase + (long long)row * p.ldc + cc * 8);
@@ -236,69 +274,78 @@ __device__ __forceinline__ void epilogue(const GemmParams& p, uint8_t* base, uin
   epi_bar();
 
   // 2. TMEM -> registers -> epilogue math -> staging
-  if (ok) {
 #pragma unroll 1
-    for (int cb = 0; cb < BN; cb += 32) {
-      float v[32];
-      __syncwarp();
-      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)cb, v);
+  for (int ch = 0; ch < 2; ++ch) {
+    const int cl = half * 64 + ch * 32;   // column inside the slab
+    float v[32];
+    __syncwarp();
+    tmem_ld32(tacc + ((uint32_t)(q * 32) << 16) + (uint32_t)(cs0 + cl), v);
+    if (store_mode) {
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         float cin[8];
-        if (use_c) unpack8(*reinterpret_cast<const uint4*>(sC + rr * SP + cb + g * 8), f16, cin);
+        if (use_c) unpack8(*reinterpret_cast<const uint4*>(sC + rr * SP + cl + g * 8), f16, cin);
+        float x[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          float x = p.alpha * v[g * 8 + e];
-          if (use_c) x = fmaf(p.beta, cin[e], x);
-          v[g * 8 + e] = x;
-        }
-      }
-      if (store_mode) {
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          float x[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            x[e] = v[g * 8 + e];
-            const int c = c0 + cb + g * 8 + e;
-            if (c == r) {
-              x[e] += p.gamma;
-              if (p.D2) d2diag[rr] = float_to_h16(x[e] + p.gamma2, f16);
-            }
-          }
-          *reinterpret_cast<uint4*>(sC + rr * SP + cb + g * 8) = pack8(x, f16);
-          if (p.sym) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) sT[(cb + g * 8 + e) * TP + rr] = float_to_h16(x[e], f16);
+          x[e] = p.alpha * v[g * 8 + e];
+          if (use_c) x[e] = fmaf(p.beta, cin[e], x[e]);
+          if (c0 + cl + g * 8 + e == r) {
+            x[e] += p.gamma;
+            if (p.D2) d2diag[rr] = float_to_h16(x[e] + p.gamma2, f16);
           }
         }
-      } else {
+        *reinterpret_cast<uint4*>(sC + rr * SP + cl + g * 8) = pack8(x, f16);
+        if (p.sym) {
 #pragma unroll
-        for (int g = 0; g < 8; ++g)
-          *reinterpret_cast<float4*>(sF + rr * FP + cb + g * 4) =
-              make_float4(v[g * 4], v[g * 4 + 1], v[g * 4 + 2], v[g * 4 + 3]);
+          for (int e = 0; e < 8; ++e) sT[(cl + g * 8 + e) * TP + rr] = float_to_h16(x[e], f16);
+        }
       }
+    } else {
+      // O = alpha acc + beta C, C read straight from global (one 64-byte row run)
+      float cin[32];
+      const uint16_t* crow = p.C + cbs + (long long)r * p.ldc + c0 + cl;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        float t8[8];
+        if (use_c && r < p.M && c0 + cl + g * 8 < p.N) {
+          unpack8(*reinterpret_cast<const uint4*>(crow + g * 8), f16, t8);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t8[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) cin[g * 8 + e] = t8[e];
+      }
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        *reinterpret_cast<float4*>(sF + rr * FP + cl + g * 4) =
+            make_float4(fmaf(p.beta, cin[g * 4], p.alpha * v[g * 4]),
+                        fmaf(p.beta, cin[g * 4 + 1], p.alpha * v[g * 4 + 1]),
+                        fmaf(p.beta, cin[g * 4 + 2], p.alpha * v[g * 4 + 2]),
+                        fmaf(p.beta, cin[g * 4 + 3], p.alpha * v[g * 4 + 3]));
     }
   }
+  if (last_slab) {
+    // every TMEM read of this accumulator is done: hand it back to the MMA warp
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acc_empty_bar);
+  }
   epi_bar();
-  if (!ok) return;
-  (void)r;
 
   // 3. staging -> global (coalesced)
-  if (store_mode) {
-    constexpr int CPR = BN / 8;
-    const bool diag = p.sym && ti == tj;
-    uint16_t* dbase = p.D + (long long)bz * p.d_bs;
-    uint16_t* d2base = p.D2 ? p.D2 + (long long)bz * p.d_bs : nullptr;
-    // direct tile (on diagonal tiles: lower triangle from sC, upper from sT)
-    for (int idx = et; idx < BM * CPR; idx += 128) {
-      const int row = idx / CPR, cc = idx % CPR;
-      if (row >= rows_valid || cc * 8 >= cols_valid) continue;
-      uint4 w = *reinterpret_cast<const uint4*>(sC + row * SP + cc * 8);
-      if (diag && cc * 8 + 7 > row) {
-        if (cc * 8 > row) {
-          w = *reinterpret_cast<const uint4*>(sT + row * TP + cc * 8);
-        } else {
+  if (cols_valid > 0) {
+    if (store_mode) {
+      const bool diag = p.sym && tc.ti == tc.tj;
+      uint16_t* dbase = p.D + (long long)tc.bz * p.d_bs;
+      uint16_t* d2base = p.D2 ? p.D2 + (long long)tc.bz * p.d_bs : nullptr;
+      for (int idx = et; idx < BM * 16; idx += kEpiThreads) {
+        const int row = idx >> 4, cc = idx & 15;
+        if (row >= rows_valid || cc * 8 >= cols_valid) continue;
+        uint4 w = *reinterpret_cast<const uint4*>(sC + row * SP + cc * 8);
+        if (diag && cc * 8 + 7 > row) {
+          // upper part of a diagonal tile = mirror of its lower part
           uint16_t hv[8];
           *reinterpret_cast<uint4*>(hv) = w;
 #pragma unroll
@@ -306,117 +353,126 @@ __device__ __forceinline__ void epilogue(const GemmParams& p, uint8_t* base, uin
             if (cc * 8 + e > row) hv[e] = sT[row * TP + cc * 8 + e];
           w = *reinterpret_cast<const uint4*>(hv);
         }
-      }
-      const long long goff = (long long)(r0 + row) * p.ldd + c0 + cc * 8;
-      *reinterpret_cast<uint4*>(dbase + goff) = w;
-      if (d2base) {
-        if (diag && cc * 8 <= row && row < cc * 8 + 8) {
-          uint16_t hv[8];
-          *reinterpret_cast<uint4*>(hv) = w;
-          hv[row - cc * 8] = d2diag[row];
-          w = *reinterpret_cast<const uint4*>(hv);
-        }
-        *reinterpret_cast<uint4*>(d2base + goff) = w;
-      }
-    }
-    // mirrored tile D[c0 + j][r0 + i] = sT[j][i] (off-diagonal tiles)
-    if (p.sym && !diag) {
-      constexpr int TPR = BM / 8;
-      for (int idx = et; idx < BN * TPR; idx += 128) {
-        const int row = idx / TPR, cc = idx % TPR;   // row: tile column j; cc: chunk of tile rows
-        if (row >= cols_valid || cc * 8 >= rows_valid) continue;
-        const uint4 w = *reinterpret_cast<const uint4*>(sT + row * TP + cc * 8);
-        const long long goff = (long long)(c0 + row) * p.ldd + r0 + cc * 8;
+        const long long goff = (long long)(r0 + row) * p.ldd + c0 + cc * 8;
         *reinterpret_cast<uint4*>(dbase + goff) = w;
-        if (d2base) *reinterpret_cast<uint4*>(d2base + goff) = w;
-      }
-    }
-  } else {
-    // fp32 values -> O (any dtype) or W -= eta (O + wd W), natural orientation.
-    // Eight 16-byte accesses per thread are issued before any is consumed.
-    const int ld = p.mode == EPI_OUT ? p.ldo : p.ldw;
-    constexpr int NB = 8;
-    constexpr int kChunks = BM * BN / 4;
-    const bool tr = p.transpose_out != 0;
-    for (int b0 = 0; b0 < kChunks; b0 += 128 * NB) {
-      float4 val[NB], wv[NB];
-      long long off[NB];
-      bool okc[NB];
-#pragma unroll
-      for (int u = 0; u < NB; ++u) {
-        const int idx = b0 + u * 128 + et;
-        int row, col;   // tile coordinates of the first of four consecutive natural elements
-        if (!tr) {
-          row = idx / (BN / 4);
-          col = (idx % (BN / 4)) * 4;
-          okc[u] = row < rows_valid && col < cols_valid;
-          off[u] = (long long)(r0 + row) * ld + c0 + col;
-          if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + row * FP + col);
-        } else {
-          col = idx / (BM / 4);            // tile column = natural row
-          row = (idx % (BM / 4)) * 4;      // tile rows = natural columns
-          okc[u] = col < cols_valid && row < rows_valid;
-          off[u] = (long long)(c0 + col) * ld + r0 + row;
-          if (okc[u])
-            val[u] = make_float4(sF[row * FP + col], sF[(row + 1) * FP + col],
-                                 sF[(row + 2) * FP + col], sF[(row + 3) * FP + col]);
+        if (d2base) {
+          if (diag && cc * 8 <= row && row < cc * 8 + 8) {
+            uint16_t hv[8];
+            *reinterpret_cast<uint4*>(hv) = w;
+            hv[row - cc * 8] = d2diag[row];
+            w = *reinterpret_cast<const uint4*>(hv);
+          }
+          *reinterpret_cast<uint4*>(d2base + goff) = w;
         }
-        if (p.mode == EPI_WUPDATE && okc[u])
-          wv[u] = *reinterpret_cast<const float4*>(p.W + (long long)bz * p.w_bs + off[u]);
       }
+      if (p.sym && !diag) {
+        // mirrored tile D[c0 + j][r0 + i] = sT[j][i]
+        for (int idx = et; idx < 128 * (BM / 8); idx += kEpiThreads) {
+          const int row = idx / (BM / 8), cc = idx % (BM / 8);
+          if (row >= cols_valid || cc * 8 >= rows_valid) continue;
+          const uint4 w = *reinterpret_cast<const uint4*>(sT + row * TP + cc * 8);
+          const long long goff = (long long)(c0 + row) * p.ldd + r0 + cc * 8;
+          *reinterpret_cast<uint4*>(dbase + goff) = w;
+          if (d2base) *reinterpret_cast<uint4*>(d2base + goff) = w;
+        }
+      }
+    } else {
+      // fp32 values -> O (any dtype) or W -= eta (O + wd W), natural orientation;
+      // eight 16-byte accesses per thread are issued before any is consumed
+      const int ld = p.mode == EPI_OUT ? p.ldo : p.ldw;
+      constexpr int NB = 4;
+      constexpr int kChunks = BM * 128 / 4;
+      const bool tr = p.transpose_out != 0;
+      for (int b0 = 0; b0 < kChunks; b0 += kEpiThreads * NB) {
+        float4 val[NB], wv[NB];
+        long long off[NB];
+        bool okc[NB];
 #pragma unroll
-      for (int u = 0; u < NB; ++u) {
-        if (!okc[u]) continue;
-        if (p.mode == EPI_OUT) {
-          store4_from_float(p.O, (long long)bz * p.o_bs + off[u], p.odt, val[u]);
-        } else {
-          float4 w = wv[u];
-          w.x -= p.eta * (val[u].x + p.wd * w.x);
-          w.y -= p.eta * (val[u].y + p.wd * w.y);
-          w.z -= p.eta * (val[u].z + p.wd * w.z);
-          w.w -= p.eta * (val[u].w + p.wd * w.w);
-          *reinterpret_cast<float4*>(p.W + (long long)bz * p.w_bs + off[u]) = w;
+        for (int u = 0; u < NB; ++u) {
+          const int idx = b0 + u * kEpiThreads + et;
+          int row, col;
+          if (!tr) {
+            row = idx >> 5;
+            col = (idx & 31) * 4;
+            okc[u] = row < rows_valid && col < cols_valid;
+            off[u] = (long long)(r0 + row) * ld + c0 + col;
+            if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + row * FP + col);
+          } else {
+            col = idx >> 5;             // slab column = natural row
+            row = (idx & 31) * 4;       // tile rows = natural columns
+            okc[u] = col < cols_valid && row < rows_valid;
+            off[u] = (long long)(c0 + col) * ld + r0 + row;
+            if (okc[u])
+              val[u] = make_float4(sF[row * FP + col], sF[(row + 1) * FP + col],
+                                   sF[(row + 2) * FP + col], sF[(row + 3) * FP + col]);
+          }
+          if (p.mode == EPI_WUPDATE && okc[u])
+            wv[u] = *reinterpret_cast<const float4*>(p.W + (long long)tc.bz * p.w_bs + off[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < NB; ++u) {
+          if (!okc[u]) continue;
+          if (p.mode == EPI_OUT) {
+            store4_from_float(p.O, (long long)tc.bz * p.o_bs + off[u], p.odt, val[u]);
+          } else {
+            float4 w = wv[u];
+            w.x -= p.eta * (val[u].x + p.wd * w.x);
+            w.y -= p.eta * (val[u].y + p.wd * w.y);
+            w.z -= p.eta * (val[u].z + p.wd * w.z);
+            w.w -= p.eta * (val[u].w + p.wd * w.w);
+            *reinterpret_cast<float4*>(p.W + (long long)tc.bz * p.w_bs + off[u]) = w;
+          }
         }
       }
     }
   }
+  epi_bar();   // staging free for the next slab / tile
 }
 
 // ------------------------------------------------------------------ kernel
-template <int BN, bool B_MN>
-__global__ void __launch_bounds__(kGemmThreads, 2)
+// Persistent: one CTA per SM walks the flattened (batch, tile) list with a
+// stride of gridDim.x. Warp 0 streams operand k-blocks through a STAGES-deep
+// ring, continuously across tiles; warp 1 accumulates each tile into one of two
+// TMEM accumulators; warps 2..9 drain the other accumulator meanwhile.
+template <int BN, bool B_MN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreadsP, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const GemmParams p) {
   if (p.skip && *p.skip) return;
   constexpr uint32_t kABytes = BM * BK * 2;
   constexpr uint32_t kBBytes = BN * BK * 2;
   constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  constexpr uint32_t kTmemCols = BN;   // fp32 accumulator columns (power of 2 >= 32)
+  constexpr uint32_t kTmemCols = 2 * BN;   // two accumulators (power of two, <= 512)
 
   extern __shared__ __align__(1024) uint8_t dsm[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + smem_data_bytes<BN>());
-  uint64_t* empty = full + kStages;
-  uint64_t* accum = empty + kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  uint8_t* stg = base + STAGES * kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg + kStagingBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;     // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2]
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  int* consumed = abort_flag + 1;   // k-blocks whose full barrier the MMA warp waited on
-  uint16_t* d2diag = reinterpret_cast<uint16_t*>(consumed + 2);   // [BM] second-output diagonal
+  int* consumed = abort_flag + 1;
+  uint16_t* d2diag = reinterpret_cast<uint16_t*>(consumed + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bz = blockIdx.y;
-  int ti, tj;
-  if (p.sym) tri_tile(blockIdx.x, ti, tj);
-  else { ti = blockIdx.x % p.tiles_m; tj = blockIdx.x / p.tiles_m; }
+  const int tiles_per = p.sym ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
+  const int total = p.batch * tiles_per;
   const int nk = cdiv(p.K, BK);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    mbar_init(smem_u32(accum), 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&acc_full[a]), 1);
+      mbar_init(smem_u32(&acc_empty[a]), kEpiWarps);
+    }
+    mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     *consumed = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -437,64 +493,96 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   const uint32_t tmem = *tmem_slot;
 
   int issued = 0;   // producer only
-  if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kStages;
-      const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
-      if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err)) { *abort_flag = 1; break; }
-      const uint32_t a_dst = smem_u32(base + s * kStageBytes);
-      const uint32_t b_dst = a_dst + kABytes;
-      const uint32_t bar = smem_u32(&full[s]);
-      mbar_expect_tx(bar, kStageBytes);
-      tma_load_3d(a_dst, &tmA, bar, kb * BK, ti * BM, bz);
-      if (!B_MN) {
-        tma_load_3d(b_dst, &tmB, bar, kb * BK, tj * BN, bz);
-      } else {
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      uint32_t g = 0;
+      bool ok = true;
+      for (int T = blockIdx.x; T < total && ok; T += gridDim.x) {
+        const TileCoord tc = decode_tile(p, T, tiles_per);
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int s = (int)(g % STAGES);
+          const uint32_t ph = (g / STAGES) & 1u;
+          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err)) { ok = false; break; }
+          const uint32_t a_dst = smem_u32(base + s * kStageBytes);
+          const uint32_t b_dst = a_dst + kABytes;
+          const uint32_t bar = smem_u32(&full[s]);
+          mbar_expect_tx(bar, kStageBytes);
+          tma_load_3d(a_dst, &tmA, bar, kb * BK, tc.ti * BM, tc.bz);
+          if (!B_MN) {
+            tma_load_3d(b_dst, &tmB, bar, kb * BK, tc.tj * BN, tc.bz);
+          } else {
 #pragma unroll
-        for (int c = 0; c < BN / 64; ++c)
-          tma_load_3d(b_dst + c * (BK * 128), &tmB, bar, tj * BN + c * 64, kb * BK, bz);
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_3d(b_dst + c * (BK * 128), &tmB, bar, tc.tj * BN + c * 64, kb * BK, tc.bz);
+          }
+        }
       }
-      issued = kb + 1;
+      if (!ok) *abort_flag = 1;
+      issued = (int)g;
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
-    constexpr uint32_t idesc = idesc_f16(false, B_MN, BN);
-    const uint32_t idesc_rt = p.f16 ? idesc_f16(true, B_MN, BN) : idesc;
-    bool ok = true;
-    int kb = 0;
-    for (; kb < nk; ++kb) {
-      const int s = kb % kStages;
-      const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
-      if (!mbar_wait(smem_u32(&full[s]), ph, p.err)) { ok = false; break; }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      const uint32_t idesc = idesc_f16(p.f16 != 0, B_MN, BN);
+      uint32_t g = 0;
+      bool ok = true;
+      int it = 0;
+      for (int T = blockIdx.x; T < total && ok; T += gridDim.x, ++it) {
+        const int ab = it & 1;
+        const uint32_t use = (uint32_t)(it >> 1);
+        if (!mbar_wait(smem_u32(&acc_empty[ab]), (use & 1u) ^ 1u, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(ab * BN);
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int s = (int)(g % STAGES);
+          const uint32_t ph = (g / STAGES) & 1u;
+          if (!mbar_wait(smem_u32(&full[s]), ph, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(base + s * kStageBytes);
+          const uint32_t b_base = a_base + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = sdesc(a_base + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc(b_base + kk * 2048, BK * 128, 1024)
+                                     : sdesc(b_base + kk * 32, 16, 1024);
+            umma(d, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&empty[s]));
+        }
+        if (!ok) break;
+        umma_commit(smem_u32(&acc_full[ab]));
+      }
+      *consumed = (int)g;
+      if (!ok) *abort_flag = 1;
+      // every MMA issued above has completed once this barrier fires
+      umma_commit(smem_u32(drain));
+      mbar_wait(smem_u32(drain), 0, p.err);
+    }
+  } else {
+    // ---------------- epilogue warps
+    int it = 0;
+    for (int T = blockIdx.x; T < total; T += gridDim.x, ++it) {
+      const int ab = it & 1;
+      const uint32_t use = (uint32_t)(it >> 1);
+      const TileCoord tc = decode_tile(p, T, tiles_per);
+      const bool ok = mbar_wait(smem_u32(&acc_full[ab]), use & 1u, p.err);
       tc_fence_after();
-      const uint32_t a_base = smem_u32(base + s * kStageBytes);
-      const uint32_t b_base = a_base + kABytes;
-#pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk) {
-        const uint64_t ad = sdesc(a_base + kk * 32, 16, 1024);
-        const uint64_t bd = B_MN ? sdesc(b_base + kk * 2048, BK * 128, 1024)
-                                 : sdesc(b_base + kk * 32, 16, 1024);
-        umma(tmem, ad, bd, idesc_rt, (kb | kk) ? 1u : 0u);
-      }
-      umma_commit(smem_u32(&empty[s]));   // frees the stage once these MMAs finish
+      // the eight epilogue warps share named barriers: leave together or not at all
+      if (epi_any(!ok || *abort_flag)) break;
+      const uint32_t tacc = tmem + (uint32_t)(ab * BN);
+#pragma unroll 1
+      for (int slab = 0; slab < BN / 128; ++slab)
+        epilogue_slab<BN>(p, stg, tacc, tc, slab, warp, lane, d2diag, slab == BN / 128 - 1,
+                          smem_u32(&acc_empty[ab]));
     }
-    *consumed = kb;
-    if (!ok) *abort_flag = 1;
-    // Arrives once every MMA issued above has completed, abort or not.
-    umma_commit(smem_u32(accum));
-  } else if (warp >= 2) {
-    // ---------------- epilogue
-    const bool ok = mbar_wait(smem_u32(accum), 0, p.err);
-    tc_fence_after();
-    epilogue<BN>(p, base, tmem, ok && !*abort_flag, ti, tj, bz, warp, lane, d2diag);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0 && lane == 0) {
-    // After an abort, let the copies still in flight land before the CTA exits.
-    for (int kb = *consumed; kb < issued; ++kb)
-      mbar_wait(smem_u32(&full[kb % kStages]), (uint32_t)(kb / kStages) & 1u, p.err);
+    // after an abort, let the copies still in flight land before the CTA exits
+    for (int g = *consumed; g < issued; ++g)
+      mbar_wait(smem_u32(&full[g % STAGES]), (uint32_t)(g / STAGES) & 1u, p.err);
   }
   if (warp == 1) {
     tc_fence_after();
@@ -534,20 +622,40 @@ bool make_map(CUtensorMap* map, const void* base, bool f16, int rows, int cols, 
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool B_MN>
-cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int batch,
-                        cudaStream_t s) {
-  constexpr int smem = smem_data_bytes<BN>() + 1024 + 512;
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int BN, bool B_MN, int STAGES>
+cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b, GemmParams p, int batch,
+                          cudaStream_t s) {
+  constexpr int smem = (int)gemm_smem_bytes<BN, STAGES>();
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm<BN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(k_gemm<BN, B_MN, STAGES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
+  p.batch = batch;
   const int tiles = p.sym ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
-  dim3 grid(tiles, batch);
-  k_gemm<BN, B_MN><<<grid, kGemmThreads, smem, s>>>(a, b, p);
+  const int total = tiles * batch;
+  const int grid = total < num_sms() ? total : num_sms();
+  k_gemm<BN, B_MN, STAGES><<<grid, kGemmThreadsP, smem, s>>>(a, b, p);
   return cudaGetLastError();
+}
+
+template <int BN, bool B_MN>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int batch,
+                        cudaStream_t s) {
+  return launch_gemm_t<BN, B_MN, BN == 128 ? 4 : 3>(a, b, p, batch, s);
 }
 
 GemmParams base_params(int M, int N, int K, bool f16, const int32_t* skip, int32_t* err) {
