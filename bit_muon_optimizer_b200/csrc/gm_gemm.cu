@@ -169,19 +169,22 @@ __device__ __forceinline__ void tri_tile(int x, int& ti, int& tj) {
 
 // ------------------------------------------------------------------ epilogue
 // Staging buffers (separate from the operand ring, which keeps streaming the
-// next tile while this one is written out), one 128-column slab at a time:
-//   EPI_STORE : sC [BM][SP] 16-bit (C tile in, output out, in place)
-//               sT [128][TP] 16-bit (transposed output, for mirrored stores)
-//   otherwise : sF [BM][FP] fp32 output values
+// next tile while this one is written out), one 32-column slab at a time:
+//   EPI_STORE : sC [BM][SP] 16-bit (C slab in, output out, in place)
+//               sT [32][TP] 16-bit (transposed output, for mirrored stores)
+//   otherwise : sF [BM][FP] fp32, or its transpose [32][FT] for transposed output
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kGemmThreadsP = 64 + kEpiThreads;
-constexpr int SP = 128 + 8;
+constexpr int SLAB = 32;
+constexpr int SP = SLAB + 8;
 constexpr int TP = BM + 8;
-constexpr int FP = 128 + 4;
+constexpr int FP = SLAB + 4;
+constexpr int FT = BM + 4;
+constexpr uint32_t cmax_u(uint32_t a, uint32_t b) { return a > b ? a : b; }
 constexpr uint32_t kStagingBytes =
-    (uint32_t)(BM * SP * 2 + 128 * TP * 2) > (uint32_t)(BM * FP * 4) ? (uint32_t)(BM * SP * 2 + 128 * TP * 2)
-                                                                     : (uint32_t)(BM * FP * 4);
+    cmax_u(cmax_u(BM * SP * 2 + SLAB * TP * 2, BM * FP * 4), SLAB * FT * 4);
+constexpr int kPrefetchDist = 12;  // k-blocks prefetched into L2 ahead of the loads
 
 template <int BN, int STAGES>
 __host__ __device__ constexpr uint32_t gemm_smem_bytes() {
@@ -208,7 +211,28 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void unpack8(const uint4 w, bool f16, float (&o)[8]) {
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void unpack8(const uint4 w, bool f16, float* o) {
   const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
@@ -216,7 +240,7 @@ __device__ __forceinline__ void unpack8(const uint4 w, bool f16, float (&o)[8]) 
     o[2 * e + 1] = h16_to_float(u[e] >> 16, f16);
   }
 }
-__device__ __forceinline__ uint4 pack8(const float (&v)[8], bool f16) {
+__device__ __forceinline__ uint4 pack8(const float* v, bool f16) {
   uint32_t u[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e)
@@ -236,35 +260,37 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int T, int
   return c;
 }
 
-// One output slab (128 columns of the tile) from TMEM through staging to global.
-// Returns false if the tile's accumulator could not be waited for.
+// One 32-column slab of the tile: TMEM -> registers -> staging -> global.
 template <int BN>
 __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg, uint32_t tacc,
                                               const TileCoord& tc, int slab, int warp, int lane,
                                               uint16_t* d2diag, bool last_slab, uint32_t acc_empty_bar) {
   const int et = threadIdx.x - 64;          // 0..255
   const int q = warp & 3;                   // TMEM lane quarter of this warp
-  const int half = (warp - 2) >> 2;         // 64-column half of the slab
+  const int sub = (warp - 2) >> 2;          // 16-column half of the slab
   const int rr = q * 32 + lane;             // tile row owned by this thread
   const int r0 = tc.ti * BM;
-  const int cs0 = slab * 128;               // slab column offset inside the tile
+  const int cs0 = slab * SLAB;              // slab column offset inside the tile
   const int c0 = tc.tj * BN + cs0;          // global column of the slab
   const int r = r0 + rr;
   const bool f16 = p.f16 != 0;
   const bool store_mode = p.mode == EPI_STORE;
+  const bool tr = p.transpose_out != 0;
   uint16_t* sC = reinterpret_cast<uint16_t*>(stg);
   uint16_t* sT = sC + BM * SP;
   float* sF = reinterpret_cast<float*>(stg);
   const int rows_valid = min(BM, p.M - r0);
-  const int cols_valid = min(128, p.N - c0);   // may be <= 0 for a ragged last slab
+  const int cols_valid = min(SLAB, p.N - c0);   // may be <= 0 for a ragged tile
   const bool use_c = p.C && p.beta != 0.f;
   const long long cbs = (long long)tc.bz * p.c_bs;
 
   // 1. C slab -> sC (store mode; coalesced 16-byte loads)
   if (store_mode && use_c) {
     const uint16_t* cbase = p.C + cbs + (long long)r0 * p.ldc + c0;
-    for (int idx = et; idx < BM * 16; idx += kEpiThreads) {
-      const int row = idx >> 4, cc = idx & 15;
+#pragma unroll
+    for (int u = 0; u < (BM * SLAB / 8) / kEpiThreads; ++u) {
+      const int idx = et + u * kEpiThreads;
+      const int row = idx >> 2, cc = idx & 3;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (row < rows_valid && cc * 8 < cols_valid)
         v = *reinterpret_cast<const uint4*>(cbase + (long long)row * p.ldc + cc * 8);
@@ -274,15 +300,13 @@ __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg,
   epi_bar();
 
   // 2. TMEM -> registers -> epilogue math -> staging
-#pragma unroll 1
-  for (int ch = 0; ch < 2; ++ch) {
-    const int cl = half * 64 + ch * 32;   // column inside the slab
-    float v[32];
-    __syncwarp();
-    tmem_ld32(tacc + ((uint32_t)(q * 32) << 16) + (uint32_t)(cs0 + cl), v);
+  {
+    const int cl = sub * 16;   // column inside the slab
+    float v[16];
+    tmem_ld16(tacc + ((uint32_t)(q * 32) << 16) + (uint32_t)(cs0 + cl), v);
     if (store_mode) {
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
+      for (int g = 0; g < 2; ++g) {
         float cin[8];
         if (use_c) unpack8(*reinterpret_cast<const uint4*>(sC + rr * SP + cl + g * 8), f16, cin);
         float x[8];
@@ -302,28 +326,24 @@ __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg,
         }
       }
     } else {
-      // O = alpha acc + beta C, C read straight from global (one 64-byte row run)
-      float cin[32];
+      // O = alpha acc + beta C, C read straight from global (32-byte row runs)
       const uint16_t* crow = p.C + cbs + (long long)r * p.ldc + c0 + cl;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        float t8[8];
+      for (int g = 0; g < 2; ++g) {
+        float cin[8];
         if (use_c && r < p.M && c0 + cl + g * 8 < p.N) {
-          unpack8(*reinterpret_cast<const uint4*>(crow + g * 8), f16, t8);
+          unpack8(*reinterpret_cast<const uint4*>(crow + g * 8), f16, cin);
         } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) t8[e] = 0.f;
+          for (int e = 0; e < 8; ++e) cin[e] = 0.f;
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) cin[g * 8 + e] = t8[e];
+        for (int e = 0; e < 8; ++e) {
+          const float val = fmaf(p.beta, cin[e], p.alpha * v[g * 8 + e]);
+          if (!tr) sF[rr * FP + cl + g * 8 + e] = val;
+          else sF[(cl + g * 8 + e) * FT + rr] = val;
+        }
       }
-#pragma unroll
-      for (int g = 0; g < 8; ++g)
-        *reinterpret_cast<float4*>(sF + rr * FP + cl + g * 4) =
-            make_float4(fmaf(p.beta, cin[g * 4], p.alpha * v[g * 4]),
-                        fmaf(p.beta, cin[g * 4 + 1], p.alpha * v[g * 4 + 1]),
-                        fmaf(p.beta, cin[g * 4 + 2], p.alpha * v[g * 4 + 2]),
-                        fmaf(p.beta, cin[g * 4 + 3], p.alpha * v[g * 4 + 3]));
     }
   }
   if (last_slab) {
@@ -340,93 +360,100 @@ __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg,
       const bool diag = p.sym && tc.ti == tc.tj;
       uint16_t* dbase = p.D + (long long)tc.bz * p.d_bs;
       uint16_t* d2base = p.D2 ? p.D2 + (long long)tc.bz * p.d_bs : nullptr;
-      for (int idx = et; idx < BM * 16; idx += kEpiThreads) {
-        const int row = idx >> 4, cc = idx & 15;
-        if (row >= rows_valid || cc * 8 >= cols_valid) continue;
-        uint4 w = *reinterpret_cast<const uint4*>(sC + row * SP + cc * 8);
-        if (diag && cc * 8 + 7 > row) {
-          // upper part of a diagonal tile = mirror of its lower part
-          uint16_t hv[8];
-          *reinterpret_cast<uint4*>(hv) = w;
+      // direct pass; on a diagonal tile only positions on or below the diagonal
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            if (cc * 8 + e > row) hv[e] = sT[row * TP + cc * 8 + e];
-          w = *reinterpret_cast<const uint4*>(hv);
-        }
+      for (int u = 0; u < (BM * SLAB / 8) / kEpiThreads; ++u) {
+        const int idx = et + u * kEpiThreads;
+        const int row = idx >> 2, cc = idx & 3;
+        if (row >= rows_valid || cc * 8 >= cols_valid) continue;
+        const int gc = cs0 + cc * 8;          // tile column of the chunk
+        if (diag && gc > row) continue;
+        uint16_t hv[8], h2[8];
+        *reinterpret_cast<uint4*>(hv) = *reinterpret_cast<const uint4*>(sC + row * SP + cc * 8);
+        *reinterpret_cast<uint4*>(h2) = *reinterpret_cast<const uint4*>(hv);
+        if (diag && row < gc + 8) h2[row - gc] = d2diag[row];
         const long long goff = (long long)(r0 + row) * p.ldd + c0 + cc * 8;
-        *reinterpret_cast<uint4*>(dbase + goff) = w;
-        if (d2base) {
-          if (diag && cc * 8 <= row && row < cc * 8 + 8) {
-            uint16_t hv[8];
-            *reinterpret_cast<uint4*>(hv) = w;
-            hv[row - cc * 8] = d2diag[row];
-            w = *reinterpret_cast<const uint4*>(hv);
+        if (diag && gc + 7 > row) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (gc + e <= row) {
+              dbase[goff + e] = hv[e];
+              if (d2base) d2base[goff + e] = h2[e];
+            }
           }
-          *reinterpret_cast<uint4*>(d2base + goff) = w;
+        } else {
+          *reinterpret_cast<uint4*>(dbase + goff) = *reinterpret_cast<const uint4*>(hv);
+          if (d2base) *reinterpret_cast<uint4*>(d2base + goff) = *reinterpret_cast<const uint4*>(h2);
         }
       }
-      if (p.sym && !diag) {
-        // mirrored tile D[c0 + j][r0 + i] = sT[j][i]
-        for (int idx = et; idx < 128 * (BM / 8); idx += kEpiThreads) {
-          const int row = idx / (BM / 8), cc = idx % (BM / 8);
+      if (p.sym) {
+        // mirror pass: D[c0 + j][r0 + i] = value(i, j); on a diagonal tile only i > j
+#pragma unroll
+        for (int u = 0; u < (SLAB * BM / 8) / kEpiThreads; ++u) {
+          const int idx = et + u * kEpiThreads;
+          const int row = idx >> 4, cc = idx & 15;   // row: slab column j; cc: chunk of tile rows
           if (row >= cols_valid || cc * 8 >= rows_valid) continue;
-          const uint4 w = *reinterpret_cast<const uint4*>(sT + row * TP + cc * 8);
+          const int tcol = cs0 + row;                 // tile column j
+          if (diag && cc * 8 + 7 <= tcol) continue;
+          uint16_t hv[8];
+          *reinterpret_cast<uint4*>(hv) = *reinterpret_cast<const uint4*>(sT + row * TP + cc * 8);
           const long long goff = (long long)(c0 + row) * p.ldd + r0 + cc * 8;
-          *reinterpret_cast<uint4*>(dbase + goff) = w;
-          if (d2base) *reinterpret_cast<uint4*>(d2base + goff) = w;
+          if (diag && cc * 8 <= tcol) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              if (cc * 8 + e > tcol) {
+                dbase[goff + e] = hv[e];
+                if (d2base) d2base[goff + e] = hv[e];
+              }
+            }
+          } else {
+            *reinterpret_cast<uint4*>(dbase + goff) = *reinterpret_cast<const uint4*>(hv);
+            if (d2base) *reinterpret_cast<uint4*>(d2base + goff) = *reinterpret_cast<const uint4*>(hv);
+          }
         }
       }
     } else {
       // fp32 values -> O (any dtype) or W -= eta (O + wd W), natural orientation;
-      // eight 16-byte accesses per thread are issued before any is consumed
+      // all of a thread's 16-byte accesses are issued before any is consumed
       const int ld = p.mode == EPI_OUT ? p.ldo : p.ldw;
-      constexpr int NB = 4;
-      constexpr int kChunks = BM * 128 / 4;
-      const bool tr = p.transpose_out != 0;
-      for (int b0 = 0; b0 < kChunks; b0 += kEpiThreads * NB) {
-        float4 val[NB], wv[NB];
-        long long off[NB];
-        bool okc[NB];
+      constexpr int NB = (BM * SLAB / 4) / kEpiThreads;   // 4
+      float4 val[NB], wv[NB];
+      long long off[NB];
+      bool okc[NB];
 #pragma unroll
-        for (int u = 0; u < NB; ++u) {
-          const int idx = b0 + u * kEpiThreads + et;
-          int row, col;
-          if (!tr) {
-            row = idx >> 5;
-            col = (idx & 31) * 4;
-            okc[u] = row < rows_valid && col < cols_valid;
-            off[u] = (long long)(r0 + row) * ld + c0 + col;
-            if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + row * FP + col);
-          } else {
-            col = idx >> 5;             // slab column = natural row
-            row = (idx & 31) * 4;       // tile rows = natural columns
-            okc[u] = col < cols_valid && row < rows_valid;
-            off[u] = (long long)(c0 + col) * ld + r0 + row;
-            if (okc[u])
-              val[u] = make_float4(sF[row * FP + col], sF[(row + 1) * FP + col],
-                                   sF[(row + 2) * FP + col], sF[(row + 3) * FP + col]);
-          }
-          if (p.mode == EPI_WUPDATE && okc[u])
-            wv[u] = *reinterpret_cast<const float4*>(p.W + (long long)tc.bz * p.w_bs + off[u]);
+      for (int u = 0; u < NB; ++u) {
+        const int idx = et + u * kEpiThreads;
+        if (!tr) {
+          const int row = idx >> 3, col = (idx & 7) * 4;
+          okc[u] = row < rows_valid && col < cols_valid;
+          off[u] = (long long)(r0 + row) * ld + c0 + col;
+          if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + row * FP + col);
+        } else {
+          const int col = idx >> 5, row = (idx & 31) * 4;   // slab column = natural row
+          okc[u] = col < cols_valid && row < rows_valid;
+          off[u] = (long long)(c0 + col) * ld + r0 + row;
+          if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + col * FT + row);
         }
+        if (p.mode == EPI_WUPDATE && okc[u])
+          wv[u] = *reinterpret_cast<const float4*>(p.W + (long long)tc.bz * p.w_bs + off[u]);
+      }
 #pragma unroll
-        for (int u = 0; u < NB; ++u) {
-          if (!okc[u]) continue;
-          if (p.mode == EPI_OUT) {
-            store4_from_float(p.O, (long long)tc.bz * p.o_bs + off[u], p.odt, val[u]);
-          } else {
-            float4 w = wv[u];
-            w.x -= p.eta * (val[u].x + p.wd * w.x);
-            w.y -= p.eta * (val[u].y + p.wd * w.y);
-            w.z -= p.eta * (val[u].z + p.wd * w.z);
-            w.w -= p.eta * (val[u].w + p.wd * w.w);
-            *reinterpret_cast<float4*>(p.W + (long long)tc.bz * p.w_bs + off[u]) = w;
-          }
+      for (int u = 0; u < NB; ++u) {
+        if (!okc[u]) continue;
+        if (p.mode == EPI_OUT) {
+          store4_from_float(p.O, (long long)tc.bz * p.o_bs + off[u], p.odt, val[u]);
+        } else {
+          float4 w = wv[u];
+          w.x -= p.eta * (val[u].x + p.wd * w.x);
+          w.y -= p.eta * (val[u].y + p.wd * w.y);
+          w.z -= p.eta * (val[u].z + p.wd * w.z);
+          w.w -= p.eta * (val[u].w + p.wd * w.w);
+          *reinterpret_cast<float4*>(p.W + (long long)tc.bz * p.w_bs + off[u]) = w;
         }
       }
     }
   }
-  epi_bar();   // staging free for the next slab / tile
+  epi_bar();   // staging free for the next slab
 }
 
 // ------------------------------------------------------------------ kernel
@@ -498,11 +525,28 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
       // ---------------- TMA producer
       uint32_t g = 0;
       bool ok = true;
+      // L2 prefetch cursor, kPrefetchDist k-blocks ahead of the loads
+      const int my_tiles = (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+      const long long gtotal = (long long)my_tiles * nk;
+      auto prefetch = [&](long long gp) {
+        if (gp >= gtotal) return;
+        const TileCoord pc = decode_tile(p, (int)blockIdx.x + (int)(gp / nk) * (int)gridDim.x, tiles_per);
+        const int pkb = (int)(gp % nk);
+        tma_prefetch_3d(&tmA, pkb * BK, pc.ti * BM, pc.bz);
+        if (!B_MN) {
+          tma_prefetch_3d(&tmB, pkb * BK, pc.tj * BN, pc.bz);
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN / 64; ++c) tma_prefetch_3d(&tmB, pc.tj * BN + c * 64, pkb * BK, pc.bz);
+        }
+      };
+      for (int i = 0; i < kPrefetchDist; ++i) prefetch(i);
       for (int T = blockIdx.x; T < total && ok; T += gridDim.x) {
         const TileCoord tc = decode_tile(p, T, tiles_per);
         for (int kb = 0; kb < nk; ++kb, ++g) {
           const int s = (int)(g % STAGES);
           const uint32_t ph = (g / STAGES) & 1u;
+          prefetch((long long)g + kPrefetchDist);
           if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err)) { ok = false; break; }
           const uint32_t a_dst = smem_u32(base + s * kStageBytes);
           const uint32_t b_dst = a_dst + kABytes;
@@ -572,8 +616,8 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
       if (epi_any(!ok || *abort_flag)) break;
       const uint32_t tacc = tmem + (uint32_t)(ab * BN);
 #pragma unroll 1
-      for (int slab = 0; slab < BN / 128; ++slab)
-        epilogue_slab<BN>(p, stg, tacc, tc, slab, warp, lane, d2diag, slab == BN / 128 - 1,
+      for (int slab = 0; slab < BN / SLAB; ++slab)
+        epilogue_slab<BN>(p, stg, tacc, tc, slab, warp, lane, d2diag, slab == BN / SLAB - 1,
                           smem_u32(&acc_empty[ab]));
     }
   }
@@ -655,8 +699,10 @@ cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b, GemmParams
 template <int BN, bool B_MN>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int batch,
                         cudaStream_t s) {
-  return launch_gemm_t<BN, B_MN, BN == 128 ? 4 : 3>(a, b, p, batch, s);
+  return launch_gemm_t<BN, B_MN, BN == 128 ? 6 : 4>(a, b, p, batch, s);
 }
+
+constexpr int kLeftBN = 256;   // output tile width of the S X products
 
 GemmParams base_params(int M, int N, int K, bool f16, const int32_t* skip, int32_t* err) {
   GemmParams p;
@@ -717,7 +763,7 @@ cudaError_t leftmul(const Ns& c, const uint16_t* S, const uint16_t* X, float alp
   if (!make_map(&mb, X, c.f16, c.N, c.Mp, c.Mp, c.B, (long long)c.N * c.Mp, BK)) return cudaErrorInvalidValue;
   GemmParams p = base_params(c.N, c.Mp, c.N, c.f16, c.skip, c.err);
   p.tiles_m = cdiv(c.N, BM);
-  p.tiles_n = cdiv(c.Mp, 128);
+  p.tiles_n = cdiv(c.Mp, kLeftBN);
   p.alpha = alpha; p.beta = beta;
   p.C = X; p.c_bs = (long long)c.N * c.Mp; p.ldc = c.Mp;
   if (!out) {
@@ -735,7 +781,7 @@ cudaError_t leftmul(const Ns& c, const uint16_t* S, const uint16_t* X, float alp
       p.eta = out->eta; p.wd = out->wd;
     }
   }
-  return launch_gemm<128, true>(ma, mb, p, c.B, c.s);
+  return launch_gemm<kLeftBN, true>(ma, mb, p, c.B, c.s);
 }
 
 #define GM_TRY(x)                          \
