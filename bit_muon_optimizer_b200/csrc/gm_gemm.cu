@@ -260,11 +260,42 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int T, int
   return c;
 }
 
+// C values of one slab, fetched into registers one slab ahead of their use.
+// Store mode: thread et holds rows et/4 (+64), 8-column chunk et%4 (the sC fill
+// pattern). Output modes: the thread's own row, its 16-column half of the slab.
+template <int BN>
+__device__ __forceinline__ void c_prefetch(const GemmParams& p, const TileCoord& tc, int slab,
+                                           int warp, int lane, uint4 (&cpre)[2]) {
+  cpre[0] = cpre[1] = make_uint4(0, 0, 0, 0);
+  if (!p.C || p.beta == 0.f) return;
+  const int r0 = tc.ti * BM;
+  const int c0 = tc.tj * BN + slab * SLAB;
+  const long long cbs = (long long)tc.bz * p.c_bs;
+  if (p.mode == EPI_STORE) {
+    const int et = threadIdx.x - 64;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int idx = et + u * kEpiThreads;
+      const int row = idx >> 2, cc = idx & 3;
+      if (r0 + row < p.M && c0 + cc * 8 < p.N)
+        cpre[u] = *reinterpret_cast<const uint4*>(p.C + cbs + (long long)(r0 + row) * p.ldc + c0 + cc * 8);
+    }
+  } else {
+    const int r = r0 + (warp & 3) * 32 + lane;
+    const int cl = ((warp - 2) >> 2) * 16;
+#pragma unroll
+    for (int g = 0; g < 2; ++g)
+      if (r < p.M && c0 + cl + g * 8 < p.N)
+        cpre[g] = *reinterpret_cast<const uint4*>(p.C + cbs + (long long)r * p.ldc + c0 + cl + g * 8);
+  }
+}
+
 // One 32-column slab of the tile: TMEM -> registers -> staging -> global.
 template <int BN>
 __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg, uint32_t tacc,
                                               const TileCoord& tc, int slab, int warp, int lane,
-                                              uint16_t* d2diag, bool last_slab, uint32_t acc_empty_bar) {
+                                              uint16_t* d2diag, bool last_slab, uint32_t acc_empty_bar,
+                                              uint4 (&cpre)[2]) {
   const int et = threadIdx.x - 64;          // 0..255
   const int q = warp & 3;                   // TMEM lane quarter of this warp
   const int sub = (warp - 2) >> 2;          // 16-column half of the slab
@@ -282,21 +313,17 @@ __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg,
   const int rows_valid = min(BM, p.M - r0);
   const int cols_valid = min(SLAB, p.N - c0);   // may be <= 0 for a ragged tile
   const bool use_c = p.C && p.beta != 0.f;
-  const long long cbs = (long long)tc.bz * p.c_bs;
 
-  // 1. C slab -> sC (store mode; coalesced 16-byte loads)
+  // 1. C slab (fetched one slab ahead) -> sC; start fetching the next slab
+  uint4 cnow[2] = {cpre[0], cpre[1]};
   if (store_mode && use_c) {
-    const uint16_t* cbase = p.C + cbs + (long long)r0 * p.ldc + c0;
 #pragma unroll
-    for (int u = 0; u < (BM * SLAB / 8) / kEpiThreads; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int idx = et + u * kEpiThreads;
-      const int row = idx >> 2, cc = idx & 3;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (row < rows_valid && cc * 8 < cols_valid)
-        v = *reinterpret_cast<const uint4*>(cbase + (long long)row * p.ldc + cc * 8);
-      *reinterpret_cast<uint4*>(sC + row * SP + cc * 8) = v;
+      *reinterpret_cast<uint4*>(sC + (idx >> 2) * SP + (idx & 3) * 8) = cnow[u];
     }
   }
+  if (!last_slab) c_prefetch<BN>(p, tc, slab + 1, warp, lane, cpre);
   epi_bar();
 
   // 2. TMEM -> registers -> epilogue math -> staging
@@ -326,17 +353,11 @@ __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg,
         }
       }
     } else {
-      // O = alpha acc + beta C, C read straight from global (32-byte row runs)
-      const uint16_t* crow = p.C + cbs + (long long)r * p.ldc + c0 + cl;
+      // O = alpha acc + beta C (this thread's C values were fetched a slab ahead)
 #pragma unroll
       for (int g = 0; g < 2; ++g) {
         float cin[8];
-        if (use_c && r < p.M && c0 + cl + g * 8 < p.N) {
-          unpack8(*reinterpret_cast<const uint4*>(crow + g * 8), f16, cin);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) cin[e] = 0.f;
-        }
+        unpack8(cnow[g], f16, cin);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float val = fmaf(p.beta, cin[e], p.alpha * v[g * 8 + e]);
@@ -525,13 +546,11 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
       // ---------------- TMA producer
       uint32_t g = 0;
       bool ok = true;
-      // L2 prefetch cursor, kPrefetchDist k-blocks ahead of the loads
-      const int my_tiles = (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-      const long long gtotal = (long long)my_tiles * nk;
-      auto prefetch = [&](long long gp) {
-        if (gp >= gtotal) return;
-        const TileCoord pc = decode_tile(p, (int)blockIdx.x + (int)(gp / nk) * (int)gridDim.x, tiles_per);
-        const int pkb = (int)(gp % nk);
+      // L2 prefetch cursor (tile pT, k-block pkb), kPrefetchDist k-blocks ahead of the loads
+      int pT = blockIdx.x, pkb = 0;
+      TileCoord pc = decode_tile(p, pT, tiles_per);
+      auto prefetch_next = [&]() {
+        if (pT >= total) return;
         tma_prefetch_3d(&tmA, pkb * BK, pc.ti * BM, pc.bz);
         if (!B_MN) {
           tma_prefetch_3d(&tmB, pkb * BK, pc.tj * BN, pc.bz);
@@ -539,14 +558,19 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
 #pragma unroll
           for (int c = 0; c < BN / 64; ++c) tma_prefetch_3d(&tmB, pc.tj * BN + c * 64, pkb * BK, pc.bz);
         }
+        if (++pkb == nk) {
+          pkb = 0;
+          pT += gridDim.x;
+          if (pT < total) pc = decode_tile(p, pT, tiles_per);
+        }
       };
-      for (int i = 0; i < kPrefetchDist; ++i) prefetch(i);
+      for (int i = 0; i < kPrefetchDist; ++i) prefetch_next();
       for (int T = blockIdx.x; T < total && ok; T += gridDim.x) {
         const TileCoord tc = decode_tile(p, T, tiles_per);
         for (int kb = 0; kb < nk; ++kb, ++g) {
           const int s = (int)(g % STAGES);
           const uint32_t ph = (g / STAGES) & 1u;
-          prefetch((long long)g + kPrefetchDist);
+          prefetch_next();
           if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err)) { ok = false; break; }
           const uint32_t a_dst = smem_u32(base + s * kStageBytes);
           const uint32_t b_dst = a_dst + kABytes;
@@ -610,6 +634,8 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
       const int ab = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
       const TileCoord tc = decode_tile(p, T, tiles_per);
+      uint4 cpre[2];
+      c_prefetch<BN>(p, tc, 0, warp, lane, cpre);   // overlaps the MMAs of this tile
       const bool ok = mbar_wait(smem_u32(&acc_full[ab]), use & 1u, p.err);
       tc_fence_after();
       // the eight epilogue warps share named barriers: leave together or not at all
@@ -618,7 +644,7 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
 #pragma unroll 1
       for (int slab = 0; slab < BN / SLAB; ++slab)
         epilogue_slab<BN>(p, stg, tacc, tc, slab, warp, lane, d2diag, slab == BN / SLAB - 1,
-                          smem_u32(&acc_empty[ab]));
+                          smem_u32(&acc_empty[ab]), cpre);
     }
   }
   tc_fence_before();
