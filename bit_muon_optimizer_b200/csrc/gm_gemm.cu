@@ -176,7 +176,16 @@ __device__ __forceinline__ void tri_tile(int x, int& ti, int& tj) {
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kGemmThreadsP = 64 + kEpiThreads;
-constexpr int SLAB = 32;
+#ifndef GM_EPI_SLAB
+#define GM_EPI_SLAB 32
+#endif
+#ifndef GM_PREFETCH_DIST
+#define GM_PREFETCH_DIST 12
+#endif
+#ifndef GM_LEFT_BN
+#define GM_LEFT_BN 256
+#endif
+constexpr int SLAB = GM_EPI_SLAB;      // epilogue columns staged at a time (32, 64 or 128)
 constexpr int SP = SLAB + 8;
 constexpr int TP = BM + 8;
 constexpr int FP = SLAB + 4;
@@ -184,7 +193,7 @@ constexpr int FT = BM + 4;
 constexpr uint32_t cmax_u(uint32_t a, uint32_t b) { return a > b ? a : b; }
 constexpr uint32_t kStagingBytes =
     cmax_u(cmax_u(BM * SP * 2 + SLAB * TP * 2, BM * FP * 4), SLAB * FT * 4);
-constexpr int kPrefetchDist = 12;  // k-blocks prefetched into L2 ahead of the loads
+constexpr int kPrefetchDist = GM_PREFETCH_DIST;  // k-blocks prefetched into L2 ahead (0: none)
 
 template <int BN, int STAGES>
 __host__ __device__ constexpr uint32_t gemm_smem_bytes() {
@@ -261,12 +270,15 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int T, int
 }
 
 // C values of one slab, fetched into registers one slab ahead of their use.
-// Store mode: thread et holds rows et/4 (+64), 8-column chunk et%4 (the sC fill
-// pattern). Output modes: the thread's own row, its 16-column half of the slab.
+// Store mode: thread et holds the sC fill chunks idx = et + u * 256. Output
+// modes: the thread's own row, its SLAB/2-column half of the slab.
+constexpr int NCH = SLAB / 16;   // 16-byte C chunks per thread per slab
+
 template <int BN>
 __device__ __forceinline__ void c_prefetch(const GemmParams& p, const TileCoord& tc, int slab,
-                                           int warp, int lane, uint4 (&cpre)[2]) {
-  cpre[0] = cpre[1] = make_uint4(0, 0, 0, 0);
+                                           int warp, int lane, uint4 (&cpre)[NCH]) {
+#pragma unroll
+  for (int u = 0; u < NCH; ++u) cpre[u] = make_uint4(0, 0, 0, 0);
   if (!p.C || p.beta == 0.f) return;
   const int r0 = tc.ti * BM;
   const int c0 = tc.tj * BN + slab * SLAB;
@@ -274,31 +286,41 @@ __device__ __forceinline__ void c_prefetch(const GemmParams& p, const TileCoord&
   if (p.mode == EPI_STORE) {
     const int et = threadIdx.x - 64;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < NCH; ++u) {
       const int idx = et + u * kEpiThreads;
-      const int row = idx >> 2, cc = idx & 3;
+      const int row = idx / (SLAB / 8), cc = idx % (SLAB / 8);
       if (r0 + row < p.M && c0 + cc * 8 < p.N)
         cpre[u] = *reinterpret_cast<const uint4*>(p.C + cbs + (long long)(r0 + row) * p.ldc + c0 + cc * 8);
     }
   } else {
     const int r = r0 + (warp & 3) * 32 + lane;
-    const int cl = ((warp - 2) >> 2) * 16;
+    const int cl = ((warp - 2) >> 2) * (SLAB / 2);
 #pragma unroll
-    for (int g = 0; g < 2; ++g)
+    for (int g = 0; g < NCH; ++g)
       if (r < p.M && c0 + cl + g * 8 < p.N)
         cpre[g] = *reinterpret_cast<const uint4*>(p.C + cbs + (long long)r * p.ldc + c0 + cl + g * 8);
   }
 }
 
-// One 32-column slab of the tile: TMEM -> registers -> staging -> global.
+__device__ __forceinline__ uint32_t pack2(float a, float b, bool f16) {
+  if (f16) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// One SLAB-column slab of the tile: TMEM -> registers -> staging -> global.
 template <int BN>
 __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg, uint32_t tacc,
                                               const TileCoord& tc, int slab, int warp, int lane,
                                               uint16_t* d2diag, bool last_slab, uint32_t acc_empty_bar,
-                                              uint4 (&cpre)[2]) {
+                                              uint4 (&cpre)[NCH]) {
+  constexpr int CPW = SLAB / 2;             // columns per warp
   const int et = threadIdx.x - 64;          // 0..255
   const int q = warp & 3;                   // TMEM lane quarter of this warp
-  const int sub = (warp - 2) >> 2;          // 16-column half of the slab
+  const int sub = (warp - 2) >> 2;          // column half of the slab
   const int rr = q * 32 + lane;             // tile row owned by this thread
   const int r0 = tc.ti * BM;
   const int cs0 = slab * SLAB;              // slab column offset inside the tile
@@ -313,43 +335,64 @@ __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg,
   const int rows_valid = min(BM, p.M - r0);
   const int cols_valid = min(SLAB, p.N - c0);   // may be <= 0 for a ragged tile
   const bool use_c = p.C && p.beta != 0.f;
+  const float alpha = p.alpha, beta = p.beta;
 
   // 1. C slab (fetched one slab ahead) -> sC; start fetching the next slab
-  uint4 cnow[2] = {cpre[0], cpre[1]};
+  uint4 cnow[NCH];
+#pragma unroll
+  for (int u = 0; u < NCH; ++u) cnow[u] = cpre[u];
   if (store_mode && use_c) {
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < NCH; ++u) {
       const int idx = et + u * kEpiThreads;
-      *reinterpret_cast<uint4*>(sC + (idx >> 2) * SP + (idx & 3) * 8) = cnow[u];
+      *reinterpret_cast<uint4*>(sC + (idx / (SLAB / 8)) * SP + (idx % (SLAB / 8)) * 8) = cnow[u];
     }
   }
   if (!last_slab) c_prefetch<BN>(p, tc, slab + 1, warp, lane, cpre);
   epi_bar();
 
   // 2. TMEM -> registers -> epilogue math -> staging
-  {
-    const int cl = sub * 16;   // column inside the slab
+#pragma unroll
+  for (int h = 0; h < CPW / 16; ++h) {
+    const int cl = sub * CPW + h * 16;   // column inside the slab
     float v[16];
     tmem_ld16(tacc + ((uint32_t)(q * 32) << 16) + (uint32_t)(cs0 + cl), v);
+    const bool has_diag = r >= c0 + cl && r < c0 + cl + 16;
     if (store_mode) {
 #pragma unroll
       for (int g = 0; g < 2; ++g) {
-        float cin[8];
-        if (use_c) unpack8(*reinterpret_cast<const uint4*>(sC + rr * SP + cl + g * 8), f16, cin);
         float x[8];
+        if (use_c) {
+          float cin[8];
+          unpack8(*reinterpret_cast<const uint4*>(sC + rr * SP + cl + g * 8), f16, cin);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          x[e] = p.alpha * v[g * 8 + e];
-          if (use_c) x[e] = fmaf(p.beta, cin[e], x[e]);
-          if (c0 + cl + g * 8 + e == r) {
-            x[e] += p.gamma;
-            if (p.D2) d2diag[rr] = float_to_h16(x[e] + p.gamma2, f16);
+          for (int e = 0; e < 8; ++e) x[e] = fmaf(beta, cin[e], alpha * v[g * 8 + e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = alpha * v[g * 8 + e];
+        }
+        if (has_diag) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (c0 + cl + g * 8 + e == r) {
+              x[e] += p.gamma;
+              if (p.D2) d2diag[rr] = float_to_h16(x[e] + p.gamma2, f16);
+            }
           }
         }
-        *reinterpret_cast<uint4*>(sC + rr * SP + cl + g * 8) = pack8(x, f16);
+        uint4 w;
+        w.x = pack2(x[0], x[1], f16);
+        w.y = pack2(x[2], x[3], f16);
+        w.z = pack2(x[4], x[5], f16);
+        w.w = pack2(x[6], x[7], f16);
+        *reinterpret_cast<uint4*>(sC + rr * SP + cl + g * 8) = w;
         if (p.sym) {
+          const uint32_t u4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) sT[(cl + g * 8 + e) * TP + rr] = float_to_h16(x[e], f16);
+          for (int e = 0; e < 4; ++e) {
+            sT[(cl + g * 8 + 2 * e) * TP + rr] = (uint16_t)(u4[e] & 0xFFFF);
+            sT[(cl + g * 8 + 2 * e + 1) * TP + rr] = (uint16_t)(u4[e] >> 16);
+          }
         }
       }
     } else {
@@ -357,10 +400,10 @@ __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg,
 #pragma unroll
       for (int g = 0; g < 2; ++g) {
         float cin[8];
-        unpack8(cnow[g], f16, cin);
+        unpack8(cnow[h * 2 + g], f16, cin);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float val = fmaf(p.beta, cin[e], p.alpha * v[g * 8 + e]);
+          const float val = fmaf(beta, cin[e], alpha * v[g * 8 + e]);
           if (!tr) sF[rr * FP + cl + g * 8 + e] = val;
           else sF[(cl + g * 8 + e) * FT + rr] = val;
         }
@@ -383,43 +426,43 @@ __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg,
       uint16_t* d2base = p.D2 ? p.D2 + (long long)tc.bz * p.d_bs : nullptr;
       // direct pass; on a diagonal tile only positions on or below the diagonal
 #pragma unroll
-      for (int u = 0; u < (BM * SLAB / 8) / kEpiThreads; ++u) {
+      for (int u = 0; u < NCH; ++u) {
         const int idx = et + u * kEpiThreads;
-        const int row = idx >> 2, cc = idx & 3;
+        const int row = idx / (SLAB / 8), cc = idx % (SLAB / 8);
         if (row >= rows_valid || cc * 8 >= cols_valid) continue;
         const int gc = cs0 + cc * 8;          // tile column of the chunk
         if (diag && gc > row) continue;
-        uint16_t hv[8], h2[8];
-        *reinterpret_cast<uint4*>(hv) = *reinterpret_cast<const uint4*>(sC + row * SP + cc * 8);
-        *reinterpret_cast<uint4*>(h2) = *reinterpret_cast<const uint4*>(hv);
-        if (diag && row < gc + 8) h2[row - gc] = d2diag[row];
+        const uint4 w = *reinterpret_cast<const uint4*>(sC + row * SP + cc * 8);
         const long long goff = (long long)(r0 + row) * p.ldd + c0 + cc * 8;
-        if (diag && gc + 7 > row) {
+        if (diag && gc + 7 >= row) {
+          uint16_t hv[8];
+          *reinterpret_cast<uint4*>(hv) = w;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             if (gc + e <= row) {
               dbase[goff + e] = hv[e];
-              if (d2base) d2base[goff + e] = h2[e];
+              if (d2base) d2base[goff + e] = (gc + e == row) ? d2diag[row] : hv[e];
             }
           }
         } else {
-          *reinterpret_cast<uint4*>(dbase + goff) = *reinterpret_cast<const uint4*>(hv);
-          if (d2base) *reinterpret_cast<uint4*>(d2base + goff) = *reinterpret_cast<const uint4*>(h2);
+          *reinterpret_cast<uint4*>(dbase + goff) = w;
+          if (d2base) *reinterpret_cast<uint4*>(d2base + goff) = w;
         }
       }
       if (p.sym) {
         // mirror pass: D[c0 + j][r0 + i] = value(i, j); on a diagonal tile only i > j
 #pragma unroll
-        for (int u = 0; u < (SLAB * BM / 8) / kEpiThreads; ++u) {
+        for (int u = 0; u < NCH; ++u) {
           const int idx = et + u * kEpiThreads;
           const int row = idx >> 4, cc = idx & 15;   // row: slab column j; cc: chunk of tile rows
           if (row >= cols_valid || cc * 8 >= rows_valid) continue;
           const int tcol = cs0 + row;                 // tile column j
           if (diag && cc * 8 + 7 <= tcol) continue;
-          uint16_t hv[8];
-          *reinterpret_cast<uint4*>(hv) = *reinterpret_cast<const uint4*>(sT + row * TP + cc * 8);
+          const uint4 w = *reinterpret_cast<const uint4*>(sT + row * TP + cc * 8);
           const long long goff = (long long)(c0 + row) * p.ldd + r0 + cc * 8;
           if (diag && cc * 8 <= tcol) {
+            uint16_t hv[8];
+            *reinterpret_cast<uint4*>(hv) = w;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               if (cc * 8 + e > tcol) {
@@ -428,48 +471,52 @@ __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg,
               }
             }
           } else {
-            *reinterpret_cast<uint4*>(dbase + goff) = *reinterpret_cast<const uint4*>(hv);
-            if (d2base) *reinterpret_cast<uint4*>(d2base + goff) = *reinterpret_cast<const uint4*>(hv);
+            *reinterpret_cast<uint4*>(dbase + goff) = w;
+            if (d2base) *reinterpret_cast<uint4*>(d2base + goff) = w;
           }
         }
       }
     } else {
       // fp32 values -> O (any dtype) or W -= eta (O + wd W), natural orientation;
-      // all of a thread's 16-byte accesses are issued before any is consumed
+      // four 16-byte accesses per thread in flight at a time
       const int ld = p.mode == EPI_OUT ? p.ldo : p.ldw;
-      constexpr int NB = (BM * SLAB / 4) / kEpiThreads;   // 4
-      float4 val[NB], wv[NB];
-      long long off[NB];
-      bool okc[NB];
+      constexpr int NB = 4;
+      constexpr int kQ = BM * SLAB / 4;   // float4 chunks per slab
+#pragma unroll 1
+      for (int b0 = 0; b0 < kQ; b0 += kEpiThreads * NB) {
+        float4 val[NB], wv[NB];
+        long long off[NB];
+        bool okc[NB];
 #pragma unroll
-      for (int u = 0; u < NB; ++u) {
-        const int idx = et + u * kEpiThreads;
-        if (!tr) {
-          const int row = idx >> 3, col = (idx & 7) * 4;
-          okc[u] = row < rows_valid && col < cols_valid;
-          off[u] = (long long)(r0 + row) * ld + c0 + col;
-          if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + row * FP + col);
-        } else {
-          const int col = idx >> 5, row = (idx & 31) * 4;   // slab column = natural row
-          okc[u] = col < cols_valid && row < rows_valid;
-          off[u] = (long long)(c0 + col) * ld + r0 + row;
-          if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + col * FT + row);
+        for (int u = 0; u < NB; ++u) {
+          const int idx = b0 + et + u * kEpiThreads;
+          if (!tr) {
+            const int row = idx / (SLAB / 4), col = (idx % (SLAB / 4)) * 4;
+            okc[u] = row < rows_valid && col < cols_valid;
+            off[u] = (long long)(r0 + row) * ld + c0 + col;
+            if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + row * FP + col);
+          } else {
+            const int col = idx >> 5, row = (idx & 31) * 4;   // slab column = natural row
+            okc[u] = col < cols_valid && row < rows_valid;
+            off[u] = (long long)(c0 + col) * ld + r0 + row;
+            if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + col * FT + row);
+          }
+          if (p.mode == EPI_WUPDATE && okc[u])
+            wv[u] = *reinterpret_cast<const float4*>(p.W + (long long)tc.bz * p.w_bs + off[u]);
         }
-        if (p.mode == EPI_WUPDATE && okc[u])
-          wv[u] = *reinterpret_cast<const float4*>(p.W + (long long)tc.bz * p.w_bs + off[u]);
-      }
 #pragma unroll
-      for (int u = 0; u < NB; ++u) {
-        if (!okc[u]) continue;
-        if (p.mode == EPI_OUT) {
-          store4_from_float(p.O, (long long)tc.bz * p.o_bs + off[u], p.odt, val[u]);
-        } else {
-          float4 w = wv[u];
-          w.x -= p.eta * (val[u].x + p.wd * w.x);
-          w.y -= p.eta * (val[u].y + p.wd * w.y);
-          w.z -= p.eta * (val[u].z + p.wd * w.z);
-          w.w -= p.eta * (val[u].w + p.wd * w.w);
-          *reinterpret_cast<float4*>(p.W + (long long)tc.bz * p.w_bs + off[u]) = w;
+        for (int u = 0; u < NB; ++u) {
+          if (!okc[u]) continue;
+          if (p.mode == EPI_OUT) {
+            store4_from_float(p.O, (long long)tc.bz * p.o_bs + off[u], p.odt, val[u]);
+          } else {
+            float4 w = wv[u];
+            w.x -= p.eta * (val[u].x + p.wd * w.x);
+            w.y -= p.eta * (val[u].y + p.wd * w.y);
+            w.z -= p.eta * (val[u].z + p.wd * w.z);
+            w.w -= p.eta * (val[u].w + p.wd * w.w);
+            *reinterpret_cast<float4*>(p.W + (long long)tc.bz * p.w_bs + off[u]) = w;
+          }
         }
       }
     }
@@ -565,12 +612,13 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
         }
       };
       for (int i = 0; i < kPrefetchDist; ++i) prefetch_next();
+      const bool do_prefetch = kPrefetchDist > 0;
       for (int T = blockIdx.x; T < total && ok; T += gridDim.x) {
         const TileCoord tc = decode_tile(p, T, tiles_per);
         for (int kb = 0; kb < nk; ++kb, ++g) {
           const int s = (int)(g % STAGES);
           const uint32_t ph = (g / STAGES) & 1u;
-          prefetch_next();
+          if (do_prefetch) prefetch_next();
           if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err)) { ok = false; break; }
           const uint32_t a_dst = smem_u32(base + s * kStageBytes);
           const uint32_t b_dst = a_dst + kABytes;
@@ -634,7 +682,7 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
       const int ab = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
       const TileCoord tc = decode_tile(p, T, tiles_per);
-      uint4 cpre[2];
+      uint4 cpre[NCH];
       c_prefetch<BN>(p, tc, 0, warp, lane, cpre);   // overlaps the MMAs of this tile
       const bool ok = mbar_wait(smem_u32(&acc_full[ab]), use & 1u, p.err);
       tc_fence_after();
@@ -725,10 +773,13 @@ cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b, GemmParams
 template <int BN, bool B_MN>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int batch,
                         cudaStream_t s) {
-  return launch_gemm_t<BN, B_MN, BN == 128 ? 6 : 4>(a, b, p, batch, s);
+  constexpr uint32_t kBudget = 227 * 1024 - 2048 - kStagingBytes;   // ring budget per CTA
+  constexpr int kStagesFit = (int)(kBudget / (BM * BK * 2 + BN * BK * 2));
+  constexpr int kStagesUse = kStagesFit > 8 ? 8 : kStagesFit;
+  return launch_gemm_t<BN, B_MN, kStagesUse>(a, b, p, batch, s);
 }
 
-constexpr int kLeftBN = 256;   // output tile width of the S X products
+constexpr int kLeftBN = GM_LEFT_BN;   // output tile width of the S X products
 
 GemmParams base_params(int M, int N, int K, bool f16, const int32_t* skip, int32_t* err) {
   GemmParams p;
