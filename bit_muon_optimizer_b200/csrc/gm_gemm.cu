@@ -177,10 +177,10 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kGemmThreadsP = 64 + kEpiThreads;
 #ifndef GM_EPI_SLAB
-#define GM_EPI_SLAB 32
+#define GM_EPI_SLAB 64
 #endif
 #ifndef GM_PREFETCH_DIST
-#define GM_PREFETCH_DIST 12
+#define GM_PREFETCH_DIST 0
 #endif
 #ifndef GM_LEFT_BN
 #define GM_LEFT_BN 256
