@@ -70,6 +70,8 @@ _sig("gm_grid_quant4", c_int, [c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, v
 _sig("gm_quant8", c_int, [c_int, c_int, c_int, vp, vp, vp, vp])
 _sig("gm_newton_schulz", c_int, [c_int, c_int, c_int, vp, c_int, vp, c_int, c_float, vp, c_int,
                                  vp, c_size_t, vp])
+_sig("gm_newton_schulz_noalloc", c_int, [c_int, c_int, c_int, vp, c_int, vp, c_int, c_float, vp,
+                                         c_int, vp])
 _sig("gm_gram_ns", c_int, [c_int, c_int, c_int, vp, c_int, vp, c_int, vp, c_int, c_float, vp,
                            c_int, vp, c_size_t, vp])
 _sig("gm_grasp_step", c_int, [c_int, c_int, c_int, ctypes.POINTER(GraspParams),
@@ -210,6 +212,21 @@ def newton_schulz(X, abc=None, T=5, eps=1e-7, out_dtype=torch.float32, out=None,
     _check(lib.gm_newton_schulz(B, m, n, _ptr(X), _DT[X.dtype], abc_table(abc, T), T, eps,
                                 _ptr(O), _DT[out_dtype], _ptr(ws), nb, _stream()),
            "gm_newton_schulz")
+    return O
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def newton_schulz_noalloc(X, abc=None, T=5, eps=1e-7, out_dtype=torch.float32, out=None):
+    """gm_newton_schulz through the entry point that allocates no device memory
+    (its scratch is a fixed 64 MiB array inside the library). ``out`` must be
+    preallocated by callers that cannot allocate either."""
+    B, m, n = _bmn(X)
+    O = out if out is not None else torch.empty((B, m, n), dtype=out_dtype, device=X.device)
+    _check(lib.gm_newton_schulz_noalloc(B, m, n, _ptr(X), _DT[X.dtype], abc_table(abc, T), T, eps,
+                                        _ptr(O), _DT[O.dtype], _stream()),
+           "gm_newton_schulz_noalloc")
     return O
 
 

@@ -150,6 +150,34 @@ gm_status gm_newton_schulz(int B, int m, int n, const void* X, gm_dtype xdt,
                            void* ws, size_t ws_bytes, gm_stream_t stream);
 
 /*
+ * gm_newton_schulz without any device allocation (the paper has no counterpart:
+ * this is a deployment convenience of this library).
+ *
+ * For callers that cannot allocate GPU memory where they need the update --
+ * code running inside a framework that owns every allocation through its own
+ * pool, plugins that may not call the device allocator, or paths where an
+ * allocation would synchronise the device. Same arguments and result as
+ * gm_newton_schulz, minus the workspace: the scratch is a fixed device array of
+ * GM_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits. The call makes no cudaMalloc,
+ * cudaFree or other allocating call.
+ *  - Shapes whose workspace (gm_workspace_bytes(GM_OP_NEWTON_SCHULZ, ...))
+ *    exceeds GM_NOALLOC_SCRATCH_BYTES are rejected with GM_E_WORKSPACE before
+ *    any launch; gm_last_error() states the bytes needed.
+ *  - The first call on a device looks up the scratch array's device address
+ *    (cudaGetSymbolAddress) with that device current and caches it; make that
+ *    first call before any stream capture.
+ *  - All calls share the one scratch array and it keeps the last call's
+ *    contents (nothing in it needs to start at zero: every byte a call reads,
+ *    it first writes). Calls that overlap on the GPU -- different streams, or
+ *    threads enqueueing concurrently -- race on it: serialise them.
+ */
+#define GM_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+gm_status gm_newton_schulz_noalloc(int B, int m, int n, const void* X, gm_dtype xdt,
+                                   const float* abc, int T, float eps,
+                                   void* O, gm_dtype odt, gm_stream_t stream);
+
+/*
  * Stabilized Gram Newton-Schulz [GramNS Algorithm 2; Algorithm 1 with
  * n_restart = 0]: fp16 operands, fp32 accumulation, a_t added in fp32
  * epilogues:
