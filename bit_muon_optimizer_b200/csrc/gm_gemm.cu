@@ -257,15 +257,20 @@ __device__ __forceinline__ uint4 pack8(const float* v, bool f16) {
   return make_uint4(u[0], u[1], u[2], u[3]);
 }
 
+// A tile of the flattened (batch, tile) list. r0 / c0 are the global row /
+// column origins of this CTA's part of the output tile (a CTA owns 128 rows).
 struct TileCoord {
-  int bz, ti, tj;
+  int bz, ti, tj, r0, c0;
 };
-__device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int T, int tiles_per) {
+__device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int T, int tiles_per,
+                                                 int tile_m, int tile_n, int row_off) {
   TileCoord c;
   c.bz = T / tiles_per;
   const int x = T - c.bz * tiles_per;
   if (p.sym) tri_tile(x, c.ti, c.tj);
   else { c.ti = x % p.tiles_m; c.tj = x / p.tiles_m; }
+  c.r0 = c.ti * tile_m + row_off;
+  c.c0 = c.tj * tile_n;
   return c;
 }
 
@@ -280,8 +285,8 @@ __device__ __forceinline__ void c_prefetch(const GemmParams& p, const TileCoord&
 #pragma unroll
   for (int u = 0; u < NCH; ++u) cpre[u] = make_uint4(0, 0, 0, 0);
   if (!p.C || p.beta == 0.f) return;
-  const int r0 = tc.ti * BM;
-  const int c0 = tc.tj * BN + slab * SLAB;
+  const int r0 = tc.r0;
+  const int c0 = tc.c0 + slab * SLAB;
   const long long cbs = (long long)tc.bz * p.c_bs;
   if (p.mode == EPI_STORE) {
     const int et = threadIdx.x - 64;
@@ -316,15 +321,17 @@ template <int BN>
 __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg, uint32_t tacc,
                                               const TileCoord& tc, int slab, int warp, int lane,
                                               uint16_t* d2diag, bool last_slab, uint32_t acc_empty_bar,
-                                              uint4 (&cpre)[NCH]) {
+                                              uint4 (&cpre)[NCH], bool cluster_arrive = false) {
   constexpr int CPW = SLAB / 2;             // columns per warp
   const int et = threadIdx.x - 64;          // 0..255
   const int q = warp & 3;                   // TMEM lane quarter of this warp
   const int sub = (warp - 2) >> 2;          // column half of the slab
   const int rr = q * 32 + lane;             // tile row owned by this thread
-  const int r0 = tc.ti * BM;
+  const int r0 = tc.r0;
   const int cs0 = slab * SLAB;              // slab column offset inside the tile
-  const int c0 = tc.tj * BN + cs0;          // global column of the slab
+  const int c0 = tc.c0 + cs0;               // global column of the slab
+  const int dlt = tc.r0 - tc.c0;            // element (row, tile col j) lies below the
+                                            // diagonal iff dlt + row - j > 0
   const int r = r0 + rr;
   const bool f16 = p.f16 != 0;
   const bool store_mode = p.mode == EPI_STORE;
@@ -414,34 +421,36 @@ __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg,
     // every TMEM read of this accumulator is done: hand it back to the MMA warp
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(acc_empty_bar);
+    if (lane == 0) {
+      if (cluster_arrive) asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(acc_empty_bar) : "memory");
+      else mbar_arrive(acc_empty_bar);
+    }
   }
   epi_bar();
 
   // 3. staging -> global (coalesced)
   if (cols_valid > 0) {
     if (store_mode) {
-      const bool diag = p.sym && tc.ti == tc.tj;
       uint16_t* dbase = p.D + (long long)tc.bz * p.d_bs;
       uint16_t* d2base = p.D2 ? p.D2 + (long long)tc.bz * p.d_bs : nullptr;
-      // direct pass; on a diagonal tile only positions on or below the diagonal
+      // direct pass; for symmetric products only positions on or below the diagonal
 #pragma unroll
       for (int u = 0; u < NCH; ++u) {
         const int idx = et + u * kEpiThreads;
         const int row = idx / (SLAB / 8), cc = idx % (SLAB / 8);
         if (row >= rows_valid || cc * 8 >= cols_valid) continue;
-        const int gc = cs0 + cc * 8;          // tile column of the chunk
-        if (diag && gc > row) continue;
+        const int rel0 = dlt + row - (cs0 + cc * 8);   // for the chunk's first column
+        if (p.sym && rel0 < 0) continue;
         const uint4 w = *reinterpret_cast<const uint4*>(sC + row * SP + cc * 8);
         const long long goff = (long long)(r0 + row) * p.ldd + c0 + cc * 8;
-        if (diag && gc + 7 >= row) {
+        if (p.sym && rel0 < 8) {
           uint16_t hv[8];
           *reinterpret_cast<uint4*>(hv) = w;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            if (gc + e <= row) {
+            if (rel0 - e >= 0) {
               dbase[goff + e] = hv[e];
-              if (d2base) d2base[goff + e] = (gc + e == row) ? d2diag[row] : hv[e];
+              if (d2base) d2base[goff + e] = (rel0 == e) ? d2diag[row] : hv[e];
             }
           }
         } else {
@@ -450,22 +459,22 @@ __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg,
         }
       }
       if (p.sym) {
-        // mirror pass: D[c0 + j][r0 + i] = value(i, j); on a diagonal tile only i > j
+        // mirror pass: D[c0 + j][r0 + i] = value(i, j) for i strictly below the diagonal
 #pragma unroll
         for (int u = 0; u < NCH; ++u) {
           const int idx = et + u * kEpiThreads;
           const int row = idx >> 4, cc = idx & 15;   // row: slab column j; cc: chunk of tile rows
           if (row >= cols_valid || cc * 8 >= rows_valid) continue;
-          const int tcol = cs0 + row;                 // tile column j
-          if (diag && cc * 8 + 7 <= tcol) continue;
+          const int relf = dlt + cc * 8 - (cs0 + row);   // for the chunk's first tile row
+          if (relf + 7 <= 0) continue;
           const uint4 w = *reinterpret_cast<const uint4*>(sT + row * TP + cc * 8);
           const long long goff = (long long)(c0 + row) * p.ldd + r0 + cc * 8;
-          if (diag && cc * 8 <= tcol) {
+          if (relf <= 0) {
             uint16_t hv[8];
             *reinterpret_cast<uint4*>(hv) = w;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              if (cc * 8 + e > tcol) {
+              if (relf + e > 0) {
                 dbase[goff + e] = hv[e];
                 if (d2base) d2base[goff + e] = hv[e];
               }
@@ -595,26 +604,26 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
       bool ok = true;
       // L2 prefetch cursor (tile pT, k-block pkb), kPrefetchDist k-blocks ahead of the loads
       int pT = blockIdx.x, pkb = 0;
-      TileCoord pc = decode_tile(p, pT, tiles_per);
+      TileCoord pc = decode_tile(p, pT, tiles_per, BM, BN, 0);
       auto prefetch_next = [&]() {
         if (pT >= total) return;
-        tma_prefetch_3d(&tmA, pkb * BK, pc.ti * BM, pc.bz);
+        tma_prefetch_3d(&tmA, pkb * BK, pc.r0, pc.bz);
         if (!B_MN) {
-          tma_prefetch_3d(&tmB, pkb * BK, pc.tj * BN, pc.bz);
+          tma_prefetch_3d(&tmB, pkb * BK, pc.c0, pc.bz);
         } else {
 #pragma unroll
-          for (int c = 0; c < BN / 64; ++c) tma_prefetch_3d(&tmB, pc.tj * BN + c * 64, pkb * BK, pc.bz);
+          for (int c = 0; c < BN / 64; ++c) tma_prefetch_3d(&tmB, pc.c0 + c * 64, pkb * BK, pc.bz);
         }
         if (++pkb == nk) {
           pkb = 0;
           pT += gridDim.x;
-          if (pT < total) pc = decode_tile(p, pT, tiles_per);
+          if (pT < total) pc = decode_tile(p, pT, tiles_per, BM, BN, 0);
         }
       };
       for (int i = 0; i < kPrefetchDist; ++i) prefetch_next();
       const bool do_prefetch = kPrefetchDist > 0;
       for (int T = blockIdx.x; T < total && ok; T += gridDim.x) {
-        const TileCoord tc = decode_tile(p, T, tiles_per);
+        const TileCoord tc = decode_tile(p, T, tiles_per, BM, BN, 0);
         for (int kb = 0; kb < nk; ++kb, ++g) {
           const int s = (int)(g % STAGES);
           const uint32_t ph = (g / STAGES) & 1u;
@@ -624,13 +633,13 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
           const uint32_t b_dst = a_dst + kABytes;
           const uint32_t bar = smem_u32(&full[s]);
           mbar_expect_tx(bar, kStageBytes);
-          tma_load_3d(a_dst, &tmA, bar, kb * BK, tc.ti * BM, tc.bz);
+          tma_load_3d(a_dst, &tmA, bar, kb * BK, tc.r0, tc.bz);
           if (!B_MN) {
-            tma_load_3d(b_dst, &tmB, bar, kb * BK, tc.tj * BN, tc.bz);
+            tma_load_3d(b_dst, &tmB, bar, kb * BK, tc.c0, tc.bz);
           } else {
 #pragma unroll
             for (int c = 0; c < BN / 64; ++c)
-              tma_load_3d(b_dst + c * (BK * 128), &tmB, bar, tc.tj * BN + c * 64, kb * BK, tc.bz);
+              tma_load_3d(b_dst + c * (BK * 128), &tmB, bar, tc.c0 + c * 64, kb * BK, tc.bz);
           }
         }
       }
@@ -681,7 +690,7 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
     for (int T = blockIdx.x; T < total; T += gridDim.x, ++it) {
       const int ab = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
-      const TileCoord tc = decode_tile(p, T, tiles_per);
+      const TileCoord tc = decode_tile(p, T, tiles_per, BM, BN, 0);
       uint4 cpre[NCH];
       c_prefetch<BN>(p, tc, 0, warp, lane, cpre);   // overlaps the MMAs of this tile
       const bool ok = mbar_wait(smem_u32(&acc_full[ab]), use & 1u, p.err);
@@ -705,6 +714,227 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ 2-SM kernel
+// A CTA pair (cluster of 2) computes 256 x 256 output tiles with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256): each CTA stages its own 128 rows
+// of A and 128 of the 256 B rows (columns, for an MN-major B) per k-block, so a
+// pair moves 32 KB per SM for 4.2 MFLOP per SM -- half the operand traffic per
+// FLOP of a 128 x 128 tile. Both CTAs' TMA loads complete on the leader's
+// (rank 0) full barrier; the leader's MMA thread commits to both CTAs' empty
+// and accumulator barriers; each CTA drains its own 128 TMEM lanes. No load uses
+// multicast.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// Address of the same shared-memory variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void umma_pair(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the barrier at this offset in both CTAs once the issued MMAs finish.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+  const uint16_t both = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(both)
+      : "memory");
+}
+
+template <bool B_MN, int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreadsP, 1)
+    k_gemm2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            const GemmParams p) {
+  constexpr int BN = 256;                     // tile columns (per CTA accumulator width)
+  constexpr uint32_t kABytes = BM * BK * 2;   // 128 rows of A
+  constexpr uint32_t kBBytes = 128 * BK * 2;  // this CTA's half of B
+  constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  constexpr uint32_t kTmemCols = 2 * BN;      // two 256-column accumulators
+
+  // The skip flag is read by both CTAs of a pair before any cluster-level
+  // operation, so they return together.
+  if (p.skip && *p.skip) return;
+
+  extern __shared__ __align__(1024) uint8_t dsm[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stg = base + STAGES * kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg + kStagingBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;     // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2]
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* consumed = abort_flag + 1;
+  uint16_t* d2diag = reinterpret_cast<uint16_t*>(consumed + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t cr = cluster_rank();
+  const bool leader = cr == 0;
+  const int pid = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int tiles_per = p.sym ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
+  const int total = p.batch * tiles_per;
+  const int nk = cdiv(p.K, BK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&acc_full[a]), 1);
+      mbar_init(smem_u32(&acc_empty[a]), 2 * kEpiWarps);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    *consumed = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    prefetch_map(&tmA);
+    prefetch_map(&tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();   // barriers of both CTAs initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  int issued = 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs)
+      uint32_t g = 0;
+      bool ok = true;
+      for (int T = pid; T < total && ok; T += npairs) {
+        const TileCoord tc = decode_tile(p, T, tiles_per, 2 * BM, BN, (int)cr * BM);
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int s = (int)(g % STAGES);
+          const uint32_t ph = (g / STAGES) & 1u;
+          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err)) { ok = false; break; }
+          const uint32_t a_dst = smem_u32(base + s * kStageBytes);
+          const uint32_t b_dst = a_dst + kABytes;
+          const uint32_t bar = map_to_rank(smem_u32(&full[s]), 0);   // the leader's barrier
+          if (leader) mbar_expect_tx(smem_u32(&full[s]), 2 * kStageBytes);
+          tma_load_3d_pair(a_dst, &tmA, bar, kb * BK, tc.r0, tc.bz);
+          if (!B_MN) {
+            tma_load_3d_pair(b_dst, &tmB, bar, kb * BK, tc.c0 + (int)cr * 128, tc.bz);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              tma_load_3d_pair(b_dst + c * (BK * 128), &tmB, bar, tc.c0 + (int)cr * 128 + c * 64,
+                               kb * BK, tc.bz);
+          }
+        }
+      }
+      if (!ok) *abort_flag = 1;
+      issued = (int)g;
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (leader CTA only)
+      // M = 256 across the pair: replace the descriptor's M field (bits 24..28)
+      const uint32_t idesc = (idesc_f16(p.f16 != 0, B_MN, BN) & ~(0x1Fu << 24)) |
+                             ((uint32_t)((2 * BM) >> 4) << 24);
+      uint32_t g = 0;
+      bool ok = true;
+      int it = 0;
+      for (int T = pid; T < total && ok; T += npairs, ++it) {
+        const int ab = it & 1;
+        const uint32_t use = (uint32_t)(it >> 1);
+        if (!mbar_wait(smem_u32(&acc_empty[ab]), (use & 1u) ^ 1u, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(ab * BN);
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int s = (int)(g % STAGES);
+          const uint32_t ph = (g / STAGES) & 1u;
+          if (!mbar_wait(smem_u32(&full[s]), ph, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(base + s * kStageBytes);
+          const uint32_t b_base = a_base + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = sdesc(a_base + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc(b_base + kk * 2048, BK * 128, 1024)
+                                     : sdesc(b_base + kk * 32, 16, 1024);
+            umma_pair(d, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+          }
+          umma_commit_pair(smem_u32(&empty[s]));
+        }
+        if (!ok) break;
+        umma_commit_pair(smem_u32(&acc_full[ab]));
+      }
+      *consumed = (int)g;
+      if (!ok) *abort_flag = 1;
+      umma_commit_pair(smem_u32(drain));
+      mbar_wait(smem_u32(drain), 0, p.err);
+    }
+  } else {
+    // ---------------- epilogue warps (both CTAs, 128 TMEM lanes each)
+    const uint32_t empty_remote0 = map_to_rank(smem_u32(&acc_empty[0]), 0);
+    const uint32_t empty_remote1 = map_to_rank(smem_u32(&acc_empty[1]), 0);
+    int it = 0;
+    for (int T = pid; T < total; T += npairs, ++it) {
+      const int ab = it & 1;
+      const uint32_t use = (uint32_t)(it >> 1);
+      const TileCoord tc = decode_tile(p, T, tiles_per, 2 * BM, BN, (int)cr * BM);
+      uint4 cpre[NCH];
+      c_prefetch<BN>(p, tc, 0, warp, lane, cpre);
+      const bool ok = mbar_wait(smem_u32(&acc_full[ab]), use & 1u, p.err);
+      tc_fence_after();
+      if (epi_any(!ok || *abort_flag)) break;
+      const uint32_t tacc = tmem + (uint32_t)(ab * BN);
+#pragma unroll 1
+      for (int slab = 0; slab < BN / SLAB; ++slab)
+        epilogue_slab<BN>(p, stg, tacc, tc, slab, warp, lane, d2diag, slab == BN / SLAB - 1,
+                          ab ? empty_remote1 : empty_remote0, cpre, true);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0 && lane == 0 && leader) {
+    // after an abort, let the copies still in flight (from both CTAs) land
+    for (int g = *consumed; g < issued; ++g)
+      mbar_wait(smem_u32(&full[g % STAGES]), (uint32_t)(g / STAGES) & 1u, p.err);
+  }
+  cluster_sync_all();   // neither CTA leaves while the other may still signal it
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
 }
@@ -770,6 +1000,33 @@ cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b, GemmParams
   return cudaGetLastError();
 }
 
+#ifndef GM_PAIR
+#define GM_PAIR 1
+#endif
+constexpr bool kPair = GM_PAIR != 0;   // 2-SM (cta_group::2) 256 x 256 tiles
+
+template <bool B_MN>
+cudaError_t launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, GemmParams p, int batch,
+                             cudaStream_t s) {
+  constexpr uint32_t kBudget = 227 * 1024 - 2048 - kStagingBytes;
+  constexpr int kStagesFit = (int)(kBudget / (2 * BM * BK * 2));
+  constexpr int STAGES = kStagesFit > 8 ? 8 : kStagesFit;
+  constexpr int smem = (int)gemm_smem_bytes<128, STAGES>();
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm2<B_MN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  p.batch = batch;
+  const int tiles = p.sym ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
+  const int total = tiles * batch;
+  const int pairs = total < num_sms() / 2 ? total : num_sms() / 2;
+  k_gemm2<B_MN, STAGES><<<2 * pairs, kGemmThreadsP, smem, s>>>(a, b, p);
+  return cudaGetLastError();
+}
+
 template <int BN, bool B_MN>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int batch,
                         cudaStream_t s) {
@@ -806,9 +1063,10 @@ cudaError_t xxt(const Ns& c, const uint16_t* X, uint16_t* D) {
   CUtensorMap ma;
   if (!make_map(&ma, X, c.f16, c.N, c.Mp, c.Mp, c.B, (long long)c.N * c.Mp, BM)) return cudaErrorInvalidValue;
   GemmParams p = base_params(c.N, c.N, c.Mp, c.f16, c.skip, c.err);
-  p.tiles_m = p.tiles_n = cdiv(c.N, BM);
+  p.tiles_m = p.tiles_n = cdiv(c.N, kPair ? 2 * BM : BM);
   p.sym = 1;
   p.D = D; p.d_bs = (long long)c.N * c.N; p.ldd = c.N;
+  if (kPair) return launch_gemm_pair<false>(ma, ma, p, c.B, c.s);
   return launch_gemm<128, false>(ma, ma, p, c.B, c.s);
 }
 
@@ -821,12 +1079,13 @@ cudaError_t symmul(const Ns& c, const uint16_t* S1, const uint16_t* S2, float al
   if (!make_map(&ma, S1, c.f16, c.N, c.N, c.N, c.B, bs, BM)) return cudaErrorInvalidValue;
   if (!make_map(&mb, S2, c.f16, c.N, c.N, c.N, c.B, bs, 128)) return cudaErrorInvalidValue;
   GemmParams p = base_params(c.N, c.N, c.N, c.f16, c.skip, c.err);
-  p.tiles_m = p.tiles_n = cdiv(c.N, BM);
+  p.tiles_m = p.tiles_n = cdiv(c.N, kPair ? 2 * BM : BM);
   p.sym = 1;
   p.alpha = alpha; p.beta = beta; p.gamma = gamma;
   p.C = Cin; p.c_bs = bs; p.ldc = c.N;
   p.D = D; p.d_bs = bs; p.ldd = c.N;
   p.D2 = D2; p.gamma2 = gamma2;
+  if (kPair) return launch_gemm_pair<false>(ma, mb, p, c.B, c.s);
   return launch_gemm<128, false>(ma, mb, p, c.B, c.s);
 }
 
@@ -839,8 +1098,8 @@ cudaError_t leftmul(const Ns& c, const uint16_t* S, const uint16_t* X, float alp
   // MN-major B operand: rows of X are the K index, columns the N index.
   if (!make_map(&mb, X, c.f16, c.N, c.Mp, c.Mp, c.B, (long long)c.N * c.Mp, BK)) return cudaErrorInvalidValue;
   GemmParams p = base_params(c.N, c.Mp, c.N, c.f16, c.skip, c.err);
-  p.tiles_m = cdiv(c.N, BM);
-  p.tiles_n = cdiv(c.Mp, kLeftBN);
+  p.tiles_m = cdiv(c.N, kPair ? 2 * BM : BM);
+  p.tiles_n = cdiv(c.Mp, kPair ? 256 : kLeftBN);
   p.alpha = alpha; p.beta = beta;
   p.C = X; p.c_bs = (long long)c.N * c.Mp; p.ldc = c.Mp;
   if (!out) {
@@ -858,6 +1117,7 @@ cudaError_t leftmul(const Ns& c, const uint16_t* S, const uint16_t* X, float alp
       p.eta = out->eta; p.wd = out->wd;
     }
   }
+  if (kPair) return launch_gemm_pair<true>(ma, mb, p, c.B, c.s);
   return launch_gemm<kLeftBN, true>(ma, mb, p, c.B, c.s);
 }
 
