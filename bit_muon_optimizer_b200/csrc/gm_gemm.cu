@@ -173,7 +173,10 @@ __device__ __forceinline__ void tri_tile(int x, int& ti, int& tj) {
 //   EPI_STORE : sC [BM][SP] 16-bit (C slab in, output out, in place)
 //               sT [32][TP] 16-bit (transposed output, for mirrored stores)
 //   otherwise : sF [BM][FP] fp32, or its transpose [32][FT] for transposed output
-constexpr int kEpiWarps = 8;
+#ifndef GM_EPI_WARPS
+#define GM_EPI_WARPS 8
+#endif
+constexpr int kEpiWarps = GM_EPI_WARPS;   // 8 or 16: two or four warps per TMEM lane quarter
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kGemmThreadsP = 64 + kEpiThreads;
 #ifndef GM_EPI_SLAB
@@ -201,17 +204,17 @@ __host__ __device__ constexpr uint32_t gemm_smem_bytes() {
          BM * 2 /* second-output diagonal */ + 1024 /* alignment slack */;
 }
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
 
 __device__ __forceinline__ bool epi_any(bool pred) {
   uint32_t res;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 256, p;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}\n"
       : "=r"(res)
-      : "r"((uint32_t)pred)
+      : "r"((uint32_t)pred), "n"(kEpiThreads)
       : "memory");
   return res != 0;
 }
@@ -277,7 +280,10 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int T, int
 // C values of one slab, fetched into registers one slab ahead of their use.
 // Store mode: thread et holds the sC fill chunks idx = et + u * 256. Output
 // modes: the thread's own row, its SLAB/2-column half of the slab.
-constexpr int NCH = SLAB / 16;   // 16-byte C chunks per thread per slab
+constexpr int kWarpsPerQuarter = kEpiWarps / 4;
+constexpr int CPW = SLAB / kWarpsPerQuarter;          // slab columns per epilogue warp
+constexpr int NCH = BM * SLAB / 8 / kEpiThreads;      // 16-byte C chunks per thread per slab
+static_assert(CPW % 16 == 0 && NCH >= 1, "slab too narrow for the epilogue warp count");
 
 template <int BN>
 __device__ __forceinline__ void c_prefetch(const GemmParams& p, const TileCoord& tc, int slab,
@@ -299,7 +305,7 @@ __device__ __forceinline__ void c_prefetch(const GemmParams& p, const TileCoord&
     }
   } else {
     const int r = r0 + (warp & 3) * 32 + lane;
-    const int cl = ((warp - 2) >> 2) * (SLAB / 2);
+    const int cl = ((warp - 2) >> 2) * CPW;
 #pragma unroll
     for (int g = 0; g < NCH; ++g)
       if (r < p.M && c0 + cl + g * 8 < p.N)
@@ -322,10 +328,9 @@ __device__ __forceinline__ void epilogue_slab(const GemmParams& p, uint8_t* stg,
                                               const TileCoord& tc, int slab, int warp, int lane,
                                               uint16_t* d2diag, bool last_slab, uint32_t acc_empty_bar,
                                               uint4 (&cpre)[NCH], bool cluster_arrive = false) {
-  constexpr int CPW = SLAB / 2;             // columns per warp
   const int et = threadIdx.x - 64;          // 0..255
   const int q = warp & 3;                   // TMEM lane quarter of this warp
-  const int sub = (warp - 2) >> 2;          // column half of the slab
+  const int sub = (warp - 2) >> 2;          // column part of the slab
   const int rr = q * 32 + lane;             // tile row owned by this thread
   const int r0 = tc.r0;
   const int cs0 = slab * SLAB;              // slab column offset inside the tile
