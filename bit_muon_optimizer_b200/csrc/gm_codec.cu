@@ -23,7 +23,6 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kTargetCtas = 2 * 148;   // two waves' worth of CTAs on a B200
 
-__device__ __forceinline__ int sext4(int v) { return (v & 0x8) ? (v | ~0xF) : (v & 0xF); }
 
 __device__ __forceinline__ float deq8(int8_t q, float s) {
   return __fmul_rn(__fdiv_rn((float)q, 127.0f), s);
@@ -242,13 +241,15 @@ __global__ void __launch_bounds__(kThreads, 2) k_rebuild_proj(
 
   // 2. factors of the tile into shared memory
   if (t < 16) deq4[t] = __fdiv_rn((float)((t & 8) ? t - 16 : t), 7.0f);
-  for (int e = t; e < kRB * kk; e += kThreads) {
-    const int rr = e / kk, l = e % kk, gi = r0 + rr;
-    Ps[l * kRB + rr] = (gi < m) ? deq8(P8[((long long)b * m + gi) * kk + l], Pscale[b * kk + l]) : 0.f;
-  }
-  for (int e = t; e < kGrid * kk; e += kThreads) {
-    const int cc = e / kk, l = e % kk, gj = c0 + cc;
-    Rs[l * kGrid + cc] = (gj < n) ? deq8(R8[((long long)b * n + gj) * kk + l], Rscale[b * kk + l]) : 0.f;
+  if constexpr (SRC == SRC_STATE) {
+    for (int e = t; e < kRB * kk; e += kThreads) {
+      const int rr = e / kk, l = e % kk, gi = r0 + rr;
+      Ps[l * kRB + rr] = (gi < m) ? deq8(P8[((long long)b * m + gi) * kk + l], Pscale[b * kk + l]) : 0.f;
+    }
+    for (int e = t; e < kGrid * kk; e += kThreads) {
+      const int cc = e / kk, l = e % kk, gj = c0 + cc;
+      Rs[l * kGrid + cc] = (gj < n) ? deq8(R8[((long long)b * n + gj) * kk + l], Rscale[b * kk + l]) : 0.f;
+    }
   }
   for (int e = t; e < kGrid * kq; e += kThreads) {
     const int cc = e / kq, l = e % kq, gj = c0 + cc;

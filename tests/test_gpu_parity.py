@@ -167,7 +167,11 @@ def test_powerit_dead_columns(cuda_lib):
 
 # --------------------------------------------------------------- Newton-Schulz
 
-NS_SHAPES = [(2, 256, 512), (2, 512, 256), (1, 384, 384), (2, 144, 400), (1, 768, 2048)]
+# multiples of 256, ragged 256-row pair tiles (384, 320: a 128-row half entirely
+# outside the matrix or a 64-row box at the edge), a single 64-row block, and
+# shapes that the chains zero-pad to multiples of 64 (144 x 400)
+NS_SHAPES = [(2, 256, 512), (2, 512, 256), (1, 384, 384), (1, 320, 640), (3, 64, 192),
+             (2, 144, 400), (1, 768, 2048)]
 
 
 @pytest.mark.parametrize("B,m,n", NS_SHAPES)
