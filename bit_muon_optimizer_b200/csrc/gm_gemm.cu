@@ -19,11 +19,12 @@
 //   warp 1      : allocates TMEM; lane 0 of the leader CTA issues the MMAs into one
 //                 of two 256-column accumulators while the epilogue drains the other
 //   warp 2      : TMA producer of B     (this CTA's 128 of the 256 B rows or columns)
-//   warp 3      : TMA loads of the epilogue input C, up to two slabs ahead
-//   warp 4      : TMA bulk stores of the staged 16-bit results
-//   warps 5..20 : epilogue: tcgen05.ld (32 lanes x 16 columns), fp32 math, staging
+//   warp 3      : TMA bulk stores of the staged 16-bit results
+//   warps 4..19 : epilogue: tcgen05.ld (32 lanes x 16 columns), fp32 math, staging
 // A thread's bulk-tensor copies are processed one after another, so operand
-// loads come from two threads and each copy moves two k-blocks (32 KB).
+// loads come from two threads and each copy moves two k-blocks (32 KB). Loads
+// take ~1.4 us under load, so the ring keeps three 64 KB stages in flight and
+// the epilogue makes do with two 16 KB staging buffers.
 // Every wait is bounded (~2 s of %globaltimer) and also gives up once another
 // role has flagged an abort; a timeout records GM_E_TIMEOUT in an error word
 // and every role unwinds.
@@ -47,14 +48,14 @@ constexpr int BM = 128;                // output rows per CTA
 constexpr int BN = 256;                // output columns per tile
 constexpr int BK = 64;                 // 64 x 16-bit = 128 B = one swizzle row
 constexpr int KPS = 2;                 // k-blocks per pipeline stage
-constexpr int STAGES = 2;
+constexpr int STAGES = 3;
 constexpr uint32_t kKBlockBytes = 128 * BK * 2;          // 128 rows (or columns) x one k-block
 constexpr uint32_t kABytes = KPS * kKBlockBytes;         // 32 KB
 constexpr uint32_t kBBytes = KPS * kKBlockBytes;         // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;      // 64 KB per CTA
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-constexpr int kEpiWarp0 = 5;
+constexpr int kEpiWarp0 = 4;
 constexpr int kEpiWarps = 16;                            // four per TMEM lane quarter
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
@@ -65,12 +66,10 @@ constexpr int NCH = CPW / 8;                             // 16-byte C chunks per
 static_assert(CPW == 16, "one tcgen05.ld x16 per thread per slab");
 
 constexpr uint32_t kBoxBytes = 64 * 128;                 // 64 x 64 16-bit values
-constexpr uint32_t kOutBufBytes = 4 * kBoxBytes;         // sC (2 boxes) + sT (2 boxes)
-constexpr uint32_t kCBufBytes = 2 * kBoxBytes;           // C rows 0..127 of a slab
-constexpr int FP = SLAB + 4, FT = BM + 4;                // fp32 staging pitches (output modes)
-static_assert(BM * FP * 4 <= 2 * kOutBufBytes && SLAB * FT * 4 <= 2 * kOutBufBytes, "fp32 staging");
+constexpr uint32_t kOutBufBytes = 2 * kBoxBytes;         // rows 0..63 and 64..127 of a slab
+static_assert(BM * SLAB * 4 <= 2 * kOutBufBytes, "fp32 staging (output modes) fits the slab buffers");
 constexpr uint32_t kSmemBytes =
-    STAGES * kStageBytes + 2 * kOutBufBytes + 2 * kCBufBytes + 1024 /* barriers */ + 1024 /* align */;
+    STAGES * kStageBytes + 2 * kOutBufBytes + 1024 /* barriers */ + 1024 /* align */;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 __device__ int32_t g_device_error = 0;
@@ -86,6 +85,7 @@ struct GemmParams {
   int f16;                     // operand / 16-bit output type: 1 fp16, 0 bf16
   float alpha, beta, gamma;    // v = alpha acc + beta Cin + gamma [r == c]
   const uint16_t* C; long long c_bs; int ldc;
+  uint16_t* D; uint16_t* D2; long long d_bs; int ldd;   // 16-bit outputs (EPI_STORE)
   int has_d2; float gamma2;    // symmetric products: D2 = v + gamma2 [r == c]
   int mode;
   int transpose_out;           // EPI_OUT / EPI_WUPDATE: natural = transpose of the tile
@@ -146,15 +146,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
-// 3-D tile load into this CTA's shared memory, completing on this CTA's barrier.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
 // 4-D tile load into this CTA's shared memory, completing on the pair
 // leader's barrier (`bar` is a cluster shared-memory address).
 __device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
@@ -172,14 +163,6 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t sr
                    reinterpret_cast<uint64_t>(map)),
                "r"(src), "r"(c0), "r"(c1), "r"(c2)
                : "memory");
-}
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1,
-                                             int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Bulk stores committed so far have finished reading shared memory.
@@ -299,19 +282,18 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int T, int
 }
 
 // ------------------------------------------------------------------ epilogue
-// 16-bit results (EPI_STORE) leave through 64 x 64 boxes in the 128-byte
-// swizzled layout, two slab buffers alternating:
-//   sC [2 boxes] : rows 0..63 / 64..127 of the tile, the slab's 64 columns
-//   sT [2 boxes] : the same values transposed (mirror stores of symmetric
-//                  products), or, in a diagonal box, the second output D2.
-// For a symmetric product every 64 x 64 box strictly below the diagonal is
-// stored with its transpose; a box on the diagonal is made exactly symmetric in
-// shared memory (each lower value written at (i, j) and (j, i)) and stored once;
-// boxes strictly above are not stored. The C input of a slab arrives by TMA in
-// the same swizzled layout. The epilogue warps never wait for one another:
-// slab_full (all epilogue warps staged a slab), buf_free (the stores of a
-// buffer have read it) and cfull (a C slab has landed) order them against the
-// storer and C-loader threads.
+// 16-bit results (EPI_STORE) leave through two 64 x 64 boxes per slab (rows
+// 0..63 and 64..127 of the tile, the slab's 64 columns) in the 128-byte
+// swizzled layout, two slab buffers alternating, written out by bulk tensor
+// stores from one thread. For a symmetric product every 64 x 64 box strictly
+// below the diagonal is stored as is and, from the epilogue threads'
+// registers, transposed into the upper triangle (coalesced 2-byte stores: the
+// 32 lanes of a warp hold 32 consecutive rows); a box on the diagonal is made
+// exactly symmetric in shared memory (each lower value written at (i, j) and
+// (j, i)) and stored once; boxes strictly above are not stored. The C input of
+// a slab is fetched into registers one slab ahead. The epilogue warps never
+// wait for one another: slab_full (all epilogue warps staged a slab) and
+// buf_free (the stores of a buffer have read it) order them against the storer.
 //
 // fp32 results (EPI_OUT, EPI_WUPDATE: the last product of a chain) go through
 // an fp32 staging tile and per-thread coalesced stores.
@@ -341,20 +323,25 @@ __device__ __forceinline__ uint32_t swz(int row, int col) {
 }
 
 // Hand an accumulator back to the leader's MMA thread once this warp's TMEM
-// reads are done.
+// reads are done (tcgen05.wait::ld has returned for all of them). The arrive is
+// relaxed: a release at cluster scope waits for the SM's outstanding memory
+// traffic (the operand TMA loads among it) and costs about a microsecond.
 __device__ __forceinline__ void release_acc(uint32_t leader_bar, int lane) {
   tc_fence_before();
   __syncwarp();
   if (lane == 0)
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(leader_bar)
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(leader_bar)
                  : "memory");
 }
 
 // One slab of a 16-bit result, one warp: TMEM -> registers -> swizzled boxes.
-// `cb` is the slab's C buffer (null without C input).
-__device__ __forceinline__ void stage_slab(const GemmParams& p, uint8_t* buf, const uint8_t* cb,
+// `cin` holds this thread's C values for the slab; `d2diag` the D2 values on
+// the diagonal of this slab buffer. Returns true when the box lies strictly
+// below the diagonal of a symmetric product: its transpose, packed in `w`,
+// still has to be written (mirror_slab, after the slab is handed over).
+__device__ __forceinline__ bool stage_slab(const GemmParams& p, uint8_t* buf, const uint4 (&cin)[NCH],
                                            uint32_t tacc, const TileCoord& tc, int slab, int q,
-                                           int sub, int lane) {
+                                           int sub, int lane, uint16_t* d2diag, uint32_t (&w)[8]) {
   const int h = q >> 1;                     // 64-row box of this warp
   const int a = (q & 1) * 32 + lane;        // row inside the box
   const int cs0 = slab * SLAB;
@@ -364,18 +351,16 @@ __device__ __forceinline__ void stage_slab(const GemmParams& p, uint8_t* buf, co
   const bool sym = p.sym != 0;
   const bool f16 = p.f16 != 0;
   uint8_t* bC = buf + h * kBoxBytes;
-  uint8_t* bT = buf + (2 + h) * kBoxBytes;
   float v[16];
   tmem_ld16(tacc + (uint32_t)(cs0 + cl), v);
   float x[16];
-  if (cb) {
-    const uint8_t* cbox = cb + h * kBoxBytes;
+  if (p.C && p.beta != 0.f) {
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
-      float cin[8];
-      unpack8(*reinterpret_cast<const uint4*>(cbox + swz(a, cl + 8 * g)), f16, cin);
+      float c8[8];
+      unpack8(cin[g], f16, c8);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[g * 8 + e] = fmaf(p.beta, cin[e], p.alpha * v[g * 8 + e]);
+      for (int e = 0; e < 8; ++e) x[g * 8 + e] = fmaf(p.beta, c8[e], p.alpha * v[g * 8 + e]);
     }
   } else {
 #pragma unroll
@@ -384,10 +369,13 @@ __device__ __forceinline__ void stage_slab(const GemmParams& p, uint8_t* buf, co
   if (rel == 0) {
 #pragma unroll
     for (int e = 0; e < 16; ++e)
-      if (cl + e == a) x[e] += p.gamma;
+      if (cl + e == a) {
+        x[e] += p.gamma;
+        if (p.has_d2) d2diag[a] = float_to_h16(x[e] + p.gamma2, f16);
+      }
   }
   if (sym && rel == 0) {
-    // diagonal box: lower values at (a, b) and (b, a); the D2 version in sT
+    // diagonal box: lower values at (a, b) and (b, a)
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       const int b = cl + e;
@@ -395,77 +383,67 @@ __device__ __forceinline__ void stage_slab(const GemmParams& p, uint8_t* buf, co
       const uint16_t hv = float_to_h16(x[e], f16);
       *reinterpret_cast<uint16_t*>(bC + swz(a, b)) = hv;
       if (b < a) *reinterpret_cast<uint16_t*>(bC + swz(b, a)) = hv;
-      if (p.has_d2) {
-        const uint16_t hv2 = b == a ? float_to_h16(x[e] + p.gamma2, f16) : hv;
-        *reinterpret_cast<uint16_t*>(bT + swz(a, b)) = hv2;
-        if (b < a) *reinterpret_cast<uint16_t*>(bT + swz(b, a)) = hv2;
-      }
     }
-  } else {
-    uint32_t w[8];
+    return false;
+  }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) w[e] = pack2(x[2 * e], x[2 * e + 1], f16);
-    *reinterpret_cast<uint4*>(bC + swz(a, cl)) = make_uint4(w[0], w[1], w[2], w[3]);
-    *reinterpret_cast<uint4*>(bC + swz(a, cl + 8)) = make_uint4(w[4], w[5], w[6], w[7]);
-    if (sym) {
-      // transposed copy for the mirror store: element (b, a) of the sT box
+  for (int e = 0; e < 8; ++e) w[e] = pack2(x[2 * e], x[2 * e + 1], f16);
+  *reinterpret_cast<uint4*>(bC + swz(a, cl)) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(bC + swz(a, cl + 8)) = make_uint4(w[4], w[5], w[6], w[7]);
+  return sym;
+}
+
+// The transposed copy of a box strictly below the diagonal: D[c][r] = value
+// (r, c) for the upper triangle, straight from registers (the 32 lanes of a
+// warp hold 32 consecutive rows, so each 2-byte store instruction is coalesced).
+__device__ __forceinline__ void mirror_slab(const GemmParams& p, const TileCoord& tc, int slab, int q,
+                                            int sub, int lane, const uint32_t (&w)[8]) {
+  const int mrow = tc.c0 + slab * SLAB + sub * CPW;       // mirror row of column cl
+  const int mcol = tc.r0 + 64 * (q >> 1) + (q & 1) * 32 + lane;   // mirror column of this row
+  if (mcol >= p.N) return;
+  const long long off = (long long)tc.bz * p.d_bs + (long long)mrow * p.ldd + mcol;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        *reinterpret_cast<uint16_t*>(bT + swz(cl + 2 * e, a)) = (uint16_t)(w[e] & 0xFFFF);
-        *reinterpret_cast<uint16_t*>(bT + swz(cl + 2 * e + 1, a)) = (uint16_t)(w[e] >> 16);
-      }
-    }
+  for (int e = 0; e < 16; ++e) {
+    if (mrow + e >= p.M) break;
+    const uint16_t hv = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
+    p.D[off + (long long)e * p.ldd] = hv;
+    if (p.has_d2) p.D2[off + (long long)e * p.ldd] = hv;
   }
 }
 
-// Stores of one staged slab (storer thread). Maps: D / D2 with 64 x 128 boxes
-// (direct), 64 x 64 x 2 boxes over (row, 64-column chunk) (mirror: both row
-// boxes of a slab at once), and 64 x 64 boxes (single).
+// Stores of one staged slab (storer thread): D (and D2) with 64 x 128 boxes
+// (both row boxes of the slab) or 64 x 64 boxes (one). D2 differs from D on the
+// diagonal only: its diagonal box is stored from the same staging and its
+// diagonal then rewritten once that copy has completed.
 struct StoreMaps {
-  const CUtensorMap *D, *Dm, *Ds, *D2, *D2m, *D2s;
+  const CUtensorMap *D, *Ds, *D2, *D2s;
 };
 __device__ __forceinline__ void store_slab(const GemmParams& p, const StoreMaps& m, uint8_t* buf,
-                                           const TileCoord& tc, int slab) {
+                                           const TileCoord& tc, int slab, const uint16_t* d2diag) {
   const int xcol = tc.c0 + slab * SLAB;
   if (xcol >= p.N || tc.r0 >= p.M) return;
-  const uint32_t sC0 = smem_u32(buf), sC1 = sC0 + kBoxBytes;
-  const uint32_t sT0 = sC0 + 2 * kBoxBytes, sT1 = sC0 + 3 * kBoxBytes;
+  const uint32_t s0 = smem_u32(buf), s1 = s0 + kBoxBytes;
   const bool d2 = p.has_d2 != 0;
-  if (!p.sym) {
-    tma_store_3d(m.D, sC0, xcol, tc.r0, tc.bz);
-    return;
-  }
   const int rel0 = tc.r0 - tc.c0 - slab * SLAB;   // box 0; box 1 is rel0 + 64
-  if (rel0 > 0) {
-    // both boxes strictly below the diagonal
-    tma_store_3d(m.D, sC0, xcol, tc.r0, tc.bz);
-    tma_store_4d(m.Dm, sT0, 0, xcol, tc.r0 / 64, tc.bz);
-    if (d2) {
-      tma_store_3d(m.D2, sC0, xcol, tc.r0, tc.bz);
-      tma_store_4d(m.D2m, sT0, 0, xcol, tc.r0 / 64, tc.bz);
-    }
-  } else if (rel0 == 0) {
-    // box 0 on the diagonal, box 1 below
-    if (!d2) {
-      tma_store_3d(m.D, sC0, xcol, tc.r0, tc.bz);
-    } else {
-      tma_store_3d(m.Ds, sC0, xcol, tc.r0, tc.bz);
-      tma_store_3d(m.D2s, sT0, xcol, tc.r0, tc.bz);
-      if (tc.r0 + 64 < p.M) {
-        tma_store_3d(m.Ds, sC1, xcol, tc.r0 + 64, tc.bz);
-        tma_store_3d(m.D2s, sC1, xcol, tc.r0 + 64, tc.bz);
-      }
-    }
-    if (tc.r0 + 64 < p.M) {
-      tma_store_3d(m.Ds, sT1, tc.r0 + 64, xcol, tc.bz);
-      if (d2) tma_store_3d(m.D2s, sT1, tc.r0 + 64, xcol, tc.bz);
-    }
-  } else if (rel0 == -64) {
+  int diag_row = -1;                              // first row of a diagonal box
+  if (!p.sym || rel0 >= 0) {
+    // both boxes on or below the diagonal
+    tma_store_3d(m.D, s0, xcol, tc.r0, tc.bz);
+    if (d2) tma_store_3d(m.D2, s0, xcol, tc.r0, tc.bz);
+    if (p.sym && rel0 == 0) diag_row = tc.r0;
+  } else if (rel0 == -64 && tc.r0 + 64 < p.M) {
     // box 0 above the diagonal, box 1 on it
-    if (tc.r0 + 64 < p.M) {
-      tma_store_3d(m.Ds, sC1, xcol, tc.r0 + 64, tc.bz);
-      if (d2) tma_store_3d(m.D2s, sT1, xcol, tc.r0 + 64, tc.bz);
-    }
+    tma_store_3d(m.Ds, s1, xcol, tc.r0 + 64, tc.bz);
+    if (d2) tma_store_3d(m.D2s, s1, xcol, tc.r0 + 64, tc.bz);
+    diag_row = tc.r0 + 64;
+  }
+  if (d2 && diag_row >= 0) {
+    bulk_commit();
+    bulk_wait_all();
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    uint16_t* dst = p.D2 + (long long)tc.bz * p.d_bs;
+    for (int i = 0; i < 64 && diag_row + i < p.M && xcol + i < p.N; ++i)
+      dst[(long long)(diag_row + i) * p.ldd + xcol + i] = d2diag[i];
   }
 }
 
@@ -478,6 +456,7 @@ __device__ __forceinline__ void c_prefetch(const GemmParams& p, const TileCoord&
   for (int u = 0; u < NCH; ++u) cpre[u] = make_uint4(0, 0, 0, 0);
   if (!p.C || p.beta == 0.f) return;
   const int c0 = tc.c0 + slab * SLAB;
+  if (p.sym && tc.r0 + 64 * (q >> 1) < c0) return;   // box strictly above the diagonal
   const int r = tc.r0 + q * 32 + lane;
   const int cl = sub * CPW;
   const long long cbs = (long long)tc.bz * p.c_bs;
@@ -502,6 +481,9 @@ __device__ __forceinline__ void epilogue_out_slab(const GemmParams& p, uint8_t* 
   const int rows_valid = min(BM, p.vm - r0);
   const int cols_valid = min(SLAB, p.vn - c0);   // may be <= 0 for a ragged tile
   const float alpha = p.alpha, beta = p.beta;
+  // natural layout: row-major 128 x 64 with 16-byte chunk c of row r at c ^ (r mod 16);
+  // transposed: column-major (64 x 128), no padding needed
+  auto fidx = [](int r, int c) { return r * SLAB + ((((c >> 2) ^ r) & 15) << 2) + (c & 3); };
 
   uint4 cnow[NCH];
 #pragma unroll
@@ -513,16 +495,22 @@ __device__ __forceinline__ void epilogue_out_slab(const GemmParams& p, uint8_t* 
     const int cl = sub * CPW;
     float v[16];
     tmem_ld16(tacc + (uint32_t)(cs0 + cl), v);
+    float val[16];
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
       float cin[8];
       unpack8(cnow[g], f16, cin);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float val = fmaf(beta, cin[e], alpha * v[g * 8 + e]);
-        if (!tr) sF[rr * FP + cl + g * 8 + e] = val;
-        else sF[(cl + g * 8 + e) * FT + rr] = val;
-      }
+      for (int e = 0; e < 8; ++e) val[g * 8 + e] = fmaf(beta, cin[e], alpha * v[g * 8 + e]);
+    }
+    if (!tr) {
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4)
+        *reinterpret_cast<float4*>(sF + fidx(rr, cl + 4 * c4)) =
+            make_float4(val[4 * c4], val[4 * c4 + 1], val[4 * c4 + 2], val[4 * c4 + 3]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) sF[(cl + e) * BM + rr] = val[e];
     }
   }
   if (last_slab) release_acc(leader_bar, lane);
@@ -545,12 +533,12 @@ __device__ __forceinline__ void epilogue_out_slab(const GemmParams& p, uint8_t* 
           const int row = idx / (SLAB / 4), col = (idx % (SLAB / 4)) * 4;
           okc[u] = row < rows_valid && col < cols_valid;
           off[u] = (long long)(r0 + row) * ld + c0 + col;
-          if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + row * FP + col);
+          if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + fidx(row, col));
         } else {
           const int col = idx >> 5, row = (idx & 31) * 4;   // slab column = natural row
           okc[u] = col < cols_valid && row < rows_valid;
           off[u] = (long long)(c0 + col) * ld + r0 + row;
-          if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + col * FT + row);
+          if (okc[u]) val[u] = *reinterpret_cast<const float4*>(sF + col * BM + row);
         }
         if (p.mode == EPI_WUPDATE && okc[u])
           wv[u] = *reinterpret_cast<const float4*>(p.W + (long long)tc.bz * p.w_bs + off[u]);
@@ -578,10 +566,9 @@ __device__ __forceinline__ void epilogue_out_slab(const GemmParams& p, uint8_t* 
 template <bool B_MN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-           const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
-           const __grid_constant__ CUtensorMap tmDm, const __grid_constant__ CUtensorMap tmDs,
-           const __grid_constant__ CUtensorMap tmD2, const __grid_constant__ CUtensorMap tmD2m,
-           const __grid_constant__ CUtensorMap tmD2s, const GemmParams p) {
+           const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmDs,
+           const __grid_constant__ CUtensorMap tmD2, const __grid_constant__ CUtensorMap tmD2s,
+           const GemmParams p) {
   // The skip flag is read by both CTAs of a pair before any cluster-level
   // operation, so they return together.
   if (p.skip && *p.skip) return;
@@ -590,17 +577,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* outbuf = base + STAGES * kStageBytes;            // [2] slab buffers
-  uint8_t* cbuf = outbuf + 2 * kOutBufBytes;                // [2] C slabs
-  uint64_t* full = reinterpret_cast<uint64_t*>(cbuf + 2 * kCBufBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(outbuf + 2 * kOutBufBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;     // [2]
   uint64_t* acc_empty = acc_full + 2;      // [2] (the leader's are used)
   uint64_t* slab_full = acc_empty + 2;     // [2]
   uint64_t* buf_free = slab_full + 2;      // [2]
-  uint64_t* cfull = buf_free + 2;          // [2]
-  uint64_t* drain = cfull + 2;
+  uint64_t* drain = buf_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   int* flags = reinterpret_cast<int*>(tmem_slot + 1);
+  uint16_t* d2diag = reinterpret_cast<uint16_t*>(flags + 4);   // [2][64]
   volatile int* abort_flag = flags;
   int* consumed = flags + 1;
   int* issued = flags + 2;
@@ -614,7 +600,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int nkb = p.K / BK;
   const int nst = cdiv(nkb, KPS);
   const bool store_mode = p.mode == EPI_STORE;
-  const bool use_c = p.C != nullptr && p.beta != 0.f;
   constexpr uint32_t kTmemCols = 2 * BN;   // two 256-column accumulators
 
   if (threadIdx.x == 0) {
@@ -627,7 +612,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&acc_empty[a]), 2 * kEpiWarps);
       mbar_init(smem_u32(&slab_full[a]), kEpiWarps);
       mbar_init(smem_u32(&buf_free[a]), 1);
-      mbar_init(smem_u32(&cfull[a]), 1);
     }
     mbar_init(smem_u32(drain), 1);
     flags[0] = 0;
@@ -639,11 +623,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     prefetch_map(&tmB);
     if (store_mode) {
       prefetch_map(&tmD);
-      if (p.sym) {
-        prefetch_map(&tmDm);
-        prefetch_map(&tmDs);
-      }
-      if (use_c) prefetch_map(&tmC);
+      if (p.sym) prefetch_map(&tmDs);
     }
   }
   if (warp == 1) {
@@ -731,33 +711,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_wait(smem_u32(drain), 0, p.err, nullptr);
     }
   } else if (warp == 3) {
-    if (lane == 0 && store_mode && use_c) {
-      // ---------------- C loader: slab g into C buffer g & 1, up to two slabs ahead
-      uint32_t g = 0;
-      bool ok = true;
-      for (int T = pid; T < total && ok; T += npairs) {
-        const TileCoord tc = decode_tile(p, T, tiles_per, (int)cr);
-        for (int slab = 0; slab < kSlabs; ++slab, ++g) {
-          const int b = (int)(g & 1u);
-          const uint32_t n = g >> 1;
-          if (n >= 1 && !mbar_wait(smem_u32(&slab_full[b]), (n - 1) & 1u, p.err, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const int xcol = tc.c0 + slab * SLAB;
-          // skip slabs outside the matrix and, for symmetric products, slabs whose
-          // two row boxes both lie strictly above the diagonal
-          const bool need = xcol < p.N && tc.r0 < p.M && !(p.sym && tc.r0 + 64 < xcol);
-          mbar_expect_tx(smem_u32(&cfull[b]), need ? kCBufBytes : 0u);
-          if (need)
-            tma_load_3d(smem_u32(cbuf + b * kCBufBytes), &tmC, smem_u32(&cfull[b]), xcol, tc.r0, tc.bz);
-        }
-      }
-    }
-  } else if (warp == 4) {
     if (lane == 0 && store_mode) {
       // ---------------- storer: bulk tensor stores of each staged slab
-      const StoreMaps maps{&tmD, &tmDm, &tmDs, &tmD2, &tmD2m, &tmD2s};
+      const StoreMaps maps{&tmD, &tmDs, &tmD2, &tmD2s};
       uint32_t g = 0;
       bool ok = true;
       for (int T = pid; T < total && ok; T += npairs) {
@@ -766,7 +722,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int b = (int)(g & 1u);
           const uint32_t n = g >> 1;
           if (!mbar_wait(smem_u32(&slab_full[b]), n & 1u, p.err, abort_flag)) { ok = false; break; }
-          store_slab(p, maps, outbuf + b * kOutBufBytes, tc, slab);
+          store_slab(p, maps, outbuf + b * kOutBufBytes, tc, slab, d2diag + b * 64);
           bulk_commit();
           bulk_wait_read_all();
           mbar_arrive(smem_u32(&buf_free[b]));
@@ -789,6 +745,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int ab = it & 1;
         const uint32_t use = (uint32_t)(it >> 1);
         const TileCoord tc = decode_tile(p, T, tiles_per, (int)cr);
+        uint4 cpre[NCH];
+        c_prefetch(p, tc, 0, q, sub, lane, cpre);   // overlaps the MMAs of this tile
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[ab]), use & 1u, p.err, abort_flag));
         if (!ok) break;
         tc_fence_after();
@@ -797,6 +755,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int slab = 0; slab < kSlabs; ++slab, ++g) {
           const int b = (int)(g & 1u);
           const uint32_t n = g >> 1;
+          uint4 cnow[NCH];
+#pragma unroll
+          for (int u = 0; u < NCH; ++u) cnow[u] = cpre[u];
           if (n >= 1) {
             ok = __all_sync(0xffffffffu,
                             mbar_wait(smem_u32(&buf_free[b]), (n - 1) & 1u, p.err, abort_flag));
@@ -804,18 +765,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           // a box strictly above the diagonal of a symmetric product is never stored
           const bool skip = p.sym && tc.r0 - tc.c0 + 64 * (q >> 1) - slab * SLAB < 0;
-          if (!skip) {
-            if (use_c) {
-              ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&cfull[b]), n & 1u, p.err, abort_flag));
-              if (!ok) break;
-            }
-            stage_slab(p, outbuf + b * kOutBufBytes, use_c ? cbuf + b * kCBufBytes : nullptr, tacc,
-                       tc, slab, q, sub, lane);
-          }
+          uint32_t w[8];
+          const bool mirror =
+              !skip && stage_slab(p, outbuf + b * kOutBufBytes, cnow, tacc, tc, slab, q, sub, lane,
+                                  d2diag + b * 64, w);
           if (slab == kSlabs - 1) release_acc(ab ? leader_empty1 : leader_empty0, lane);
           fence_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&slab_full[b]));
+          // global stores and the next slab's C loads only after the hand-over, so
+          // that neither the proxy fence nor the (releasing) arrive waits for them
+          if (mirror) mirror_slab(p, tc, slab, q, sub, lane, w);
+          if (slab + 1 < kSlabs) c_prefetch(p, tc, slab + 1, q, sub, lane, cpre);
         }
       }
     } else {
@@ -902,9 +863,9 @@ bool map_tile(CUtensorMap* m, const void* base, bool f16, int rows, int cols, in
 // The same matrix viewed as [batch][cols / 64][rows][64] (64-column chunks as a
 // dimension) with {64, box_rows, 2, 1} boxes: box_rows rows of two consecutive
 // chunks in one copy, each chunk landing as its own box_rows x 128 B block.
-// Used for K-major operands (rows x K, box_rows 128: two k-blocks), the
-// MN-major B (K rows x N, box_rows 128: two k-blocks of rows, 128 columns) and
-// mirror stores (box_rows 64). Requires cols % 64 == 0.
+// Used for K-major operands (rows x K, box_rows 128: two k-blocks) and the
+// MN-major B (K rows x N, box_rows 128: two k-blocks of rows, 128 columns).
+// Requires cols % 64 == 0.
 bool map_chunks(CUtensorMap* m, const void* base, bool f16, int rows, int cols, int ld, int batch,
                 long long bs, int box_rows) {
   const cuuint64_t dims[4] = {64, (cuuint64_t)rows, (cuuint64_t)(cols / 64), (cuuint64_t)batch};
@@ -925,7 +886,7 @@ int num_sms() {
 }
 
 struct Maps {
-  CUtensorMap A, B, C, D, Dm, Ds, D2, D2m, D2s;
+  CUtensorMap A, B, D, Ds, D2, D2s;
 };
 
 template <bool B_MN>
@@ -940,8 +901,7 @@ cudaError_t launch_gemm(const Maps& m, const GemmParams& p, cudaStream_t s) {
   const int tiles = p.sym ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
   const int total = tiles * p.batch;
   const int pairs = total < num_sms() / 2 ? total : num_sms() / 2;
-  k_gemm<B_MN><<<2 * pairs, kThreads, kSmemBytes, s>>>(m.A, m.B, m.C, m.D, m.Dm, m.Ds, m.D2, m.D2m,
-                                                        m.D2s, p);
+  k_gemm<B_MN><<<2 * pairs, kThreads, kSmemBytes, s>>>(m.A, m.B, m.D, m.Ds, m.D2, m.D2s, p);
   return cudaGetLastError();
 }
 
@@ -968,17 +928,17 @@ struct Ns {
   cudaStream_t s;
 };
 
-// Output maps of a symmetric N x N result.
-bool sym_out_maps(Maps& m, const Ns& c, uint16_t* D, uint16_t* D2) {
+// Output maps and pointers of a symmetric N x N result.
+bool sym_out(Maps& m, GemmParams& p, const Ns& c, uint16_t* D, uint16_t* D2) {
   const long long bs = (long long)c.N * c.N;
   if (!map_tile(&m.D, D, c.f16, c.N, c.N, c.N, c.B, bs, 128) ||
-      !map_chunks(&m.Dm, D, c.f16, c.N, c.N, c.N, c.B, bs, 64) ||
       !map_tile(&m.Ds, D, c.f16, c.N, c.N, c.N, c.B, bs, 64))
     return false;
   if (D2 && (!map_tile(&m.D2, D2, c.f16, c.N, c.N, c.N, c.B, bs, 128) ||
-             !map_chunks(&m.D2m, D2, c.f16, c.N, c.N, c.N, c.B, bs, 64) ||
              !map_tile(&m.D2s, D2, c.f16, c.N, c.N, c.N, c.B, bs, 64)))
     return false;
+  p.D = D; p.D2 = D2; p.d_bs = bs; p.ldd = c.N;
+  p.has_d2 = D2 ? 1 : 0;
   return true;
 }
 
@@ -989,8 +949,8 @@ cudaError_t xxt(const Ns& c, const uint16_t* X, uint16_t* D) {
   const long long xbs = (long long)c.N * c.Mp;
   if (!map_chunks(&m.A, X, c.f16, c.N, c.Mp, c.Mp, c.B, xbs, 128)) return cudaErrorInvalidValue;
   m.B = m.A;
-  if (!sym_out_maps(m, c, D, nullptr)) return cudaErrorInvalidValue;
   GemmParams p = base_params(c.N, c.N, c.Mp, c.B, c.f16, c.skip, c.err);
+  if (!sym_out(m, p, c, D, nullptr)) return cudaErrorInvalidValue;
   p.tiles_m = p.tiles_n = cdiv(c.N, 2 * BM);
   p.sym = 1;
   return launch_gemm<false>(m, p, c.s);
@@ -1006,15 +966,13 @@ cudaError_t symmul(const Ns& c, const uint16_t* S1, const uint16_t* S2, float al
   if (!map_chunks(&m.A, S1, c.f16, c.N, c.N, c.N, c.B, bs, 128) ||
       !map_chunks(&m.B, S2, c.f16, c.N, c.N, c.N, c.B, bs, 128))
     return cudaErrorInvalidValue;
-  const bool with_c = Cin && beta != 0.f;
-  if (with_c && !map_tile(&m.C, Cin, c.f16, c.N, c.N, c.N, c.B, bs, 128)) return cudaErrorInvalidValue;
-  if (!sym_out_maps(m, c, D, D2)) return cudaErrorInvalidValue;
   GemmParams p = base_params(c.N, c.N, c.N, c.B, c.f16, c.skip, c.err);
+  if (!sym_out(m, p, c, D, D2)) return cudaErrorInvalidValue;
   p.tiles_m = p.tiles_n = cdiv(c.N, 2 * BM);
   p.sym = 1;
   p.alpha = alpha; p.beta = beta; p.gamma = gamma;
-  p.C = with_c ? Cin : nullptr; p.c_bs = bs; p.ldc = c.N;
-  p.has_d2 = D2 ? 1 : 0; p.gamma2 = gamma2;
+  p.C = (Cin && beta != 0.f) ? Cin : nullptr; p.c_bs = bs; p.ldc = c.N;
+  p.gamma2 = gamma2;
   return launch_gemm<false>(m, p, c.s);
 }
 
@@ -1037,7 +995,7 @@ cudaError_t leftmul(const Ns& c, const uint16_t* S, const uint16_t* X, float alp
   if (!out) {
     p.mode = EPI_STORE;
     if (!map_tile(&m.D, D, c.f16, c.N, c.Mp, c.Mp, c.B, xbs, 128)) return cudaErrorInvalidValue;
-    if (p.C && !map_tile(&m.C, X, c.f16, c.N, c.Mp, c.Mp, c.B, xbs, 128)) return cudaErrorInvalidValue;
+    p.D = D; p.d_bs = xbs; p.ldd = c.Mp;
   } else {
     p.vm = c.vN; p.vn = c.vMp;
     p.transpose_out = c.tall ? 1 : 0;
