@@ -204,48 +204,77 @@ def run_reference(args, world, rank):
 
 GRAD_POOL = 6   # distinct gradient buffers per group, used cyclically step after step
 
+# DRAM bytes per k_gemm launch (average over one step's 45 NS products of the
+# LLaMA-130M set, standard NS), from the ncu capture summarised in
+# profiles/k_gemm_llama130m.md; reported only while gm_gemm.cu is the source
+# that capture measured.
+GEMM_TRAFFIC = {"config": 2, "ns": "standard", "bytes_per_launch": 88.12e6,
+                "source_sha256": "71ddb81c923aae0552d646128a7517d4ccfdb97ae75dac5ec043ec8a7b442da8"}
 
-def build_set(gm, w: WL.Workload, ns_mode: int, rank: int, steps_total: int, dev):
-    groups = []
-    rank_offset = rank * sum(g.count for g in w.groups)
-    for gi, g in enumerate(w.groups):
-        B, m, n = g.count, g.m, g.n
-        base = rank_offset + w.group_base(gi)
-        step = gm.GraspStep(B, m, n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=ns_mode,
-                            seed=w.seed + rank, device=dev)
-        st = gm.GraspState.zeros(B, m, n, w.k, dev)
-        W = torch.empty((B, m, n), dtype=torch.float32, device=dev)
+
+def gemm_traffic(config: int, ns: str):
+    import hashlib
+    path = os.path.join(ROOT, "bit_muon_optimizer_b200", "csrc", "gm_gemm.cu")
+    try:
+        with open(path, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    t = GEMM_TRAFFIC
+    if sha != t["source_sha256"] or config != t["config"] or ns != t["ns"]:
+        return None
+    return t["bytes_per_launch"]
+
+
+def est_bytes(w: WL.Workload, pool: int) -> int:
+    """Device bytes of the benchmark per parameter-set element: fp32 W, the
+    gradient pool, the step workspace (fp32 M, the 16-bit iterate, NS buffers),
+    and the separately timed NS / codec passes (fp32 O, their workspace, codes)."""
+    elems = sum(g.count * g.m * g.n for g in w.groups)
+    return elems * (22 + 2 * pool)
+
+
+def matrix_base(w: WL.Workload, gi: int, rank: int) -> int:
+    """Index of the first matrix of shape group gi in rank's parameter set: rank r
+    steps matrices r * count ... (r + 1) * count - 1 of the workload's sequence."""
+    return rank * sum(x.count for x in w.groups) + w.group_base(gi)
+
+
+def build_group(gm, w: WL.Workload, gi: int, ns_mode: int, rank: int, pool: int, dev):
+    g = w.groups[gi]
+    B, m, n = g.count, g.m, g.n
+    base = matrix_base(w, gi, rank)
+    step = gm.GraspStep(B, m, n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=ns_mode,
+                        seed=w.seed + rank, device=dev)
+    st = gm.GraspState.zeros(B, m, n, w.k, dev)
+    W = torch.empty((B, m, n), dtype=torch.float32, device=dev)
+    for b in range(B):
+        W[b] = WL.initial_weight(w, base + b, m, n, device=dev)
+    grads = []
+    for t in range(1, pool + 1):
+        G = torch.empty((B, m, n), dtype=w.gdtype, device=dev)
         for b in range(B):
-            W[b] = WL.initial_weight(w, base + b, m, n, device=dev)
-        grads = []
-        for t in range(1, min(steps_total, GRAD_POOL) + 1):
-            G = torch.empty((B, m, n), dtype=w.gdtype, device=dev)
-            for b in range(B):
-                WL.gradient(w, base + b, t, m, n, device=dev, out=G[b])
-            grads.append(G)
-        groups.append(dict(step=step, st=st, W=W, grads=grads, B=B, m=m, n=n))
-    return groups
+            WL.gradient(w, base + b, t, m, n, device=dev, out=G[b])
+        grads.append(G)
+    return dict(step=step, st=st, W=W, grads=grads, B=B, m=m, n=n)
 
 
-def run_ours(args, world, rank, local):
-    from bit_muon_optimizer_b200 import gmuon as gm
-    dev = torch.device("cuda", local)
-    w = WL.WORKLOADS[args.config]
-    ns_mode = gm.GM_NS_GRAM if args.ns == "gram" else gm.GM_NS_STANDARD
-    hbm, bf16, bf16_sus, peak_kind = _peaks()
-    total = args.warmup + args.steps
-    groups = build_set(gm, w, ns_mode, rank, total, dev)
+def measure(gm, w, groups, ns_mode, args, world, local, do_e2e):
+    """Times args.steps graph-replayed GRASP steps over `groups` (each group on
+    its own stream), then the NS chains and the codec passes alone, then (if
+    asked) steps end to end through pinned host buffers."""
+    dev = groups[0]["W"].device
     streams = [torch.cuda.Stream(device=dev) for _ in groups]
     main = torch.cuda.Stream(device=dev)        # graphs are captured on a side stream
 
-    def one_step(t):
+    def fork(enqueue):
         ev = torch.cuda.Event()
         ev.record(main)
         done = []
         for g, s in zip(groups, streams):
             s.wait_event(ev)
             with torch.cuda.stream(s):
-                g["step"](g["st"], g["W"], g["grads"][t])
+                enqueue(g)
             e = torch.cuda.Event()
             e.record(s)
             done.append(e)
@@ -255,13 +284,13 @@ def run_ours(args, world, rank, local):
     # eager warm-up (also sets kernel attributes), then one graph per gradient slot
     main.wait_stream(torch.cuda.current_stream(dev))
     npool = len(groups[0]["grads"])
-    one_step(0)
+    fork(lambda g: g["step"](g["st"], g["W"], g["grads"][0]))
     torch.cuda.synchronize()
     graphs = []
     for t in range(npool):
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=main):
-            one_step(t)
+            fork(lambda g, t=t: g["step"](g["st"], g["W"], g["grads"][t]))
         graphs.append(gr)
     torch.cuda.synchronize()
     with torch.cuda.stream(main):
@@ -282,34 +311,20 @@ def run_ours(args, world, rank, local):
             end.record(main)
         torch.cuda.synchronize()
         barrier(world)
-    ms_step = start.elapsed_time(end) / args.steps
-    ms_step = max_over_ranks(ms_step, world)
-    clocks = clk.summary()
+    ms_step = max_over_ranks(start.elapsed_time(end) / args.steps, world)
     status = [int(g["st"].dev_status.item()) for g in groups]
     if any(status):
         raise RuntimeError(f"device status {status}")
+    del graphs
 
     # ---- NS chain alone (tensor-core roofline) and codec passes alone (HBM), each
-    # replayed from a graph with the three groups on their own streams, as in the step
+    # replayed from a graph with the groups on their own streams, as in the step
     def graph_ms(enqueue, reps):
-        def fork():
-            ev = torch.cuda.Event()
-            ev.record(main)
-            done = []
-            for g, s in zip(groups, streams):
-                s.wait_event(ev)
-                with torch.cuda.stream(s):
-                    enqueue(g)
-                e = torch.cuda.Event()
-                e.record(s)
-                done.append(e)
-            for e in done:
-                main.wait_event(e)
-        fork()                                   # eager once (attributes, workspaces)
+        fork(enqueue)                            # eager once (attributes, workspaces)
         torch.cuda.synchronize()
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=main):
-            fork()
+            fork(enqueue)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(main):       # replay on the stream the events are recorded on
             for _ in range(3):
@@ -320,12 +335,12 @@ def run_ours(args, world, rank, local):
                 gr.replay()
             s1.record(main)
         torch.cuda.synchronize()
+        del gr
         return s0.elapsed_time(s1) / reps
 
     for g in groups:
-        g["Mx"] = g["step"].stage_M().clone()
-        g["Mout"] = torch.empty_like(g["Mx"])
-        g["O"] = torch.empty_like(g["Mx"])
+        g["Mx"] = g["step"].stage_M()            # the last step's fp32 M_t, read-only below
+        g["O"] = torch.empty_like(g["Mx"])       # NS output, then the codec's rebuilt M
         g["ws_ns"] = torch.empty(gm.workspace_bytes(gm.GM_OP_GRAM_NS if ns_mode == gm.GM_NS_GRAM
                                                     else gm.GM_OP_NEWTON_SCHULZ, g["B"], g["m"], g["n"]),
                                  dtype=torch.uint8, device=dev)
@@ -341,21 +356,22 @@ def run_ours(args, world, rank, local):
     def codec_enqueue(g):
         st = g["st"]
         gm.dequant_rebuild(st.codes4, st.rscale, st.cscale, st.P8, st.Pscale, st.R8, st.Rscale,
-                           out=g["Mout"])
+                           out=g["O"])
         gm.grid_quant4(g["Mx"], g["step"].stage_P(), g["step"].stage_R(), out=g["codes"])
 
-    ns_ms = graph_ms(ns_enqueue, 20)
+    reps = 20 if sum(g["B"] * g["m"] * g["n"] for g in groups) < 5e8 else 5
+    ns_ms = graph_ms(ns_enqueue, reps)
     ns_flops = sum(gm.ns_flops(ns_mode, g["m"], g["n"], w.T)[0] * g["B"] for g in groups)
-    ns_tflops = ns_flops / (ns_ms * 1e-3) / 1e12
-    cod_ms = graph_ms(codec_enqueue, 20)
+    cod_ms = graph_ms(codec_enqueue, reps)
     # algorithmic bytes: rebuild reads codes + scales and writes fp32 M; quant reads fp32 M
     # and writes codes + scales (the k (m + n) factor bytes are ignored)
     cod_bytes = sum(2 * g["B"] * g["m"] * g["n"] * (4 + 0.5 + 0.0625) for g in groups)
-    codec_gbs = cod_bytes / (cod_ms * 1e-3) / 1e9
+    for g in groups:
+        del g["Mx"], g["O"], g["ws_ns"], g["codes"]
 
     # ---- end to end through host buffers: H2D W and G, the step, D2H W
     e2e = None
-    if not args.no_e2e:
+    if do_e2e:
         host = []
         for g in groups:
             host.append(dict(W=g["W"].cpu().pin_memory(), G=g["grads"][-1].cpu().pin_memory()))
@@ -377,21 +393,69 @@ def run_ours(args, world, rank, local):
         s1.record()
         torch.cuda.synchronize()
         barrier(world)
-        e_ms = max_over_ranks(s0.elapsed_time(s1) / e_steps, world)
+        e2e = (max_over_ranks(s0.elapsed_time(s1) / e_steps, world), h2d, d2h)
+    return dict(ms_step=ms_step, clocks=clk.summary(), ns_ms=ns_ms, ns_flops=ns_flops,
+                cod_ms=cod_ms, cod_bytes=cod_bytes, e2e=e2e)
+
+
+def run_ours(args, world, rank, local):
+    from bit_muon_optimizer_b200 import gmuon as gm
+    dev = torch.device("cuda", local)
+    w = WL.WORKLOADS[args.config]
+    ns_mode = gm.GM_NS_GRAM if args.ns == "gram" else gm.GM_NS_STANDARD
+    hbm, bf16, bf16_sus, peak_kind = _peaks()
+    total_mem = torch.cuda.get_device_properties(dev).total_memory
+    pool = min(GRAD_POOL, args.warmup + args.steps)
+    if est_bytes(w, pool) > 0.7 * total_mem:
+        pool = 2
+    # a set too large to hold at once is measured one shape group at a time; the
+    # groups are independent and each fills the GPU, so the set's time is the sum
+    per_group = est_bytes(w, pool) > 0.7 * total_mem
+    batches = [[gi] for gi in range(len(w.groups))] if per_group else [list(range(len(w.groups)))]
+    do_e2e = not args.no_e2e and not per_group
+    res = []
+    for gis in batches:
+        groups = [build_group(gm, w, gi, ns_mode, rank, pool, dev) for gi in gis]
+        res.append(measure(gm, w, groups, ns_mode, args, world, local, do_e2e))
+        del groups
+        torch.cuda.empty_cache()
+    ms_step = sum(r["ms_step"] for r in res)
+    ns_ms = sum(r["ns_ms"] for r in res)
+    ns_flops = sum(r["ns_flops"] for r in res)
+    cod_ms = sum(r["cod_ms"] for r in res)
+    cod_bytes = sum(r["cod_bytes"] for r in res)
+    ns_tflops = ns_flops / (ns_ms * 1e-3) / 1e12
+    codec_gbs = cod_bytes / (cod_ms * 1e-3) / 1e9
+    clk = [r["clocks"] for r in res if r["clocks"]]
+    clocks = None
+    if clk:
+        clocks = {"sm_mhz": statistics.median([c["sm_mhz"] for c in clk]),
+                  "sm_max_mhz": clk[0]["sm_max_mhz"],
+                  "reasons": sorted(set(x for c in clk for x in c["reasons"])),
+                  "samples": sum(c["samples"] for c in clk)}
+    e2e = None
+    if res[0]["e2e"] is not None:
+        e_ms, h2d, d2h = res[0]["e2e"]
         e2e = {"value": e_ms / world, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h)}
 
-    # ---- kernel count inside the timed region
-    per_call = 11 + gm.ns_flops(ns_mode, 768, 768, w.T)[1]   # 11 codec kernels + NS products
-    launches = per_call * len(groups) * args.steps
+    # ---- our kernels launched per step: per group 10 codec kernels (column norms,
+    # warm start, rebuild + projection, three orthonormalisation kernels, back
+    # projection, its finalisation, 4-bit and 8-bit quantisation), the NS
+    # products, and the zero-padding copy when a dimension is not a multiple of 64
+    launches = 0
+    for g in w.groups:
+        pad = int(min(g.m, g.n) % 64 != 0 or max(g.m, g.n) % 64 != 0)
+        launches += 10 + gm.ns_flops(ns_mode, g.m, g.n, w.T)[1] + pad
+    launches *= args.steps
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         ms_cpu, sample, cores = oracle_sample_seconds(w, args.ns, 20.0)
         cpu = {"value": ms_cpu, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
 
-    elements = sum(g["B"] * g["m"] * g["n"] for g in groups)
-    step_flops = sum(gm.ns_flops(ns_mode, g["m"], g["n"], w.T)[0] * g["B"] for g in groups)
+    elements = sum(g.count * g.m * g.n for g in w.groups)
+    step_flops = sum(gm.ns_flops(ns_mode, g.m, g.n, w.T)[0] * g.count for g in w.groups)
     step_bytes = elements * FL.step_bytes_per_element(2 if w.gdtype != torch.float32 else 4)
     t_roof = max(step_flops / (bf16 * 1e12), step_bytes / (hbm * 1e9)) * 1e3
     if rank == 0:
@@ -402,15 +466,17 @@ def run_ours(args, world, rank, local):
             "dtype": "bf16" if ns_mode == gm.GM_NS_STANDARD else "f16",
             "data": "synthetic",
             "config": {"workload": w.name, "ns": args.ns, "k": w.k,
-                       "shapes": [[g["m"], g["n"], g["B"]] for g in groups],
+                       "shapes": [[g.m, g.n, g.count] for g in w.groups],
                        "elements": elements, "grad_dtype": str(w.gdtype).replace("torch.", ""),
                        "l2": "per-step working set (G, W, state, fp32 M) > L2; no flush",
                        "parallelism": f"weak x{world}, one parameter set per rank",
-                       "graph": "one CUDA graph per gradient slot, 3 streams",
-                       "grad_pool": GRAD_POOL},
+                       "graph": ("one CUDA graph per gradient slot, one stream per shape group"
+                                 + ("; shape groups measured one at a time (device memory), "
+                                    "set time = sum" if per_group else "")),
+                       "grad_pool": pool},
             "roofline": {"bound": "tensor", "achieved": ns_tflops, "peak": bf16, "unit": "TFLOP/s",
-                         "frac": ns_tflops / bf16, "traffic": None,
-                         "kernel": "NS chain (k_gemm tcgen05 products) of all groups, graph-replayed alone",
+                         "frac": ns_tflops / bf16, "traffic": gemm_traffic(args.config, args.ns),
+                         "kernel": "k_gemm: the NS chains' tcgen05 products of all groups, graph-replayed alone",
                          "peak_kind": f"{peak_kind} bf16 dense burst"},
             "ns": {"tflops": ns_tflops, "ms": ns_ms, "flops": ns_flops},
             "codec": {"gbs": codec_gbs, "peak_gbs": hbm, "frac": codec_gbs / hbm,
@@ -423,8 +489,6 @@ def run_ours(args, world, rank, local):
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    # graphs hold no NCCL work; release them before the process group goes
-    del graphs
 
 
 def main():
