@@ -179,7 +179,8 @@ __device__ __forceinline__ void reduce_scatter16(float (&v)[16], int tx) {
 
 enum RebuildSrc { SRC_STATE = 0, SRC_DENSE = 1, SRC_ZERO = 2 };
 
-template <int SRC, bool G32>
+// KP: the factor width k rounded up to 8, 16 or 32 (columns beyond k are zero).
+template <int SRC, bool G32, int KP>
 __global__ void __launch_bounds__(kThreads, 2) k_rebuild_proj(
     int m, int n, int k, const uint8_t* __restrict__ codes4, const float* __restrict__ rscale,
     const float* __restrict__ cscale, const int8_t* __restrict__ P8,
@@ -192,12 +193,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_rebuild_proj(
   const int mb = cdiv(m, kGrid);
   const int r0 = bh * kRB, c0 = bj * kGrid, bi = r0 / kGrid;
   const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
-  const int kk = SRC == SRC_STATE ? k : 0;
-  const int kq = Q ? ((k + 3) & ~3) : 0;
+  constexpr int KK = SRC == SRC_STATE ? KP : 0;
   extern __shared__ __align__(16) float sm[];
-  float* Ps = sm;                  // [kk][64]
-  float* Rs = Ps + kk * kRB;       // [kk][128]
-  float* Qs = Rs + kk * kGrid;     // [kq][128]
+  float* Ps = sm;                  // [KK][64]
+  float* Rs = Ps + KK * kRB;       // [KK][128]
+  float* Qs = Rs + KK * kGrid;     // [KP][128] (with Q)
   __shared__ float deq4[16];
   __shared__ double red[kThreads / 32];
   const long long mn = (long long)m * n;
@@ -242,18 +242,23 @@ __global__ void __launch_bounds__(kThreads, 2) k_rebuild_proj(
   // 2. factors of the tile into shared memory
   if (t < 16) deq4[t] = __fdiv_rn((float)((t & 8) ? t - 16 : t), 7.0f);
   if constexpr (SRC == SRC_STATE) {
-    for (int e = t; e < kRB * kk; e += kThreads) {
-      const int rr = e / kk, l = e % kk, gi = r0 + rr;
-      Ps[l * kRB + rr] = (gi < m) ? deq8(P8[((long long)b * m + gi) * kk + l], Pscale[b * kk + l]) : 0.f;
+#pragma unroll 4
+    for (int e = t; e < kRB * KK; e += kThreads) {
+      const int rr = e / KK, l = e % KK, gi = r0 + rr;
+      Ps[l * kRB + rr] = (gi < m && l < k) ? deq8(P8[((long long)b * m + gi) * k + l], Pscale[b * k + l]) : 0.f;
     }
-    for (int e = t; e < kGrid * kk; e += kThreads) {
-      const int cc = e / kk, l = e % kk, gj = c0 + cc;
-      Rs[l * kGrid + cc] = (gj < n) ? deq8(R8[((long long)b * n + gj) * kk + l], Rscale[b * kk + l]) : 0.f;
+#pragma unroll 4
+    for (int e = t; e < kGrid * KK; e += kThreads) {
+      const int cc = e / KK, l = e % KK, gj = c0 + cc;
+      Rs[l * kGrid + cc] = (gj < n && l < k) ? deq8(R8[((long long)b * n + gj) * k + l], Rscale[b * k + l]) : 0.f;
     }
   }
-  for (int e = t; e < kGrid * kq; e += kThreads) {
-    const int cc = e / kq, l = e % kq, gj = c0 + cc;
-    Qs[l * kGrid + cc] = (gj < n && l < k) ? Q[((long long)b * n + gj) * k + l] : 0.f;
+  if (Q) {
+#pragma unroll 4
+    for (int e = t; e < kGrid * KP; e += kThreads) {
+      const int cc = e / KP, l = e % KP, gj = c0 + cc;
+      Qs[l * kGrid + cc] = (gj < n && l < k) ? Q[((long long)b * n + gj) * k + l] : 0.f;
+    }
   }
   __syncthreads();
 
@@ -263,7 +268,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_rebuild_proj(
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  for (int l = 0; l < kk; ++l) {
+#pragma unroll 4
+  for (int l = 0; l < KK; ++l) {
     const float4 ra = *reinterpret_cast<const float4*>(Rs + l * kGrid + 4 * tx);
     const float4 rb = *reinterpret_cast<const float4*>(Rs + l * kGrid + 64 + 4 * tx);
     const float rv[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
@@ -324,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_rebuild_proj(
 
   // 5. projection partials: this tile's share of M Q, four columns of Q at a time
   if (Q) {
-    for (int l0 = 0; l0 < kq; l0 += 4) {
+    for (int l0 = 0; l0 < KP; l0 += 4) {
       float v[16];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -410,13 +416,36 @@ __global__ void __launch_bounds__(32) k_orth_chol(int k, int rsplit, const doubl
   __shared__ double L[kMaxK][kMaxK + 1];
   __shared__ double Li[kMaxK][kMaxK + 1];
   __shared__ int live[kMaxK];
-  for (int e = lane; e < k * k; e += 32) {
-    double s = 0.0;
-    for (int p = 0; p < rsplit; ++p) s += gram_part[((long long)b * rsplit + p) * k * k + e];
-    G[e / k][e % k] = s;
-    L[e / k][e % k] = 0.0;
-    Li[e / k][e % k] = 0.0;
+  {
+    // element e = lane + 32 u of the k x k Gram, summed over the row splits in order;
+    // the loads of all u are independent and issued together
+    constexpr int U = kMaxK * kMaxK / 32;
+    double acc[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) acc[u] = 0.0;
+    const double* gp = gram_part + (long long)b * rsplit * k * k;
+    for (int p = 0; p < rsplit; ++p) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int e = lane + 32 * u;
+        if (e < k * k) acc[u] += gp[(long long)p * k * k + e];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int e = lane + 32 * u;
+      if (e < k * k) {
+        G[e / k][e % k] = acc[u];
+        L[e / k][e % k] = 0.0;
+        Li[e / k][e % k] = 0.0;
+      }
+    }
   }
+  // |M_t|^2 from the rebuild's partials: lane-strided sums, then a fixed shuffle tree
+  double ns2 = 0.0;
+  for (int p = lane; p < ntiles; p += 32) ns2 += norm2_part[(long long)b * ntiles + p];
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ns2 += __shfl_xor_sync(0xffffffffu, ns2, off);
   __syncwarp();
   double maxn2 = 0.0;
   for (int l = 0; l < k; ++l) maxn2 = fmax(maxn2, G[l][l]);
@@ -454,11 +483,7 @@ __global__ void __launch_bounds__(32) k_orth_chol(int k, int rsplit, const doubl
     const int a = e / k, c = e % k;
     Tmat[(long long)b * k * k + e] = Li[c][a];   // T = L^-T
   }
-  if (lane == 0 && scale) {
-    double s = 0.0;
-    for (int p = 0; p < ntiles; ++p) s += norm2_part[(long long)b * ntiles + p];
-    scale[b] = (float)(1.0 / (sqrt(s) + (double)eps));
-  }
+  if (lane == 0 && scale) scale[b] = (float)(1.0 / (sqrt(ns2) + (double)eps));
 }
 
 // (c) P = P~ T (fp64), stored fp32.
@@ -723,7 +748,11 @@ __global__ void __launch_bounds__(512, 2) k_residual_quant4(
 }
 
 // ------------------------------------------------------------------ S6
-// blockIdx.x selects the matrix (0: X0 with rows0 rows, 1: X1), blockIdx.y the batch.
+// blockIdx.x selects the matrix (0: X0 with rows0 rows, 1: X1), blockIdx.y the batch,
+// blockIdx.z a share of the rows. Every block reduces the column absmax over all
+// rows (the factors are small and L2-resident), then quantizes its share; thread
+// t owns column t % k of rows t / k, t / k + 256 / k, ... (no division per element).
+constexpr int kQuant8Split = 8;
 __global__ void __launch_bounds__(kThreads) k_quant8(int rows0, int rows1, int k,
                                                       const float* __restrict__ X0,
                                                       int8_t* __restrict__ c0, float* __restrict__ s0,
@@ -731,7 +760,7 @@ __global__ void __launch_bounds__(kThreads) k_quant8(int rows0, int rows1, int k
                                                       int8_t* __restrict__ c1, float* __restrict__ s1,
                                                       int64_t* step, const int32_t* skip) {
   if (skip && *skip) return;
-  const int which = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  const int which = blockIdx.x, b = blockIdx.y, z = blockIdx.z, t = threadIdx.x;
   const int rows = which ? rows1 : rows0;
   const float* X = (which ? X1 : X0) + (long long)b * rows * k;
   int8_t* C = (which ? c1 : c0) + (long long)b * rows * k;
@@ -739,31 +768,35 @@ __global__ void __launch_bounds__(kThreads) k_quant8(int rows0, int rows1, int k
   __shared__ float red[kThreads];
   __shared__ float sc[kMaxK];
   const int groups = kThreads / k;
+  const int l = t % k, g = t / k;
+  const bool active = t < groups * k;
   float mx = 0.f;
-  if (t < groups * k) {
-    const int l = t % k, g = t / k;
+  if (active)
     for (int i = g; i < rows; i += groups) mx = fmaxf(mx, fabsf(X[(long long)i * k + l]));
-  }
   red[t] = mx;
   __syncthreads();
   if (t < k) {
     float v = 0.f;
-    for (int g = 0; g < groups; ++g) v = fmaxf(v, red[g * k + t]);
+    for (int gg = 0; gg < groups; ++gg) v = fmaxf(v, red[gg * k + t]);
     sc[t] = v;
-    S[t] = v;
+    if (z == 0) S[t] = v;
   }
   __syncthreads();
-  for (long long e = t; e < (long long)rows * k; e += kThreads) {
-    const int l = (int)(e % k);
+  const int per = cdiv(rows, kQuant8Split);
+  const int i0 = z * per, i1 = min(rows, i0 + per);
+  if (active) {
     const float s = sc[l];
-    int q = 0;
-    if (s > 0.f) {
-      q = (int)rintf(__fmul_rn(__fdiv_rn(X[e], s), 127.0f));
-      q = max(-127, min(127, q));
+    for (int i = i0 + g; i < i1; i += groups) {
+      const long long e = (long long)i * k + l;
+      int q = 0;
+      if (s > 0.f) {
+        q = (int)rintf(__fmul_rn(__fdiv_rn(X[e], s), 127.0f));
+        q = max(-127, min(127, q));
+      }
+      C[e] = (int8_t)q;
     }
-    C[e] = (int8_t)q;
   }
-  if (step && which == 0 && b == 0 && t == 0) *step += 1;
+  if (step && which == 0 && b == 0 && z == 0 && t == 0) *step += 1;
 }
 
 // ------------------------------------------------------------- NS input prep
@@ -877,7 +910,7 @@ cudaError_t launch_warm_start(int B, int n, int k, const int8_t* R8, const float
   return cudaGetLastError();
 }
 
-template <int SRC, bool G32>
+template <int SRC, bool G32, int KP>
 cudaError_t launch_rebuild_t(dim3 grid, size_t smem, cudaStream_t s, int m, int n, int k,
                              const uint8_t* codes4, const float* rscale, const float* cscale,
                              const int8_t* P8, const float* Pscale, const int8_t* R8,
@@ -886,13 +919,13 @@ cudaError_t launch_rebuild_t(dim3 grid, size_t smem, cudaStream_t s, int m, int 
                              int32_t* status) {
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_rebuild_proj<SRC, G32>,
+    cudaError_t e = cudaFuncSetAttribute(k_rebuild_proj<SRC, G32, KP>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)((2 * kMaxK * kGrid + kMaxK * kRB) * sizeof(float)));
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  k_rebuild_proj<SRC, G32><<<grid, kThreads, smem, s>>>(m, n, k, codes4, rscale, cscale, P8, Pscale,
+  k_rebuild_proj<SRC, G32, KP><<<grid, kThreads, smem, s>>>(m, n, k, codes4, rscale, cscale, P8, Pscale,
                                                         R8, Rscale, Mprev32, mu, G, gdt, Q, M,
                                                         norm2_part, Ppart, status);
   return cudaGetLastError();
@@ -904,16 +937,19 @@ cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4, co
                            const void* G, int gdt, const float* Q, float* M, double* norm2_part,
                            float* Ppart, int32_t* status, cudaStream_t s) {
   dim3 grid(cdiv(n, kGrid), cdiv(m, kRB), B);
-  const int kk = codes4 ? k : 0;
-  const int kq = Q ? ((k + 3) & ~3) : 0;
+  const int kp = k <= 8 ? 8 : (k <= 16 ? 16 : 32);
+  const int kk = codes4 ? kp : 0;
+  const int kq = Q ? kp : 0;
   const size_t smem = (size_t)(kk * kRB + kk * kGrid + kq * kGrid) * sizeof(float);
   const bool g32 = (G == nullptr) || gdt == GM_F32;
   const int src = codes4 ? SRC_STATE : (Mprev32 ? SRC_DENSE : SRC_ZERO);
-#define GM_RB(S, W) launch_rebuild_t<S, W>(grid, smem, s, m, n, k, codes4, rscale, cscale, P8, Pscale, \
-                                           R8, Rscale, Mprev32, mu, G, gdt, Q, M, norm2_part, Ppart, status)
-  if (src == SRC_STATE) return g32 ? GM_RB(SRC_STATE, true) : GM_RB(SRC_STATE, false);
-  if (src == SRC_DENSE) return g32 ? GM_RB(SRC_DENSE, true) : GM_RB(SRC_DENSE, false);
-  return g32 ? GM_RB(SRC_ZERO, true) : GM_RB(SRC_ZERO, false);
+#define GM_RB(S, W, K) launch_rebuild_t<S, W, K>(grid, smem, s, m, n, k, codes4, rscale, cscale, P8, Pscale, \
+                                                 R8, Rscale, Mprev32, mu, G, gdt, Q, M, norm2_part, Ppart, status)
+#define GM_RBK(S, W) (kp == 8 ? GM_RB(S, W, 8) : (kp == 16 ? GM_RB(S, W, 16) : GM_RB(S, W, 32)))
+  if (src == SRC_STATE) return g32 ? GM_RBK(SRC_STATE, true) : GM_RBK(SRC_STATE, false);
+  if (src == SRC_DENSE) return g32 ? GM_RBK(SRC_DENSE, true) : GM_RBK(SRC_DENSE, false);
+  return g32 ? GM_RBK(SRC_ZERO, true) : GM_RBK(SRC_ZERO, false);
+#undef GM_RBK
 #undef GM_RB
 }
 
@@ -959,7 +995,7 @@ cudaError_t launch_residual_quant4(int B, int m, int n, int k, const float* X, c
 cudaError_t launch_quant8(int B, int rows0, int rows1, int k, const float* X0, int8_t* c0,
                           float* s0, const float* X1, int8_t* c1, float* s1, int64_t* step,
                           const int32_t* skip, cudaStream_t s) {
-  dim3 grid(X1 ? 2 : 1, B);
+  dim3 grid(X1 ? 2 : 1, B, kQuant8Split);
   k_quant8<<<grid, kThreads, 0, s>>>(rows0, rows1, k, X0, c0, s0, X1, c1, s1, step, skip);
   return cudaGetLastError();
 }
