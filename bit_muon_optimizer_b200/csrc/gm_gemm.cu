@@ -638,6 +638,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();   // barriers of both CTAs initialised before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Products of a chain are launched as programmatic dependents: a CTA of the
+  // next product may start (and run the prologue above) on an SM this launch
+  // has left once every CTA here has finished its work; no thread touches
+  // global memory before the previous product has completed and its writes are
+  // visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // Role dispatch by warp; within a role warp only the lanes named below work,
   // the others go straight to the final barrier.
@@ -798,6 +804,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
   }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   if (warp == 0 && lane == 0 && leader) {
@@ -901,8 +908,17 @@ cudaError_t launch_gemm(const Maps& m, const GemmParams& p, cudaStream_t s) {
   const int tiles = p.sym ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
   const int total = tiles * p.batch;
   const int pairs = total < num_sms() / 2 ? total : num_sms() / 2;
-  k_gemm<B_MN><<<2 * pairs, kThreads, kSmemBytes, s>>>(m.A, m.B, m.D, m.Ds, m.D2, m.D2s, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_gemm<B_MN>, m.A, m.B, m.D, m.Ds, m.D2, m.D2s, p);
 }
 
 GemmParams base_params(int M, int N, int K, int batch, bool f16, const int32_t* skip, int32_t* err) {
