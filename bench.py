@@ -363,6 +363,28 @@ def measure(gm, w, groups, ns_mode, args, world, local, do_e2e):
     ns_ms = graph_ms(ns_enqueue, reps)
     ns_flops = sum(gm.ns_flops(ns_mode, g["m"], g["n"], w.T)[0] * g["B"] for g in groups)
     cod_ms = graph_ms(codec_enqueue, reps)
+
+    # comparator: the same standard NS chain written with torch.matmul (cuBLAS,
+    # bf16, no symmetry), on the same normalised wide-form inputs
+    abc = [(3.4445, -4.7750, 2.0315)] * w.T
+    for g in groups:
+        g["Xc"] = g["step"].stage_X().to(torch.bfloat16).clone()
+        g["Xw"] = torch.empty_like(g["Xc"])
+
+    def cublas_enqueue(g):
+        X = g["Xc"]
+        for a, b_, c in abc:
+            A = torch.matmul(X, X.mT)
+            B = torch.baddbmm(A, A, A, beta=b_, alpha=c)
+            X = torch.baddbmm(X, B, X, beta=a, alpha=1.0)
+        g["Xw"].copy_(X)
+
+    cub_ms = graph_ms(cublas_enqueue, reps)
+    cub_flops_dense = sum(T_ * g["B"] * (2.0 * min(g["m"], g["n"]) ** 2 * max(g["m"], g["n"]) * 2
+                                         + 2.0 * min(g["m"], g["n"]) ** 3)
+                          for g in groups for T_ in [w.T])
+    for g in groups:
+        del g["Xc"], g["Xw"]
     # algorithmic bytes: rebuild reads codes + scales and writes fp32 M; quant reads fp32 M
     # and writes codes + scales (the k (m + n) factor bytes are ignored)
     cod_bytes = sum(2 * g["B"] * g["m"] * g["n"] * (4 + 0.5 + 0.0625) for g in groups)
@@ -395,7 +417,8 @@ def measure(gm, w, groups, ns_mode, args, world, local, do_e2e):
         barrier(world)
         e2e = (max_over_ranks(s0.elapsed_time(s1) / e_steps, world), h2d, d2h)
     return dict(ms_step=ms_step, clocks=clk.summary(), ns_ms=ns_ms, ns_flops=ns_flops,
-                cod_ms=cod_ms, cod_bytes=cod_bytes, e2e=e2e)
+                cod_ms=cod_ms, cod_bytes=cod_bytes, e2e=e2e, cub_ms=cub_ms,
+                cub_flops_dense=cub_flops_dense)
 
 
 def run_ours(args, world, rank, local):
@@ -424,6 +447,8 @@ def run_ours(args, world, rank, local):
     ns_flops = sum(r["ns_flops"] for r in res)
     cod_ms = sum(r["cod_ms"] for r in res)
     cod_bytes = sum(r["cod_bytes"] for r in res)
+    cub_ms = sum(r["cub_ms"] for r in res)
+    cub_dense = sum(r["cub_flops_dense"] for r in res)
     ns_tflops = ns_flops / (ns_ms * 1e-3) / 1e12
     codec_gbs = cod_bytes / (cod_ms * 1e-3) / 1e9
     clk = [r["clocks"] for r in res if r["clocks"]]
@@ -479,6 +504,11 @@ def run_ours(args, world, rank, local):
                          "kernel": "k_gemm: the NS chains' tcgen05 products of all groups, graph-replayed alone",
                          "peak_kind": f"{peak_kind} bf16 dense burst"},
             "ns": {"tflops": ns_tflops, "ms": ns_ms, "flops": ns_flops},
+            "cublas_ns": {"ms": cub_ms, "tflops_algorithmic": ns_flops / (cub_ms * 1e-3) / 1e12
+                          if args.ns == "standard" else None,
+                          "tflops_dense": cub_dense / (cub_ms * 1e-3) / 1e12,
+                          "what": "standard NS, T steps of torch.matmul / baddbmm (cuBLAS bf16, "
+                                  "dense products), same inputs and streams"},
             "codec": {"gbs": codec_gbs, "peak_gbs": hbm, "frac": codec_gbs / hbm,
                       "ms": cod_ms, "kernels": "k_rebuild + k_residual_quant4"},
             "step_roofline": {"ms": t_roof, "frac": t_roof / ms_step, "flops": step_flops,

@@ -1,0 +1,106 @@
+"""Parity at full parameter-set sizes, in the benchmark's launch configuration.
+
+A whole shape group (every same-shape matrix of the parameter set, batched in
+one gm_grasp_step call as the benchmark launches it) runs two steps from a
+zero state. For the first and the last matrix of the batch, step 2 is checked
+teacher-forced against the oracle: the rebuilt momentum M_t, the power
+iteration's P and R (relative Frobenius error <= 1e-5), the 8-bit codes
+(bit-exact on the GPU's own P, R) and the 4-bit grid codes (one step apart in
+at most 1e-4 of the elements).
+
+The fp64 oracle's Newton-Schulz is too slow at these sizes, so the update
+direction O = (W_before - W_after) / eta (weight decay 0) is checked through
+the property Proposition 1 of "优化器 (3)（Gram Newton-Schulz）" states for any
+size: NS(X) = U f(S) V^T for X = U S V^T, f the composed scalar quintic. So
+the sorted singular values of O equal the sorted f(s_i) of the normalised
+momentum, up to the bf16 arithmetic's spectral-norm error (Weyl: sorted
+singular values move by at most ||E||_2).
+"""
+
+import pytest
+import torch
+
+import oracle as O
+from bit_muon_optimizer_b200 import workloads as WL
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def rel(a, b):
+    a, b = a.double().cpu(), b.double().cpu()
+    return float((a - b).norm() / b.norm())
+
+
+def _oracle_state(st, b):
+    return O.GraspState(st.codes4[b].cpu(), st.rscale[b].cpu(), st.cscale[b].cpu(),
+                        st.P8[b].cpu(), st.Pscale[b].cpu(), st.R8[b].cpu(), st.Rscale[b].cpu(),
+                        int(st.step.item()))
+
+
+def _singular_values(X):
+    """Singular values (ascending) of a matrix on the GPU, fp64, wide Gram."""
+    Xw = X.double() if X.shape[0] <= X.shape[1] else X.double().T
+    ev = torch.linalg.eigvalsh(Xw @ Xw.T)
+    return ev.clamp_min(0).sqrt()
+
+
+# (workload, shape group): LLaMA-1.1B 5632 x 2048 (tall) and 256 x 2048;
+# Qwen2.5-7B 3584 x 18944 (wide, the largest matrices) and 512 x 3584.
+FULL = [(3, 2), (3, 1), (4, 3), (4, 1)]
+
+
+@pytest.mark.parametrize("cid,gi", FULL)
+def test_full_size_group_step(cuda_lib, cid, gi):
+    gm = cuda_lib
+    w = WL.WORKLOADS[cid]
+    g = w.groups[gi]
+    B, m, n, k = g.count, g.m, g.n, w.k
+    base = w.group_base(gi)
+    sample = (0, B - 1)
+    step = gm.GraspStep(B, m, n, k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=gm.GM_NS_STANDARD,
+                        seed=w.seed, device=DEV)
+    st = gm.GraspState.zeros(B, m, n, k, DEV)
+    W = torch.empty((B, m, n), dtype=torch.float32, device=DEV)
+    G = torch.empty((B, m, n), dtype=w.gdtype, device=DEV)
+    for b in range(B):
+        W[b] = WL.initial_weight(w, base + b, m, n, device=DEV)
+    for t in (1, 2):
+        for b in range(B):
+            WL.gradient(w, base + b, t, m, n, device=DEV, out=G[b])
+        before = {b: _oracle_state(st, b) for b in sample}
+        W0 = {b: W[b].clone() for b in sample}
+        step(st, W, G)
+        torch.cuda.synchronize()
+        assert int(st.dev_status.item()) == 0
+        assert int(st.step.item()) == t
+    for b in sample:
+        Mg = step.stage_M()[b]
+        M = w.mu * O.rebuild_momentum(before[b]) + G[b].cpu().double()
+        assert rel(Mg, M) <= 1e-5, f"M_t of matrix {b}"
+        Q = O.warm_start(O.dequant8(before[b].R8, before[b].Rscale), w.seed, b)
+        P, R, _, _ = O.power_iteration(M, Q)
+        Pg, Rg = step.stage_P()[b].cpu(), step.stage_R()[b].cpu()
+        assert rel(Pg, P) <= 1e-5 and rel(Rg, R) <= 1e-5, f"P, R of matrix {b}"
+        q, s = O.quant8(Pg)
+        assert torch.equal(st.P8[b].cpu(), q) and torch.equal(st.Pscale[b].cpu(), s)
+        q, s = O.quant8(Rg)
+        assert torch.equal(st.R8[b].cpu(), q) and torch.equal(st.Rscale[b].cpu(), s)
+        q4, _, _ = O.grid_quant4((M - P @ R.T).to(torch.float32))
+        diff = (O.unpack_nibbles(st.codes4[b].cpu()).int() - q4.int()).abs()
+        assert int(diff.max()) <= 1 and float((diff > 0).double().mean()) <= 1e-4
+        # update direction vs the scalar quintic on the momentum's spectrum
+        s_in = _singular_values(Mg)
+        want = O.quintic_scalar(s_in / s_in.pow(2).sum().sqrt(), T=w.T).sort().values
+        got = _singular_values((W0[b] - W[b]) / w.eta)
+        err = (got - want).abs()
+        print(f"\n[{w.name} {m}x{n} b={b}] sigma(O) in [{float(got.min()):.4f}, "
+              f"{float(got.max()):.4f}], |sorted diff| max {float(err.max()):.4f} "
+              f"mean {float(err.mean()):.5f}")
+        # bf16 stores each product with unit roundoff u = 2^-8; over T steps the
+        # errors add and the quintic's slope (<= a = 3.4445 near 0) can amplify
+        # them for the smallest singular values, so single values may move by a
+        # few u; on the flat part of the band, where most values sit, the mean
+        # stays well below u.
+        assert float(err.max()) <= 0.06 and float(err.mean()) <= 0.004
