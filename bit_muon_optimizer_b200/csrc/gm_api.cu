@@ -45,7 +45,8 @@ void expand_abc(const float* abc, int T, float* out) {
 }
 
 struct StepLayout {
-  size_t M, Q, P, R, X, scale, norm2, Ppart, Ptil, gram, Tm, Rpart, qnorm, ns, total;
+  size_t M, Q, P, R, X, scale, norm2, Ppart, Ptil, gram, Tm, Rpart, qnorm, QF, RF, PF, PA, RB, PB,
+      ns, total;
   int csplit, rsplit_b, rsplit_g, ntiles;
 };
 
@@ -72,6 +73,13 @@ StepLayout step_layout(int B, int m, int n, int k, int ns_mode, bool with_ns) {
   L.Tm = take(Bz * kz * kz * 8);
   L.Rpart = take(Bz * L.rsplit_b * nz * kz * 8);
   L.qnorm = take(Bz * kz * 4);
+  const FactorFrags fw = factor_frag_words(B, m, n, k);
+  L.QF = take((size_t)fw.QF * 4);
+  L.RF = take((size_t)fw.RF * 4);
+  L.PF = take((size_t)fw.PF * 4);
+  L.PA = take((size_t)fw.PA * 4);
+  L.RB = take((size_t)fw.RB * 4);
+  L.PB = take((size_t)fw.PB * 4);
   if (with_ns)
     L.ns = take(ns_mode == GM_NS_GRAM ? ns_gram_ws_bytes(B, m, n) : ns_standard_ws_bytes(B, m, n));
   L.total = off;
@@ -96,6 +104,8 @@ NsLayout ns_layout(int B, int m, int n, bool gram) {
 }
 
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+// NULL counts as aligned (optional arguments are checked for presence separately).
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 }  // namespace
 
@@ -204,10 +214,14 @@ gm_status gm_dequant_rebuild(int B, int m, int n, int k, const uint8_t* codes4,
   GM_CHECK_ARG(k >= 0 && k <= kMaxK, "k=%d out of [0, %d]", k, kMaxK);
   GM_CHECK_ARG(codes4 && rscale && cscale && M_out, "NULL state or output pointer");
   GM_CHECK_ARG(k == 0 || (P8 && Pscale && R8 && Rscale), "k > 0 needs P8, Pscale, R8, Rscale");
+  GM_CHECK_ARG(al16(codes4) && al16(rscale) && al16(cscale) && al16(P8) && al16(Pscale) &&
+                   al16(R8) && al16(Rscale) && al16(M_out),
+               "device arrays must be 16-byte aligned");
   GM_DEVICE();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   GM_CUDA(launch_rebuild(B, m, n, k, codes4, rscale, cscale, P8, Pscale, R8, Rscale, nullptr, 1.0f,
-                         nullptr, GM_F32, nullptr, M_out, nullptr, nullptr, nullptr, s));
+                         nullptr, GM_F32, nullptr, nullptr, nullptr, nullptr, M_out, nullptr, nullptr,
+                         nullptr, s));
   return GM_OK;
 }
 
@@ -219,6 +233,8 @@ gm_status gm_momentum_powerit(int B, int m, int n, int k, float mu, const float*
   GM_CHECK_ARG(k >= 1 && k <= kMaxK, "k=%d out of [1, %d]", k, kMaxK);
   GM_CHECK_ARG(G && M_out && P_out && R_out, "NULL G or output pointer");
   GM_CHECK_ARG(gdt == GM_F32 || gdt == GM_BF16 || gdt == GM_F16, "bad gdt %d", (int)gdt);
+  GM_CHECK_ARG(al16(M_prev) && al16(G) && al16(R_prev) && al16(M_out) && al16(P_out) && al16(R_out),
+               "device arrays must be 16-byte aligned");
   StepLayout L = step_layout(B, m, n, k, GM_NS_STANDARD, false);
   if (!ws || ws_bytes < L.total || !aligned256(ws))
     return set_error(GM_E_WORKSPACE, "workspace needs %zu bytes, 256-aligned", L.total);
@@ -233,12 +249,15 @@ gm_status gm_momentum_powerit(int B, int m, int n, int k, float mu, const float*
   double* Tm = reinterpret_cast<double*>(w + L.Tm);
   double* Rpart = reinterpret_cast<double*>(w + L.Rpart);
   float* scale = reinterpret_cast<float*>(w + L.scale);
-  GM_CUDA(launch_warm_start(B, n, k, nullptr, nullptr, R_prev, seed, Q, nullptr, nullptr, s));
+  uint32_t* QF = reinterpret_cast<uint32_t*>(w + L.QF);
+  uint32_t* PB = reinterpret_cast<uint32_t*>(w + L.PB);
+  GM_CUDA(launch_warm_start(B, m, n, k, nullptr, nullptr, nullptr, nullptr, R_prev, seed, Q, nullptr,
+                            QF, nullptr, nullptr, nullptr, s));
   GM_CUDA(launch_rebuild(B, m, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-                         M_prev, mu, G, gdt, Q, M_out, norm2, Ppart, nullptr, s));
+                         M_prev, mu, G, gdt, Q, QF, nullptr, nullptr, M_out, norm2, Ppart, nullptr, s));
   GM_CUDA(launch_orth(B, m, k, L.csplit, Ppart, Ptil, gram, Tm, norm2, L.ntiles, 1e-7f, scale,
-                      P_out, nullptr, s));
-  GM_CUDA(launch_backproject(B, m, n, k, M_out, P_out, nullptr, nullptr, false, Rpart, R_out,
+                      P_out, PB, nullptr, nullptr, s));
+  GM_CUDA(launch_backproject(B, m, n, k, M_out, PB, nullptr, nullptr, false, Rpart, R_out, nullptr,
                              nullptr, s));
   return GM_OK;
 }
@@ -250,9 +269,12 @@ gm_status gm_grid_quant4(int B, int m, int n, int k, const float* X, const float
   GM_CHECK_ARG(X && codes4 && rscale && cscale, "NULL input or output pointer");
   GM_CHECK_ARG((P == nullptr) == (R == nullptr), "P and R must both be NULL or both set");
   GM_CHECK_ARG(!P || (k >= 1 && k <= kMaxK), "k=%d out of [1, %d]", k, kMaxK);
+  GM_CHECK_ARG(al16(X) && al16(P) && al16(R) && al16(codes4) && al16(rscale) && al16(cscale),
+               "device arrays must be 16-byte aligned");
   GM_DEVICE();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  GM_CUDA(launch_residual_quant4(B, m, n, P ? k : 0, X, P, R, codes4, rscale, cscale, nullptr, s));
+  GM_CUDA(launch_residual_quant4(B, m, n, P ? k : 0, X, P, R, nullptr, nullptr, codes4, rscale,
+                                 cscale, nullptr, s));
   return GM_OK;
 }
 
@@ -273,6 +295,7 @@ static gm_status ns_common(int B, int m, int n, const void* X, gm_dtype xdt, con
                            gm_dtype odt, void* ws, size_t ws_bytes, gm_stream_t stream, bool gram) {
   GM_CHECK_ARG(shape_ok(B, m, n), "bad shape B=%d m=%d n=%d", B, m, n);
   GM_CHECK_ARG(X && O, "NULL X or O");
+  GM_CHECK_ARG(al16(X) && al16(O), "device arrays must be 16-byte aligned");
   GM_CHECK_ARG(xdt == GM_F32 || xdt == GM_BF16 || xdt == GM_F16, "bad xdt");
   GM_CHECK_ARG(odt == GM_F32 || odt == GM_BF16 || odt == GM_F16, "bad odt");
   GM_CHECK_ARG(T >= 1 && T <= GM_MAX_T, "T=%d out of [1, %d]", T, GM_MAX_T);
@@ -327,6 +350,9 @@ gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* prm, const g
                    st->Rscale && st->step && st->dev_status,
                "NULL state pointer");
   GM_CHECK_ARG(W && G, "NULL W or G");
+  GM_CHECK_ARG(al16(W) && al16(G) && al16(st->codes4) && al16(st->rscale) && al16(st->cscale) &&
+                   al16(st->P8) && al16(st->Pscale) && al16(st->R8) && al16(st->Rscale),
+               "device arrays must be 16-byte aligned");
   GM_CHECK_ARG(gdt == GM_F32 || gdt == GM_BF16 || gdt == GM_F16, "bad gdt");
   StepLayout L = step_layout(B, m, n, k, prm->ns, true);
   if (!ws || ws_bytes < L.total || !aligned256(ws))
@@ -346,6 +372,12 @@ gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* prm, const g
   double* gram = reinterpret_cast<double*>(w + L.gram);
   double* Tm = reinterpret_cast<double*>(w + L.Tm);
   double* Rpart = reinterpret_cast<double*>(w + L.Rpart);
+  uint32_t* QF = reinterpret_cast<uint32_t*>(w + L.QF);
+  uint32_t* RF = reinterpret_cast<uint32_t*>(w + L.RF);
+  uint32_t* PF = reinterpret_cast<uint32_t*>(w + L.PF);
+  uint32_t* PA = reinterpret_cast<uint32_t*>(w + L.PA);
+  uint32_t* RB = reinterpret_cast<uint32_t*>(w + L.RB);
+  uint32_t* PB = reinterpret_cast<uint32_t*>(w + L.PB);
   int32_t* status = st->dev_status;
   float tab[3 * GM_MAX_T];
   expand_abc(prm->abc, prm->T, tab);
@@ -353,18 +385,21 @@ gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* prm, const g
 
   GM_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
   // worked step 2: warm start from the stored R (read before it is overwritten)
-  GM_CUDA(launch_warm_start(B, n, k, st->R8, st->Rscale, nullptr, prm->seed, Q,
-                            reinterpret_cast<int*>(w + L.qnorm), status, s));
+  // (with the fragment copies of Q, R and P that the rebuild reads)
+  GM_CUDA(launch_warm_start(B, m, n, k, st->R8, st->Rscale, st->P8, st->Pscale, nullptr, prm->seed,
+                            Q, reinterpret_cast<int*>(w + L.qnorm), QF, RF, PF, status, s));
   // worked steps 1 and 3: rebuild M_{t-1}, M_t = mu M_{t-1} + G
   // (with the projection P~ = M Q of worked step 4 fused in)
   GM_CUDA(launch_rebuild(B, m, n, k, st->codes4, st->rscale, st->cscale, st->P8, st->Pscale,
-                         st->R8, st->Rscale, nullptr, prm->mu, G, gdt, Q, M, norm2, Ppart, status, s));
+                         st->R8, st->Rscale, nullptr, prm->mu, G, gdt, Q, QF, RF, PF, M, norm2, Ppart,
+                         status, s));
   // worked step 4: P = orth(P~), R = M^T P
   GM_CUDA(launch_orth(B, m, k, L.csplit, Ppart, Ptil, gram, Tm, norm2, L.ntiles, prm->eps, scale,
-                      P, status, s));
-  GM_CUDA(launch_backproject(B, m, n, k, M, P, scale, X, gramns, Rpart, R, status, s));
+                      P, PB, PA, status, s));
+  GM_CUDA(launch_backproject(B, m, n, k, M, PB, scale, X, gramns, Rpart, R, RB, status, s));
   // worked step 5: residual -> 4-bit grid codes; P, R -> 8-bit codes (state in place)
-  GM_CUDA(launch_residual_quant4(B, m, n, k, M, P, R, st->codes4, st->rscale, st->cscale, status, s));
+  GM_CUDA(launch_residual_quant4(B, m, n, k, M, P, R, PA, RB, st->codes4, st->rscale, st->cscale,
+                                 status, s));
   GM_CUDA(launch_quant8(B, m, n, k, P, st->P8, st->Pscale, R, st->R8, st->Rscale, st->step, status, s));
   // worked step 6: O = NS(M_t); W <- W - eta (O + wd W) in the last product's epilogue
   NsOutput out{1, nullptr, 0, W, prm->eta, prm->wd};

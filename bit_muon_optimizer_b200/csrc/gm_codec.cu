@@ -42,10 +42,129 @@ __device__ __forceinline__ double block_sum_d(double v, double* red) {
   return s;   // valid in thread 0
 }
 
+// ------------------------------------------------- warp tensor-core helpers
+// The rank-k contractions of the codec passes (at most 32 deep) run as
+// warp-level mma.sync: too shallow for the tcgen05 pipeline to pay, and on the
+// FMA pipe they made these HBM-bound passes issue-bound. Fragment layouts follow
+// the PTX ISA for mma.m16n8k8 .tf32 and mma.m16n8k16 .bf16 (row.col): lane =
+// 4 g + t; A holds rows g and g + 8, B column g, C/D rows g and g + 8 at
+// columns 2 t and 2 t + 1.
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// x = hi + lo + rest, |rest| <= 2^-22 |x|: hi keeps the top 11 significant bits
+// (a tf32 by truncation, exact), lo is the remainder rounded to tf32. Products
+// of two such pairs summed as lo*hi + hi*lo + hi*hi reach fp32-level accuracy
+// (the 3xTF32 emulation); the small terms go first.
+__device__ __forceinline__ uint32_t tf32_hi(float x) { return __float_as_uint(x) & 0xFFFFE000u; }
+__device__ __forceinline__ uint32_t tf32_lo(float x, uint32_t hi) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(__fsub_rn(x, __uint_as_float(hi))));
+  return r;
+}
+
+// x = p0 + p1 + p2 with every part a bf16: exact for normal fp32 (3 x 8
+// significant bits). Two values per word, the first in the low half.
+__device__ __forceinline__ void bf16_split3(float x, float y, uint32_t (&w)[3]) {
+#pragma unroll
+  for (int p = 0; p < 3; ++p) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    w[p] = *reinterpret_cast<const uint32_t*>(&h);
+    x = __fsub_rn(x, __low2float(h));
+    y = __fsub_rn(y, __high2float(h));
+  }
+}
+
+// 16-byte asynchronous global -> shared copies (zero-filled when !valid; the
+// source address is then not read).
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Copy `bytes` (a multiple of 16, both ends 16-byte aligned) from global to
+// shared memory with all threads of the block; the copies stay in flight.
+__device__ __forceinline__ void cp_async_block(void* smem, const void* gmem, int bytes) {
+  for (int c = threadIdx.x; c < (bytes >> 4); c += blockDim.x)
+    cp_async16(static_cast<uint8_t*>(smem) + 16 * c, static_cast<const uint8_t*>(gmem) + 16 * c, true);
+}
+
+// As above, zero-filling the bytes at and beyond `valid`.
+__device__ __forceinline__ void cp_async_block_zf(void* smem, const void* gmem, int bytes, int valid) {
+  for (int c = threadIdx.x; c < (bytes >> 4); c += blockDim.x) {
+    const bool ok = 16 * c < valid;
+    cp_async16(static_cast<uint8_t*>(smem) + 16 * c,
+               ok ? static_cast<const uint8_t*>(gmem) + 16 * c : gmem, ok);
+  }
+}
+
+constexpr int kCT = 512;   // threads of the 128 x 128 codec CTAs (16 warps)
+
+__host__ __device__ constexpr int kb16(int KP) { return KP < 16 ? 16 : KP; }
+
+// ---------------------------------------------- fragment-ordered factor copies
+// The rank-k factors are small (rows x k), so each is laid out once per step in
+// the order the warps' MMA fragments read it; a CTA then copies its slice into
+// shared memory with cp.async, as is. kp = factor_width(k), nl = kp / 8,
+// ksb = max(kp, 16) / 16, nsl = ceil(n / 64) column slabs; padding is zero.
+//   QF [B][nsl][8 s][nl][32][4]    Q hi, lo: B operand of the projection
+//   RF [B][nsl][8 nt][ksb][32][2]  R codes as bf16: B operand of the rebuild
+//   PF [B][m/16][ksb][3][32][4]    P codes x c_l, three bf16 parts: its A operand
+//   PA [B][m/16][nl][2][32][4]     -P hi, lo: A operand of the residual
+//   RB [B][nsl][8 nt][nl][32][4]   R hi, lo: B operand of the residual
+//   PB [B][m/8][nl][32][4]         P hi, lo: B operand of the back-projection
+// Column j of a slab sits in n-tile ((j & 15) >> 1) at fragment column
+// 2 (j >> 4 & 3) + (j & 1) for the rebuild / residual, and at k-step
+// ((j & 15) >> 1), k-slot (j >> 4 & 3) (+4 when j is odd) for the projection.
+__device__ __forceinline__ long long qf_at(int b, int nsl, int nl, int j, int l) {   // + 0/1 hi, + 2/3 lo
+  const int slab = j >> 6, jj = j & 63;
+  return ((((long long)(b * nsl + slab) * 8 + ((jj & 15) >> 1)) * nl + (l >> 3)) * 32 + 4 * (l & 7) +
+          (jj >> 4)) * 4 + (jj & 1);
+}
+__device__ __forceinline__ long long rf_at16(int b, int nsl, int ksb, int j, int l) {   // 16-bit index
+  const int slab = j >> 6, jj = j & 63, ll = l & 15;
+  return (((((long long)(b * nsl + slab) * 8 + ((jj & 15) >> 1)) * ksb + (l >> 4)) * 32 +
+           4 * (2 * (jj >> 4) + (jj & 1)) + ((ll >> 1) & 3)) * 2 + (ll >> 3)) * 2 + (ll & 1);
+}
+__device__ __forceinline__ long long pf_at16(int b, int m16, int ksb, int i, int l, int part) {
+  const int r = i & 15, ll = l & 15;
+  return (((((long long)(b * m16 + (i >> 4)) * ksb + (l >> 4)) * 3 + part) * 32 + 4 * (r & 7) +
+           ((ll >> 1) & 3)) * 4 + (r >> 3) + 2 * (ll >> 3)) * 2 + (ll & 1);
+}
+__device__ __forceinline__ long long pa_at(int b, int m16, int nl, int i, int l) {   // + 128 lo
+  const int r = i & 15, ll = l & 7;
+  return (((((long long)(b * m16 + (i >> 4)) * nl + (l >> 3)) * 2) * 32 + 4 * (r & 7) + (ll & 3)) * 4 +
+          (r >> 3) + 2 * (ll >> 2));
+}
+__device__ __forceinline__ long long rb_at(int b, int nsl, int nl, int j, int l) {   // + 2 lo
+  const int slab = j >> 6, jj = j & 63, ll = l & 7;
+  return ((((long long)(b * nsl + slab) * 8 + ((jj & 15) >> 1)) * nl + (l >> 3)) * 32 +
+          4 * (2 * (jj >> 4) + (jj & 1)) + (ll & 3)) * 4 + (ll >> 2);
+}
+__device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+
 // ------------------------------------------------------------------ S2
 __global__ void __launch_bounds__(kThreads) k_warm_start(int n, int k, const int8_t* R8,
                                                           const float* Rscale, const float* Rprev,
-                                                          uint64_t seed, float* Q,
+                                                          uint64_t seed, float* Q, uint32_t* QF,
                                                           const int32_t* skip) {
   if (skip && *skip) return;
   const int b = blockIdx.x, t = threadIdx.x;
@@ -75,17 +194,26 @@ __global__ void __launch_bounds__(kThreads) k_warm_start(int n, int k, const int
   }
   __syncthreads();
   const float rad = (float)(1.0 / sqrt((double)n));
-  for (long long e = t; e < (long long)n * k; e += kThreads) {
-    const int j = (int)(e / k), l = (int)(e % k);
-    const double inv = nrm2[l];
-    float q;
-    if (inv == 0.0) {
-      const uint64_t ctr = seed ^ ((uint64_t)b << 48) ^ ((uint64_t)j << 16) ^ (uint64_t)l;
-      q = (splitmix64(ctr) >> 63) ? -rad : rad;
-    } else {
-      q = (float)((double)rhat(j, l) * inv);
+  const int kp = factor_width(k), nsl = cdiv(n, 64);
+  for (long long e = t; e < (long long)nsl * 64 * kp; e += kThreads) {
+    const int j = (int)(e / kp), l = (int)(e % kp);
+    float q = 0.f;
+    if (j < n && l < k) {
+      const double inv = nrm2[l];
+      if (inv == 0.0) {
+        const uint64_t ctr = seed ^ ((uint64_t)b << 48) ^ ((uint64_t)j << 16) ^ (uint64_t)l;
+        q = (splitmix64(ctr) >> 63) ? -rad : rad;
+      } else {
+        q = (float)((double)rhat(j, l) * inv);
+      }
+      Q[off + (long long)j * k + l] = q;
     }
-    Q[off + e] = q;
+    if (QF) {
+      const long long at = qf_at(b, nsl, kp / 8, j, l);
+      const uint32_t hi = tf32_hi(q);
+      QF[at] = hi;
+      QF[at + 2] = tf32_lo(q, hi);
+    }
   }
 }
 
@@ -120,234 +248,378 @@ __global__ void __launch_bounds__(kThreads) k_colnorm_int(int n, int k, const in
   }
 }
 
-__global__ void __launch_bounds__(kThreads) k_warm_q(int n, int k, const int8_t* __restrict__ R8,
+// Blocks [0, nbq) cover the nsl * 64 x kb elements of Q and R: Q, its fragments
+// QF and the R code fragments RF; blocks [nbq, ..) the m x kb elements of P:
+// the P code fragments PF (c_l = Pscale_l Rscale_l / 127^2).
+__global__ void __launch_bounds__(kThreads) k_warm_q(int m, int n, int k, int nbq,
+                                                      const int8_t* __restrict__ R8,
                                                       const float* __restrict__ Rscale,
+                                                      const int8_t* __restrict__ P8,
+                                                      const float* __restrict__ Pscale,
                                                       const int* __restrict__ norm2, uint64_t seed,
-                                                      float* __restrict__ Q, const int32_t* skip) {
+                                                      float* __restrict__ Q, uint32_t* __restrict__ QF,
+                                                      uint16_t* __restrict__ RF, uint16_t* __restrict__ PF,
+                                                      const int32_t* skip) {
   if (skip && *skip) return;
   const int b = blockIdx.y, t = threadIdx.x;
+  const int kp = factor_width(k), kb = kb16(kp), nsl = cdiv(n, 64);
   __shared__ double inv[kMaxK];
+  __shared__ float cf[kMaxK];
   if (t < k) {
     const int s2 = norm2[b * k + t];
     const float sc = Rscale[b * k + t];
     inv[t] = (s2 > 0 && sc != 0.f) ? (sc > 0.f ? 1.0 : -1.0) / sqrt((double)s2) : 0.0;
+    cf[t] = __fdiv_rn(__fmul_rn(Pscale[b * k + t], sc), 16129.0f);
   }
   __syncthreads();
-  const float rad = (float)(1.0 / sqrt((double)n));
-  const long long base = (long long)blockIdx.x * kThreads * 4;
+  if ((int)blockIdx.x < nbq) {
+    const float rad = (float)(1.0 / sqrt((double)n));
+    const long long base = (long long)blockIdx.x * kThreads * 4;
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const long long e = base + u * kThreads + t;
-    if (e >= (long long)n * k) break;
-    const int j = (int)(e / k), l = (int)(e % k);
-    const double iv = inv[l];
-    float q;
-    if (iv == 0.0) {
-      const uint64_t ctr = seed ^ ((uint64_t)b << 48) ^ ((uint64_t)j << 16) ^ (uint64_t)l;
-      q = (splitmix64(ctr) >> 63) ? -rad : rad;
-    } else {
-      q = (float)((double)R8[(long long)b * n * k + e] * iv);
+    for (int u = 0; u < 4; ++u) {
+      const long long e = base + u * kThreads + t;
+      if (e >= (long long)nsl * 64 * kb) break;
+      const int j = (int)(e / kb), l = (int)(e % kb);
+      const bool valid = j < n && l < k;
+      const float rq = valid ? (float)R8[((long long)b * n + j) * k + l] : 0.f;
+      if (l < kp) {
+        float q = 0.f;
+        if (valid) {
+          const double iv = inv[l];
+          if (iv == 0.0) {
+            const uint64_t ctr = seed ^ ((uint64_t)b << 48) ^ ((uint64_t)j << 16) ^ (uint64_t)l;
+            q = (splitmix64(ctr) >> 63) ? -rad : rad;
+          } else {
+            q = (float)((double)rq * iv);
+          }
+          Q[((long long)b * n + j) * k + l] = q;
+        }
+        const long long at = qf_at(b, nsl, kp / 8, j, l);
+        const uint32_t hi = tf32_hi(q);
+        QF[at] = hi;
+        QF[at + 2] = tf32_lo(q, hi);
+      }
+      RF[rf_at16(b, nsl, kb / 16, j, l)] = bf16_bits(rq);
     }
-    Q[(long long)b * n * k + e] = q;
+  } else {
+    const long long base = (long long)(blockIdx.x - nbq) * kThreads * 4;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const long long e = base + u * kThreads + t;
+      if (e >= (long long)m * kb) break;
+      const int i = (int)(e / kb), l = (int)(e % kb);
+      float x = l < k ? __fmul_rn((float)P8[((long long)b * m + i) * k + l], cf[l]) : 0.f;
+#pragma unroll
+      for (int part = 0; part < 3; ++part) {
+        const uint16_t h = bf16_bits(x);
+        PF[pf_at16(b, m >> 4, kb / 16, i, l, part)] = h;
+        x = __fsub_rn(x, __bfloat162float(__ushort_as_bfloat16(h)));
+      }
+    }
   }
 }
 
 // ------------------------------------------------------------------ S1 + S3
 // Rebuild + momentum, fused with the projection P~ = M Q.
-// CTA: 64 rows x 128 columns (half a grid block); thread (ty, tx) owns rows
-// ty + 16 i (i < 4) and columns 4 tx + {0..3}, 64 + 4 tx + {0..3}.
-// Global loads of the tile are issued before the rank-k product. The decoded
-// nibble value q / 7 comes from a 16-entry table filled with IEEE divisions, so it
-// is bit-identical to (float)q / 7.0f. P~ partials of the tile (sum over its 128
-// columns, fp32) go to Ppart[b][bj][row][l]; the orthonormalisation sums the
-// column blocks in fp64 in a fixed order.
-constexpr int kRB = 64;   // rows per rebuild CTA
+// CTA: 64 rows x 128 columns (half a grid block), 8 warps, two CTAs per SM.
+// Warp w owns the rows 16 (w & 3) .. + 15 and the 64-column slab w >> 2; lane
+// (g, t) the rows g and g + 8 of the
+// warp's 16 and the 16 consecutive columns 16 t .. 16 t + 15 of the slab, so its
+// loads and stores are whole 16-column runs. Column 16 t + 2 s + e of the slab
+// is column 2 t + e of n-tile s in the C fragments, which makes
+//   * the rank-k rebuild P^ R^T eight n-tiles of bf16 mma.m16n8k16 with
+//     A = the 8-bit P codes times c_l = Pscale_l Rscale_l / 127^2, split into
+//     three bf16 parts (exact), and B = the R codes (exact in bf16);
+//   * the projection a tf32 mma.m16n8k8 whose A operand is M read straight from
+//     those fragments (k-step s = slab columns 16 t + 2 s + {0, 1} of every t)
+//     and whose B is Q, both split hi + lo (3xTF32).
+// The tile's raw factors (R and P codes, Q) are copied to shared memory with
+// cp.async while the element loads are in flight, then laid out as fragments.
+// The decoded nibble value q / 7 comes from a 16-entry table filled with IEEE
+// divisions, so it is bit-identical to (float)q / 7.0f. P~ partials of the tile
+// (sum over its 128 columns, the two slabs added in order) go to
+// Ppart[b][bj][row][l]; the orthonormalisation sums the column blocks in fp64 in
+// a fixed order.
+constexpr int kRB = 64;     // rows per rebuild CTA
+constexpr int kRBT = 256;  // threads per rebuild CTA
 
-__device__ __forceinline__ void reduce_scatter16(float (&v)[16], int tx) {
-  // After the four steps lane tx (of a 16-lane group) holds the group sum of v[tx].
-#pragma unroll
-  for (int s = 8; s >= 1; s >>= 1) {
-    const bool up = (tx & s) != 0;
-#pragma unroll
-    for (int j = 0; j < s; ++j) {
-      const float send = up ? v[j] : v[j + s];
-      const float keep = up ? v[j + s] : v[j];
-      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-    }
-  }
+// 32-bit words of the rebuild CTA's dynamic shared memory: Q fragments, slab
+// reduction, raw Q, then (state) R and P code fragments and raw R and P codes
+__host__ __device__ constexpr int rebuild_smem_words(int KP, bool state) {
+  return 2 * 8 * (KP / 8) * 32 * 4 + kRB * KP + kGrid * KP +
+         (state ? 2 * 8 * (kb16(KP) / 16) * 32 * 2 + 4 * (kb16(KP) / 16) * 3 * 32 * 4 +
+                      (kGrid + kRB) * KP / 4
+                : 0);
 }
 
 enum RebuildSrc { SRC_STATE = 0, SRC_DENSE = 1, SRC_ZERO = 2 };
 
 // KP: the factor width k rounded up to 8, 16 or 32 (columns beyond k are zero).
-template <int SRC, bool G32, int KP>
-__global__ void __launch_bounds__(kThreads, 2) k_rebuild_proj(
+// FR: the fragments come ready-made (QF, RF, PF in global memory); otherwise the
+// CTA builds them from the raw factors.
+template <int SRC, bool G32, int KP, bool FR>
+__global__ void __launch_bounds__(kRBT, 2) k_rebuild_proj(
     int m, int n, int k, const uint8_t* __restrict__ codes4, const float* __restrict__ rscale,
     const float* __restrict__ cscale, const int8_t* __restrict__ P8,
     const float* __restrict__ Pscale, const int8_t* __restrict__ R8,
     const float* __restrict__ Rscale, const float* __restrict__ Mprev, float mu,
-    const void* __restrict__ G, int gdt, const float* __restrict__ Q, float* __restrict__ M,
-    double* __restrict__ norm2_part, float* __restrict__ Ppart, int32_t* status) {
-  const int bj = blockIdx.x, bh = blockIdx.y, b = blockIdx.z;
-  const int nb = gridDim.x;
-  const int mb = cdiv(m, kGrid);
-  const int r0 = bh * kRB, c0 = bj * kGrid, bi = r0 / kGrid;
-  const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
-  constexpr int KK = SRC == SRC_STATE ? KP : 0;
-  extern __shared__ __align__(16) float sm[];
-  float* Ps = sm;                  // [KK][64]
-  float* Rs = Ps + KK * kRB;       // [KK][128]
-  float* Qs = Rs + KK * kGrid;     // [KP][128] (with Q)
+    const void* __restrict__ G, int gdt, const float* __restrict__ Q,
+    const uint32_t* __restrict__ QFg, const uint32_t* __restrict__ RFg,
+    const uint32_t* __restrict__ PFg, float* __restrict__ M, double* __restrict__ norm2_part,
+    float* __restrict__ Ppart, int32_t* status) {
+  constexpr bool ST = SRC == SRC_STATE;
+  constexpr int NL = KP / 8, KSB = kb16(KP) / 16;
+  const int bj = blockIdx.x, bi = blockIdx.y, b = blockIdx.z;
+  const int nb = gridDim.x, mb = gridDim.y;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int g = lane >> 2, tq = lane & 3, rb = warp & 3, slab = warp >> 2;
+  const int r0 = bi * kRB, c0 = bj * kGrid;
+  const int nrows = min(kRB, m - r0), ncols = min(kGrid, n - c0);   // multiples of 16
+  extern __shared__ __align__(16) uint32_t smr[];
+  uint32_t* QF = smr;                                             // [slab][s][NL][lane][4]
+  float* RED = reinterpret_cast<float*>(QF + 2 * 8 * NL * 32 * 4);   // [64][KP]
+  float* Qraw = RED + kRB * KP;                                      // [128][k]
+  uint32_t* RF = reinterpret_cast<uint32_t*>(Qraw + kGrid * KP);     // [slab][nt][KSB][lane][2]
+  uint32_t* PF = RF + 2 * 8 * KSB * 32 * 2;                          // [rb][KSB][part][lane][4]
+  int8_t* R8raw = reinterpret_cast<int8_t*>(PF + 4 * KSB * 3 * 32 * 4);   // [128][k]
+  int8_t* P8raw = R8raw + kGrid * KP;                                     // [64][k]
   __shared__ float deq4[16];
-  __shared__ double red[kThreads / 32];
+  __shared__ float cfac[32];
+  __shared__ double red[kRBT / 32];
   const long long mn = (long long)m * n;
   const bool f16 = gdt == GM_F16;
+  const int cb = c0 + 64 * slab + 16 * tq;   // n % 16 == 0: the run is all in or all out
+  const bool colok = cb < n;
 
-  // 1. global loads of this thread's 32 elements, all issued up front
-  uint32_t cw[4][2];      // four nibbles per (row, half)
-  float4 mpv[4][2];       // dense M_prev
-  uint2 gw[4][2];         // 16-bit gradient
-  float4 gf[4][2];        // fp32 gradient
-  float rsc[4];
+  // 1. global loads of this thread's 2 x 16 elements, issued before the staging
+  uint32_t gw[2][8];   // 16-bit gradient, two per word
+  float gf[2][16];     // fp32 gradient
+  float mpv[2][16];    // dense M_prev
+  uint2 cw[2];         // 16 nibbles per row
+  float rsc[2], cs[16];
+  bool ok[2];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int gi = r0 + ty + 16 * i;
-    if (SRC == SRC_STATE) rsc[i] = gi < m ? rscale[((long long)b * m + gi) * nb + bj] : 0.f;
+  for (int h = 0; h < 2; ++h) {
+    const int gi = r0 + 16 * rb + g + 8 * h;
+    ok[h] = gi < m && colok;
+    const long long base = (long long)b * mn + (long long)gi * n + cb;
+    if constexpr (G32) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int cb = c0 + 64 * h + 4 * tx;
-      const bool ok = gi < m && cb < n;
-      const long long base = (long long)b * mn + (long long)gi * n + cb;
-      if (SRC == SRC_STATE)
-        cw[i][h] = ok ? *reinterpret_cast<const uint16_t*>(codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2) : 0u;
-      if (SRC == SRC_DENSE)
-        mpv[i][h] = ok ? *reinterpret_cast<const float4*>(Mprev + base) : make_float4(0.f, 0.f, 0.f, 0.f);
-      if (G32) gf[i][h] = (ok && G) ? *reinterpret_cast<const float4*>(static_cast<const float*>(G) + base)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-      else gw[i][h] = (ok && G) ? *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(G) + base)
-                                : make_uint2(0u, 0u);
-    }
-  }
-  float cs[8];
-  if (SRC == SRC_STATE) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int gj = c0 + 64 * h + 4 * tx + e;
-        cs[4 * h + e] = gj < n ? cscale[((long long)b * mb + bi) * n + gj] : 0.f;
+      for (int u = 0; u < 4; ++u) {
+        const float4 v = (ok[h] && G)
+                             ? reinterpret_cast<const float4*>(static_cast<const float*>(G) + base)[u]
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        gf[h][4 * u] = v.x; gf[h][4 * u + 1] = v.y; gf[h][4 * u + 2] = v.z; gf[h][4 * u + 3] = v.w;
       }
+    } else {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint4 v = (ok[h] && G)
+                            ? reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(G) + base)[u]
+                            : make_uint4(0u, 0u, 0u, 0u);
+        gw[h][4 * u] = v.x; gw[h][4 * u + 1] = v.y; gw[h][4 * u + 2] = v.z; gw[h][4 * u + 3] = v.w;
+      }
+    }
+    if constexpr (ST) {
+      cw[h] = ok[h] ? *reinterpret_cast<const uint2*>(codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2)
+                    : make_uint2(0u, 0u);
+      rsc[h] = gi < m ? rscale[((long long)b * m + gi) * nb + bj] : 0.f;
+    }
+    if constexpr (SRC == SRC_DENSE) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 v = ok[h] ? reinterpret_cast<const float4*>(Mprev + base)[u]
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        mpv[h][4 * u] = v.x; mpv[h][4 * u + 1] = v.y; mpv[h][4 * u + 2] = v.z; mpv[h][4 * u + 3] = v.w;
+      }
+    }
+  }
+  if constexpr (ST) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float4 v = colok ? *reinterpret_cast<const float4*>(cscale + ((long long)b * cdiv(m, kGrid) + r0 / kGrid) * n + cb + 4 * u)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      cs[4 * u] = v.x; cs[4 * u + 1] = v.y; cs[4 * u + 2] = v.z; cs[4 * u + 3] = v.w;
+    }
   }
 
-  // 2. factors of the tile into shared memory
+  // 2. the tile's factors: fragment slices (FR) or raw rows of k values
+  if constexpr (FR) {
+    const int nsl = cdiv(n, 64), vs = min(2, nsl - 2 * bj), vb = min(kRB / 16, (m >> 4) - r0 / 16);
+    constexpr int qw = 8 * NL * 128, rw = 8 * KSB * 64, pw = KSB * 3 * 128;   // words per slab / block
+    if (Q) cp_async_block_zf(QF, QFg + ((long long)b * nsl + 2 * bj) * qw, 2 * qw * 4, vs * qw * 4);
+    if constexpr (ST) {
+      cp_async_block_zf(RF, RFg + ((long long)b * nsl + 2 * bj) * rw, 2 * rw * 4, vs * rw * 4);
+      cp_async_block_zf(PF, PFg + ((long long)b * (m >> 4) + r0 / 16) * pw, (kRB / 16) * pw * 4, vb * pw * 4);
+    }
+  } else {
+    if (Q) cp_async_block(Qraw, Q + ((long long)b * n + c0) * k, ncols * k * 4);
+    if constexpr (ST) {
+      cp_async_block(R8raw, R8 + ((long long)b * n + c0) * k, ncols * k);
+      cp_async_block(P8raw, P8 + ((long long)b * m + r0) * k, nrows * k);
+    }
+  }
+  cp_async_commit();
   if (t < 16) deq4[t] = __fdiv_rn((float)((t & 8) ? t - 16 : t), 7.0f);
-  if constexpr (SRC == SRC_STATE) {
-#pragma unroll 4
-    for (int e = t; e < kRB * KK; e += kThreads) {
-      const int rr = e / KK, l = e % KK, gi = r0 + rr;
-      Ps[l * kRB + rr] = (gi < m && l < k) ? deq8(P8[((long long)b * m + gi) * k + l], Pscale[b * k + l]) : 0.f;
-    }
-#pragma unroll 4
-    for (int e = t; e < kGrid * KK; e += kThreads) {
-      const int cc = e / KK, l = e % KK, gj = c0 + cc;
-      Rs[l * kGrid + cc] = (gj < n && l < k) ? deq8(R8[((long long)b * n + gj) * k + l], Rscale[b * k + l]) : 0.f;
-    }
+  if constexpr (ST && !FR) {
+    if (t < 32)
+      cfac[t] = t < k ? __fdiv_rn(__fmul_rn(Pscale[b * k + t], Rscale[b * k + t]), 16129.0f) : 0.f;
   }
-  if (Q) {
-#pragma unroll 4
-    for (int e = t; e < kGrid * KP; e += kThreads) {
-      const int cc = e / KP, l = e % KP, gj = c0 + cc;
-      Qs[l * kGrid + cc] = (gj < n && l < k) ? Q[((long long)b * n + gj) * k + l] : 0.f;
-    }
-  }
+  cp_async_wait<0>();
   __syncthreads();
 
-  // 3. rank-k rebuild P^ R^T
-  float acc[4][8];
+  // 3. factor fragments from the raw rows
+  if constexpr (ST && !FR) {
+    // R codes as the B operand of n-tile (jj & 15) / 2, column 2 (jj / 16) + jj % 2
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int it = 0; it < kGrid * KSB * 8 / kRBT; ++it) {
+      const int e = t + it * kRBT;
+      const int jl = e / (KSB * 8), l = 2 * (e % (KSB * 8));
+      const int8_t* rr = R8raw + jl * k;
+      const float v0 = (jl < ncols && l < k) ? (float)rr[l] : 0.f;
+      const float v1 = (jl < ncols && l + 1 < k) ? (float)rr[l + 1] : 0.f;
+      const int jj = jl & 63, ll = l & 15;
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
+      RF[((((jl >> 6) * 8 + ((jj & 15) >> 1)) * KSB + (l >> 4)) * 32 + 4 * (2 * (jj >> 4) + (jj & 1)) +
+           ((ll >> 1) & 3)) * 2 + (ll >> 3)] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+  }
+  if (Q && !FR) {
+    // Q as the projection's B operand: k-step (jj & 15) / 2, k-slot jj / 16 (+4 for odd jj)
 #pragma unroll 4
-  for (int l = 0; l < KK; ++l) {
-    const float4 ra = *reinterpret_cast<const float4*>(Rs + l * kGrid + 4 * tx);
-    const float4 rb = *reinterpret_cast<const float4*>(Rs + l * kGrid + 64 + 4 * tx);
-    const float rv[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+    for (int it = 0; it < kGrid * KP / kRBT; ++it) {
+      const int e = t + it * kRBT;
+      const int jl = e / KP, l = e % KP;
+      const float v = (jl < ncols && l < k) ? Qraw[jl * k + l] : 0.f;
+      const int jj = jl & 63;
+      uint32_t* q4 = QF + ((((jl >> 6) * 8 + ((jj & 15) >> 1)) * NL + (l >> 3)) * 32 + 4 * (l & 7) + (jj >> 4)) * 4;
+      const uint32_t hi = tf32_hi(v);
+      q4[jj & 1] = hi;
+      q4[2 + (jj & 1)] = tf32_lo(v, hi);
+    }
+  }
+  if constexpr (ST && !FR) {
+    // P codes x c_l as the A operand, three bf16 parts
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float pv = Ps[l * kRB + ty + 16 * i];
+    for (int it = 0; it < kRB * KSB * 8 / kRBT; ++it) {
+      const int e = t + it * kRBT;
+      const int il = e / (KSB * 8), l = 2 * (e % (KSB * 8));
+      const int8_t* pr = P8raw + il * k;
+      const float v0 = (il < nrows && l < k) ? __fmul_rn((float)pr[l], cfac[l]) : 0.f;
+      const float v1 = (il < nrows && l + 1 < k) ? __fmul_rn((float)pr[l + 1], cfac[l + 1]) : 0.f;
+      uint32_t w3[3];
+      bf16_split3(v0, v1, w3);
+      const int r = il & 15, ll = l & 15;
+      uint32_t* dst = PF + (((il >> 4) * KSB + (l >> 4)) * 3) * 128 +
+                      (4 * (r & 7) + ((ll >> 1) & 3)) * 4 + (r >> 3) + 2 * (ll >> 3);
+      dst[0] = w3[0];
+      dst[128] = w3[1];
+      dst[256] = w3[2];
+    }
+  }
+  if constexpr (!FR) __syncthreads();
+
+  // 4. rank-k rebuild P^ R^T
+  float acc[8][4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(pv, rv[j], acc[i][j]);
+  for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+  if constexpr (ST) {
+#pragma unroll
+    for (int ks = 0; ks < KSB; ++ks) {
+      uint32_t a[3][4];
+#pragma unroll
+      for (int p = 0; p < 3; ++p) {
+        const uint4 v = reinterpret_cast<const uint4*>(PF)[((rb * KSB + ks) * 3 + p) * 32 + lane];
+        a[p][0] = v.x; a[p][1] = v.y; a[p][2] = v.z; a[p][3] = v.w;
+      }
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const uint2 bv = reinterpret_cast<const uint2*>(RF)[((slab * 8 + nt) * KSB + ks) * 32 + lane];
+        mma_bf16(acc[nt], a[2], bv.x, bv.y);
+        mma_bf16(acc[nt], a[1], bv.x, bv.y);
+        mma_bf16(acc[nt], a[0], bv.x, bv.y);
+      }
     }
   }
 
-  // 4. M = mu M_prev + G, with M_prev = deq4 + P^R^T (state) or dense
+  // 5. M = mu M_prev + G, with M_prev = deq4 + P^R^T (state) or dense or zero
   float nsq = 0.f;
   bool bad = false;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int gi = r0 + ty + 16 * i;
+  for (int h = 0; h < 2; ++h) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int cb = c0 + 64 * h + 4 * tx;
-      const bool ok = gi < m && cb < n;
-      float g[4], mp[4];
-      if (G32) {
-        g[0] = gf[i][h].x; g[1] = gf[i][h].y; g[2] = gf[i][h].z; g[3] = gf[i][h].w;
-      } else {
-        g[0] = h16_to_float(gw[i][h].x & 0xFFFF, f16);
-        g[1] = h16_to_float(gw[i][h].x >> 16, f16);
-        g[2] = h16_to_float(gw[i][h].y & 0xFFFF, f16);
-        g[3] = h16_to_float(gw[i][h].y >> 16, f16);
-      }
-      if (SRC == SRC_STATE) {
+    for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float sc = fminf(rsc[i], cs[4 * h + e]);
-          mp[e] = __fmul_rn(deq4[(cw[i][h] >> (4 * e)) & 0xF], sc) + acc[i][4 * h + e];
+      for (int e = 0; e < 2; ++e) {
+        const int ce = 2 * nt + e;
+        float gv;
+        if constexpr (G32) gv = gf[h][ce];
+        else gv = h16_to_float((uint16_t)(gw[h][ce >> 1] >> (16 * (ce & 1))), f16);
+        float mp = 0.f;
+        if constexpr (ST) {
+          const uint32_t word = ce < 8 ? cw[h].x : cw[h].y;
+          const float sc = fminf(rsc[h], cs[ce]);
+          mp = __fadd_rn(__fmul_rn(deq4[(word >> (4 * (ce & 7))) & 0xF], sc), acc[nt][2 * h + e]);
+        } else if constexpr (SRC == SRC_DENSE) {
+          mp = mpv[h][ce];
         }
-      } else if (SRC == SRC_DENSE) {
-        mp[0] = mpv[i][h].x; mp[1] = mpv[i][h].y; mp[2] = mpv[i][h].z; mp[3] = mpv[i][h].w;
-      } else {
-        mp[0] = mp[1] = mp[2] = mp[3] = 0.f;
+        const float o = ok[h] ? __fadd_rn(__fmul_rn(mu, mp), gv) : 0.f;
+        acc[nt][2 * h + e] = o;   // keep M for the projection
+        bad |= !isfinite(o);
+        nsq = fmaf(o, o, nsq);
       }
-      float o[4];
+    }
+    if (ok[h]) {
+      float4* dst = reinterpret_cast<float4*>(M + (long long)b * mn + (long long)(r0 + 16 * rb + g + 8 * h) * n + cb);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        o[e] = ok ? __fadd_rn(__fmul_rn(mu, mp[e]), g[e]) : 0.f;
-        acc[i][4 * h + e] = o[e];        // keep M for the projection
-        bad |= !isfinite(o[e]);
-        nsq = fmaf(o[e], o[e], nsq);
-      }
-      if (ok)
-        *reinterpret_cast<float4*>(M + (long long)b * mn + (long long)gi * n + cb) =
-            make_float4(o[0], o[1], o[2], o[3]);
+      for (int u = 0; u < 4; ++u)
+        dst[u] = make_float4(acc[2 * u][2 * h], acc[2 * u][2 * h + 1], acc[2 * u + 1][2 * h],
+                             acc[2 * u + 1][2 * h + 1]);
     }
   }
   const double tot = block_sum_d((double)nsq, red);
-  if (t == 0 && norm2_part) norm2_part[((long long)b * cdiv(m, kRB) + bh) * nb + bj] = tot;
+  if (t == 0 && norm2_part) norm2_part[((long long)b * mb + bi) * nb + bj] = tot;
   if (bad && status) atomicExch(status, GM_E_NONFINITE);
 
-  // 5. projection partials: this tile's share of M Q, four columns of Q at a time
+  // 6. projection partials: this tile's share of M Q
   if (Q) {
-    for (int l0 = 0; l0 < KP; l0 += 4) {
-      float v[16];
+    float pt[NL][4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float4 qa = *reinterpret_cast<const float4*>(Qs + (l0 + j) * kGrid + 4 * tx);
-        const float4 qb = *reinterpret_cast<const float4*>(Qs + (l0 + j) * kGrid + 64 + 4 * tx);
-        const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+    for (int nl = 0; nl < NL; ++nl) pt[nl][0] = pt[nl][1] = pt[nl][2] = pt[nl][3] = 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float sacc = 0.f;
+    for (int s = 0; s < 8; ++s) {
+      const float xa[4] = {acc[s][0], acc[s][2], acc[s][1], acc[s][3]};
+      uint32_t ah[4], al[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) sacc = fmaf(acc[i][e], qv[e], sacc);
-          v[i * 4 + j] = sacc;
-        }
+      for (int i = 0; i < 4; ++i) {
+        ah[i] = tf32_hi(xa[i]);
+        al[i] = tf32_lo(xa[i], ah[i]);
       }
-      reduce_scatter16(v, tx);
-      const int row = r0 + ty + 16 * (tx >> 2), l = l0 + (tx & 3);
-      if (row < m && l < k) Ppart[(((long long)b * nb + bj) * m + row) * k + l] = v[0];
+#pragma unroll
+      for (int nl = 0; nl < NL; ++nl) {
+        const uint4 qv = reinterpret_cast<const uint4*>(QF)[((slab * 8 + s) * NL + nl) * 32 + lane];
+        mma_tf32(pt[nl], al, qv.x, qv.y);
+        mma_tf32(pt[nl], ah, qv.z, qv.w);
+        mma_tf32(pt[nl], ah, qv.x, qv.y);
+      }
+    }
+    if (slab == 1) {
+#pragma unroll
+      for (int nl = 0; nl < NL; ++nl)
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          RED[(16 * rb + g + 8 * (r >> 1)) * KP + 8 * nl + 2 * tq + (r & 1)] = pt[nl][r];
+    }
+    __syncthreads();
+    if (slab == 0) {
+#pragma unroll
+      for (int nl = 0; nl < NL; ++nl)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int rl = 16 * rb + g + 8 * (r >> 1), l = 8 * nl + 2 * tq + (r & 1);
+          if (r0 + rl < m && l < k)
+            Ppart[(((long long)b * nb + bj) * m + r0 + rl) * k + l] = pt[nl][r] + RED[rl * KP + l];
+        }
     }
   }
 }
@@ -486,10 +758,15 @@ __global__ void __launch_bounds__(32) k_orth_chol(int k, int rsplit, const doubl
   if (lane == 0 && scale) scale[b] = (float)(1.0 / (sqrt(ns2) + (double)eps));
 }
 
-// (c) P = P~ T (fp64), stored fp32.
-__global__ void __launch_bounds__(kThreads) k_orth_apply(int m, int k, const double* __restrict__ Ptil,
+// (c) P = P~ T (fp64), stored fp32, and as fragments: PB for the back-projection
+// (PB[b][i / 8][l / 8][lane][4] = {hi(P[8 s + t][l]), hi(P[8 s + t + 4][l]), lo, lo},
+// lane = 4 (l % 8) + t) and PA (-P) for the residual; zero for k <= l < kp.
+__global__ void __launch_bounds__(kThreads) k_orth_apply(int m, int k, int kp,
+                                                          const double* __restrict__ Ptil,
                                                           const double* __restrict__ Tmat,
                                                           float* __restrict__ P,
+                                                          uint32_t* __restrict__ PB,
+                                                          uint32_t* __restrict__ PA,
                                                           const int32_t* skip) {
   if (skip && *skip) return;
   const int b = blockIdx.y, t = threadIdx.x;
@@ -499,251 +776,426 @@ __global__ void __launch_bounds__(kThreads) k_orth_apply(int m, int k, const dou
   const long long base = (long long)blockIdx.x * kThreads * 4;
   for (int s = 0; s < 4; ++s) {
     const long long e = base + s * kThreads + t;
-    if (e >= (long long)m * k) break;
-    const long long i = e / k;
-    const int l = (int)(e % k);
-    const double* row = Ptil + ((long long)b * m + i) * k;
-    double v = 0.0;
-    for (int a = 0; a <= l; ++a) v = fma(row[a], Ts[a][l], v);   // T upper triangular
-    P[(long long)b * m * k + e] = (float)v;
+    if (e >= (long long)m * kp) break;
+    const long long i = e / kp;
+    const int l = (int)(e % kp);
+    float f = 0.f;
+    if (l < k) {
+      const double* row = Ptil + ((long long)b * m + i) * k;
+      double v = 0.0;
+      for (int a = 0; a <= l; ++a) v = fma(row[a], Ts[a][l], v);   // T upper triangular
+      f = (float)v;
+      P[((long long)b * m + i) * k + l] = f;
+    }
+    if (PB) {
+      const int c = (int)(i & 7);
+      uint32_t* dst = PB + ((((long long)b * (m >> 3) + (i >> 3)) * (kp >> 3) + (l >> 3)) * 32 +
+                            4 * (l & 7) + (c & 3)) * 4 + (c >> 2);
+      const uint32_t hi = tf32_hi(f);
+      dst[0] = hi;
+      dst[2] = tf32_lo(f, hi);
+    }
+    if (PA) {
+      const long long at = pa_at(b, m >> 4, kp >> 3, (int)i, l);
+      const uint32_t hi = tf32_hi(-f);
+      PA[at] = hi;
+      PA[at + 128] = tf32_lo(-f, hi);
+    }
   }
 }
 
 // ------------------------------------------------------------------ S5
 // R = M^T P over row splits, and the normalised wide-form NS input
 // X = round16(scale * M) (X = M^T when m > n).
-// CTA: 64 columns x the rows of its split, in chunks of 128 rows. Warp w owns
-// rows 16 w .. 16 w + 15 of a chunk, lane c the columns 2c, 2c + 1, so every
-// warp reads whole 256-byte row segments of M straight into registers; P rows
-// are broadcast from shared memory. fp32 sums over at most 1024 rows per split,
-// fp64 across splits.
+// CTA: 64 columns x the rows of its split, in chunks of 128 rows; 8 warps. Warp
+// w owns the 32-column half w & 1 and the rows 32 (w >> 1) .. + 31 of each chunk
+// as four k-steps of 8 rows. Per k-step, lane (g, t) loads the float4
+// M[i][4 g .. 4 g + 3] of rows i = 8 s + t and 8 s + t + 4 (one load instruction
+// reads four whole 128-byte row segments), through a two-stage cp.async ring
+// in shared memory (each thread reads back only its own copies, so the next
+// chunk streams in while this one is multiplied); element 2 mt + h of the float4 is row
+// g + 8 h of m-tile mt in the A fragment of M^T (tf32 mma.m16n8k8, 3xTF32
+// against P's precomputed fragments). fp32 sums over at most 1024 rows per
+// split, the four row warps added in order, fp64 across splits.
 template <int KP>
 __global__ void __launch_bounds__(kThreads, 2) k_backproject(int m, int n, int k, int rsplit,
                                                               const float* __restrict__ M,
-                                                              const float* __restrict__ P,
+                                                              const uint32_t* __restrict__ PB,
                                                               const float* __restrict__ scale,
                                                               uint16_t* __restrict__ X16, int f16,
                                                               double* __restrict__ Rpart,
                                                               const int32_t* skip) {
   if (skip && *skip) return;
-  constexpr int CB = 64, CH = 128, RPW = 16, XS = CH + 2;
-  extern __shared__ __align__(16) float smb[];
-  float* Ps = smb;                                             // [CH][KP]
-  uint16_t* Xt = reinterpret_cast<uint16_t*>(Ps + CH * KP);     // [CB][XS], tall staging
+  constexpr int NL = KP / 8, CH = 128, XS = 40;
+  __shared__ __align__(16) uint16_t Xt[8][32][XS];   // per-warp transpose tile [col][row]
+  __shared__ float redR[64][KP + 1];
+  extern __shared__ __align__(16) float4 Ms[];       // [stage][warp][slot][lane]
   const int cbk = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
-  const int t = threadIdx.x, cq = t & 31, rg = t >> 5;
-  const int c0 = cbk * CB;
-  const int col = c0 + 2 * cq;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int g = lane >> 2, tq = lane & 3, half = warp & 1, rg = warp >> 1;
+  const int c0 = cbk * 64 + 32 * half;   // the warp's 32 columns
+  const int cq = c0 + 4 * g;             // this lane's float4 (n % 16 == 0: all in or out)
+  const bool colok = cq < n;
   const int nchunks = cdiv(m, CH);
   const int per = cdiv(nchunks, rsplit);
   const int ch0 = split * per, ch1 = min(nchunks, ch0 + per);
   const float* Mb = M + (long long)b * m * n;
-  const float* Pb = P + (long long)b * m * k;
+  const uint4* PBb = reinterpret_cast<const uint4*>(PB) + (long long)b * (m >> 3) * NL * 32;
   const bool tall = m > n;
   const float sc = X16 ? scale[b] : 0.f;
   uint16_t* Xb = X16 ? X16 + (long long)b * m * n : nullptr;
 
-  float acc[2][KP];
+  float acc[2][NL][4];
 #pragma unroll
-  for (int c = 0; c < 2; ++c)
+  for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-    for (int l = 0; l < KP; ++l) acc[c][l] = 0.f;
+    for (int nl = 0; nl < NL; ++nl) acc[mt][nl][0] = acc[mt][nl][1] = acc[mt][nl][2] = acc[mt][nl][3] = 0.f;
 
-  for (int ch = ch0; ch < ch1; ++ch) {
-    const int i0 = ch * CH;
-    float2 mv[RPW];
+  auto issue = [&](int chn, int st) {
+    const int i0 = chn * CH + 32 * rg;
 #pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      const int gi = i0 + rg * RPW + r;
-      mv[r] = (gi < m && col < n) ? *reinterpret_cast<const float2*>(Mb + (long long)gi * n + col)
-                                  : make_float2(0.f, 0.f);
+    for (int j = 0; j < 8; ++j) {
+      const int gi = i0 + 8 * (j >> 1) + tq + 4 * (j & 1);
+      const bool ok = gi < m && colok;
+      cp_async16(&Ms[((st * 8 + warp) * 8 + j) * 32 + lane], ok ? Mb + (long long)gi * n + cq : Mb, ok);
     }
-    for (int e = t; e < CH * KP; e += kThreads) {
-      const int ii = e / KP, l = e % KP, gi = i0 + ii;
-      Ps[e] = (gi < m && l < k) ? Pb[(long long)gi * k + l] : 0.f;
+    cp_async_commit();
+  };
+  // P fragments of the warp's k-step sequence (chunk c, step s: rows c * 128 +
+  // 32 rg + 8 s), loaded one k-step ahead from L2
+  const int nq = (ch1 - ch0) * 4;
+  auto pb_load = [&](int q, uint4 (&dst)[NL]) {
+    const int i8 = (ch0 + (q >> 2)) * CH + 32 * rg + 8 * (q & 3);
+    const bool ok = q < nq && i8 < m;
+#pragma unroll
+    for (int nl = 0; nl < NL; ++nl)
+      dst[nl] = ok ? PBb[((long long)(i8 >> 3) * NL + nl) * 32 + lane] : make_uint4(0u, 0u, 0u, 0u);
+  };
+  uint4 pbn[NL];
+  pb_load(0, pbn);
+  if (ch0 < ch1) issue(ch0, 0);
+  for (int chn = ch0; chn < ch1; ++chn) {
+    const int i0 = chn * CH + 32 * rg;   // the warp's 32 rows
+    const int st = (chn - ch0) & 1;
+    if (chn + 1 < ch1) {
+      issue(chn + 1, st ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    float4 v[4][2];
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) v[s][hh] = Ms[((st * 8 + warp) * 8 + 2 * s + hh) * 32 + lane];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int i8 = i0 + 8 * s;
+      uint4 pb[NL];
+#pragma unroll
+      for (int nl = 0; nl < NL; ++nl) pb[nl] = pbn[nl];
+      pb_load((chn - ch0) * 4 + s + 1, pbn);
+      if (i8 >= m) continue;   // m % 8 == 0: a k-step is all in or all out (warp-uniform)
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const float xa[4] = {mt ? v[s][0].z : v[s][0].x, mt ? v[s][0].w : v[s][0].y,
+                             mt ? v[s][1].z : v[s][1].x, mt ? v[s][1].w : v[s][1].y};
+        uint32_t ah[4], al[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          ah[i] = tf32_hi(xa[i]);
+          al[i] = tf32_lo(xa[i], ah[i]);
+        }
+#pragma unroll
+        for (int nl = 0; nl < NL; ++nl) {
+          mma_tf32(acc[mt][nl], al, pb[nl].x, pb[nl].y);
+          mma_tf32(acc[mt][nl], ah, pb[nl].z, pb[nl].w);
+          mma_tf32(acc[mt][nl], ah, pb[nl].x, pb[nl].y);
+        }
+      }
     }
     if (Xb) {
+      if (!tall) {
 #pragma unroll
-      for (int r = 0; r < RPW; ++r) {
-        const int gi = i0 + rg * RPW + r;
-        const uint16_t x0 = float_to_h16(mv[r].x * sc, f16), x1 = float_to_h16(mv[r].y * sc, f16);
-        if (!tall) {
-          if (gi < m && col < n)
-            *reinterpret_cast<uint32_t*>(Xb + (long long)gi * n + col) = (uint32_t)x0 | ((uint32_t)x1 << 16);
-        } else {
-          Xt[(2 * cq) * XS + rg * RPW + r] = x0;
-          Xt[(2 * cq + 1) * XS + rg * RPW + r] = x1;
+        for (int s = 0; s < 4; ++s)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int gi = i0 + 8 * s + tq + 4 * hh;
+            if (gi < m && colok) {
+              const float4 x = v[s][hh];
+              uint2 w;
+              w.x = (uint32_t)float_to_h16(x.x * sc, f16) | ((uint32_t)float_to_h16(x.y * sc, f16) << 16);
+              w.y = (uint32_t)float_to_h16(x.z * sc, f16) | ((uint32_t)float_to_h16(x.w * sc, f16) << 16);
+              *reinterpret_cast<uint2*>(Xb + (long long)gi * n + cq) = w;
+            }
+          }
+      } else {
+        // X[j][i] = M[i][j]: through the warp's tile, then 32-byte row runs of X
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int ii = 8 * s + tq + 4 * hh;
+            const float4 x = v[s][hh];
+            Xt[warp][4 * g][ii] = float_to_h16(x.x * sc, f16);
+            Xt[warp][4 * g + 1][ii] = float_to_h16(x.y * sc, f16);
+            Xt[warp][4 * g + 2][ii] = float_to_h16(x.z * sc, f16);
+            Xt[warp][4 * g + 3][ii] = float_to_h16(x.w * sc, f16);
+          }
+        __syncwarp();
+        if (c0 + lane < n) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            if (i0 + 16 * q < m) {   // m % 16 == 0: 16-row runs are all in or all out
+              const uint4* src = reinterpret_cast<const uint4*>(&Xt[warp][lane][16 * q]);
+              uint4* dst = reinterpret_cast<uint4*>(Xb + (long long)(c0 + lane) * m + i0 + 16 * q);
+              dst[0] = src[0];
+              dst[1] = src[1];
+            }
+          }
         }
+        __syncwarp();
       }
     }
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      const float* prow = Ps + (rg * RPW + r) * KP;
-#pragma unroll
-      for (int l = 0; l < KP; l += 4) {
-        const float4 pv = *reinterpret_cast<const float4*>(prow + l);
-        acc[0][l] = fmaf(mv[r].x, pv.x, acc[0][l]);
-        acc[0][l + 1] = fmaf(mv[r].x, pv.y, acc[0][l + 1]);
-        acc[0][l + 2] = fmaf(mv[r].x, pv.z, acc[0][l + 2]);
-        acc[0][l + 3] = fmaf(mv[r].x, pv.w, acc[0][l + 3]);
-        acc[1][l] = fmaf(mv[r].y, pv.x, acc[1][l]);
-        acc[1][l + 1] = fmaf(mv[r].y, pv.y, acc[1][l + 1]);
-        acc[1][l + 2] = fmaf(mv[r].y, pv.z, acc[1][l + 2]);
-        acc[1][l + 3] = fmaf(mv[r].y, pv.w, acc[1][l + 3]);
-      }
-    }
-    if (Xb && tall) {
-      // X[j][i] = M[i][j]: rows of X are 256-byte runs of this chunk
-      for (int idx = t; idx < CB * (CH / 2); idx += kThreads) {
-        const int j = idx / (CH / 2), i2 = idx % (CH / 2);
-        const int gj = c0 + j, gi = i0 + 2 * i2;
-        if (gj < n && gi < m)
-          *reinterpret_cast<uint32_t*>(Xb + (long long)gj * m + gi) =
-              *reinterpret_cast<const uint32_t*>(Xt + j * XS + 2 * i2);
-      }
-    }
-    __syncthreads();
   }
-  // ordered reduction over the eight warps
-  float* red = smb;   // [CB][KP]
-  for (int w = (kThreads / 32) - 1; w >= 0; --w) {
+  // the four row warps of each half, added in order
+  for (int w = 3; w >= 0; --w) {
     if (rg == w) {
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
+      for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int l = 0; l < KP; ++l) {
-          float* slot = red + (2 * cq + c) * KP + l;
-          *slot = (w == (kThreads / 32) - 1) ? acc[c][l] : (*slot + acc[c][l]);
-        }
+        for (int nl = 0; nl < NL; ++nl)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            float* slot = &redR[32 * half + 4 * g + 2 * mt + (r >> 1)][8 * nl + 2 * tq + (r & 1)];
+            *slot = (w == 3) ? acc[mt][nl][r] : (*slot + acc[mt][nl][r]);
+          }
     }
     __syncthreads();
   }
   double* out = Rpart + ((long long)b * rsplit + split) * n * k;
-  for (int e = t; e < CB * k; e += kThreads) {
+  for (int e = t; e < 64 * k; e += kThreads) {
     const int cc = e / k, l = e % k;
-    if (c0 + cc < n) out[(long long)(c0 + cc) * k + l] = (double)red[cc * KP + l];
+    if (cbk * 64 + cc < n) out[(long long)(cbk * 64 + cc) * k + l] = (double)redR[cc][l];
   }
 }
 
+// R = the sum of the row splits (fp64, in order), and its residual fragments RB
+// over the padded nsl * 64 x kp range (zero outside n x k).
 __global__ void __launch_bounds__(kThreads) k_finalize_r(int n, int k, int rsplit,
                                                           const double* __restrict__ Rpart,
                                                           float* __restrict__ R,
+                                                          uint32_t* __restrict__ RB,
                                                           const int32_t* skip) {
   if (skip && *skip) return;
   const int b = blockIdx.y;
+  const int kp = factor_width(k), nsl = cdiv(n, 64);
   const long long e = (long long)blockIdx.x * kThreads + threadIdx.x;
-  if (e >= (long long)n * k) return;
-  double s = 0.0;
-  for (int p = 0; p < rsplit; ++p) s += Rpart[((long long)b * rsplit + p) * n * k + e];
-  R[(long long)b * n * k + e] = (float)s;
+  if (e >= (long long)nsl * 64 * kp) return;
+  const int j = (int)(e / kp), l = (int)(e % kp);
+  float f = 0.f;
+  if (j < n && l < k) {
+    double s = 0.0;
+    for (int p = 0; p < rsplit; ++p) s += Rpart[(((long long)b * rsplit + p) * n + j) * k + l];
+    f = (float)s;
+    R[((long long)b * n + j) * k + l] = f;
+  }
+  if (RB) {
+    const long long at = rb_at(b, nsl, kp >> 3, j, l);
+    const uint32_t hi = tf32_hi(f);
+    RB[at] = hi;
+    RB[at + 2] = tf32_lo(f, hi);
+  }
 }
 
 // ------------------------------------------------------------------ S7
-// One 128 x 128 grid block per CTA of 512 threads; thread (ty, tx) owns rows
-// ty + 32 i (i < 4) and columns 4 tx + {0..3}, 64 + 4 tx + {0..3}. The residual
-// x = M - sum_l P_il R_jl is formed in place (fp32 FMA), then the block's row and
-// column absolute maxima, then the codes q = rint(fp32(x / s) * 7).
-__global__ void __launch_bounds__(512, 2) k_residual_quant4(
+// One 128 x 128 grid block per CTA of 16 warps, laid out as in the rebuild:
+// warp w owns the rows 16 (w & 7) + {g, g + 8} and the columns 64 (w >> 3) +
+// 16 t .. + 15. The residual x = M - P R^T is formed in the C fragments: M is
+// loaded as the accumulator, A = -P and B = R^T are tf32 hi + lo pairs
+// (3xTF32, mma.m16n8k8; the raw P and R rows of the block are copied to shared
+// memory with cp.async while M loads). Then the block's row and column absolute maxima, and
+// the codes q = rint(fp32(x / s) * 7) with s = min(row max, column max). Since
+// |x| <= s, the quotient taken as z = x * fl(7 / s) is within 7 * 2^-22 of
+// fp32(x / s) * 7; where z lies at least 2^-16 away from a rounding tie, rint(z)
+// is the code, elsewhere the IEEE division decides.
+// FR: -P and R come as ready-made fragments (PA, RB); otherwise from raw rows.
+template <int KP, bool FR>   // KP = 0: no rank-k term
+__global__ void __launch_bounds__(kCT, 1) k_residual_quant4(
     int m, int n, int k, const float* __restrict__ X, const float* __restrict__ P,
-    const float* __restrict__ R, uint8_t* __restrict__ codes4, float* __restrict__ rscale,
-    float* __restrict__ cscale, const int32_t* skip) {
+    const float* __restrict__ R, const uint32_t* __restrict__ PA, const uint32_t* __restrict__ RB,
+    uint8_t* __restrict__ codes4, float* __restrict__ rscale, float* __restrict__ cscale,
+    const int32_t* skip) {
   if (skip && *skip) return;
+  constexpr int NL = KP / 8;
   const int bj = blockIdx.x, bi = blockIdx.y, b = blockIdx.z;
   const int nb = gridDim.x, mb = gridDim.y;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int g = lane >> 2, tq = lane & 3, rb = warp & 7, slab = warp >> 3;
   const int r0 = bi * kGrid, c0 = bj * kGrid;
-  const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
-  const int kk = (P && R) ? k : 0;
-  extern __shared__ __align__(16) float smq[];
-  float* Ps = smq;                 // [kk][128]
-  float* Rs = Ps + kk * kGrid;     // [kk][128]
-  __shared__ float cm[32][kGrid];
-  __shared__ float cmax[kGrid];
+  const int cb = c0 + 64 * slab + 16 * tq;   // n % 16 == 0: the run is all in or all out
+  const bool colok = cb < n;
+  extern __shared__ __align__(16) uint32_t smq[];
+  uint32_t* AF = smq;                      // [rb][ks][part][lane][4]: -P hi, lo
+  uint32_t* BF = smq + 8 * NL * 2 * 128;   // [slab][nt][ks][lane][4]: {b0, b1} hi, {b0, b1} lo
+  float* Praw = reinterpret_cast<float*>(BF + 2 * 8 * NL * 32 * 4);   // [128][k]
+  float* Rraw = Praw + kGrid * KP;                                     // [128][k]
+  const int nrows = min(kGrid, m - r0), ncols = min(kGrid, n - c0);   // multiples of 16
+  __shared__ __align__(16) float CM[64][kGrid];   // per (warp row block, g): column maxima of 2 rows
+  __shared__ float CQ[4][kGrid];
+  __shared__ float RM[2][kGrid];
+  __shared__ __align__(16) float smax_c[kGrid], r7c[kGrid];
+  __shared__ float smax_r[kGrid], r7r[kGrid];
 
-  float x[4][8];
+  float acc[8][4];   // C fragments: element (h, 2 nt + e) of the run at acc[nt][2 h + e]
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int gi = r0 + ty + 32 * i;
+  for (int h = 0; h < 2; ++h) {
+    const int gi = r0 + 16 * rb + g + 8 * h;
+    const bool ok = gi < m && colok;
+    const float4* src = reinterpret_cast<const float4*>(X + ((long long)b * m + gi) * n + cb);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int cb = c0 + 64 * h + 4 * tx;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (gi < m && cb < n) v = *reinterpret_cast<const float4*>(X + ((long long)b * m + gi) * n + cb);
-      x[i][4 * h] = v.x; x[i][4 * h + 1] = v.y; x[i][4 * h + 2] = v.z; x[i][4 * h + 3] = v.w;
+    for (int u = 0; u < 4; ++u) {
+      const float4 v = ok ? src[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+      acc[2 * u][2 * h] = v.x;
+      acc[2 * u][2 * h + 1] = v.y;
+      acc[2 * u + 1][2 * h] = v.z;
+      acc[2 * u + 1][2 * h + 1] = v.w;
     }
   }
-  for (int e = t; e < kGrid * kk; e += 512) {
-    const int rr = e / kk, l = e % kk;
-    const int gi = r0 + rr, gj = c0 + rr;
-    Ps[l * kGrid + rr] = (gi < m) ? P[((long long)b * m + gi) * kk + l] : 0.f;
-    Rs[l * kGrid + rr] = (gj < n) ? R[((long long)b * n + gj) * kk + l] : 0.f;
+  if constexpr (KP > 0 && FR) {
+    const int nsl = cdiv(n, 64), vs = min(2, nsl - 2 * bj), vb = min(8, (m >> 4) - r0 / 16);
+    constexpr int aw = NL * 2 * 128, bw = 8 * NL * 128;   // words per row block / slab
+    cp_async_block_zf(AF, PA + ((long long)b * (m >> 4) + r0 / 16) * aw, 8 * aw * 4, vb * aw * 4);
+    cp_async_block_zf(BF, RB + ((long long)b * nsl + 2 * bj) * bw, 2 * bw * 4, vs * bw * 4);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
   }
-  __syncthreads();
-  for (int l = 0; l < kk; ++l) {
-    const float4 ra = *reinterpret_cast<const float4*>(Rs + l * kGrid + 4 * tx);
-    const float4 rb = *reinterpret_cast<const float4*>(Rs + l * kGrid + 64 + 4 * tx);
-    const float rv[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+  if constexpr (KP > 0 && !FR) {
+    cp_async_block(Praw, P + ((long long)b * m + r0) * k, nrows * k * 4);
+    cp_async_block(Rraw, R + ((long long)b * n + c0) * k, ncols * k * 4);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+#pragma unroll 4
+    for (int it = 0; it < kGrid * KP / kCT; ++it) {
+      const int e = t + it * kCT;
+      const int il = e / KP, l = e % KP;
+      const float pv = (il < nrows && l < k) ? -Praw[il * k + l] : 0.f;
+      const float rv = (il < ncols && l < k) ? Rraw[il * k + l] : 0.f;
+      {
+        const int r = il & 15;
+        uint32_t* dst = AF + (((il >> 4) * NL + (l >> 3)) * 2) * 128 + (4 * (r & 7) + (l & 3)) * 4 +
+                        (r >> 3) + 2 * ((l & 7) >> 2);
+        const uint32_t hi = tf32_hi(pv);
+        dst[0] = hi;
+        dst[128] = tf32_lo(pv, hi);
+      }
+      {
+        const int jj = il & 63;
+        uint32_t* dst = BF + ((((il >> 6) * 8 + ((jj & 15) >> 1)) * NL + (l >> 3)) * 32 +
+                              4 * (2 * (jj >> 4) + (jj & 1)) + (l & 3)) * 4 + ((l & 7) >> 2);
+        const uint32_t hi = tf32_hi(rv);
+        dst[0] = hi;
+        dst[2] = tf32_lo(rv, hi);
+      }
+    }
+    __syncthreads();
+  }
+  if constexpr (KP > 0) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float pv = -Ps[l * kGrid + ty + 32 * i];
+    for (int ks = 0; ks < NL; ++ks) {
+      uint32_t ah[4], al[4];
+      {
+        const uint4 h4 = reinterpret_cast<const uint4*>(AF)[((rb * NL + ks) * 2) * 32 + lane];
+        const uint4 l4 = reinterpret_cast<const uint4*>(AF)[((rb * NL + ks) * 2 + 1) * 32 + lane];
+        ah[0] = h4.x; ah[1] = h4.y; ah[2] = h4.z; ah[3] = h4.w;
+        al[0] = l4.x; al[1] = l4.y; al[2] = l4.z; al[3] = l4.w;
+      }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) x[i][j] = fmaf(pv, rv[j], x[i][j]);
+      for (int nt = 0; nt < 8; ++nt) {
+        const uint4 bv = reinterpret_cast<const uint4*>(BF)[((slab * 8 + nt) * NL + ks) * 32 + lane];
+        mma_tf32(acc[nt], al, bv.x, bv.y);
+        mma_tf32(acc[nt], ah, bv.z, bv.w);
+        mma_tf32(acc[nt], ah, bv.x, bv.y);
+      }
     }
   }
-  // rows and columns outside the matrix are 0 (loaded as 0; their P, R rows are 0)
-  float cmx[8];
+  // rows outside the matrix are 0 (loaded as 0; their P rows are 0), as are columns
+  // row maxima: the thread's 16 columns, then the 4 lanes of the row (64 columns)
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int h = 0; h < 2; ++h) {
     float v = 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v = fmaxf(v, fabsf(x[i][j]));
-    cmx[j] = v;
+    for (int nt = 0; nt < 8; ++nt) v = fmaxf(v, fmaxf(fabsf(acc[nt][2 * h]), fabsf(acc[nt][2 * h + 1])));
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+    if (tq == 0) RM[slab][16 * rb + g + 8 * h] = v;
   }
+  // column maxima over the thread's two rows
+  {
+    float4* dst = reinterpret_cast<float4*>(&CM[8 * rb + g][64 * slab + 16 * tq]);
 #pragma unroll
-  for (int h = 0; h < 2; ++h)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) cm[ty][64 * h + 4 * tx + e] = cmx[4 * h + e];
-  __syncthreads();
-  if (t < kGrid) {
-    float v = 0.f;
-#pragma unroll 8
-    for (int g = 0; g < 32; ++g) v = fmaxf(v, cm[g][t]);
-    cmax[t] = v;
-    if (c0 + t < n) cscale[((long long)b * mb + bi) * n + c0 + t] = v;
-  }
-  __syncthreads();
-  float cs[8];
-#pragma unroll
-  for (int h = 0; h < 2; ++h)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) cs[4 * h + e] = cmax[64 * h + 4 * tx + e];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int gi = r0 + ty + 32 * i;
-    float rmx = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) rmx = fmaxf(rmx, fabsf(x[i][j]));
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) rmx = fmaxf(rmx, __shfl_xor_sync(0xffffffffu, rmx, o));
-    if (gi >= m) continue;
-    if (tx == 0) rscale[((long long)b * m + gi) * nb + bj] = rmx;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int cb = c0 + 64 * h + 4 * tx;
-      if (cb >= n) continue;
-      uint32_t packed = 0;
+    for (int u = 0; u < 4; ++u) {
+      float c4[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float sv = fminf(rmx, cs[4 * h + e]);
-        int q = 0;
-        if (sv > 0.f) {
-          q = (int)rintf(__fmul_rn(__fdiv_rn(x[i][4 * h + e], sv), 7.0f));
-          q = max(-7, min(7, q));
-        }
-        packed |= (uint32_t)(q & 0xF) << (4 * e);
+        const int nt = 2 * u + (e >> 1), ee = e & 1;
+        c4[e] = fmaxf(fabsf(acc[nt][ee]), fabsf(acc[nt][2 + ee]));
       }
-      *reinterpret_cast<uint16_t*>(codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2) = (uint16_t)packed;
+      dst[u] = make_float4(c4[0], c4[1], c4[2], c4[3]);
     }
+  }
+  __syncthreads();
+  {
+    const int c = t & (kGrid - 1), q = t >> 7;
+    float v = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v = fmaxf(v, CM[16 * q + i][c]);
+    CQ[q][c] = v;
+  }
+  __syncthreads();
+  if (t < kGrid) {
+    const float v = fmaxf(fmaxf(CQ[0][t], CQ[1][t]), fmaxf(CQ[2][t], CQ[3][t]));
+    smax_c[t] = v;
+    r7c[t] = v > 0.f ? __fdiv_rn(7.0f, v) : 0.f;
+    if (c0 + t < n) cscale[((long long)b * mb + bi) * n + c0 + t] = v;
+  } else if (t < 2 * kGrid) {
+    const int r = t - kGrid;
+    const float v = fmaxf(RM[0][r], RM[1][r]);
+    smax_r[r] = v;
+    r7r[r] = v > 0.f ? __fdiv_rn(7.0f, v) : 0.f;
+    if (r0 + r < m) rscale[((long long)b * m + r0 + r) * nb + bj] = v;
+  }
+  __syncthreads();
+  float rc7[16];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float4 v = *reinterpret_cast<const float4*>(&r7c[64 * slab + 16 * tq + 4 * u]);
+    rc7[4 * u] = v.x; rc7[4 * u + 1] = v.y; rc7[4 * u + 2] = v.z; rc7[4 * u + 3] = v.w;
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int rl = 16 * rb + g + 8 * h, gi = r0 + rl;
+    if (gi >= m || !colok) continue;
+    const float rr7 = r7r[rl];
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int ce = 0; ce < 16; ++ce) {
+      const float x = acc[ce >> 1][2 * h + (ce & 1)];
+      const float z = __fmul_rn(x, fmaxf(rr7, rc7[ce]));
+      const float zr = rintf(z);
+      int q;
+      if (fabsf(__fsub_rn(z, zr)) < 0.49998474f) {   // 0.5 - 2^-16
+        q = (int)zr;
+      } else {
+        const float sv = fminf(smax_r[rl], smax_c[64 * slab + 16 * tq + ce]);
+        q = sv > 0.f ? (int)rintf(__fmul_rn(__fdiv_rn(x, sv), 7.0f)) : 0;
+      }
+      q = max(-7, min(7, q));
+      w[ce >> 3] |= (uint32_t)(q & 0xF) << (4 * (ce & 7));
+    }
+    *reinterpret_cast<uint2*>(codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2) = make_uint2(w[0], w[1]);
   }
 }
 
@@ -852,26 +1304,45 @@ __global__ void __launch_bounds__(kThreads) k_cast_wide(int m, int n, const void
 }
 
 template <int KP>
-cudaError_t launch_backproject_t(int B, int m, int n, int k, const float* M, const float* P,
+cudaError_t launch_backproject_t(int B, int m, int n, int k, const float* M, const uint32_t* PB,
                                  const float* scale, void* X16, bool f16, double* Rpart,
-                                 float* R, const int32_t* skip, cudaStream_t s) {
+                                 float* R, uint32_t* RB, const int32_t* skip, cudaStream_t s) {
   const int rs = backproject_row_splits(B, m, n);
-  const size_t smem = (size_t)128 * KP * sizeof(float) + (size_t)64 * 130 * sizeof(uint16_t);
+  const size_t smem = (size_t)2 * 8 * 8 * 32 * sizeof(float4);
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_backproject<KP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_backproject<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   dim3 grid(cdiv(n, 64), rs, B);
-  k_backproject<KP><<<grid, kThreads, smem, s>>>(m, n, k, rs, M, P, scale,
-                                              static_cast<uint16_t*>(X16), f16 ? 1 : 0, Rpart,
-                                              skip);
+  k_backproject<KP><<<grid, kThreads, smem, s>>>(m, n, k, rs, M, PB, scale,
+                                                 static_cast<uint16_t*>(X16), f16 ? 1 : 0, Rpart,
+                                                 skip);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 g2(cdiv(n * k, kThreads), B);
-  k_finalize_r<<<g2, kThreads, 0, s>>>(n, k, rs, Rpart, R, skip);
+  dim3 g2((int)cdivll((long long)cdiv(n, 64) * 64 * KP, kThreads), B);
+  k_finalize_r<<<g2, kThreads, 0, s>>>(n, k, rs, Rpart, R, RB, skip);
+  return cudaGetLastError();
+}
+
+template <int KP, bool FR>
+cudaError_t launch_residual_t(int B, int m, int n, int k, const float* X, const float* P,
+                              const float* R, const uint32_t* PA, const uint32_t* RB,
+                              uint8_t* codes4, float* rscale, float* cscale, const int32_t* skip,
+                              cudaStream_t s) {
+  const size_t smem = (size_t)(2 * 8 * (KP / 8) * 2 * 128 + (FR ? 0 : 2 * kGrid * KP)) * sizeof(uint32_t);
+  static bool attr = false;
+  if (!attr && smem > 0) {
+    cudaError_t e = cudaFuncSetAttribute(k_residual_quant4<KP, FR>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid(cdiv(n, kGrid), cdiv(m, kGrid), B);
+  k_residual_quant4<KP, FR><<<grid, kCT, smem, s>>>(m, n, k, X, P, R, PA, RB, codes4, rscale, cscale,
+                                                    skip);
   return cudaGetLastError();
 }
 
@@ -892,12 +1363,26 @@ int gram_row_splits(int B, int m) {
 }
 int ns_prep_parts(int m, int n) { return (int)cdivll((long long)m * n, kPrepChunk); }
 
+FactorFrags factor_frag_words(int B, int m, int n, int k) {
+  const long long kp = factor_width(k), kb = kp < 16 ? 16 : kp;
+  const long long np = (long long)cdiv(n, 64) * 64, bm = (long long)B * m, bn = (long long)B * np;
+  FactorFrags f;
+  f.QF = bn * kp * 2;
+  f.RF = bn * kb / 2;
+  f.PF = bm * kb * 3 / 2;
+  f.PA = bm * kp * 2;
+  f.RB = bn * kp * 2;
+  f.PB = bm * kp * 2;
+  return f;
+}
+
 // ---------------------------------------------------------------- launchers
-cudaError_t launch_warm_start(int B, int n, int k, const int8_t* R8, const float* Rscale,
-                              const float* Rprev, uint64_t seed, float* Q, int* norm2_int,
-                              const int32_t* skip, cudaStream_t s) {
+cudaError_t launch_warm_start(int B, int m, int n, int k, const int8_t* R8, const float* Rscale,
+                              const int8_t* P8, const float* Pscale, const float* Rprev,
+                              uint64_t seed, float* Q, int* norm2_int, uint32_t* QF, uint32_t* RF,
+                              uint32_t* PF, const int32_t* skip, cudaStream_t s) {
   if (Rprev || !R8 || !norm2_int) {
-    k_warm_start<<<B, kThreads, 0, s>>>(n, k, R8, Rscale, Rprev, seed, Q, skip);
+    k_warm_start<<<B, kThreads, 0, s>>>(n, k, R8, Rscale, Rprev, seed, Q, QF, skip);
     return cudaGetLastError();
   }
   cudaError_t e = cudaMemsetAsync(norm2_int, 0, sizeof(int) * (size_t)B * k, s);
@@ -905,57 +1390,68 @@ cudaError_t launch_warm_start(int B, int n, int k, const int8_t* R8, const float
   k_colnorm_int<<<dim3(cdiv(n, kThreads), B), kThreads, 0, s>>>(n, k, R8, norm2_int, skip);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_warm_q<<<dim3((int)cdivll((long long)n * k, kThreads * 4), B), kThreads, 0, s>>>(
-      n, k, R8, Rscale, norm2_int, seed, Q, skip);
+  const int kb = kb16(factor_width(k));
+  const int nbq = (int)cdivll((long long)cdiv(n, 64) * 64 * kb, kThreads * 4);
+  const int nbp = (int)cdivll((long long)m * kb, kThreads * 4);
+  k_warm_q<<<dim3(nbq + nbp, B), kThreads, 0, s>>>(m, n, k, nbq, R8, Rscale, P8, Pscale, norm2_int,
+                                                   seed, Q, QF, reinterpret_cast<uint16_t*>(RF),
+                                                   reinterpret_cast<uint16_t*>(PF), skip);
   return cudaGetLastError();
 }
 
-template <int SRC, bool G32, int KP>
-cudaError_t launch_rebuild_t(dim3 grid, size_t smem, cudaStream_t s, int m, int n, int k,
+template <int SRC, bool G32, int KP, bool FR>
+cudaError_t launch_rebuild_t(dim3 grid, cudaStream_t s, int m, int n, int k,
                              const uint8_t* codes4, const float* rscale, const float* cscale,
                              const int8_t* P8, const float* Pscale, const int8_t* R8,
                              const float* Rscale, const float* Mprev32, float mu, const void* G,
-                             int gdt, const float* Q, float* M, double* norm2_part, float* Ppart,
+                             int gdt, const float* Q, const uint32_t* QF, const uint32_t* RF,
+                             const uint32_t* PF, float* M, double* norm2_part, float* Ppart,
                              int32_t* status) {
+  const size_t smem = (size_t)rebuild_smem_words(KP, SRC == SRC_STATE) * sizeof(uint32_t);
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_rebuild_proj<SRC, G32, KP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)((2 * kMaxK * kGrid + kMaxK * kRB) * sizeof(float)));
+    cudaError_t e = cudaFuncSetAttribute(k_rebuild_proj<SRC, G32, KP, FR>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  k_rebuild_proj<SRC, G32, KP><<<grid, kThreads, smem, s>>>(m, n, k, codes4, rscale, cscale, P8, Pscale,
-                                                        R8, Rscale, Mprev32, mu, G, gdt, Q, M,
-                                                        norm2_part, Ppart, status);
+  k_rebuild_proj<SRC, G32, KP, FR><<<grid, kRBT, smem, s>>>(m, n, k, codes4, rscale, cscale, P8,
+                                                            Pscale, R8, Rscale, Mprev32, mu, G, gdt,
+                                                            Q, QF, RF, PF, M, norm2_part, Ppart,
+                                                            status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4, const float* rscale,
                            const float* cscale, const int8_t* P8, const float* Pscale,
                            const int8_t* R8, const float* Rscale, const float* Mprev32, float mu,
-                           const void* G, int gdt, const float* Q, float* M, double* norm2_part,
+                           const void* G, int gdt, const float* Q, const uint32_t* QF,
+                           const uint32_t* RF, const uint32_t* PF, float* M, double* norm2_part,
                            float* Ppart, int32_t* status, cudaStream_t s) {
   dim3 grid(cdiv(n, kGrid), cdiv(m, kRB), B);
-  const int kp = k <= 8 ? 8 : (k <= 16 ? 16 : 32);
-  const int kk = codes4 ? kp : 0;
-  const int kq = Q ? kp : 0;
-  const size_t smem = (size_t)(kk * kRB + kk * kGrid + kq * kGrid) * sizeof(float);
+  const int kp = factor_width(k);
   const bool g32 = (G == nullptr) || gdt == GM_F32;
   const int src = codes4 ? SRC_STATE : (Mprev32 ? SRC_DENSE : SRC_ZERO);
-#define GM_RB(S, W, K) launch_rebuild_t<S, W, K>(grid, smem, s, m, n, k, codes4, rscale, cscale, P8, Pscale, \
-                                                 R8, Rscale, Mprev32, mu, G, gdt, Q, M, norm2_part, Ppart, status)
-#define GM_RBK(S, W) (kp == 8 ? GM_RB(S, W, 8) : (kp == 16 ? GM_RB(S, W, 16) : GM_RB(S, W, 32)))
-  if (src == SRC_STATE) return g32 ? GM_RBK(SRC_STATE, true) : GM_RBK(SRC_STATE, false);
-  if (src == SRC_DENSE) return g32 ? GM_RBK(SRC_DENSE, true) : GM_RBK(SRC_DENSE, false);
-  return g32 ? GM_RBK(SRC_ZERO, true) : GM_RBK(SRC_ZERO, false);
+  // ready-made fragments: QF whenever Q is given, RF and PF for the state source
+  const bool fr = (!Q || QF) && (src != SRC_STATE || (RF && PF)) && (Q || src == SRC_STATE);
+#define GM_RB(S, W, K, F) launch_rebuild_t<S, W, K, F>(grid, s, m, n, k, codes4, rscale, cscale, P8, \
+    Pscale, R8, Rscale, Mprev32, mu, G, gdt, Q, QF, RF, PF, M, norm2_part, Ppart, status)
+#define GM_RBK(S, W, F) (kp == 8 ? GM_RB(S, W, 8, F) : (kp == 16 ? GM_RB(S, W, 16, F) : GM_RB(S, W, 32, F)))
+  if (src == SRC_STATE) {
+    if (fr) return g32 ? GM_RBK(SRC_STATE, true, true) : GM_RBK(SRC_STATE, false, true);
+    return g32 ? GM_RBK(SRC_STATE, true, false) : GM_RBK(SRC_STATE, false, false);
+  }
+  if (!fr) return cudaErrorInvalidValue;   // dense / zero sources always come with QF
+  if (src == SRC_DENSE) return g32 ? GM_RBK(SRC_DENSE, true, true) : GM_RBK(SRC_DENSE, false, true);
+  return g32 ? GM_RBK(SRC_ZERO, true, true) : GM_RBK(SRC_ZERO, false, true);
 #undef GM_RBK
 #undef GM_RB
 }
 
 cudaError_t launch_orth(int B, int m, int k, int csplit, const float* Ppart, double* Ptil,
                         double* gram_part, double* Tmat, const double* norm2_part, int ntiles,
-                        float eps, float* scale, float* P, const int32_t* skip, cudaStream_t s) {
+                        float eps, float* scale, float* P, uint32_t* PB, uint32_t* PA,
+                        const int32_t* skip, cudaStream_t s) {
   const int rs = gram_row_splits(B, m);
   k_orth_gram<<<dim3(rs, B), kThreads, 0, s>>>(m, k, csplit, rs, Ppart, Ptil, gram_part, skip);
   cudaError_t e = cudaGetLastError();
@@ -963,33 +1459,37 @@ cudaError_t launch_orth(int B, int m, int k, int csplit, const float* Ppart, dou
   k_orth_chol<<<B, 32, 0, s>>>(k, rs, gram_part, Tmat, norm2_part, ntiles, eps, scale, skip);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int blocks = (int)cdivll((long long)m * k, kThreads * 4);
-  k_orth_apply<<<dim3(blocks, B), kThreads, 0, s>>>(m, k, Ptil, Tmat, P, skip);
+  const int kp = factor_width(k);
+  const int blocks = (int)cdivll((long long)m * kp, kThreads * 4);
+  k_orth_apply<<<dim3(blocks, B), kThreads, 0, s>>>(m, k, kp, Ptil, Tmat, P, PB, PA, skip);
   return cudaGetLastError();
 }
 
-cudaError_t launch_backproject(int B, int m, int n, int k, const float* M, const float* P,
+cudaError_t launch_backproject(int B, int m, int n, int k, const float* M, const uint32_t* PB,
                                const float* scale, void* X16, bool f16, double* Rpart, float* R,
-                               const int32_t* skip, cudaStream_t s) {
-  if (k <= 8) return launch_backproject_t<8>(B, m, n, k, M, P, scale, X16, f16, Rpart, R, skip, s);
-  if (k <= 16) return launch_backproject_t<16>(B, m, n, k, M, P, scale, X16, f16, Rpart, R, skip, s);
-  return launch_backproject_t<32>(B, m, n, k, M, P, scale, X16, f16, Rpart, R, skip, s);
+                               uint32_t* RB, const int32_t* skip, cudaStream_t s) {
+  const int kp = factor_width(k);
+  if (kp == 8) return launch_backproject_t<8>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, skip, s);
+  if (kp == 16) return launch_backproject_t<16>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, skip, s);
+  return launch_backproject_t<32>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, skip, s);
 }
 
 cudaError_t launch_residual_quant4(int B, int m, int n, int k, const float* X, const float* P,
-                                   const float* R, uint8_t* codes4, float* rscale, float* cscale,
+                                   const float* R, const uint32_t* PA, const uint32_t* RB,
+                                   uint8_t* codes4, float* rscale, float* cscale,
                                    const int32_t* skip, cudaStream_t s) {
-  dim3 grid(cdiv(n, kGrid), cdiv(m, kGrid), B);
-  const size_t smem = (size_t)2 * k * kGrid * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_residual_quant4, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(2 * kMaxK * kGrid * sizeof(float)));
-    if (e != cudaSuccess) return e;
-    attr = true;
+  if (k == 0 || !P || !R)
+    return launch_residual_t<0, false>(B, m, n, 0, X, nullptr, nullptr, nullptr, nullptr, codes4,
+                                       rscale, cscale, skip, s);
+  const int kp = factor_width(k);
+  if (PA && RB) {
+    if (kp == 8) return launch_residual_t<8, true>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, skip, s);
+    if (kp == 16) return launch_residual_t<16, true>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, skip, s);
+    return launch_residual_t<32, true>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, skip, s);
   }
-  k_residual_quant4<<<grid, 512, smem, s>>>(m, n, k, X, P, R, codes4, rscale, cscale, skip);
-  return cudaGetLastError();
+  if (kp == 8) return launch_residual_t<8, false>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, skip, s);
+  if (kp == 16) return launch_residual_t<16, false>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, skip, s);
+  return launch_residual_t<32, false>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, skip, s);
 }
 
 cudaError_t launch_quant8(int B, int rows0, int rows1, int k, const float* X0, int8_t* c0,

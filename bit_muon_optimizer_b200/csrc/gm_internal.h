@@ -8,39 +8,62 @@ namespace gm {
 
 // Column / row split counts of the power-iteration reductions. They depend
 // only on the problem shape, so the workspace layout is a pure function of it.
-int rebuild_row_blocks(int m);   // 64-row blocks of the fused rebuild / projection
+int rebuild_row_blocks(int m);   // 128-row blocks of the fused rebuild / projection
 int backproject_row_splits(int B, int m, int n);
 int gram_row_splits(int B, int m);
+// The factor width k rounded up to 8, 16 or 32: the depth of the codec kernels'
+// warp MMA fragments (components beyond k are zero).
+__host__ __device__ inline int factor_width(int k) { return k <= 8 ? 8 : (k <= 16 ? 16 : 32); }
+
+// 32-bit words of the fragment-ordered factor copies of B matrices (layouts in
+// gm_codec.cu): QF, RF, PF feed the rebuild / projection, PA, RB the residual,
+// PB the back-projection.
+struct FactorFrags {
+  long long QF, RF, PF, PA, RB, PB;
+};
+FactorFrags factor_frag_words(int B, int m, int n, int k);
 
 // ---- codec / power-iteration kernels (gm_codec.cu) ------------------------
-// Q from the stored 8-bit R (norm2_int: scratch int [B][k]) or from fp32 Rprev.
-cudaError_t launch_warm_start(int B, int n, int k, const int8_t* R8, const float* Rscale,
-                              const float* Rprev, uint64_t seed, float* Q, int* norm2_int,
-                              const int32_t* skip, cudaStream_t s);
+// Q from the stored 8-bit R (norm2_int: scratch int [B][k]) or from fp32 Rprev,
+// with its fragments QF; from the stored state also the R and P code fragments
+// RF, PF (P8, Pscale needed then).
+cudaError_t launch_warm_start(int B, int m, int n, int k, const int8_t* R8, const float* Rscale,
+                              const int8_t* P8, const float* Pscale, const float* Rprev,
+                              uint64_t seed, float* Q, int* norm2_int, uint32_t* QF, uint32_t* RF,
+                              uint32_t* PF, const int32_t* skip, cudaStream_t s);
 
 // M = mu * Mprev + G where Mprev is either the rebuilt state (codes4 != NULL)
 // or a dense fp32 matrix (Mprev32 != NULL) or zero; with Q != NULL also the
 // projection partials Ppart f32 [B][ceil(n/128)][m][k] (sum over one column
-// block each). norm2_part gets one fp64 partial |M|^2 per 64 x 128 tile
-// ([B][ceil(m/64)][ceil(n/128)]); status (nullable) gets GM_E_NONFINITE.
+// block each). norm2_part gets one fp64 partial |M|^2 per 128 x 128 tile
+// ([B][ceil(m/128)][ceil(n/128)]); status (nullable) gets GM_E_NONFINITE.
+// Data pointers are 16-byte aligned; m and n are multiples of 16. QF (with Q)
+// and RF, PF (with the state) are the ready-made fragments; NULL builds them in
+// each CTA from Q, R8, P8 (the dense and zero sources need QF).
 cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4,
                            const float* rscale, const float* cscale, const int8_t* P8,
                            const float* Pscale, const int8_t* R8, const float* Rscale,
                            const float* Mprev32, float mu, const void* G, int gdt, const float* Q,
-                           float* M, double* norm2_part, float* Ppart, int32_t* status,
-                           cudaStream_t s);
+                           const uint32_t* QF, const uint32_t* RF, const uint32_t* PF, float* M,
+                           double* norm2_part, float* Ppart, int32_t* status, cudaStream_t s);
 
+// P = orth(P~) (fp32 [B][m][k]) with its fragments PB (back-projection) and PA
+// (residual, nullable).
 cudaError_t launch_orth(int B, int m, int k, int csplit, const float* Ppart, double* Ptil,
                         double* gram_part, double* Tmat, const double* norm2_part, int ntiles,
-                        float eps, float* scale, float* P, const int32_t* skip, cudaStream_t s);
+                        float eps, float* scale, float* P, uint32_t* PB, uint32_t* PA,
+                        const int32_t* skip, cudaStream_t s);
 
-cudaError_t launch_backproject(int B, int m, int n, int k, const float* M, const float* P,
+// R = M^T P from PB, with its residual fragments RB (nullable).
+cudaError_t launch_backproject(int B, int m, int n, int k, const float* M, const uint32_t* PB,
                                const float* scale, void* X16, bool f16, double* Rpart,
-                               float* R, const int32_t* skip, cudaStream_t s);
+                               float* R, uint32_t* RB, const int32_t* skip, cudaStream_t s);
 
+// PA, RB: ready-made fragments of -P and R (both or neither; NULL stages P, R).
 cudaError_t launch_residual_quant4(int B, int m, int n, int k, const float* X, const float* P,
-                                   const float* R, uint8_t* codes4, float* rscale,
-                                   float* cscale, const int32_t* skip, cudaStream_t s);
+                                   const float* R, const uint32_t* PA, const uint32_t* RB,
+                                   uint8_t* codes4, float* rscale, float* cscale,
+                                   const int32_t* skip, cudaStream_t s);
 
 cudaError_t launch_quant8(int B, int rows0, int rows1, int k, const float* X0, int8_t* c0,
                           float* s0, const float* X1, int8_t* c1, float* s1,

@@ -5,6 +5,8 @@
  * All matrices are row-major and batch-contiguous: a call operates on B
  * same-shape matrices stored back to back (batch stride = rows * cols).
  * Shapes: m, n multiples of 16, 16 <= m, n <= 65536; top rank 1 <= k <= 32.
+ * Every device array pointer must be 16-byte aligned (the kernels move
+ * 16-byte vectors); a misaligned pointer returns GM_E_ARG.
  * The 4-bit grid uses fixed 128 x 128 blocks (ragged edge blocks allowed).
  *
  * Ownership: the caller allocates every buffer (typically torch tensors) and
