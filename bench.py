@@ -464,14 +464,15 @@ def run_ours(args, world, rank, local):
         e2e = {"value": e_ms / world, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h)}
 
-    # ---- our kernels launched per step: per group 10 codec kernels (column norms,
-    # warm start, rebuild + projection, three orthonormalisation kernels, back
-    # projection, its finalisation, 4-bit and 8-bit quantisation), the NS
-    # products, and the zero-padding copy when a dimension is not a multiple of 64
+    # ---- our kernels launched per step: per group 9 codec kernels (column norms,
+    # warm start with the factor fragments, rebuild + projection, three
+    # orthonormalisation kernels, back projection, its finalisation, the 4-bit
+    # quantisation with the 8-bit one folded in), the NS products, and the
+    # zero-padding copy when a dimension is not a multiple of 64
     launches = 0
     for g in w.groups:
         pad = int(min(g.m, g.n) % 64 != 0 or max(g.m, g.n) % 64 != 0)
-        launches += 10 + gm.ns_flops(ns_mode, g.m, g.n, w.T)[1] + pad
+        launches += 9 + gm.ns_flops(ns_mode, g.m, g.n, w.T)[1] + pad
     launches *= args.steps
 
     cpu = None

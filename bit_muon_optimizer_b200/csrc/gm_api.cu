@@ -72,7 +72,7 @@ StepLayout step_layout(int B, int m, int n, int k, int ns_mode, bool with_ns) {
   L.gram = take(Bz * L.rsplit_g * kz * kz * 8);
   L.Tm = take(Bz * kz * kz * 8);
   L.Rpart = take(Bz * L.rsplit_b * nz * kz * 8);
-  L.qnorm = take(Bz * kz * 4);
+  L.qnorm = take(Bz * kz * 4 * 3);   // column norms of R8, then the P and R column maxima
   const FactorFrags fw = factor_frag_words(B, m, n, k);
   L.QF = take((size_t)fw.QF * 4);
   L.RF = take((size_t)fw.RF * 4);
@@ -256,9 +256,9 @@ gm_status gm_momentum_powerit(int B, int m, int n, int k, float mu, const float*
   GM_CUDA(launch_rebuild(B, m, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                          M_prev, mu, G, gdt, Q, QF, nullptr, nullptr, M_out, norm2, Ppart, nullptr, s));
   GM_CUDA(launch_orth(B, m, k, L.csplit, Ppart, Ptil, gram, Tm, norm2, L.ntiles, 1e-7f, scale,
-                      P_out, PB, nullptr, nullptr, s));
+                      P_out, PB, nullptr, nullptr, nullptr, s));
   GM_CUDA(launch_backproject(B, m, n, k, M_out, PB, nullptr, nullptr, false, Rpart, R_out, nullptr,
-                             nullptr, s));
+                             nullptr, nullptr, s));
   return GM_OK;
 }
 
@@ -274,7 +274,8 @@ gm_status gm_grid_quant4(int B, int m, int n, int k, const float* X, const float
   GM_DEVICE();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   GM_CUDA(launch_residual_quant4(B, m, n, P ? k : 0, X, P, R, nullptr, nullptr, codes4, rscale,
-                                 cscale, nullptr, s));
+                                 cscale, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                 nullptr, s));
   return GM_OK;
 }
 
@@ -394,13 +395,14 @@ gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* prm, const g
                          st->R8, st->Rscale, nullptr, prm->mu, G, gdt, Q, QF, RF, PF, M, norm2, Ppart,
                          status, s));
   // worked step 4: P = orth(P~), R = M^T P
+  unsigned* PRmax = reinterpret_cast<unsigned*>(w + L.qnorm) + (size_t)B * k;
   GM_CUDA(launch_orth(B, m, k, L.csplit, Ppart, Ptil, gram, Tm, norm2, L.ntiles, prm->eps, scale,
-                      P, PB, PA, status, s));
-  GM_CUDA(launch_backproject(B, m, n, k, M, PB, scale, X, gramns, Rpart, R, RB, status, s));
+                      P, PB, PA, PRmax, status, s));
+  GM_CUDA(launch_backproject(B, m, n, k, M, PB, scale, X, gramns, Rpart, R, RB, PRmax + (size_t)B * k,
+                             status, s));
   // worked step 5: residual -> 4-bit grid codes; P, R -> 8-bit codes (state in place)
   GM_CUDA(launch_residual_quant4(B, m, n, k, M, P, R, PA, RB, st->codes4, st->rscale, st->cscale,
-                                 status, s));
-  GM_CUDA(launch_quant8(B, m, n, k, P, st->P8, st->Pscale, R, st->R8, st->Rscale, st->step, status, s));
+                                 PRmax, st->P8, st->Pscale, st->R8, st->Rscale, st->step, status, s));
   // worked step 6: O = NS(M_t); W <- W - eta (O + wd W) in the last product's epilogue
   NsOutput out{1, nullptr, 0, W, prm->eta, prm->wd};
   if (gramns)

@@ -357,7 +357,8 @@ enum RebuildSrc { SRC_STATE = 0, SRC_DENSE = 1, SRC_ZERO = 2 };
 // KP: the factor width k rounded up to 8, 16 or 32 (columns beyond k are zero).
 // FR: the fragments come ready-made (QF, RF, PF in global memory); otherwise the
 // CTA builds them from the raw factors.
-template <int SRC, bool G32, int KP, bool FR>
+// GDT: the gradient's dtype (GM_F32, GM_BF16 or GM_F16).
+template <int SRC, int GDT, int KP, bool FR>
 __global__ void __launch_bounds__(kRBT, 2) k_rebuild_proj(
     int m, int n, int k, const uint8_t* __restrict__ codes4, const float* __restrict__ rscale,
     const float* __restrict__ cscale, const int8_t* __restrict__ P8,
@@ -387,7 +388,7 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_proj(
   __shared__ float cfac[32];
   __shared__ double red[kRBT / 32];
   const long long mn = (long long)m * n;
-  const bool f16 = gdt == GM_F16;
+  constexpr bool G32 = GDT == GM_F32;
   const int cb = c0 + 64 * slab + 16 * tq;   // n % 16 == 0: the run is all in or all out
   const bool colok = cb < n;
 
@@ -554,7 +555,7 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_proj(
         const int ce = 2 * nt + e;
         float gv;
         if constexpr (G32) gv = gf[h][ce];
-        else gv = h16_to_float((uint16_t)(gw[h][ce >> 1] >> (16 * (ce & 1))), f16);
+        else gv = h16_to_float((uint16_t)(gw[h][ce >> 1] >> (16 * (ce & 1))), GDT == GM_F16);
         float mp = 0.f;
         if constexpr (ST) {
           const uint32_t word = ce < 8 ? cw[h].x : cw[h].y;
@@ -565,7 +566,7 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_proj(
         }
         const float o = ok[h] ? __fadd_rn(__fmul_rn(mu, mp), gv) : 0.f;
         acc[nt][2 * h + e] = o;   // keep M for the projection
-        bad |= !isfinite(o);
+        bad |= !(fabsf(o) <= 3.402823466e38f);   // NaN or infinite
         nsq = fmaf(o, o, nsq);
       }
     }
@@ -676,132 +677,138 @@ __global__ void __launch_bounds__(kThreads) k_orth_gram(int m, int k, int csplit
   }
 }
 
-// (b) Cholesky of the Gram with dead-column exclusion; T = L^-T; NS scale.
+// (b) Cholesky G = L L^T of the Gram (fp64) with dead-column exclusion, right
+// looking: lane i holds row i of G in registers; after step j it holds L[i][j] in
+// slot j and has subtracted L[i][j] L[c][j] from its slots c > j (L[c][j] by
+// shuffle from lane c), in ascending j as the textbook left-looking sums do.
+// Writes L below the diagonal and the reciprocal diagonal on it (0 for a dead
+// column) for the forward substitution in (c); NS scale 1 / (|M_t|_F + eps).
 __global__ void __launch_bounds__(32) k_orth_chol(int k, int rsplit, const double* __restrict__ gram_part,
-                                                   double* __restrict__ Tmat,
+                                                   double* __restrict__ Lmat,
                                                    const double* __restrict__ norm2_part, int ntiles,
                                                    float eps, float* __restrict__ scale,
                                                    const int32_t* skip) {
   if (skip && *skip) return;
   const int b = blockIdx.x, lane = threadIdx.x;
-  __shared__ double G[kMaxK][kMaxK + 1];
-  __shared__ double L[kMaxK][kMaxK + 1];
-  __shared__ double Li[kMaxK][kMaxK + 1];
-  __shared__ int live[kMaxK];
-  {
-    // element e = lane + 32 u of the k x k Gram, summed over the row splits in order;
-    // the loads of all u are independent and issued together
-    constexpr int U = kMaxK * kMaxK / 32;
-    double acc[U];
+  constexpr unsigned kAll = 0xffffffffu;
+  // row `lane` of the Gram, summed over the row splits in order
+  double g[kMaxK];
 #pragma unroll
-    for (int u = 0; u < U; ++u) acc[u] = 0.0;
-    const double* gp = gram_part + (long long)b * rsplit * k * k;
+  for (int c = 0; c < kMaxK; ++c) g[c] = 0.0;
+  if (lane < k) {
+    const double* gp = gram_part + (long long)b * rsplit * k * k + (long long)lane * k;
+#pragma unroll 2
     for (int p = 0; p < rsplit; ++p) {
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int e = lane + 32 * u;
-        if (e < k * k) acc[u] += gp[(long long)p * k * k + e];
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int e = lane + 32 * u;
-      if (e < k * k) {
-        G[e / k][e % k] = acc[u];
-        L[e / k][e % k] = 0.0;
-        Li[e / k][e % k] = 0.0;
-      }
+      for (int c = 0; c < kMaxK; ++c)
+        if (c < k) g[c] += gp[(long long)p * k * k + c];
     }
   }
-  // |M_t|^2 from the rebuild's partials: lane-strided sums, then a fixed shuffle tree
-  double ns2 = 0.0;
-  for (int p = lane; p < ntiles; p += 32) ns2 += norm2_part[(long long)b * ntiles + p];
+  // |M_t|^2 from the rebuild's partials: eight lane-strided chains, then a fixed tree
+  double nsq[8];
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) ns2 += __shfl_xor_sync(0xffffffffu, ns2, off);
-  __syncwarp();
+  for (int u = 0; u < 8; ++u) nsq[u] = 0.0;
+  const double* np = norm2_part + (long long)b * ntiles;
+  for (int p0 = 0; p0 < ntiles; p0 += 256) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int p = p0 + 32 * u + lane;
+      if (p < ntiles) nsq[u] += np[p];
+    }
+  }
+  double ns2 = ((nsq[0] + nsq[1]) + (nsq[2] + nsq[3])) + ((nsq[4] + nsq[5]) + (nsq[6] + nsq[7]));
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ns2 += __shfl_xor_sync(kAll, ns2, off);
+  // dead-column tolerance: (1e-6 * max column norm)^2
   double maxn2 = 0.0;
-  for (int l = 0; l < k; ++l) maxn2 = fmax(maxn2, G[l][l]);
-  const double tol2 = 1e-12 * maxn2;   // (1e-6 * max column norm)^2
-  for (int j = 0; j < k; ++j) {
-    double d = G[j][j];
-    for (int l = 0; l < j; ++l) d -= L[j][l] * L[j][l];   // dead columns hold zeros
+#pragma unroll
+  for (int c = 0; c < kMaxK; ++c)
+    if (c == lane) maxn2 = g[c];
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) maxn2 = fmax(maxn2, __shfl_xor_sync(kAll, maxn2, off));
+  const double tol2 = 1e-12 * maxn2;
+  double rinv = 0.0;
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    if (j >= k) break;
+    const double d = __shfl_sync(kAll, g[j], j);
     const bool alive = (d > tol2) && (d > 0.0);
     const double ljj = alive ? sqrt(d) : 0.0;
-    __syncwarp();
-    if (lane == 0) { live[j] = alive; L[j][j] = ljj; }
-    for (int i = j + 1 + lane; i < k; i += 32) {
-      double v = 0.0;
-      if (alive) {
-        v = G[i][j];
-        for (int l = 0; l < j; ++l) v -= L[i][l] * L[j][l];
-        v /= ljj;
-      }
-      L[i][j] = v;
-    }
-    __syncwarp();
-  }
-  // Li = L^-1 on the live columns (forward substitution, one column per lane).
-  for (int c = lane; c < k; c += 32) {
-    if (!live[c]) continue;
-    for (int i = c; i < k; ++i) {
-      if (!live[i]) continue;
-      double v = (i == c) ? 1.0 : 0.0;
-      for (int l = c; l < i; ++l) v -= L[i][l] * Li[l][c];
-      Li[i][c] = v / L[i][i];
+    const double rj = alive ? 1.0 / ljj : 0.0;
+    const double lij = lane > j ? g[j] * rj : (lane == j ? ljj : 0.0);
+    if (lane >= j) g[j] = lij;
+    if (lane == j) rinv = rj;
+#pragma unroll
+    for (int c = j + 1; c < kMaxK; ++c) {
+      const double lcj = __shfl_sync(kAll, lij, c);
+      if (lane >= c && c < k) g[c] = fma(-lij, lcj, g[c]);
     }
   }
-  __syncwarp();
-  for (int e = lane; e < k * k; e += 32) {
-    const int a = e / k, c = e % k;
-    Tmat[(long long)b * k * k + e] = Li[c][a];   // T = L^-T
+  if (lane < k) {
+    double* out = Lmat + ((long long)b * k + lane) * k;
+#pragma unroll
+    for (int c = 0; c < kMaxK; ++c)
+      if (c < k) out[c] = c < lane ? g[c] : (c == lane ? rinv : 0.0);
   }
   if (lane == 0 && scale) scale[b] = (float)(1.0 / (sqrt(ns2) + (double)eps));
 }
 
-// (c) P = P~ T (fp64), stored fp32, and as fragments: PB for the back-projection
-// (PB[b][i / 8][l / 8][lane][4] = {hi(P[8 s + t][l]), hi(P[8 s + t + 4][l]), lo, lo},
-// lane = 4 (l % 8) + t) and PA (-P) for the residual; zero for k <= l < kp.
-__global__ void __launch_bounds__(kThreads) k_orth_apply(int m, int k, int kp,
-                                                          const double* __restrict__ Ptil,
-                                                          const double* __restrict__ Tmat,
+// (c) P = P~ L^-T by forward substitution (fp64), one row of P per thread:
+// P[i][l] = (P~[i][l] - sum_{a<l} P[i][a] L[l][a]) / L[l][l], zero for a dead
+// column. Stored fp32 and as fragments: PB for the back-projection (PB[b][i / 8]
+// [l / 8][lane][4] = {hi(P[8 s + t][l]), hi(P[8 s + t + 4][l]), lo, lo}, lane =
+// 4 (l % 8) + t) and PA (-P) for the residual (nullable); zero for k <= l < KP.
+// The column absolute maxima of P go to Pmax (fp32 bits, atomicMax; nullable).
+template <int KP>
+__global__ void __launch_bounds__(kThreads) k_orth_apply(int m, int k, const double* __restrict__ Ptil,
+                                                          const double* __restrict__ Lmat,
                                                           float* __restrict__ P,
                                                           uint32_t* __restrict__ PB,
                                                           uint32_t* __restrict__ PA,
+                                                          unsigned* __restrict__ Pmax,
                                                           const int32_t* skip) {
   if (skip && *skip) return;
-  const int b = blockIdx.y, t = threadIdx.x;
-  __shared__ double Ts[kMaxK][kMaxK];
-  for (int e = t; e < k * k; e += kThreads) Ts[e / k][e % k] = Tmat[(long long)b * k * k + e];
+  const int b = blockIdx.y, t = threadIdx.x, lane = t & 31;
+  __shared__ double Ls[KP][KP];   // L below the diagonal, 1 / L[l][l] on it
+  __shared__ unsigned cmax[KP];
+  for (int e = t; e < KP * KP; e += kThreads) {
+    const int l = e / KP, a = e % KP;
+    Ls[l][a] = (a < k && l < k) ? Lmat[((long long)b * k + l) * k + a] : 0.0;
+  }
+  if (t < KP) cmax[t] = 0u;
   __syncthreads();
-  const long long base = (long long)blockIdx.x * kThreads * 4;
-  for (int s = 0; s < 4; ++s) {
-    const long long e = base + s * kThreads + t;
-    if (e >= (long long)m * kp) break;
-    const long long i = e / kp;
-    const int l = (int)(e % kp);
-    float f = 0.f;
-    if (l < k) {
-      const double* row = Ptil + ((long long)b * m + i) * k;
-      double v = 0.0;
-      for (int a = 0; a <= l; ++a) v = fma(row[a], Ts[a][l], v);   // T upper triangular
-      f = (float)v;
-      P[((long long)b * m + i) * k + l] = f;
-    }
+  const int i = blockIdx.x * kThreads + t;
+  const bool in = i < m;
+  double row[KP];
+#pragma unroll
+  for (int a = 0; a < KP; ++a) row[a] = (in && a < k) ? Ptil[((long long)b * m + i) * k + a] : 0.0;
+#pragma unroll
+  for (int l = 0; l < KP; ++l) {
+    double v = row[l];
+#pragma unroll
+    for (int a = 0; a < l; ++a) v = fma(-row[a], Ls[l][a], v);   // row[a] holds P[i][a] by now
+    row[l] = v * Ls[l][l];
+    const float f = (float)row[l];   // 0 outside the matrix
+    const unsigned mx = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(f)));
+    if (lane == 0 && mx) atomicMax(&cmax[l], mx);
+    if (!in) continue;
+    if (l < k) P[((long long)b * m + i) * k + l] = f;
     if (PB) {
-      const int c = (int)(i & 7);
-      uint32_t* dst = PB + ((((long long)b * (m >> 3) + (i >> 3)) * (kp >> 3) + (l >> 3)) * 32 +
-                            4 * (l & 7) + (c & 3)) * 4 + (c >> 2);
+      uint32_t* dst = PB + ((((long long)b * (m >> 3) + (i >> 3)) * (KP / 8) + (l >> 3)) * 32 +
+                            4 * (l & 7) + (i & 3)) * 4 + ((i & 7) >> 2);
       const uint32_t hi = tf32_hi(f);
       dst[0] = hi;
       dst[2] = tf32_lo(f, hi);
     }
     if (PA) {
-      const long long at = pa_at(b, m >> 4, kp >> 3, (int)i, l);
+      const long long at = pa_at(b, m >> 4, KP / 8, i, l);
       const uint32_t hi = tf32_hi(-f);
       PA[at] = hi;
       PA[at + 128] = tf32_lo(-f, hi);
     }
   }
+  __syncthreads();
+  if (Pmax && t < k && cmax[t]) atomicMax(&Pmax[b * k + t], cmax[t]);
 }
 
 // ------------------------------------------------------------------ S5
@@ -982,24 +989,33 @@ __global__ void __launch_bounds__(kThreads, 2) k_backproject(int m, int n, int k
 
 // R = the sum of the row splits (fp64, in order), and its residual fragments RB
 // over the padded nsl * 64 x kp range (zero outside n x k).
+// The column absolute maxima of R go to Rmax (fp32 bits, atomicMax; nullable).
 __global__ void __launch_bounds__(kThreads) k_finalize_r(int n, int k, int rsplit,
                                                           const double* __restrict__ Rpart,
                                                           float* __restrict__ R,
                                                           uint32_t* __restrict__ RB,
+                                                          unsigned* __restrict__ Rmax,
                                                           const int32_t* skip) {
   if (skip && *skip) return;
-  const int b = blockIdx.y;
+  const int b = blockIdx.y, t = threadIdx.x;
   const int kp = factor_width(k), nsl = cdiv(n, 64);
-  const long long e = (long long)blockIdx.x * kThreads + threadIdx.x;
-  if (e >= (long long)nsl * 64 * kp) return;
+  __shared__ unsigned cmax[kMaxK];
+  if (t < kMaxK) cmax[t] = 0u;
+  __syncthreads();
+  const long long e = (long long)blockIdx.x * kThreads + t;
+  const bool in = e < (long long)nsl * 64 * kp;
   const int j = (int)(e / kp), l = (int)(e % kp);
   float f = 0.f;
-  if (j < n && l < k) {
+  if (in && j < n && l < k) {
     double s = 0.0;
     for (int p = 0; p < rsplit; ++p) s += Rpart[(((long long)b * rsplit + p) * n + j) * k + l];
     f = (float)s;
     R[((long long)b * n + j) * k + l] = f;
+    if (f != 0.f) atomicMax(&cmax[l], __float_as_uint(fabsf(f)));
   }
+  __syncthreads();
+  if (Rmax && t < k && cmax[t]) atomicMax(&Rmax[b * k + t], cmax[t]);
+  if (!in) return;
   if (RB) {
     const long long at = rb_at(b, nsl, kp >> 3, j, l);
     const uint32_t hi = tf32_hi(f);
@@ -1020,12 +1036,41 @@ __global__ void __launch_bounds__(kThreads) k_finalize_r(int n, int k, int rspli
 // fp32(x / s) * 7; where z lies at least 2^-16 away from a rounding tie, rint(z)
 // is the code, elsewhere the IEEE division decides.
 // FR: -P and R come as ready-made fragments (PA, RB); otherwise from raw rows.
+// Q8 (given with the P and R column maxima): the CTAs of block column 0 also
+// write the 8-bit codes of their 128 rows of P, those of block row 0 of their
+// 128 rows of R (q = rint(fp32(x / s) * 127), s the column absolute maximum;
+// the worked step's step 5), and block (0, 0) the scales and the step count.
+struct Quant8Out {
+  const unsigned* Pmax;
+  const unsigned* Rmax;
+  int8_t* P8;
+  float* Pscale;
+  int8_t* R8;
+  float* Rscale;
+  int64_t* step;
+};
+
+// q = rint(fp32(x / s) * 127) for |x| <= s. Taken as rint(x * fl(127 / s)) where
+// that product lies at least 2^-12 away from a rounding tie (the two differ by at
+// most 127 * 2^-22), else by the IEEE division.
+__device__ __forceinline__ int8_t code8(float x, float s, float r127) {
+  if (!(s > 0.f)) return 0;
+  const float z = __fmul_rn(x, r127), zr = rintf(z);
+  int q;
+  if (fabsf(__fsub_rn(z, zr)) < 0.49975586f)   // 0.5 - 2^-12
+    q = (int)zr;
+  else
+    q = (int)rintf(__fmul_rn(__fdiv_rn(x, s), 127.0f));
+  return (int8_t)max(-127, min(127, q));
+}
+constexpr int kQ8PerThread = kGrid * kMaxK / kCT;   // P or R values per thread, 128 rows
+
 template <int KP, bool FR>   // KP = 0: no rank-k term
 __global__ void __launch_bounds__(kCT, 1) k_residual_quant4(
     int m, int n, int k, const float* __restrict__ X, const float* __restrict__ P,
     const float* __restrict__ R, const uint32_t* __restrict__ PA, const uint32_t* __restrict__ RB,
     uint8_t* __restrict__ codes4, float* __restrict__ rscale, float* __restrict__ cscale,
-    const int32_t* skip) {
+    Quant8Out q8, const int32_t* skip) {
   if (skip && *skip) return;
   constexpr int NL = KP / 8;
   const int bj = blockIdx.x, bi = blockIdx.y, b = blockIdx.z;
@@ -1046,6 +1091,26 @@ __global__ void __launch_bounds__(kCT, 1) k_residual_quant4(
   __shared__ float RM[2][kGrid];
   __shared__ __align__(16) float smax_c[kGrid], r7c[kGrid];
   __shared__ float smax_r[kGrid], r7r[kGrid];
+  __shared__ float s8[2][kMaxK], r127[2][kMaxK];
+  // 8-bit codes of P (block column 0) and R (block row 0): values loaded up front
+  const bool doP = q8.Pmax && bj == 0, doR = q8.Pmax && bi == 0;
+  float pq[kQ8PerThread], rq[kQ8PerThread];
+  if (doP) {
+    const float* src = P + ((long long)b * m + r0) * k;
+#pragma unroll
+    for (int u = 0; u < kQ8PerThread; ++u) pq[u] = t + u * kCT < nrows * k ? src[t + u * kCT] : 0.f;
+  }
+  if (doR) {
+    const float* src = R + ((long long)b * n + c0) * k;
+#pragma unroll
+    for (int u = 0; u < kQ8PerThread; ++u) rq[u] = t + u * kCT < ncols * k ? src[t + u * kCT] : 0.f;
+  }
+  if (q8.Pmax && t < 2 * kMaxK) {
+    const int w = t / kMaxK, l = t % kMaxK;
+    const float sv = l < k ? __uint_as_float((w ? q8.Rmax : q8.Pmax)[b * k + l]) : 0.f;
+    s8[w][l] = sv;
+    r127[w][l] = sv > 0.f ? __fdiv_rn(127.0f, sv) : 0.f;
+  }
 
   float acc[8][4];   // C fragments: element (h, 2 nt + e) of the run at acc[nt][2 h + e]
 #pragma unroll
@@ -1197,6 +1262,27 @@ __global__ void __launch_bounds__(kCT, 1) k_residual_quant4(
     }
     *reinterpret_cast<uint2*>(codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2) = make_uint2(w[0], w[1]);
   }
+  if (doP) {
+    int8_t* dst = q8.P8 + ((long long)b * m + r0) * k;
+#pragma unroll
+    for (int u = 0; u < kQ8PerThread; ++u) {
+      const int e = t + u * kCT;
+      if (e < nrows * k) dst[e] = code8(pq[u], s8[0][e % k], r127[0][e % k]);
+    }
+  }
+  if (doR) {
+    int8_t* dst = q8.R8 + ((long long)b * n + c0) * k;
+#pragma unroll
+    for (int u = 0; u < kQ8PerThread; ++u) {
+      const int e = t + u * kCT;
+      if (e < ncols * k) dst[e] = code8(rq[u], s8[1][e % k], r127[1][e % k]);
+    }
+  }
+  if (doP && bi == 0 && t < k) {
+    q8.Pscale[b * k + t] = s8[0][t];
+    q8.Rscale[b * k + t] = s8[1][t];
+  }
+  if (q8.step && b == 0 && bi == 0 && bj == 0 && t == 0) *q8.step += 1;
 }
 
 // ------------------------------------------------------------------ S6
@@ -1306,7 +1392,8 @@ __global__ void __launch_bounds__(kThreads) k_cast_wide(int m, int n, const void
 template <int KP>
 cudaError_t launch_backproject_t(int B, int m, int n, int k, const float* M, const uint32_t* PB,
                                  const float* scale, void* X16, bool f16, double* Rpart,
-                                 float* R, uint32_t* RB, const int32_t* skip, cudaStream_t s) {
+                                 float* R, uint32_t* RB, unsigned* Rmax, const int32_t* skip,
+                                 cudaStream_t s) {
   const int rs = backproject_row_splits(B, m, n);
   const size_t smem = (size_t)2 * 8 * 8 * 32 * sizeof(float4);
   static bool attr = false;
@@ -1323,15 +1410,15 @@ cudaError_t launch_backproject_t(int B, int m, int n, int k, const float* M, con
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g2((int)cdivll((long long)cdiv(n, 64) * 64 * KP, kThreads), B);
-  k_finalize_r<<<g2, kThreads, 0, s>>>(n, k, rs, Rpart, R, RB, skip);
+  k_finalize_r<<<g2, kThreads, 0, s>>>(n, k, rs, Rpart, R, RB, Rmax, skip);
   return cudaGetLastError();
 }
 
 template <int KP, bool FR>
 cudaError_t launch_residual_t(int B, int m, int n, int k, const float* X, const float* P,
                               const float* R, const uint32_t* PA, const uint32_t* RB,
-                              uint8_t* codes4, float* rscale, float* cscale, const int32_t* skip,
-                              cudaStream_t s) {
+                              uint8_t* codes4, float* rscale, float* cscale, const Quant8Out& q8,
+                              const int32_t* skip, cudaStream_t s) {
   const size_t smem = (size_t)(2 * 8 * (KP / 8) * 2 * 128 + (FR ? 0 : 2 * kGrid * KP)) * sizeof(uint32_t);
   static bool attr = false;
   if (!attr && smem > 0) {
@@ -1342,7 +1429,7 @@ cudaError_t launch_residual_t(int B, int m, int n, int k, const float* X, const 
   }
   dim3 grid(cdiv(n, kGrid), cdiv(m, kGrid), B);
   k_residual_quant4<KP, FR><<<grid, kCT, smem, s>>>(m, n, k, X, P, R, PA, RB, codes4, rscale, cscale,
-                                                    skip);
+                                                    q8, skip);
   return cudaGetLastError();
 }
 
@@ -1358,8 +1445,8 @@ int backproject_row_splits(int B, int m, int n) {
   return max(1, min(rs, nchunks));
 }
 int gram_row_splits(int B, int m) {
-  int rs = cdiv(kTargetCtas, B);
-  return max(1, min(rs, cdiv(m, 256)));
+  const int rs = cdiv(2 * kTargetCtas, B);   // about four CTAs per SM, 128 rows or more each
+  return max(1, min(rs, cdiv(m, 128)));
 }
 int ns_prep_parts(int m, int n) { return (int)cdivll((long long)m * n, kPrepChunk); }
 
@@ -1385,7 +1472,7 @@ cudaError_t launch_warm_start(int B, int m, int n, int k, const int8_t* R8, cons
     k_warm_start<<<B, kThreads, 0, s>>>(n, k, R8, Rscale, Rprev, seed, Q, QF, skip);
     return cudaGetLastError();
   }
-  cudaError_t e = cudaMemsetAsync(norm2_int, 0, sizeof(int) * (size_t)B * k, s);
+  cudaError_t e = cudaMemsetAsync(norm2_int, 0, sizeof(int) * (size_t)3 * B * k, s);
   if (e != cudaSuccess) return e;
   k_colnorm_int<<<dim3(cdiv(n, kThreads), B), kThreads, 0, s>>>(n, k, R8, norm2_int, skip);
   e = cudaGetLastError();
@@ -1399,7 +1486,7 @@ cudaError_t launch_warm_start(int B, int m, int n, int k, const int8_t* R8, cons
   return cudaGetLastError();
 }
 
-template <int SRC, bool G32, int KP, bool FR>
+template <int SRC, int GDT, int KP, bool FR>
 cudaError_t launch_rebuild_t(dim3 grid, cudaStream_t s, int m, int n, int k,
                              const uint8_t* codes4, const float* rscale, const float* cscale,
                              const int8_t* P8, const float* Pscale, const int8_t* R8,
@@ -1410,12 +1497,12 @@ cudaError_t launch_rebuild_t(dim3 grid, cudaStream_t s, int m, int n, int k,
   const size_t smem = (size_t)rebuild_smem_words(KP, SRC == SRC_STATE) * sizeof(uint32_t);
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_rebuild_proj<SRC, G32, KP, FR>,
+    cudaError_t e = cudaFuncSetAttribute(k_rebuild_proj<SRC, GDT, KP, FR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  k_rebuild_proj<SRC, G32, KP, FR><<<grid, kRBT, smem, s>>>(m, n, k, codes4, rscale, cscale, P8,
+  k_rebuild_proj<SRC, GDT, KP, FR><<<grid, kRBT, smem, s>>>(m, n, k, codes4, rscale, cscale, P8,
                                                             Pscale, R8, Rscale, Mprev32, mu, G, gdt,
                                                             Q, QF, RF, PF, M, norm2_part, Ppart,
                                                             status);
@@ -1430,66 +1517,69 @@ cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4, co
                            float* Ppart, int32_t* status, cudaStream_t s) {
   dim3 grid(cdiv(n, kGrid), cdiv(m, kRB), B);
   const int kp = factor_width(k);
-  const bool g32 = (G == nullptr) || gdt == GM_F32;
+  const int gd = (G == nullptr) ? GM_F32 : gdt;
   const int src = codes4 ? SRC_STATE : (Mprev32 ? SRC_DENSE : SRC_ZERO);
   // ready-made fragments: QF whenever Q is given, RF and PF for the state source
   const bool fr = (!Q || QF) && (src != SRC_STATE || (RF && PF)) && (Q || src == SRC_STATE);
 #define GM_RB(S, W, K, F) launch_rebuild_t<S, W, K, F>(grid, s, m, n, k, codes4, rscale, cscale, P8, \
     Pscale, R8, Rscale, Mprev32, mu, G, gdt, Q, QF, RF, PF, M, norm2_part, Ppart, status)
 #define GM_RBK(S, W, F) (kp == 8 ? GM_RB(S, W, 8, F) : (kp == 16 ? GM_RB(S, W, 16, F) : GM_RB(S, W, 32, F)))
-  if (src == SRC_STATE) {
-    if (fr) return g32 ? GM_RBK(SRC_STATE, true, true) : GM_RBK(SRC_STATE, false, true);
-    return g32 ? GM_RBK(SRC_STATE, true, false) : GM_RBK(SRC_STATE, false, false);
+#define GM_RBD(S, F) (gd == GM_F32 ? GM_RBK(S, GM_F32, F) : (gd == GM_BF16 ? GM_RBK(S, GM_BF16, F) : GM_RBK(S, GM_F16, F)))
+  if (src == SRC_STATE) {   // the raw-factor path serves the rebuild-only call (no gradient)
+    if (fr) return GM_RBD(SRC_STATE, true);
+    return gd == GM_F32 ? GM_RBK(SRC_STATE, GM_F32, false) : cudaErrorInvalidValue;
   }
   if (!fr) return cudaErrorInvalidValue;   // dense / zero sources always come with QF
-  if (src == SRC_DENSE) return g32 ? GM_RBK(SRC_DENSE, true, true) : GM_RBK(SRC_DENSE, false, true);
-  return g32 ? GM_RBK(SRC_ZERO, true, true) : GM_RBK(SRC_ZERO, false, true);
+  if (src == SRC_DENSE) return GM_RBD(SRC_DENSE, true);
+  return GM_RBD(SRC_ZERO, true);
+#undef GM_RBD
 #undef GM_RBK
 #undef GM_RB
 }
 
 cudaError_t launch_orth(int B, int m, int k, int csplit, const float* Ppart, double* Ptil,
-                        double* gram_part, double* Tmat, const double* norm2_part, int ntiles,
+                        double* gram_part, double* Lmat, const double* norm2_part, int ntiles,
                         float eps, float* scale, float* P, uint32_t* PB, uint32_t* PA,
-                        const int32_t* skip, cudaStream_t s) {
+                        unsigned* Pmax, const int32_t* skip, cudaStream_t s) {
   const int rs = gram_row_splits(B, m);
   k_orth_gram<<<dim3(rs, B), kThreads, 0, s>>>(m, k, csplit, rs, Ppart, Ptil, gram_part, skip);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_orth_chol<<<B, 32, 0, s>>>(k, rs, gram_part, Tmat, norm2_part, ntiles, eps, scale, skip);
+  k_orth_chol<<<B, 32, 0, s>>>(k, rs, gram_part, Lmat, norm2_part, ntiles, eps, scale, skip);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int kp = factor_width(k);
-  const int blocks = (int)cdivll((long long)m * kp, kThreads * 4);
-  k_orth_apply<<<dim3(blocks, B), kThreads, 0, s>>>(m, k, kp, Ptil, Tmat, P, PB, PA, skip);
+  const dim3 grid(cdiv(m, kThreads), B);
+  if (kp == 8) k_orth_apply<8><<<grid, kThreads, 0, s>>>(m, k, Ptil, Lmat, P, PB, PA, Pmax, skip);
+  else if (kp == 16) k_orth_apply<16><<<grid, kThreads, 0, s>>>(m, k, Ptil, Lmat, P, PB, PA, Pmax, skip);
+  else k_orth_apply<32><<<grid, kThreads, 0, s>>>(m, k, Ptil, Lmat, P, PB, PA, Pmax, skip);
   return cudaGetLastError();
 }
 
 cudaError_t launch_backproject(int B, int m, int n, int k, const float* M, const uint32_t* PB,
                                const float* scale, void* X16, bool f16, double* Rpart, float* R,
-                               uint32_t* RB, const int32_t* skip, cudaStream_t s) {
+                               uint32_t* RB, unsigned* Rmax, const int32_t* skip, cudaStream_t s) {
   const int kp = factor_width(k);
-  if (kp == 8) return launch_backproject_t<8>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, skip, s);
-  if (kp == 16) return launch_backproject_t<16>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, skip, s);
-  return launch_backproject_t<32>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, skip, s);
+  if (kp == 8) return launch_backproject_t<8>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, Rmax, skip, s);
+  if (kp == 16) return launch_backproject_t<16>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, Rmax, skip, s);
+  return launch_backproject_t<32>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, Rmax, skip, s);
 }
 
 cudaError_t launch_residual_quant4(int B, int m, int n, int k, const float* X, const float* P,
                                    const float* R, const uint32_t* PA, const uint32_t* RB,
                                    uint8_t* codes4, float* rscale, float* cscale,
-                                   const int32_t* skip, cudaStream_t s) {
+                                   const unsigned* PRmax, int8_t* P8, float* Pscale, int8_t* R8,
+                                   float* Rscale, int64_t* step, const int32_t* skip,
+                                   cudaStream_t s) {
+  const Quant8Out q8{PRmax, PRmax ? PRmax + (size_t)B * k : nullptr, P8, Pscale, R8, Rscale, step};
   if (k == 0 || !P || !R)
     return launch_residual_t<0, false>(B, m, n, 0, X, nullptr, nullptr, nullptr, nullptr, codes4,
-                                       rscale, cscale, skip, s);
+                                       rscale, cscale, Quant8Out{}, skip, s);
   const int kp = factor_width(k);
-  if (PA && RB) {
-    if (kp == 8) return launch_residual_t<8, true>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, skip, s);
-    if (kp == 16) return launch_residual_t<16, true>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, skip, s);
-    return launch_residual_t<32, true>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, skip, s);
-  }
-  if (kp == 8) return launch_residual_t<8, false>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, skip, s);
-  if (kp == 16) return launch_residual_t<16, false>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, skip, s);
-  return launch_residual_t<32, false>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, skip, s);
+#define GM_RQ(K, F) launch_residual_t<K, F>(B, m, n, k, X, P, R, PA, RB, codes4, rscale, cscale, q8, skip, s)
+  if (PA && RB) return kp == 8 ? GM_RQ(8, true) : (kp == 16 ? GM_RQ(16, true) : GM_RQ(32, true));
+  return kp == 8 ? GM_RQ(8, false) : (kp == 16 ? GM_RQ(16, false) : GM_RQ(32, false));
+#undef GM_RQ
 }
 
 cudaError_t launch_quant8(int B, int rows0, int rows1, int k, const float* X0, int8_t* c0,

@@ -24,7 +24,9 @@ struct FactorFrags {
 FactorFrags factor_frag_words(int B, int m, int n, int k);
 
 // ---- codec / power-iteration kernels (gm_codec.cu) ------------------------
-// Q from the stored 8-bit R (norm2_int: scratch int [B][k]) or from fp32 Rprev,
+// Q from the stored 8-bit R (norm2_int: scratch int [3][B][k], zeroed here: the
+// column norms, then the P and R column maxima of launch_orth / launch_backproject)
+// or from fp32 Rprev,
 // with its fragments QF; from the stored state also the R and P code fragments
 // RF, PF (P8, Pscale needed then).
 cudaError_t launch_warm_start(int B, int m, int n, int k, const int8_t* R8, const float* Rscale,
@@ -49,21 +51,27 @@ cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4,
 
 // P = orth(P~) (fp32 [B][m][k]) with its fragments PB (back-projection) and PA
 // (residual, nullable).
+// Pmax (nullable): the column absolute maxima of P (fp32 bits, atomicMax into zeroed words).
 cudaError_t launch_orth(int B, int m, int k, int csplit, const float* Ppart, double* Ptil,
-                        double* gram_part, double* Tmat, const double* norm2_part, int ntiles,
+                        double* gram_part, double* Lmat, const double* norm2_part, int ntiles,
                         float eps, float* scale, float* P, uint32_t* PB, uint32_t* PA,
-                        const int32_t* skip, cudaStream_t s);
+                        unsigned* Pmax, const int32_t* skip, cudaStream_t s);
 
 // R = M^T P from PB, with its residual fragments RB (nullable).
 cudaError_t launch_backproject(int B, int m, int n, int k, const float* M, const uint32_t* PB,
                                const float* scale, void* X16, bool f16, double* Rpart,
-                               float* R, uint32_t* RB, const int32_t* skip, cudaStream_t s);
+                               float* R, uint32_t* RB, unsigned* Rmax, const int32_t* skip,
+                               cudaStream_t s);
 
 // PA, RB: ready-made fragments of -P and R (both or neither; NULL stages P, R).
+// PRmax (nullable): the P then R column maxima; with it the kernel also writes the
+// 8-bit state P8, Pscale, R8, Rscale and increments step.
 cudaError_t launch_residual_quant4(int B, int m, int n, int k, const float* X, const float* P,
                                    const float* R, const uint32_t* PA, const uint32_t* RB,
                                    uint8_t* codes4, float* rscale, float* cscale,
-                                   const int32_t* skip, cudaStream_t s);
+                                   const unsigned* PRmax, int8_t* P8, float* Pscale, int8_t* R8,
+                                   float* Rscale, int64_t* step, const int32_t* skip,
+                                   cudaStream_t s);
 
 cudaError_t launch_quant8(int B, int rows0, int rows1, int k, const float* X0, int8_t* c0,
                           float* s0, const float* X1, int8_t* c1, float* s1,
