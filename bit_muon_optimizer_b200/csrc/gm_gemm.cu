@@ -734,8 +734,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           mbar_arrive(smem_u32(&buf_free[b]));
         }
       }
-      // shared memory stays allocated until the bulk stores have completed
-      bulk_wait_all();
+      // every slab's bulk store has read its staging by now (waited above); the
+      // writes themselves complete with the grid, before any dependent launch reads them
     }
   } else {
     // ---------------- epilogue warps (both CTAs, 128 TMEM lanes each)
