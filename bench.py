@@ -208,8 +208,8 @@ GRAD_POOL = 6   # distinct gradient buffers per group, used cyclically step afte
 # LLaMA-130M set, standard NS), from the ncu capture summarised in
 # profiles/k_gemm_llama130m.md; reported only while gm_gemm.cu is the source
 # that capture measured.
-GEMM_TRAFFIC = {"config": 2, "ns": "standard", "bytes_per_launch": 88.63e6,
-                "source_sha256": "e243e07758da123732a4cd7b3bc5875ee9f181e121419ee0443d32d2c79d87be"}
+GEMM_TRAFFIC = {"config": 2, "ns": "standard", "bytes_per_launch": 87.56e6,
+                "source_sha256": "aa52586b7c8ef53cef64f66392279f880c35c449ce72813d6b82ec7d5a190d0a"}
 
 
 def gemm_traffic(config: int, ns: str):
