@@ -46,20 +46,24 @@ def _singular_values(X):
     return ev.clamp_min(0).sqrt()
 
 
-# (workload, shape group): LLaMA-1.1B 5632 x 2048 (tall) and 256 x 2048;
-# Qwen2.5-7B 3584 x 18944 (wide, the largest matrices) and 512 x 3584.
-FULL = [(3, 2), (3, 1), (4, 3), (4, 1)]
+# (workload, shape group, NS form): LLaMA-1.1B 5632 x 2048 (tall) and 256 x 2048;
+# Qwen2.5-7B 3584 x 18944 (wide, the largest matrices) and 512 x 3584; the Gram NS
+# form on the MoE experts (1408 x 2048, k = 32, Student-t gradients) and on
+# LLaMA-130M's 2048 x 768.
+FULL = [(3, 2, "standard"), (3, 1, "standard"), (4, 3, "standard"), (4, 1, "standard"),
+        (5, 0, "gram"), (2, 1, "gram")]
 
 
-@pytest.mark.parametrize("cid,gi", FULL)
-def test_full_size_group_step(cuda_lib, cid, gi):
+@pytest.mark.parametrize("cid,gi,ns", FULL)
+def test_full_size_group_step(cuda_lib, cid, gi, ns):
     gm = cuda_lib
     w = WL.WORKLOADS[cid]
     g = w.groups[gi]
     B, m, n, k = g.count, g.m, g.n, w.k
     base = w.group_base(gi)
     sample = (0, B - 1)
-    step = gm.GraspStep(B, m, n, k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=gm.GM_NS_STANDARD,
+    nsmode = gm.GM_NS_GRAM if ns == "gram" else gm.GM_NS_STANDARD
+    step = gm.GraspStep(B, m, n, k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=nsmode,
                         seed=w.seed, device=DEV)
     st = gm.GraspState.zeros(B, m, n, k, DEV)
     W = torch.empty((B, m, n), dtype=torch.float32, device=DEV)
@@ -95,12 +99,12 @@ def test_full_size_group_step(cuda_lib, cid, gi):
         want = O.quintic_scalar(s_in / s_in.pow(2).sum().sqrt(), T=w.T).sort().values
         got = _singular_values((W0[b] - W[b]) / w.eta)
         err = (got - want).abs()
-        print(f"\n[{w.name} {m}x{n} b={b}] sigma(O) in [{float(got.min()):.4f}, "
+        print(f"\n[{w.name} {m}x{n} {ns} b={b}] sigma(O) in [{float(got.min()):.4f}, "
               f"{float(got.max()):.4f}], |sorted diff| max {float(err.max()):.4f} "
               f"mean {float(err.mean()):.5f}")
-        # bf16 stores each product with unit roundoff u = 2^-8; over T steps the
-        # errors add and the quintic's slope (<= a = 3.4445 near 0) can amplify
-        # them for the smallest singular values, so single values may move by a
-        # few u; on the flat part of the band, where most values sit, the mean
-        # stays well below u.
+        # bf16 (standard NS) stores each product with unit roundoff u = 2^-8, fp16
+        # (Gram NS) with 2^-11; over T steps the errors add and the quintic's
+        # slope (<= a = 3.4445 near 0) can amplify them for the smallest singular
+        # values, so single values may move by a few u; on the flat part of the
+        # band, where most values sit, the mean stays well below u.
         assert float(err.max()) <= 0.06 and float(err.mean()) <= 0.004

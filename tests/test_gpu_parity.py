@@ -221,7 +221,7 @@ def _to_oracle_state(st, b):
                         int(st.step.item()))
 
 
-def _run_teacher_forced(gm, cid, group, B, steps, ns):
+def _run_teacher_forced(gm, cid, group, B, steps, ns, gdtype=None):
     w = WL.WORKLOADS[cid]
     g = w.groups[group]
     m, n, k = g.m, g.n, w.k
@@ -233,6 +233,8 @@ def _run_teacher_forced(gm, cid, group, B, steps, ns):
     W = torch.stack([WL.initial_weight(w, base + b, m, n) for b in range(B)]).to(DEV)
     for t in range(1, steps + 1):
         G = torch.stack([WL.gradient(w, base + b, t, m, n) for b in range(B)]).to(DEV)
+        if gdtype is not None:
+            G = G.to(gdtype)
         before = [_to_oracle_state(st, b) for b in range(B)]
         W0 = W.clone()
         step(st, W, G)
@@ -271,6 +273,11 @@ def test_grasp_step_llama130m_shapes(cuda_lib, ns):
     """2048 x 768 (tall) and 768 x 2048 gradients in bf16, k = 16."""
     _run_teacher_forced(cuda_lib, 2, 1, 2, 2, ns)
     _run_teacher_forced(cuda_lib, 2, 2, 1, 2, ns)
+
+
+def test_grasp_step_fp16_gradients(cuda_lib):
+    """fp16 gradients (the third gradient dtype of the C ABI), 768 x 2048, 2 steps."""
+    _run_teacher_forced(cuda_lib, 2, 2, 2, 2, "standard", gdtype=torch.float16)
 
 
 def test_grasp_step_nonfinite_leaves_state_and_weights(cuda_lib):
