@@ -625,6 +625,274 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_proj(
   }
 }
 
+// Pipelined form of the same pass for ready-made fragments: a CTA owns one
+// 128-column block and walks up to kRebuildTiles 64-row tiles of it (rows
+// blockIdx.y, + gridDim.y, ...). Q's and R's fragments are copied once; every
+// input of tile i + 1 (its P fragments, gradient, codes, row and column scales,
+// dense M_{t-1}) streams into the other of two shared-memory stages with
+// cp.async while tile i is multiplied, so the memory latency of one tile hides
+// behind the work of the previous one. Each thread copies its own gradient (and
+// M_{t-1}) chunks and reads only those back; the shared inputs become visible at
+// the barrier after the copies complete. The arithmetic per element is the one
+// of k_rebuild_proj.
+constexpr int kRebuildTiles = 4;
+
+__host__ __device__ constexpr int pipe_g_chunks(int GDT) { return GDT == GM_F32 ? 8 : 4; }
+// words of one stage: P fragments, codes (64 rows x 64 B), column and row scales,
+// the per-thread gradient chunks, the per-thread dense M_{t-1} chunks
+__host__ __device__ constexpr int pipe_stage_words(int SRC, int GDT, int KP) {
+  return (SRC == SRC_STATE ? 4 * (kb16(KP) / 16) * 3 * 128 + 64 * 16 + kGrid + kRB : 0) +
+         pipe_g_chunks(GDT) * kRBT * 4 + (SRC == SRC_DENSE ? 8 * kRBT * 4 : 0);
+}
+__host__ __device__ constexpr int pipe_smem_words(int SRC, int GDT, int KP) {
+  return 2 * 8 * (KP / 8) * 32 * 4 + (SRC == SRC_STATE ? 2 * 8 * (kb16(KP) / 16) * 32 * 2 : 0) +
+         2 * pipe_stage_words(SRC, GDT, KP);
+}
+
+template <int SRC, int GDT, int KP>
+__global__ void __launch_bounds__(kRBT, 2) k_rebuild_pipe(
+    int m, int n, int k, const uint8_t* __restrict__ codes4, const float* __restrict__ rscale,
+    const float* __restrict__ cscale, const float* __restrict__ Mprev, float mu,
+    const void* __restrict__ G, const uint32_t* __restrict__ QFg, const uint32_t* __restrict__ RFg,
+    const uint32_t* __restrict__ PFg, float* __restrict__ M, double* __restrict__ norm2_part,
+    float* __restrict__ Ppart, int32_t* status) {
+  constexpr bool ST = SRC == SRC_STATE, DN = SRC == SRC_DENSE, G32 = GDT == GM_F32;
+  constexpr int NL = KP / 8, KSB = kb16(KP) / 16, GCH = pipe_g_chunks(GDT);
+  constexpr int QW = 8 * NL * 128, RW = 8 * KSB * 64, PW = KSB * 3 * 128;   // words per slab / block
+  constexpr int SW = pipe_stage_words(SRC, GDT, KP);
+  const int bj = blockIdx.x, b = blockIdx.z;
+  const int nb = gridDim.x, nrb = cdiv(m, kRB), mbg = cdiv(m, kGrid);
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int g = lane >> 2, tq = lane & 3, rb = warp & 3, slab = warp >> 2;
+  const int c0 = bj * kGrid;
+  const int cb = c0 + 64 * slab + 16 * tq;   // n % 16 == 0: the run is all in or all out
+  const bool colok = cb < n;
+  const int ncols = min(kGrid, n - c0);
+  const int nsl = cdiv(n, 64), vs = min(2, nsl - 2 * bj);
+  const long long mn = (long long)m * n;
+  extern __shared__ __align__(16) uint32_t smp[];
+  uint32_t* QF = smp;                          // [slab][s][NL][lane][4]
+  uint32_t* RF = QF + 2 * QW;                  // [slab][nt][KSB][lane][2]
+  uint32_t* stg = RF + (ST ? 2 * RW : 0);      // two stages of SW words
+  __shared__ float deq4[16];
+  __shared__ double red[kRBT / 32];
+
+  // stage layout
+  auto PFs = [&](int s) { return stg + s * SW; };                                  // [rb][KSB][part][lane][4]
+  auto CDs = [&](int s) { return stg + s * SW + (ST ? 4 * PW : 0); };              // codes [64][16 words]
+  auto CSs = [&](int s) { return reinterpret_cast<float*>(CDs(s) + (ST ? 64 * 16 : 0)); };   // [128]
+  auto RSs = [&](int s) { return CSs(s) + (ST ? kGrid : 0); };                     // [64]
+  auto GSs = [&](int s) { return reinterpret_cast<uint4*>(RSs(s) + (ST ? kRB : 0)); };        // [GCH][256]
+  auto MPs = [&](int s) { return GSs(s) + GCH * kRBT; };                           // [8][256]
+
+  auto issue = [&](int rbi, int s) {
+    const int r0 = rbi * kRB;
+    if constexpr (ST) {
+      const int vb = min(kRB / 16, (m >> 4) - r0 / 16);
+      cp_async_block_zf(PFs(s), PFg + ((long long)b * (m >> 4) + r0 / 16) * PW, (kRB / 16) * PW * 4, vb * PW * 4);
+      {   // codes: 64 rows x 64 bytes, one 16-byte chunk (32 columns) per thread; a
+          // chunk half past the last column (ncols % 32 == 16) copies 8 bytes
+        const int r = t >> 2, ch = t & 3, gi = r0 + r;
+        const int nbytes = gi < m ? max(0, min(16, (ncols - 32 * ch) / 2)) : 0;
+        const uint32_t sa = (uint32_t)__cvta_generic_to_shared(CDs(s) + r * 16 + ch * 4);
+        const uint8_t* src = nbytes ? codes4 + ((long long)b * m + gi) * (n / 2) + c0 / 2 + 16 * ch : codes4;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sa), "l"(src), "r"(nbytes)
+                     : "memory");
+      }
+      if (t < kGrid / 4) {   // column scales of the grid-block row
+        const bool ok = 4 * t < ncols;
+        cp_async16(CSs(s) + 4 * t, ok ? cscale + ((long long)b * mbg + r0 / kGrid) * n + c0 + 4 * t : cscale, ok);
+      }
+      if (t < kRB) {   // row scales (stride ceil(n / 128) in memory)
+        const int gi = r0 + t;
+        const uint32_t sa = (uint32_t)__cvta_generic_to_shared(RSs(s) + t);
+        if (gi < m)
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sa),
+                       "l"(rscale + ((long long)b * m + gi) * nb + bj) : "memory");
+        else
+          RSs(s)[t] = 0.f;
+      }
+    }
+    // this thread's gradient (and dense M_{t-1}) chunks: rows g, g + 8 of its warp's 16
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int gi = r0 + 16 * rb + g + 8 * h;
+      const bool ok = gi < m && colok && G;
+      const long long base = (long long)b * mn + (long long)gi * n + cb;
+#pragma unroll
+      for (int u = 0; u < GCH / 2; ++u) {
+        const void* src = ok ? (G32 ? (const void*)(static_cast<const float*>(G) + base + 4 * u)
+                                    : (const void*)(static_cast<const uint16_t*>(G) + base + 8 * u))
+                             : G ? G : (const void*)M;
+        cp_async16(&GSs(s)[(h * (GCH / 2) + u) * kRBT + t], src, ok);
+      }
+      if constexpr (DN) {
+        const bool okm = gi < m && colok;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          cp_async16(&MPs(s)[(h * 4 + u) * kRBT + t], okm ? Mprev + base + 4 * u : Mprev, okm);
+      }
+    }
+  };
+
+  const int first = blockIdx.y, stride = gridDim.y;
+  int ntl = 0;
+  for (int rbi = first; rbi < nrb && ntl < kRebuildTiles; rbi += stride) ++ntl;
+  // Q and R fragments of the column block, and the first tile's stage
+  cp_async_block_zf(QF, QFg + ((long long)b * nsl + 2 * bj) * QW, 2 * QW * 4, vs * QW * 4);
+  if constexpr (ST) cp_async_block_zf(RF, RFg + ((long long)b * nsl + 2 * bj) * RW, 2 * RW * 4, vs * RW * 4);
+  if (t < 16) deq4[t] = __fdiv_rn((float)((t & 8) ? t - 16 : t), 7.0f);
+  if (ntl > 0) issue(first, 0);
+  cp_async_commit();
+
+  bool bad = false;
+  for (int i = 0; i < ntl; ++i) {
+    const int s = i & 1, rbi = first + i * stride, r0 = rbi * kRB;
+    __syncthreads();   // every thread is done with stage s ^ 1 (tile i - 1)
+    if (i + 1 < ntl) {
+      issue(rbi + stride, s ^ 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();   // stage s (and the fragments) complete and visible
+
+    // rank-k rebuild P^ R^T
+    float acc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    if constexpr (ST) {
+      const uint32_t* PF = PFs(s);
+#pragma unroll
+      for (int ks = 0; ks < KSB; ++ks) {
+        uint32_t a[3][4];
+#pragma unroll
+        for (int p = 0; p < 3; ++p) {
+          const uint4 v = reinterpret_cast<const uint4*>(PF)[((rb * KSB + ks) * 3 + p) * 32 + lane];
+          a[p][0] = v.x; a[p][1] = v.y; a[p][2] = v.z; a[p][3] = v.w;
+        }
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          const uint2 bv = reinterpret_cast<const uint2*>(RF)[((slab * 8 + nt) * KSB + ks) * 32 + lane];
+          mma_bf16(acc[nt], a[2], bv.x, bv.y);
+          mma_bf16(acc[nt], a[1], bv.x, bv.y);
+          mma_bf16(acc[nt], a[0], bv.x, bv.y);
+        }
+      }
+    }
+
+    // M = mu M_prev + G
+    float cs[16];
+    if constexpr (ST) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 v = reinterpret_cast<const float4*>(CSs(s))[16 * slab + 4 * tq + u];
+        cs[4 * u] = v.x; cs[4 * u + 1] = v.y; cs[4 * u + 2] = v.z; cs[4 * u + 3] = v.w;
+      }
+    }
+    float nsq = 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int rl = 16 * rb + g + 8 * h, gi = r0 + rl;
+      const bool ok = gi < m && colok;
+      uint32_t gw[GCH / 2 * 4];
+#pragma unroll
+      for (int u = 0; u < GCH / 2; ++u) {
+        const uint4 v = GSs(s)[(h * (GCH / 2) + u) * kRBT + t];
+        gw[4 * u] = v.x; gw[4 * u + 1] = v.y; gw[4 * u + 2] = v.z; gw[4 * u + 3] = v.w;
+      }
+      uint2 cw = make_uint2(0u, 0u);
+      float rsc = 0.f;
+      if constexpr (ST) {
+        cw = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(CDs(s)) + rl * 64 + 32 * slab + 8 * tq);
+        rsc = RSs(s)[rl];
+      }
+      float mpv[16];
+      if constexpr (DN) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 v = reinterpret_cast<const float4*>(MPs(s))[(h * 4 + u) * kRBT + t];
+          mpv[4 * u] = v.x; mpv[4 * u + 1] = v.y; mpv[4 * u + 2] = v.z; mpv[4 * u + 3] = v.w;
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int ce = 2 * nt + e;
+          float gv;
+          if constexpr (G32) gv = __uint_as_float(gw[ce]);
+          else gv = h16_to_float((uint16_t)(gw[ce >> 1] >> (16 * (ce & 1))), GDT == GM_F16);
+          float mp = 0.f;
+          if constexpr (ST) {
+            const uint32_t word = ce < 8 ? cw.x : cw.y;
+            const float sc = fminf(rsc, cs[ce]);
+            mp = __fadd_rn(__fmul_rn(deq4[(word >> (4 * (ce & 7))) & 0xF], sc), acc[nt][2 * h + e]);
+          } else if constexpr (DN) {
+            mp = mpv[ce];
+          }
+          const float o = ok ? __fadd_rn(__fmul_rn(mu, mp), gv) : 0.f;
+          acc[nt][2 * h + e] = o;
+          bad |= !(fabsf(o) <= 3.402823466e38f);
+          nsq = fmaf(o, o, nsq);
+        }
+      }
+      if (ok) {
+        float4* dst = reinterpret_cast<float4*>(M + (long long)b * mn + (long long)gi * n + cb);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          dst[u] = make_float4(acc[2 * u][2 * h], acc[2 * u][2 * h + 1], acc[2 * u + 1][2 * h],
+                               acc[2 * u + 1][2 * h + 1]);
+      }
+    }
+    const double tot = block_sum_d((double)nsq, red);
+    if (t == 0 && norm2_part) norm2_part[((long long)b * nrb + rbi) * nb + bj] = tot;
+
+    // projection partials; the slab reduction reuses this stage's gradient slots
+    float pt[NL][4];
+#pragma unroll
+    for (int nl = 0; nl < NL; ++nl) pt[nl][0] = pt[nl][1] = pt[nl][2] = pt[nl][3] = 0.f;
+#pragma unroll
+    for (int sk = 0; sk < 8; ++sk) {
+      const float xa[4] = {acc[sk][0], acc[sk][2], acc[sk][1], acc[sk][3]};
+      uint32_t ah[4], al[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        ah[j] = tf32_hi(xa[j]);
+        al[j] = tf32_lo(xa[j], ah[j]);
+      }
+#pragma unroll
+      for (int nl = 0; nl < NL; ++nl) {
+        const uint4 qv = reinterpret_cast<const uint4*>(QF)[((slab * 8 + sk) * NL + nl) * 32 + lane];
+        mma_tf32(pt[nl], al, qv.x, qv.y);
+        mma_tf32(pt[nl], ah, qv.z, qv.w);
+        mma_tf32(pt[nl], ah, qv.x, qv.y);
+      }
+    }
+    float* RED = reinterpret_cast<float*>(GSs(s));   // [64][KP], within the gradient slots
+    if (slab == 1) {
+#pragma unroll
+      for (int nl = 0; nl < NL; ++nl)
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          RED[(16 * rb + g + 8 * (r >> 1)) * KP + 8 * nl + 2 * tq + (r & 1)] = pt[nl][r];
+    }
+    __syncthreads();
+    if (slab == 0) {
+#pragma unroll
+      for (int nl = 0; nl < NL; ++nl)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int rl = 16 * rb + g + 8 * (r >> 1), l = 8 * nl + 2 * tq + (r & 1);
+          if (r0 + rl < m && l < k)
+            Ppart[(((long long)b * nb + bj) * m + r0 + rl) * k + l] = pt[nl][r] + RED[rl * KP + l];
+        }
+    }
+  }
+  if (bad && status) atomicExch(status, GM_E_NONFINITE);
+}
+
 // ------------------------------------------------------------------ S4
 // (a) P~ = sum of column-split partials (fixed order); partial Gram P~^T P~.
 __global__ void __launch_bounds__(kThreads) k_orth_gram(int m, int k, int csplit, int rsplit,
@@ -1509,6 +1777,29 @@ cudaError_t launch_rebuild_t(dim3 grid, cudaStream_t s, int m, int n, int k,
   return cudaGetLastError();
 }
 
+template <int SRC, int GDT, int KP>
+cudaError_t launch_pipe_t(int B, int m, int n, cudaStream_t s, int k, const uint8_t* codes4,
+                          const float* rscale, const float* cscale, const float* Mprev32, float mu,
+                          const void* G, const uint32_t* QF, const uint32_t* RF, const uint32_t* PF,
+                          float* M, double* norm2_part, float* Ppart, int32_t* status) {
+  const size_t smem = (size_t)pipe_smem_words(SRC, GDT, KP) * sizeof(uint32_t);
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_rebuild_pipe<SRC, GDT, KP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int nb = cdiv(n, kGrid), nrb = cdiv(m, kRB);
+  // tiles per CTA: up to kRebuildTiles while the grid keeps about four CTAs per SM
+  const long long tiles = (long long)nb * nrb * B;
+  const int per = (int)max(1LL, min((long long)kRebuildTiles, tiles / (4 * 148)));
+  dim3 grid(nb, cdiv(nrb, per), B);
+  k_rebuild_pipe<SRC, GDT, KP><<<grid, kRBT, smem, s>>>(m, n, k, codes4, rscale, cscale, Mprev32, mu, G,
+                                                         QF, RF, PF, M, norm2_part, Ppart, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4, const float* rscale,
                            const float* cscale, const int8_t* P8, const float* Pscale,
                            const int8_t* R8, const float* Rscale, const float* Mprev32, float mu,
@@ -1521,8 +1812,10 @@ cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4, co
   const int src = codes4 ? SRC_STATE : (Mprev32 ? SRC_DENSE : SRC_ZERO);
   // ready-made fragments: QF whenever Q is given, RF and PF for the state source
   const bool fr = (!Q || QF) && (src != SRC_STATE || (RF && PF)) && (Q || src == SRC_STATE);
-#define GM_RB(S, W, K, F) launch_rebuild_t<S, W, K, F>(grid, s, m, n, k, codes4, rscale, cscale, P8, \
-    Pscale, R8, Rscale, Mprev32, mu, G, gdt, Q, QF, RF, PF, M, norm2_part, Ppart, status)
+#define GM_RB(S, W, K, F) ((F) ? launch_pipe_t<S, W, K>(B, m, n, s, k, codes4, rscale, cscale, Mprev32, \
+    mu, G, QF, RF, PF, M, norm2_part, Ppart, status) : launch_rebuild_t<S, W, K, F>(grid, s, m, n, k, \
+    codes4, rscale, cscale, P8, Pscale, R8, Rscale, Mprev32, mu, G, gdt, Q, QF, RF, PF, M, norm2_part, \
+    Ppart, status))
 #define GM_RBK(S, W, F) (kp == 8 ? GM_RB(S, W, 8, F) : (kp == 16 ? GM_RB(S, W, 16, F) : GM_RB(S, W, 32, F)))
 #define GM_RBD(S, F) (gd == GM_F32 ? GM_RBK(S, GM_F32, F) : (gd == GM_BF16 ? GM_RBK(S, GM_BF16, F) : GM_RBK(S, GM_F16, F)))
   if (src == SRC_STATE) {   // the raw-factor path serves the rebuild-only call (no gradient)
