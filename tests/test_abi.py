@@ -76,3 +76,16 @@ def test_argument_errors_are_reported_before_any_launch():
     st2 = gm.GraspStateC(256, 256, 256, 256, 256, 256, 256, 256, 256)
     r = gm.lib.gm_grasp_step(1, 256, 512, ctypes.byref(prm2), ctypes.byref(st2), p, p, 0, p, 16, None)
     assert r == gm.GM_E_WORKSPACE
+
+
+def test_misaligned_arrays_are_rejected_before_any_launch():
+    """Every device array must be 16-byte aligned (the kernels move 16-byte vectors)."""
+    ok, bad = ctypes.c_void_p(4096), ctypes.c_void_p(4096 + 8)
+    r = gm.lib.gm_grid_quant4(1, 256, 512, 0, bad, None, None, ok, ok, ok, None)
+    assert r == gm.GM_E_ARG and b"aligned" in gm.lib.gm_last_error()
+    prm = gm.GraspParams(0.95, 0.02, 0.0, 8, 5, 0, None, None, 0, 1e-7, 0)
+    st = gm.GraspStateC(4096, 4096, 4096, 4096, 4096, 4096, 4096 + 4, 4096, 4096)   # Rscale off by 4
+    r = gm.lib.gm_grasp_step(1, 256, 512, ctypes.byref(prm), ctypes.byref(st), ok, ok, 1, ok, 1 << 30, None)
+    assert r == gm.GM_E_ARG and b"aligned" in gm.lib.gm_last_error()
+    r = gm.lib.gm_newton_schulz(1, 256, 512, bad, 1, None, 5, 1e-7, ok, 0, ok, 1 << 30, None)
+    assert r == gm.GM_E_ARG
