@@ -320,321 +320,164 @@ __global__ void __launch_bounds__(kThreads) k_warm_q(int m, int n, int k, int nb
 }
 
 // ------------------------------------------------------------------ S1 + S3
-// Rebuild + momentum, fused with the projection P~ = M Q.
-// CTA: 64 rows x 128 columns (half a grid block), 8 warps, two CTAs per SM.
+// Rebuild + momentum, fused with the projection P~ = M Q (k_rebuild_pipe below).
+// Tile: 64 rows x 128 columns (half a grid block), 8 warps, two CTAs per SM.
 // Warp w owns the rows 16 (w & 3) .. + 15 and the 64-column slab w >> 2; lane
-// (g, t) the rows g and g + 8 of the
-// warp's 16 and the 16 consecutive columns 16 t .. 16 t + 15 of the slab, so its
-// loads and stores are whole 16-column runs. Column 16 t + 2 s + e of the slab
-// is column 2 t + e of n-tile s in the C fragments, which makes
+// (g, t) the rows g and g + 8 of the warp's 16 and the 16 consecutive columns
+// 16 t .. 16 t + 15 of the slab, so its loads and stores are whole 16-column runs.
+// Column 16 t + 2 s + e of the slab is column 2 t + e of n-tile s in the C
+// fragments, which makes
 //   * the rank-k rebuild P^ R^T eight n-tiles of bf16 mma.m16n8k16 with
 //     A = the 8-bit P codes times c_l = Pscale_l Rscale_l / 127^2, split into
 //     three bf16 parts (exact), and B = the R codes (exact in bf16);
 //   * the projection a tf32 mma.m16n8k8 whose A operand is M read straight from
 //     those fragments (k-step s = slab columns 16 t + 2 s + {0, 1} of every t)
 //     and whose B is Q, both split hi + lo (3xTF32).
-// The tile's raw factors (R and P codes, Q) are copied to shared memory with
-// cp.async while the element loads are in flight, then laid out as fragments.
 // The decoded nibble value q / 7 comes from a 16-entry table filled with IEEE
-// divisions, so it is bit-identical to (float)q / 7.0f. P~ partials of the tile
+// divisions, so it is bit-identical to (float)q / 7.0f. P~ partials of a tile
 // (sum over its 128 columns, the two slabs added in order) go to
 // Ppart[b][bj][row][l]; the orthonormalisation sums the column blocks in fp64 in
 // a fixed order.
-constexpr int kRB = 64;     // rows per rebuild CTA
+constexpr int kRB = 64;     // rows per rebuild tile
 constexpr int kRBT = 256;  // threads per rebuild CTA
-
-// 32-bit words of the rebuild CTA's dynamic shared memory: Q fragments, slab
-// reduction, raw Q, then (state) R and P code fragments and raw R and P codes
-__host__ __device__ constexpr int rebuild_smem_words(int KP, bool state) {
-  return 2 * 8 * (KP / 8) * 32 * 4 + kRB * KP + kGrid * KP +
-         (state ? 2 * 8 * (kb16(KP) / 16) * 32 * 2 + 4 * (kb16(KP) / 16) * 3 * 32 * 4 +
-                      (kGrid + kRB) * KP / 4
-                : 0);
-}
 
 enum RebuildSrc { SRC_STATE = 0, SRC_DENSE = 1, SRC_ZERO = 2 };
 
-// KP: the factor width k rounded up to 8, 16 or 32 (columns beyond k are zero).
-// FR: the fragments come ready-made (QF, RF, PF in global memory); otherwise the
-// CTA builds them from the raw factors.
-// GDT: the gradient's dtype (GM_F32, GM_BF16 or GM_F16).
-template <int SRC, int GDT, int KP, bool FR>
-__global__ void __launch_bounds__(kRBT, 2) k_rebuild_proj(
+// The rebuild alone (the rebuild-only entry point: M_{t-1} from the stored
+// state, no gradient, no step workspace): one tile per CTA, the factors' MMA
+// fragments built in the CTA from the raw codes, which are copied to shared
+// memory with cp.async while the element loads are in flight.
+__host__ __device__ constexpr int dequant_smem_words(int KP) {
+  return 2 * 8 * (kb16(KP) / 16) * 32 * 2 + 4 * (kb16(KP) / 16) * 3 * 32 * 4 + (kGrid + kRB) * KP / 4;
+}
+
+template <int KP>   // the factor width k rounded up to 8, 16 or 32 (columns beyond k are zero)
+__global__ void __launch_bounds__(kRBT, 2) k_dequant_rebuild(
     int m, int n, int k, const uint8_t* __restrict__ codes4, const float* __restrict__ rscale,
     const float* __restrict__ cscale, const int8_t* __restrict__ P8,
     const float* __restrict__ Pscale, const int8_t* __restrict__ R8,
-    const float* __restrict__ Rscale, const float* __restrict__ Mprev, float mu,
-    const void* __restrict__ G, int gdt, const float* __restrict__ Q,
-    const uint32_t* __restrict__ QFg, const uint32_t* __restrict__ RFg,
-    const uint32_t* __restrict__ PFg, float* __restrict__ M, double* __restrict__ norm2_part,
-    float* __restrict__ Ppart, int32_t* status) {
-  constexpr bool ST = SRC == SRC_STATE;
-  constexpr int NL = KP / 8, KSB = kb16(KP) / 16;
+    const float* __restrict__ Rscale, float* __restrict__ M) {
+  constexpr int KSB = kb16(KP) / 16;
   const int bj = blockIdx.x, bi = blockIdx.y, b = blockIdx.z;
-  const int nb = gridDim.x, mb = gridDim.y;
+  const int nb = gridDim.x;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int g = lane >> 2, tq = lane & 3, rb = warp & 3, slab = warp >> 2;
   const int r0 = bi * kRB, c0 = bj * kGrid;
   const int nrows = min(kRB, m - r0), ncols = min(kGrid, n - c0);   // multiples of 16
-  extern __shared__ __align__(16) uint32_t smr[];
-  uint32_t* QF = smr;                                             // [slab][s][NL][lane][4]
-  float* RED = reinterpret_cast<float*>(QF + 2 * 8 * NL * 32 * 4);   // [64][KP]
-  float* Qraw = RED + kRB * KP;                                      // [128][k]
-  uint32_t* RF = reinterpret_cast<uint32_t*>(Qraw + kGrid * KP);     // [slab][nt][KSB][lane][2]
+  extern __shared__ __align__(16) uint32_t smd[];
+  uint32_t* RF = smd;                                                // [slab][nt][KSB][lane][2]
   uint32_t* PF = RF + 2 * 8 * KSB * 32 * 2;                          // [rb][KSB][part][lane][4]
   int8_t* R8raw = reinterpret_cast<int8_t*>(PF + 4 * KSB * 3 * 32 * 4);   // [128][k]
   int8_t* P8raw = R8raw + kGrid * KP;                                     // [64][k]
   __shared__ float deq4[16];
   __shared__ float cfac[32];
-  __shared__ double red[kRBT / 32];
   const long long mn = (long long)m * n;
-  constexpr bool G32 = GDT == GM_F32;
   const int cb = c0 + 64 * slab + 16 * tq;   // n % 16 == 0: the run is all in or all out
   const bool colok = cb < n;
 
-  // 1. global loads of this thread's 2 x 16 elements, issued before the staging
-  uint32_t gw[2][8];   // 16-bit gradient, two per word
-  float gf[2][16];     // fp32 gradient
-  float mpv[2][16];    // dense M_prev
-  uint2 cw[2];         // 16 nibbles per row
+  // 1. element loads (codes, scales), then the raw factors
+  uint2 cw[2];
   float rsc[2], cs[16];
   bool ok[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int gi = r0 + 16 * rb + g + 8 * h;
     ok[h] = gi < m && colok;
-    const long long base = (long long)b * mn + (long long)gi * n + cb;
-    if constexpr (G32) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float4 v = (ok[h] && G)
-                             ? reinterpret_cast<const float4*>(static_cast<const float*>(G) + base)[u]
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        gf[h][4 * u] = v.x; gf[h][4 * u + 1] = v.y; gf[h][4 * u + 2] = v.z; gf[h][4 * u + 3] = v.w;
-      }
-    } else {
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const uint4 v = (ok[h] && G)
-                            ? reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(G) + base)[u]
-                            : make_uint4(0u, 0u, 0u, 0u);
-        gw[h][4 * u] = v.x; gw[h][4 * u + 1] = v.y; gw[h][4 * u + 2] = v.z; gw[h][4 * u + 3] = v.w;
-      }
-    }
-    if constexpr (ST) {
-      cw[h] = ok[h] ? *reinterpret_cast<const uint2*>(codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2)
-                    : make_uint2(0u, 0u);
-      rsc[h] = gi < m ? rscale[((long long)b * m + gi) * nb + bj] : 0.f;
-    }
-    if constexpr (SRC == SRC_DENSE) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float4 v = ok[h] ? reinterpret_cast<const float4*>(Mprev + base)[u]
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-        mpv[h][4 * u] = v.x; mpv[h][4 * u + 1] = v.y; mpv[h][4 * u + 2] = v.z; mpv[h][4 * u + 3] = v.w;
-      }
-    }
+    cw[h] = ok[h] ? *reinterpret_cast<const uint2*>(codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2)
+                  : make_uint2(0u, 0u);
+    rsc[h] = gi < m ? rscale[((long long)b * m + gi) * nb + bj] : 0.f;
   }
-  if constexpr (ST) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float4 v = colok ? *reinterpret_cast<const float4*>(cscale + ((long long)b * cdiv(m, kGrid) + r0 / kGrid) * n + cb + 4 * u)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-      cs[4 * u] = v.x; cs[4 * u + 1] = v.y; cs[4 * u + 2] = v.z; cs[4 * u + 3] = v.w;
-    }
+  for (int u = 0; u < 4; ++u) {
+    const float4 v = colok ? *reinterpret_cast<const float4*>(cscale + ((long long)b * cdiv(m, kGrid) + r0 / kGrid) * n + cb + 4 * u)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    cs[4 * u] = v.x; cs[4 * u + 1] = v.y; cs[4 * u + 2] = v.z; cs[4 * u + 3] = v.w;
   }
-
-  // 2. the tile's factors: fragment slices (FR) or raw rows of k values
-  if constexpr (FR) {
-    const int nsl = cdiv(n, 64), vs = min(2, nsl - 2 * bj), vb = min(kRB / 16, (m >> 4) - r0 / 16);
-    constexpr int qw = 8 * NL * 128, rw = 8 * KSB * 64, pw = KSB * 3 * 128;   // words per slab / block
-    if (Q) cp_async_block_zf(QF, QFg + ((long long)b * nsl + 2 * bj) * qw, 2 * qw * 4, vs * qw * 4);
-    if constexpr (ST) {
-      cp_async_block_zf(RF, RFg + ((long long)b * nsl + 2 * bj) * rw, 2 * rw * 4, vs * rw * 4);
-      cp_async_block_zf(PF, PFg + ((long long)b * (m >> 4) + r0 / 16) * pw, (kRB / 16) * pw * 4, vb * pw * 4);
-    }
-  } else {
-    if (Q) cp_async_block(Qraw, Q + ((long long)b * n + c0) * k, ncols * k * 4);
-    if constexpr (ST) {
-      cp_async_block(R8raw, R8 + ((long long)b * n + c0) * k, ncols * k);
-      cp_async_block(P8raw, P8 + ((long long)b * m + r0) * k, nrows * k);
-    }
-  }
+  cp_async_block(R8raw, R8 + ((long long)b * n + c0) * k, ncols * k);
+  cp_async_block(P8raw, P8 + ((long long)b * m + r0) * k, nrows * k);
   cp_async_commit();
   if (t < 16) deq4[t] = __fdiv_rn((float)((t & 8) ? t - 16 : t), 7.0f);
-  if constexpr (ST && !FR) {
-    if (t < 32)
-      cfac[t] = t < k ? __fdiv_rn(__fmul_rn(Pscale[b * k + t], Rscale[b * k + t]), 16129.0f) : 0.f;
-  }
+  if (t < 32) cfac[t] = t < k ? __fdiv_rn(__fmul_rn(Pscale[b * k + t], Rscale[b * k + t]), 16129.0f) : 0.f;
   cp_async_wait<0>();
   __syncthreads();
 
-  // 3. factor fragments from the raw rows
-  if constexpr (ST && !FR) {
-    // R codes as the B operand of n-tile (jj & 15) / 2, column 2 (jj / 16) + jj % 2
+  // 2. fragments: R codes as the B operand of n-tile (jj & 15) / 2, column
+  // 2 (jj / 16) + jj % 2; P codes x c_l as the A operand in three bf16 parts
 #pragma unroll
-    for (int it = 0; it < kGrid * KSB * 8 / kRBT; ++it) {
-      const int e = t + it * kRBT;
-      const int jl = e / (KSB * 8), l = 2 * (e % (KSB * 8));
-      const int8_t* rr = R8raw + jl * k;
-      const float v0 = (jl < ncols && l < k) ? (float)rr[l] : 0.f;
-      const float v1 = (jl < ncols && l + 1 < k) ? (float)rr[l + 1] : 0.f;
-      const int jj = jl & 63, ll = l & 15;
-      const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
-      RF[((((jl >> 6) * 8 + ((jj & 15) >> 1)) * KSB + (l >> 4)) * 32 + 4 * (2 * (jj >> 4) + (jj & 1)) +
-           ((ll >> 1) & 3)) * 2 + (ll >> 3)] = *reinterpret_cast<const uint32_t*>(&h2);
-    }
+  for (int it = 0; it < kGrid * KSB * 8 / kRBT; ++it) {
+    const int e = t + it * kRBT;
+    const int jl = e / (KSB * 8), l = 2 * (e % (KSB * 8));
+    const int8_t* rr = R8raw + jl * k;
+    const float v0 = (jl < ncols && l < k) ? (float)rr[l] : 0.f;
+    const float v1 = (jl < ncols && l + 1 < k) ? (float)rr[l + 1] : 0.f;
+    const int jj = jl & 63, ll = l & 15;
+    const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
+    RF[((((jl >> 6) * 8 + ((jj & 15) >> 1)) * KSB + (l >> 4)) * 32 + 4 * (2 * (jj >> 4) + (jj & 1)) +
+        ((ll >> 1) & 3)) * 2 + (ll >> 3)] = *reinterpret_cast<const uint32_t*>(&h2);
   }
-  if (Q && !FR) {
-    // Q as the projection's B operand: k-step (jj & 15) / 2, k-slot jj / 16 (+4 for odd jj)
-#pragma unroll 4
-    for (int it = 0; it < kGrid * KP / kRBT; ++it) {
-      const int e = t + it * kRBT;
-      const int jl = e / KP, l = e % KP;
-      const float v = (jl < ncols && l < k) ? Qraw[jl * k + l] : 0.f;
-      const int jj = jl & 63;
-      uint32_t* q4 = QF + ((((jl >> 6) * 8 + ((jj & 15) >> 1)) * NL + (l >> 3)) * 32 + 4 * (l & 7) + (jj >> 4)) * 4;
-      const uint32_t hi = tf32_hi(v);
-      q4[jj & 1] = hi;
-      q4[2 + (jj & 1)] = tf32_lo(v, hi);
-    }
-  }
-  if constexpr (ST && !FR) {
-    // P codes x c_l as the A operand, three bf16 parts
 #pragma unroll
-    for (int it = 0; it < kRB * KSB * 8 / kRBT; ++it) {
-      const int e = t + it * kRBT;
-      const int il = e / (KSB * 8), l = 2 * (e % (KSB * 8));
-      const int8_t* pr = P8raw + il * k;
-      const float v0 = (il < nrows && l < k) ? __fmul_rn((float)pr[l], cfac[l]) : 0.f;
-      const float v1 = (il < nrows && l + 1 < k) ? __fmul_rn((float)pr[l + 1], cfac[l + 1]) : 0.f;
-      uint32_t w3[3];
-      bf16_split3(v0, v1, w3);
-      const int r = il & 15, ll = l & 15;
-      uint32_t* dst = PF + (((il >> 4) * KSB + (l >> 4)) * 3) * 128 +
-                      (4 * (r & 7) + ((ll >> 1) & 3)) * 4 + (r >> 3) + 2 * (ll >> 3);
-      dst[0] = w3[0];
-      dst[128] = w3[1];
-      dst[256] = w3[2];
-    }
+  for (int it = 0; it < kRB * KSB * 8 / kRBT; ++it) {
+    const int e = t + it * kRBT;
+    const int il = e / (KSB * 8), l = 2 * (e % (KSB * 8));
+    const int8_t* pr = P8raw + il * k;
+    const float v0 = (il < nrows && l < k) ? __fmul_rn((float)pr[l], cfac[l]) : 0.f;
+    const float v1 = (il < nrows && l + 1 < k) ? __fmul_rn((float)pr[l + 1], cfac[l + 1]) : 0.f;
+    uint32_t w3[3];
+    bf16_split3(v0, v1, w3);
+    const int r = il & 15, ll = l & 15;
+    uint32_t* dst = PF + (((il >> 4) * KSB + (l >> 4)) * 3) * 128 +
+                    (4 * (r & 7) + ((ll >> 1) & 3)) * 4 + (r >> 3) + 2 * (ll >> 3);
+    dst[0] = w3[0];
+    dst[128] = w3[1];
+    dst[256] = w3[2];
   }
-  if constexpr (!FR) __syncthreads();
+  __syncthreads();
 
-  // 4. rank-k rebuild P^ R^T
+  // 3. rank-k rebuild P^ R^T, then M = q/7 * s + P^ R^T
   float acc[8][4];
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-  if constexpr (ST) {
 #pragma unroll
-    for (int ks = 0; ks < KSB; ++ks) {
-      uint32_t a[3][4];
+  for (int ks = 0; ks < KSB; ++ks) {
+    uint32_t a[3][4];
 #pragma unroll
-      for (int p = 0; p < 3; ++p) {
-        const uint4 v = reinterpret_cast<const uint4*>(PF)[((rb * KSB + ks) * 3 + p) * 32 + lane];
-        a[p][0] = v.x; a[p][1] = v.y; a[p][2] = v.z; a[p][3] = v.w;
-      }
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const uint2 bv = reinterpret_cast<const uint2*>(RF)[((slab * 8 + nt) * KSB + ks) * 32 + lane];
-        mma_bf16(acc[nt], a[2], bv.x, bv.y);
-        mma_bf16(acc[nt], a[1], bv.x, bv.y);
-        mma_bf16(acc[nt], a[0], bv.x, bv.y);
-      }
+    for (int p = 0; p < 3; ++p) {
+      const uint4 v = reinterpret_cast<const uint4*>(PF)[((rb * KSB + ks) * 3 + p) * 32 + lane];
+      a[p][0] = v.x; a[p][1] = v.y; a[p][2] = v.z; a[p][3] = v.w;
     }
-  }
-
-  // 5. M = mu M_prev + G, with M_prev = deq4 + P^R^T (state) or dense or zero
-  float nsq = 0.f;
-  bool bad = false;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int ce = 2 * nt + e;
-        float gv;
-        if constexpr (G32) gv = gf[h][ce];
-        else gv = h16_to_float((uint16_t)(gw[h][ce >> 1] >> (16 * (ce & 1))), GDT == GM_F16);
-        float mp = 0.f;
-        if constexpr (ST) {
-          const uint32_t word = ce < 8 ? cw[h].x : cw[h].y;
-          const float sc = fminf(rsc[h], cs[ce]);
-          mp = __fadd_rn(__fmul_rn(deq4[(word >> (4 * (ce & 7))) & 0xF], sc), acc[nt][2 * h + e]);
-        } else if constexpr (SRC == SRC_DENSE) {
-          mp = mpv[h][ce];
-        }
-        const float o = ok[h] ? __fadd_rn(__fmul_rn(mu, mp), gv) : 0.f;
-        acc[nt][2 * h + e] = o;   // keep M for the projection
-        bad |= !(fabsf(o) <= 3.402823466e38f);   // NaN or infinite
-        nsq = fmaf(o, o, nsq);
-      }
-    }
-    if (ok[h]) {
-      float4* dst = reinterpret_cast<float4*>(M + (long long)b * mn + (long long)(r0 + 16 * rb + g + 8 * h) * n + cb);
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        dst[u] = make_float4(acc[2 * u][2 * h], acc[2 * u][2 * h + 1], acc[2 * u + 1][2 * h],
-                             acc[2 * u + 1][2 * h + 1]);
+      const uint2 bv = reinterpret_cast<const uint2*>(RF)[((slab * 8 + nt) * KSB + ks) * 32 + lane];
+      mma_bf16(acc[nt], a[2], bv.x, bv.y);
+      mma_bf16(acc[nt], a[1], bv.x, bv.y);
+      mma_bf16(acc[nt], a[0], bv.x, bv.y);
     }
   }
-  const double tot = block_sum_d((double)nsq, red);
-  if (t == 0 && norm2_part) norm2_part[((long long)b * mb + bi) * nb + bj] = tot;
-  if (bad && status) atomicExch(status, GM_E_NONFINITE);
-
-  // 6. projection partials: this tile's share of M Q
-  if (Q) {
-    float pt[NL][4];
 #pragma unroll
-    for (int nl = 0; nl < NL; ++nl) pt[nl][0] = pt[nl][1] = pt[nl][2] = pt[nl][3] = 0.f;
+  for (int h = 0; h < 2; ++h) {
+    if (!ok[h]) continue;
+    float o[16];
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const float xa[4] = {acc[s][0], acc[s][2], acc[s][1], acc[s][3]};
-      uint32_t ah[4], al[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        ah[i] = tf32_hi(xa[i]);
-        al[i] = tf32_lo(xa[i], ah[i]);
-      }
-#pragma unroll
-      for (int nl = 0; nl < NL; ++nl) {
-        const uint4 qv = reinterpret_cast<const uint4*>(QF)[((slab * 8 + s) * NL + nl) * 32 + lane];
-        mma_tf32(pt[nl], al, qv.x, qv.y);
-        mma_tf32(pt[nl], ah, qv.z, qv.w);
-        mma_tf32(pt[nl], ah, qv.x, qv.y);
-      }
+    for (int ce = 0; ce < 16; ++ce) {
+      const uint32_t word = ce < 8 ? cw[h].x : cw[h].y;
+      const float sc = fminf(rsc[h], cs[ce]);
+      o[ce] = __fadd_rn(__fmul_rn(deq4[(word >> (4 * (ce & 7))) & 0xF], sc), acc[ce >> 1][2 * h + (ce & 1)]);
     }
-    if (slab == 1) {
+    float4* dst = reinterpret_cast<float4*>(M + (long long)b * mn + (long long)(r0 + 16 * rb + g + 8 * h) * n + cb);
 #pragma unroll
-      for (int nl = 0; nl < NL; ++nl)
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-          RED[(16 * rb + g + 8 * (r >> 1)) * KP + 8 * nl + 2 * tq + (r & 1)] = pt[nl][r];
-    }
-    __syncthreads();
-    if (slab == 0) {
-#pragma unroll
-      for (int nl = 0; nl < NL; ++nl)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int rl = 16 * rb + g + 8 * (r >> 1), l = 8 * nl + 2 * tq + (r & 1);
-          if (r0 + rl < m && l < k)
-            Ppart[(((long long)b * nb + bj) * m + r0 + rl) * k + l] = pt[nl][r] + RED[rl * KP + l];
-        }
-    }
+    for (int u = 0; u < 4; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
   }
 }
 
-// Pipelined form of the same pass for ready-made fragments: a CTA owns one
-// 128-column block and walks up to kRebuildTiles 64-row tiles of it (rows
+// The fused pass, pipelined: a CTA owns one 128-column block and walks up to
+// kRebuildTiles 64-row tiles of it (rows
 // blockIdx.y, + gridDim.y, ...). Q's and R's fragments are copied once; every
 // input of tile i + 1 (its P fragments, gradient, codes, row and column scales,
 // dense M_{t-1}) streams into the other of two shared-memory stages with
 // cp.async while tile i is multiplied, so the memory latency of one tile hides
 // behind the work of the previous one. Each thread copies its own gradient (and
 // M_{t-1}) chunks and reads only those back; the shared inputs become visible at
-// the barrier after the copies complete. The arithmetic per element is the one
-// of k_rebuild_proj.
+// the barrier after the copies complete.
 constexpr int kRebuildTiles = 4;
 
 __host__ __device__ constexpr int pipe_g_chunks(int GDT) { return GDT == GM_F32 ? 8 : 4; }
@@ -1754,26 +1597,20 @@ cudaError_t launch_warm_start(int B, int m, int n, int k, const int8_t* R8, cons
   return cudaGetLastError();
 }
 
-template <int SRC, int GDT, int KP, bool FR>
-cudaError_t launch_rebuild_t(dim3 grid, cudaStream_t s, int m, int n, int k,
-                             const uint8_t* codes4, const float* rscale, const float* cscale,
-                             const int8_t* P8, const float* Pscale, const int8_t* R8,
-                             const float* Rscale, const float* Mprev32, float mu, const void* G,
-                             int gdt, const float* Q, const uint32_t* QF, const uint32_t* RF,
-                             const uint32_t* PF, float* M, double* norm2_part, float* Ppart,
-                             int32_t* status) {
-  const size_t smem = (size_t)rebuild_smem_words(KP, SRC == SRC_STATE) * sizeof(uint32_t);
+template <int KP>
+cudaError_t launch_dequant_t(int B, int m, int n, int k, const uint8_t* codes4, const float* rscale,
+                             const float* cscale, const int8_t* P8, const float* Pscale,
+                             const int8_t* R8, const float* Rscale, float* M, cudaStream_t s) {
+  const size_t smem = (size_t)dequant_smem_words(KP) * sizeof(uint32_t);
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_rebuild_proj<SRC, GDT, KP, FR>,
+    cudaError_t e = cudaFuncSetAttribute(k_dequant_rebuild<KP>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  k_rebuild_proj<SRC, GDT, KP, FR><<<grid, kRBT, smem, s>>>(m, n, k, codes4, rscale, cscale, P8,
-                                                            Pscale, R8, Rscale, Mprev32, mu, G, gdt,
-                                                            Q, QF, RF, PF, M, norm2_part, Ppart,
-                                                            status);
+  dim3 grid(cdiv(n, kGrid), cdiv(m, kRB), B);
+  k_dequant_rebuild<KP><<<grid, kRBT, smem, s>>>(m, n, k, codes4, rscale, cscale, P8, Pscale, R8, Rscale, M);
   return cudaGetLastError();
 }
 
@@ -1806,25 +1643,23 @@ cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4, co
                            const void* G, int gdt, const float* Q, const uint32_t* QF,
                            const uint32_t* RF, const uint32_t* PF, float* M, double* norm2_part,
                            float* Ppart, int32_t* status, cudaStream_t s) {
-  dim3 grid(cdiv(n, kGrid), cdiv(m, kRB), B);
   const int kp = factor_width(k);
-  const int gd = (G == nullptr) ? GM_F32 : gdt;
   const int src = codes4 ? SRC_STATE : (Mprev32 ? SRC_DENSE : SRC_ZERO);
-  // ready-made fragments: QF whenever Q is given, RF and PF for the state source
-  const bool fr = (!Q || QF) && (src != SRC_STATE || (RF && PF)) && (Q || src == SRC_STATE);
-#define GM_RB(S, W, K, F) ((F) ? launch_pipe_t<S, W, K>(B, m, n, s, k, codes4, rscale, cscale, Mprev32, \
-    mu, G, QF, RF, PF, M, norm2_part, Ppart, status) : launch_rebuild_t<S, W, K, F>(grid, s, m, n, k, \
-    codes4, rscale, cscale, P8, Pscale, R8, Rscale, Mprev32, mu, G, gdt, Q, QF, RF, PF, M, norm2_part, \
-    Ppart, status))
-#define GM_RBK(S, W, F) (kp == 8 ? GM_RB(S, W, 8, F) : (kp == 16 ? GM_RB(S, W, 16, F) : GM_RB(S, W, 32, F)))
-#define GM_RBD(S, F) (gd == GM_F32 ? GM_RBK(S, GM_F32, F) : (gd == GM_BF16 ? GM_RBK(S, GM_BF16, F) : GM_RBK(S, GM_F16, F)))
-  if (src == SRC_STATE) {   // the raw-factor path serves the rebuild-only call (no gradient)
-    if (fr) return GM_RBD(SRC_STATE, true);
-    return gd == GM_F32 ? GM_RBK(SRC_STATE, GM_F32, false) : cudaErrorInvalidValue;
+  if (!G && !Q && src == SRC_STATE && !QF) {   // the rebuild alone, from the raw codes
+    if (kp == 8) return launch_dequant_t<8>(B, m, n, k, codes4, rscale, cscale, P8, Pscale, R8, Rscale, M, s);
+    if (kp == 16) return launch_dequant_t<16>(B, m, n, k, codes4, rscale, cscale, P8, Pscale, R8, Rscale, M, s);
+    return launch_dequant_t<32>(B, m, n, k, codes4, rscale, cscale, P8, Pscale, R8, Rscale, M, s);
   }
-  if (!fr) return cudaErrorInvalidValue;   // dense / zero sources always come with QF
-  if (src == SRC_DENSE) return GM_RBD(SRC_DENSE, true);
-  return GM_RBD(SRC_ZERO, true);
+  // the fused pass needs Q's fragments, and R's and P's for the stored state
+  if (!Q || !QF || (src == SRC_STATE && (!RF || !PF))) return cudaErrorInvalidValue;
+  const int gd = (G == nullptr) ? GM_F32 : gdt;
+#define GM_RB(S, W, K) launch_pipe_t<S, W, K>(B, m, n, s, k, codes4, rscale, cscale, Mprev32, mu, G, QF, \
+                                              RF, PF, M, norm2_part, Ppart, status)
+#define GM_RBK(S, W) (kp == 8 ? GM_RB(S, W, 8) : (kp == 16 ? GM_RB(S, W, 16) : GM_RB(S, W, 32)))
+#define GM_RBD(S) (gd == GM_F32 ? GM_RBK(S, GM_F32) : (gd == GM_BF16 ? GM_RBK(S, GM_BF16) : GM_RBK(S, GM_F16)))
+  if (src == SRC_STATE) return GM_RBD(SRC_STATE);
+  if (src == SRC_DENSE) return GM_RBD(SRC_DENSE);
+  return GM_RBD(SRC_ZERO);
 #undef GM_RBD
 #undef GM_RBK
 #undef GM_RB

@@ -39,9 +39,10 @@ cudaError_t launch_warm_start(int B, int m, int n, int k, const int8_t* R8, cons
 // projection partials Ppart f32 [B][ceil(n/128)][m][k] (sum over one column
 // block each). norm2_part gets one fp64 partial |M|^2 per 128 x 128 tile
 // ([B][ceil(m/128)][ceil(n/128)]); status (nullable) gets GM_E_NONFINITE.
-// Data pointers are 16-byte aligned; m and n are multiples of 16. QF (with Q)
-// and RF, PF (with the state) are the ready-made fragments; NULL builds them in
-// each CTA from Q, R8, P8 (the dense and zero sources need QF).
+// Data pointers are 16-byte aligned; m and n are multiples of 16. The fused pass
+// takes the ready-made fragments QF (with Q) and RF, PF (with the state); the
+// rebuild alone (state, no G, no Q, no fragments) builds its fragments in each
+// CTA from R8, P8.
 cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4,
                            const float* rscale, const float* cscale, const int8_t* P8,
                            const float* Pscale, const int8_t* R8, const float* Rscale,
