@@ -511,7 +511,11 @@ def run_ours(args, world, rank, local):
                           "what": "standard NS, T steps of torch.matmul / baddbmm (cuBLAS bf16, "
                                   "dense products), same inputs and streams"},
             "codec": {"gbs": codec_gbs, "peak_gbs": hbm, "frac": codec_gbs / hbm,
-                      "ms": cod_ms, "kernels": "k_rebuild + k_residual_quant4"},
+                      "ms": cod_ms,
+                      "kernels": "rebuild (k_dequant_rebuild) + residual grid quantisation "
+                                 "(k_residual_quant4) through the standalone entry points, "
+                                 "which stage the factor fragments in each CTA"},
+            "step_minus_ns_ms": ms_step - ns_ms,
             "step_roofline": {"ms": t_roof, "frac": t_roof / ms_step, "flops": step_flops,
                               "bytes": step_bytes},
             "gpu_launches": launches,
