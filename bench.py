@@ -205,9 +205,9 @@ def run_reference(args, world, rank):
 GRAD_POOL = 6   # distinct gradient buffers per group, used cyclically step after step
 
 # DRAM bytes per k_gemm launch (average over one step's 45 NS products of the
-# LLaMA-130M set, standard NS), from the ncu capture summarised in
-# profiles/k_gemm_llama130m.md; reported only while gm_gemm.cu is the source
-# that capture measured.
+# LLaMA-130M set, standard NS), from an ncu capture of dram__bytes_read.sum +
+# dram__bytes_write.sum (the k_gemm summary under profiles/); reported only while
+# gm_gemm.cu is the source that capture measured.
 GEMM_TRAFFIC = {"config": 2, "ns": "standard", "bytes_per_launch": 87.56e6,
                 "source_sha256": "aa52586b7c8ef53cef64f66392279f880c35c449ce72813d6b82ec7d5a190d0a"}
 

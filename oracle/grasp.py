@@ -6,7 +6,7 @@ matmul is the only library primitive used as a step. Quantization decisions
 kernels decide them in: IEEE fp32 division, fp32 multiply by 7 or 127,
 round-half-to-even, clamp. All other arithmetic is fp64.
 
-Readings of points the pages leave open (each also listed in the design doc):
+Readings of points the pages leave open:
 
 * NS coefficients: T=5 steps of the constant quintic (a,b,c) =
   (3.4445, -4.7750, 2.0315) [LiMuon, key design 3], for both the standard
