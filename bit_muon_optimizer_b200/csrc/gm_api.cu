@@ -53,10 +53,10 @@ struct StepLayout {
 StepLayout step_layout(int B, int m, int n, int k, int ns_mode, bool with_ns) {
   StepLayout L;
   memset(&L, 0, sizeof(L));
-  L.csplit = cdiv(n, kGrid);                        // projection partials: one per column block
+  L.csplit = cdiv(n, 64);                           // projection partials: one per 64-column slab
   L.rsplit_b = backproject_row_splits(B, m, n);
   L.rsplit_g = gram_row_splits(B, m);
-  L.ntiles = rebuild_row_blocks(m) * cdiv(n, kGrid);  // |M|^2 partials
+  L.ntiles = rebuild_row_blocks(m) * cdiv(n, kGrid) * 8;  // |M|^2 partials: one per warp of a tile
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off += al256(bytes); return o; };
   const size_t Bz = (size_t)B, mz = (size_t)m, nz = (size_t)n, kz = (size_t)k;

@@ -334,10 +334,11 @@ __global__ void __launch_bounds__(kThreads) k_warm_q(int m, int n, int k, int nb
 //     those fragments (k-step s = slab columns 16 t + 2 s + {0, 1} of every t)
 //     and whose B is Q, both split hi + lo (3xTF32).
 // The decoded nibble value q / 7 comes from a 16-entry table filled with IEEE
-// divisions, so it is bit-identical to (float)q / 7.0f. P~ partials of a tile
-// (sum over its 128 columns, the two slabs added in order) go to
-// Ppart[b][bj][row][l]; the orthonormalisation sums the column blocks in fp64 in
-// a fixed order.
+// divisions, so it is bit-identical to (float)q / 7.0f. Each warp writes its own
+// partials, so no block-wide reduction (and no barrier) is needed per tile: P~
+// over its 64-column slab to Ppart[b][slab][row][l] and |M|^2 over its 16 x 64
+// part to norm2_part[b][row tile][column block][warp]; the orthonormalisation
+// sums them in fp64 in a fixed order.
 constexpr int kRB = 64;     // rows per rebuild tile
 constexpr int kRBT = 256;  // threads per rebuild CTA
 
@@ -518,7 +519,6 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_pipe(
   uint32_t* RF = QF + 2 * QW;                  // [slab][nt][KSB][lane][2]
   uint32_t* stg = RF + (ST ? 2 * RW : 0);      // two stages of SW words
   __shared__ float deq4[16];
-  __shared__ double red[kRBT / 32];
 
   // stage layout
   auto PFs = [&](int s) { return stg + s * SW; };                                  // [rb][KSB][part][lane][4]
@@ -689,10 +689,13 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_pipe(
                                acc[2 * u + 1][2 * h + 1]);
       }
     }
-    const double tot = block_sum_d((double)nsq, red);
-    if (t == 0 && norm2_part) norm2_part[((long long)b * nrb + rbi) * nb + bj] = tot;
+    // |M|^2 partial of this warp's 16 x 64 part of the tile (fixed shuffle tree)
+    double wsq = (double)nsq;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsq += __shfl_xor_sync(0xffffffffu, wsq, o);
+    if (lane == 0 && norm2_part) norm2_part[(((long long)b * nrb + rbi) * nb + bj) * (kRBT / 32) + warp] = wsq;
 
-    // projection partials; the slab reduction reuses this stage's gradient slots
+    // projection partials of this warp's 64-column slab
     float pt[NL][4];
 #pragma unroll
     for (int nl = 0; nl < NL; ++nl) pt[nl][0] = pt[nl][1] = pt[nl][2] = pt[nl][3] = 0.f;
@@ -713,23 +716,14 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_pipe(
         mma_tf32(pt[nl], ah, qv.x, qv.y);
       }
     }
-    float* RED = reinterpret_cast<float*>(GSs(s));   // [64][KP], within the gradient slots
-    if (slab == 1) {
-#pragma unroll
-      for (int nl = 0; nl < NL; ++nl)
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-          RED[(16 * rb + g + 8 * (r >> 1)) * KP + 8 * nl + 2 * tq + (r & 1)] = pt[nl][r];
-    }
-    __syncthreads();
-    if (slab == 0) {
+    if (2 * bj + slab < nsl) {
+      const long long pbase = ((long long)b * nsl + 2 * bj + slab) * m;
 #pragma unroll
       for (int nl = 0; nl < NL; ++nl)
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const int rl = 16 * rb + g + 8 * (r >> 1), l = 8 * nl + 2 * tq + (r & 1);
-          if (r0 + rl < m && l < k)
-            Ppart[(((long long)b * nb + bj) * m + r0 + rl) * k + l] = pt[nl][r] + RED[rl * KP + l];
+          if (r0 + rl < m && l < k) Ppart[(pbase + r0 + rl) * k + l] = pt[nl][r];
         }
     }
   }

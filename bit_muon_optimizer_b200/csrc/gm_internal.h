@@ -8,7 +8,7 @@ namespace gm {
 
 // Column / row split counts of the power-iteration reductions. They depend
 // only on the problem shape, so the workspace layout is a pure function of it.
-int rebuild_row_blocks(int m);   // 128-row blocks of the fused rebuild / projection
+int rebuild_row_blocks(int m);   // 64-row tiles of the fused rebuild / projection
 int backproject_row_splits(int B, int m, int n);
 int gram_row_splits(int B, int m);
 // The factor width k rounded up to 8, 16 or 32: the depth of the codec kernels'
@@ -36,9 +36,9 @@ cudaError_t launch_warm_start(int B, int m, int n, int k, const int8_t* R8, cons
 
 // M = mu * Mprev + G where Mprev is either the rebuilt state (codes4 != NULL)
 // or a dense fp32 matrix (Mprev32 != NULL) or zero; with Q != NULL also the
-// projection partials Ppart f32 [B][ceil(n/128)][m][k] (sum over one column
-// block each). norm2_part gets one fp64 partial |M|^2 per 128 x 128 tile
-// ([B][ceil(m/128)][ceil(n/128)]); status (nullable) gets GM_E_NONFINITE.
+// projection partials Ppart f32 [B][ceil(n/64)][m][k] (sum over one 64-column
+// slab each). norm2_part gets one fp64 partial |M|^2 per warp of a 64 x 128 tile
+// ([B][ceil(m/64)][ceil(n/128)][8]); status (nullable) gets GM_E_NONFINITE.
 // Data pointers are 16-byte aligned; m and n are multiples of 16. The fused pass
 // takes the ready-made fragments QF (with Q) and RF, PF (with the state); the
 // rebuild alone (state, no G, no Q, no fragments) builds its fragments in each
