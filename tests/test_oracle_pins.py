@@ -398,6 +398,33 @@ def test_step_mu_zero_momentum_is_gradient_and_k_full_is_lossless():
     assert float(torch.linalg.matrix_norm(r2.residual)) < 1e-12 * float(torch.linalg.matrix_norm(r2.M))
 
 
+@pytest.mark.parametrize("m,n", [(96, 48), (48, 96)])
+@pytest.mark.parametrize("ns", ["standard", "gram"])
+def test_step_weight_update_closed_form_on_rank_one_gradient(m, n, ns):
+    """From a zero state, M_1 = G. For G = sigma u v^T (unit u, v) the
+    Frobenius norm is sigma, so NS sees one singular value s = sigma /
+    (sigma + eps) and, by Proposition 1 of the Gram Newton-Schulz page,
+    returns f(s) u v^T with f the composed scalar quintic. The update
+    W <- W - eta (O + wd W) of "Achieving low-bit Muon through subspace
+    preservation and grid quantization" (worked step 6) then has the closed
+    form (1 - eta wd) W - eta f(s) u v^T: a flipped sign, a missing eta on the
+    decay term or a mis-oriented O for a tall matrix all break it."""
+    gen = torch.Generator().manual_seed(17)
+    u = torch.randn(m, generator=gen, dtype=DT)
+    v = torch.randn(n, generator=gen, dtype=DT)
+    u, v = u / u.norm(), v / v.norm()
+    sigma, eta, wd = 0.37, 0.02, 0.1
+    G = sigma * torch.outer(u, v)
+    W = torch.randn(m, n, generator=gen, dtype=DT)
+    r = O.grasp_step(O.zero_state(m, n, 4, block=16), W, G, mu=0.95, eta=eta, wd=wd,
+                     ns=ns, block=16)
+    f = O.quintic_scalar(sigma / (sigma + O.NS_EPS))
+    assert 0.5 < f < 1.5
+    want = (1 - eta * wd) * W - eta * f * torch.outer(u, v)
+    assert float((r.W - want).abs().max()) <= 1e-12
+    assert float((r.O - f * torch.outer(u, v)).abs().max()) <= 1e-10
+
+
 def test_step_rebuild_roundtrip():
     """After a step, rebuilding from the new state reproduces M_t up to the
     codes' half-step bounds: |M - M^| <= s/14 + 8-bit factor error."""
