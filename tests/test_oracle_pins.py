@@ -398,6 +398,34 @@ def test_step_mu_zero_momentum_is_gradient_and_k_full_is_lossless():
     assert float(torch.linalg.matrix_norm(r2.residual)) < 1e-12 * float(torch.linalg.matrix_norm(r2.M))
 
 
+def test_step_momentum_is_undamped_heavy_ball():
+    """Muon's momentum M_t = mu M_{t-1} + G_t ("Achieving low-bit Muon through
+    subspace preservation and grid quantization", worked step 3) carries no
+    (1 - mu) damping on the gradient. From a fixed non-zero state, M is
+    therefore affine in G with unit slope and, at G = 0, linear in mu: a
+    damped EMA or swapped operands break one of the two."""
+    gen = torch.Generator().manual_seed(18)
+    m, n, k = 32, 64, 4
+    st = O.zero_state(m, n, k, block=16)
+    st.codes4 = torch.randint(0, 255, (m, n // 2), generator=gen, dtype=torch.uint8)
+    st.rscale = torch.rand(st.rscale.shape, generator=gen)
+    st.cscale = torch.rand(st.cscale.shape, generator=gen)
+    st.P8 = torch.randint(-127, 128, (m, k), generator=gen, dtype=torch.int8)
+    st.R8 = torch.randint(-127, 128, (n, k), generator=gen, dtype=torch.int8)
+    st.Pscale, st.Rscale = torch.rand(k, generator=gen), torch.rand(k, generator=gen)
+    G = torch.randn(m, n, generator=gen)
+    Z = torch.zeros(m, n)
+
+    def M(mu, g):
+        return O.grasp_step(st, Z, g, mu=mu, eta=0.0, block=16).M
+
+    M1 = M(1.0, Z)
+    assert float(M1.abs().max()) > 0.1
+    assert float((M(0.9, G) - M(0.9, Z) - G.double()).abs().max()) <= 1e-12
+    assert float((M(0.9, Z) - 0.9 * M1).abs().max()) <= 1e-12
+    assert float((M(0.0, G) - G.double()).abs().max()) == 0.0
+
+
 @pytest.mark.parametrize("m,n", [(96, 48), (48, 96)])
 @pytest.mark.parametrize("ns", ["standard", "gram"])
 def test_step_weight_update_closed_form_on_rank_one_gradient(m, n, ns):
