@@ -426,6 +426,29 @@ def test_step_momentum_is_undamped_heavy_ball():
     assert float((M(0.0, G) - G.double()).abs().max()) == 0.0
 
 
+def test_step_warm_start_takes_the_stored_right_factor():
+    """The warm start of step t is built from the stored R_{t-1} (the right
+    factor, n x k), not P_{t-1} ("Achieving low-bit Muon through subspace
+    preservation and grid quantization", worked step 2). Step 1 stores the
+    exact factors of a square rank-k momentum U S V^T. Step 2 adds the gradient
+    X S' U^T, with U, V, X mutually orthogonal k-frames, so M_2 = U S V^T +
+    X S' U^T. One power iteration from Q ~ V gives M_2 Q ~ U S: P spans U.
+    From Q ~ U (the left factor) it would give M_2 Q ~ X S': P would span X."""
+    gen = torch.Generator().manual_seed(19)
+    n, k = 64, 4
+    Qo = _orthogonal(n, gen)
+    U, V, X = Qo[:, :k], Qo[:, k:2 * k], Qo[:, 2 * k:3 * k]
+    S = torch.diag(torch.tensor([0.4, 0.3, 0.2, 0.1], dtype=DT))
+    Z = torch.zeros(n, n)
+    r1 = O.grasp_step(O.zero_state(n, n, k, block=16), Z, U @ S @ V.T, mu=0.95, eta=0.0,
+                      block=16)
+    assert float(torch.linalg.matrix_norm(r1.residual)) < 1e-12
+    r2 = O.grasp_step(r1.state, Z, X @ (0.3 * S) @ U.T, mu=1.0, eta=0.0, block=16)
+    off = float(torch.linalg.matrix_norm(r2.P - U @ (U.T @ r2.P)))
+    assert off < 0.05, off
+    assert float(torch.linalg.matrix_norm(U.T @ r2.P)) > 0.99 * math.sqrt(k)
+
+
 @pytest.mark.parametrize("m,n", [(96, 48), (48, 96)])
 @pytest.mark.parametrize("ns", ["standard", "gram"])
 def test_step_weight_update_closed_form_on_rank_one_gradient(m, n, ns):
