@@ -534,13 +534,25 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_pipe(
       const int vb = min(kRB / 16, (m >> 4) - r0 / 16);
       cp_async_block_zf(PFs(s), PFg + ((long long)b * (m >> 4) + r0 / 16) * PW, (kRB / 16) * PW * 4, vb * PW * 4);
       {   // codes: 64 rows x 64 bytes, one 16-byte chunk (32 columns) per thread; a
-          // chunk half past the last column (ncols % 32 == 16) copies 8 bytes
+          // chunk half past the last column (ncols % 32 == 16) copies 8 bytes. A codes
+          // row is n / 2 bytes, so rows start 16-byte aligned only when n % 32 == 0;
+          // otherwise (n % 32 == 16) the chunk goes as two 8-byte copies, which need
+          // only the 8-byte alignment that n % 16 == 0 gives.
         const int r = t >> 2, ch = t & 3, gi = r0 + r;
         const int nbytes = gi < m ? max(0, min(16, (ncols - 32 * ch) / 2)) : 0;
         const uint32_t sa = (uint32_t)__cvta_generic_to_shared(CDs(s) + r * 16 + ch * 4);
         const uint8_t* src = nbytes ? codes4 + ((long long)b * m + gi) * (n / 2) + c0 / 2 + 16 * ch : codes4;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sa), "l"(src), "r"(nbytes)
-                     : "memory");
+        if ((n & 31) == 0) {
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sa), "l"(src), "r"(nbytes)
+                       : "memory");
+        } else {
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(sa), "l"(src),
+                       "r"(min(nbytes, 8))
+                       : "memory");
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(sa + 8u),
+                       "l"(nbytes > 8 ? src + 8 : codes4), "r"(max(nbytes - 8, 0))
+                       : "memory");
+        }
       }
       if (t < kGrid / 4) {   // column scales of the grid-block row
         const bool ok = 4 * t < ncols;

@@ -340,3 +340,67 @@ def test_grasp_step_checkpoint_and_batch_consistency(cuda_lib):
     run(1, slice(0, 1), st1, W1, range(5))
     assert torch.equal(W1[0], WA[0])
     assert torch.equal(st1.codes4[0], stA.codes4[0])
+
+
+@pytest.mark.parametrize("m,n,ns", [(144, 272, "standard"), (272, 144, "gram")])
+def test_grasp_step_ragged_shape(cuda_lib, m, n, ns):
+    """The whole step at sizes that are not multiples of the 128-row grid
+    blocks, the 64-row codec tiles or the NS tiles (144 = 128 + 16,
+    272 = 2*128 + 16), wide and tall, teacher-forced for two steps."""
+    gm = cuda_lib
+    B, k, mu, eta, seed = 2, 8, 0.95, 0.02, 77
+    nsmode = gm.GM_NS_GRAM if ns == "gram" else gm.GM_NS_STANDARD
+    step = gm.GraspStep(B, m, n, k, mu=mu, eta=eta, ns=nsmode, seed=seed, device=DEV)
+    st = gm.GraspState.zeros(B, m, n, k, DEV)
+    W = WL.random_matrix((B, m, n), 41, std=0.02).to(DEV)
+    for t in (1, 2):
+        G = _outlier_matrix(B, m, n, 50 + t, dtype=torch.bfloat16).to(DEV)
+        before = [_to_oracle_state(st, b) for b in range(B)]
+        W0 = W.clone()
+        step(st, W, G)
+        torch.cuda.synchronize()
+        assert int(st.dev_status.item()) == 0
+        for b in range(B):
+            r = O.grasp_step(before[b], W0[b].cpu(), G[b].cpu(), mu=mu, eta=eta, seed=seed,
+                             b=b, ns=ns)
+            assert rel(step.stage_M()[b], r.M) <= 1e-5
+            assert rel(step.stage_P()[b], r.P) <= 1e-5
+            assert rel(step.stage_R()[b], r.R) <= 1e-5
+            q, s = O.quant8(step.stage_P()[b].cpu())
+            assert torch.equal(st.P8[b].cpu(), q) and torch.equal(st.Pscale[b].cpu(), s)
+            q, s = O.quant8(step.stage_R()[b].cpu())
+            assert torch.equal(st.R8[b].cpu(), q) and torch.equal(st.Rscale[b].cpu(), s)
+            assert torch.equal(st.rscale[b].cpu() > 0, r.state.rscale > 0)
+            diff = (O.unpack_nibbles(st.codes4[b].cpu()).int()
+                    - O.unpack_nibbles(r.state.codes4).int()).abs()
+            assert int(diff.max()) <= 1 and int((diff > 0).sum()) <= 4
+            Og = (W0[b].double() - W[b].double()).cpu() / eta
+            assert rel(Og, r.O) <= 2e-2
+
+
+@pytest.mark.parametrize("m,n", [(256, 512), (512, 256)])
+@pytest.mark.parametrize("ns", ["standard", "gram"])
+def test_grasp_step_weight_decay(cuda_lib, m, n, ns):
+    """W <- W - eta (O + wd W). One step from a zero state with wd = 0.1 and
+    with wd = 0: O and the new state depend only on the state and G, so the
+    states match bit for bit and the updated weights differ by -eta wd W_0
+    up to fp32 rounding (relative size ~1e-4 here). Wide and tall, both NS
+    forms: the decay term sits in the epilogue of the last NS product."""
+    gm = cuda_lib
+    B, k, eta, wd = 2, 8, 0.02, 0.1
+    nsmode = gm.GM_NS_GRAM if ns == "gram" else gm.GM_NS_STANDARD
+    W0 = WL.random_matrix((B, m, n), 43, std=0.02).to(DEV)
+    G = _outlier_matrix(B, m, n, 44, dtype=torch.bfloat16).to(DEV)
+    out = {}
+    for lam in (0.0, wd):
+        step = gm.GraspStep(B, m, n, k, eta=eta, wd=lam, ns=nsmode, seed=3, device=DEV)
+        st = gm.GraspState.zeros(B, m, n, k, DEV)
+        W = W0.clone()
+        step(st, W, G)
+        torch.cuda.synchronize()
+        assert int(st.dev_status.item()) == 0
+        out[lam] = (W, st)
+    (W_a, st_a), (W_b, st_b) = out[0.0], out[wd]
+    for a, b in zip(st_a.tensors(), st_b.tensors()):
+        assert torch.equal(a, b)
+    assert rel(W_b - W_a, -eta * wd * W0) <= 1e-3
