@@ -342,13 +342,16 @@ def test_grasp_step_checkpoint_and_batch_consistency(cuda_lib):
     assert torch.equal(st1.codes4[0], stA.codes4[0])
 
 
-@pytest.mark.parametrize("m,n,ns", [(144, 272, "standard"), (272, 144, "gram")])
-def test_grasp_step_ragged_shape(cuda_lib, m, n, ns):
+@pytest.mark.parametrize("m,n,ns,k", [(144, 272, "standard", 8), (272, 144, "gram", 8),
+                                      (256, 384, "standard", 12), (208, 336, "gram", 5)])
+def test_grasp_step_ragged_shape(cuda_lib, m, n, ns, k):
     """The whole step at sizes that are not multiples of the 128-row grid
     blocks, the 64-row codec tiles or the NS tiles (144 = 128 + 16,
-    272 = 2*128 + 16), wide and tall, teacher-forced for two steps."""
+    272 = 2*128 + 16, 208, 336), wide and tall, and at ranks k that are not
+    the factor widths 8, 16, 32 the MMA fragments are padded to, teacher-forced
+    for two steps."""
     gm = cuda_lib
-    B, k, mu, eta, seed = 2, 8, 0.95, 0.02, 77
+    B, mu, eta, seed = 2, 0.95, 0.02, 77
     nsmode = gm.GM_NS_GRAM if ns == "gram" else gm.GM_NS_STANDARD
     step = gm.GraspStep(B, m, n, k, mu=mu, eta=eta, ns=nsmode, seed=seed, device=DEV)
     st = gm.GraspState.zeros(B, m, n, k, DEV)
