@@ -407,3 +407,22 @@ def test_grasp_step_weight_decay(cuda_lib, m, n, ns):
     for a, b in zip(st_a.tensors(), st_b.tensors()):
         assert torch.equal(a, b)
     assert rel(W_b - W_a, -eta * wd * W0) <= 1e-3
+
+
+@pytest.mark.parametrize("odt", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("B,m,n,form", [(2, 256, 512, "standard"), (1, 400, 144, "gram")])
+def test_ns_half_precision_outputs(cuda_lib, odt, B, m, n, form):
+    """The NS entry points' 16-bit output dtypes (wide and tall, both forms):
+    the same 2e-2 bar against fp64 NS, and the 16-bit output equal to the fp32
+    output of the same call rounded to that dtype, up to one ulp of the fp32
+    result's own rounding order."""
+    gm = cuda_lib
+    X = _outlier_matrix(B, m, n, 61).to(DEV)
+    f = gm.gram_ns if form == "gram" else gm.newton_schulz
+    O32 = f(X)
+    O16 = f(X, out_dtype=odt)
+    torch.cuda.synchronize()
+    assert O16.dtype == odt
+    for b in range(B):
+        assert rel(O16[b], O.ns_standard(X[b].cpu().double())) <= 2e-2
+    assert rel(O16, O32.to(odt)) <= 1e-2
