@@ -1,0 +1,64 @@
+"""Host logic of bench.py that needs no GPU: the clock-sample summary that goes
+into the JSON line's ``clocks`` object, and the roofline denominators."""
+
+import json
+import os
+
+import bench
+
+
+def _sampler_with(tmp_path, lines):
+    s = bench.ClockSampler(0)
+    path = tmp_path / "clocks.csv"
+    path.write_text("\n".join(lines) + "\n")
+
+    class _F:
+        name = str(path)
+    s.file = _F()
+    return s
+
+
+def test_clock_summary_median_max_and_reasons(tmp_path):
+    # nvidia-smi --format=csv,noheader,nounits rows in the sampler's field order:
+    # index, clocks.sm, clocks.max.sm, power.draw, reasons bitmask, hw_slowdown,
+    # hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap
+    rows = [
+        "0, 1965, 1965, 410.20, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1860, 1965, 998.70, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1830, 1965, 1001.30, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, [N/A], 1965, [N/A], [N/A], [N/A], [N/A], [N/A], [N/A]",   # skipped: no clock
+        "garbage",                                                    # skipped: short row
+    ]
+    s = _sampler_with(tmp_path, rows)
+    out = s.summary()
+    assert out == {"sm_mhz": 1860.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                   "samples": 3}
+    assert not os.path.exists(s.file.name)          # the temporary file is removed
+
+
+def test_clock_summary_reports_every_slowdown_reason(tmp_path):
+    rows = [
+        "0, 1200, 1965, 700.0, 0x48, Active, Not Active, Not Active, Not Active",
+        "0, 1100, 1965, 700.0, 0x68, Not Active, Active, Active, Not Active",
+    ]
+    out = _sampler_with(tmp_path, rows).summary()
+    assert out["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+    assert out["sm_mhz"] == 1150.0
+
+
+def test_clock_summary_without_samples_is_none(tmp_path):
+    assert _sampler_with(tmp_path, ["0, [N/A], [N/A], 0, 0, x, x, x, x"]).summary() is None
+    s = bench.ClockSampler(0)
+    assert s.summary() is None                      # sampler never started
+
+
+def test_peaks_come_from_the_measured_file_when_present():
+    hbm, bf16, bf16_sus, kind = bench._peaks()
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                        "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        assert kind == "measured"
+        assert (hbm, bf16) == (d["hbm_gbs"], d["bf16_tflops"])
+    else:
+        assert kind == "fallback" and (hbm, bf16, bf16_sus) == (6650.0, 1590.0, 1400.0)
