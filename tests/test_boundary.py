@@ -1,0 +1,82 @@
+"""The product's boundary rules, checked on the host.
+
+* The Python binding is argument marshalling over libgmuon: importing it
+  without the built library fails loudly (no silent fallback of any kind).
+* The oracle is test infrastructure: nothing in the package imports it, and
+  bench.py imports it only inside the function that times the CPU baseline.
+* The oracle is independent of the CUDA path: it imports nothing from the
+  package or the bench, and no CUDA or C source includes anything of it.
+"""
+
+import ast
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+PKG = os.path.join(ROOT, "bit_muon_optimizer_b200")
+ORACLE = os.path.join(ROOT, "oracle")
+
+
+def _py_files(top):
+    for dirpath, _, files in os.walk(top):
+        for f in files:
+            if f.endswith(".py"):
+                yield os.path.join(dirpath, f)
+
+
+def _top_imports(node):
+    """Top-level package names imported anywhere under an AST node."""
+    names = set()
+    for n in ast.walk(node):
+        if isinstance(n, ast.Import):
+            names |= {a.name.split(".")[0] for a in n.names}
+        elif isinstance(n, ast.ImportFrom) and n.level == 0 and n.module:
+            names.add(n.module.split(".")[0])
+    return names
+
+
+def _parse(path):
+    with open(path) as f:
+        return ast.parse(f.read(), path)
+
+
+def test_binding_import_fails_loudly_without_the_library():
+    code = ("import os\n"
+            "real = os.path.exists\n"
+            "os.path.exists = lambda p: False if str(p).endswith('libgmuon.so') else real(p)\n"
+            "import bit_muon_optimizer_b200.gmuon\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "libgmuon.so is missing" in r.stderr
+
+
+def test_package_never_imports_the_oracle():
+    for path in _py_files(PKG):
+        assert "oracle" not in _top_imports(_parse(path)), path
+
+
+def test_bench_imports_the_oracle_only_for_the_cpu_baseline():
+    tree = _parse(os.path.join(ROOT, "bench.py"))
+    module_level = set()
+    for n in tree.body:
+        if isinstance(n, (ast.Import, ast.ImportFrom)):
+            module_level |= _top_imports(n)
+    assert "oracle" not in module_level
+    users = {f.name for f in ast.walk(tree)
+             if isinstance(f, ast.FunctionDef) and "oracle" in _top_imports(f)}
+    assert users == {"oracle_sample_seconds"}
+
+
+def test_oracle_is_independent_of_the_cuda_path():
+    for path in _py_files(ORACLE):
+        imps = _top_imports(_parse(path))
+        assert not imps & {"bit_muon_optimizer_b200", "bench", "__graft_entry__", "ctypes"}, path
+    for dirpath, _, files in os.walk(PKG):
+        for f in files:
+            if f.endswith((".cu", ".cuh", ".h", ".c", ".cpp")):
+                with open(os.path.join(dirpath, f)) as fh:
+                    for line in fh:
+                        if line.lstrip().startswith("#include"):
+                            assert "oracle" not in line, (f, line)
