@@ -284,6 +284,7 @@ gm_status gm_quant8(int B, int rows, int k, const float* X, int8_t* codes, float
   GM_CHECK_ARG(B >= 1 && B <= 65535 && rows >= 1 && rows <= (1 << 20), "bad B=%d rows=%d", B, rows);
   GM_CHECK_ARG(k >= 1 && k <= kMaxK, "k=%d out of [1, %d]", k, kMaxK);
   GM_CHECK_ARG(X && codes && colscale, "NULL pointer");
+  GM_CHECK_ARG(al16(X) && al16(codes) && al16(colscale), "device arrays must be 16-byte aligned");
   GM_DEVICE();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   GM_CUDA(launch_quant8(B, rows, 0, k, X, codes, colscale, nullptr, nullptr, nullptr, nullptr,

@@ -4,7 +4,9 @@
  * C ABI. Every pointer argument is a DEVICE pointer unless marked "host".
  * All matrices are row-major and batch-contiguous: a call operates on B
  * same-shape matrices stored back to back (batch stride = rows * cols).
- * Shapes: m, n multiples of 16, 16 <= m, n <= 65536; top rank 1 <= k <= 32.
+ * Shapes: batch 1 <= B <= 65535; m, n multiples of 16, 16 <= m, n <= 65536;
+ * top rank 1 <= k <= 32. An empty batch or matrix (B, m or n = 0) is an
+ * argument error (GM_E_ARG), not a no-op: a caller skips empty groups itself.
  * Every device array pointer must be 16-byte aligned (the kernels move
  * 16-byte vectors); a misaligned pointer returns GM_E_ARG.
  * The 4-bit grid uses fixed 128 x 128 blocks (ragged edge blocks allowed).
@@ -130,7 +132,8 @@ gm_status gm_grid_quant4(int B, int m, int n, int k, const float* X,
  * 8-bit per-column absmax quantization of P or R [GRASP, worked step 5;
  * training strategy: INT8 factors]:
  *   s_l = max_i |x_il|; q = clamp(rint(fp32(x / s_l) * 127), -127, 127); s = 0 -> 0.
- *   X f32 [B][rows][k] -> codes int8 [B][rows][k], colscale f32 [B][k].
+ *   X f32 [B][rows][k] -> codes int8 [B][rows][k], colscale f32 [B][k];
+ *   1 <= rows <= 2^20 (any count, not only multiples of 16).
  */
 gm_status gm_quant8(int B, int rows, int k, const float* X,
                     int8_t* codes, float* colscale, gm_stream_t stream);

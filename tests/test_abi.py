@@ -89,3 +89,33 @@ def test_misaligned_arrays_are_rejected_before_any_launch():
     assert r == gm.GM_E_ARG and b"aligned" in gm.lib.gm_last_error()
     r = gm.lib.gm_newton_schulz(1, 256, 512, bad, 1, None, 5, 1e-7, ok, 0, ok, 1 << 30, None)
     assert r == gm.GM_E_ARG
+    r = gm.lib.gm_quant8(1, 777, 3, ok, bad, ok, None)
+    assert r == gm.GM_E_ARG and b"aligned" in gm.lib.gm_last_error()
+
+
+@pytest.mark.parametrize("B,m,n", [(0, 256, 512), (65536, 256, 512), (1, 0, 512), (1, 256, 0),
+                                   (1, 8, 512), (1, 256, 65552), (1, 250, 512)])
+def test_empty_and_out_of_range_shapes_are_argument_errors(B, m, n):
+    """An empty batch or matrix is GM_E_ARG (not a silent no-op), as are sizes
+    outside 16 <= m, n <= 65536 (multiples of 16) and 1 <= B <= 65535; all
+    are caught on the host before any launch (this runs without a GPU)."""
+    ok = ctypes.c_void_p(4096)
+    prm = gm.GraspParams(0.95, 0.02, 0.0, 8, 5, 0, None, None, 0, 1e-7, 0)
+    st = gm.GraspStateC(*([4096] * 9))
+    calls = [
+        lambda: gm.lib.gm_grasp_step(B, m, n, ctypes.byref(prm), ctypes.byref(st), ok, ok, 1, ok,
+                                     1 << 40, None),
+        lambda: gm.lib.gm_newton_schulz(B, m, n, ok, 1, None, 5, 1e-7, ok, 0, ok, 1 << 40, None),
+        lambda: gm.lib.gm_grid_quant4(B, m, n, 0, ok, None, None, ok, ok, ok, None),
+        lambda: gm.lib.gm_dequant_rebuild(B, m, n, 0, ok, ok, ok, None, None, None, None, ok, None),
+    ]
+    for call in calls:
+        assert call() == gm.GM_E_ARG
+        assert b"shape" in gm.lib.gm_last_error()
+    assert gm.workspace_bytes(gm.GM_OP_GRASP_STEP, B, m, n, 8) == 0
+
+
+def test_quant8_row_range():
+    ok = ctypes.c_void_p(4096)
+    for B, rows in [(0, 16), (1, 0), (1, (1 << 20) + 1)]:
+        assert gm.lib.gm_quant8(B, rows, 8, ok, ok, ok, None) == gm.GM_E_ARG
