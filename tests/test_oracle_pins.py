@@ -330,6 +330,33 @@ def test_grid_quant4_brute_force_codes():
         assert torch.all(err <= s.double() / 14 * (1 + 1e-6) + 1e-30)
 
 
+@pytest.mark.parametrize("m,n,blk", [(13, 22, 8), (21, 10, 4), (9, 9, 16)])
+def test_grid_scales_brute_force_ragged(m, n, blk):
+    """Element by element with plain loops, on ragged edge blocks: s_ij is the
+    smaller of |x| maxima over row i and over column j, each taken only inside
+    the block that holds (i, j) ("Achieving low-bit Muon through subspace
+    preservation and grid quantization", key design 2); the oracle's row and
+    column scales and its per-element scale must match, and its dequantized
+    value must lie within half a step s_ij / 14 of x."""
+    gen = torch.Generator().manual_seed(20 + m * n)
+    X = (torch.randn(m, n, generator=gen) * torch.rand(1, n, generator=gen)).to(torch.float32)
+    X[m - 1, :] = 0.0
+    codes, rs, cs = O.grid_quant4(X, block=blk)
+    s_or = O.grid_scale_matrix(rs, cs, m, n, blk)
+    xh = O.grid_dequant4(codes, rs, cs, blk)
+    for i in range(m):
+        bi0 = (i // blk) * blk
+        for j in range(n):
+            bj0 = (j // blk) * blk
+            r = max(abs(float(X[i, c])) for c in range(bj0, min(n, bj0 + blk)))
+            c = max(abs(float(X[a, j])) for a in range(bi0, min(m, bi0 + blk)))
+            assert float(rs[i, j // blk]) == r
+            assert float(cs[i // blk, j]) == c
+            s = min(r, c)
+            assert float(s_or[i, j]) == s
+            assert abs(float(X[i, j]) - float(xh[i, j])) <= s / 14 * (1 + 1e-6)
+
+
 def test_grid_quant4_invariants():
     gen = torch.Generator().manual_seed(13)
     m, n, blk = 256, 384, 128
