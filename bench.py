@@ -177,18 +177,43 @@ def oracle_sample_seconds(w: WL.Workload, ns: str, budget_s: float):
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the fp64 CPU oracle as it stands, on this host's cores.
+
+    Each step (warm-up or timed) is one oracle step of one sample matrix of
+    every shape group, with each sample's state and weight carried from step
+    to step, so the timed steps start from a warm quantized state like the
+    GPU arm's; the step's time per parameter set is sum over groups of
+    (matrices in the group) x (the sample's step time). The whole run costs
+    (W + K) times one oracle step per group, about 0.4 s a step for LLaMA-130M.
+    Only rank 0 works; the other ranks return at once."""
     if rank != 0:
         return
+    import oracle as O
     w = WL.WORKLOADS[args.config]
-    budget = max(3.0, 90.0 / max(1, args.steps + args.warmup))
+    samples = []
+    for gi, g in enumerate(w.groups):
+        b = w.group_base(gi)
+        samples.append([g, b, O.zero_state(g.m, g.n, w.k), WL.initial_weight(w, b, g.m, g.n)])
     vals = []
-    sample = ""
-    cores = torch.get_num_threads()
     for i in range(args.warmup + args.steps):
-        ms, sample, cores = oracle_sample_seconds(w, args.ns, budget)
+        t = i + 1
+        ms = 0.0
+        for smp in samples:
+            g, b, st, W = smp
+            G = WL.gradient(w, b, t, g.m, g.n)
+            t0 = time.perf_counter()
+            r = O.grasp_step(st, W, G, mu=w.mu, eta=w.eta, wd=w.wd, seed=w.seed, b=0, ns=args.ns,
+                             T=w.T)
+            ms += 1e3 * g.count * (time.perf_counter() - t0)
+            smp[2], smp[3] = r.state, r.W.float()
         if i >= args.warmup:
             vals.append(ms)
     v = statistics.median(vals)
+    cores = torch.get_num_threads()
+    sample = ("fp64 oracle, one matrix per shape group ("
+              + ", ".join(f"{g.m}x{g.n}" for g, _, _, _ in samples)
+              + "), one step of each per reference step from a state carried across steps, "
+              "extrapolated by the group counts; median over the timed steps")
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
