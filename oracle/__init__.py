@@ -1,8 +1,8 @@
 """Plain, slow fp64 CPU oracle of one 4-bit-Muon-GRASP optimizer step.
 
 TEST INFRASTRUCTURE ONLY. Nothing in the product path imports this package:
-only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
-``bench.py`` may use it. It shares no code with the CUDA library; the only
+only ``tests/``, ``__graft_entry__.smoke()`` and the two legs of ``bench.py``
+that time the oracle (the CPU baseline and the reference arm) may use it. It shares no code with the CUDA library; the only
 module both sides use is the seeded input generator
 (``bit_muon_optimizer_b200.workloads``), which holds none of the method's
 arithmetic.

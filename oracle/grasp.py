@@ -24,6 +24,9 @@ Readings of points the pages leave open:
 * The residual uses the unquantized new P and R.
 * NS runs on the fp64 momentum of this step; tall matrices (rows > cols) are
   transposed first, square ones are not.
+* The 4bit-Muon-base codec the note compares against quantizes the whole
+  matrix in groups of 128 consecutive row-major elements, one absmax scale
+  per group, codes in [-7, 7] like the grid codec.
 """
 
 from __future__ import annotations
@@ -50,7 +53,7 @@ __all__ = [
     "splitmix64", "rademacher_sign", "rademacher_column", "warm_start",
     "orth_positive", "power_iteration",
     "quant8", "dequant8", "grid_quant4", "grid_scale_matrix", "grid_dequant4",
-    "pack_nibbles", "unpack_nibbles",
+    "pack_nibbles", "unpack_nibbles", "group_quant4", "group_dequant4",
     "ns_standard", "gram_ns", "quintic_scalar",
     "GraspState", "zero_state", "rebuild_momentum", "grasp_step",
 ]
@@ -224,6 +227,36 @@ def grid_dequant4(codes, rscale, cscale, block: int = GRID_BLOCK) -> torch.Tenso
     m, n = codes.shape
     s = grid_scale_matrix(rscale, cscale, m, n, block).to(DT)
     return codes.to(DT) / 7.0 * s
+
+
+def group_quant4(X: torch.Tensor, group: int = 128):
+    """The 4bit-Muon-base codec the GRASP note compares against (its results
+    tables' "4bit-Muon-base" rows; the motivation's direct quantization of
+    Muon's momentum): blockwise 4-bit of the whole matrix with one absmax
+    scale per group of `group` consecutive elements in row-major order (a
+    shorter last group when the count is not a multiple of `group`);
+    q = clamp(rint(fp32(x / s) * 7), -7, 7), s = 0 giving 0.
+
+    Returns (codes int8 (m, n), scales fp32 (ceil(m n / group),))."""
+    x = X.to(F32).reshape(-1)
+    ng = -(-x.numel() // group)
+    scales = torch.zeros(ng, dtype=F32)
+    codes = torch.zeros(x.numel(), dtype=torch.int8)
+    for gi in range(ng):
+        seg = x[gi * group:(gi + 1) * group]
+        s = seg.abs().max()
+        scales[gi] = s
+        if s > 0:
+            r = (seg / s) * torch.tensor(7.0, dtype=F32)
+            codes[gi * group:(gi + 1) * group] = torch.clamp(torch.round(r), -7, 7).to(torch.int8)
+    return codes.view(X.shape), scales
+
+
+def group_dequant4(codes: torch.Tensor, scales: torch.Tensor, group: int = 128) -> torch.Tensor:
+    """x^ = (q / 7) * s of the element's group, in fp64."""
+    q = codes.reshape(-1).to(DT)
+    s = scales.to(DT).repeat_interleave(group)[: q.numel()]
+    return (q / 7.0 * s).view(codes.shape)
 
 
 def pack_nibbles(codes: torch.Tensor) -> torch.Tensor:
