@@ -105,6 +105,26 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _expect(t, shape, dtypes, name):
+    """Checks the shape (a [m, n] matrix also stands for a batch of one) and
+    dtype of a tensor handed to the library as a raw pointer."""
+    shape = tuple(shape)
+    got = tuple(t.shape)
+    if got != shape and not (len(shape) == 3 and shape[0] == 1 and got == shape[1:]):
+        raise ValueError(f"{name}: expected shape {shape}, got {got}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype} is not one of {tuple(dtypes)}")
+
+
+def _placed(tensors, names):
+    """Checks that tensors are contiguous CUDA tensors."""
+    for t, name in zip(tensors, names):
+        if not t.is_cuda:
+            raise ValueError(f"{name}: expected a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: expected a contiguous tensor")
+
+
 def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
@@ -285,6 +305,23 @@ class GraspState:
         return [self.codes4, self.rscale, self.cscale, self.P8, self.Pscale, self.R8,
                 self.Rscale, self.step, self.dev_status]
 
+    def check(self, B, m, n, k):
+        """Raises ValueError unless every tensor has the layout gm_grasp_step
+        reads and writes for B matrices of m x n at top rank k."""
+        mb, nb = -(-m // GRID_BLOCK), -(-n // GRID_BLOCK)
+        f32, i8 = (torch.float32,), (torch.int8,)
+        _expect(self.codes4, (B, m, n // 2), (torch.uint8,), "codes4")
+        _expect(self.rscale, (B, m, nb), f32, "rscale")
+        _expect(self.cscale, (B, mb, n), f32, "cscale")
+        _expect(self.P8, (B, m, k), i8, "P8")
+        _expect(self.Pscale, (B, k), f32, "Pscale")
+        _expect(self.R8, (B, n, k), i8, "R8")
+        _expect(self.Rscale, (B, k), f32, "Rscale")
+        _expect(self.step, (1,), (torch.int64,), "step")
+        _expect(self.dev_status, (1,), (torch.int32,), "dev_status")
+        _placed(self.tensors(), ["codes4", "rscale", "cscale", "P8", "Pscale", "R8", "Rscale",
+                                 "step", "dev_status"])
+
     def c_struct(self):
         return GraspStateC(*[t.data_ptr() for t in self.tensors()])
 
@@ -316,6 +353,11 @@ class GraspStep:
         self.ns = ns
 
     def __call__(self, state: GraspState, W, G):
+        B, m, n = self.B, self.m, self.n
+        _expect(W, (B, m, n), (torch.float32,), "W")
+        _expect(G, (B, m, n), tuple(_DT), "G")
+        state.check(B, m, n, self.k)
+        _placed((W, G), ("W", "G"))
         st = state.c_struct()
         _check(lib.gm_grasp_step(self.B, self.m, self.n, ctypes.byref(self.params), ctypes.byref(st),
                                  _ptr(W), _ptr(G), _DT[G.dtype], _ptr(self.ws), self.ws_bytes,

@@ -81,3 +81,33 @@ def test_oracle_is_independent_of_the_cuda_path():
                     for line in fh:
                         if line.lstrip().startswith("#include"):
                             assert "oracle" not in line, (f, line)
+
+
+def test_step_binding_checks_tensors_before_passing_pointers():
+    """GraspStep hands W, G and the state to the library as raw pointers, so
+    the binding checks their shapes, dtypes, device and layout first; every
+    call here is rejected in Python, before the library is reached."""
+    import pytest
+    import torch
+
+    from bit_muon_optimizer_b200 import gmuon as gm
+    B, m, n, k = 2, 64, 96, 8
+    step = gm.GraspStep(B, m, n, k, ws=torch.empty(0, dtype=torch.uint8))
+    st = gm.GraspState.zeros(B, m, n, k, device="cpu")
+    W = torch.zeros(B, m, n)
+    G = torch.zeros(B, m, n, dtype=torch.bfloat16)
+    bad = [
+        (st, torch.zeros(B, m, n + 16), G, "W: expected shape"),
+        (st, W, torch.zeros(B, m, n, dtype=torch.float64), "G: dtype"),
+        (st, W.double(), G, "W: dtype"),
+        (gm.GraspState.zeros(B, m, n, k + 1, device="cpu"), W, G, "P8: expected shape"),
+        (gm.GraspState.zeros(B + 1, m, n, k, device="cpu"), W, G, "codes4: expected shape"),
+        (st, W, G, "expected a CUDA tensor"),               # right layout, host memory
+    ]
+    for state, w_, g_, msg in bad:
+        with pytest.raises(ValueError, match=msg):
+            step(state, w_, g_)
+    # a batch of one also takes plain [m, n] matrices
+    one = gm.GraspStep(1, m, n, k, ws=torch.empty(0, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="expected a CUDA tensor"):
+        one(gm.GraspState.zeros(1, m, n, k, device="cpu"), torch.zeros(m, n), torch.zeros(m, n))
