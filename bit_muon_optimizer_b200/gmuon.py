@@ -110,10 +110,17 @@ def _expect(t, shape, dtypes, name):
     dtype of a tensor handed to the library as a raw pointer."""
     shape = tuple(shape)
     got = tuple(t.shape)
-    if got != shape and not (len(shape) == 3 and shape[0] == 1 and got == shape[1:]):
+    if got != shape and not (len(shape) >= 2 and shape[0] == 1 and got == shape[1:]):
         raise ValueError(f"{name}: expected shape {shape}, got {got}")
     if t.dtype not in dtypes:
         raise ValueError(f"{name}: dtype {t.dtype} is not one of {tuple(dtypes)}")
+
+
+def _ws_fits(ws, nbytes, name="ws"):
+    """Checks that a caller-supplied workspace holds at least `nbytes`."""
+    have = ws.numel() * ws.element_size()
+    if have < nbytes:
+        raise ValueError(f"{name}: {have} bytes, the call needs {nbytes}")
 
 
 def _placed(tensors, names):
@@ -178,8 +185,18 @@ def dequant_rebuild(codes4, rscale, cscale, P8=None, Pscale=None, R8=None, Rscal
     B, m, n2 = _bmn(codes4)
     n = 2 * n2
     k = 0 if P8 is None else P8.shape[-1]
+    mb, nb = -(-m // GRID_BLOCK), -(-n // GRID_BLOCK)
+    _expect(codes4, (B, m, n2), (torch.uint8,), "codes4")
+    _expect(rscale, (B, m, nb), (torch.float32,), "rscale")
+    _expect(cscale, (B, mb, n), (torch.float32,), "cscale")
+    if k:
+        _expect(P8, (B, m, k), (torch.int8,), "P8")
+        _expect(Pscale, (B, k), (torch.float32,), "Pscale")
+        _expect(R8, (B, n, k), (torch.int8,), "R8")
+        _expect(Rscale, (B, k), (torch.float32,), "Rscale")
     if out is None:
         out = torch.empty((B, m, n), dtype=torch.float32, device=codes4.device)
+    _expect(out, (B, m, n), (torch.float32,), "out")
     _check(lib.gm_dequant_rebuild(B, m, n, k, _ptr(codes4), _ptr(rscale), _ptr(cscale), _ptr(P8),
                                   _ptr(Pscale), _ptr(R8), _ptr(Rscale), _ptr(out), _stream()),
            "gm_dequant_rebuild")
@@ -188,6 +205,11 @@ def dequant_rebuild(codes4, rscale, cscale, P8=None, Pscale=None, R8=None, Rscal
 
 def momentum_powerit(G, k, mu=0.95, M_prev=None, R_prev=None, seed=0):
     B, m, n = _bmn(G)
+    _expect(G, (B, m, n), tuple(_DT), "G")
+    if M_prev is not None:
+        _expect(M_prev, (B, m, n), (torch.float32,), "M_prev")
+    if R_prev is not None:
+        _expect(R_prev, (B, n, k), (torch.float32,), "R_prev")
     dev = G.device
     M = torch.empty((B, m, n), dtype=torch.float32, device=dev)
     P = torch.empty((B, m, k), dtype=torch.float32, device=dev)
@@ -204,8 +226,17 @@ def grid_quant4(X, P=None, R=None, out=None):
     B, m, n = _bmn(X)
     dev = X.device
     k = 0 if P is None else P.shape[-1]
+    _expect(X, (B, m, n), (torch.float32,), "X")
+    if (P is None) != (R is None):
+        raise ValueError("P and R must both be given or both be None")
+    if k:
+        _expect(P, (B, m, k), (torch.float32,), "P")
+        _expect(R, (B, n, k), (torch.float32,), "R")
     if out is not None:
         codes, rs, cs = out
+        _expect(codes, (B, m, n // 2), (torch.uint8,), "codes")
+        _expect(rs, (B, m, -(-n // GRID_BLOCK)), (torch.float32,), "rscale")
+        _expect(cs, (B, -(-m // GRID_BLOCK), n), (torch.float32,), "cscale")
     else:
         codes = torch.empty((B, m, n // 2), dtype=torch.uint8, device=dev)
         rs = torch.empty((B, m, -(-n // GRID_BLOCK)), dtype=torch.float32, device=dev)
@@ -217,6 +248,7 @@ def grid_quant4(X, P=None, R=None, out=None):
 
 def quant8(X):
     B, rows, k = _bmn(X)
+    _expect(X, (B, rows, k), (torch.float32,), "X")
     codes = torch.empty((B, rows, k), dtype=torch.int8, device=X.device)
     scale = torch.empty((B, k), dtype=torch.float32, device=X.device)
     _check(lib.gm_quant8(B, rows, k, _ptr(X), _ptr(codes), _ptr(scale), _stream()), "gm_quant8")
@@ -225,10 +257,13 @@ def quant8(X):
 
 def newton_schulz(X, abc=None, T=5, eps=1e-7, out_dtype=torch.float32, out=None, ws=None):
     B, m, n = _bmn(X)
+    _expect(X, (B, m, n), tuple(_DT), "X")
     O = out if out is not None else torch.empty((B, m, n), dtype=out_dtype, device=X.device)
+    _expect(O, (B, m, n), tuple(_DT), "out")
     out_dtype = O.dtype
     nb = workspace_bytes(GM_OP_NEWTON_SCHULZ, B, m, n)
     ws = ws if ws is not None else workspace(nb, X.device)
+    _ws_fits(ws, nb)
     _check(lib.gm_newton_schulz(B, m, n, _ptr(X), _DT[X.dtype], abc_table(abc, T), T, eps,
                                 _ptr(O), _DT[out_dtype], _ptr(ws), nb, _stream()),
            "gm_newton_schulz")
@@ -243,7 +278,9 @@ def newton_schulz_noalloc(X, abc=None, T=5, eps=1e-7, out_dtype=torch.float32, o
     (its scratch is a fixed 64 MiB array inside the library). ``out`` must be
     preallocated by callers that cannot allocate either."""
     B, m, n = _bmn(X)
+    _expect(X, (B, m, n), tuple(_DT), "X")
     O = out if out is not None else torch.empty((B, m, n), dtype=out_dtype, device=X.device)
+    _expect(O, (B, m, n), tuple(_DT), "out")
     _check(lib.gm_newton_schulz_noalloc(B, m, n, _ptr(X), _DT[X.dtype], abc_table(abc, T), T, eps,
                                         _ptr(O), _DT[O.dtype], _stream()),
            "gm_newton_schulz_noalloc")
@@ -253,10 +290,13 @@ def newton_schulz_noalloc(X, abc=None, T=5, eps=1e-7, out_dtype=torch.float32, o
 def gram_ns(X, abc=None, T=5, restart_after=(2,), eps=1e-7, out_dtype=torch.float32, out=None,
             ws=None):
     B, m, n = _bmn(X)
+    _expect(X, (B, m, n), tuple(_DT), "X")
     O = out if out is not None else torch.empty((B, m, n), dtype=out_dtype, device=X.device)
+    _expect(O, (B, m, n), tuple(_DT), "out")
     out_dtype = O.dtype
     nb = workspace_bytes(GM_OP_GRAM_NS, B, m, n)
     ws = ws if ws is not None else workspace(nb, X.device)
+    _ws_fits(ws, nb)
     rl = list(restart_after)
     rarr = (c_int * max(1, len(rl)))(*rl) if rl else None
     _check(lib.gm_gram_ns(B, m, n, _ptr(X), _DT[X.dtype], abc_table(abc, T), T, rarr, len(rl),
@@ -358,6 +398,7 @@ class GraspStep:
         _expect(G, (B, m, n), tuple(_DT), "G")
         state.check(B, m, n, self.k)
         _placed((W, G), ("W", "G"))
+        _ws_fits(self.ws, self.ws_bytes)
         st = state.c_struct()
         _check(lib.gm_grasp_step(self.B, self.m, self.n, ctypes.byref(self.params), ctypes.byref(st),
                                  _ptr(W), _ptr(G), _DT[G.dtype], _ptr(self.ws), self.ws_bytes,

@@ -111,3 +111,37 @@ def test_step_binding_checks_tensors_before_passing_pointers():
     one = gm.GraspStep(1, m, n, k, ws=torch.empty(0, dtype=torch.uint8))
     with pytest.raises(ValueError, match="expected a CUDA tensor"):
         one(gm.GraspState.zeros(1, m, n, k, device="cpu"), torch.zeros(m, n), torch.zeros(m, n))
+
+
+def test_entry_point_bindings_check_tensors_before_passing_pointers():
+    import pytest
+    import torch
+
+    from bit_muon_optimizer_b200 import gmuon as gm
+    B, m, n, k = 2, 64, 256, 8
+    f = lambda *s: torch.zeros(*s)                                   # noqa: E731
+    st = gm.GraspState.zeros(B, m, n, k, device="cpu")
+    parts = [st.codes4, st.rscale, st.cscale, st.P8, st.Pscale, st.R8, st.Rscale]
+    cases = [
+        (lambda: gm.dequant_rebuild(st.codes4, f(B, m, 1), *parts[2:]), "rscale: expected shape"),
+        (lambda: gm.dequant_rebuild(*parts[:5], st.R8[:, :-16], st.Rscale), "R8: expected shape"),
+        (lambda: gm.dequant_rebuild(*parts, out=f(B, m, n - 16)), "out: expected shape"),
+        (lambda: gm.momentum_powerit(f(B, m, n), k, M_prev=f(B, m, n + 16)), "M_prev: expected"),
+        (lambda: gm.momentum_powerit(f(B, m, n), k, R_prev=f(B, n, k + 1)), "R_prev: expected"),
+        (lambda: gm.momentum_powerit(f(B, m, n).double(), k), "G: dtype"),
+        (lambda: gm.grid_quant4(f(B, m, n), f(B, m, k)), "both be given"),
+        (lambda: gm.grid_quant4(f(B, m, n), f(B, m, k), f(B, n + 16, k)), "R: expected shape"),
+        (lambda: gm.grid_quant4(f(B, m, n).half()), "X: dtype"),
+        (lambda: gm.quant8(f(B, m, k).double()), "X: dtype"),
+        (lambda: gm.newton_schulz(f(B, m, n), out=f(B, n, m)), "out: expected shape"),
+        (lambda: gm.newton_schulz(f(B, m, n), ws=torch.empty(16, dtype=torch.uint8)), "ws: 16 bytes"),
+        (lambda: gm.gram_ns(f(B, m, n).double()), "X: dtype"),
+        (lambda: gm.newton_schulz_noalloc(f(B, m, n), out=f(B, m, n).double()), "out: dtype"),
+        # right shapes and dtypes, host memory: stopped before the library call
+        (lambda: gm.dequant_rebuild(*parts), "expected a CUDA tensor"),
+        (lambda: gm.grid_quant4(f(B, m, n), f(B, m, k), f(B, n, k)), "expected a CUDA tensor"),
+        (lambda: gm.quant8(f(B, m, k)), "expected a CUDA tensor"),
+    ]
+    for call, msg in cases:
+        with pytest.raises(ValueError, match=msg):
+            call()
