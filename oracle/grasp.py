@@ -54,7 +54,7 @@ __all__ = [
     "orth_positive", "power_iteration",
     "quant8", "dequant8", "grid_quant4", "grid_scale_matrix", "grid_dequant4",
     "pack_nibbles", "unpack_nibbles", "group_quant4", "group_dequant4",
-    "ns_standard", "gram_ns", "quintic_scalar",
+    "ns_standard", "gram_ns", "quintic_scalar", "POLAR_EXPRESS_ABC", "safety_scaled",
     "GraspState", "zero_state", "rebuild_momentum", "grasp_step",
 ]
 
@@ -307,13 +307,18 @@ def ns_standard(X: torch.Tensor, abc=None, T: int = 5, eps: float = NS_EPS) -> t
 
 
 def gram_ns(X: torch.Tensor, abc=None, T: int = 5, restart_after=(2,),
-            eps: float = NS_EPS) -> torch.Tensor:
+            eps: float = NS_EPS, trace: list | None = None) -> torch.Tensor:
     """Gram Newton-Schulz [GramNS, Algorithm 2; Algorithm 1 when no restart].
 
     X <- X / (|X|_F + eps); R = X X^T; Q = I; for each step
     Z = b R + c R^2, Q <- Q Z + a Q, RZ = R Z + a R, R <- Z RZ + a RZ.
     After each step listed in ``restart_after`` (1-based, before the last
     step): X <- Q X, R <- X X^T, Q <- I. Returns Q X.
+
+    With a list as ``trace``, every step t appends (t, smallest eigenvalue of
+    R_t, condition number of Q_t), taken after the step's update and before
+    any restart: the two quantities [GramNS §3.2] bounds for its restart
+    choice.
     """
     if abc is None:
         abc = [QUINTIC_ABC] * T
@@ -329,12 +334,29 @@ def gram_ns(X: torch.Tensor, abc=None, T: int = 5, restart_after=(2,),
         Q = Q @ Z + a * Q
         RZ = R @ Z + a * R
         R = Z @ RZ + a * RZ
+        if trace is not None:
+            sq = torch.linalg.svdvals(Q)
+            trace.append((t, float(torch.linalg.eigvalsh(R)[0]), float(sq[0] / sq[-1])))
         if t in restart_after and t < T:
             Y = Q @ Y
             R = Y @ Y.T
             Q = I.clone()
     O = Q @ Y
     return O.T if tall else O
+
+
+#: The Polar Express quintics as printed in [GramNS §3.2] (one per step).
+POLAR_EXPRESS_ABC = ((8.123737, -22.232240, 16.373715), (4.026529, -2.776323, 0.514551),
+                     (3.870284, -2.739120, 0.520999), (3.253351, -2.343223, 0.481420),
+                     (2.300652, -1.668904, 0.418807))
+
+
+def safety_scaled(abc, s: float = 1.05):
+    """A coefficient table whose every step evaluates p_t(x / s): (a / s,
+    b / s^3, c / s^5). Reading of the safety factor of [GramNS §3.3], whose
+    formula (eq. (12)) is lost from the page: only its purpose, convergence
+    for singular values up to 1.05, survives."""
+    return [(a / s, b / s ** 3, c / s ** 5) for a, b, c in abc]
 
 
 def quintic_scalar(x: float, abc=None, T: int = 5) -> float:

@@ -160,6 +160,84 @@ def test_gram_ns_negative_eigenvalue_grows():
     assert abs(float(R[0, 0]) - 1.0) < 0.05
 
 
+def _composed(x, abc):
+    for a, b, c in abc:
+        x = a * x + b * x ** 3 + c * x ** 5
+    return x
+
+
+@pytest.mark.parametrize("restart", [(), (2,), (1, 3)])
+def test_gram_ns_trace_closed_form(restart):
+    """In exact arithmetic every iterate keeps X_0's singular vectors [GramNS
+    Prop. 1, Theorem 1], so for X = U S V^T with normalised values s_i: R_t
+    has eigenvalues f_t(s_i)^2 (f_t the first t polynomials composed) and Q_t,
+    which maps the iterate at the last restart r (r = 0 at the start) to
+    X_t, is U diag(f_t(s_i) / f_r(s_i)) U^T. The trace's smallest eigenvalue
+    of R_t and condition number of Q_t must follow."""
+    gen = torch.Generator().manual_seed(40)
+    m, n = 24, 40
+    U = _orthogonal(m, gen)
+    V = _orthogonal(n, gen)[:, :m]
+    s = torch.logspace(0, -3, m, dtype=DT)
+    X = U @ torch.diag(s) @ V.T
+    abc = O.safety_scaled(O.POLAR_EXPRESS_ABC)
+    tr = []
+    O.gram_ns(X, abc=abc, restart_after=restart, trace=tr)
+    sh = s / (torch.linalg.matrix_norm(X) + O.NS_EPS)
+    r = 0
+    for t, lam, cond in tr:
+        ft = _composed(sh, abc[:t])
+        fr = _composed(sh, abc[:r])
+        ratio = ft / fr
+        assert lam == pytest.approx(float((ft * ft).min()), rel=1e-6, abs=1e-12)
+        assert cond == pytest.approx(float(ratio.max() / ratio.min()), rel=1e-6)
+        if t in restart:
+            r = t
+
+
+def test_polar_express_table_and_safety_factor_reading():
+    """The Polar Express quintics printed in [GramNS §3.2] diverge as printed
+    for singular values near 1 (the first maps 1 to 2.27); with the lost
+    safety factor read as evaluating every step at x / 1.05 [GramNS §3.3],
+    every normalised singular value in [1e-3, 1] lands in [0.68, 1.13]."""
+    pe = O.POLAR_EXPRESS_ABC
+    assert _composed(1.0, pe) > 1e6
+    scaled = O.safety_scaled(pe, 1.05)
+    xs = torch.cat([torch.logspace(-3, 0, 4001, dtype=DT)])
+    y = _composed(xs, scaled)
+    assert 0.68 < float(y.min()) and float(y.max()) < 1.13
+    # the scaled coefficients evaluate each printed polynomial at x / 1.05
+    gen = torch.Generator().manual_seed(41)
+    x = torch.rand(50, generator=gen, dtype=DT) * 1.2
+    for (a, b, c), (a2, b2, c2) in zip(pe, scaled):
+        z = x / 1.05
+        assert torch.allclose(a2 * x + b2 * x ** 3 + c2 * x ** 5, a * z + b * z ** 3 + c * z ** 5,
+                              rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("smallest", [1e-3, 1e-4])
+def test_restart_after_step_two_bounds_cond_q(smallest):
+    """[GramNS §3.2]: with the Polar Express quintics, restarting after the
+    second step keeps the condition number of Q_t below about 100. In exact
+    arithmetic (no rounding) this already separates the two schedules on an
+    input whose singular values fall to `smallest`: with the restart every
+    cond(Q_t) stays below 100, without it some cond(Q_t) exceeds 100."""
+    gen = torch.Generator().manual_seed(42)
+    m, n = 24, 40
+    U = _orthogonal(m, gen)
+    V = _orthogonal(n, gen)[:, :m]
+    X = U @ torch.diag(torch.logspace(0, math.log10(smallest), m, dtype=DT)) @ V.T
+    abc = O.safety_scaled(O.POLAR_EXPRESS_ABC)
+    with_restart, without = [], []
+    O.gram_ns(X, abc=abc, restart_after=(2,), trace=with_restart)
+    O.gram_ns(X, abc=abc, restart_after=(), trace=without)
+    assert max(c for _, _, c in with_restart) < 100
+    assert max(c for _, _, c in without) > 100
+    # and R_t stays positive semidefinite in exact arithmetic (the negative
+    # eigenvalues the page bounds by -0.4 come from rounding)
+    assert min(lam for _, lam, _ in with_restart + without) > -1e-12
+
+
 # ------------------------------------------------------------ FLOP counters
 
 def test_flop_counters_match_printed_savings():
