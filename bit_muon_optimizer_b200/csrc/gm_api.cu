@@ -292,6 +292,27 @@ gm_status gm_quant8(int B, int rows, int k, const float* X, int8_t* codes, float
   return GM_OK;
 }
 
+gm_status gm_group_quant4(int B, int m, int n, const float* X, uint8_t* codes4, float* gscale,
+                          gm_stream_t stream) {
+  GM_CHECK_ARG(shape_ok(B, m, n), "bad shape B=%d m=%d n=%d", B, m, n);
+  GM_CHECK_ARG(X && codes4 && gscale, "NULL pointer");
+  GM_CHECK_ARG(al16(X) && al16(codes4) && al16(gscale), "device arrays must be 16-byte aligned");
+  GM_DEVICE();
+  GM_CUDA(launch_group_quant4(B, m, n, X, codes4, gscale, reinterpret_cast<cudaStream_t>(stream)));
+  return GM_OK;
+}
+
+gm_status gm_group_dequant4(int B, int m, int n, const uint8_t* codes4, const float* gscale,
+                            float* X_out, gm_stream_t stream) {
+  GM_CHECK_ARG(shape_ok(B, m, n), "bad shape B=%d m=%d n=%d", B, m, n);
+  GM_CHECK_ARG(codes4 && gscale && X_out, "NULL pointer");
+  GM_CHECK_ARG(al16(codes4) && al16(gscale) && al16(X_out), "device arrays must be 16-byte aligned");
+  GM_DEVICE();
+  GM_CUDA(launch_group_dequant4(B, m, n, codes4, gscale, X_out,
+                                reinterpret_cast<cudaStream_t>(stream)));
+  return GM_OK;
+}
+
 static gm_status ns_common(int B, int m, int n, const void* X, gm_dtype xdt, const float* abc,
                            int T, const int* restart_after, int n_restart, float eps, void* O,
                            gm_dtype odt, void* ws, size_t ws_bytes, gm_stream_t stream, bool gram) {

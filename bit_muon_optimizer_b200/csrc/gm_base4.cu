@@ -1,0 +1,112 @@
+// The 4bit-Muon-base codec: blockwise 4-bit quantization of the whole
+// momentum matrix, the direct quantization of Muon's state that the GRASP
+// note ("Achieving low-bit Muon through subspace preservation and grid
+// quantization") measures its own codec against.
+//
+// Layout: groups of 128 consecutive row-major elements, one absmax scale each.
+// m and n are multiples of 16, so m n is a multiple of 256: no group is ragged
+// or straddles two matrices of the batch, and the batch is one flat run of
+// B m n / 128 groups.
+//
+// Both passes are HBM-bound (4.53 B per element in total): one warp owns one
+// group at a time, lane l holds its elements 4l .. 4l + 3 as one float4, so a
+// warp moves the group's 512 bytes in one coalesced request and its 64 code
+// bytes as 32 two-byte stores. A grid of eight CTAs per SM walks the groups.
+
+#include "gm_common.cuh"
+#include "gm_internal.h"
+
+namespace gm {
+namespace {
+
+constexpr int kGroup = 128;
+constexpr int kB4Threads = 256;
+constexpr int kB4Warps = kB4Threads / 32;
+constexpr int kB4MaxBlocks = 8 * 148;
+
+// q = clamp(rint(fp32(x / s) * 7), -7, 7) for |x| <= s, as a nibble. The
+// product z = x * fl(7 / s) differs from fl(x / s) * 7 by a few units in the
+// last place, so away from a rounding tie (|z - rint(z)| < 0.5 - 2^-16) both
+// round alike; near one the IEEE division decides.
+__device__ __forceinline__ uint32_t code4(float x, float s, float r7) {
+  const float z = __fmul_rn(x, r7), zr = rintf(z);
+  int q;
+  if (fabsf(__fsub_rn(z, zr)) < 0.49998474f)   // 0.5 - 2^-16
+    q = (int)zr;
+  else
+    q = (int)rintf(__fmul_rn(__fdiv_rn(x, s), 7.0f));
+  q = max(-7, min(7, q));
+  return (uint32_t)q & 0xFu;
+}
+
+__global__ void __launch_bounds__(kB4Threads) k_group_quant4(long long ngroups,
+                                                              const float* __restrict__ X,
+                                                              uint8_t* __restrict__ codes4,
+                                                              float* __restrict__ gscale) {
+  const int lane = threadIdx.x & 31;
+  const long long stride = (long long)gridDim.x * kB4Warps;
+  for (long long g = (long long)blockIdx.x * kB4Warps + (threadIdx.x >> 5); g < ngroups;
+       g += stride) {
+    const float4 v = reinterpret_cast<const float4*>(X)[g * 32 + lane];
+    // |x| as unsigned bits orders like the values, and a NaN (above every
+    // other pattern) carries into the scale: its group then keeps code 0
+    const uint32_t a = max(max(__float_as_uint(fabsf(v.x)), __float_as_uint(fabsf(v.y))),
+                           max(__float_as_uint(fabsf(v.z)), __float_as_uint(fabsf(v.w))));
+    const float s = __uint_as_float(__reduce_max_sync(0xffffffffu, a));
+    uint32_t w = 0;
+    if (s > 0.f) {
+      const float r7 = __fdiv_rn(7.0f, s);
+      // element 4 lane + e sits in nibble e: low nibble = even column
+      w = code4(v.x, s, r7) | (code4(v.y, s, r7) << 4) | (code4(v.z, s, r7) << 8) |
+          (code4(v.w, s, r7) << 12);
+    }
+    reinterpret_cast<uint16_t*>(codes4)[g * 32 + lane] = (uint16_t)w;
+    if (lane == 0) gscale[g] = s;
+  }
+}
+
+__global__ void __launch_bounds__(kB4Threads) k_group_dequant4(long long ngroups,
+                                                                const uint8_t* __restrict__ codes4,
+                                                                const float* __restrict__ gscale,
+                                                                float* __restrict__ X) {
+  __shared__ float deq[16];   // fl(q / 7) for the nibble q (two's complement)
+  if (threadIdx.x < 16)
+    deq[threadIdx.x] = __fdiv_rn((float)((threadIdx.x & 8) ? (int)threadIdx.x - 16 : (int)threadIdx.x),
+                                 7.0f);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const long long stride = (long long)gridDim.x * kB4Warps;
+  for (long long g = (long long)blockIdx.x * kB4Warps + (threadIdx.x >> 5); g < ngroups;
+       g += stride) {
+    const float s = gscale[g];
+    const uint32_t w = reinterpret_cast<const uint16_t*>(codes4)[g * 32 + lane];
+    float4 o;
+    o.x = __fmul_rn(deq[w & 0xF], s);
+    o.y = __fmul_rn(deq[(w >> 4) & 0xF], s);
+    o.z = __fmul_rn(deq[(w >> 8) & 0xF], s);
+    o.w = __fmul_rn(deq[(w >> 12) & 0xF], s);
+    reinterpret_cast<float4*>(X)[g * 32 + lane] = o;
+  }
+}
+
+int base4_blocks(long long ngroups) {
+  return (int)max(1LL, min((long long)kB4MaxBlocks, cdivll(ngroups, kB4Warps)));
+}
+
+}  // namespace
+
+cudaError_t launch_group_quant4(int B, int m, int n, const float* X, uint8_t* codes4,
+                                float* gscale, cudaStream_t s) {
+  const long long ngroups = (long long)B * m * n / kGroup;
+  k_group_quant4<<<base4_blocks(ngroups), kB4Threads, 0, s>>>(ngroups, X, codes4, gscale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_group_dequant4(int B, int m, int n, const uint8_t* codes4, const float* gscale,
+                                  float* X, cudaStream_t s) {
+  const long long ngroups = (long long)B * m * n / kGroup;
+  k_group_dequant4<<<base4_blocks(ngroups), kB4Threads, 0, s>>>(ngroups, codes4, gscale, X);
+  return cudaGetLastError();
+}
+
+}  // namespace gm

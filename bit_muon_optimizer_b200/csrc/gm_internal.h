@@ -78,6 +78,13 @@ cudaError_t launch_quant8(int B, int rows0, int rows1, int k, const float* X0, i
                           float* s0, const float* X1, int8_t* c1, float* s1,
                           int64_t* step, const int32_t* skip, cudaStream_t s);
 
+// The 4bit-Muon-base group codec (gm_base4.cu): 128 consecutive elements per
+// absmax scale, codes packed as in the grid codec.
+cudaError_t launch_group_quant4(int B, int m, int n, const float* X, uint8_t* codes4,
+                                float* gscale, cudaStream_t s);
+cudaError_t launch_group_dequant4(int B, int m, int n, const uint8_t* codes4, const float* gscale,
+                                  float* X, cudaStream_t s);
+
 // Standalone NS input: scale = 1/(|X|_F + eps) per matrix, then the wide
 // 16-bit copy Y = round(scale * X) (transposed when m > n).
 cudaError_t launch_ns_prep(int B, int m, int n, const void* X, int xdt, float eps,

@@ -68,6 +68,8 @@ _sig("gm_momentum_powerit", c_int, [c_int, c_int, c_int, c_int, c_float, vp, vp,
                                     c_uint64, vp, vp, vp, vp, c_size_t, vp])
 _sig("gm_grid_quant4", c_int, [c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, vp])
 _sig("gm_quant8", c_int, [c_int, c_int, c_int, vp, vp, vp, vp])
+_sig("gm_group_quant4", c_int, [c_int, c_int, c_int, vp, vp, vp, vp])
+_sig("gm_group_dequant4", c_int, [c_int, c_int, c_int, vp, vp, vp, vp])
 _sig("gm_newton_schulz", c_int, [c_int, c_int, c_int, vp, c_int, vp, c_int, c_float, vp, c_int,
                                  vp, c_size_t, vp])
 _sig("gm_newton_schulz_noalloc", c_int, [c_int, c_int, c_int, vp, c_int, vp, c_int, c_float, vp,
@@ -253,6 +255,40 @@ def quant8(X):
     scale = torch.empty((B, k), dtype=torch.float32, device=X.device)
     _check(lib.gm_quant8(B, rows, k, _ptr(X), _ptr(codes), _ptr(scale), _stream()), "gm_quant8")
     return codes, scale
+
+
+GROUP = 128   # elements per scale of the 4bit-Muon-base codec
+
+
+def group_quant4(X, out=None):
+    """4bit-Muon-base codes of fp32 [B, m, n] (or [m, n]): (codes [B, m, n/2]
+    uint8, scales [B, m n / 128] fp32)."""
+    B, m, n = _bmn(X)
+    _expect(X, (B, m, n), (torch.float32,), "X")
+    if out is not None:
+        codes, gs = out
+    else:
+        codes = torch.empty((B, m, n // 2), dtype=torch.uint8, device=X.device)
+        gs = torch.empty((B, m * n // GROUP), dtype=torch.float32, device=X.device)
+    _expect(codes, (B, m, n // 2), (torch.uint8,), "codes")
+    _expect(gs, (B, m * n // GROUP), (torch.float32,), "gscale")
+    _check(lib.gm_group_quant4(B, m, n, _ptr(X), _ptr(codes), _ptr(gs), _stream()),
+           "gm_group_quant4")
+    return codes, gs
+
+
+def group_dequant4(codes, gscale, out=None):
+    """fp32 [B, m, n] from 4bit-Muon-base codes and scales."""
+    B, m, n2 = _bmn(codes)
+    n = 2 * n2
+    _expect(codes, (B, m, n2), (torch.uint8,), "codes")
+    _expect(gscale, (B, m * n // GROUP), (torch.float32,), "gscale")
+    if out is None:
+        out = torch.empty((B, m, n), dtype=torch.float32, device=codes.device)
+    _expect(out, (B, m, n), (torch.float32,), "out")
+    _check(lib.gm_group_dequant4(B, m, n, _ptr(codes), _ptr(gscale), _ptr(out), _stream()),
+           "gm_group_dequant4")
+    return out
 
 
 def newton_schulz(X, abc=None, T=5, eps=1e-7, out_dtype=torch.float32, out=None, ws=None):

@@ -139,6 +139,24 @@ gm_status gm_quant8(int B, int rows, int k, const float* X,
                     int8_t* codes, float* colscale, gm_stream_t stream);
 
 /*
+ * The 4bit-Muon-base codec: direct 4-bit quantization of the whole momentum,
+ * the baseline [GRASP] compares its codec with (research background: the
+ * error NS amplifies; the results tables' "4bit-Muon-base" rows). The page
+ * does not describe its grouping; this library's reading: one absmax scale per
+ * group of 128 consecutive row-major elements (m n is a multiple of 256, so no
+ * group is ragged or spans two matrices):
+ *   s_g = max |x| over the group; q = clamp(rint(fp32(x / s_g) * 7), -7, 7);
+ *   s_g = 0 -> q = 0; a NaN in a group makes s_g NaN and its codes 0.
+ *   X f32 [B][m][n] -> codes4 uint8 [B][m][n/2] (nibbles as in
+ *   gm_dequant_rebuild), gscale f32 [B][m*n/128].
+ */
+gm_status gm_group_quant4(int B, int m, int n, const float* X, uint8_t* codes4, float* gscale,
+                          gm_stream_t stream);
+/* The inverse: X_out[e] = fp32(q_e / 7) * s_g (f32 [B][m][n]). */
+gm_status gm_group_dequant4(int B, int m, int n, const uint8_t* codes4, const float* gscale,
+                            float* X_out, gm_stream_t stream);
+
+/*
  * Standard quintic Newton-Schulz [GramNS §1.2, eq. (2); Algorithm 1 first
  * line for the normalisation; LiMuon key design 3 for the coefficients]:
  *   wide form Y = X (m <= n) or X^T (m > n); Y <- Y / (|Y|_F + eps);

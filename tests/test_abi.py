@@ -119,3 +119,16 @@ def test_quant8_row_range():
     ok = ctypes.c_void_p(4096)
     for B, rows in [(0, 16), (1, 0), (1, (1 << 20) + 1)]:
         assert gm.lib.gm_quant8(B, rows, 8, ok, ok, ok, None) == gm.GM_E_ARG
+
+
+def test_group_codec_argument_errors():
+    """The 4bit-Muon-base entry points reject bad shapes, NULL and misaligned
+    arrays on the host, before any launch (this runs without a GPU)."""
+    ok, bad = ctypes.c_void_p(4096), ctypes.c_void_p(4096 + 8)
+    for B, m, n in [(0, 256, 512), (1, 250, 512), (1, 256, 8)]:
+        assert gm.lib.gm_group_quant4(B, m, n, ok, ok, ok, None) == gm.GM_E_ARG
+        assert gm.lib.gm_group_dequant4(B, m, n, ok, ok, ok, None) == gm.GM_E_ARG
+    assert gm.lib.gm_group_quant4(1, 256, 512, None, ok, ok, None) == gm.GM_E_ARG
+    assert gm.lib.gm_group_quant4(1, 256, 512, bad, ok, ok, None) == gm.GM_E_ARG
+    assert b"aligned" in gm.lib.gm_last_error()
+    assert gm.lib.gm_group_dequant4(1, 256, 512, ok, bad, ok, None) == gm.GM_E_ARG

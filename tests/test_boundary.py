@@ -137,7 +137,12 @@ def test_entry_point_bindings_check_tensors_before_passing_pointers():
         (lambda: gm.newton_schulz(f(B, m, n), ws=torch.empty(16, dtype=torch.uint8)), "ws: 16 bytes"),
         (lambda: gm.gram_ns(f(B, m, n).double()), "X: dtype"),
         (lambda: gm.newton_schulz_noalloc(f(B, m, n), out=f(B, m, n).double()), "out: dtype"),
+        (lambda: gm.group_quant4(f(B, m, n).double()), "X: dtype"),
+        (lambda: gm.group_dequant4(st.codes4, f(B, m * n // 64)), "gscale: expected shape"),
+        (lambda: gm.group_dequant4(st.codes4, f(B, m * n // 128), out=f(B, m, n).half()),
+         "out: dtype"),
         # right shapes and dtypes, host memory: stopped before the library call
+        (lambda: gm.group_quant4(f(B, m, n)), "expected a CUDA tensor"),
         (lambda: gm.dequant_rebuild(*parts), "expected a CUDA tensor"),
         (lambda: gm.grid_quant4(f(B, m, n), f(B, m, k), f(B, n, k)), "expected a CUDA tensor"),
         (lambda: gm.quant8(f(B, m, k)), "expected a CUDA tensor"),

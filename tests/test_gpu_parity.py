@@ -426,3 +426,26 @@ def test_ns_half_precision_outputs(cuda_lib, odt, B, m, n, form):
     for b in range(B):
         assert rel(O16[b], O.ns_standard(X[b].cpu().double())) <= 2e-2
     assert rel(O16, O32.to(odt)) <= 1e-2
+
+
+@pytest.mark.parametrize("B,m,n", [(2, 256, 512), (3, 144, 272), (1, 16, 48)])
+def test_group_codec_bit_exact(cuda_lib, B, m, n):
+    """The 4bit-Muon-base codec (128 consecutive elements per absmax scale)
+    against the oracle: codes and scales bit-exact, including a zero group and
+    a group of exact rounding ties (s = 7, x = k + 1/2), which take the
+    division path; the dequantized values within fp32 rounding."""
+    gm = cuda_lib
+    X = _outlier_matrix(B, m, n, 71)
+    flat = X[0].view(-1)
+    flat[:128] = 0.0
+    ties = torch.tensor([7.0] + [k + 0.5 for k in range(-7, 7)], dtype=torch.float32)
+    flat[128:256] = ties.repeat(10)[:128]
+    codes, gs = gm.group_quant4(X.to(DEV))
+    Xh = gm.group_dequant4(codes, gs)
+    torch.cuda.synchronize()
+    for b in range(B):
+        q, s = O.group_quant4(X[b])
+        assert torch.equal(codes[b].cpu(), O.pack_nibbles(q))
+        assert torch.equal(gs[b].cpu(), s)
+        assert rel(Xh[b], O.group_dequant4(q, s)) <= 1e-6
+    assert float(gs[0, 0]) == 0.0 and int(codes[0].view(-1)[:64].abs().max()) == 0
