@@ -1,0 +1,130 @@
+"""Ownership sharding of one parameter set across data-parallel ranks.
+
+Muon needs each weight's whole gradient matrix, and every matrix's GRASP step
+is independent of the others ("Achieving low-bit Muon through subspace
+preservation and grid quantization": overall framework; its limitations
+section describes quantizing per partition on top of distributed Muon). So a
+set of 2-D weights splits by ownership: each matrix has one owner rank, which
+alone keeps its quantized momentum and runs its step; the owners' updated
+weights are then all-gathered so that every rank holds the whole set again.
+
+Owners come from LPT greedy (longest processing time first) on a per-matrix
+cost, by default the step's Newton-Schulz FLOP scaling m n min(m, n). Every
+rank computes the same assignment from the same shapes, so no communication
+decides it.
+
+The per-matrix update is injected: ``make_step(B, m, n)`` returns a callable
+``step(W, G)`` that updates a contiguous [B, m, n] fp32 weight batch in place
+from a gradient batch of the same shape and keeps whatever state it needs
+(the library's GRASP step on a GPU; any stand-in in tests). The exchange is
+one all-gather per shape group through ``torch.distributed`` (NCCL on GPUs),
+each rank sending its owned matrices padded to the largest owner's count.
+"""
+
+from __future__ import annotations
+
+from typing import Callable, Sequence
+
+import torch
+import torch.distributed as dist
+
+
+def ns_cost(m: int, n: int) -> float:
+    """NS FLOPs of one m x n matrix up to a constant factor: N^2 M' = m n min(m, n)."""
+    return float(m) * n * min(m, n)
+
+
+def lpt_owners(costs: Sequence[float], world: int) -> list[int]:
+    """LPT greedy: items in order of decreasing cost (ties by index), each to
+    the rank with the smallest load so far (ties to the lower rank). Returns the
+    owner of every item."""
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    order = sorted(range(len(costs)), key=lambda i: (-costs[i], i))
+    load = [0.0] * world
+    owner = [0] * len(costs)
+    for i in order:
+        r = min(range(world), key=lambda q: (load[q], q))
+        owner[i] = r
+        load[r] += costs[i]
+    return owner
+
+
+class ShardedStep:
+    """One optimizer step of a parameter set split by ownership.
+
+    ``shapes`` lists the set's shape groups as (m, n, count), in order; the
+    call takes, per group, the [count, m, n] weights (updated in place on
+    every rank) and the matching gradients (every rank holds all of them, as
+    after a data-parallel all-reduce)."""
+
+    def __init__(self, shapes: Sequence[tuple[int, int, int]], world: int, rank: int,
+                 make_step: Callable[[int, int, int], Callable], cost=ns_cost, group=None):
+        if not 0 <= rank < world:
+            raise ValueError(f"rank {rank} outside world {world}")
+        self.shapes = [tuple(s) for s in shapes]
+        self.world, self.rank, self.group = world, rank, group
+        costs = [cost(m, n) for m, n, count in self.shapes for _ in range(count)]
+        flat = lpt_owners(costs, world)
+        self.owner: list[list[int]] = []          # owner of matrix i of group g
+        self.owned: list[list[list[int]]] = []    # owned[g][r]: indices rank r owns in g
+        pos = 0
+        for m, n, count in self.shapes:
+            own = flat[pos:pos + count]
+            pos += count
+            self.owner.append(own)
+            self.owned.append([[i for i in range(count) if own[i] == r] for r in range(world)])
+        self.steps = [make_step(len(o[rank]), m, n) if o[rank] else None
+                      for (m, n, _), o in zip(self.shapes, self.owned)]
+
+    def loads(self, cost=ns_cost) -> list[float]:
+        """Total cost each rank owns."""
+        load = [0.0] * self.world
+        for (m, n, _), own in zip(self.shapes, self.owner):
+            for r in own:
+                load[r] += cost(m, n)
+        return load
+
+    def __call__(self, Ws: Sequence[torch.Tensor], Gs: Sequence[torch.Tensor]) -> None:
+        if len(Ws) != len(self.shapes) or len(Gs) != len(self.shapes):
+            raise ValueError("one weight and one gradient tensor per shape group")
+        for g, ((m, n, count), W, G) in enumerate(zip(self.shapes, Ws, Gs)):
+            if tuple(W.shape) != (count, m, n) or tuple(G.shape) != (count, m, n):
+                raise ValueError(f"group {g}: expected [{count}, {m}, {n}] weights and gradients")
+            mine = self.owned[g][self.rank]
+            Wb = None
+            if mine:
+                idx = torch.tensor(mine, device=W.device)
+                Wb = W.index_select(0, idx)
+                self.steps[g](Wb, G.index_select(0, idx))
+            if self.world == 1:
+                if Wb is not None:
+                    W.copy_(Wb)
+                continue
+            width = max(len(o) for o in self.owned[g])
+            send = torch.zeros((width, m, n), dtype=W.dtype, device=W.device)
+            if Wb is not None:
+                send[:len(mine)] = Wb
+            recv = [torch.empty_like(send) for _ in range(self.world)]
+            dist.all_gather(recv, send, group=self.group)
+            for r, own in enumerate(self.owned[g]):
+                if own:
+                    W.index_copy_(0, torch.tensor(own, device=W.device), recv[r][:len(own)])
+
+
+def grasp_make_step(k: int, device=None, **params) -> Callable[[int, int, int], Callable]:
+    """``make_step`` for the library's GRASP step: each owner batch gets its own
+    step object and zero state (its quantized momentum lives on this rank only)."""
+    from . import gmuon as gm
+
+    def make(B: int, m: int, n: int):
+        step = gm.GraspStep(B, m, n, k, device=device, **params)
+        state = gm.GraspState.zeros(B, m, n, k, device)
+
+        def run(W: torch.Tensor, G: torch.Tensor) -> None:
+            step(state, W, G)
+
+        run.state = state
+        return run
+
+    return make

@@ -1,0 +1,112 @@
+"""Ownership sharding of one parameter set across ranks, on CPU.
+
+The assignment is checked against a hand-worked LPT example and against the
+textbook bound for LPT (Graham, 1969: makespan <= (4/3 - 1/(3w)) x optimum),
+the optimum found by brute force. The exchange runs as gloo processes with a
+stateful CPU stand-in for the per-matrix step: every rank must end with the
+weights a single process computes, and every matrix must have one owner.
+"""
+
+import itertools
+import os
+import random
+import socket
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+from bit_muon_optimizer_b200 import sharding as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SHAPES = [(8, 16, 5), (16, 8, 3), (16, 16, 1), (8, 8, 4)]
+
+
+def test_lpt_hand_worked_example():
+    # 7 -> r0; 6 -> r1; 5 -> r1 (6 < 7); 4 -> r0 (7 < 11); 3 -> r0 (11 = 11, lower rank);
+    # 2 -> r1 (11 < 14): loads 14 and 13
+    assert S.lpt_owners([7, 6, 5, 4, 3, 2], 2) == [0, 1, 1, 0, 0, 1]
+    assert S.lpt_owners([5.0], 3) == [0]
+    assert S.lpt_owners([], 2) == []
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_lpt_within_graham_bound(world):
+    rnd = random.Random(world)
+    for _ in range(20):
+        costs = [rnd.randint(1, 50) for _ in range(rnd.randint(world, 8))]
+        own = S.lpt_owners(costs, world)
+        lpt = max(sum(c for c, o in zip(costs, own) if o == r) for r in range(world))
+        best = min(max(sum(c for c, o in zip(costs, a) if o == r) for r in range(world))
+                   for a in itertools.product(range(world), repeat=len(costs)))
+        assert lpt <= (4 / 3 - 1 / (3 * world)) * best + 1e-9
+
+
+class _StandIn:
+    """Per-batch state: the number of steps taken; W -= 0.1 t G per matrix."""
+
+    def __init__(self, B, m, n):
+        self.t = 0
+
+    def __call__(self, W, G):
+        self.t += 1
+        W.sub_(0.1 * self.t * G)
+
+
+def _inputs(step):
+    g = torch.Generator().manual_seed(100 + step)
+    return [torch.randn((c, m, n), generator=g) for m, n, c in SHAPES]
+
+
+def _run(world, rank, steps=2):
+    sh = S.ShardedStep(SHAPES, world, rank, _StandIn)
+    W = [x.clone() for x in _inputs(0)]
+    for t in range(1, steps + 1):
+        sh(W, _inputs(t))
+    return sh, W
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        sh, W = _run(world, rank)
+        q.put((rank, sh.owner, W))
+    finally:
+        dist.destroy_process_group()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_gloo_ranks_end_with_the_single_process_weights(world):
+    _, W_ref = _run(1, 0)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    owners = out[0][1]
+    for rank, own, W in out:
+        assert own == owners                                   # same assignment everywhere
+        for a, b in zip(W, W_ref):
+            assert torch.equal(a, b)
+    # one owner per matrix; the 1-matrix group leaves some ranks without work in it
+    assert [len(o) for o in owners] == [c for _, _, c in SHAPES]
+    assert all(0 <= r < world for o in owners for r in o)
+    assert len(set(owners[2])) == 1
