@@ -27,6 +27,8 @@ Readings of points the pages leave open:
 * The 4bit-Muon-base codec the note compares against quantizes the whole
   matrix in groups of 128 consecutive row-major elements, one absmax scale
   per group, codes in [-7, 7] like the grid codec.
+* MuonQ's mu-law codec (only its abstract is on the pages): the same groups
+  and absmax normalisation, mu = 255, codes rint(7 F(x / s)) in [-7, 7].
 """
 
 from __future__ import annotations
@@ -54,6 +56,7 @@ __all__ = [
     "orth_positive", "power_iteration",
     "quant8", "dequant8", "grid_quant4", "grid_scale_matrix", "grid_dequant4",
     "pack_nibbles", "unpack_nibbles", "group_quant4", "group_dequant4",
+    "MULAW_MU", "mulaw_compress", "mulaw_expand", "mulaw_quant4", "mulaw_dequant4",
     "ns_standard", "gram_ns", "quintic_scalar", "POLAR_EXPRESS_ABC", "safety_scaled",
     "GraspState", "zero_state", "rebuild_momentum", "grasp_step",
 ]
@@ -257,6 +260,51 @@ def group_dequant4(codes: torch.Tensor, scales: torch.Tensor, group: int = 128) 
     q = codes.reshape(-1).to(DT)
     s = scales.to(DT).repeat_interleave(group)[: q.numel()]
     return (q / 7.0 * s).view(codes.shape)
+
+
+#: mu of the mu-law companding codec (the G.711 value; MuonQ states none).
+MULAW_MU = 255.0
+
+
+def mulaw_compress(x: torch.Tensor, mu: float = MULAW_MU) -> torch.Tensor:
+    """F(x) = sign(x) ln(1 + mu |x|) / ln(1 + mu) for |x| <= 1, in fp64."""
+    x = x.to(DT)
+    return torch.sign(x) * torch.log1p(mu * x.abs()) / math.log1p(mu)
+
+
+def mulaw_expand(y: torch.Tensor, mu: float = MULAW_MU) -> torch.Tensor:
+    """F^-1(y) = sign(y) ((1 + mu)^|y| - 1) / mu, in fp64."""
+    y = y.to(DT)
+    return torch.sign(y) * torch.expm1(y.abs() * math.log1p(mu)) / mu
+
+
+def mulaw_quant4(X: torch.Tensor, group: int = 128, mu: float = MULAW_MU):
+    """4-bit mu-law companding codes, the third part of MuonQ (its abstract:
+    finer steps where momentum values are dense, coarser at the outliers).
+    Each group of `group` consecutive row-major elements is normalised by its
+    absmax s (the plainest reading of MuonQ's unstated pre-quantization
+    normalisation) and q = clamp(rint(7 F(x / s)), -7, 7); s = 0 gives 0.
+    Returns (codes int8 (m, n), scales fp32 (ceil(m n / group),))."""
+    x = X.to(F32).reshape(-1)
+    ng = -(-x.numel() // group)
+    scales = torch.zeros(ng, dtype=F32)
+    codes = torch.zeros(x.numel(), dtype=torch.int8)
+    for gi in range(ng):
+        seg = x[gi * group:(gi + 1) * group]
+        s = seg.abs().max()
+        scales[gi] = s
+        if s > 0:
+            y = mulaw_compress(seg.to(DT) / float(s), mu)
+            codes[gi * group:(gi + 1) * group] = torch.clamp(torch.round(7.0 * y), -7, 7).to(torch.int8)
+    return codes.view(X.shape), scales
+
+
+def mulaw_dequant4(codes: torch.Tensor, scales: torch.Tensor, group: int = 128,
+                   mu: float = MULAW_MU) -> torch.Tensor:
+    """x^ = s F^-1(q / 7), in fp64."""
+    q = codes.reshape(-1).to(DT)
+    s = scales.to(DT).repeat_interleave(group)[: q.numel()]
+    return (s * mulaw_expand(q / 7.0, mu)).view(codes.shape)
 
 
 def pack_nibbles(codes: torch.Tensor) -> torch.Tensor:

@@ -486,6 +486,60 @@ def test_group_quant4_by_explicit_loops(m, n, group):
         assert abs(float(flat[e]) - float(xh.reshape(-1)[e])) <= s / 14 * (1 + 1e-6)
 
 
+def test_mulaw_function_inverse_and_endpoints():
+    """The textbook mu-law pair: F maps [-1, 1] onto itself, odd and
+    increasing, F(0) = 0, F(+-1) = +-1, and F^-1 undoes it."""
+    x = torch.linspace(-1, 1, 2001, dtype=DT)
+    y = O.mulaw_compress(x)
+    assert float(y[0]) == pytest.approx(-1.0, abs=1e-15) and float(y[-1]) == pytest.approx(1.0, abs=1e-15)
+    assert float(O.mulaw_compress(torch.zeros(1, dtype=DT))) == 0.0
+    assert torch.all(y[1:] > y[:-1])
+    assert torch.allclose(y, -O.mulaw_compress(-x), atol=0, rtol=0)
+    assert float((O.mulaw_expand(y) - x).abs().max()) < 1e-14
+    # mu = 255 at x = 0.5: ln(128.5) / ln(256)
+    assert float(O.mulaw_compress(torch.tensor([0.5]))) == pytest.approx(math.log(128.5) / math.log(256))
+
+
+def test_mulaw_codes_by_brute_force_and_small_mu_limit():
+    """Each code is the nibble nearest 7 F(x / s) (ties to even); as mu -> 0,
+    F -> identity and the codec becomes the uniform group codec."""
+    gen = torch.Generator().manual_seed(50)
+    X = (torch.randn(16, 64, generator=gen) * torch.rand(16, 1, generator=gen)).to(torch.float32)
+    codes, scales = O.mulaw_quant4(X)
+    s = scales.to(DT).repeat_interleave(128).view(X.shape)
+    target = 7.0 * O.mulaw_compress(X.to(DT) / s)
+    cand = torch.arange(-8, 8, dtype=DT)
+    dist = (target.unsqueeze(-1) - cand).abs()
+    best = dist.min(dim=-1).values
+    chosen = dist.gather(-1, (codes.to(torch.int64) + 8).unsqueeze(-1)).squeeze(-1)
+    assert torch.all(chosen == best)
+    cu, su = O.group_quant4(X)
+    cm, sm = O.mulaw_quant4(X, mu=1e-9)
+    assert torch.equal(su, sm)
+    diff = (cu.int() - cm.int()).abs()
+    assert int(diff.max()) <= 1 and float((diff > 0).double().mean()) <= 1e-3
+
+
+@pytest.mark.parametrize("dist", ["gauss", "student3"])
+def test_mulaw_finer_in_the_dense_region(dist):
+    """MuonQ's abstract: mu-law companding gives more resolution where momentum
+    values are dense. Below the median magnitude its mean error is lower than
+    the uniform group codec's, on Gaussian and on heavy-tailed data."""
+    gen = torch.Generator().manual_seed(51)
+    if dist == "gauss":
+        X = torch.randn(128, 256, generator=gen)
+    else:                                   # Student-t, 3 degrees of freedom
+        z = torch.randn(128, 256, generator=gen, dtype=DT)
+        chi2 = (torch.randn(3, 128, 256, generator=gen, dtype=DT) ** 2).sum(0)
+        X = (z / torch.sqrt(chi2 / 3)).float()
+    dense = X.abs() <= X.abs().median()
+    cu, su = O.group_quant4(X)
+    cm, sm = O.mulaw_quant4(X)
+    eu = (O.group_dequant4(cu, su) - X.double()).abs()
+    em = (O.mulaw_dequant4(cm, sm) - X.double()).abs()
+    assert float(em[dense].mean()) < 0.8 * float(eu[dense].mean())
+
+
 def _low_rank_plus_outliers(m, n, r, seed, noise=0.05, outlier=10.0):
     """Synthetic momentum: rank-r part with singular values from 1 down to
     10^-1.5, a Gaussian floor, and 1 % of rows and of columns scaled by 10."""
