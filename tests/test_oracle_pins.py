@@ -537,6 +537,14 @@ def test_mulaw_finer_in_the_dense_region(dist):
     cm, sm = O.mulaw_quant4(X)
     eu = (O.group_dequant4(cu, su) - X.double()).abs()
     em = (O.mulaw_dequant4(cm, sm) - X.double()).abs()
+    xn = float(X.double().norm())
+    sweep = []
+    for mu in (15.0, 63.0):
+        c, sc = O.mulaw_quant4(X, mu=mu)
+        sweep.append(float((O.mulaw_dequant4(c, sc, mu=mu) - X.double()).norm()) / xn)
+    print(f"\n[{dist}] mean |error| below the median: uniform {float(eu[dense].mean()):.3f}, "
+          f"mu-law {float(em[dense].mean()):.3f}; relative error: uniform {float(eu.norm()) / xn:.3f}, "
+          f"mu = 15 / 63 / 255: {sweep[0]:.3f} / {sweep[1]:.3f} / {float(em.norm()) / xn:.3f}")
     assert float(em[dense].mean()) < 0.8 * float(eu[dense].mean())
 
 
