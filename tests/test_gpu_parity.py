@@ -449,3 +449,16 @@ def test_group_codec_bit_exact(cuda_lib, B, m, n):
         assert torch.equal(gs[b].cpu(), s)
         assert rel(Xh[b], O.group_dequant4(q, s)) <= 1e-6
     assert float(gs[0, 0]) == 0.0 and int(codes[0].view(-1)[:64].abs().max()) == 0
+
+
+def test_dequant_rebuild_residual_only(cuda_lib):
+    """k = 0: gm_dequant_rebuild rebuilds the 4-bit residual alone (no factor
+    arrays passed), at a ragged size."""
+    gm = cuda_lib
+    B, m, n = 2, 144, 272
+    s = _random_state(B, m, n, 8, 12)
+    M = gm.dequant_rebuild(s["codes4"].to(DEV), s["rscale"].to(DEV), s["cscale"].to(DEV))
+    torch.cuda.synchronize()
+    for b in range(B):
+        want = O.grid_dequant4(O.unpack_nibbles(s["codes4"][b]), s["rscale"][b], s["cscale"][b])
+        assert rel(M[b], want) <= 1e-6
