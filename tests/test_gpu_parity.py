@@ -462,3 +462,27 @@ def test_dequant_rebuild_residual_only(cuda_lib):
     for b in range(B):
         want = O.grid_dequant4(O.unpack_nibbles(s["codes4"][b]), s["rscale"][b], s["cscale"][b])
         assert rel(M[b], want) <= 1e-6
+
+
+@pytest.mark.parametrize("ns", ["standard", "gram"])
+def test_grasp_step_zero_gradient(cuda_lib, ns):
+    """The degenerate step: a zero gradient on a zero state gives M = 0, every
+    power-iteration column dead (P = R = 0), zero codes and scales, O = 0, so
+    W is unchanged bit for bit; twice, so the second step's warm start falls
+    back to the Rademacher columns of an all-zero R."""
+    gm = cuda_lib
+    B, m, n, k = 2, 256, 512, 8
+    nsmode = gm.GM_NS_GRAM if ns == "gram" else gm.GM_NS_STANDARD
+    step = gm.GraspStep(B, m, n, k, ns=nsmode, seed=9, device=DEV)
+    st = gm.GraspState.zeros(B, m, n, k, DEV)
+    W = WL.random_matrix((B, m, n), 81, std=0.02).to(DEV)
+    W0 = W.clone()
+    G = torch.zeros((B, m, n), dtype=torch.bfloat16, device=DEV)
+    for t in (1, 2):
+        step(st, W, G)
+        torch.cuda.synchronize()
+        assert int(st.dev_status.item()) == 0 and int(st.step.item()) == t
+    assert torch.equal(W, W0)
+    for x in (st.codes4, st.rscale, st.cscale, st.P8, st.Pscale, st.R8, st.Rscale):
+        assert int(torch.count_nonzero(x)) == 0
+    assert int(torch.count_nonzero(step.stage_P())) == 0
