@@ -99,7 +99,7 @@ class ShardedStep:
                 self.steps[g](Wb, G.index_select(0, idx))
             if self.world == 1:
                 if Wb is not None:
-                    W.copy_(Wb)
+                    W.index_copy_(0, idx, Wb)
                 continue
             width = max(len(o) for o in self.owned[g])
             send = torch.zeros((width, m, n), dtype=W.dtype, device=W.device)
