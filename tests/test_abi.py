@@ -132,3 +132,15 @@ def test_group_codec_argument_errors():
     assert gm.lib.gm_group_quant4(1, 256, 512, bad, ok, ok, None) == gm.GM_E_ARG
     assert b"aligned" in gm.lib.gm_last_error()
     assert gm.lib.gm_group_dequant4(1, 256, 512, ok, bad, ok, None) == gm.GM_E_ARG
+
+
+def test_every_cuda_source_is_built():
+    """The in-tree build compiles every .cu file of the package's csrc/ into
+    libgmuon.so (a kernel file left out would only fail at link or call time)."""
+    import os
+
+    from bit_muon_optimizer_b200 import build as Bd
+    on_disk = sorted(f for f in os.listdir(Bd.CSRC) if f.endswith(".cu"))
+    assert sorted(Bd.SOURCES) == on_disk
+    headers = sorted(f for f in os.listdir(Bd.CSRC) if f.endswith((".cuh", ".h")))
+    assert sorted(Bd.HEADERS) == headers
