@@ -1,21 +1,24 @@
 """Benchmark of one GRASP optimizer step over a parameter set, on B200s.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--ns standard|gram]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--ns standard|gram]
                     [--impl ours|reference]
 
 A "step" is one full GRASP step (rebuild, momentum, power iteration, 4/8-bit
 re-quantization, Newton-Schulz, weight update) over every matrix of the
 parameter set, with that step's synthetic gradients already resident in HBM.
-Each shape group is one batched gm_grasp_step call; the three calls of a step
-run on three streams and are replayed from a CUDA graph (one graph per step,
-since each step has its own gradient buffer). N > 1 (torchrun): every rank
-steps its own parameter set (weak scaling, no collective on the data path);
-the time is the max over ranks.
+The default parameter set is the largest one that fits one GPU: the
+Qwen2.5-7B-shaped set (6.5e9 weight elements), measured one shape group at a
+time (each group batched in one gm_grasp_step call and replayed from CUDA
+graphs); the set's time is the sum over its groups. N > 1 (torchrun): the set
+is split by ownership across the ranks (each matrix's step runs on one owner,
+then one NCCL all-gather per shape group gives every rank the updated set:
+strong scaling); the time is the max over ranks.
 
 Printed (rank 0): one JSON line with value = ms per parameter set for the
-whole job, the NS chain's tensor-core roofline, the codec passes' HBM rate,
-an end-to-end number through host buffers, and the fp64 CPU oracle timed on a
-bounded sample as the CPU baseline.
+whole job; the NS chain's tensor-core roofline and the codec half's HBM rate,
+both timed with CUDA events around the step's own two halves
+(gm_grasp_state_update, gm_grasp_apply); an end-to-end number through pinned
+host buffers; and the fp64 CPU oracle timed on a bounded sample.
 """
 
 from __future__ import annotations
@@ -144,48 +147,38 @@ def max_over_ranks(v: float, world: int) -> float:
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_sample_seconds(w: WL.Workload, ns: str, budget_s: float):
-    """Time the fp64 oracle on one matrix of every shape group, step 1 and 2,
-    repeated until ~budget_s; returns (ms per parameter set, sample text, cores)."""
+def oracle_sample_seconds(w: WL.Workload, ns: str):
+    """Time the fp64 oracle: one step (from a zero state) of one matrix of every
+    shape group; returns (ms per parameter set = sum over groups of the group's
+    count x its sample's time, sample text, cores)."""
     import oracle as O
     per_shape = []
-    t_all = time.perf_counter()
     for gi, g in enumerate(w.groups):
-        m, n, k = g.m, g.n, w.k
         b = w.group_base(gi)
-        st = O.zero_state(m, n, k)
-        W = WL.initial_weight(w, b, m, n)
-        times = []
-        t = 1
-        while True:
-            G = WL.gradient(w, b, t, m, n)
-            t0 = time.perf_counter()
-            r = O.grasp_step(st, W, G, mu=w.mu, eta=w.eta, wd=w.wd, seed=w.seed, b=0, ns=ns, T=w.T)
-            times.append(time.perf_counter() - t0)
-            st, W = r.state, r.W.float()
-            t += 1
-            if t > 2 and (time.perf_counter() - t_all) > budget_s * (gi + 1) / len(w.groups):
-                break
-            if t > 6:
-                break
-        per_shape.append((g, statistics.median(times[1:] if len(times) > 1 else times)))
+        W = WL.initial_weight(w, b, g.m, g.n)
+        G = WL.gradient(w, b, 1, g.m, g.n)
+        t0 = time.perf_counter()
+        O.grasp_step(O.zero_state(g.m, g.n, w.k), W, G, mu=w.mu, eta=w.eta, wd=w.wd, seed=w.seed,
+                     b=b, ns=ns, T=w.T)
+        per_shape.append((g, time.perf_counter() - t0))
     ms = 1e3 * sum(g.count * s for g, s in per_shape)
-    sample = ("fp64 oracle, one matrix per shape group ("
-              + ", ".join(f"{g.m}x{g.n}" for g, _ in per_shape)
-              + "), median of its steps 2+, extrapolated by the group counts")
+    sample = ("fp64 oracle, one step of one matrix per shape group ("
+              + ", ".join(f"{g.m}x{g.n}: {s:.2f} s" for g, s in per_shape)
+              + "), extrapolated by the group counts")
     return ms, sample, torch.get_num_threads()
 
 
 def run_reference(args, world, rank):
     """The reference arm: the fp64 CPU oracle as it stands, on this host's cores.
 
-    Each step (warm-up or timed) is one oracle step of one sample matrix of
-    every shape group, with each sample's state and weight carried from step
-    to step, so the timed steps start from a warm quantized state like the
-    GPU arm's; the step's time per parameter set is sum over groups of
-    (matrices in the group) x (the sample's step time). The whole run costs
-    (W + K) times one oracle step per group, about 0.4 s a step for LLaMA-130M.
-    Only rank 0 works; the other ranks return at once."""
+    Every shape group has one sample matrix whose state and weight carry over
+    from one of its steps to the next. Each reference step (warm-up or timed)
+    runs one oracle step of one sample, the groups taken in turn, so a step
+    costs one matrix step however large the set; it reports the parameter
+    set's time as the sum over groups of (matrices in the group) x (the latest
+    step time of the group's sample). Samples not yet timed after the warm-up
+    steps get one untimed step first. Only rank 0 works; the other ranks
+    return at once."""
     if rank != 0:
         return
     import oracle as O
@@ -193,31 +186,40 @@ def run_reference(args, world, rank):
     samples = []
     for gi, g in enumerate(w.groups):
         b = w.group_base(gi)
-        samples.append([g, b, O.zero_state(g.m, g.n, w.k), WL.initial_weight(w, b, g.m, g.n)])
+        samples.append({"g": g, "b": b, "st": O.zero_state(g.m, g.n, w.k),
+                        "W": WL.initial_weight(w, b, g.m, g.n), "t": 0, "s": None})
+
+    def one(smp):
+        g, b = smp["g"], smp["b"]
+        smp["t"] += 1
+        G = WL.gradient(w, b, smp["t"], g.m, g.n)
+        t0 = time.perf_counter()
+        r = O.grasp_step(smp["st"], smp["W"], G, mu=w.mu, eta=w.eta, wd=w.wd, seed=w.seed, b=b,
+                         ns=args.ns, T=w.T)
+        smp["s"] = time.perf_counter() - t0
+        smp["st"], smp["W"] = r.state, r.W.float()
+
+    ng = len(samples)
+    for i in range(args.warmup):
+        one(samples[i % ng])
+    for smp in samples:
+        if smp["s"] is None:
+            one(smp)
     vals = []
-    for i in range(args.warmup + args.steps):
-        t = i + 1
-        ms = 0.0
-        for smp in samples:
-            g, b, st, W = smp
-            G = WL.gradient(w, b, t, g.m, g.n)
-            t0 = time.perf_counter()
-            r = O.grasp_step(st, W, G, mu=w.mu, eta=w.eta, wd=w.wd, seed=w.seed, b=0, ns=args.ns,
-                             T=w.T)
-            ms += 1e3 * g.count * (time.perf_counter() - t0)
-            smp[2], smp[3] = r.state, r.W.float()
-        if i >= args.warmup:
-            vals.append(ms)
+    for i in range(args.steps):
+        one(samples[(args.warmup + i) % ng])
+        vals.append(1e3 * sum(smp["g"].count * smp["s"] for smp in samples))
     v = statistics.median(vals)
     cores = torch.get_num_threads()
-    sample = ("fp64 oracle, one matrix per shape group ("
-              + ", ".join(f"{g.m}x{g.n}" for g, _, _, _ in samples)
-              + "), one step of each per reference step from a state carried across steps, "
-              "extrapolated by the group counts; median over the timed steps")
+    sample = ("fp64 oracle, one sample matrix per shape group ("
+              + ", ".join(f"{s['g'].m}x{s['g'].n}" for s in samples)
+              + ") with its state carried across its steps; each reference step runs one "
+              "sample's step, groups in turn; per-set time = sum over groups of the count x "
+              "the sample's latest step time; median over the timed steps")
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "ns": args.ns, "k": w.k, "matrices": sum(g.count for g in w.groups)},
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -229,10 +231,10 @@ def run_reference(args, world, rank):
 
 GRAD_POOL = 6   # distinct gradient buffers per group, used cyclically step after step
 
-# DRAM bytes per k_gemm launch (average over one step's 45 NS products of the
-# LLaMA-130M set, standard NS), from an ncu capture of dram__bytes_read.sum +
-# dram__bytes_write.sum (the k_gemm summary under profiles/); reported only while
-# gm_gemm.cu is the source that capture measured.
+# DRAM bytes per k_gemm launch (average over one step's NS products of the named
+# workload), from an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum
+# (the k_gemm summaries under profiles/); reported only while gm_gemm.cu is the
+# source that capture measured.
 GEMM_TRAFFIC = {"config": 2, "ns": "standard", "bytes_per_launch": 87.56e6,
                 "source_sha256": "aa52586b7c8ef53cef64f66392279f880c35c449ce72813d6b82ec7d5a190d0a"}
 
@@ -253,24 +255,19 @@ def gemm_traffic(config: int, ns: str):
 
 def est_bytes(w: WL.Workload, pool: int) -> int:
     """Device bytes of the benchmark per parameter-set element: fp32 W, the
-    gradient pool, the step workspace (fp32 M, the 16-bit iterate, NS buffers),
-    and the separately timed NS / codec passes (fp32 O, their workspace, codes)."""
+    gradient pool, the step workspace (fp32 M, the 16-bit iterate, NS buffers)
+    and the comparator's copies."""
     elems = sum(g.count * g.m * g.n for g in w.groups)
     return elems * (22 + 2 * pool)
 
 
-def matrix_base(w: WL.Workload, gi: int, rank: int) -> int:
-    """Index of the first matrix of shape group gi in rank's parameter set: rank r
-    steps matrices r * count ... (r + 1) * count - 1 of the workload's sequence."""
-    return rank * sum(x.count for x in w.groups) + w.group_base(gi)
-
-
-def build_group(gm, w: WL.Workload, gi: int, ns_mode: int, rank: int, pool: int, dev):
+def build_group(gm, w: WL.Workload, gi: int, ns_mode: int, pool: int, dev):
     g = w.groups[gi]
     B, m, n = g.count, g.m, g.n
-    base = matrix_base(w, gi, rank)
+    base = w.group_base(gi)
+    ids = list(range(base, base + B))
     step = gm.GraspStep(B, m, n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=ns_mode,
-                        seed=w.seed + rank, device=dev)
+                        seed=w.seed, device=dev, matrix_ids=ids)
     st = gm.GraspState.zeros(B, m, n, w.k, dev)
     W = torch.empty((B, m, n), dtype=torch.float32, device=dev)
     for b in range(B):
@@ -284,10 +281,24 @@ def build_group(gm, w: WL.Workload, gi: int, ns_mode: int, rank: int, pool: int,
     return dict(step=step, st=st, W=W, grads=grads, B=B, m=m, n=n)
 
 
+def our_launches(gm, w: WL.Workload, ns_mode: int, groups=None) -> int:
+    """Our kernels per step: per group 9 codec kernels (column norms, warm start
+    with the factor fragments, rebuild + projection, three orthonormalisation
+    kernels, back projection, its finalisation, the 4-bit quantisation with the
+    8-bit one folded in), the NS products, and the zero-padding copy when a
+    dimension is not a multiple of 64."""
+    launches = 0
+    for (m, n) in (groups if groups is not None else [(g.m, g.n) for g in w.groups]):
+        pad = int(min(m, n) % 64 != 0 or max(m, n) % 64 != 0)
+        launches += 9 + gm.ns_flops(ns_mode, m, n, w.T)[1] + pad
+    return launches
+
+
 def measure(gm, w, groups, ns_mode, args, world, local, do_e2e):
     """Times args.steps graph-replayed GRASP steps over `groups` (each group on
-    its own stream), then the NS chains and the codec passes alone, then (if
-    asked) steps end to end through pinned host buffers."""
+    its own stream); then the step's two halves with CUDA events around each
+    (codec half: gm_grasp_state_update; NS half: gm_grasp_apply); the cuBLAS
+    comparator; and (if asked) steps end to end through pinned host buffers."""
     dev = groups[0]["W"].device
     streams = [torch.cuda.Stream(device=dev) for _ in groups]
     main = torch.cuda.Stream(device=dev)        # graphs are captured on a side stream
@@ -342,55 +353,28 @@ def measure(gm, w, groups, ns_mode, args, world, local, do_e2e):
         raise RuntimeError(f"device status {status}")
     del graphs
 
-    # ---- NS chain alone (tensor-core roofline) and codec passes alone (HBM), each
-    # replayed from a graph with the groups on their own streams, as in the step
-    def graph_ms(enqueue, reps):
-        fork(enqueue)                            # eager once (attributes, workspaces)
-        torch.cuda.synchronize()
-        gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr, stream=main):
-            fork(enqueue)
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(main):       # replay on the stream the events are recorded on
-            for _ in range(3):
-                gr.replay()
-            torch.cuda.synchronize()
-            s0.record(main)
-            for _ in range(reps):
-                gr.replay()
-            s1.record(main)
-        torch.cuda.synchronize()
-        del gr
-        return s0.elapsed_time(s1) / reps
-
-    for g in groups:
-        g["Mx"] = g["step"].stage_M()            # the last step's fp32 M_t, read-only below
-        g["O"] = torch.empty_like(g["Mx"])       # NS output, then the codec's rebuilt M
-        g["ws_ns"] = torch.empty(gm.workspace_bytes(gm.GM_OP_GRAM_NS if ns_mode == gm.GM_NS_GRAM
-                                                    else gm.GM_OP_NEWTON_SCHULZ, g["B"], g["m"], g["n"]),
-                                 dtype=torch.uint8, device=dev)
-        g["codes"] = (torch.empty_like(g["st"].codes4), torch.empty_like(g["st"].rscale),
-                      torch.empty_like(g["st"].cscale))
-
-    def ns_enqueue(g):
-        if ns_mode == gm.GM_NS_GRAM:
-            gm.gram_ns(g["Mx"], T=w.T, out=g["O"], ws=g["ws_ns"])
-        else:
-            gm.newton_schulz(g["Mx"], T=w.T, out=g["O"], ws=g["ws_ns"])
-
-    def codec_enqueue(g):
-        st = g["st"]
-        gm.dequant_rebuild(st.codes4, st.rscale, st.cscale, st.P8, st.Pscale, st.R8, st.Rscale,
-                           out=g["O"])
-        gm.grid_quant4(g["Mx"], g["step"].stage_P(), g["step"].stage_R(), out=g["codes"])
-
-    reps = 20 if sum(g["B"] * g["m"] * g["n"] for g in groups) < 5e8 else 5
-    ns_ms = graph_ms(ns_enqueue, reps)
+    # ---- the step's two halves, each bracketed by CUDA events on the stream
+    # that launches it; groups one after another (no overlap between groups)
+    nb = max(2, min(args.steps, 5))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nb * len(groups))]
+    with torch.cuda.stream(main):
+        for i in range(nb):
+            for j, g in enumerate(groups):
+                e0, e1, e2 = evs[i * len(groups) + j]
+                G = g["grads"][(args.warmup + args.steps + i) % npool]
+                e0.record(main)
+                g["step"].state_update(g["st"], G)
+                e1.record(main)
+                g["step"].apply(g["st"], g["W"])
+                e2.record(main)
+    torch.cuda.synchronize()
+    cod_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in evs) / nb
+    ns_ms = sum(e1.elapsed_time(e2) for _, e1, e2 in evs) / nb
     ns_flops = sum(gm.ns_flops(ns_mode, g["m"], g["n"], w.T)[0] * g["B"] for g in groups)
-    cod_ms = graph_ms(codec_enqueue, reps)
+    ns_launches = sum(gm.ns_flops(ns_mode, g["m"], g["n"], w.T)[1] for g in groups)
 
-    # comparator: the same standard NS chain written with torch.matmul (cuBLAS,
-    # bf16, no symmetry), on the same normalised wide-form inputs
+    # ---- comparator: the same standard NS chain written with torch.matmul
+    # (cuBLAS, bf16, no symmetry) on the same normalised inputs, graph-replayed
     abc = [(3.4445, -4.7750, 2.0315)] * w.T
     for g in groups:
         g["Xc"] = g["step"].stage_X().to(torch.bfloat16).clone()
@@ -404,17 +388,27 @@ def measure(gm, w, groups, ns_mode, args, world, local, do_e2e):
             X = torch.baddbmm(X, B, X, beta=a, alpha=1.0)
         g["Xw"].copy_(X)
 
-    cub_ms = graph_ms(cublas_enqueue, reps)
-    cub_flops_dense = sum(T_ * g["B"] * (2.0 * min(g["m"], g["n"]) ** 2 * max(g["m"], g["n"]) * 2
-                                         + 2.0 * min(g["m"], g["n"]) ** 3)
-                          for g in groups for T_ in [w.T])
+    reps = 20 if sum(g["B"] * g["m"] * g["n"] for g in groups) < 5e8 else 3
+    fork(cublas_enqueue)
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=main):
+        fork(cublas_enqueue)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(main):
+        gr.replay()
+        torch.cuda.synchronize()
+        s0.record(main)
+        for _ in range(reps):
+            gr.replay()
+        s1.record(main)
+    torch.cuda.synchronize()
+    cub_ms = s0.elapsed_time(s1) / reps
+    del gr
+    cub_flops_dense = sum(w.T * g["B"] * (2.0 * min(g["m"], g["n"]) ** 2 * max(g["m"], g["n"]) * 2
+                                          + 2.0 * min(g["m"], g["n"]) ** 3) for g in groups)
     for g in groups:
         del g["Xc"], g["Xw"]
-    # algorithmic bytes: rebuild reads codes + scales and writes fp32 M; quant reads fp32 M
-    # and writes codes + scales (the k (m + n) factor bytes are ignored)
-    cod_bytes = sum(2 * g["B"] * g["m"] * g["n"] * (4 + 0.5 + 0.0625) for g in groups)
-    for g in groups:
-        del g["Mx"], g["O"], g["ws_ns"], g["codes"]
 
     # ---- end to end through host buffers: H2D W and G, the step, D2H W
     e2e = None
@@ -424,34 +418,37 @@ def measure(gm, w, groups, ns_mode, args, world, local, do_e2e):
             host.append(dict(W=g["W"].cpu().pin_memory(), G=g["grads"][-1].cpu().pin_memory()))
         h2d = sum(h["W"].numel() * 4 + h["G"].numel() * h["G"].element_size() for h in host)
         d2h = sum(h["W"].numel() * 4 for h in host)
-        Wd = [torch.empty_like(g["W"]) for g in groups]
-        Gd = [torch.empty_like(g["grads"][-1]) for g in groups]
-        e_steps = max(2, min(args.steps, 5))
+        e_steps = 3 if h2d < 4e9 else 2
         torch.cuda.synchronize()
         barrier(world)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record()
         for _ in range(e_steps):
-            for g, h, wd_, gd_ in zip(groups, host, Wd, Gd):
-                wd_.copy_(h["W"], non_blocking=True)
-                gd_.copy_(h["G"], non_blocking=True)
-                g["step"](g["st"], wd_, gd_)
-                h["W"].copy_(wd_, non_blocking=True)
+            for g, h in zip(groups, host):
+                g["W"].copy_(h["W"], non_blocking=True)
+                g["grads"][-1].copy_(h["G"], non_blocking=True)
+                g["step"](g["st"], g["W"], g["grads"][-1])
+                h["W"].copy_(g["W"], non_blocking=True)
         s1.record()
         torch.cuda.synchronize()
         barrier(world)
         e2e = (max_over_ranks(s0.elapsed_time(s1) / e_steps, world), h2d, d2h)
+        del host
     return dict(ms_step=ms_step, clocks=clk.summary(), ns_ms=ns_ms, ns_flops=ns_flops,
-                cod_ms=cod_ms, cod_bytes=cod_bytes, e2e=e2e, cub_ms=cub_ms,
+                ns_launches=ns_launches, cod_ms=cod_ms, e2e=e2e, cub_ms=cub_ms,
                 cub_flops_dense=cub_flops_dense)
 
 
-def run_ours(args, world, rank, local):
-    from bit_muon_optimizer_b200 import gmuon as gm
+def codec_bytes(w: WL.Workload, groups) -> float:
+    """Algorithmic HBM bytes of the codec half (worked steps 1-5) per step: read
+    G and the old 4-bit codes and grid scales, write the new ones and the
+    16-bit NS input (the k (m + n) factor bytes are ignored)."""
+    gb = 2 if w.gdtype != torch.float32 else 4
+    return sum(g["B"] * g["m"] * g["n"] for g in groups) * (gb + 2 * (0.5 + 0.0625) + 2)
+
+
+def run_single(gm, w, ns_mode, args, local):
     dev = torch.device("cuda", local)
-    w = WL.WORKLOADS[args.config]
-    ns_mode = gm.GM_NS_GRAM if args.ns == "gram" else gm.GM_NS_STANDARD
-    hbm, bf16, bf16_sus, peak_kind = _peaks()
     total_mem = torch.cuda.get_device_properties(dev).total_memory
     pool = min(GRAD_POOL, args.warmup + args.steps)
     if est_bytes(w, pool) > 0.7 * total_mem:
@@ -460,103 +457,173 @@ def run_ours(args, world, rank, local):
     # groups are independent and each fills the GPU, so the set's time is the sum
     per_group = est_bytes(w, pool) > 0.7 * total_mem
     batches = [[gi] for gi in range(len(w.groups))] if per_group else [list(range(len(w.groups)))]
-    do_e2e = not args.no_e2e and not per_group
     res = []
     for gis in batches:
-        groups = [build_group(gm, w, gi, ns_mode, rank, pool, dev) for gi in gis]
-        res.append(measure(gm, w, groups, ns_mode, args, world, local, do_e2e))
+        groups = [build_group(gm, w, gi, ns_mode, pool, dev) for gi in gis]
+        r = measure(gm, w, groups, ns_mode, args, 1, local, not args.no_e2e)
+        r["codec_bytes"] = codec_bytes(w, groups)
+        res.append(r)
         del groups
         torch.cuda.empty_cache()
-    ms_step = sum(r["ms_step"] for r in res)
-    ns_ms = sum(r["ns_ms"] for r in res)
-    ns_flops = sum(r["ns_flops"] for r in res)
-    cod_ms = sum(r["cod_ms"] for r in res)
-    cod_bytes = sum(r["cod_bytes"] for r in res)
-    cub_ms = sum(r["cub_ms"] for r in res)
-    cub_dense = sum(r["cub_flops_dense"] for r in res)
-    ns_tflops = ns_flops / (ns_ms * 1e-3) / 1e12
-    codec_gbs = cod_bytes / (cod_ms * 1e-3) / 1e9
+    out = {k: sum(r[k] for r in res) for k in ("ms_step", "ns_ms", "ns_flops", "ns_launches",
+                                                 "cod_ms", "cub_ms", "cub_flops_dense",
+                                                 "codec_bytes")}
     clk = [r["clocks"] for r in res if r["clocks"]]
-    clocks = None
+    out["clocks"] = None
     if clk:
-        clocks = {"sm_mhz": statistics.median([c["sm_mhz"] for c in clk]),
-                  "sm_max_mhz": clk[0]["sm_max_mhz"],
-                  "reasons": sorted(set(x for c in clk for x in c["reasons"])),
-                  "samples": sum(c["samples"] for c in clk)}
-    e2e = None
-    if res[0]["e2e"] is not None:
-        e_ms, h2d, d2h = res[0]["e2e"]
-        e2e = {"value": e_ms / world, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h)}
+        out["clocks"] = {"sm_mhz": statistics.median([c["sm_mhz"] for c in clk]),
+                         "sm_max_mhz": clk[0]["sm_max_mhz"],
+                         "reasons": sorted(set(x for c in clk for x in c["reasons"])),
+                         "samples": sum(c["samples"] for c in clk)}
+    out["e2e"] = None
+    if all(r["e2e"] is not None for r in res):
+        out["e2e"] = {"value": sum(r["e2e"][0] for r in res), "unit": UNIT,
+                      "h2d_bytes_per_step": int(sum(r["e2e"][1] for r in res)),
+                      "d2h_bytes_per_step": int(sum(r["e2e"][2] for r in res))}
+    out["graph"] = ("one CUDA graph per gradient slot, one stream per shape group"
+                    + ("; shape groups measured one at a time (device memory), set time = sum"
+                       if per_group else ""))
+    out["pool"] = pool
+    out["launches"] = our_launches(gm, w, ns_mode) * args.steps
+    return out
 
-    # ---- our kernels launched per step: per group 9 codec kernels (column norms,
-    # warm start with the factor fragments, rebuild + projection, three
-    # orthonormalisation kernels, back projection, its finalisation, the 4-bit
-    # quantisation with the 8-bit one folded in), the NS products, and the
-    # zero-padding copy when a dimension is not a multiple of 64
-    launches = 0
-    for g in w.groups:
-        pad = int(min(g.m, g.n) % 64 != 0 or max(g.m, g.n) % 64 != 0)
-        launches += 9 + gm.ns_flops(ns_mode, g.m, g.n, w.T)[1] + pad
-    launches *= args.steps
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
-        ms_cpu, sample, cores = oracle_sample_seconds(w, args.ns, 20.0)
-        cpu = {"value": ms_cpu, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+def run_sharded(gm, w, ns_mode, args, world, rank, local):
+    """N > 1: the set split by ownership (sharding.ShardedStep: LPT owners, the
+    owners' GRASP steps, one NCCL all-gather of the updated fp32 weights per
+    shape group), one shape group at a time; eager launches (the exchange is
+    torch.distributed). Returns the max over ranks of the summed group times."""
+    from bit_muon_optimizer_b200 import sharding as S
+    dev = torch.device("cuda", local)
+    make = S.grasp_make_step(w.k, dev, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=ns_mode, seed=w.seed)
+    ms_total, clocks, launches, owned = 0.0, [], 0, []
+    for gi, g in enumerate(w.groups):
+        base = w.group_base(gi)
+        sh = S.ShardedStep([(g.m, g.n, g.count)], world, rank, make, first_index=base)
+        W = torch.empty((g.count, g.m, g.n), dtype=torch.float32, device=dev)
+        grads = []
+        for b in range(g.count):
+            W[b] = WL.initial_weight(w, base + b, g.m, g.n, device=dev)
+        for t in (1, 2):
+            G = torch.empty((g.count, g.m, g.n), dtype=w.gdtype, device=dev)
+            for b in range(g.count):
+                WL.gradient(w, base + b, t, g.m, g.n, device=dev, out=G[b])
+            grads.append(G)
+        for t in range(args.warmup):
+            sh([W], [grads[t % 2]])
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local) as clk:
+            torch.cuda.synchronize()
+            barrier(world)
+            e0.record()
+            for t in range(args.steps):
+                sh([W], [grads[t % 2]])
+            e1.record()
+            torch.cuda.synchronize()
+            barrier(world)
+        ms_total += max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+        if clk.summary():
+            clocks.append(clk.summary())
+        mine = len(sh.owned[0][rank])
+        owned.append(mine)
+        if mine:
+            launches += our_launches(gm, w, ns_mode, [(g.m, g.n)])
+        del sh, W, grads
+        torch.cuda.empty_cache()
+    clk = None
+    if clocks:
+        clk = {"sm_mhz": statistics.median([c["sm_mhz"] for c in clocks]),
+               "sm_max_mhz": clocks[0]["sm_max_mhz"],
+               "reasons": sorted(set(x for c in clocks for x in c["reasons"])),
+               "samples": sum(c["samples"] for c in clocks)}
+    return ms_total, clk, launches * args.steps, owned
 
+
+def run_ours(args, world, rank, local):
+    from bit_muon_optimizer_b200 import gmuon as gm
+    w = WL.WORKLOADS[args.config]
+    ns_mode = gm.GM_NS_GRAM if args.ns == "gram" else gm.GM_NS_STANDARD
+    hbm, bf16, bf16_sus, peak_kind = _peaks()
     elements = sum(g.count * g.m * g.n for g in w.groups)
     step_flops = sum(gm.ns_flops(ns_mode, g.m, g.n, w.T)[0] * g.count for g in w.groups)
     step_bytes = elements * FL.step_bytes_per_element(2 if w.gdtype != torch.float32 else 4)
     t_roof = max(step_flops / (bf16 * 1e12), step_bytes / (hbm * 1e9)) * 1e3
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": ms_step / world, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if ns_mode == gm.GM_NS_STANDARD else "f16",
-            "data": "synthetic",
-            "config": {"workload": w.name, "ns": args.ns, "k": w.k,
-                       "shapes": [[g.m, g.n, g.count] for g in w.groups],
-                       "elements": elements, "grad_dtype": str(w.gdtype).replace("torch.", ""),
-                       "l2": "per-step working set (G, W, state, fp32 M) > L2; no flush",
-                       "parallelism": f"weak x{world}, one parameter set per rank",
-                       "graph": ("one CUDA graph per gradient slot, one stream per shape group"
-                                 + ("; shape groups measured one at a time (device memory), "
-                                    "set time = sum" if per_group else "")),
-                       "grad_pool": pool},
-            "roofline": {"bound": "tensor", "achieved": ns_tflops, "peak": bf16, "unit": "TFLOP/s",
-                         "frac": ns_tflops / bf16, "traffic": gemm_traffic(args.config, args.ns),
-                         "kernel": "k_gemm: the NS chains' tcgen05 products of all groups, graph-replayed alone",
-                         "peak_kind": f"{peak_kind} bf16 dense burst"},
-            "ns": {"tflops": ns_tflops, "ms": ns_ms, "flops": ns_flops},
-            "cublas_ns": {"ms": cub_ms, "tflops_algorithmic": ns_flops / (cub_ms * 1e-3) / 1e12
-                          if args.ns == "standard" else None,
-                          "tflops_dense": cub_dense / (cub_ms * 1e-3) / 1e12,
-                          "what": "standard NS, T steps of torch.matmul / baddbmm (cuBLAS bf16, "
-                                  "dense products), same inputs and streams"},
-            "codec": {"gbs": codec_gbs, "peak_gbs": hbm, "frac": codec_gbs / hbm,
-                      "ms": cod_ms,
-                      "kernels": "rebuild (k_dequant_rebuild) + residual grid quantisation "
-                                 "(k_residual_quant4) through the standalone entry points, "
-                                 "which stage the factor fragments in each CTA"},
-            "step_minus_ns_ms": ms_step - ns_ms,
-            "step_roofline": {"ms": t_roof, "frac": t_roof / ms_step, "flops": step_flops,
-                              "bytes": step_bytes},
-            "gpu_launches": launches,
-            "clocks": clocks,
-            "e2e": e2e,
-            "cpu_baseline": cpu,
-        }
-        print(json.dumps(line), flush=True)
+    config = {"workload": w.name, "ns": args.ns, "k": w.k,
+              "shapes": [[g.m, g.n, g.count] for g in w.groups],
+              "elements": elements, "grad_dtype": str(w.gdtype).replace("torch.", ""),
+              "l2": "per-step working set (G, W, state, fp32 M) > L2; no flush"}
+    dtype = "bf16" if ns_mode == gm.GM_NS_STANDARD else "f16"
+    if world > 1:
+        ms_step, clocks, launches, owned = run_sharded(gm, w, ns_mode, args, world, rank, local)
+        if rank == 0:
+            config.update(parallelism=f"ownership sharding x{world}: LPT owners per shape group, "
+                                      "one NCCL all-gather of the updated fp32 weights per group",
+                          graph="eager launches, shape groups one at a time, set time = sum",
+                          owned_per_group_rank0=owned)
+            line = {"metric": METRIC, "value": ms_step, "unit": UNIT, "n_gpus": world,
+                    "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                    "higher_is_better": False, "scaling": "strong", "vs_baseline": None,
+                    "dtype": dtype, "data": "synthetic", "config": config,
+                    "step_roofline": {"ms": t_roof, "frac": t_roof / world / ms_step,
+                                      "flops": step_flops, "bytes": step_bytes,
+                                      "note": "single-GPU roofline / N"},
+                    "gpu_launches": launches, "clocks": clocks, "e2e": None, "cpu_baseline": None}
+            print(json.dumps(line), flush=True)
+        return
+    r = run_single(gm, w, ns_mode, args, local)
+    ns_tflops = r["ns_flops"] / (r["ns_ms"] * 1e-3) / 1e12
+    codec_gbs = r["codec_bytes"] / (r["cod_ms"] * 1e-3) / 1e9
+    long_step = r["ms_step"] > 50.0
+    peak = bf16_sus if long_step else bf16
+    cpu = None
+    if not args.no_cpu:
+        ms_cpu, sample, cores = oracle_sample_seconds(w, args.ns)
+        cpu = {"value": ms_cpu, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+    config.update(parallelism="single GPU", graph=r["graph"], grad_pool=r["pool"])
+    line = {
+        "metric": METRIC, "value": r["ms_step"], "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_step"],
+        "higher_is_better": False, "scaling": "strong", "vs_baseline": None,
+        "dtype": dtype, "data": "synthetic", "config": config,
+        "roofline": {"bound": "tensor", "achieved": ns_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": ns_tflops / peak, "traffic": gemm_traffic(args.config, args.ns),
+                     "kernel": "k_gemm: the NS half of the step (gm_grasp_apply: "
+                               f"{r['ns_launches']} tcgen05 products per step), CUDA events "
+                               "around it on its launching stream",
+                     "peak_kind": f"{peak_kind} bf16 dense "
+                                  + ("sustained (kernel timed inside a step of "
+                                     f"{r['ms_step']:.0f} ms)" if long_step else "burst")},
+        "ns": {"tflops": ns_tflops, "ms": r["ns_ms"], "flops": r["ns_flops"],
+               "frac_of_burst_peak": ns_tflops / bf16},
+        "cublas_ns": {"ms": r["cub_ms"],
+                      "tflops_algorithmic": r["ns_flops"] / (r["cub_ms"] * 1e-3) / 1e12
+                      if args.ns == "standard" else None,
+                      "tflops_dense": r["cub_flops_dense"] / (r["cub_ms"] * 1e-3) / 1e12,
+                      "what": "standard NS, T steps of torch.matmul / baddbmm (cuBLAS bf16, "
+                              "dense products), same inputs"},
+        "codec": {"gbs": codec_gbs, "peak_gbs": hbm, "frac": codec_gbs / hbm, "ms": r["cod_ms"],
+                  "bytes": r["codec_bytes"],
+                  "kernels": "the codec half of the step (gm_grasp_state_update: 9 kernels per "
+                             "group), CUDA events around it; algorithmic bytes G + old and new "
+                             "codes and scales + the 16-bit NS input"},
+        "step_roofline": {"ms": t_roof, "frac": t_roof / r["ms_step"], "flops": step_flops,
+                          "bytes": step_bytes},
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+        "e2e": r["e2e"],
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--ns", choices=["standard", "gram"], default="standard")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")

@@ -18,19 +18,21 @@ size_t al256(size_t b) { return (b + 255) & ~size_t(255); }
 
 const float kQuintic[3] = {3.4445f, -4.7750f, 2.0315f};
 
+// The current device is an sm_100 part (checked once per device).
 bool device_ok() {
-  static int checked_dev = -1;
-  static bool ok = false;
+  static std::atomic<int> verdict[kMaxDevices];   // 0 unknown, 1 sm_100, 2 other
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  if (dev != checked_dev) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  int v = verdict[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
     int major = 0, minor = 0;
-    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-    ok = (major == 10 && minor == 0);
-    checked_dev = dev;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return false;
+    v = (major == 10 && minor == 0) ? 1 : 2;
+    verdict[dev].store(v, std::memory_order_relaxed);
   }
-  return ok;
+  return v == 1;
 }
 
 bool shape_ok(int B, int m, int n) {
@@ -251,8 +253,8 @@ gm_status gm_momentum_powerit(int B, int m, int n, int k, float mu, const float*
   float* scale = reinterpret_cast<float*>(w + L.scale);
   uint32_t* QF = reinterpret_cast<uint32_t*>(w + L.QF);
   uint32_t* PB = reinterpret_cast<uint32_t*>(w + L.PB);
-  GM_CUDA(launch_warm_start(B, m, n, k, nullptr, nullptr, nullptr, nullptr, R_prev, seed, Q, nullptr,
-                            QF, nullptr, nullptr, nullptr, s));
+  GM_CUDA(launch_warm_start(B, m, n, k, nullptr, nullptr, nullptr, nullptr, R_prev, seed, nullptr, Q,
+                            nullptr, QF, nullptr, nullptr, nullptr, s));
   GM_CUDA(launch_rebuild(B, m, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                          M_prev, mu, G, gdt, Q, QF, nullptr, nullptr, M_out, norm2, Ppart, nullptr, s));
   GM_CUDA(launch_orth(B, m, k, L.csplit, Ppart, Ptil, gram, Tm, norm2, L.ntiles, 1e-7f, scale,
@@ -357,9 +359,11 @@ gm_status gm_gram_ns(int B, int m, int n, const void* X, gm_dtype xdt, const flo
                    stream, true);
 }
 
-gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* prm, const gm_grasp_state* st,
-                        float* W, const void* G, gm_dtype gdt, void* ws, size_t ws_bytes,
-                        gm_stream_t stream) {
+// Argument checks shared by the step and its two halves (W, G: NULL where the
+// half does not take them).
+static gm_status step_checks(int B, int m, int n, const gm_grasp_params* prm, const gm_grasp_state* st,
+                             const float* W, bool need_w, const void* G, bool need_g, gm_dtype gdt,
+                             void* ws, size_t ws_bytes, StepLayout* L) {
   GM_CHECK_ARG(prm && st, "NULL params or state");
   GM_CHECK_ARG(shape_ok(B, m, n), "bad shape B=%d m=%d n=%d", B, m, n);
   const int k = prm->k;
@@ -369,18 +373,34 @@ gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* prm, const g
   GM_CHECK_ARG(prm->n_restart >= 0 && (prm->n_restart == 0 || prm->restart_after),
                "bad restart list");
   GM_CHECK_ARG(prm->eps >= 0.f, "eps < 0");
+  GM_CHECK_ARG(prm->power_steps >= 0 && prm->power_steps <= 3, "power_steps=%d out of [0, 3]",
+               prm->power_steps);
+  GM_CHECK_ARG(prm->residual_from_codes == 0 || prm->residual_from_codes == 1,
+               "residual_from_codes must be 0 or 1");
+  GM_CHECK_ARG(al16(prm->matrix_ids), "matrix_ids must be 16-byte aligned");
   GM_CHECK_ARG(st->codes4 && st->rscale && st->cscale && st->P8 && st->Pscale && st->R8 &&
                    st->Rscale && st->step && st->dev_status,
                "NULL state pointer");
-  GM_CHECK_ARG(W && G, "NULL W or G");
+  GM_CHECK_ARG(!need_w || W, "NULL W");
+  GM_CHECK_ARG(!need_g || G, "NULL G");
   GM_CHECK_ARG(al16(W) && al16(G) && al16(st->codes4) && al16(st->rscale) && al16(st->cscale) &&
                    al16(st->P8) && al16(st->Pscale) && al16(st->R8) && al16(st->Rscale),
                "device arrays must be 16-byte aligned");
-  GM_CHECK_ARG(gdt == GM_F32 || gdt == GM_BF16 || gdt == GM_F16, "bad gdt");
-  StepLayout L = step_layout(B, m, n, k, prm->ns, true);
-  if (!ws || ws_bytes < L.total || !aligned256(ws))
-    return set_error(GM_E_WORKSPACE, "workspace needs %zu bytes, 256-aligned", L.total);
+  GM_CHECK_ARG(!need_g || gdt == GM_F32 || gdt == GM_BF16 || gdt == GM_F16, "bad gdt");
+  *L = step_layout(B, m, n, k, prm->ns, true);
+  if (!ws || ws_bytes < L->total || !aligned256(ws))
+    return set_error(GM_E_WORKSPACE, "workspace needs %zu bytes, 256-aligned", L->total);
   GM_DEVICE();
+  return GM_OK;
+}
+
+gm_status gm_grasp_state_update(int B, int m, int n, const gm_grasp_params* prm,
+                                const gm_grasp_state* st, const void* G, gm_dtype gdt, void* ws,
+                                size_t ws_bytes, gm_stream_t stream) {
+  StepLayout L;
+  const gm_status chk = step_checks(B, m, n, prm, st, nullptr, false, G, true, gdt, ws, ws_bytes, &L);
+  if (chk != GM_OK) return chk;
+  const int k = prm->k;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);
   float* M = reinterpret_cast<float*>(w + L.M);
@@ -402,37 +422,79 @@ gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* prm, const g
   uint32_t* RB = reinterpret_cast<uint32_t*>(w + L.RB);
   uint32_t* PB = reinterpret_cast<uint32_t*>(w + L.PB);
   int32_t* status = st->dev_status;
-  float tab[3 * GM_MAX_T];
-  expand_abc(prm->abc, prm->T, tab);
   const bool gramns = prm->ns == GM_NS_GRAM;
+  const int psteps = prm->power_steps < 1 ? 1 : prm->power_steps;
+  unsigned* PRmax = reinterpret_cast<unsigned*>(w + L.qnorm) + (size_t)B * k;
 
   GM_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
   // worked step 2: warm start from the stored R (read before it is overwritten)
   // (with the fragment copies of Q, R and P that the rebuild reads)
   GM_CUDA(launch_warm_start(B, m, n, k, st->R8, st->Rscale, st->P8, st->Pscale, nullptr, prm->seed,
-                            Q, reinterpret_cast<int*>(w + L.qnorm), QF, RF, PF, status, s));
+                            prm->matrix_ids, Q, reinterpret_cast<int*>(w + L.qnorm), QF, RF, PF,
+                            status, s));
   // worked steps 1 and 3: rebuild M_{t-1}, M_t = mu M_{t-1} + G
   // (with the projection P~ = M Q of worked step 4 fused in)
   GM_CUDA(launch_rebuild(B, m, n, k, st->codes4, st->rscale, st->cscale, st->P8, st->Pscale,
                          st->R8, st->Rscale, nullptr, prm->mu, G, gdt, Q, QF, RF, PF, M, norm2, Ppart,
                          status, s));
-  // worked step 4: P = orth(P~), R = M^T P
-  unsigned* PRmax = reinterpret_cast<unsigned*>(w + L.qnorm) + (size_t)B * k;
+  // worked step 4: P = orth(P~), R = M^T P (and the normalised NS input X)
   GM_CUDA(launch_orth(B, m, k, L.csplit, Ppart, Ptil, gram, Tm, norm2, L.ntiles, prm->eps, scale,
                       P, PB, PA, PRmax, status, s));
   GM_CUDA(launch_backproject(B, m, n, k, M, PB, scale, X, gramns, Rpart, R, RB, PRmax + (size_t)B * k,
                              status, s));
+  // further power-iteration steps: Q = column-normalised R, P~ = M Q (a projection
+  // pass over the stored M_t), P = orth(P~), R = M^T P
+  for (int it = 1; it < psteps; ++it) {
+    GM_CUDA(launch_warm_start(B, m, n, k, nullptr, nullptr, nullptr, nullptr, R, prm->seed,
+                              prm->matrix_ids, Q, nullptr, QF, nullptr, nullptr, status, s));
+    GM_CUDA(launch_rebuild(B, m, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                           nullptr, M, 1.0f, nullptr, GM_F32, Q, QF, nullptr, nullptr, nullptr,
+                           nullptr, Ppart, status, s));
+    GM_CUDA(cudaMemsetAsync(PRmax, 0, sizeof(unsigned) * 2 * (size_t)B * k, s));
+    GM_CUDA(launch_orth(B, m, k, L.csplit, Ppart, Ptil, gram, Tm, norm2, L.ntiles, prm->eps, scale,
+                        P, PB, PA, PRmax, status, s));
+    GM_CUDA(launch_backproject(B, m, n, k, M, PB, nullptr, nullptr, gramns, Rpart, R, RB,
+                               PRmax + (size_t)B * k, status, s));
+  }
+  // worked step 5 variant: the residual from the dequantized 8-bit factors
+  if (prm->residual_from_codes)
+    GM_CUDA(launch_codes_frags(B, m, n, k, P, R, PRmax, PRmax + (size_t)B * k, PA, RB, status, s));
   // worked step 5: residual -> 4-bit grid codes; P, R -> 8-bit codes (state in place)
   GM_CUDA(launch_residual_quant4(B, m, n, k, M, P, R, PA, RB, st->codes4, st->rscale, st->cscale,
                                  PRmax, st->P8, st->Pscale, st->R8, st->Rscale, st->step, status, s));
+  return GM_OK;
+}
+
+gm_status gm_grasp_apply(int B, int m, int n, const gm_grasp_params* prm, const gm_grasp_state* st,
+                         float* W, void* ws, size_t ws_bytes, gm_stream_t stream) {
+  StepLayout L;
+  const gm_status chk = step_checks(B, m, n, prm, st, W, true, nullptr, false, GM_F32, ws, ws_bytes, &L);
+  if (chk != GM_OK) return chk;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* X = reinterpret_cast<uint16_t*>(w + L.X);
+  int32_t* status = st->dev_status;
+  float tab[3 * GM_MAX_T];
+  expand_abc(prm->abc, prm->T, tab);
   // worked step 6: O = NS(M_t); W <- W - eta (O + wd W) in the last product's epilogue
   NsOutput out{1, nullptr, 0, W, prm->eta, prm->wd};
-  if (gramns)
+  if (prm->ns == GM_NS_GRAM)
     GM_CUDA(run_ns_gram(B, m, n, X, tab, prm->T, prm->restart_after, prm->n_restart, out,
                         w + L.ns, status, status, s));
   else
     GM_CUDA(run_ns_standard(B, m, n, X, tab, prm->T, out, w + L.ns, status, status, s));
   return GM_OK;
+}
+
+gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* prm, const gm_grasp_state* st,
+                        float* W, const void* G, gm_dtype gdt, void* ws, size_t ws_bytes,
+                        gm_stream_t stream) {
+  StepLayout L;
+  const gm_status chk = step_checks(B, m, n, prm, st, W, true, G, true, gdt, ws, ws_bytes, &L);
+  if (chk != GM_OK) return chk;
+  const gm_status a = gm_grasp_state_update(B, m, n, prm, st, G, gdt, ws, ws_bytes, stream);
+  if (a != GM_OK) return a;
+  return gm_grasp_apply(B, m, n, prm, st, W, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -164,10 +164,12 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_us
 // ------------------------------------------------------------------ S2
 __global__ void __launch_bounds__(kThreads) k_warm_start(int n, int k, const int8_t* R8,
                                                           const float* Rscale, const float* Rprev,
-                                                          uint64_t seed, float* Q, uint32_t* QF,
+                                                          uint64_t seed, const int64_t* ids,
+                                                          float* Q, uint32_t* QF,
                                                           const int32_t* skip) {
   if (skip && *skip) return;
   const int b = blockIdx.x, t = threadIdx.x;
+  const uint64_t bid = ids ? (uint64_t)ids[b] : (uint64_t)b;   // the matrix's counter index
   const long long off = (long long)b * n * k;
   __shared__ double red[kThreads];
   __shared__ double nrm2[kMaxK];
@@ -201,7 +203,7 @@ __global__ void __launch_bounds__(kThreads) k_warm_start(int n, int k, const int
     if (j < n && l < k) {
       const double inv = nrm2[l];
       if (inv == 0.0) {
-        const uint64_t ctr = seed ^ ((uint64_t)b << 48) ^ ((uint64_t)j << 16) ^ (uint64_t)l;
+        const uint64_t ctr = seed ^ (bid << 48) ^ ((uint64_t)j << 16) ^ (uint64_t)l;
         q = (splitmix64(ctr) >> 63) ? -rad : rad;
       } else {
         q = (float)((double)rhat(j, l) * inv);
@@ -257,6 +259,7 @@ __global__ void __launch_bounds__(kThreads) k_warm_q(int m, int n, int k, int nb
                                                       const int8_t* __restrict__ P8,
                                                       const float* __restrict__ Pscale,
                                                       const int* __restrict__ norm2, uint64_t seed,
+                                                      const int64_t* __restrict__ ids,
                                                       float* __restrict__ Q, uint32_t* __restrict__ QF,
                                                       uint16_t* __restrict__ RF, uint16_t* __restrict__ PF,
                                                       const int32_t* skip) {
@@ -287,7 +290,8 @@ __global__ void __launch_bounds__(kThreads) k_warm_q(int m, int n, int k, int nb
         if (valid) {
           const double iv = inv[l];
           if (iv == 0.0) {
-            const uint64_t ctr = seed ^ ((uint64_t)b << 48) ^ ((uint64_t)j << 16) ^ (uint64_t)l;
+            const uint64_t bid = ids ? (uint64_t)ids[b] : (uint64_t)b;
+            const uint64_t ctr = seed ^ (bid << 48) ^ ((uint64_t)j << 16) ^ (uint64_t)l;
             q = (splitmix64(ctr) >> 63) ? -rad : rad;
           } else {
             q = (float)((double)rq * iv);
@@ -578,7 +582,7 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_pipe(
       for (int u = 0; u < GCH / 2; ++u) {
         const void* src = ok ? (G32 ? (const void*)(static_cast<const float*>(G) + base + 4 * u)
                                     : (const void*)(static_cast<const uint16_t*>(G) + base + 8 * u))
-                             : G ? G : (const void*)M;
+                             : G ? G : (Mprev ? (const void*)Mprev : (const void*)M);
         cp_async16(&GSs(s)[(h * (GCH / 2) + u) * kRBT + t], src, ok);
       }
       if constexpr (DN) {
@@ -693,7 +697,7 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_pipe(
           nsq = fmaf(o, o, nsq);
         }
       }
-      if (ok) {
+      if (ok && M) {   // M == NULL: the projection alone (a repeated power-iteration step)
         float4* dst = reinterpret_cast<float4*>(M + (long long)b * mn + (long long)gi * n + cb);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -1182,6 +1186,52 @@ __device__ __forceinline__ int8_t code8(float x, float s, float r127) {
 }
 constexpr int kQ8PerThread = kGrid * kMaxK / kCT;   // P or R values per thread, 128 rows
 
+// The residual-from-codes variant: the residual pass's factor fragments PA (-P^)
+// and RB (R^) rebuilt from this step's 8-bit codes, P^ = deq8(code8(P)) and
+// R^ = deq8(code8(R)), instead of the unquantized P and R. Pmax / Rmax hold the
+// complete column absolute maxima (the 8-bit scales). Elements [0, m k) are P's,
+// [m k, (m + n) k) R's; fragment slots of columns l >= k keep their zeros.
+template <int KP>
+__global__ void __launch_bounds__(kThreads) k_codes_frags(int m, int n, int k,
+                                                           const float* __restrict__ P,
+                                                           const float* __restrict__ R,
+                                                           const unsigned* __restrict__ Pmax,
+                                                           const unsigned* __restrict__ Rmax,
+                                                           uint32_t* __restrict__ PA,
+                                                           uint32_t* __restrict__ RB,
+                                                           const int32_t* skip) {
+  if (skip && *skip) return;
+  const int b = blockIdx.y, t = threadIdx.x;
+  __shared__ float s8[2][kMaxK], r127[2][kMaxK];
+  if (t < 2 * kMaxK) {
+    const int w = t / kMaxK, l = t % kMaxK;
+    const float sv = l < k ? __uint_as_float((w ? Rmax : Pmax)[b * k + l]) : 0.f;
+    s8[w][l] = sv;
+    r127[w][l] = sv > 0.f ? __fdiv_rn(127.0f, sv) : 0.f;
+  }
+  __syncthreads();
+  const long long e = (long long)blockIdx.x * kThreads + t;
+  const long long np = (long long)m * k, nr = (long long)n * k;
+  if (e < np) {
+    const int i = (int)(e / k), l = (int)(e % k);
+    const float x = P[(long long)b * np + e];
+    const float v = -deq8(code8(x, s8[0][l], r127[0][l]), s8[0][l]);
+    const long long at = pa_at(b, m >> 4, KP / 8, i, l);
+    const uint32_t hi = tf32_hi(v);
+    PA[at] = hi;
+    PA[at + 128] = tf32_lo(v, hi);
+  } else if (e < np + nr) {
+    const long long e2 = e - np;
+    const int j = (int)(e2 / k), l = (int)(e2 % k);
+    const float x = R[(long long)b * nr + e2];
+    const float v = deq8(code8(x, s8[1][l], r127[1][l]), s8[1][l]);
+    const long long at = rb_at(b, cdiv(n, 64), KP / 8, j, l);
+    const uint32_t hi = tf32_hi(v);
+    RB[at] = hi;
+    RB[at + 2] = tf32_lo(v, hi);
+  }
+}
+
 template <int KP, bool FR>   // KP = 0: no rank-k term
 __global__ void __launch_bounds__(kCT, 1) k_residual_quant4(
     int m, int n, int k, const float* __restrict__ X, const float* __restrict__ P,
@@ -1513,12 +1563,10 @@ cudaError_t launch_backproject_t(int B, int m, int n, int k, const float* M, con
                                  cudaStream_t s) {
   const int rs = backproject_row_splits(B, m, n);
   const size_t smem = (size_t)2 * 8 * 8 * 32 * sizeof(float4);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_backproject<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+  static DeviceOnce attr;
+  {
+    const cudaError_t e = smem_attr_once(attr, k_backproject<KP>, smem);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   dim3 grid(cdiv(n, 64), rs, B);
   k_backproject<KP><<<grid, kThreads, smem, s>>>(m, n, k, rs, M, PB, scale,
@@ -1537,12 +1585,10 @@ cudaError_t launch_residual_t(int B, int m, int n, int k, const float* X, const 
                               uint8_t* codes4, float* rscale, float* cscale, const Quant8Out& q8,
                               const int32_t* skip, cudaStream_t s) {
   const size_t smem = (size_t)(2 * 8 * (KP / 8) * 2 * 128 + (FR ? 0 : 2 * kGrid * KP)) * sizeof(uint32_t);
-  static bool attr = false;
-  if (!attr && smem > 0) {
-    cudaError_t e = cudaFuncSetAttribute(k_residual_quant4<KP, FR>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static DeviceOnce attr;
+  if (smem > 0) {
+    const cudaError_t e = smem_attr_once(attr, k_residual_quant4<KP, FR>, smem);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   dim3 grid(cdiv(n, kGrid), cdiv(m, kGrid), B);
   k_residual_quant4<KP, FR><<<grid, kCT, smem, s>>>(m, n, k, X, P, R, PA, RB, codes4, rscale, cscale,
@@ -1583,10 +1629,11 @@ FactorFrags factor_frag_words(int B, int m, int n, int k) {
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_warm_start(int B, int m, int n, int k, const int8_t* R8, const float* Rscale,
                               const int8_t* P8, const float* Pscale, const float* Rprev,
-                              uint64_t seed, float* Q, int* norm2_int, uint32_t* QF, uint32_t* RF,
-                              uint32_t* PF, const int32_t* skip, cudaStream_t s) {
+                              uint64_t seed, const int64_t* ids, float* Q, int* norm2_int,
+                              uint32_t* QF, uint32_t* RF, uint32_t* PF, const int32_t* skip,
+                              cudaStream_t s) {
   if (Rprev || !R8 || !norm2_int) {
-    k_warm_start<<<B, kThreads, 0, s>>>(n, k, R8, Rscale, Rprev, seed, Q, QF, skip);
+    k_warm_start<<<B, kThreads, 0, s>>>(n, k, R8, Rscale, Rprev, seed, ids, Q, QF, skip);
     return cudaGetLastError();
   }
   cudaError_t e = cudaMemsetAsync(norm2_int, 0, sizeof(int) * (size_t)3 * B * k, s);
@@ -1598,7 +1645,7 @@ cudaError_t launch_warm_start(int B, int m, int n, int k, const int8_t* R8, cons
   const int nbq = (int)cdivll((long long)cdiv(n, 64) * 64 * kb, kThreads * 4);
   const int nbp = (int)cdivll((long long)m * kb, kThreads * 4);
   k_warm_q<<<dim3(nbq + nbp, B), kThreads, 0, s>>>(m, n, k, nbq, R8, Rscale, P8, Pscale, norm2_int,
-                                                   seed, Q, QF, reinterpret_cast<uint16_t*>(RF),
+                                                   seed, ids, Q, QF, reinterpret_cast<uint16_t*>(RF),
                                                    reinterpret_cast<uint16_t*>(PF), skip);
   return cudaGetLastError();
 }
@@ -1608,12 +1655,10 @@ cudaError_t launch_dequant_t(int B, int m, int n, int k, const uint8_t* codes4, 
                              const float* cscale, const int8_t* P8, const float* Pscale,
                              const int8_t* R8, const float* Rscale, float* M, cudaStream_t s) {
   const size_t smem = (size_t)dequant_smem_words(KP) * sizeof(uint32_t);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_dequant_rebuild<KP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static DeviceOnce attr;
+  {
+    const cudaError_t e = smem_attr_once(attr, k_dequant_rebuild<KP>, smem);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   dim3 grid(cdiv(n, kGrid), cdiv(m, kRB), B);
   k_dequant_rebuild<KP><<<grid, kRBT, smem, s>>>(m, n, k, codes4, rscale, cscale, P8, Pscale, R8, Rscale, M);
@@ -1626,12 +1671,10 @@ cudaError_t launch_pipe_t(int B, int m, int n, cudaStream_t s, int k, const uint
                           const void* G, const uint32_t* QF, const uint32_t* RF, const uint32_t* PF,
                           float* M, double* norm2_part, float* Ppart, int32_t* status) {
   const size_t smem = (size_t)pipe_smem_words(SRC, GDT, KP) * sizeof(uint32_t);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_rebuild_pipe<SRC, GDT, KP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static DeviceOnce attr;
+  {
+    const cudaError_t e = smem_attr_once(attr, k_rebuild_pipe<SRC, GDT, KP>, smem);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   const int nb = cdiv(n, kGrid), nrb = cdiv(m, kRB);
   // tiles per CTA: up to kRebuildTiles while the grid keeps about four CTAs per SM
@@ -1714,6 +1757,17 @@ cudaError_t launch_residual_quant4(int B, int m, int n, int k, const float* X, c
   if (PA && RB) return kp == 8 ? GM_RQ(8, true) : (kp == 16 ? GM_RQ(16, true) : GM_RQ(32, true));
   return kp == 8 ? GM_RQ(8, false) : (kp == 16 ? GM_RQ(16, false) : GM_RQ(32, false));
 #undef GM_RQ
+}
+
+cudaError_t launch_codes_frags(int B, int m, int n, int k, const float* P, const float* R,
+                               const unsigned* Pmax, const unsigned* Rmax, uint32_t* PA,
+                               uint32_t* RB, const int32_t* skip, cudaStream_t s) {
+  const dim3 grid((unsigned)cdivll((long long)(m + n) * k, kThreads), B);
+  const int kp = factor_width(k);
+  if (kp == 8) k_codes_frags<8><<<grid, kThreads, 0, s>>>(m, n, k, P, R, Pmax, Rmax, PA, RB, skip);
+  else if (kp == 16) k_codes_frags<16><<<grid, kThreads, 0, s>>>(m, n, k, P, R, Pmax, Rmax, PA, RB, skip);
+  else k_codes_frags<32><<<grid, kThreads, 0, s>>>(m, n, k, P, R, Pmax, Rmax, PA, RB, skip);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_quant8(int B, int rows0, int rows1, int k, const float* X0, int8_t* c0,

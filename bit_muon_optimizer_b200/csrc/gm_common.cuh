@@ -7,6 +7,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/gmuon.h"
 
 namespace gm {
@@ -59,6 +62,43 @@ __host__ __device__ inline uint64_t splitmix64(uint64_t x) {
   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
   z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
   return z ^ (z >> 31);
+}
+
+// ------------------------------------------------- per-device one-time set-up
+// Kernel attributes and looked-up device addresses belong to a device (its
+// primary context), so every cache of them is keyed by the current device.
+constexpr int kMaxDevices = 64;
+
+// Runs `fn` once per device (the current one when called), thread-safe; a
+// failed `fn` is retried on the next call.
+class DeviceOnce {
+ public:
+  template <typename F>
+  cudaError_t run(F&& fn) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    const uint64_t bit = 1ull << dev;
+    if (done_.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (done_.load(std::memory_order_relaxed) & bit) return cudaSuccess;
+    e = fn();
+    if (e == cudaSuccess) done_.fetch_or(bit, std::memory_order_release);
+    return e;
+  }
+
+ private:
+  std::mutex mu_;
+  std::atomic<uint64_t> done_{0};
+};
+
+// cudaFuncSetAttribute(kernel, MaxDynamicSharedMemorySize, bytes) once per device.
+template <typename K>
+cudaError_t smem_attr_once(DeviceOnce& once, K kernel, size_t bytes) {
+  return once.run([&] {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  });
 }
 
 // --------------------------------------------------------------- errors

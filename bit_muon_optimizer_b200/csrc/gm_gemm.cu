@@ -834,17 +834,21 @@ __global__ void k_pad16(int B, int rows, int cols, int prow, int pcol, const uin
 }
 
 // ------------------------------------------------------------------ host side
+// The driver's tensor-map encoder (one function for every device of the process).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+  PFN_cuTensorMapEncodeTiled_v12000 f = fn.load(std::memory_order_acquire);
+  if (!f) {
     cudaDriverEntryPointQueryResult q;
     void* ptr = nullptr;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
             cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        q == cudaDriverEntryPointSuccess) {
+      f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+      fn.store(f, std::memory_order_release);
+    }
   }
-  return fn;
+  return f;
 }
 
 // Map over 16-bit elements with the 128-byte swizzle (innermost box extent 64).
@@ -881,13 +885,16 @@ bool map_chunks(CUtensorMap* m, const void* base, bool f16, int rows, int cols, 
   return encode(m, base, f16, 4, dims, strides, box);
 }
 
+// SM count of the current device (cached per device).
 int num_sms() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      return 148;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
   return n;
 }
@@ -898,12 +905,10 @@ struct Maps {
 
 template <bool B_MN>
 cudaError_t launch_gemm(const Maps& m, const GemmParams& p, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm<B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+  static DeviceOnce attr;
+  {
+    const cudaError_t e = smem_attr_once(attr, k_gemm<B_MN>, kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   const int tiles = p.sym ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
   const int total = tiles * p.batch;
@@ -1185,11 +1190,18 @@ void ns_schedule_flops(int ns_mode, int m, int n, int T, const int* restart_afte
   if (products) *products = cnt;
 }
 
+// Device address of the error word on the current device (looked up with that
+// device current, cached per device).
 int32_t* device_error_word() {
-  static int32_t* ptr = nullptr;
+  static std::atomic<int32_t*> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  int32_t* ptr = cache[dev].load(std::memory_order_acquire);
   if (!ptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) ptr = static_cast<int32_t*>(p);
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    ptr = static_cast<int32_t*>(p);
+    cache[dev].store(ptr, std::memory_order_release);
   }
   return ptr;
 }

@@ -29,10 +29,12 @@ FactorFrags factor_frag_words(int B, int m, int n, int k);
 // or from fp32 Rprev,
 // with its fragments QF; from the stored state also the R and P code fragments
 // RF, PF (P8, Pscale needed then).
+// ids (nullable, device int64 [B]): the matrices' indices in the Rademacher counter.
 cudaError_t launch_warm_start(int B, int m, int n, int k, const int8_t* R8, const float* Rscale,
                               const int8_t* P8, const float* Pscale, const float* Rprev,
-                              uint64_t seed, float* Q, int* norm2_int, uint32_t* QF, uint32_t* RF,
-                              uint32_t* PF, const int32_t* skip, cudaStream_t s);
+                              uint64_t seed, const int64_t* ids, float* Q, int* norm2_int,
+                              uint32_t* QF, uint32_t* RF, uint32_t* PF, const int32_t* skip,
+                              cudaStream_t s);
 
 // M = mu * Mprev + G where Mprev is either the rebuilt state (codes4 != NULL)
 // or a dense fp32 matrix (Mprev32 != NULL) or zero; with Q != NULL also the
@@ -73,6 +75,12 @@ cudaError_t launch_residual_quant4(int B, int m, int n, int k, const float* X, c
                                    const unsigned* PRmax, int8_t* P8, float* Pscale, int8_t* R8,
                                    float* Rscale, int64_t* step, const int32_t* skip,
                                    cudaStream_t s);
+
+// Residual-from-codes variant: PA, RB from the dequantized 8-bit codes of P, R
+// (Pmax, Rmax: their complete column absolute maxima).
+cudaError_t launch_codes_frags(int B, int m, int n, int k, const float* P, const float* R,
+                               const unsigned* Pmax, const unsigned* Rmax, uint32_t* PA,
+                               uint32_t* RB, const int32_t* skip, cudaStream_t s);
 
 cudaError_t launch_quant8(int B, int rows0, int rows1, int k, const float* X0, int8_t* c0,
                           float* s0, const float* X1, int8_t* c1, float* s1,

@@ -23,7 +23,6 @@ constexpr size_t kNoallocScratchBytes = GM_NOALLOC_SCRATCH_BYTES;   // 64 MiB pe
 // Every GPU that loads this library holds this array until the process exits.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {nullptr};
 

@@ -39,7 +39,8 @@ class GraspParams(ctypes.Structure):
     _fields_ = [("mu", c_float), ("eta", c_float), ("wd", c_float), ("k", c_int), ("T", c_int),
                 ("ns", c_int), ("abc", ctypes.POINTER(c_float)),
                 ("restart_after", ctypes.POINTER(c_int)), ("n_restart", c_int),
-                ("eps", c_float), ("seed", c_uint64)]
+                ("eps", c_float), ("seed", c_uint64), ("power_steps", c_int),
+                ("residual_from_codes", c_int), ("matrix_ids", vp)]
 
 
 class GraspStateC(ctypes.Structure):
@@ -78,6 +79,10 @@ _sig("gm_gram_ns", c_int, [c_int, c_int, c_int, vp, c_int, vp, c_int, vp, c_int,
                            c_int, vp, c_size_t, vp])
 _sig("gm_grasp_step", c_int, [c_int, c_int, c_int, ctypes.POINTER(GraspParams),
                               ctypes.POINTER(GraspStateC), vp, vp, c_int, vp, c_size_t, vp])
+_sig("gm_grasp_state_update", c_int, [c_int, c_int, c_int, ctypes.POINTER(GraspParams),
+                                      ctypes.POINTER(GraspStateC), vp, c_int, vp, c_size_t, vp])
+_sig("gm_grasp_apply", c_int, [c_int, c_int, c_int, ctypes.POINTER(GraspParams),
+                               ctypes.POINTER(GraspStateC), vp, vp, c_size_t, vp])
 _sig("gm_grasp_workspace_layout", c_int, [c_int, c_int, c_int, c_int, c_int,
                                           ctypes.POINTER(GraspWsLayout)])
 _sig("gm_ns_flops", c_int, [c_int, c_int, c_int, c_int, vp, c_int,
@@ -406,21 +411,34 @@ class GraspState:
 
 
 class GraspStep:
-    """Marshals one gm_grasp_step call for a fixed shape batch."""
+    """Marshals one gm_grasp_step call for a fixed shape batch.
+
+    ``matrix_ids`` (optional): each matrix's index in the whole parameter set,
+    used by the Rademacher start vectors (default 0 .. B-1); ``power_steps``
+    (1..3) and ``residual_from_codes`` select the ablation variants."""
 
     def __init__(self, B, m, n, k, mu=0.95, eta=0.02, wd=0.0, T=5, ns=GM_NS_STANDARD, abc=None,
-                 restart_after=(2,), eps=1e-7, seed=0, device=None, ws=None):
+                 restart_after=(2,), eps=1e-7, seed=0, device=None, ws=None, power_steps=1,
+                 residual_from_codes=False, matrix_ids=None):
         self.B, self.m, self.n, self.k = B, m, n, k
         self._abc = abc_table(abc, T)
         rl = list(restart_after) if ns == GM_NS_GRAM else []
         self._rarr = (c_int * max(1, len(rl)))(*rl)
+        dev = device or torch.device("cuda")
+        self.ids = None
+        if matrix_ids is not None:
+            ids = [int(i) for i in matrix_ids]
+            if len(ids) != B or not all(0 <= i < 65536 for i in ids):
+                raise ValueError("matrix_ids: B indices in [0, 65536) expected")
+            self.ids = torch.tensor(ids, dtype=torch.int64, device=dev)
         self.params = GraspParams(mu, eta, wd, k, T, ns,
                                   ctypes.cast(self._abc, ctypes.POINTER(c_float)) if self._abc else None,
                                   ctypes.cast(self._rarr, ctypes.POINTER(c_int)) if rl else None,
-                                  len(rl), eps, seed)
+                                  len(rl), eps, seed, int(power_steps), int(bool(residual_from_codes)),
+                                  self.ids.data_ptr() if self.ids is not None else None)
         self.ws_bytes = workspace_bytes(GM_OP_GRASP_STEP, B, m, n, k, ns)
         if ws is None:
-            ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device or torch.device("cuda"))
+            ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
         self.ws = ws
         lay = GraspWsLayout()
         _check(lib.gm_grasp_workspace_layout(B, m, n, k, ns, ctypes.byref(lay)),
@@ -439,6 +457,29 @@ class GraspStep:
         _check(lib.gm_grasp_step(self.B, self.m, self.n, ctypes.byref(self.params), ctypes.byref(st),
                                  _ptr(W), _ptr(G), _DT[G.dtype], _ptr(self.ws), self.ws_bytes,
                                  _stream()), "gm_grasp_step")
+
+    def state_update(self, state: GraspState, G):
+        """Worked steps 1-5 alone (gm_grasp_state_update)."""
+        B, m, n = self.B, self.m, self.n
+        _expect(G, (B, m, n), tuple(_DT), "G")
+        state.check(B, m, n, self.k)
+        _placed((G,), ("G",))
+        _ws_fits(self.ws, self.ws_bytes)
+        st = state.c_struct()
+        _check(lib.gm_grasp_state_update(B, m, n, ctypes.byref(self.params), ctypes.byref(st),
+                                         _ptr(G), _DT[G.dtype], _ptr(self.ws), self.ws_bytes,
+                                         _stream()), "gm_grasp_state_update")
+
+    def apply(self, state: GraspState, W):
+        """Worked step 6 alone (gm_grasp_apply) on the NS input the state update left."""
+        B, m, n = self.B, self.m, self.n
+        _expect(W, (B, m, n), (torch.float32,), "W")
+        state.check(B, m, n, self.k)
+        _placed((W,), ("W",))
+        _ws_fits(self.ws, self.ws_bytes)
+        st = state.c_struct()
+        _check(lib.gm_grasp_apply(B, m, n, ctypes.byref(self.params), ctypes.byref(st), _ptr(W),
+                                  _ptr(self.ws), self.ws_bytes, _stream()), "gm_grasp_apply")
 
     # stage buffers inside the workspace (views; valid after the step ran)
     def _view(self, off, shape, dtype):

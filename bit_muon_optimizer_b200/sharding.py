@@ -13,12 +13,16 @@ cost, by default the step's Newton-Schulz FLOP scaling m n min(m, n). Every
 rank computes the same assignment from the same shapes, so no communication
 decides it.
 
-The per-matrix update is injected: ``make_step(B, m, n)`` returns a callable
-``step(W, G)`` that updates a contiguous [B, m, n] fp32 weight batch in place
-from a gradient batch of the same shape and keeps whatever state it needs
-(the library's GRASP step on a GPU; any stand-in in tests). The exchange is
-one all-gather per shape group through ``torch.distributed`` (NCCL on GPUs),
-each rank sending its owned matrices padded to the largest owner's count.
+The per-matrix update is injected: ``make_step(m, n, ids)`` returns a callable
+``step(W, G)`` that updates a contiguous [len(ids), m, n] fp32 weight batch in
+place from a gradient batch of the same shape and keeps whatever state it
+needs (the library's GRASP step on a GPU; any stand-in in tests). ``ids`` are
+the batch's indices in the whole parameter set (groups in order, matrices in
+order within a group): the step seeds its per-matrix random draws (the
+Rademacher start vectors) from them, so a matrix's results do not depend on
+the number of ranks or on which rank owns it. The exchange is one all-gather
+per shape group through ``torch.distributed`` (NCCL on GPUs), each rank
+sending its owned matrices padded to the largest owner's count.
 """
 
 from __future__ import annotations
@@ -56,10 +60,12 @@ class ShardedStep:
     ``shapes`` lists the set's shape groups as (m, n, count), in order; the
     call takes, per group, the [count, m, n] weights (updated in place on
     every rank) and the matching gradients (every rank holds all of them, as
-    after a data-parallel all-reduce)."""
+    after a data-parallel all-reduce). ``first_index`` is the set index of the
+    first matrix (for a part of a larger set handled on its own)."""
 
     def __init__(self, shapes: Sequence[tuple[int, int, int]], world: int, rank: int,
-                 make_step: Callable[[int, int, int], Callable], cost=ns_cost, group=None):
+                 make_step: Callable[[int, int, list], Callable], cost=ns_cost, group=None,
+                 first_index: int = 0):
         if not 0 <= rank < world:
             raise ValueError(f"rank {rank} outside world {world}")
         self.shapes = [tuple(s) for s in shapes]
@@ -68,14 +74,16 @@ class ShardedStep:
         flat = lpt_owners(costs, world)
         self.owner: list[list[int]] = []          # owner of matrix i of group g
         self.owned: list[list[list[int]]] = []    # owned[g][r]: indices rank r owns in g
+        self.base: list[int] = []                 # set index of each group's first matrix
         pos = 0
         for m, n, count in self.shapes:
             own = flat[pos:pos + count]
+            self.base.append(first_index + pos)
             pos += count
             self.owner.append(own)
             self.owned.append([[i for i in range(count) if own[i] == r] for r in range(world)])
-        self.steps = [make_step(len(o[rank]), m, n) if o[rank] else None
-                      for (m, n, _), o in zip(self.shapes, self.owned)]
+        self.steps = [make_step(m, n, [base + i for i in o[rank]]) if o[rank] else None
+                      for (m, n, _), o, base in zip(self.shapes, self.owned, self.base)]
 
     def loads(self, cost=ns_cost) -> list[float]:
         """Total cost each rank owns."""
@@ -112,13 +120,15 @@ class ShardedStep:
                     W.index_copy_(0, torch.tensor(own, device=W.device), recv[r][:len(own)])
 
 
-def grasp_make_step(k: int, device=None, **params) -> Callable[[int, int, int], Callable]:
+def grasp_make_step(k: int, device=None, **params) -> Callable[[int, int, list], Callable]:
     """``make_step`` for the library's GRASP step: each owner batch gets its own
-    step object and zero state (its quantized momentum lives on this rank only)."""
+    step object and zero state (its quantized momentum lives on this rank only),
+    with the batch's set indices as the step's matrix ids."""
     from . import gmuon as gm
 
-    def make(B: int, m: int, n: int):
-        step = gm.GraspStep(B, m, n, k, device=device, **params)
+    def make(m: int, n: int, ids: list):
+        B = len(ids)
+        step = gm.GraspStep(B, m, n, k, device=device, matrix_ids=ids, **params)
         state = gm.GraspState.zeros(B, m, n, k, device)
 
         def run(W: torch.Tensor, G: torch.Tensor) -> None:

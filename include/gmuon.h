@@ -14,6 +14,15 @@
  * Ownership: the caller allocates every buffer (typically torch tensors) and
  * keeps it alive until the stream work completes. The library never
  * allocates or frees device memory and keeps no per-call device state.
+ * Library-wide device state is limited to two file-scope arrays that every
+ * GPU loading the library holds: one int32 error word (see
+ * gm_device_errors) and the scratch of gm_newton_schulz_noalloc.
+ *
+ * Devices: one process may drive several GPUs; each call works on the
+ * current device. Kernel attributes and looked-up device addresses are set
+ * up once per device on first use (thread-safe). These caches do not survive
+ * cudaDeviceReset (or any other primary-context reset): do not reset a
+ * device between calls into the library.
  *
  * Execution: every call enqueues work on `stream` and returns without
  * synchronising. Argument errors are detected on the host before any launch
@@ -189,7 +198,8 @@ gm_status gm_newton_schulz(int B, int m, int n, const void* X, gm_dtype xdt,
  *    any launch; gm_last_error() states the bytes needed.
  *  - The first call on a device looks up the scratch array's device address
  *    (cudaGetSymbolAddress) with that device current and caches it; make that
- *    first call before any stream capture.
+ *    first call before any stream capture. The cached address does not survive
+ *    cudaDeviceReset: do not reset the device between calls.
  *  - All calls share the one scratch array and it keeps the last call's
  *    contents (nothing in it needs to start at zero: every byte a call reads,
  *    it first writes). Calls that overlap on the GPU -- different streams, or
@@ -229,6 +239,18 @@ typedef struct {
   int n_restart;
   float eps;                 /* Frobenius normalisation epsilon (1e-7) */
   uint64_t seed;             /* Rademacher start vectors */
+  /* The fields below may be left zero (their defaults): */
+  int power_steps;           /* power-iteration steps per GRASP step, 1..3 (0 = 1). Each
+                                step after the first restarts from Q = column-normalised R
+                                of the one before ([GRASP] ablation table: 1/2/3 steps) */
+  int residual_from_codes;   /* 0: residual M_t - P R^T with the unquantized P, R
+                                ([GRASP] worked step 5); 1: M_t - P^ R^T with P^, R^ the
+                                dequantized 8-bit codes of this step */
+  const int64_t* matrix_ids; /* device int64 [B] or NULL: the index b that the Rademacher
+                                counter uses for each matrix (NULL: 0 .. B-1). Giving each
+                                matrix its index in the whole parameter set makes the start
+                                vectors independent of how a set is split into calls (e.g.
+                                across ranks); ids lie in [0, 65536) */
 } gm_grasp_params;
 
 /* The quantized momentum state [GRASP, worked step, last paragraph];
@@ -252,6 +274,9 @@ typedef struct {
  *   rebuild M_{t-1}; warm start Q; M_t = mu M_{t-1} + G; P, R = PowerIter(M_t, Q);
  *   residual M_t - P R^T -> 4-bit grid codes; P, R -> 8-bit codes (state updated
  *   in place); O = NS(M_t) (standard or Gram); W <- W - eta (O + wd W).
+ * The Rademacher start column of matrix b (step 1, or a zero column of the
+ * stored R) takes its sign from splitmix64(seed ^ id<<48 ^ j<<16 ^ l), id =
+ * matrix_ids[b] or b.
  *   W f32 [B][m][n] (in place), G [B][m][n] of dtype gdt.
  * If G or M_t holds a NaN/Inf, *dev_status = GM_E_NONFINITE and W and the
  * state are left unchanged (the step counter too).
@@ -259,6 +284,25 @@ typedef struct {
 gm_status gm_grasp_step(int B, int m, int n, const gm_grasp_params* params,
                         const gm_grasp_state* state, float* W, const void* G, gm_dtype gdt,
                         void* ws, size_t ws_bytes, gm_stream_t stream);
+
+/*
+ * gm_grasp_step in its two halves, on the same arguments and workspace
+ * (gm_grasp_step = gm_grasp_state_update, then gm_grasp_apply):
+ *  - gm_grasp_state_update: worked steps 1-5 (rebuild, warm start, momentum,
+ *    power iteration, re-quantization into `state`); it resets and then writes
+ *    *dev_status and leaves M_t, P, R and the normalised NS input X in `ws`.
+ *  - gm_grasp_apply: worked step 6 on the X that the state update left in
+ *    `ws`: O = NS(X), W <- W - eta (O + wd W); nothing happens (W unchanged)
+ *    when *dev_status is non-zero. The NS chain overwrites X.
+ * A caller may run other work between the halves on the same stream, as long
+ * as it leaves `ws` and the state alone.
+ */
+gm_status gm_grasp_state_update(int B, int m, int n, const gm_grasp_params* params,
+                                const gm_grasp_state* state, const void* G, gm_dtype gdt,
+                                void* ws, size_t ws_bytes, gm_stream_t stream);
+gm_status gm_grasp_apply(int B, int m, int n, const gm_grasp_params* params,
+                         const gm_grasp_state* state, float* W,
+                         void* ws, size_t ws_bytes, gm_stream_t stream);
 
 /* Byte offsets of the stage buffers inside the gm_grasp_step workspace, for
  * inspection by tests: M f32 [B][m][n]; Q f32 [B][n][k]; P, R f32; X the NS
@@ -274,8 +318,11 @@ gm_status gm_grasp_workspace_layout(int B, int m, int n, int k, int ns_mode,
 gm_status gm_ns_flops(int ns_mode, int m, int n, int T, const int* restart_after,
                       int n_restart, double* flops, int* products);
 
-/* Synchronises `stream`, then reads and clears the library's device error
- * word (set when a kernel's bounded wait ran out). Returns GM_OK or
+/* Synchronises `stream`, then reads and clears the current device's error
+ * word, which the standalone NS entry points' kernels set when a bounded wait
+ * ran out (gm_grasp_step reports through its state's dev_status instead).
+ * The word is shared by every stream and thread on that device: a timeout is
+ * reported to whichever caller reads the word first. Returns GM_OK or
  * GM_E_TIMEOUT (or GM_E_CUDA). */
 gm_status gm_device_errors(gm_stream_t stream);
 

@@ -144,15 +144,24 @@ def orth_positive(Ptil: torch.Tensor, tol: float = QR_DEAD_TOL):
     return P, live
 
 
-def power_iteration(M: torch.Tensor, Q: torch.Tensor):
-    """P, R = PowerIter(M, Q) with one step [GRASP, worked step 4].
+def power_iteration(M: torch.Tensor, Q: torch.Tensor, steps: int = 1, seed: int = 0, b: int = 0):
+    """P, R = PowerIter(M, Q) [GRASP, worked step 4; ablation table, 1/2/3
+    power-iteration steps].
 
-    P~ = M Q; P = orth(P~); R = M^T P. Returns (P, R, P~, live).
+    One step: P~ = M Q; P = orth(P~); R = M^T P. Each further step starts
+    again from Q = column-normalised R of the step before, the same rule as
+    the warm start (so a zero column of R, a dead one, restarts from its
+    Rademacher column, drawn with ``seed`` and ``b``). Returns
+    (P, R, P~, live) of the last step.
     """
     M = M.to(DT)
-    Ptil = M @ Q.to(DT)
-    P, live = orth_positive(Ptil)
-    R = M.T @ P
+    Q = Q.to(DT)
+    for s in range(steps):
+        if s > 0:
+            Q = warm_start(R, seed, b)
+        Ptil = M @ Q
+        P, live = orth_positive(Ptil)
+        R = M.T @ P
     return P, R, Ptil, live
 
 
@@ -465,24 +474,36 @@ class StepResult:
 
 def grasp_step(st: GraspState, W: torch.Tensor, G: torch.Tensor, *, mu: float, eta: float,
                wd: float = 0.0, seed: int = 0, b: int = 0, ns: str = "standard",
-               abc=None, T: int = 5, restart_after=(2,), block: int = GRID_BLOCK) -> StepResult:
+               abc=None, T: int = 5, restart_after=(2,), block: int = GRID_BLOCK,
+               power_steps: int = 1, residual: str = "exact") -> StepResult:
     """One GRASP step for one matrix, in the order of [GRASP, worked step]:
 
     1. rebuild M_{t-1} from the stored codes;
     2. warm start Q_t = column-normalised R_{t-1};
     3. M_t = mu M_{t-1} + G;
-    4. P, R = PowerIter(M_t, Q_t);
-    5. M_res = M_t - P R^T -> 4-bit grid codes; P, R -> 8-bit codes;
+    4. P, R = PowerIter(M_t, Q_t) (``power_steps`` steps: the ablation table's
+       1/2/3-step rows; the method uses one);
+    5. M_res = M_t - P R^T -> 4-bit grid codes; P, R -> 8-bit codes.
+       ``residual="codes"`` is the variant that subtracts the dequantized
+       8-bit factors instead, M_t - P^ R^T (the worked step writes the
+       unquantized P, R, the default);
     6. O = NS(M_t); W <- W - eta (O + wd W).
+
+    ``b`` is the matrix's index in the Rademacher counter.
     """
     M_prev = rebuild_momentum(st, block)
     Q = warm_start(dequant8(st.R8, st.Rscale), seed, b)
     M = mu * M_prev + G.to(DT)
-    P, R, Ptil, live = power_iteration(M, Q)
-    residual = M - P @ R.T
-    q4, rs, cs = grid_quant4(residual.to(F32), block)
+    P, R, Ptil, live = power_iteration(M, Q, power_steps, seed, b)
     P8, Ps = quant8(P.to(F32))
     R8, Rs = quant8(R.to(F32))
+    if residual == "exact":
+        residual = M - P @ R.T
+    elif residual == "codes":
+        residual = M - dequant8(P8, Ps) @ dequant8(R8, Rs).T
+    else:
+        raise ValueError(residual)
+    q4, rs, cs = grid_quant4(residual.to(F32), block)
     if ns == "standard":
         O = ns_standard(M, abc, T)
     elif ns == "gram":

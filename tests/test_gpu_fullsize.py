@@ -8,12 +8,14 @@ iteration's P and R (relative Frobenius error <= 1e-5), the 8-bit codes
 (bit-exact on the GPU's own P, R) and the 4-bit grid codes (one step apart in
 at most 1e-4 of the elements).
 
-The fp64 oracle's Newton-Schulz is too slow at these sizes, so the update
-direction O = (W_before - W_after) / eta (weight decay 0) is checked through
-the property Proposition 1 of "优化器 (3)（Gram Newton-Schulz）" states for any
-size: NS(X) = U f(S) V^T for X = U S V^T, f the composed scalar quintic. So
-the sorted singular values of O equal the sorted f(s_i) of the normalised
-momentum, up to the bf16 arithmetic's spectral-norm error (Weyl: sorted
+The update direction O = (W_before - W_after) / eta (weight decay 0) of each
+sampled matrix is compared element by element with the oracle's fp64
+Newton-Schulz of the same momentum (standard, or Gram with its restart):
+relative Frobenius error <= 2e-2. It is also checked through the property
+Proposition 1 of "优化器 (3)（Gram Newton-Schulz）" states for any size:
+NS(X) = U f(S) V^T for X = U S V^T, f the composed scalar quintic, so the
+sorted singular values of O equal the sorted f(s_i) of the normalised
+momentum, up to the 16-bit arithmetic's spectral-norm error (Weyl: sorted
 singular values move by at most ||E||_2).
 """
 
@@ -46,12 +48,16 @@ def _singular_values(X):
     return ev.clamp_min(0).sqrt()
 
 
-# (workload, shape group, NS form): LLaMA-1.1B 5632 x 2048 (tall) and 256 x 2048;
-# Qwen2.5-7B 3584 x 18944 (wide, the largest matrices) and 512 x 3584; the Gram NS
-# form on the MoE experts (1408 x 2048, k = 32, Student-t gradients) and on
-# LLaMA-130M's 2048 x 768. The largest group of all runs from test_gpu_size_limits.py.
-FULL = [(3, 2, "standard"), (3, 1, "standard"), (4, 3, "standard"), (4, 1, "standard"),
-        (5, 0, "gram"), (2, 1, "gram")]
+# (workload, shape group, NS form): every shape group of the LLaMA-1.1B set
+# (2048^2, 256 x 2048, 5632 x 2048 tall, 2048 x 5632 wide); Qwen2.5-7B 3584^2,
+# 512 x 3584 and 3584 x 18944 (wide, the largest matrices); the MoE experts
+# (1408 x 2048, k = 32, Student-t gradients) and the 4096 x 16384 alpha = 4 matrix
+# under both NS forms; LLaMA-130M's 2048 x 768 under Gram NS. The largest group of
+# all (18944 x 3584 x 56) runs from test_gpu_size_limits.py.
+FULL = [(3, 0, "standard"), (3, 1, "standard"), (3, 2, "standard"), (3, 3, "standard"),
+        (4, 0, "standard"), (4, 1, "standard"), (4, 3, "standard"),
+        (5, 0, "standard"), (5, 0, "gram"), (5, 1, "standard"), (5, 1, "gram"),
+        (2, 1, "gram")]
 
 
 @pytest.mark.parametrize("cid,gi,ns", FULL)
@@ -61,7 +67,7 @@ def test_full_size_group_step(cuda_lib, cid, gi, ns):
     g = w.groups[gi]
     B, m, n, k = g.count, g.m, g.n, w.k
     base = w.group_base(gi)
-    sample = (0, B - 1)
+    sample = sorted({0, B - 1})
     nsmode = gm.GM_NS_GRAM if ns == "gram" else gm.GM_NS_STANDARD
     step = gm.GraspStep(B, m, n, k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=nsmode,
                         seed=w.seed, device=DEV)
@@ -94,6 +100,12 @@ def test_full_size_group_step(cuda_lib, cid, gi, ns):
         q4, _, _ = O.grid_quant4((M - P @ R.T).to(torch.float32))
         diff = (O.unpack_nibbles(st.codes4[b].cpu()).int() - q4.int()).abs()
         assert int(diff.max()) <= 1 and float((diff > 0).double().mean()) <= 1e-4
+        # update direction, element by element, vs the oracle's fp64 NS of M_t
+        Og = ((W0[b] - W[b]) / w.eta).cpu()
+        Oref = O.gram_ns(M, T=w.T) if ns == "gram" else O.ns_standard(M, T=w.T)
+        e_ns = rel(Og, Oref)
+        print(f"\n[{w.name} {m}x{n} {ns} b={b}] |O - O_fp64| / |O_fp64| = {e_ns:.2e}")
+        assert e_ns <= 2e-2, f"O of matrix {b}"
         # update direction vs the scalar quintic on the momentum's spectrum
         s_in = _singular_values(Mg)
         want = O.quintic_scalar(s_in / s_in.pow(2).sum().sqrt(), T=w.T).sort().values

@@ -196,21 +196,59 @@ def test_newton_schulz_single_terms(cuda_lib, abc, B, m, n):
         assert rel(Og[b], O.ns_standard(X[b].double(), abc=abc, T=1)) <= 1e-2
 
 
+def _conditioned_matrix(B, m, n, seed, smin=0.1):
+    """U diag(s) V^T with random orthogonal frames and s spread evenly over
+    [smin, 1]: a matrix whose Gram has no near-zero eigenvalue."""
+    g = torch.Generator().manual_seed(seed)
+    N = min(m, n)
+    out = torch.empty(B, m, n)
+    for b in range(B):
+        U, _ = torch.linalg.qr(torch.randn(m, N, generator=g, dtype=torch.float64))
+        V, _ = torch.linalg.qr(torch.randn(n, N, generator=g, dtype=torch.float64))
+        s = torch.linspace(1.0, smin, N, dtype=torch.float64)
+        out[b] = (U @ torch.diag(s) @ V.T).float() * 1e-2
+    return out
+
+
 @pytest.mark.parametrize("restart", [(2,), (1, 3), (1, 2, 3, 4), ()])
 @pytest.mark.parametrize("B,m,n", NS_SHAPES)
 def test_gram_ns_vs_oracle(cuda_lib, B, m, n, restart):
     """Stabilized Gram NS (restarts) within 2e-2 of fp64 NS on every shape. The
-    restart-free (naive) form is held to it only on well-conditioned inputs: in
-    half precision it is unstable when R has near-zero eigenvalues (Gram NS
-    page, §3.1), as the square random case (sigma_min / sigma_max ~ 1e-5) has."""
-    if restart == () and m == n:
-        pytest.skip("naive Gram NS on a near-singular square input")
+    restart-free (naive) form on a square matrix gets a well-conditioned input
+    (singular values spread over [0.1, 1]): in half precision naive Gram NS is
+    unstable when R has near-zero eigenvalues (Gram NS page, §3.1, Proposition
+    2), which a square random matrix (sigma_min / sigma_max ~ 1e-5) has."""
     gm = cuda_lib
-    X = _outlier_matrix(B, m, n, 51)
+    if restart == () and m == n:
+        X = _conditioned_matrix(B, m, n, 52)
+    else:
+        X = _outlier_matrix(B, m, n, 51)
     Og = gm.gram_ns(X.to(DEV), restart_after=restart)
     for b in range(B):
         ref = O.ns_standard(X[b].double())          # Gram NS equals NS in exact arithmetic
         assert rel(Og[b], ref) <= 2e-2
+
+
+# Batches with more output tiles per product than the 74 CTA pairs of the
+# persistent GEMM, so every pair walks several (matrix, tile) pairs: the
+# accumulator double buffer flips, the operand ring wraps across tiles and
+# the batch index advances inside one launch. 48 x 768^2: 288 lower-triangle
+# tiles per symmetric product, 432 per left product; 8 x 768 x 2048: 192 left
+# tiles; 160 x 256 x 512: 160 tiles of one matrix each.
+MULTI_TILE = [(48, 768, 768), (8, 768, 2048), (160, 256, 512), (6, 2048, 768)]
+
+
+@pytest.mark.parametrize("B,m,n", MULTI_TILE)
+@pytest.mark.parametrize("form", ["standard", "gram"])
+def test_ns_many_tiles_per_cta_pair(cuda_lib, B, m, n, form):
+    gm = cuda_lib
+    X = _outlier_matrix(B, m, n, 53)
+    f = gm.gram_ns if form == "gram" else gm.newton_schulz
+    Og = f(X.to(DEV)).cpu()
+    torch.cuda.synchronize()
+    for b in range(B):
+        ref = O.gram_ns(X[b].double()) if form == "gram" else O.ns_standard(X[b].double())
+        assert rel(Og[b], ref) <= 2e-2, f"matrix {b}"
 
 
 # ----------------------------------------------------------------- full step
@@ -486,3 +524,88 @@ def test_grasp_step_zero_gradient(cuda_lib, ns):
     for x in (st.codes4, st.rscale, st.cscale, st.P8, st.Pscale, st.R8, st.Rscale):
         assert int(torch.count_nonzero(x)) == 0
     assert int(torch.count_nonzero(step.stage_P())) == 0
+
+
+# ------------------------------------------------- step options and halves
+
+@pytest.mark.parametrize("power_steps,residual,ns", [(2, "exact", "standard"), (3, "exact", "gram"),
+                                                     (1, "codes", "standard"), (2, "codes", "gram")])
+def test_grasp_step_power_steps_and_residual_variant(cuda_lib, power_steps, residual, ns):
+    """The ablation variants of the step ([GRASP] ablation table: 1/2/3
+    power-iteration steps; the residual from the dequantized 8-bit factors),
+    teacher-forced for two steps at a ragged wide and a tall size, with the
+    matrices' Rademacher counter indices given explicitly (ids 5 and 11)."""
+    gm = cuda_lib
+    nsmode = gm.GM_NS_GRAM if ns == "gram" else gm.GM_NS_STANDARD
+    ids = [5, 11]
+    for m, n, k in ((144, 400, 8), (400, 144, 16)):
+        B, seed = 2, 321
+        step = gm.GraspStep(B, m, n, k, ns=nsmode, seed=seed, device=DEV, power_steps=power_steps,
+                            residual_from_codes=residual == "codes", matrix_ids=ids)
+        st = gm.GraspState.zeros(B, m, n, k, DEV)
+        W = WL.random_matrix((B, m, n), 91, std=0.02).to(DEV)
+        for t in (1, 2):
+            G = _outlier_matrix(B, m, n, 90 + t, dtype=torch.bfloat16).to(DEV)
+            before = [_to_oracle_state(st, b) for b in range(B)]
+            W0 = W.clone()
+            step(st, W, G)
+            torch.cuda.synchronize()
+            assert int(st.dev_status.item()) == 0
+            for b in range(B):
+                r = O.grasp_step(before[b], W0[b].cpu(), G[b].cpu(), mu=0.95, eta=0.02, seed=seed,
+                                 b=ids[b], ns=ns, power_steps=power_steps, residual=residual)
+                assert rel(step.stage_M()[b], r.M) <= 1e-5
+                assert rel(step.stage_P()[b], r.P) <= 1e-5
+                assert rel(step.stage_R()[b], r.R) <= 1e-5
+                q, s = O.quant8(step.stage_P()[b].cpu())
+                assert torch.equal(st.P8[b].cpu(), q) and torch.equal(st.Pscale[b].cpu(), s)
+                q, s = O.quant8(step.stage_R()[b].cpu())
+                assert torch.equal(st.R8[b].cpu(), q) and torch.equal(st.Rscale[b].cpu(), s)
+                diff = (O.unpack_nibbles(st.codes4[b].cpu()).int()
+                        - O.unpack_nibbles(r.state.codes4).int()).abs()
+                assert int(diff.max()) <= 1 and float((diff > 0).double().mean()) <= 1e-4
+                assert rel((W0[b].double() - W[b].double()).cpu() / 0.02, r.O) <= 2e-2
+
+
+def test_grasp_step_halves_equal_the_step(cuda_lib):
+    """gm_grasp_state_update followed by gm_grasp_apply is gm_grasp_step, bit for
+    bit (state, weights and the stage buffers), over two steps."""
+    gm = cuda_lib
+    B, m, n, k = 3, 256, 640, 16
+    W0 = WL.random_matrix((B, m, n), 95, std=0.02).to(DEV)
+    grads = [_outlier_matrix(B, m, n, 96 + t, dtype=torch.bfloat16).to(DEV) for t in (1, 2)]
+    runs = []
+    for split in (False, True):
+        step = gm.GraspStep(B, m, n, k, seed=4, device=DEV)
+        st = gm.GraspState.zeros(B, m, n, k, DEV)
+        W = W0.clone()
+        for G in grads:
+            if split:
+                step.state_update(st, G)
+                step.apply(st, W)
+            else:
+                step(st, W, G)
+        torch.cuda.synchronize()
+        runs.append((st, W, step.stage_M().clone(), step.stage_P().clone()))
+    (sa, Wa, Ma, Pa), (sb, Wb, Mb, Pb) = runs
+    assert torch.equal(Wa, Wb) and torch.equal(Ma, Mb) and torch.equal(Pa, Pb)
+    for a, b in zip(sa.tensors(), sb.tensors()):
+        assert torch.equal(a, b)
+
+
+def test_grasp_apply_skips_after_a_nonfinite_state_update(cuda_lib):
+    """A NaN in G: the state update flags GM_E_NONFINITE and leaves the state
+    alone; the apply half then leaves W alone too."""
+    gm = cuda_lib
+    B, m, n, k = 1, 256, 256, 8
+    step = gm.GraspStep(B, m, n, k, device=DEV)
+    st = gm.GraspState.zeros(B, m, n, k, DEV)
+    W = WL.random_matrix((B, m, n), 97, std=0.02).to(DEV)
+    G = WL.random_matrix((B, m, n), 98, std=1e-3).to(DEV)
+    G[0, 3, 3] = float("inf")
+    W1 = W.clone()
+    step.state_update(st, G)
+    step.apply(st, W)
+    torch.cuda.synchronize()
+    assert int(st.dev_status.item()) == gm.GM_E_NONFINITE
+    assert torch.equal(W, W1) and int(st.step.item()) == 0

@@ -1,6 +1,8 @@
 """The bench's multi-rank logic on CPU: two gloo processes take the same barrier
-and max-over-ranks steps as the GPU ranks do, and draw disjoint parameter sets
-(weak scaling: no collective on the data path)."""
+and max-over-ranks steps as the GPU ranks do, and split each shape group of the
+benchmarked parameter set into disjoint owner batches that cover it (the
+ownership sharding the bench drives at N > 1); the reference arm runs on rank 0
+only."""
 
 import os
 import socket
@@ -30,16 +32,22 @@ def _rank_main(rank, world, port, q):
     try:
         bench.barrier(w_)
         t = bench.max_over_ranks(1.5 * (r_ + 1), w_)
-        wl = WL.WORKLOADS[2]
-        bases = [(bench.matrix_base(wl, gi, r_), wl.groups[gi].count) for gi in range(len(wl.groups))]
+        from bit_muon_optimizer_b200 import sharding as S
+        wl = WL.WORKLOADS[4]
+        owned = []
+        for gi, g in enumerate(wl.groups):
+            ids = []
+            S.ShardedStep([(g.m, g.n, g.count)], w_, r_, lambda m, n, i: ids.extend(i) or (lambda W, G: None),
+                          first_index=wl.group_base(gi))
+            owned.append(ids)
         ref = bench.run_reference(None, w_, r_) if r_ != 0 else None   # rank != 0: no work
         bench.barrier(w_)
-        q.put((r_, w_, t, bases, ref))
+        q.put((r_, w_, t, owned, ref))
     finally:
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_barrier_max_and_disjoint_sets():
+def test_two_gloo_ranks_barrier_max_and_owner_split():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -54,11 +62,10 @@ def test_two_gloo_ranks_barrier_max_and_disjoint_sets():
     assert [o[0] for o in out] == [0, 1] and all(o[1] == 2 for o in out)
     assert all(o[2] == pytest.approx(3.0) for o in out)            # max over ranks of 1.5, 3.0
     assert out[1][4] is None
-    sets = []
-    for _, _, _, bases, _ in out:
-        idx = set()
-        for base, count in bases:
-            idx.update(range(base, base + count))
-        sets.append(idx)
-    assert len(sets[0]) == len(sets[1]) == 84                      # 48 + 24 + 12 matrices per rank
-    assert not (sets[0] & sets[1])
+    from bit_muon_optimizer_b200 import workloads as WL
+    wl = WL.WORKLOADS[4]
+    for gi, g in enumerate(wl.groups):
+        a, b = set(out[0][3][gi]), set(out[1][3][gi])
+        assert not (a & b)
+        assert a | b == set(range(wl.group_base(gi), wl.group_base(gi) + g.count))
+        assert abs(len(a) - len(b)) <= 1                            # equal costs: balanced

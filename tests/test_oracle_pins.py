@@ -363,6 +363,72 @@ def test_power_iteration_subspace_bound():
             assert rel <= 0.01
 
 
+def test_power_iteration_steps_contract_the_subspace_angle_geometrically():
+    """s steps of subspace iteration from Q_0 (each step restarting from the
+    column-normalised R of the one before, which spans the same space as
+    M^T P): tan(theta_s) <= (s_{k+1}/s_k)^s tan(theta_0), the textbook bound
+    ([GRASP] ablation table: 1, 2 and 3 power-iteration steps). Also: two
+    steps equal one step started from the normalised R of one step."""
+    gen = torch.Generator().manual_seed(12)
+    m, n, k = 200, 150, 6
+    U = _orthogonal(m, gen)
+    V = _orthogonal(n, gen)
+    s = torch.cat([torch.linspace(10, 6, k, dtype=DT), torch.linspace(3.0, 0.1, n - k, dtype=DT)])
+    M = U[:, :n] @ torch.diag(s) @ V.T
+    Uk, Vk = U[:, :k], V[:, :k]
+
+    def tan_theta(B, target):
+        B, _ = torch.linalg.qr(B)
+        c = torch.linalg.svdvals(target.T @ B).min()
+        return math.sqrt(max(0.0, 1 - float(c) ** 2)) / float(c)
+
+    Q0 = Vk + 0.4 * torch.randn(n, k, generator=gen, dtype=DT)
+    Q0 = Q0 / torch.linalg.vector_norm(Q0, dim=0)
+    t0 = tan_theta(Q0, Vk)
+    ratio = float(s[k] / s[k - 1])
+    prev = None
+    for steps in (1, 2, 3):
+        P, R, _, live = O.power_iteration(M, Q0, steps, seed=3, b=1)
+        assert all(live)
+        t = tan_theta(P, Uk)
+        assert t <= ratio ** steps * t0 * (1 + 1e-9)
+        if prev is not None:
+            assert t < prev                     # each step gains
+        prev = t
+    P1, R1, _, _ = O.power_iteration(M, Q0, 1)
+    P2, R2, _, _ = O.power_iteration(M, Q0, 2)
+    Pc, Rc, _, _ = O.power_iteration(M, R1 / torch.linalg.vector_norm(R1, dim=0), 1)
+    assert torch.allclose(P2, Pc, atol=1e-12) and torch.allclose(R2, Rc, atol=1e-11)
+
+
+def test_residual_from_codes_bounds_the_rebuild_by_the_grid_half_step():
+    """The residual-from-codes variant stores M_t - P^ R^T, so the next rebuild
+    deq4 + P^ R^T misses M_t only by the 4-bit grid error: every element within
+    half a code step s_ij / 14 (plus fp32 rounding of the residual). The
+    worked step's own residual M_t - P R^T leaves the 8-bit factor error
+    (P R^T - P^ R^T) in the rebuild on top, which this outlier input makes
+    larger than the half step somewhere."""
+    gen = torch.Generator().manual_seed(13)
+    m, n, k = 256, 384, 8
+    U = _orthogonal(m, gen)[:, :k]
+    V = _orthogonal(n, gen)[:, :k]
+    M = U @ torch.diag(torch.logspace(0, -1, k, dtype=DT)) @ V.T
+    M = M + 1e-3 * torch.randn(m, n, generator=gen, dtype=DT)
+    M[:, 5] *= 30.0
+    st = O.zero_state(m, n, k)
+    worst = {}
+    for mode in ("codes", "exact"):
+        r = O.grasp_step(st, torch.zeros(m, n), M.float(), mu=0.0, eta=0.0, seed=1, b=0,
+                         residual=mode)
+        M_t = r.M
+        rebuilt = O.rebuild_momentum(r.state)
+        s_ij = O.grid_scale_matrix(r.state.rscale, r.state.cscale, m, n).to(DT)
+        excess = (rebuilt - M_t).abs() - s_ij / 14.0
+        worst[mode] = float((excess / M_t.abs().max()).max())
+    assert worst["codes"] <= 1e-6
+    assert worst["exact"] > 1e-4
+
+
 def test_warm_start_normalises_columns_and_uses_rademacher_for_zero_columns():
     Rh = torch.zeros(40, 3, dtype=DT)
     Rh[:, 0] = torch.arange(40, dtype=DT) - 20.0

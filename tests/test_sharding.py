@@ -5,6 +5,10 @@ textbook bound for LPT (Graham, 1969: makespan <= (4/3 - 1/(3w)) x optimum),
 the optimum found by brute force. The exchange runs as gloo processes with a
 stateful CPU stand-in for the per-matrix step: every rank must end with the
 weights a single process computes, and every matrix must have one owner.
+With the oracle's GRASP step as the per-matrix step (seeded by each matrix's
+index in the set), weights and quantized states after two steps are the same
+for 1, 2 and 3 ranks; seeded by the index inside each owner's batch instead,
+they are not (the step-1 Rademacher start vectors move with the split).
 """
 
 import itertools
@@ -46,7 +50,7 @@ def test_lpt_within_graham_bound(world):
 class _StandIn:
     """Per-batch state: the number of steps taken; W -= 0.1 t G per matrix."""
 
-    def __init__(self, B, m, n):
+    def __init__(self, m, n, ids):
         self.t = 0
 
     def __call__(self, W, G):
@@ -67,19 +71,84 @@ def _run(world, rank, steps=2):
     return sh, W
 
 
-def _rank_main(rank, world, port, q):
+# the oracle's step on small shapes: k = 2, T = 2 NS steps
+O_SHAPES = [(16, 32, 3), (32, 16, 2), (16, 16, 2)]
+O_K, O_SEED = 2, 7
+
+
+class _OracleStep:
+    """The oracle's GRASP step for an owner batch; the Rademacher counter index b
+    is each matrix's set index (``set_ids``) or its place in the batch."""
+
+    def __init__(self, m, n, ids, set_ids=True):
+        import oracle as O
+        self.O = O
+        self.ids = list(ids) if set_ids else list(range(len(ids)))
+        self.states = [O.zero_state(m, n, O_K) for _ in ids]
+
+    def __call__(self, W, G):
+        for i, b in enumerate(self.ids):
+            r = self.O.grasp_step(self.states[i], W[i], G[i], mu=0.95, eta=0.02, seed=O_SEED, b=b,
+                                  T=2)
+            self.states[i] = r.state
+            W[i] = r.W.float()
+
+
+def _oracle_inputs(step):
+    g = torch.Generator().manual_seed(300 + step)
+    return [torch.randn((c, m, n), generator=g, dtype=torch.float64).float() * 1e-3
+            for m, n, c in O_SHAPES]
+
+
+def _run_oracle(world, rank, set_ids):
+    steps = []
+
+    def make(m, n, ids):
+        st = _OracleStep(m, n, ids, set_ids)
+        steps.append((m, n, ids, st))
+        return st
+
+    sh = S.ShardedStep(O_SHAPES, world, rank, make)
+    W = [x.clone() * 20 for x in _oracle_inputs(0)]
+    for t in (1, 2):
+        sh(W, _oracle_inputs(t))
+    codes = {(m, n, b): st.states[i].codes4 for m, n, ids, st in steps for i, b in enumerate(ids)}
+    return W, codes
+
+
+def _rank_main(rank, world, port, q, kind="standin", set_ids=True):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world))
     sys.path.insert(0, ROOT)
+    torch.set_num_threads(1)
     import datetime
 
     import torch.distributed as dist
     dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     try:
-        sh, W = _run(world, rank)
-        q.put((rank, sh.owner, W))
+        if kind == "standin":
+            sh, W = _run(world, rank)
+            q.put((rank, sh.owner, W))
+        else:
+            W, codes = _run_oracle(world, rank, set_ids)
+            q.put((rank, W, codes))
     finally:
         dist.destroy_process_group()
+
+
+def _spawn(world, kind="standin", set_ids=True):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q, kind, set_ids))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=300) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return sorted(out, key=lambda x: x[0])
 
 
 def _free_port():
@@ -91,16 +160,7 @@ def _free_port():
 @pytest.mark.parametrize("world", [2, 3])
 def test_gloo_ranks_end_with_the_single_process_weights(world):
     _, W_ref = _run(1, 0)
-    ctx = mp.get_context("spawn")
-    q = ctx.Queue()
-    port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
-    for p in procs:
-        p.start()
-    out = [q.get(timeout=120) for _ in procs]
-    for p in procs:
-        p.join(timeout=60)
-        assert p.exitcode == 0
+    out = _spawn(world)
     owners = out[0][1]
     for rank, own, W in out:
         assert own == owners                                   # same assignment everywhere
@@ -110,3 +170,25 @@ def test_gloo_ranks_end_with_the_single_process_weights(world):
     assert [len(o) for o in owners] == [c for _, _, c in SHAPES]
     assert all(0 <= r < world for o in owners for r in o)
     assert len(set(owners[2])) == 1
+
+
+def test_oracle_step_results_do_not_depend_on_the_world_size():
+    """Two oracle GRASP steps of a small set on 1, 2 and 3 gloo ranks: every
+    rank ends with the same weights, and each matrix's quantized state is the
+    same whichever rank owns it, because the step is seeded by the matrix's
+    index in the set. Seeded by its place in the owner's batch, the two-rank
+    run departs from the one-rank run."""
+    ref = _spawn(1, "oracle")[0]
+    W1, codes1 = ref[1], ref[2]
+    for world in (2, 3):
+        out = _spawn(world, "oracle")
+        codes = {}
+        for _, W, c in out:
+            for a, b in zip(W, W1):
+                assert torch.equal(a, b)
+            codes.update(c)
+        assert codes.keys() == codes1.keys()
+        for key in codes1:
+            assert torch.equal(codes[key], codes1[key])
+    local = _spawn(2, "oracle", set_ids=False)
+    assert any(not torch.equal(a, b) for a, b in zip(local[0][1], W1))

@@ -38,6 +38,27 @@ def test_noalloc_matches_allocating_entry_point_twice(cuda_lib):
         assert _rel(got, ref) <= 2e-2
 
 
+def test_noalloc_call_allocates_no_device_memory(cuda_lib):
+    """The property the entry point exists for. One warm-up call loads the
+    library's kernels (and with them the built-in scratch array) on the device;
+    after it, with the input and the output preallocated, a call on a new shape
+    and new dtypes leaves the device's free memory exactly where it was. Both
+    shapes are multiples of 64, so the two calls launch the same kernels."""
+    gm = cuda_lib
+    X0 = WL.random_matrix((2, 256, 512), 910, std=1e-2).cuda()
+    gm.newton_schulz_noalloc(X0, out=torch.empty_like(X0))
+    X1 = WL.random_matrix((3, 384, 640), 911, std=1e-2).to(torch.bfloat16).cuda()
+    out = torch.empty((3, 384, 640), dtype=torch.float16, device="cuda")
+    ref = gm.newton_schulz(X1)
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    gm.newton_schulz_noalloc(X1, out=out)
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert free_after == free_before
+    assert _rel(out, ref) <= 2e-2
+
+
 def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_lib):
     gm = cuda_lib
     B, m, n = 64, 1024, 1024          # needs far more than the built-in 64 MiB
