@@ -373,6 +373,35 @@ def measure(gm, w, groups, ns_mode, args, world, local, do_e2e):
     ns_flops = sum(gm.ns_flops(ns_mode, g["m"], g["n"], w.T)[0] * g["B"] for g in groups)
     ns_launches = sum(gm.ns_flops(ns_mode, g["m"], g["n"], w.T)[1] for g in groups)
 
+    # ---- the standalone 4-bit codecs of the same entry points a user calls
+    # (4bit-Muon-base group codec, MuonQ's mu-law codec), on the first group's
+    # fp32 M_t: HBM GB/s of their algorithmic bytes (4 + 0.5 + 4/128 B per element)
+    codecs = None
+    if args.codecs:
+        g = groups[0]
+        M = g["step"].stage_M()
+        codes = torch.empty((g["B"], g["m"], g["n"] // 2), dtype=torch.uint8, device=dev)
+        gsc = torch.empty((g["B"], g["m"] * g["n"] // 128), dtype=torch.float32, device=dev)
+        Xo = torch.empty_like(M)
+        calls = {"group_quant4": lambda: gm.group_quant4(M, out=(codes, gsc)),
+                 "group_dequant4": lambda: gm.group_dequant4(codes, gsc, out=Xo),
+                 "mulaw_quant4": lambda: gm.mulaw_quant4(M, out=(codes, gsc)),
+                 "mulaw_dequant4": lambda: gm.mulaw_dequant4(codes, gsc, out=Xo)}
+        nbytes = M.numel() * (4 + 0.5 + 4 / 128)
+        codecs = {"elements": M.numel(), "bytes_per_call": nbytes}
+        with torch.cuda.stream(main):
+            for name, call in calls.items():
+                call()
+                c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                c0.record(main)
+                for _ in range(5):
+                    call()
+                c1.record(main)
+                torch.cuda.synchronize()
+                ms = c0.elapsed_time(c1) / 5
+                codecs[name] = {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9}
+        del codes, gsc, Xo
+
     # ---- comparator: the same standard NS chain written with torch.matmul
     # (cuBLAS, bf16, no symmetry) on the same normalised inputs, graph-replayed
     abc = [(3.4445, -4.7750, 2.0315)] * w.T
@@ -436,7 +465,7 @@ def measure(gm, w, groups, ns_mode, args, world, local, do_e2e):
         del host
     return dict(ms_step=ms_step, clocks=clk.summary(), ns_ms=ns_ms, ns_flops=ns_flops,
                 ns_launches=ns_launches, cod_ms=cod_ms, e2e=e2e, cub_ms=cub_ms,
-                cub_flops_dense=cub_flops_dense)
+                cub_flops_dense=cub_flops_dense, codecs=codecs)
 
 
 def codec_bytes(w: WL.Workload, groups) -> float:
@@ -458,8 +487,9 @@ def run_single(gm, w, ns_mode, args, local):
     per_group = est_bytes(w, pool) > 0.7 * total_mem
     batches = [[gi] for gi in range(len(w.groups))] if per_group else [list(range(len(w.groups)))]
     res = []
-    for gis in batches:
+    for i, gis in enumerate(batches):
         groups = [build_group(gm, w, gi, ns_mode, pool, dev) for gi in gis]
+        args.codecs = i == 0
         r = measure(gm, w, groups, ns_mode, args, 1, local, not args.no_e2e)
         r["codec_bytes"] = codec_bytes(w, groups)
         res.append(r)
@@ -484,6 +514,7 @@ def run_single(gm, w, ns_mode, args, local):
                     + ("; shape groups measured one at a time (device memory), set time = sum"
                        if per_group else ""))
     out["pool"] = pool
+    out["codecs"] = res[0]["codecs"]
     out["launches"] = our_launches(gm, w, ns_mode) * args.steps
     return out
 
@@ -610,6 +641,10 @@ def run_ours(args, world, rank, local):
                              "codes and scales + the 16-bit NS input"},
         "step_roofline": {"ms": t_roof, "frac": t_roof / r["ms_step"], "flops": step_flops,
                           "bytes": step_bytes},
+        "standalone_codecs": dict(r["codecs"] or {}, peak_gbs=hbm,
+                                  what="gm_group_quant4 / gm_group_dequant4 (4bit-Muon-base) and "
+                                       "gm_mulaw_quant4 / gm_mulaw_dequant4 (MuonQ mu-law, mu = 255) "
+                                       "on the first shape group's fp32 M_t; not part of the step"),
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
         "e2e": r["e2e"],

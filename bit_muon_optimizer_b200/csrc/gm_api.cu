@@ -208,6 +208,16 @@ gm_status gm_device_errors(gm_stream_t stream) {
   return GM_OK;
 }
 
+gm_status gm_test_wait_timeout(const uint16_t* X, uint16_t* D, int64_t limit_ns,
+                               gm_stream_t stream) {
+  GM_CHECK_ARG(X && D, "NULL buffer");
+  GM_CHECK_ARG(al16(X) && al16(D), "device arrays must be 16-byte aligned");
+  GM_CHECK_ARG(limit_ns >= 1000000 && limit_ns <= 1000000000, "limit_ns out of [1 ms, 1 s]");
+  GM_DEVICE();
+  GM_CUDA(run_wait_timeout_probe(X, D, (uint64_t)limit_ns, reinterpret_cast<cudaStream_t>(stream)));
+  return GM_OK;
+}
+
 gm_status gm_dequant_rebuild(int B, int m, int n, int k, const uint8_t* codes4,
                              const float* rscale, const float* cscale, const int8_t* P8,
                              const float* Pscale, const int8_t* R8, const float* Rscale,
@@ -315,9 +325,33 @@ gm_status gm_group_dequant4(int B, int m, int n, const uint8_t* codes4, const fl
   return GM_OK;
 }
 
+gm_status gm_mulaw_quant4(int B, int m, int n, float mu, const float* X, uint8_t* codes4,
+                          float* gscale, gm_stream_t stream) {
+  GM_CHECK_ARG(shape_ok(B, m, n), "bad shape B=%d m=%d n=%d", B, m, n);
+  GM_CHECK_ARG(mu > 0.f && mu <= 1e6f, "mu=%g out of (0, 1e6]", (double)mu);
+  GM_CHECK_ARG(X && codes4 && gscale, "NULL pointer");
+  GM_CHECK_ARG(al16(X) && al16(codes4) && al16(gscale), "device arrays must be 16-byte aligned");
+  GM_DEVICE();
+  GM_CUDA(launch_mulaw_quant4(B, m, n, mu, X, codes4, gscale, reinterpret_cast<cudaStream_t>(stream)));
+  return GM_OK;
+}
+
+gm_status gm_mulaw_dequant4(int B, int m, int n, float mu, const uint8_t* codes4,
+                            const float* gscale, float* X_out, gm_stream_t stream) {
+  GM_CHECK_ARG(shape_ok(B, m, n), "bad shape B=%d m=%d n=%d", B, m, n);
+  GM_CHECK_ARG(mu > 0.f && mu <= 1e6f, "mu=%g out of (0, 1e6]", (double)mu);
+  GM_CHECK_ARG(codes4 && gscale && X_out, "NULL pointer");
+  GM_CHECK_ARG(al16(codes4) && al16(gscale) && al16(X_out), "device arrays must be 16-byte aligned");
+  GM_DEVICE();
+  GM_CUDA(launch_mulaw_dequant4(B, m, n, mu, codes4, gscale, X_out,
+                                reinterpret_cast<cudaStream_t>(stream)));
+  return GM_OK;
+}
+
 static gm_status ns_common(int B, int m, int n, const void* X, gm_dtype xdt, const float* abc,
                            int T, const int* restart_after, int n_restart, float eps, void* O,
-                           gm_dtype odt, void* ws, size_t ws_bytes, gm_stream_t stream, bool gram) {
+                           gm_dtype odt, void* ws, size_t ws_bytes, gm_stream_t stream, bool gram,
+                           uint16_t* Rtrace = nullptr, uint16_t* Qtrace = nullptr) {
   GM_CHECK_ARG(shape_ok(B, m, n), "bad shape B=%d m=%d n=%d", B, m, n);
   GM_CHECK_ARG(X && O, "NULL X or O");
   GM_CHECK_ARG(al16(X) && al16(O), "device arrays must be 16-byte aligned");
@@ -340,7 +374,7 @@ static gm_status ns_common(int B, int m, int n, const void* X, gm_dtype xdt, con
   NsOutput out{0, O, (int)odt, nullptr, 0.f, 0.f};
   if (gram)
     GM_CUDA(run_ns_gram(B, m, n, Y, tab, T, restart_after, n_restart, out, w + L.ns, nullptr,
-                        nullptr, s));
+                        nullptr, s, Rtrace, Qtrace));
   else
     GM_CUDA(run_ns_standard(B, m, n, Y, tab, T, out, w + L.ns, nullptr, nullptr, s));
   return GM_OK;
@@ -357,6 +391,16 @@ gm_status gm_gram_ns(int B, int m, int n, const void* X, gm_dtype xdt, const flo
                      void* ws, size_t ws_bytes, gm_stream_t stream) {
   return ns_common(B, m, n, X, xdt, abc, T, restart_after, n_restart, eps, O, odt, ws, ws_bytes,
                    stream, true);
+}
+
+gm_status gm_gram_ns_trace(int B, int m, int n, const void* X, gm_dtype xdt, const float* abc,
+                           int T, const int* restart_after, int n_restart, float eps, void* O,
+                           gm_dtype odt, uint16_t* Rtrace, uint16_t* Qtrace, void* ws,
+                           size_t ws_bytes, gm_stream_t stream) {
+  GM_CHECK_ARG(Rtrace && Qtrace, "NULL trace buffer");
+  GM_CHECK_ARG(al16(Rtrace) && al16(Qtrace), "trace buffers must be 16-byte aligned");
+  return ns_common(B, m, n, X, xdt, abc, T, restart_after, n_restart, eps, O, odt, ws, ws_bytes,
+                   stream, true, Rtrace, Qtrace);
 }
 
 // Argument checks shared by the step and its two halves (W, G: NULL where the

@@ -54,6 +54,11 @@ constexpr uint32_t kABytes = KPS * kKBlockBytes;         // 32 KB
 constexpr uint32_t kBBytes = KPS * kKBlockBytes;         // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;      // 64 KB per CTA
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+#ifndef GM_LOAD_LANES
+#define GM_LOAD_LANES 1
+#endif
+constexpr int kLoadLanes = GM_LOAD_LANES;   // operand-copy issuing threads per operand
+static_assert(kLoadLanes >= 1 && kLoadLanes <= STAGES, "one stage per loader at least");
 
 constexpr int kEpiWarp0 = 4;
 constexpr int kEpiWarps = 16;                            // four per TMEM lane quarter
@@ -93,6 +98,8 @@ struct GemmParams {
   float* W; long long w_bs; int ldw; float eta, wd;
   const int32_t* skip;
   int32_t* err;
+  uint64_t wait_ns;            // limit of every bounded wait
+  int stall;                   // test hook: the operand producers issue no copies
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -125,17 +132,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false once ~2 s have passed (error word and abort flag set),
-// or as soon as the abort flag is seen.
+// Bounded wait: false once limit_ns have passed (error word and abort flag
+// set), or as soon as the abort flag is seen.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* err,
-                                          volatile int* abort_flag) {
+                                          volatile int* abort_flag, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (abort_flag && *abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         if (err) atomicExch(err, (int32_t)GM_E_TIMEOUT);
         if (abort_flag) *abort_flag = 1;
         return false;
@@ -648,17 +655,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // Role dispatch by warp; within a role warp only the lanes named below work,
   // the others go straight to the final barrier.
   if (warp == 0 || warp == 2) {
-    if (lane == 0) {
-      // ---------------- TMA producers: warp 0 loads A, warp 2 loads B (both CTAs)
+    if (lane < kLoadLanes) {
+      // ---------------- TMA producers: warp 0 loads A, warp 2 loads B (both CTAs);
+      // lane j of each issues the stages g with g % kLoadLanes == j
       const bool isA = warp == 0;
       uint32_t g = 0;
-      bool ok = true;
+      bool ok = !p.stall;
       for (int T = pid; T < total && ok; T += npairs) {
         const TileCoord tc = decode_tile(p, T, tiles_per, (int)cr);
         for (int st = 0; st < nst; ++st, ++g) {
+          if ((int)(g % kLoadLanes) != lane) continue;
           const int s = (int)(g % STAGES);
           const uint32_t ph = (g / STAGES) & 1u;
-          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err, abort_flag, p.wait_ns)) { ok = false; break; }
           const uint32_t bar = map_to_rank(smem_u32(&full[s]), 0);   // the leader's barrier
           const uint32_t dst = smem_u32(base + s * kStageBytes) + (isA ? 0u : kABytes);
           if (isA) {
@@ -683,13 +692,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int T = pid; T < total && ok; T += npairs, ++it) {
         const int ab = it & 1;
         const uint32_t use = (uint32_t)(it >> 1);
-        if (!mbar_wait(smem_u32(&acc_empty[ab]), (use & 1u) ^ 1u, p.err, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&acc_empty[ab]), (use & 1u) ^ 1u, p.err, abort_flag, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(ab * BN);
         for (int st = 0; st < nst; ++st, ++g) {
           const int s = (int)(g % STAGES);
           const uint32_t ph = (g / STAGES) & 1u;
-          if (!mbar_wait(smem_u32(&full[s]), ph, p.err, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&full[s]), ph, p.err, abort_flag, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_base = smem_u32(base + s * kStageBytes);
           const uint32_t b_base = a_base + kABytes;
@@ -714,7 +723,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!ok) *abort_flag = 1;
       // every MMA issued above has completed once this barrier fires
       umma_commit_pair(smem_u32(drain));
-      mbar_wait(smem_u32(drain), 0, p.err, nullptr);
+      mbar_wait(smem_u32(drain), 0, p.err, nullptr, p.wait_ns);
     }
   } else if (warp == 3) {
     if (lane == 0 && store_mode) {
@@ -727,7 +736,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int slab = 0; slab < kSlabs; ++slab, ++g) {
           const int b = (int)(g & 1u);
           const uint32_t n = g >> 1;
-          if (!mbar_wait(smem_u32(&slab_full[b]), n & 1u, p.err, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&slab_full[b]), n & 1u, p.err, abort_flag, p.wait_ns)) { ok = false; break; }
           store_slab(p, maps, outbuf + b * kOutBufBytes, tc, slab, d2diag + b * 64);
           bulk_commit();
           bulk_wait_read_all();
@@ -753,7 +762,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const TileCoord tc = decode_tile(p, T, tiles_per, (int)cr);
         uint4 cpre[NCH];
         c_prefetch(p, tc, 0, q, sub, lane, cpre);   // overlaps the MMAs of this tile
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[ab]), use & 1u, p.err, abort_flag));
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[ab]), use & 1u, p.err, abort_flag, p.wait_ns));
         if (!ok) break;
         tc_fence_after();
         const uint32_t tacc = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * BN);
@@ -766,7 +775,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int u = 0; u < NCH; ++u) cnow[u] = cpre[u];
           if (n >= 1) {
             ok = __all_sync(0xffffffffu,
-                            mbar_wait(smem_u32(&buf_free[b]), (n - 1) & 1u, p.err, abort_flag));
+                            mbar_wait(smem_u32(&buf_free[b]), (n - 1) & 1u, p.err, abort_flag, p.wait_ns));
             if (!ok) break;
           }
           // a box strictly above the diagonal of a symmetric product is never stored
@@ -792,7 +801,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const TileCoord tc = decode_tile(p, T, tiles_per, (int)cr);
         uint4 cpre[NCH];
         c_prefetch(p, tc, 0, q, sub, lane, cpre);
-        const bool ok = mbar_wait(smem_u32(&acc_full[ab]), use & 1u, p.err, abort_flag);
+        const bool ok = mbar_wait(smem_u32(&acc_full[ab]), use & 1u, p.err, abort_flag, p.wait_ns);
         tc_fence_after();
         // the epilogue warps share named barriers here: leave together or not at all
         if (epi_any(!ok || *abort_flag)) break;
@@ -810,7 +819,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0 && leader) {
     // after an abort, let the copies still in flight (from both CTAs) land
     for (int g = *consumed; g < *issued; ++g)
-      mbar_wait(smem_u32(&full[g % STAGES]), (uint32_t)(g / STAGES) & 1u, p.err, nullptr);
+      mbar_wait(smem_u32(&full[g % STAGES]), (uint32_t)(g / STAGES) & 1u, p.err, nullptr, p.wait_ns);
   }
   cluster_sync_all();   // neither CTA leaves while the other may still signal it
   if (warp == 1) {
@@ -936,6 +945,7 @@ GemmParams base_params(int M, int N, int K, int batch, bool f16, const int32_t* 
   p.alpha = 1.f;
   p.skip = skip;
   p.err = err;
+  p.wait_ns = kWaitLimitNs;
   return p;
 }
 
@@ -1113,7 +1123,8 @@ cudaError_t run_ns_standard(int B, int m, int n, uint16_t* X16, const float* abc
 
 cudaError_t run_ns_gram(int B, int m, int n, uint16_t* X16, const float* abc, int T,
                         const int* restart_after, int n_restart, const NsOutput& out, void* ws,
-                        const int32_t* skip, int32_t* err, cudaStream_t s) {
+                        const int32_t* skip, int32_t* err, cudaStream_t s, uint16_t* Rtrace,
+                        uint16_t* Qtrace) {
   const NsDims d = ns_dims(m, n);
   Ns c{B, d.Np, d.Mpp, d.N, d.Mp, true, m > n, skip, err ? err : device_error_word(), s};
   uint8_t* cur = static_cast<uint8_t*>(ws);
@@ -1131,6 +1142,11 @@ cudaError_t run_ns_gram(int B, int m, int n, uint16_t* X16, const float* abc, in
     if (restart_after[i] >= 1 && restart_after[i] < T) restart_at[restart_after[i]] = true;
   GM_TRY(xxt(c, X, R));                                    // R = X X^T
   bool q_is_identity = true;
+  // optional per-step copies of R_t and Q_t (padded N x N blocks of the batch)
+  auto dump = [&](uint16_t* trace, const uint16_t* src, int t) -> cudaError_t {
+    if (!trace) return cudaSuccess;
+    return cudaMemcpyAsync(trace + (size_t)(t - 1) * B * c.N * c.N, src, nn, cudaMemcpyDeviceToDevice, s);
+  };
   for (int t = 1; t <= T; ++t) {
     const float a = abc[3 * (t - 1)], b = abc[3 * (t - 1) + 1], cc = abc[3 * (t - 1) + 2];
     const bool block_end = restart_at[t] || t == T;
@@ -1143,20 +1159,42 @@ cudaError_t run_ns_gram(int B, int m, int n, uint16_t* X16, const float* abc, in
       GM_TRY(symmul(c, Q, Z, 1.f, a, Q, 0.f, Qn));          // Q = Q Z + a Q
       uint16_t* tq = Q; Q = Qn; Qn = tq;
     }
+    GM_TRY(dump(Qtrace, Q, t));
     if (!block_end) {
       GM_TRY(symmul(c, R, Z, 1.f, a, R, 0.f, RZ));          // RZ = R Z + a R
       GM_TRY(symmul(c, Z, RZ, 1.f, a, RZ, 0.f, Rn));        // R = Z RZ + a RZ
       uint16_t* tr = R; R = Rn; Rn = tr;
+      GM_TRY(dump(Rtrace, R, t));
     } else if (t < T) {
       GM_TRY(leftmul(c, Q, X, 1.f, 0.f, Xn, nullptr));      // restart: X = Q X
       uint16_t* tx = X; X = Xn; Xn = tx;
       GM_TRY(xxt(c, X, R));
+      GM_TRY(dump(Rtrace, R, t));
       q_is_identity = true;
     } else {
       GM_TRY(leftmul(c, Q, X, 1.f, 0.f, nullptr, &out));    // O = Q X
     }
   }
   return cudaSuccess;
+}
+
+cudaError_t run_wait_timeout_probe(const uint16_t* X, uint16_t* D, uint64_t limit_ns, cudaStream_t s) {
+  // one 256 x 256 bf16 X X^T tile whose operand producers issue nothing: the MMA
+  // issuer's wait for the first stage runs out after limit_ns, records
+  // GM_E_TIMEOUT in the error word and every role unwinds
+  Ns c{1, 256, 256, 256, 256, false, false, nullptr, device_error_word(), s};
+  Maps m;
+  memset(&m, 0, sizeof(m));
+  if (!c.err) return cudaErrorInvalidValue;
+  if (!map_chunks(&m.A, X, false, 256, 256, 256, 1, 256 * 256, 128)) return cudaErrorInvalidValue;
+  m.B = m.A;
+  GemmParams p = base_params(256, 256, 256, 1, false, nullptr, c.err);
+  if (!sym_out(m, p, c, D, nullptr)) return cudaErrorInvalidValue;
+  p.tiles_m = p.tiles_n = 1;
+  p.sym = 1;
+  p.wait_ns = limit_ns;
+  p.stall = 1;
+  return launch_gemm<false>(m, p, s);
 }
 
 void ns_schedule_flops(int ns_mode, int m, int n, int T, const int* restart_after, int n_restart,

@@ -93,6 +93,12 @@ cudaError_t launch_group_quant4(int B, int m, int n, const float* X, uint8_t* co
 cudaError_t launch_group_dequant4(int B, int m, int n, const uint8_t* codes4, const float* gscale,
                                   float* X, cudaStream_t s);
 
+// MuonQ's mu-law companding codec (gm_base4.cu): the same groups and layout.
+cudaError_t launch_mulaw_quant4(int B, int m, int n, float mu, const float* X, uint8_t* codes4,
+                                float* gscale, cudaStream_t s);
+cudaError_t launch_mulaw_dequant4(int B, int m, int n, float mu, const uint8_t* codes4,
+                                  const float* gscale, float* X, cudaStream_t s);
+
 // Standalone NS input: scale = 1/(|X|_F + eps) per matrix, then the wide
 // 16-bit copy Y = round(scale * X) (transposed when m > n).
 cudaError_t launch_ns_prep(int B, int m, int n, const void* X, int xdt, float eps,
@@ -117,9 +123,17 @@ size_t ns_gram_ws_bytes(int B, int m, int n);
 cudaError_t run_ns_standard(int B, int m, int n, uint16_t* X16, const float* abc, int T,
                             const NsOutput& out, void* ws, const int32_t* skip, int32_t* err,
                             cudaStream_t s);
+// Rtrace, Qtrace (nullable): fp16 [T][B][Np][Np] (Np = N rounded up to 64) per-step
+// copies of R_t (when the chain computes it: not on the last step of a block,
+// whose R update is skipped; after a restart, the restarted Gram X X^T) and Q_t.
 cudaError_t run_ns_gram(int B, int m, int n, uint16_t* X16, const float* abc, int T,
                         const int* restart_after, int n_restart, const NsOutput& out, void* ws,
-                        const int32_t* skip, int32_t* err, cudaStream_t s);
+                        const int32_t* skip, int32_t* err, cudaStream_t s,
+                        uint16_t* Rtrace = nullptr, uint16_t* Qtrace = nullptr);
+
+// Test hook of the bounded waits: a one-tile product that never gets its
+// operands; X, D: bf16 [256][256] (never read or written).
+cudaError_t run_wait_timeout_probe(const uint16_t* X, uint16_t* D, uint64_t limit_ns, cudaStream_t s);
 
 void ns_schedule_flops(int ns_mode, int m, int n, int T, const int* restart_after,
                        int n_restart, double* flops, int* products);

@@ -71,6 +71,8 @@ _sig("gm_grid_quant4", c_int, [c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, v
 _sig("gm_quant8", c_int, [c_int, c_int, c_int, vp, vp, vp, vp])
 _sig("gm_group_quant4", c_int, [c_int, c_int, c_int, vp, vp, vp, vp])
 _sig("gm_group_dequant4", c_int, [c_int, c_int, c_int, vp, vp, vp, vp])
+_sig("gm_mulaw_quant4", c_int, [c_int, c_int, c_int, c_float, vp, vp, vp, vp])
+_sig("gm_mulaw_dequant4", c_int, [c_int, c_int, c_int, c_float, vp, vp, vp, vp])
 _sig("gm_newton_schulz", c_int, [c_int, c_int, c_int, vp, c_int, vp, c_int, c_float, vp, c_int,
                                  vp, c_size_t, vp])
 _sig("gm_newton_schulz_noalloc", c_int, [c_int, c_int, c_int, vp, c_int, vp, c_int, c_float, vp,
@@ -88,6 +90,7 @@ _sig("gm_grasp_workspace_layout", c_int, [c_int, c_int, c_int, c_int, c_int,
 _sig("gm_ns_flops", c_int, [c_int, c_int, c_int, c_int, vp, c_int,
                             ctypes.POINTER(ctypes.c_double), ctypes.POINTER(c_int)])
 _sig("gm_device_errors", c_int, [vp])
+_sig("gm_test_wait_timeout", c_int, [vp, vp, ctypes.c_int64, vp])
 
 
 class GmuonError(RuntimeError):
@@ -296,6 +299,40 @@ def group_dequant4(codes, gscale, out=None):
     return out
 
 
+MULAW_MU = 255.0
+
+
+def mulaw_quant4(X, mu=MULAW_MU, out=None):
+    """MuonQ's mu-law 4-bit codes of fp32 [B, m, n] (or [m, n]), in the group
+    layout of ``group_quant4``: (codes [B, m, n/2] uint8, scales [B, m n / 128])."""
+    B, m, n = _bmn(X)
+    _expect(X, (B, m, n), (torch.float32,), "X")
+    if out is not None:
+        codes, gs = out
+    else:
+        codes = torch.empty((B, m, n // 2), dtype=torch.uint8, device=X.device)
+        gs = torch.empty((B, m * n // GROUP), dtype=torch.float32, device=X.device)
+    _expect(codes, (B, m, n // 2), (torch.uint8,), "codes")
+    _expect(gs, (B, m * n // GROUP), (torch.float32,), "gscale")
+    _check(lib.gm_mulaw_quant4(B, m, n, float(mu), _ptr(X), _ptr(codes), _ptr(gs), _stream()),
+           "gm_mulaw_quant4")
+    return codes, gs
+
+
+def mulaw_dequant4(codes, gscale, mu=MULAW_MU, out=None):
+    """fp32 [B, m, n] from mu-law codes and group scales."""
+    B, m, n2 = _bmn(codes)
+    n = 2 * n2
+    _expect(codes, (B, m, n2), (torch.uint8,), "codes")
+    _expect(gscale, (B, m * n // GROUP), (torch.float32,), "gscale")
+    if out is None:
+        out = torch.empty((B, m, n), dtype=torch.float32, device=codes.device)
+    _expect(out, (B, m, n), (torch.float32,), "out")
+    _check(lib.gm_mulaw_dequant4(B, m, n, float(mu), _ptr(codes), _ptr(gscale), _ptr(out),
+                                 _stream()), "gm_mulaw_dequant4")
+    return out
+
+
 def newton_schulz(X, abc=None, T=5, eps=1e-7, out_dtype=torch.float32, out=None, ws=None):
     B, m, n = _bmn(X)
     _expect(X, (B, m, n), tuple(_DT), "X")
@@ -345,6 +382,31 @@ def gram_ns(X, abc=None, T=5, restart_after=(2,), eps=1e-7, out_dtype=torch.floa
     return O
 
 
+_sig("gm_gram_ns_trace", c_int, [c_int, c_int, c_int, vp, c_int, vp, c_int, vp, c_int, c_float,
+                                 vp, c_int, vp, vp, vp, c_size_t, vp])
+
+
+def gram_ns_trace(X, abc=None, T=5, restart_after=(2,), eps=1e-7, out_dtype=torch.float32):
+    """gm_gram_ns_trace: returns (O, R_trace, Q_trace), the traces fp16
+    [T, B, N, N] (N = min(m, n)): Q_t after every step, R_t where the chain
+    computes it (zeros at t = T; the restarted Gram after a restart step)."""
+    B, m, n = _bmn(X)
+    _expect(X, (B, m, n), tuple(_DT), "X")
+    N = min(m, n)
+    Np = -(-N // 64) * 64
+    O = torch.empty((B, m, n), dtype=out_dtype, device=X.device)
+    Rt = torch.zeros((T, B, Np, Np), dtype=torch.float16, device=X.device)
+    Qt = torch.zeros_like(Rt)
+    nb = workspace_bytes(GM_OP_GRAM_NS, B, m, n)
+    ws = workspace(nb, X.device)
+    rl = list(restart_after)
+    rarr = (c_int * max(1, len(rl)))(*rl) if rl else None
+    _check(lib.gm_gram_ns_trace(B, m, n, _ptr(X), _DT[X.dtype], abc_table(abc, T), T, rarr, len(rl),
+                                eps, _ptr(O), _DT[out_dtype], _ptr(Rt), _ptr(Qt), _ptr(ws), nb,
+                                _stream()), "gm_gram_ns_trace")
+    return O, Rt[..., :N, :N], Qt[..., :N, :N]
+
+
 def ns_flops(ns, m, n, T=5, restart_after=(2,)):
     rl = list(restart_after) if ns == GM_NS_GRAM else []
     rarr = (c_int * max(1, len(rl)))(*rl) if rl else None
@@ -357,6 +419,16 @@ def ns_flops(ns, m, n, T=5, restart_after=(2,)):
 
 def device_errors():
     _check(lib.gm_device_errors(_stream()), "gm_device_errors")
+
+
+def wait_timeout_probe(limit_ns=20_000_000):
+    """gm_test_wait_timeout: one product launch whose bounded wait runs out
+    after limit_ns (a test hook of the failure path)."""
+    X = torch.zeros((256, 256), dtype=torch.bfloat16, device="cuda")
+    D = torch.empty_like(X)
+    _check(lib.gm_test_wait_timeout(_ptr(X), _ptr(D), int(limit_ns), _stream()),
+           "gm_test_wait_timeout")
+    return X, D
 
 
 @dataclass

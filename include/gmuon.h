@@ -166,6 +166,24 @@ gm_status gm_group_dequant4(int B, int m, int n, const uint8_t* codes4, const fl
                             float* X_out, gm_stream_t stream);
 
 /*
+ * MuonQ's mu-law companding 4-bit codec ("MuonQ: Enhancing Low-Bit Muon
+ * Quantization via Directional Fidelity Optimization", abstract: mu-law
+ * companding gives finer steps where the momentum values are dense). The
+ * abstract states neither mu nor the pre-quantization normalisation; this
+ * library's reading: the groups, absmax scales and code layout of the
+ * 4bit-Muon-base codec above, and
+ *   F(y) = sign(y) ln(1 + mu |y|) / ln(1 + mu),  q = clamp(rint(7 F(x / s_g)), -7, 7)
+ * (s_g = 0 or NaN -> q = 0); decided exactly: |q| >= j iff |x| / s_g >=
+ * F^-1((j - 1/2) / 7) (ties of the rounding, which have measure zero, go up).
+ * Decode: X_out = s_g F^-1(|q| / 7) sign(q), the level F^-1(|q| / 7) in fp32.
+ * 0 < mu <= 1e6 (255 is the telephony value).
+ */
+gm_status gm_mulaw_quant4(int B, int m, int n, float mu, const float* X, uint8_t* codes4,
+                          float* gscale, gm_stream_t stream);
+gm_status gm_mulaw_dequant4(int B, int m, int n, float mu, const uint8_t* codes4,
+                            const float* gscale, float* X_out, gm_stream_t stream);
+
+/*
  * Standard quintic Newton-Schulz [GramNS §1.2, eq. (2); Algorithm 1 first
  * line for the normalisation; LiMuon key design 3 for the coefficients]:
  *   wide form Y = X (m <= n) or X^T (m > n); Y <- Y / (|Y|_F + eps);
@@ -225,6 +243,23 @@ gm_status gm_gram_ns(int B, int m, int n, const void* X, gm_dtype xdt,
                      const float* abc, int T, const int* restart_after, int n_restart,
                      float eps, void* O, gm_dtype odt,
                      void* ws, size_t ws_bytes, gm_stream_t stream);
+
+/*
+ * gm_gram_ns, also copying the chain's fp16 Gram and transform matrices after
+ * every step, for checking the restart bounds [GramNS §3.2: with a restart
+ * after step 2, the smallest eigenvalue of R_t stays above -0.4 and the
+ * condition number of Q_t below about 100]. Rtrace and Qtrace are fp16
+ * [T][B][Np][Np], Np = min(m, n) rounded up to a multiple of 64 (the chain's
+ * zero-padded size; the valid block is the leading min(m, n) square):
+ *   Qtrace[t-1] = Q_t after step t (before a restart resets it);
+ *   Rtrace[t-1] = R_t after step t when the chain computes it (not on the last
+ *     step of a block, whose R update is skipped); after a restart at step t,
+ *     the restarted Gram X_t X_t^T; untouched for t = T.
+ */
+gm_status gm_gram_ns_trace(int B, int m, int n, const void* X, gm_dtype xdt, const float* abc,
+                           int T, const int* restart_after, int n_restart, float eps, void* O,
+                           gm_dtype odt, uint16_t* Rtrace, uint16_t* Qtrace, void* ws,
+                           size_t ws_bytes, gm_stream_t stream);
 
 /* Hyper-parameters of one GRASP step (host struct). */
 typedef struct {
@@ -325,6 +360,19 @@ gm_status gm_ns_flops(int ns_mode, int m, int n, int T, const int* restart_after
  * reported to whichever caller reads the word first. Returns GM_OK or
  * GM_E_TIMEOUT (or GM_E_CUDA). */
 gm_status gm_device_errors(gm_stream_t stream);
+
+/*
+ * Test hook of the failure path (not part of the method): launches the NS
+ * product kernel on one 256 x 256 tile with its operand copies withheld, so
+ * that the bounded wait for the first operand stage runs out after limit_ns
+ * (1 ms .. 1 s). The kernel then records GM_E_TIMEOUT in the current device's
+ * error word, every role leaves its loop, and the tensor memory is released;
+ * gm_device_errors() then returns GM_E_TIMEOUT (and clears the word), and the
+ * device stays usable. X, D: bf16 [256][256] device buffers, never read or
+ * written (the operand and output maps need real addresses).
+ */
+gm_status gm_test_wait_timeout(const uint16_t* X, uint16_t* D, int64_t limit_ns,
+                               gm_stream_t stream);
 
 #ifdef __cplusplus
 }

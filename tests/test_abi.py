@@ -144,3 +144,44 @@ def test_every_cuda_source_is_built():
     assert sorted(Bd.SOURCES) == on_disk
     headers = sorted(f for f in os.listdir(Bd.CSRC) if f.endswith((".cuh", ".h")))
     assert sorted(Bd.HEADERS) == headers
+
+
+def test_new_entry_points_argument_errors():
+    """The step halves, the step's option fields, the mu-law codec, the Gram NS
+    trace and the timeout hook reject bad arguments on the host, before any
+    launch (this runs without a GPU)."""
+    ok, bad = ctypes.c_void_p(4096), ctypes.c_void_p(4096 + 8)
+    st = gm.GraspStateC(*([4096] * 9))
+
+    def prm(**kw):
+        p = gm.GraspParams(0.95, 0.02, 0.0, 8, 5, 0, None, None, 0, 1e-7, 0)
+        for k, v in kw.items():
+            setattr(p, k, v)
+        return p
+
+    big = 1 << 40
+    for p in (prm(power_steps=4), prm(power_steps=-1), prm(residual_from_codes=2),
+              prm(matrix_ids=4096 + 8)):
+        assert gm.lib.gm_grasp_step(1, 256, 512, ctypes.byref(p), ctypes.byref(st), ok, ok, 1, ok,
+                                    big, None) == gm.GM_E_ARG
+        assert gm.lib.gm_grasp_state_update(1, 256, 512, ctypes.byref(p), ctypes.byref(st), ok, 1,
+                                            ok, big, None) == gm.GM_E_ARG
+    p = prm()
+    assert gm.lib.gm_grasp_state_update(1, 256, 512, ctypes.byref(p), ctypes.byref(st), None, 1,
+                                        ok, big, None) == gm.GM_E_ARG
+    assert gm.lib.gm_grasp_apply(1, 256, 512, ctypes.byref(p), ctypes.byref(st), None, ok, big,
+                                 None) == gm.GM_E_ARG
+    assert gm.lib.gm_grasp_apply(1, 256, 512, ctypes.byref(p), ctypes.byref(st), ok, ok, 16,
+                                 None) == gm.GM_E_WORKSPACE
+    # mu-law codec: mu must be positive, shapes and alignment as the group codec
+    assert gm.lib.gm_mulaw_quant4(1, 256, 512, 0.0, ok, ok, ok, None) == gm.GM_E_ARG
+    assert gm.lib.gm_mulaw_quant4(1, 256, 512, -1.0, ok, ok, ok, None) == gm.GM_E_ARG
+    assert gm.lib.gm_mulaw_quant4(1, 250, 512, 255.0, ok, ok, ok, None) == gm.GM_E_ARG
+    assert gm.lib.gm_mulaw_dequant4(1, 256, 512, 255.0, ok, bad, ok, None) == gm.GM_E_ARG
+    # Gram NS trace: both trace buffers required
+    assert gm.lib.gm_gram_ns_trace(1, 256, 512, ok, 1, None, 5, None, 0, 1e-7, ok, 0, None, ok,
+                                   ok, big, None) == gm.GM_E_ARG
+    # timeout hook: the limit stays within [1 ms, 1 s]
+    assert gm.lib.gm_test_wait_timeout(ok, ok, 10, None) == gm.GM_E_ARG
+    assert gm.lib.gm_test_wait_timeout(ok, ok, 5_000_000_000, None) == gm.GM_E_ARG
+    assert gm.lib.gm_test_wait_timeout(None, ok, 20_000_000, None) == gm.GM_E_ARG

@@ -1,0 +1,112 @@
+"""The page's own Gram Newton-Schulz configuration on the GPU: fp16 operands,
+the Polar Express quintics under the safety factor, a restart after step 2
+("优化器 (3)（Gram Newton-Schulz）", §3.2-§3.4, Algorithm 2).
+
+* Parity: gm_gram_ns with that table against the oracle's fp64 Gram NS with
+  the same table, and against its fp64 standard NS (the two agree in exact
+  arithmetic, Theorem 1): relative Frobenius error <= 2e-2.
+* Restart bounds (§3.2): on inputs whose singular values fall to 1e-3, the
+  smallest eigenvalue of every R_t the fp16 chain computes stays above -0.4,
+  and the condition number of every Q_t below 100, read back from the GPU's
+  own fp16 matrices (gm_gram_ns_trace); cond(Q_t) also tracks the oracle's
+  exact-arithmetic value. Without the restart, some cond(Q_t) exceeds 100.
+
+The safety factor's formula (eq. (12)) is lost from the page; the reading used
+is that every step evaluates p_t(x / 1.05) (oracle.safety_scaled).
+"""
+
+import math
+
+import pytest
+import torch
+
+import oracle as O
+from bit_muon_optimizer_b200 import workloads as WL
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+PE = O.safety_scaled(O.POLAR_EXPRESS_ABC)
+
+
+def rel(a, b):
+    a, b = a.double().cpu(), b.double().cpu()
+    return float((a - b).norm() / b.norm())
+
+
+def _outlier_matrix(B, m, n, seed):
+    X = WL.random_matrix((B, m, n), seed, std=1e-3)
+    g = torch.Generator().manual_seed(seed + 1)
+    for b in range(B):
+        X[b, torch.randperm(m, generator=g)[:2], :] *= 10
+        X[b, :, torch.randperm(n, generator=g)[:2]] *= 10
+    return X
+
+
+def _spectrum_matrix(B, m, n, smallest, seed):
+    """U diag(s) V^T, s log-spaced from 1 down to `smallest`."""
+    g = torch.Generator().manual_seed(seed)
+    N = min(m, n)
+    out = torch.empty(B, m, n)
+    s = torch.logspace(0, math.log10(smallest), N, dtype=torch.float64)
+    for b in range(B):
+        U, _ = torch.linalg.qr(torch.randn(m, N, generator=g, dtype=torch.float64))
+        V, _ = torch.linalg.qr(torch.randn(n, N, generator=g, dtype=torch.float64))
+        out[b] = (U @ torch.diag(s) @ V.T).float()
+    return out
+
+
+@pytest.mark.parametrize("B,m,n", [(2, 256, 512), (1, 400, 144), (2, 768, 2048), (1, 512, 512)])
+def test_polar_express_gram_ns_vs_oracle(cuda_lib, B, m, n):
+    gm = cuda_lib
+    X = _outlier_matrix(B, m, n, 61 + m)
+    Og = gm.gram_ns(X.to(DEV), abc=PE, T=5, restart_after=(2,)).cpu()
+    for b in range(B):
+        Xb = X[b].double()
+        assert rel(Og[b], O.gram_ns(Xb, abc=PE, restart_after=(2,))) <= 2e-2
+        assert rel(Og[b], O.ns_standard(Xb, abc=PE)) <= 2e-2
+
+
+def _trace_stats(Rt, Qt, T, restart_after):
+    """(t, lambda_min(R_t) or None, cond(Q_t)) per step from the GPU traces."""
+    ends = set(restart_after) | {T}
+    out = []
+    for t in range(1, T + 1):
+        Q = Qt[t - 1].double()
+        sq = torch.linalg.svdvals(Q)
+        cond = (sq[:, 0] / sq[:, -1]).max().item()
+        lam = None
+        if t not in ends or t < T:
+            R = Rt[t - 1].double()
+            R = 0.5 * (R + R.mT)
+            lam = torch.linalg.eigvalsh(R)[:, 0].min().item()
+        out.append((t, lam, cond))
+    return out
+
+
+@pytest.mark.parametrize("smallest", [1e-3, 1e-4])
+@pytest.mark.parametrize("B,m,n", [(2, 256, 1024), (1, 512, 2048)])
+def test_restart_bounds_on_the_fp16_chain(cuda_lib, B, m, n, smallest):
+    gm = cuda_lib
+    X = _spectrum_matrix(B, m, n, smallest, 70 + m)
+    O_r, Rt, Qt = gm.gram_ns_trace(X.to(DEV), abc=PE, T=5, restart_after=(2,))
+    _, _, Qn = gm.gram_ns_trace(X.to(DEV), abc=PE, T=5, restart_after=())
+    torch.cuda.synchronize()
+    with_r = _trace_stats(Rt, Qt, 5, (2,))
+    cond_without = max(_trace_stats(torch.zeros_like(Qn), Qn, 5, ())[i][2] for i in range(5))
+    exact = []
+    O.gram_ns(X[0].double(), abc=PE, restart_after=(2,), trace=exact)
+    lam_min = min(l for _, l, _ in with_r if l is not None)
+    cond_max = max(c for _, _, c in with_r)
+    print(f"\n[{m}x{n}, s down to {smallest:g}] fp16 chain with restart after step 2: "
+          f"min lambda_min(R_t) = {lam_min:.4f}, max cond(Q_t) = {cond_max:.1f} "
+          f"(exact arithmetic: {max(c for _, _, c in exact):.1f}); without restart: "
+          f"max cond(Q_t) = {cond_without:.1f}")
+    assert lam_min > -0.4
+    assert cond_max < 100
+    assert cond_without > 100
+    for (t, _, c), (te, _, ce) in zip(with_r, exact):
+        assert abs(c - ce) <= 0.1 * ce, f"cond(Q_{t}) {c:.2f} vs exact {ce:.2f}"
+    # and the result is the orthogonalisation
+    for b in range(B):
+        assert rel(O_r[b], O.ns_standard(X[b].double(), abc=PE)) <= 2e-2

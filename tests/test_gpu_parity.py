@@ -609,3 +609,30 @@ def test_grasp_apply_skips_after_a_nonfinite_state_update(cuda_lib):
     torch.cuda.synchronize()
     assert int(st.dev_status.item()) == gm.GM_E_NONFINITE
     assert torch.equal(W, W1) and int(st.step.item()) == 0
+
+
+@pytest.mark.parametrize("mu", [255.0, 15.0])
+@pytest.mark.parametrize("B,m,n,dist", [(2, 256, 512, "gauss"), (3, 144, 272, "student"),
+                                        (1, 16, 48, "gauss")])
+def test_mulaw_codec_bit_exact(cuda_lib, mu, B, m, n, dist):
+    """MuonQ's mu-law companding codec against the oracle's fp64 definition
+    (codes = rint(7 F(x / s)), F the mu-law curve): codes and group scales bit
+    for bit, including a zero group; the decoded values within fp32 rounding of
+    the oracle's s F^-1(q / 7)."""
+    gm = cuda_lib
+    if dist == "gauss":
+        X = _outlier_matrix(B, m, n, 81)
+    else:
+        g = torch.Generator().manual_seed(82)
+        X = (torch.randn(B, m, n, generator=g)
+             / torch.sqrt((torch.randn(3, B, m, n, generator=g) ** 2).sum(0) / 3.0)) * 1e-3
+    X[0].view(-1)[:128] = 0.0
+    codes, gs = gm.mulaw_quant4(X.to(DEV), mu=mu)
+    Xh = gm.mulaw_dequant4(codes, gs, mu=mu)
+    torch.cuda.synchronize()
+    for b in range(B):
+        q, s = O.mulaw_quant4(X[b], mu=mu)
+        assert torch.equal(gs[b].cpu(), s)
+        assert torch.equal(codes[b].cpu(), O.pack_nibbles(q)), f"codes differ in matrix {b}"
+        assert rel(Xh[b], O.mulaw_dequant4(q, s, mu=mu)) <= 1e-6
+    assert float(gs[0, 0]) == 0.0 and int(codes[0].view(-1)[:64].abs().max()) == 0
