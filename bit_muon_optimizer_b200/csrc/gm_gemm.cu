@@ -47,8 +47,14 @@ namespace {
 constexpr int BM = 128;                // output rows per CTA
 constexpr int BN = 256;                // output columns per tile
 constexpr int BK = 64;                 // 64 x 16-bit = 128 B = one swizzle row
-constexpr int KPS = 2;                 // k-blocks per pipeline stage
-constexpr int STAGES = 3;
+#ifndef GM_KPS
+#define GM_KPS 2
+#endif
+#ifndef GM_STAGES
+#define GM_STAGES 3
+#endif
+constexpr int KPS = GM_KPS;            // k-blocks per pipeline stage
+constexpr int STAGES = GM_STAGES;
 constexpr uint32_t kKBlockBytes = 128 * BK * 2;          // 128 rows (or columns) x one k-block
 constexpr uint32_t kABytes = KPS * kKBlockBytes;         // 32 KB
 constexpr uint32_t kBBytes = KPS * kKBlockBytes;         // 32 KB
@@ -881,17 +887,28 @@ bool map_tile(CUtensorMap* m, const void* base, bool f16, int rows, int cols, in
   return encode(m, base, f16, 3, dims, strides, box);
 }
 // The same matrix viewed as [batch][cols / 64][rows][64] (64-column chunks as a
-// dimension) with {64, box_rows, 2, 1} boxes: box_rows rows of two consecutive
-// chunks in one copy, each chunk landing as its own box_rows x 128 B block.
-// Used for K-major operands (rows x K, box_rows 128: two k-blocks) and the
-// MN-major B (K rows x N, box_rows 128: two k-blocks of rows, 128 columns).
-// Requires cols % 64 == 0.
+// dimension) with {64, box_rows, box_chunks, 1} boxes: box_rows rows of
+// box_chunks consecutive chunks in one copy, each chunk landing as its own
+// box_rows x 128 B block. Used for K-major operands (rows x K: 128 rows, one
+// chunk per k-block of a stage) and the MN-major B (K rows x N: the stage's
+// k-blocks of rows, two chunks = 128 columns). Requires cols % 64 == 0.
 bool map_chunks(CUtensorMap* m, const void* base, bool f16, int rows, int cols, int ld, int batch,
-                long long bs, int box_rows) {
+                long long bs, int box_rows, int box_chunks) {
   const cuuint64_t dims[4] = {64, (cuuint64_t)rows, (cuuint64_t)(cols / 64), (cuuint64_t)batch};
   const cuuint64_t strides[3] = {(cuuint64_t)ld * 2, 128, (cuuint64_t)bs * 2};
-  const cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 2, 1};
+  const cuuint32_t box[4] = {64, (cuuint32_t)box_rows, (cuuint32_t)box_chunks, 1};
   return encode(m, base, f16, 4, dims, strides, box);
+}
+// A K-major operand: 128 rows x the KPS k-blocks of one stage per copy.
+bool map_kmajor(CUtensorMap* m, const void* base, bool f16, int rows, int cols, int ld, int batch,
+                long long bs) {
+  return map_chunks(m, base, f16, rows, cols, ld, batch, bs, 128, KPS);
+}
+// The MN-major B operand: the KPS * 64 rows of K of one stage x 128 columns
+// (two 64-column chunks) per copy.
+bool map_mnmajor(CUtensorMap* m, const void* base, bool f16, int rows, int cols, int ld, int batch,
+                 long long bs) {
+  return map_chunks(m, base, f16, rows, cols, ld, batch, bs, KPS * BK, 2);
 }
 
 // SM count of the current device (cached per device).
@@ -978,7 +995,7 @@ cudaError_t xxt(const Ns& c, const uint16_t* X, uint16_t* D) {
   Maps m;
   memset(&m, 0, sizeof(m));
   const long long xbs = (long long)c.N * c.Mp;
-  if (!map_chunks(&m.A, X, c.f16, c.N, c.Mp, c.Mp, c.B, xbs, 128)) return cudaErrorInvalidValue;
+  if (!map_kmajor(&m.A, X, c.f16, c.N, c.Mp, c.Mp, c.B, xbs)) return cudaErrorInvalidValue;
   m.B = m.A;
   GemmParams p = base_params(c.N, c.N, c.Mp, c.B, c.f16, c.skip, c.err);
   if (!sym_out(m, p, c, D, nullptr)) return cudaErrorInvalidValue;
@@ -994,8 +1011,8 @@ cudaError_t symmul(const Ns& c, const uint16_t* S1, const uint16_t* S2, float al
   Maps m;
   memset(&m, 0, sizeof(m));
   const long long bs = (long long)c.N * c.N;
-  if (!map_chunks(&m.A, S1, c.f16, c.N, c.N, c.N, c.B, bs, 128) ||
-      !map_chunks(&m.B, S2, c.f16, c.N, c.N, c.N, c.B, bs, 128))
+  if (!map_kmajor(&m.A, S1, c.f16, c.N, c.N, c.N, c.B, bs) ||
+      !map_kmajor(&m.B, S2, c.f16, c.N, c.N, c.N, c.B, bs))
     return cudaErrorInvalidValue;
   GemmParams p = base_params(c.N, c.N, c.N, c.B, c.f16, c.skip, c.err);
   if (!sym_out(m, p, c, D, D2)) return cudaErrorInvalidValue;
@@ -1014,9 +1031,9 @@ cudaError_t leftmul(const Ns& c, const uint16_t* S, const uint16_t* X, float alp
   Maps m;
   memset(&m, 0, sizeof(m));
   const long long xbs = (long long)c.N * c.Mp;
-  if (!map_chunks(&m.A, S, c.f16, c.N, c.N, c.N, c.B, (long long)c.N * c.N, 128) ||
+  if (!map_kmajor(&m.A, S, c.f16, c.N, c.N, c.N, c.B, (long long)c.N * c.N) ||
       // MN-major B operand: rows of X are the K index, 64-column chunks the N index
-      !map_chunks(&m.B, X, c.f16, c.N, c.Mp, c.Mp, c.B, xbs, 128))
+      !map_mnmajor(&m.B, X, c.f16, c.N, c.Mp, c.Mp, c.B, xbs))
     return cudaErrorInvalidValue;
   GemmParams p = base_params(c.N, c.Mp, c.N, c.B, c.f16, c.skip, c.err);
   p.tiles_m = cdiv(c.N, 2 * BM);
@@ -1186,7 +1203,7 @@ cudaError_t run_wait_timeout_probe(const uint16_t* X, uint16_t* D, uint64_t limi
   Maps m;
   memset(&m, 0, sizeof(m));
   if (!c.err) return cudaErrorInvalidValue;
-  if (!map_chunks(&m.A, X, false, 256, 256, 256, 1, 256 * 256, 128)) return cudaErrorInvalidValue;
+  if (!map_kmajor(&m.A, X, false, 256, 256, 256, 1, 256 * 256)) return cudaErrorInvalidValue;
   m.B = m.A;
   GemmParams p = base_params(256, 256, 256, 1, false, nullptr, c.err);
   if (!sym_out(m, p, c, D, nullptr)) return cudaErrorInvalidValue;
