@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--ns standard|gram]
                     [--impl ours|reference]
+    python bench.py --profile S [--config c] [--group g] [--batch B]   (launches for profilers)
 
 A "step" is one full GRASP step (rebuild, momentum, power iteration, 4/8-bit
 re-quantization, Newton-Schulz, weight update) over every matrix of the
@@ -653,6 +654,38 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(args):
+    """A fixed launch sequence for profilers: args.profile eager GRASP steps of
+    each shape group (or of group args.group only), one group after the other,
+    optionally with args.batch matrices instead of the group's count. No timing
+    and no JSON line; the device status is checked after every group."""
+    from bit_muon_optimizer_b200 import gmuon as gm
+    w = WL.WORKLOADS[args.config]
+    ns_mode = gm.GM_NS_GRAM if args.ns == "gram" else gm.GM_NS_STANDARD
+    dev = torch.device("cuda", 0)
+    gis = range(len(w.groups)) if args.group < 0 else [args.group]
+    for gi in gis:
+        g = w.groups[gi]
+        B = args.batch or g.count
+        base = w.group_base(gi)
+        step = gm.GraspStep(B, g.m, g.n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=ns_mode,
+                            seed=w.seed, device=dev, matrix_ids=list(range(base, base + B)))
+        st = gm.GraspState.zeros(B, g.m, g.n, w.k, dev)
+        W = torch.empty((B, g.m, g.n), dtype=torch.float32, device=dev)
+        G = torch.empty((B, g.m, g.n), dtype=w.gdtype, device=dev)
+        for b in range(B):
+            W[b] = WL.initial_weight(w, base + b, g.m, g.n, device=dev)
+            WL.gradient(w, base + b, 1, g.m, g.n, device=dev, out=G[b])
+        for _ in range(args.profile):
+            step(st, W, G)
+        torch.cuda.synchronize()
+        if int(st.dev_status.item()):
+            raise RuntimeError(f"device status {int(st.dev_status.item())}")
+        print(f"profile: group {gi} ({g.m} x {g.n} x {B}): {args.profile} steps", flush=True)
+        del step, st, W, G
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -663,7 +696,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--profile", type=int, default=0,
+                    help="run this many eager steps per shape group for a profiler, then exit")
+    ap.add_argument("--group", type=int, default=-1, help="--profile: this shape group only")
+    ap.add_argument("--batch", type=int, default=0, help="--profile: matrices per group")
     args = ap.parse_args()
+    if args.profile:
+        if torch.cuda.is_available():
+            torch.cuda.set_device(0)
+        run_profile(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = init_dist(args.gpus)

@@ -55,7 +55,7 @@ struct StepLayout {
 StepLayout step_layout(int B, int m, int n, int k, int ns_mode, bool with_ns) {
   StepLayout L;
   memset(&L, 0, sizeof(L));
-  L.csplit = cdiv(n, 64);                           // projection partials: one per 64-column slab
+  L.csplit = cdiv(n, kGrid);                        // projection partials: one per 128-column block
   L.rsplit_b = backproject_row_splits(B, m, n);
   L.rsplit_g = gram_row_splits(B, m);
   L.ntiles = rebuild_row_blocks(m) * cdiv(n, kGrid) * 8;  // |M|^2 partials: one per warp of a tile

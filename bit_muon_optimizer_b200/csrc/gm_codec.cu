@@ -116,7 +116,6 @@ __device__ __forceinline__ void cp_async_block_zf(void* smem, const void* gmem, 
   }
 }
 
-constexpr int kCT = 512;   // threads of the 128 x 128 codec CTAs (16 warps)
 
 __host__ __device__ constexpr int kb16(int KP) { return KP < 16 ? 16 : KP; }
 
@@ -338,12 +337,24 @@ __global__ void __launch_bounds__(kThreads) k_warm_q(int m, int n, int k, int nb
 //     those fragments (k-step s = slab columns 16 t + 2 s + {0, 1} of every t)
 //     and whose B is Q, both split hi + lo (3xTF32).
 // The decoded nibble value q / 7 comes from a 16-entry table filled with IEEE
-// divisions, so it is bit-identical to (float)q / 7.0f. Each warp writes its own
-// partials, so no block-wide reduction (and no barrier) is needed per tile: P~
-// over its 64-column slab to Ppart[b][slab][row][l] and |M|^2 over its 16 x 64
-// part to norm2_part[b][row tile][column block][warp]; the orthonormalisation
-// sums them in fp64 in a fixed order.
+// divisions, so it is bit-identical to (float)q / 7.0f. No block-wide reduction is
+// needed per tile: the two warps of the same rows (one per 64-column slab) add
+// their P~ partials through shared memory (a named barrier of the pair) and the
+// slab-0 warp writes the sum over the 128-column block to Ppart[b][bj][row][l];
+// each warp writes |M|^2 over its 16 x 64 part to norm2_part[b][row tile][column
+// block][warp]; the orthonormalisation sums them in fp64 in a fixed order.
 constexpr int kRB = 64;     // rows per rebuild tile
+
+// Named barrier of the two warps (one per 64-column slab) that own row block rb
+// of a rebuild tile (barriers 1..4; 0 is the block-wide one).
+__device__ __forceinline__ void pair_sync(int rb) {
+  switch (rb) {
+    case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
+    case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
+    case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
+    default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+  }
+}
 constexpr int kRBT = 256;  // threads per rebuild CTA
 
 enum RebuildSrc { SRC_STATE = 0, SRC_DENSE = 1, SRC_ZERO = 2 };
@@ -494,7 +505,7 @@ __host__ __device__ constexpr int pipe_stage_words(int SRC, int GDT, int KP) {
 }
 __host__ __device__ constexpr int pipe_smem_words(int SRC, int GDT, int KP) {
   return 2 * 8 * (KP / 8) * 32 * 4 + (SRC == SRC_STATE ? 2 * 8 * (kb16(KP) / 16) * 32 * 2 : 0) +
-         2 * pipe_stage_words(SRC, GDT, KP);
+         2 * pipe_stage_words(SRC, GDT, KP) + (SRC == SRC_STATE ? 0 : (kRB / 16) * (KP / 8) * 4 * 32);
 }
 
 template <int SRC, int GDT, int KP>
@@ -522,6 +533,7 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_pipe(
   uint32_t* QF = smp;                          // [slab][s][NL][lane][4]
   uint32_t* RF = QF + 2 * QW;                  // [slab][nt][KSB][lane][2]
   uint32_t* stg = RF + (ST ? 2 * RW : 0);      // two stages of SW words
+  float* PXd = reinterpret_cast<float*>(stg + 2 * SW);   // [rb][NL][4][lane] (without a state)
   __shared__ float deq4[16];
 
   // stage layout
@@ -732,14 +744,30 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_pipe(
         mma_tf32(pt[nl], ah, qv.x, qv.y);
       }
     }
-    if (2 * bj + slab < nsl) {
-      const long long pbase = ((long long)b * nsl + 2 * bj + slab) * m;
+    // the slab-1 warp hands its partials to the slab-0 warp of the same rows (a
+    // slab beyond the last column holds zeros). With a state the hand-over goes
+    // through this pair's own P-fragment rows of the current stage, which only
+    // the pair reads (in its rebuild, before the first pair barrier) and which
+    // are refilled only after the block-wide barrier at the top of the next tile
+    float* PX = ST ? reinterpret_cast<float*>(PFs(s) + rb * KSB * 3 * 128) : PXd + rb * NL * 128;
+    static_assert(!ST || NL * 4 * 32 <= KSB * 3 * 128, "hand-over fits the pair's P fragments");
+    pair_sync(rb);
+    if (slab == 1) {
+#pragma unroll
+      for (int nl = 0; nl < NL; ++nl)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) PX[(nl * 4 + r) * 32 + lane] = pt[nl][r];
+    }
+    pair_sync(rb);
+    if (slab == 0) {
+      const long long pbase = ((long long)b * nb + bj) * m;
 #pragma unroll
       for (int nl = 0; nl < NL; ++nl)
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const int rl = 16 * rb + g + 8 * (r >> 1), l = 8 * nl + 2 * tq + (r & 1);
-          if (r0 + rl < m && l < k) Ppart[(pbase + r0 + rl) * k + l] = pt[nl][r];
+          const float v = __fadd_rn(pt[nl][r], PX[(nl * 4 + r) * 32 + lane]);
+          if (r0 + rl < m && l < k) Ppart[(pbase + r0 + rl) * k + l] = v;
         }
     }
   }
@@ -1146,13 +1174,16 @@ __global__ void __launch_bounds__(kThreads) k_finalize_r(int n, int k, int rspli
 }
 
 // ------------------------------------------------------------------ S7
-// One 128 x 128 grid block per CTA of 16 warps, laid out as in the rebuild:
-// warp w owns the rows 16 (w & 7) + {g, g + 8} and the columns 64 (w >> 3) +
-// 16 t .. + 15. The residual x = M - P R^T is formed in the C fragments: M is
-// loaded as the accumulator, A = -P and B = R^T are tf32 hi + lo pairs
-// (3xTF32, mma.m16n8k8; the raw P and R rows of the block are copied to shared
-// memory with cp.async while M loads). Then the block's row and column absolute maxima, and
-// the codes q = rint(fp32(x / s) * 7) with s = min(row max, column max). Since
+// One 128 x 128 grid block per CTA of 8 warps (two CTAs per SM, so that one
+// CTA's loads overlap the other's arithmetic). Warp w owns the rows 16 w +
+// {g, g + 8} of the block and, in each of its two 64-column slabs, the columns
+// 64 slab + 16 t .. + 15 (lane = 4 g + t): the C fragments of the rank-k
+// products, as in the rebuild. The residual x = M - P R^T is formed in those
+// fragments: M is loaded as the accumulator, A = -P and B = R^T are tf32 hi + lo
+// pairs (3xTF32, mma.m16n8k8). A row's absolute maximum over the block's 128
+// columns is complete inside its warp (the four lanes of the row); the column
+// maxima need one exchange of 8 x 128 values through shared memory. Then the
+// codes q = rint(fp32(x / s) * 7) with s = min(row max, column max). Since
 // |x| <= s, the quotient taken as z = x * fl(7 / s) is within 7 * 2^-22 of
 // fp32(x / s) * 7; where z lies at least 2^-16 away from a rounding tie, rint(z)
 // is the code, elsewhere the IEEE division decides.
@@ -1160,7 +1191,9 @@ __global__ void __launch_bounds__(kThreads) k_finalize_r(int n, int k, int rspli
 // Q8 (given with the P and R column maxima): the CTAs of block column 0 also
 // write the 8-bit codes of their 128 rows of P, those of block row 0 of their
 // 128 rows of R (q = rint(fp32(x / s) * 127), s the column absolute maximum;
-// the worked step's step 5), and block (0, 0) the scales and the step count.
+// the worked step's step 5), after their 4-bit codes; block (0, 0) the scales
+// and the step count.
+constexpr int kRT = 256;   // threads of the residual CTAs (8 warps)
 struct Quant8Out {
   const unsigned* Pmax;
   const unsigned* Rmax;
@@ -1184,7 +1217,6 @@ __device__ __forceinline__ int8_t code8(float x, float s, float r127) {
     q = (int)rintf(__fmul_rn(__fdiv_rn(x, s), 127.0f));
   return (int8_t)max(-127, min(127, q));
 }
-constexpr int kQ8PerThread = kGrid * kMaxK / kCT;   // P or R values per thread, 128 rows
 
 // The residual-from-codes variant: the residual pass's factor fragments PA (-P^)
 // and RB (R^) rebuilt from this step's 8-bit codes, P^ = deq8(code8(P)) and
@@ -1233,7 +1265,7 @@ __global__ void __launch_bounds__(kThreads) k_codes_frags(int m, int n, int k,
 }
 
 template <int KP, bool FR>   // KP = 0: no rank-k term
-__global__ void __launch_bounds__(kCT, 1) k_residual_quant4(
+__global__ void __launch_bounds__(kRT, 2) k_residual_quant4(
     int m, int n, int k, const float* __restrict__ X, const float* __restrict__ P,
     const float* __restrict__ R, const uint32_t* __restrict__ PA, const uint32_t* __restrict__ RB,
     uint8_t* __restrict__ codes4, float* __restrict__ rscale, float* __restrict__ cscale,
@@ -1243,55 +1275,37 @@ __global__ void __launch_bounds__(kCT, 1) k_residual_quant4(
   const int bj = blockIdx.x, bi = blockIdx.y, b = blockIdx.z;
   const int nb = gridDim.x, mb = gridDim.y;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int g = lane >> 2, tq = lane & 3, rb = warp & 7, slab = warp >> 3;
+  const int g = lane >> 2, tq = lane & 3, rb = warp;
   const int r0 = bi * kGrid, c0 = bj * kGrid;
-  const int cb = c0 + 64 * slab + 16 * tq;   // n % 16 == 0: the run is all in or all out
-  const bool colok = cb < n;
   extern __shared__ __align__(16) uint32_t smq[];
   uint32_t* AF = smq;                      // [rb][ks][part][lane][4]: -P hi, lo
   uint32_t* BF = smq + 8 * NL * 2 * 128;   // [slab][nt][ks][lane][4]: {b0, b1} hi, {b0, b1} lo
   float* Praw = reinterpret_cast<float*>(BF + 2 * 8 * NL * 32 * 4);   // [128][k]
   float* Rraw = Praw + kGrid * KP;                                     // [128][k]
   const int nrows = min(kGrid, m - r0), ncols = min(kGrid, n - c0);   // multiples of 16
-  __shared__ __align__(16) float CM[64][kGrid];   // per (warp row block, g): column maxima of 2 rows
-  __shared__ float CQ[4][kGrid];
-  __shared__ float RM[2][kGrid];
-  __shared__ __align__(16) float smax_c[kGrid], r7c[kGrid];
-  __shared__ float smax_r[kGrid], r7r[kGrid];
-  __shared__ float s8[2][kMaxK], r127[2][kMaxK];
-  // 8-bit codes of P (block column 0) and R (block row 0): values loaded up front
-  const bool doP = q8.Pmax && bj == 0, doR = q8.Pmax && bi == 0;
-  float pq[kQ8PerThread], rq[kQ8PerThread];
-  if (doP) {
-    const float* src = P + ((long long)b * m + r0) * k;
-#pragma unroll
-    for (int u = 0; u < kQ8PerThread; ++u) pq[u] = t + u * kCT < nrows * k ? src[t + u * kCT] : 0.f;
-  }
-  if (doR) {
-    const float* src = R + ((long long)b * n + c0) * k;
-#pragma unroll
-    for (int u = 0; u < kQ8PerThread; ++u) rq[u] = t + u * kCT < ncols * k ? src[t + u * kCT] : 0.f;
-  }
-  if (q8.Pmax && t < 2 * kMaxK) {
-    const int w = t / kMaxK, l = t % kMaxK;
-    const float sv = l < k ? __uint_as_float((w ? q8.Rmax : q8.Pmax)[b * k + l]) : 0.f;
-    s8[w][l] = sv;
-    r127[w][l] = sv > 0.f ? __fdiv_rn(127.0f, sv) : 0.f;
-  }
+  __shared__ __align__(16) float CM[8][kGrid];    // per warp: column maxima of its 16 rows
+  __shared__ __align__(16) float r7c[kGrid];
+  __shared__ float smax_c[kGrid];
 
-  float acc[8][4];   // C fragments: element (h, 2 nt + e) of the run at acc[nt][2 h + e]
+  // M as the accumulator: acc[slab][nt][2 h + e] = element (row g + 8 h, column
+  // 64 slab + 16 t + 2 nt + e)
+  float acc[2][8][4];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int gi = r0 + 16 * rb + g + 8 * h;
-    const bool ok = gi < m && colok;
-    const float4* src = reinterpret_cast<const float4*>(X + ((long long)b * m + gi) * n + cb);
+  for (int sl = 0; sl < 2; ++sl) {
+    const int cb = c0 + 64 * sl + 16 * tq;   // n % 16 == 0: the run is all in or all out
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float4 v = ok ? src[u] : make_float4(0.f, 0.f, 0.f, 0.f);
-      acc[2 * u][2 * h] = v.x;
-      acc[2 * u][2 * h + 1] = v.y;
-      acc[2 * u + 1][2 * h] = v.z;
-      acc[2 * u + 1][2 * h + 1] = v.w;
+    for (int h = 0; h < 2; ++h) {
+      const int gi = r0 + 16 * rb + g + 8 * h;
+      const bool ok = gi < m && cb < n;
+      const float4* src = reinterpret_cast<const float4*>(X + ((long long)b * m + gi) * n + cb);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 v = ok ? src[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+        acc[sl][2 * u][2 * h] = v.x;
+        acc[sl][2 * u][2 * h + 1] = v.y;
+        acc[sl][2 * u + 1][2 * h] = v.z;
+        acc[sl][2 * u + 1][2 * h + 1] = v.w;
+      }
     }
   }
   if constexpr (KP > 0 && FR) {
@@ -1310,8 +1324,8 @@ __global__ void __launch_bounds__(kCT, 1) k_residual_quant4(
     cp_async_wait<0>();
     __syncthreads();
 #pragma unroll 4
-    for (int it = 0; it < kGrid * KP / kCT; ++it) {
-      const int e = t + it * kCT;
+    for (int it = 0; it < kGrid * KP / kRT; ++it) {
+      const int e = t + it * kRT;
       const int il = e / KP, l = e % KP;
       const float pv = (il < nrows && l < k) ? -Praw[il * k + l] : 0.f;
       const float rv = (il < ncols && l < k) ? Rraw[il * k + l] : 0.f;
@@ -1345,109 +1359,113 @@ __global__ void __launch_bounds__(kCT, 1) k_residual_quant4(
         al[0] = l4.x; al[1] = l4.y; al[2] = l4.z; al[3] = l4.w;
       }
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const uint4 bv = reinterpret_cast<const uint4*>(BF)[((slab * 8 + nt) * NL + ks) * 32 + lane];
-        mma_tf32(acc[nt], al, bv.x, bv.y);
-        mma_tf32(acc[nt], ah, bv.z, bv.w);
-        mma_tf32(acc[nt], ah, bv.x, bv.y);
-      }
+      for (int sl = 0; sl < 2; ++sl)
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          const uint4 bv = reinterpret_cast<const uint4*>(BF)[((sl * 8 + nt) * NL + ks) * 32 + lane];
+          mma_tf32(acc[sl][nt], al, bv.x, bv.y);
+          mma_tf32(acc[sl][nt], ah, bv.z, bv.w);
+          mma_tf32(acc[sl][nt], ah, bv.x, bv.y);
+        }
     }
   }
-  // rows outside the matrix are 0 (loaded as 0; their P rows are 0), as are columns
-  // row maxima: the thread's 16 columns, then the 4 lanes of the row (64 columns)
+  // rows and columns outside the matrix are 0 (loaded as 0; their P rows are 0)
+  // row maxima over the block's 128 columns: the thread's 32, then the 4 lanes of the row
+  float rmax[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     float v = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) v = fmaxf(v, fmaxf(fabsf(acc[nt][2 * h]), fabsf(acc[nt][2 * h + 1])));
+    for (int sl = 0; sl < 2; ++sl)
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+        v = fmaxf(v, fmaxf(fabsf(acc[sl][nt][2 * h]), fabsf(acc[sl][nt][2 * h + 1])));
     v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
     v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-    if (tq == 0) RM[slab][16 * rb + g + 8 * h] = v;
+    rmax[h] = v;
+    const int gi = r0 + 16 * rb + g + 8 * h;
+    if (tq == 0 && gi < m) rscale[((long long)b * m + gi) * nb + bj] = v;
   }
-  // column maxima over the thread's two rows
-  {
-    float4* dst = reinterpret_cast<float4*>(&CM[8 * rb + g][64 * slab + 16 * tq]);
+  // column maxima over the warp's 16 rows (the 8 lanes g of each column), then
+  // over the 8 warps
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      float c4[4];
+  for (int sl = 0; sl < 2; ++sl) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int nt = 2 * u + (e >> 1), ee = e & 1;
-        c4[e] = fmaxf(fabsf(acc[nt][ee]), fabsf(acc[nt][2 + ee]));
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float v = fmaxf(fabsf(acc[sl][nt][e]), fabsf(acc[sl][nt][2 + e]));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+        if (g == 0) CM[rb][64 * sl + 16 * tq + 2 * nt + e] = v;
       }
-      dst[u] = make_float4(c4[0], c4[1], c4[2], c4[3]);
     }
-  }
-  __syncthreads();
-  {
-    const int c = t & (kGrid - 1), q = t >> 7;
-    float v = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v = fmaxf(v, CM[16 * q + i][c]);
-    CQ[q][c] = v;
   }
   __syncthreads();
   if (t < kGrid) {
-    const float v = fmaxf(fmaxf(CQ[0][t], CQ[1][t]), fmaxf(CQ[2][t], CQ[3][t]));
+    float v = CM[0][t];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) v = fmaxf(v, CM[w][t]);
     smax_c[t] = v;
     r7c[t] = v > 0.f ? __fdiv_rn(7.0f, v) : 0.f;
     if (c0 + t < n) cscale[((long long)b * mb + bi) * n + c0 + t] = v;
-  } else if (t < 2 * kGrid) {
-    const int r = t - kGrid;
-    const float v = fmaxf(RM[0][r], RM[1][r]);
-    smax_r[r] = v;
-    r7r[r] = v > 0.f ? __fdiv_rn(7.0f, v) : 0.f;
-    if (r0 + r < m) rscale[((long long)b * m + r0 + r) * nb + bj] = v;
   }
   __syncthreads();
-  float rc7[16];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const float4 v = *reinterpret_cast<const float4*>(&r7c[64 * slab + 16 * tq + 4 * u]);
-    rc7[4 * u] = v.x; rc7[4 * u + 1] = v.y; rc7[4 * u + 2] = v.z; rc7[4 * u + 3] = v.w;
-  }
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int rl = 16 * rb + g + 8 * h, gi = r0 + rl;
-    if (gi >= m || !colok) continue;
-    const float rr7 = r7r[rl];
-    uint32_t w[2] = {0u, 0u};
+    const float rr7 = rmax[h] > 0.f ? __fdiv_rn(7.0f, rmax[h]) : 0.f;
 #pragma unroll
-    for (int ce = 0; ce < 16; ++ce) {
-      const float x = acc[ce >> 1][2 * h + (ce & 1)];
-      const float z = __fmul_rn(x, fmaxf(rr7, rc7[ce]));
-      const float zr = rintf(z);
-      int q;
-      if (fabsf(__fsub_rn(z, zr)) < 0.49998474f) {   // 0.5 - 2^-16
-        q = (int)zr;
-      } else {
-        const float sv = fminf(smax_r[rl], smax_c[64 * slab + 16 * tq + ce]);
-        q = sv > 0.f ? (int)rintf(__fmul_rn(__fdiv_rn(x, sv), 7.0f)) : 0;
+    for (int sl = 0; sl < 2; ++sl) {
+      const int cb = c0 + 64 * sl + 16 * tq;
+      if (gi >= m || cb >= n) continue;
+      float rc7[16];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 v = *reinterpret_cast<const float4*>(&r7c[64 * sl + 16 * tq + 4 * u]);
+        rc7[4 * u] = v.x; rc7[4 * u + 1] = v.y; rc7[4 * u + 2] = v.z; rc7[4 * u + 3] = v.w;
       }
-      q = max(-7, min(7, q));
-      w[ce >> 3] |= (uint32_t)(q & 0xF) << (4 * (ce & 7));
-    }
-    *reinterpret_cast<uint2*>(codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2) = make_uint2(w[0], w[1]);
-  }
-  if (doP) {
-    int8_t* dst = q8.P8 + ((long long)b * m + r0) * k;
+      uint32_t w[2] = {0u, 0u};
 #pragma unroll
-    for (int u = 0; u < kQ8PerThread; ++u) {
-      const int e = t + u * kCT;
-      if (e < nrows * k) dst[e] = code8(pq[u], s8[0][e % k], r127[0][e % k]);
+      for (int ce = 0; ce < 16; ++ce) {
+        const float x = acc[sl][ce >> 1][2 * h + (ce & 1)];
+        const float z = __fmul_rn(x, fmaxf(rr7, rc7[ce]));
+        const float zr = rintf(z);
+        int q;
+        if (fabsf(__fsub_rn(z, zr)) < 0.49998474f) {   // 0.5 - 2^-16
+          q = (int)zr;
+        } else {
+          const float sv = fminf(rmax[h], smax_c[64 * sl + 16 * tq + ce]);
+          q = sv > 0.f ? (int)rintf(__fmul_rn(__fdiv_rn(x, sv), 7.0f)) : 0;
+        }
+        q = max(-7, min(7, q));
+        w[ce >> 3] |= (uint32_t)(q & 0xF) << (4 * (ce & 7));
+      }
+      *reinterpret_cast<uint2*>(codes4 + ((long long)b * m + gi) * (n / 2) + cb / 2) = make_uint2(w[0], w[1]);
     }
   }
-  if (doR) {
-    int8_t* dst = q8.R8 + ((long long)b * n + c0) * k;
-#pragma unroll
-    for (int u = 0; u < kQ8PerThread; ++u) {
-      const int e = t + u * kCT;
-      if (e < ncols * k) dst[e] = code8(rq[u], s8[1][e % k], r127[1][e % k]);
+  // 8-bit codes of P (block column 0) and R (block row 0), after the block's own
+  // codes: the factor values are loaded only now, so they hold no registers above
+  if (q8.Pmax && (bj == 0 || bi == 0)) {
+    for (int which = 0; which < 2; ++which) {
+      const bool doit = which == 0 ? bj == 0 : bi == 0;
+      if (!doit) continue;
+      const unsigned* mx = which == 0 ? q8.Pmax : q8.Rmax;
+      const float* src = which == 0 ? P + ((long long)b * m + r0) * k : R + ((long long)b * n + c0) * k;
+      int8_t* dst = which == 0 ? q8.P8 + ((long long)b * m + r0) * k : q8.R8 + ((long long)b * n + c0) * k;
+      const int cnt = (which == 0 ? nrows : ncols) * k;
+      for (int e = t; e < cnt; e += kRT) {
+        const int l = e % k;
+        const float sv = __uint_as_float(mx[b * k + l]);
+        const float r127 = sv > 0.f ? __fdiv_rn(127.0f, sv) : 0.f;
+        dst[e] = code8(src[e], sv, r127);
+      }
     }
-  }
-  if (doP && bi == 0 && t < k) {
-    q8.Pscale[b * k + t] = s8[0][t];
-    q8.Rscale[b * k + t] = s8[1][t];
+    if (bi == 0 && bj == 0 && t < k) {
+      q8.Pscale[b * k + t] = __uint_as_float(q8.Pmax[b * k + t]);
+      q8.Rscale[b * k + t] = __uint_as_float(q8.Rmax[b * k + t]);
+    }
   }
   if (q8.step && b == 0 && bi == 0 && bj == 0 && t == 0) *q8.step += 1;
 }
@@ -1591,7 +1609,7 @@ cudaError_t launch_residual_t(int B, int m, int n, int k, const float* X, const 
     if (e != cudaSuccess) return e;
   }
   dim3 grid(cdiv(n, kGrid), cdiv(m, kGrid), B);
-  k_residual_quant4<KP, FR><<<grid, kCT, smem, s>>>(m, n, k, X, P, R, PA, RB, codes4, rscale, cscale,
+  k_residual_quant4<KP, FR><<<grid, kRT, smem, s>>>(m, n, k, X, P, R, PA, RB, codes4, rscale, cscale,
                                                     q8, skip);
   return cudaGetLastError();
 }

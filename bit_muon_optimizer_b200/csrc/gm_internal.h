@@ -38,8 +38,8 @@ cudaError_t launch_warm_start(int B, int m, int n, int k, const int8_t* R8, cons
 
 // M = mu * Mprev + G where Mprev is either the rebuilt state (codes4 != NULL)
 // or a dense fp32 matrix (Mprev32 != NULL) or zero; with Q != NULL also the
-// projection partials Ppart f32 [B][ceil(n/64)][m][k] (sum over one 64-column
-// slab each). norm2_part gets one fp64 partial |M|^2 per warp of a 64 x 128 tile
+// projection partials Ppart f32 [B][ceil(n/128)][m][k] (sum over one 128-column
+// block each). norm2_part gets one fp64 partial |M|^2 per warp of a 64 x 128 tile
 // ([B][ceil(m/64)][ceil(n/128)][8]); status (nullable) gets GM_E_NONFINITE.
 // Data pointers are 16-byte aligned; m and n are multiples of 16. The fused pass
 // takes the ready-made fragments QF (with Q) and RF, PF (with the state); the
