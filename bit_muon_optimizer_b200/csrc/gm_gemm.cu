@@ -47,24 +47,15 @@ namespace {
 constexpr int BM = 128;                // output rows per CTA
 constexpr int BN = 256;                // output columns per tile
 constexpr int BK = 64;                 // 64 x 16-bit = 128 B = one swizzle row
-#ifndef GM_KPS
-#define GM_KPS 2
-#endif
-#ifndef GM_STAGES
-#define GM_STAGES 3
-#endif
-constexpr int KPS = GM_KPS;            // k-blocks per pipeline stage
-constexpr int STAGES = GM_STAGES;
+// The operand ring holds kRingKBlocks k-blocks of A and B per CTA, cut into
+// stages of KPS k-blocks (a kernel template parameter): 3 stages of 2 k-blocks
+// (32 KB copies) for deep products, 6 stages of 1 for short ones, where finer
+// stages keep the MMAs fed across the more frequent tile changes.
+constexpr int kRingKBlocks = 6;
 constexpr uint32_t kKBlockBytes = 128 * BK * 2;          // 128 rows (or columns) x one k-block
-constexpr uint32_t kABytes = KPS * kKBlockBytes;         // 32 KB
-constexpr uint32_t kBBytes = KPS * kKBlockBytes;         // 32 KB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;      // 64 KB per CTA
+constexpr uint32_t kRingBytes = 2 * kRingKBlocks * kKBlockBytes;   // A and B: 192 KB per CTA
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-#ifndef GM_LOAD_LANES
-#define GM_LOAD_LANES 1
-#endif
-constexpr int kLoadLanes = GM_LOAD_LANES;   // operand-copy issuing threads per operand
-static_assert(kLoadLanes >= 1 && kLoadLanes <= STAGES, "one stage per loader at least");
+
 
 constexpr int kEpiWarp0 = 4;
 constexpr int kEpiWarps = 16;                            // four per TMEM lane quarter
@@ -79,8 +70,7 @@ static_assert(CPW == 16, "one tcgen05.ld x16 per thread per slab");
 constexpr uint32_t kBoxBytes = 64 * 128;                 // 64 x 64 16-bit values
 constexpr uint32_t kOutBufBytes = 2 * kBoxBytes;         // rows 0..63 and 64..127 of a slab
 static_assert(BM * SLAB * 4 <= 2 * kOutBufBytes, "fp32 staging (output modes) fits the slab buffers");
-constexpr uint32_t kSmemBytes =
-    STAGES * kStageBytes + 2 * kOutBufBytes + 1024 /* barriers */ + 1024 /* align */;
+constexpr uint32_t kSmemBytes = kRingBytes + 2 * kOutBufBytes + 1024 /* barriers */ + 1024 /* align */;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 __device__ int32_t g_device_error = 0;
@@ -576,7 +566,7 @@ __device__ __forceinline__ void epilogue_out_slab(const GemmParams& p, uint8_t* 
 }
 
 // ------------------------------------------------------------------ kernel
-template <bool B_MN>
+template <bool B_MN, int KPS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmDs,
@@ -585,6 +575,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // The skip flag is read by both CTAs of a pair before any cluster-level
   // operation, so they return together.
   if (p.skip && *p.skip) return;
+  constexpr int STAGES = kRingKBlocks / KPS;
+  constexpr uint32_t kABytes = KPS * kKBlockBytes;       // A and B per stage and CTA
+  constexpr uint32_t kStageBytes = 2 * kABytes;
+  static_assert(STAGES * KPS == kRingKBlocks, "the ring holds whole stages");
 
   extern __shared__ __align__(1024) uint8_t dsm[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm) + 1023) &
@@ -661,16 +655,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // Role dispatch by warp; within a role warp only the lanes named below work,
   // the others go straight to the final barrier.
   if (warp == 0 || warp == 2) {
-    if (lane < kLoadLanes) {
-      // ---------------- TMA producers: warp 0 loads A, warp 2 loads B (both CTAs);
-      // lane j of each issues the stages g with g % kLoadLanes == j
+    if (lane == 0) {
+      // ---------------- TMA producers: warp 0 loads A, warp 2 loads B (both CTAs)
       const bool isA = warp == 0;
       uint32_t g = 0;
       bool ok = !p.stall;
       for (int T = pid; T < total && ok; T += npairs) {
         const TileCoord tc = decode_tile(p, T, tiles_per, (int)cr);
         for (int st = 0; st < nst; ++st, ++g) {
-          if ((int)(g % kLoadLanes) != lane) continue;
           const int s = (int)(g % STAGES);
           const uint32_t ph = (g / STAGES) & 1u;
           if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err, abort_flag, p.wait_ns)) { ok = false; break; }
@@ -899,17 +891,20 @@ bool map_chunks(CUtensorMap* m, const void* base, bool f16, int rows, int cols, 
   const cuuint32_t box[4] = {64, (cuuint32_t)box_rows, (cuuint32_t)box_chunks, 1};
   return encode(m, base, f16, 4, dims, strides, box);
 }
-// A K-major operand: 128 rows x the KPS k-blocks of one stage per copy.
+// A K-major operand: 128 rows x the kps k-blocks of one stage per copy.
 bool map_kmajor(CUtensorMap* m, const void* base, bool f16, int rows, int cols, int ld, int batch,
-                long long bs) {
-  return map_chunks(m, base, f16, rows, cols, ld, batch, bs, 128, KPS);
+                long long bs, int kps) {
+  return map_chunks(m, base, f16, rows, cols, ld, batch, bs, 128, kps);
 }
-// The MN-major B operand: the KPS * 64 rows of K of one stage x 128 columns
+// The MN-major B operand: the kps * 64 rows of K of one stage x 128 columns
 // (two 64-column chunks) per copy.
 bool map_mnmajor(CUtensorMap* m, const void* base, bool f16, int rows, int cols, int ld, int batch,
-                 long long bs) {
-  return map_chunks(m, base, f16, rows, cols, ld, batch, bs, KPS * BK, 2);
+                 long long bs, int kps) {
+  return map_chunks(m, base, f16, rows, cols, ld, batch, bs, kps * BK, 2);
 }
+// k-blocks per pipeline stage for a product of reduction depth K (see kRingKBlocks)
+constexpr int kShortK = 1024;
+int stage_kblocks(int K) { return K <= kShortK ? 1 : 2; }
 
 // SM count of the current device (cached per device).
 int num_sms() {
@@ -929,11 +924,11 @@ struct Maps {
   CUtensorMap A, B, D, Ds, D2, D2s;
 };
 
-template <bool B_MN>
-cudaError_t launch_gemm(const Maps& m, const GemmParams& p, cudaStream_t s) {
+template <bool B_MN, int KPS>
+cudaError_t launch_gemm_t(const Maps& m, const GemmParams& p, cudaStream_t s) {
   static DeviceOnce attr;
   {
-    const cudaError_t e = smem_attr_once(attr, k_gemm<B_MN>, kSmemBytes);
+    const cudaError_t e = smem_attr_once(attr, k_gemm<B_MN, KPS>, kSmemBytes);
     if (e != cudaSuccess) return e;
   }
   const int tiles = p.sym ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
@@ -949,7 +944,12 @@ cudaError_t launch_gemm(const Maps& m, const GemmParams& p, cudaStream_t s) {
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_gemm<B_MN>, m.A, m.B, m.D, m.Ds, m.D2, m.D2s, p);
+  return cudaLaunchKernelEx(&cfg, k_gemm<B_MN, KPS>, m.A, m.B, m.D, m.Ds, m.D2, m.D2s, p);
+}
+// The operand maps must have been encoded for stage_kblocks(p.K).
+template <bool B_MN>
+cudaError_t launch_gemm(const Maps& m, const GemmParams& p, cudaStream_t s) {
+  return stage_kblocks(p.K) == 1 ? launch_gemm_t<B_MN, 1>(m, p, s) : launch_gemm_t<B_MN, 2>(m, p, s);
 }
 
 GemmParams base_params(int M, int N, int K, int batch, bool f16, const int32_t* skip, int32_t* err) {
@@ -995,7 +995,8 @@ cudaError_t xxt(const Ns& c, const uint16_t* X, uint16_t* D) {
   Maps m;
   memset(&m, 0, sizeof(m));
   const long long xbs = (long long)c.N * c.Mp;
-  if (!map_kmajor(&m.A, X, c.f16, c.N, c.Mp, c.Mp, c.B, xbs)) return cudaErrorInvalidValue;
+  if (!map_kmajor(&m.A, X, c.f16, c.N, c.Mp, c.Mp, c.B, xbs, stage_kblocks(c.Mp)))
+    return cudaErrorInvalidValue;
   m.B = m.A;
   GemmParams p = base_params(c.N, c.N, c.Mp, c.B, c.f16, c.skip, c.err);
   if (!sym_out(m, p, c, D, nullptr)) return cudaErrorInvalidValue;
@@ -1011,8 +1012,9 @@ cudaError_t symmul(const Ns& c, const uint16_t* S1, const uint16_t* S2, float al
   Maps m;
   memset(&m, 0, sizeof(m));
   const long long bs = (long long)c.N * c.N;
-  if (!map_kmajor(&m.A, S1, c.f16, c.N, c.N, c.N, c.B, bs) ||
-      !map_kmajor(&m.B, S2, c.f16, c.N, c.N, c.N, c.B, bs))
+  const int kps = stage_kblocks(c.N);
+  if (!map_kmajor(&m.A, S1, c.f16, c.N, c.N, c.N, c.B, bs, kps) ||
+      !map_kmajor(&m.B, S2, c.f16, c.N, c.N, c.N, c.B, bs, kps))
     return cudaErrorInvalidValue;
   GemmParams p = base_params(c.N, c.N, c.N, c.B, c.f16, c.skip, c.err);
   if (!sym_out(m, p, c, D, D2)) return cudaErrorInvalidValue;
@@ -1031,9 +1033,10 @@ cudaError_t leftmul(const Ns& c, const uint16_t* S, const uint16_t* X, float alp
   Maps m;
   memset(&m, 0, sizeof(m));
   const long long xbs = (long long)c.N * c.Mp;
-  if (!map_kmajor(&m.A, S, c.f16, c.N, c.N, c.N, c.B, (long long)c.N * c.N) ||
+  const int kps = stage_kblocks(c.N);
+  if (!map_kmajor(&m.A, S, c.f16, c.N, c.N, c.N, c.B, (long long)c.N * c.N, kps) ||
       // MN-major B operand: rows of X are the K index, 64-column chunks the N index
-      !map_mnmajor(&m.B, X, c.f16, c.N, c.Mp, c.Mp, c.B, xbs))
+      !map_mnmajor(&m.B, X, c.f16, c.N, c.Mp, c.Mp, c.B, xbs, kps))
     return cudaErrorInvalidValue;
   GemmParams p = base_params(c.N, c.Mp, c.N, c.B, c.f16, c.skip, c.err);
   p.tiles_m = cdiv(c.N, 2 * BM);
@@ -1203,7 +1206,8 @@ cudaError_t run_wait_timeout_probe(const uint16_t* X, uint16_t* D, uint64_t limi
   Maps m;
   memset(&m, 0, sizeof(m));
   if (!c.err) return cudaErrorInvalidValue;
-  if (!map_kmajor(&m.A, X, false, 256, 256, 256, 1, 256 * 256)) return cudaErrorInvalidValue;
+  if (!map_kmajor(&m.A, X, false, 256, 256, 256, 1, 256 * 256, stage_kblocks(256)))
+    return cudaErrorInvalidValue;
   m.B = m.A;
   GemmParams p = base_params(256, 256, 256, 1, false, nullptr, c.err);
   if (!sym_out(m, p, c, D, nullptr)) return cudaErrorInvalidValue;

@@ -126,12 +126,14 @@ def _rank_main(rank, world, port, q, kind="standin", set_ids=True):
     import torch.distributed as dist
     dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     try:
+        # plain arrays, pickled by value: a tensor would be shared through a file
+        # descriptor that dies with this process if it exits before the parent reads
         if kind == "standin":
             sh, W = _run(world, rank)
-            q.put((rank, sh.owner, W))
+            q.put((rank, sh.owner, [w.numpy() for w in W]))
         else:
             W, codes = _run_oracle(world, rank, set_ids)
-            q.put((rank, W, codes))
+            q.put((rank, [w.numpy() for w in W], {k: v.numpy() for k, v in codes.items()}))
     finally:
         dist.destroy_process_group()
 
@@ -148,6 +150,9 @@ def _spawn(world, kind="standin", set_ids=True):
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
+    out = [(r, a, [torch.from_numpy(x) for x in b] if kind == "standin" else b) if kind == "standin"
+           else (r, [torch.from_numpy(x) for x in a], {k: torch.from_numpy(v) for k, v in b.items()})
+           for r, a, b in out]
     return sorted(out, key=lambda x: x[0])
 
 
