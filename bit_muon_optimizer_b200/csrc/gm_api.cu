@@ -48,7 +48,7 @@ void expand_abc(const float* abc, int T, float* out) {
 
 struct StepLayout {
   size_t M, Q, P, R, X, scale, norm2, Ppart, Ptil, gram, Tm, Rpart, qnorm, QF, RF, PF, PA, RB, PB,
-      ns, total;
+      PT, RT, ns, total;
   int csplit, rsplit_b, rsplit_g, ntiles;
 };
 
@@ -82,6 +82,8 @@ StepLayout step_layout(int B, int m, int n, int k, int ns_mode, bool with_ns) {
   L.PA = take((size_t)fw.PA * 4);
   L.RB = take((size_t)fw.RB * 4);
   L.PB = take((size_t)fw.PB * 4);
+  L.PT = take(Bz * mz * 32 * 4 * 2);   // tensor-core residual operand rows: tf32 hi, lo
+  L.RT = take(Bz * nz * 32 * 4 * 2);
   if (with_ns)
     L.ns = take(ns_mode == GM_NS_GRAM ? ns_gram_ws_bytes(B, m, n) : ns_standard_ws_bytes(B, m, n));
   L.total = off;
@@ -268,9 +270,9 @@ gm_status gm_momentum_powerit(int B, int m, int n, int k, float mu, const float*
   GM_CUDA(launch_rebuild(B, m, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                          M_prev, mu, G, gdt, Q, QF, nullptr, nullptr, M_out, norm2, Ppart, nullptr, s));
   GM_CUDA(launch_orth(B, m, k, L.csplit, Ppart, Ptil, gram, Tm, norm2, L.ntiles, 1e-7f, scale,
-                      P_out, PB, nullptr, nullptr, nullptr, s));
+                      P_out, PB, nullptr, nullptr, nullptr, nullptr, s));
   GM_CUDA(launch_backproject(B, m, n, k, M_out, PB, nullptr, nullptr, false, Rpart, R_out, nullptr,
-                             nullptr, nullptr, s));
+                             nullptr, nullptr, nullptr, s));
   return GM_OK;
 }
 
@@ -465,6 +467,8 @@ gm_status gm_grasp_state_update(int B, int m, int n, const gm_grasp_params* prm,
   uint32_t* PA = reinterpret_cast<uint32_t*>(w + L.PA);
   uint32_t* RB = reinterpret_cast<uint32_t*>(w + L.RB);
   uint32_t* PB = reinterpret_cast<uint32_t*>(w + L.PB);
+  float* PT = reinterpret_cast<float*>(w + L.PT);
+  float* RT = reinterpret_cast<float*>(w + L.RT);
   int32_t* status = st->dev_status;
   const bool gramns = prm->ns == GM_NS_GRAM;
   const int psteps = prm->power_steps < 1 ? 1 : prm->power_steps;
@@ -483,9 +487,9 @@ gm_status gm_grasp_state_update(int B, int m, int n, const gm_grasp_params* prm,
                          status, s));
   // worked step 4: P = orth(P~), R = M^T P (and the normalised NS input X)
   GM_CUDA(launch_orth(B, m, k, L.csplit, Ppart, Ptil, gram, Tm, norm2, L.ntiles, prm->eps, scale,
-                      P, PB, PA, PRmax, status, s));
-  GM_CUDA(launch_backproject(B, m, n, k, M, PB, scale, X, gramns, Rpart, R, RB, PRmax + (size_t)B * k,
-                             status, s));
+                      P, PB, PA, PT, PRmax, status, s));
+  GM_CUDA(launch_backproject(B, m, n, k, M, PB, scale, X, gramns, Rpart, R, RB, RT,
+                             PRmax + (size_t)B * k, status, s));
   // further power-iteration steps: Q = column-normalised R, P~ = M Q (a projection
   // pass over the stored M_t), P = orth(P~), R = M^T P
   for (int it = 1; it < psteps; ++it) {
@@ -496,16 +500,18 @@ gm_status gm_grasp_state_update(int B, int m, int n, const gm_grasp_params* prm,
                            nullptr, Ppart, status, s));
     GM_CUDA(cudaMemsetAsync(PRmax, 0, sizeof(unsigned) * 2 * (size_t)B * k, s));
     GM_CUDA(launch_orth(B, m, k, L.csplit, Ppart, Ptil, gram, Tm, norm2, L.ntiles, prm->eps, scale,
-                        P, PB, PA, PRmax, status, s));
-    GM_CUDA(launch_backproject(B, m, n, k, M, PB, nullptr, nullptr, gramns, Rpart, R, RB,
+                        P, PB, PA, PT, PRmax, status, s));
+    GM_CUDA(launch_backproject(B, m, n, k, M, PB, nullptr, nullptr, gramns, Rpart, R, RB, RT,
                                PRmax + (size_t)B * k, status, s));
   }
   // worked step 5 variant: the residual from the dequantized 8-bit factors
   if (prm->residual_from_codes)
-    GM_CUDA(launch_codes_frags(B, m, n, k, P, R, PRmax, PRmax + (size_t)B * k, PA, RB, status, s));
-  // worked step 5: residual -> 4-bit grid codes; P, R -> 8-bit codes (state in place)
-  GM_CUDA(launch_residual_quant4(B, m, n, k, M, P, R, PA, RB, st->codes4, st->rscale, st->cscale,
-                                 PRmax, st->P8, st->Pscale, st->R8, st->Rscale, st->step, status, s));
+    GM_CUDA(launch_codes_frags(B, m, n, k, P, R, PRmax, PRmax + (size_t)B * k, PA, RB, PT, RT, status,
+                               s));
+  // worked step 5: residual -> 4-bit grid codes (tensor cores); P, R -> 8-bit codes
+  // (state in place)
+  GM_CUDA(launch_residual_tc(B, m, n, k, M, P, R, PT, RT, st->codes4, st->rscale, st->cscale, PRmax,
+                             st->P8, st->Pscale, st->R8, st->Rscale, st->step, status, status, s));
   return GM_OK;
 }
 

@@ -907,6 +907,8 @@ __global__ void __launch_bounds__(32) k_orth_chol(int k, int rsplit, const doubl
 // column. Stored fp32 and as fragments: PB for the back-projection (PB[b][i / 8]
 // [l / 8][lane][4] = {hi(P[8 s + t][l]), hi(P[8 s + t + 4][l]), lo, lo}, lane =
 // 4 (l % 8) + t) and PA (-P) for the residual (nullable); zero for k <= l < KP.
+// PT (nullable): the tensor-core residual's operand rows, tf32 hi then lo halves
+// ([2][B][m][32], columns beyond k zero).
 // The column absolute maxima of P go to Pmax (fp32 bits, atomicMax; nullable).
 template <int KP>
 __global__ void __launch_bounds__(kThreads) k_orth_apply(int m, int k, const double* __restrict__ Ptil,
@@ -914,6 +916,7 @@ __global__ void __launch_bounds__(kThreads) k_orth_apply(int m, int k, const dou
                                                           float* __restrict__ P,
                                                           uint32_t* __restrict__ PB,
                                                           uint32_t* __restrict__ PA,
+                                                          float* __restrict__ PT,
                                                           unsigned* __restrict__ Pmax,
                                                           const int32_t* skip) {
   if (skip && *skip) return;
@@ -954,6 +957,20 @@ __global__ void __launch_bounds__(kThreads) k_orth_apply(int m, int k, const dou
       const uint32_t hi = tf32_hi(-f);
       PA[at] = hi;
       PA[at + 128] = tf32_lo(-f, hi);
+    }
+    if (PT) {
+      const long long at = ((long long)b * m + i) * 32 + l;
+      const uint32_t hi = tf32_hi(f);
+      PT[at] = __uint_as_float(hi);
+      PT[(long long)gridDim.y * m * 32 + at] = __uint_as_float(tf32_lo(f, hi));
+    }
+  }
+  if (PT && in) {   // the operand tiles' columns beyond the factor width are zero
+#pragma unroll
+    for (int l = KP; l < 32; ++l) {
+      const long long at = ((long long)b * m + i) * 32 + l;
+      PT[at] = 0.f;
+      PT[(long long)gridDim.y * m * 32 + at] = 0.f;
     }
   }
   __syncthreads();
@@ -1143,6 +1160,7 @@ __global__ void __launch_bounds__(kThreads) k_finalize_r(int n, int k, int rspli
                                                           const double* __restrict__ Rpart,
                                                           float* __restrict__ R,
                                                           uint32_t* __restrict__ RB,
+                                                          float* __restrict__ RT,
                                                           unsigned* __restrict__ Rmax,
                                                           const int32_t* skip) {
   if (skip && *skip) return;
@@ -1170,6 +1188,14 @@ __global__ void __launch_bounds__(kThreads) k_finalize_r(int n, int k, int rspli
     const uint32_t hi = tf32_hi(f);
     RB[at] = hi;
     RB[at + 2] = tf32_lo(f, hi);
+  }
+  if (RT && j < n) {   // the tensor-core residual's operand rows ([2][B][n][32], tf32 hi, lo)
+    const long long row = ((long long)b * n + j) * 32, lo_off = (long long)gridDim.y * n * 32;
+    const uint32_t hi = tf32_hi(f);
+    RT[row + l] = __uint_as_float(hi);
+    RT[lo_off + row + l] = __uint_as_float(tf32_lo(f, hi));
+    if (l == kp - 1)
+      for (int c = kp; c < 32; ++c) RT[row + c] = RT[lo_off + row + c] = 0.f;
   }
 }
 
@@ -1231,6 +1257,8 @@ __global__ void __launch_bounds__(kThreads) k_codes_frags(int m, int n, int k,
                                                            const unsigned* __restrict__ Rmax,
                                                            uint32_t* __restrict__ PA,
                                                            uint32_t* __restrict__ RB,
+                                                           float* __restrict__ PT,
+                                                           float* __restrict__ RT,
                                                            const int32_t* skip) {
   if (skip && *skip) return;
   const int b = blockIdx.y, t = threadIdx.x;
@@ -1252,6 +1280,12 @@ __global__ void __launch_bounds__(kThreads) k_codes_frags(int m, int n, int k,
     const uint32_t hi = tf32_hi(v);
     PA[at] = hi;
     PA[at + 128] = tf32_lo(v, hi);
+    if (PT) {   // +P^ for the tensor-core residual
+      const long long pt = ((long long)b * m + i) * 32 + l;
+      const uint32_t ph = tf32_hi(-v);
+      PT[pt] = __uint_as_float(ph);
+      PT[(long long)gridDim.y * m * 32 + pt] = __uint_as_float(tf32_lo(-v, ph));
+    }
   } else if (e < np + nr) {
     const long long e2 = e - np;
     const int j = (int)(e2 / k), l = (int)(e2 % k);
@@ -1261,6 +1295,11 @@ __global__ void __launch_bounds__(kThreads) k_codes_frags(int m, int n, int k,
     const uint32_t hi = tf32_hi(v);
     RB[at] = hi;
     RB[at + 2] = tf32_lo(v, hi);
+    if (RT) {
+      const long long rt = ((long long)b * n + j) * 32 + l;
+      RT[rt] = __uint_as_float(hi);
+      RT[(long long)gridDim.y * n * 32 + rt] = __uint_as_float(tf32_lo(v, hi));
+    }
   }
 }
 
@@ -1470,6 +1509,309 @@ __global__ void __launch_bounds__(kRT, 2) k_residual_quant4(
   if (q8.step && b == 0 && bi == 0 && bj == 0 && t == 0) *q8.step += 1;
 }
 
+// ---------------------------------------------- S7 on the 5th-generation tensor cores
+// The step's residual pass with the rank-k product on tcgen05 (kind::tf32) and the
+// block held in tensor memory, one thread per row. Per 128 x 128 grid block:
+//   * TMA brings the block's P rows and R rows as tf32 hi / lo pairs (pre-split by
+//     the kernels that produce P and R; the k <= 32 factor columns zero-padded to
+//     32, one 128-byte swizzled row each: the K-major operand layout);
+//   * one thread issues the 3xTF32 product D = P_hi R_hi^T + P_hi R_lo^T +
+//     P_lo R_hi^T (M = N = 128, K = 8 per instruction) into 128 TMEM columns;
+//   * warp w owns the TMEM lanes (rows) 32 (w & 3) .. + 31 and the 64 columns of
+//     half w >> 2: it reads D in 16-column chunks, forms x = M - D from its rows of
+//     M (fp32 loads, one 64-byte row segment per chunk), keeps the row maxima in
+//     the thread, reduces the column maxima over its 32 rows with redux.sync and
+//     writes x back into TMEM; the two halves of a row and the four row quarters
+//     of a column meet in shared memory;
+//   * a second sweep over TMEM turns x into codes q = rint(fp32(x / s) * 7), s =
+//     min(row max, column max), with the same fl(7 / s) shortcut and IEEE fallback
+//     as k_residual_quant4, and stores each thread's 8 code bytes per chunk.
+// The 8-bit factor codes, scales and step count are written as in k_residual_quant4.
+// Every mbarrier wait is bounded; a wait that runs out records GM_E_TIMEOUT in
+// `status` and the CTA skips its outputs, always releasing its tensor memory.
+constexpr int kTcThreads = 256;
+constexpr int kTcTmemCols = 128;
+constexpr uint32_t kTcTileBytes = 128 * 32 * 4;               // 128 rows x 32 fp32
+constexpr uint32_t kTcSmemBytes = 4 * kTcTileBytes + 1024;    // P hi, lo, R hi, lo + alignment
+
+struct ResidualTcMaps {
+  CUtensorMap P, Plo, R, Rlo;   // [B][rows][32] fp32, {32, 128, 1} boxes, 128-byte swizzle
+};
+
+__device__ __forceinline__ uint32_t tc_smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ bool tc_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait on phase `parity` of an mbarrier: false after ~2 s.
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity) {
+  if (tc_try_wait(bar, parity)) return true;
+  uint64_t t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (uint32_t it = 1;; ++it) {
+    if (tc_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      uint64_t t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (t - t0 > 2000000000ull) return false;
+    }
+  }
+}
+// UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t tc_sdesc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor, kind::tf32: D f32, A and B tf32, both K-major, M = N = 128.
+constexpr uint32_t kTcIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kTcThreads, 3) k_residual_tc(
+    const __grid_constant__ ResidualTcMaps maps, int m, int n, int k,
+    const float* __restrict__ X, const float* __restrict__ P, const float* __restrict__ R,
+    uint8_t* __restrict__ codes4, float* __restrict__ rscale, float* __restrict__ cscale,
+    Quant8Out q8, const int32_t* skip, int32_t* status) {
+  if (skip && *skip) return;
+  const int bj = blockIdx.x, bi = blockIdx.y, b = blockIdx.z;
+  const int nb = gridDim.x, mb = gridDim.y;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int quarter = warp & 3, half = warp >> 2;
+  const int rl = 32 * quarter + lane;                 // this thread's row of the block
+  const int r0 = bi * kGrid, c0 = bj * kGrid, gi = r0 + rl;
+  const int cbase = c0 + 64 * half;                   // first column of this thread's half
+  const bool row_ok = gi < m;
+  extern __shared__ __align__(1024) uint8_t tsm[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bars[2];           // operands landed, product done
+  __shared__ uint32_t tmem_slot;
+  __shared__ int bad;
+  __shared__ float RMX[2][kGrid];                     // row maxima of the two column halves
+  __shared__ uint32_t CMX[4][kGrid];                  // column maxima of the four row quarters
+  __shared__ float smax_c[kGrid], r7c[kGrid];
+  const uint32_t bar_ld = tc_smem_u32(&bars[0]), bar_mma = tc_smem_u32(&bars[1]);
+
+  if (t == 0) {
+    bad = 0;
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_ld) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    const uint32_t dst = tc_smem_u32(tiles);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_ld),
+                 "r"(4 * kTcTileBytes)
+                 : "memory");
+    const CUtensorMap* mp[4] = {&maps.P, &maps.Plo, &maps.R, &maps.Rlo};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int row = q < 2 ? r0 : c0;
+      asm volatile(
+          "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+          " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst + q * kTcTileBytes),
+          "l"(reinterpret_cast<uint64_t>(mp[q])), "r"(bar_ld), "r"(0), "r"(row), "r"(b)
+          : "memory");
+    }
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     tc_smem_u32(&tmem_slot)),
+                 "r"(kTcTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = tmem_slot;
+  const uint32_t tbase = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(64 * half);
+
+  // this thread's M row segment of the first chunk, in flight while the product runs
+  const float* Mrow = X + ((long long)b * m + gi) * n;
+  float4 mnext[4];
+  auto load_m = [&](int ch, float4 (&dst)[4]) {
+    const int c = cbase + 16 * ch;    // n % 16 == 0: a 16-column run is all in or all out
+    const bool ok = row_ok && c < n;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      dst[u] = ok ? reinterpret_cast<const float4*>(Mrow + c)[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  load_m(0, mnext);
+
+  if (t == 0) {
+    if (!tc_wait(bar_ld, 0)) {
+      bad = 1;
+    } else {
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t sP = tc_smem_u32(tiles), sPlo = sP + kTcTileBytes;
+      const uint32_t sR = sP + 2 * kTcTileBytes, sRlo = sP + 3 * kTcTileBytes;
+      const uint32_t as[3] = {sP, sP, sPlo}, bs[3] = {sR, sRlo, sR};
+#pragma unroll
+      for (int term = 0; term < 3; ++term)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {   // K = 8 tf32 = 32 bytes per instruction
+          const uint64_t ad = tc_sdesc(as[term] + 32 * kk), bd = tc_sdesc(bs[term] + 32 * kk);
+          const uint32_t acc = (term | kk) ? 1u : 0u;
+          asm volatile(
+              "{\n\t.reg .pred p;\n\t"
+              "setp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+              "l"(ad), "l"(bd), "r"(kTcIdesc), "r"(acc)
+              : "memory");
+        }
+    }
+    // arrives once every MMA issued above has completed (at once when none was)
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar_mma)
+                 : "memory");
+  }
+  bool ok = tc_wait(bar_mma, 0);
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  __syncthreads();
+  ok = ok && !bad;
+
+  float rmax = 0.f;
+  if (ok) {
+    // sweep 1: x = M - P R^T, row and column maxima, x back into TMEM
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+      __syncwarp();                       // TMEM loads, stores and redux are warp collectives
+      float4 mv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) mv[u] = mnext[u];
+      if (ch + 1 < 4) load_m(ch + 1, mnext);
+      float x[16];
+      tc_ld16(tbase + 16 * ch, x);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        x[4 * u] = __fsub_rn(mv[u].x, x[4 * u]);
+        x[4 * u + 1] = __fsub_rn(mv[u].y, x[4 * u + 1]);
+        x[4 * u + 2] = __fsub_rn(mv[u].z, x[4 * u + 2]);
+        x[4 * u + 3] = __fsub_rn(mv[u].w, x[4 * u + 3]);
+      }
+      if (!row_ok || cbase + 16 * ch >= n) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e] = 0.f;   // rows and columns outside the matrix
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const uint32_t a = __float_as_uint(fabsf(x[e]));
+        rmax = fmaxf(rmax, fabsf(x[e]));
+        uint32_t cm;
+        asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(cm) : "r"(a));
+        if (lane == e) CMX[quarter][64 * half + 16 * ch + e] = cm;
+      }
+      tc_st16(tbase + 16 * ch, x);
+    }
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    RMX[half][rl] = rmax;
+  }
+  __syncthreads();
+  if (ok && t < kGrid) {
+    const uint32_t v = max(max(CMX[0][t], CMX[1][t]), max(CMX[2][t], CMX[3][t]));
+    const float f = __uint_as_float(v);
+    smax_c[t] = f;
+    r7c[t] = f > 0.f ? __fdiv_rn(7.0f, f) : 0.f;
+    if (c0 + t < n) cscale[((long long)b * mb + bi) * n + c0 + t] = f;
+  }
+  __syncthreads();
+  if (ok) {
+    rmax = fmaxf(RMX[0][rl], RMX[1][rl]);
+    if (half == 0 && row_ok) rscale[((long long)b * m + gi) * nb + bj] = rmax;
+    const float rr7 = rmax > 0.f ? __fdiv_rn(7.0f, rmax) : 0.f;
+    // sweep 2: the codes
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+      const int c = cbase + 16 * ch;
+      float x[16];
+      __syncwarp();                       // the TMEM load is a collective of the whole warp
+      tc_ld16(tbase + 16 * ch, x);
+      if (!row_ok || c >= n) continue;    // rows (and 16-column runs) outside the matrix
+      uint32_t w[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int cl = 64 * half + 16 * ch + e;
+        const float z = __fmul_rn(x[e], fmaxf(rr7, r7c[cl]));
+        const float zr = rintf(z);
+        int q;
+        if (fabsf(__fsub_rn(z, zr)) < 0.49998474f) {   // 0.5 - 2^-16
+          q = (int)zr;
+        } else {
+          const float sv = fminf(rmax, smax_c[cl]);
+          q = sv > 0.f ? (int)rintf(__fmul_rn(__fdiv_rn(x[e], sv), 7.0f)) : 0;
+        }
+        q = max(-7, min(7, q));
+        w[e >> 3] |= (uint32_t)(q & 0xF) << (4 * (e & 7));
+      }
+      *reinterpret_cast<uint2*>(codes4 + ((long long)b * m + gi) * (n / 2) + c / 2) = make_uint2(w[0], w[1]);
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols)
+                 : "memory");
+  if (!ok) {
+    if (t == 0 && status) atomicExch(status, (int32_t)GM_E_TIMEOUT);
+    return;
+  }
+  // 8-bit codes of P (block column 0) and R (block row 0), scales, step count
+  const int nrows = min(kGrid, m - r0), ncols = min(kGrid, n - c0);
+  if (q8.Pmax && (bj == 0 || bi == 0)) {
+    for (int which = 0; which < 2; ++which) {
+      const bool doit = which == 0 ? bj == 0 : bi == 0;
+      if (!doit) continue;
+      const unsigned* mx = which == 0 ? q8.Pmax : q8.Rmax;
+      const float* src = which == 0 ? P + ((long long)b * m + r0) * k : R + ((long long)b * n + c0) * k;
+      int8_t* dst = which == 0 ? q8.P8 + ((long long)b * m + r0) * k : q8.R8 + ((long long)b * n + c0) * k;
+      const int cnt = (which == 0 ? nrows : ncols) * k;
+      for (int e = t; e < cnt; e += kTcThreads) {
+        const int l = e % k;
+        const float sv = __uint_as_float(mx[b * k + l]);
+        const float r127 = sv > 0.f ? __fdiv_rn(127.0f, sv) : 0.f;
+        dst[e] = code8(src[e], sv, r127);
+      }
+    }
+    if (bi == 0 && bj == 0 && t < k) {
+      q8.Pscale[b * k + t] = __uint_as_float(q8.Pmax[b * k + t]);
+      q8.Rscale[b * k + t] = __uint_as_float(q8.Rmax[b * k + t]);
+    }
+  }
+  if (q8.step && b == 0 && bi == 0 && bj == 0 && t == 0) *q8.step += 1;
+}
+
 // ------------------------------------------------------------------ S6
 // blockIdx.x selects the matrix (0: X0 with rows0 rows, 1: X1), blockIdx.y the batch,
 // blockIdx.z a share of the rows. Every block reduces the column absmax over all
@@ -1577,8 +1919,8 @@ __global__ void __launch_bounds__(kThreads) k_cast_wide(int m, int n, const void
 template <int KP>
 cudaError_t launch_backproject_t(int B, int m, int n, int k, const float* M, const uint32_t* PB,
                                  const float* scale, void* X16, bool f16, double* Rpart,
-                                 float* R, uint32_t* RB, unsigned* Rmax, const int32_t* skip,
-                                 cudaStream_t s) {
+                                 float* R, uint32_t* RB, float* RT, unsigned* Rmax,
+                                 const int32_t* skip, cudaStream_t s) {
   const int rs = backproject_row_splits(B, m, n);
   const size_t smem = (size_t)2 * 8 * 8 * 32 * sizeof(float4);
   static DeviceOnce attr;
@@ -1593,7 +1935,7 @@ cudaError_t launch_backproject_t(int B, int m, int n, int k, const float* M, con
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g2((int)cdivll((long long)cdiv(n, 64) * 64 * KP, kThreads), B);
-  k_finalize_r<<<g2, kThreads, 0, s>>>(n, k, rs, Rpart, R, RB, Rmax, skip);
+  k_finalize_r<<<g2, kThreads, 0, s>>>(n, k, rs, Rpart, R, RB, RT, Rmax, skip);
   return cudaGetLastError();
 }
 
@@ -1734,7 +2076,7 @@ cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4, co
 
 cudaError_t launch_orth(int B, int m, int k, int csplit, const float* Ppart, double* Ptil,
                         double* gram_part, double* Lmat, const double* norm2_part, int ntiles,
-                        float eps, float* scale, float* P, uint32_t* PB, uint32_t* PA,
+                        float eps, float* scale, float* P, uint32_t* PB, uint32_t* PA, float* PT,
                         unsigned* Pmax, const int32_t* skip, cudaStream_t s) {
   const int rs = gram_row_splits(B, m);
   k_orth_gram<<<dim3(rs, B), kThreads, 0, s>>>(m, k, csplit, rs, Ppart, Ptil, gram_part, skip);
@@ -1745,19 +2087,20 @@ cudaError_t launch_orth(int B, int m, int k, int csplit, const float* Ppart, dou
   if (e != cudaSuccess) return e;
   const int kp = factor_width(k);
   const dim3 grid(cdiv(m, kThreads), B);
-  if (kp == 8) k_orth_apply<8><<<grid, kThreads, 0, s>>>(m, k, Ptil, Lmat, P, PB, PA, Pmax, skip);
-  else if (kp == 16) k_orth_apply<16><<<grid, kThreads, 0, s>>>(m, k, Ptil, Lmat, P, PB, PA, Pmax, skip);
-  else k_orth_apply<32><<<grid, kThreads, 0, s>>>(m, k, Ptil, Lmat, P, PB, PA, Pmax, skip);
+  if (kp == 8) k_orth_apply<8><<<grid, kThreads, 0, s>>>(m, k, Ptil, Lmat, P, PB, PA, PT, Pmax, skip);
+  else if (kp == 16) k_orth_apply<16><<<grid, kThreads, 0, s>>>(m, k, Ptil, Lmat, P, PB, PA, PT, Pmax, skip);
+  else k_orth_apply<32><<<grid, kThreads, 0, s>>>(m, k, Ptil, Lmat, P, PB, PA, PT, Pmax, skip);
   return cudaGetLastError();
 }
 
 cudaError_t launch_backproject(int B, int m, int n, int k, const float* M, const uint32_t* PB,
                                const float* scale, void* X16, bool f16, double* Rpart, float* R,
-                               uint32_t* RB, unsigned* Rmax, const int32_t* skip, cudaStream_t s) {
+                               uint32_t* RB, float* RT, unsigned* Rmax, const int32_t* skip,
+                               cudaStream_t s) {
   const int kp = factor_width(k);
-  if (kp == 8) return launch_backproject_t<8>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, Rmax, skip, s);
-  if (kp == 16) return launch_backproject_t<16>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, Rmax, skip, s);
-  return launch_backproject_t<32>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, Rmax, skip, s);
+  if (kp == 8) return launch_backproject_t<8>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, RT, Rmax, skip, s);
+  if (kp == 16) return launch_backproject_t<16>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, RT, Rmax, skip, s);
+  return launch_backproject_t<32>(B, m, n, k, M, PB, scale, X16, f16, Rpart, R, RB, RT, Rmax, skip, s);
 }
 
 cudaError_t launch_residual_quant4(int B, int m, int n, int k, const float* X, const float* P,
@@ -1779,12 +2122,51 @@ cudaError_t launch_residual_quant4(int B, int m, int n, int k, const float* X, c
 
 cudaError_t launch_codes_frags(int B, int m, int n, int k, const float* P, const float* R,
                                const unsigned* Pmax, const unsigned* Rmax, uint32_t* PA,
-                               uint32_t* RB, const int32_t* skip, cudaStream_t s) {
+                               uint32_t* RB, float* PT, float* RT, const int32_t* skip,
+                               cudaStream_t s) {
   const dim3 grid((unsigned)cdivll((long long)(m + n) * k, kThreads), B);
   const int kp = factor_width(k);
-  if (kp == 8) k_codes_frags<8><<<grid, kThreads, 0, s>>>(m, n, k, P, R, Pmax, Rmax, PA, RB, skip);
-  else if (kp == 16) k_codes_frags<16><<<grid, kThreads, 0, s>>>(m, n, k, P, R, Pmax, Rmax, PA, RB, skip);
-  else k_codes_frags<32><<<grid, kThreads, 0, s>>>(m, n, k, P, R, Pmax, Rmax, PA, RB, skip);
+  if (kp == 8) k_codes_frags<8><<<grid, kThreads, 0, s>>>(m, n, k, P, R, Pmax, Rmax, PA, RB, PT, RT, skip);
+  else if (kp == 16) k_codes_frags<16><<<grid, kThreads, 0, s>>>(m, n, k, P, R, Pmax, Rmax, PA, RB, PT, RT, skip);
+  else k_codes_frags<32><<<grid, kThreads, 0, s>>>(m, n, k, P, R, Pmax, Rmax, PA, RB, PT, RT, skip);
+  return cudaGetLastError();
+}
+
+// Tensor maps of the residual operand rows ([2][B][rows][32] fp32: hi then lo).
+static bool tc_operand_maps(CUtensorMap* hi, CUtensorMap* lo, const float* base, int B, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {32, (cuuint64_t)rows, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {32 * 4, (cuuint64_t)rows * 32 * 4};
+  const cuuint32_t box[3] = {32, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  for (int h = 0; h < 2; ++h) {
+    void* p = const_cast<float*>(base + (size_t)h * B * rows * 32);
+    const CUresult r = fn(h ? lo : hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p, dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+  }
+  return true;
+}
+
+cudaError_t launch_residual_tc(int B, int m, int n, int k, const float* X, const float* P,
+                               const float* R, const float* PT, const float* RT, uint8_t* codes4,
+                               float* rscale, float* cscale, const unsigned* PRmax, int8_t* P8,
+                               float* Pscale, int8_t* R8, float* Rscale, int64_t* step,
+                               const int32_t* skip, int32_t* status, cudaStream_t s) {
+  ResidualTcMaps maps;
+  if (!tc_operand_maps(&maps.P, &maps.Plo, PT, B, m) || !tc_operand_maps(&maps.R, &maps.Rlo, RT, B, n))
+    return cudaErrorInvalidValue;
+  static DeviceOnce attr;
+  {
+    const cudaError_t e = smem_attr_once(attr, k_residual_tc, kTcSmemBytes);
+    if (e != cudaSuccess) return e;
+  }
+  const Quant8Out q8{PRmax, PRmax ? PRmax + (size_t)B * k : nullptr, P8, Pscale, R8, Rscale, step};
+  dim3 grid(cdiv(n, kGrid), cdiv(m, kGrid), B);
+  k_residual_tc<<<grid, kTcThreads, kTcSmemBytes, s>>>(maps, m, n, k, X, P, R, codes4, rscale, cscale,
+                                                       q8, skip, status);
   return cudaGetLastError();
 }
 

@@ -841,6 +841,8 @@ __global__ void k_pad16(int B, int rows, int cols, int prow, int pcol, const uin
 }
 
 // ------------------------------------------------------------------ host side
+}  // namespace
+
 // The driver's tensor-map encoder (one function for every device of the process).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
@@ -857,6 +859,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   }
   return f;
 }
+
+namespace {
 
 // Map over 16-bit elements with the 128-byte swizzle (innermost box extent 64).
 bool encode(CUtensorMap* map, const void* base, bool f16, int rank, const cuuint64_t* dims,

@@ -4,7 +4,12 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cudaTypedefs.h>
+
 namespace gm {
+
+// The driver's cuTensorMapEncodeTiled (NULL if the driver does not provide it).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
 
 // Column / row split counts of the power-iteration reductions. They depend
 // only on the problem shape, so the workspace layout is a pure function of it.
@@ -53,18 +58,29 @@ cudaError_t launch_rebuild(int B, int m, int n, int k, const uint8_t* codes4,
                            double* norm2_part, float* Ppart, int32_t* status, cudaStream_t s);
 
 // P = orth(P~) (fp32 [B][m][k]) with its fragments PB (back-projection) and PA
-// (residual, nullable).
+// (residual, nullable) and the tensor-core residual's operand rows PT (nullable:
+// [2][B][m][32] fp32, tf32 hi then lo, columns beyond k zero).
 // Pmax (nullable): the column absolute maxima of P (fp32 bits, atomicMax into zeroed words).
 cudaError_t launch_orth(int B, int m, int k, int csplit, const float* Ppart, double* Ptil,
                         double* gram_part, double* Lmat, const double* norm2_part, int ntiles,
-                        float eps, float* scale, float* P, uint32_t* PB, uint32_t* PA,
+                        float eps, float* scale, float* P, uint32_t* PB, uint32_t* PA, float* PT,
                         unsigned* Pmax, const int32_t* skip, cudaStream_t s);
 
-// R = M^T P from PB, with its residual fragments RB (nullable).
+// R = M^T P from PB, with its residual fragments RB (nullable) and operand rows RT
+// (nullable, [2][B][n][32] as PT).
 cudaError_t launch_backproject(int B, int m, int n, int k, const float* M, const uint32_t* PB,
                                const float* scale, void* X16, bool f16, double* Rpart,
-                               float* R, uint32_t* RB, unsigned* Rmax, const int32_t* skip,
-                               cudaStream_t s);
+                               float* R, uint32_t* RB, float* RT, unsigned* Rmax,
+                               const int32_t* skip, cudaStream_t s);
+
+// The step's residual pass on the tensor cores (tcgen05, kind::tf32): the same
+// outputs as launch_residual_quant4 with ready-made operand rows PT, RT; status
+// gets GM_E_TIMEOUT when a bounded wait runs out.
+cudaError_t launch_residual_tc(int B, int m, int n, int k, const float* X, const float* P,
+                               const float* R, const float* PT, const float* RT, uint8_t* codes4,
+                               float* rscale, float* cscale, const unsigned* PRmax, int8_t* P8,
+                               float* Pscale, int8_t* R8, float* Rscale, int64_t* step,
+                               const int32_t* skip, int32_t* status, cudaStream_t s);
 
 // PA, RB: ready-made fragments of -P and R (both or neither; NULL stages P, R).
 // PRmax (nullable): the P then R column maxima; with it the kernel also writes the
@@ -80,7 +96,8 @@ cudaError_t launch_residual_quant4(int B, int m, int n, int k, const float* X, c
 // (Pmax, Rmax: their complete column absolute maxima).
 cudaError_t launch_codes_frags(int B, int m, int n, int k, const float* P, const float* R,
                                const unsigned* Pmax, const unsigned* Rmax, uint32_t* PA,
-                               uint32_t* RB, const int32_t* skip, cudaStream_t s);
+                               uint32_t* RB, float* PT, float* RT, const int32_t* skip,
+                               cudaStream_t s);
 
 cudaError_t launch_quant8(int B, int rows0, int rows1, int k, const float* X0, int8_t* c0,
                           float* s0, const float* X1, int8_t* c1, float* s1,
