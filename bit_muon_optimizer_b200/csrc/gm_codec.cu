@@ -958,19 +958,23 @@ __global__ void __launch_bounds__(kThreads) k_orth_apply(int m, int k, const dou
       PA[at] = hi;
       PA[at + 128] = tf32_lo(-f, hi);
     }
-    if (PT) {
-      const long long at = ((long long)b * m + i) * 32 + l;
-      const uint32_t hi = tf32_hi(f);
-      PT[at] = __uint_as_float(hi);
-      PT[(long long)gridDim.y * m * 32 + at] = __uint_as_float(tf32_lo(f, hi));
-    }
   }
-  if (PT && in) {   // the operand tiles' columns beyond the factor width are zero
+  if (PT && in) {   // the operand row, 16-byte stores; columns beyond KP are zero
+    float4* hi4 = reinterpret_cast<float4*>(PT + ((long long)b * m + i) * 32);
+    float4* lo4 = reinterpret_cast<float4*>(PT + (long long)gridDim.y * m * 32 + ((long long)b * m + i) * 32);
 #pragma unroll
-    for (int l = KP; l < 32; ++l) {
-      const long long at = ((long long)b * m + i) * 32 + l;
-      PT[at] = 0.f;
-      PT[(long long)gridDim.y * m * 32 + at] = 0.f;
+    for (int q = 0; q < 8; ++q) {
+      float h[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int l = 4 * q + e;
+        const float f = l < KP ? (float)row[l < KP ? l : 0] : 0.f;   // 0 beyond k (row is 0 there)
+        const uint32_t hb = tf32_hi(f);
+        h[e] = __uint_as_float(hb);
+        lo[e] = __uint_as_float(tf32_lo(f, hb));
+      }
+      hi4[q] = make_float4(h[0], h[1], h[2], h[3]);
+      lo4[q] = make_float4(lo[0], lo[1], lo[2], lo[3]);
     }
   }
   __syncthreads();
