@@ -276,10 +276,11 @@ gm_status gm_momentum_powerit(int B, int m, int n, int k, float mu, const float*
   return GM_OK;
 }
 
-gm_status gm_grid_quant4(int B, int m, int n, int k, const float* X, const float* P,
+gm_status gm_grid_quant4(int B, int m, int n, int block, int k, const float* X, const float* P,
                          const float* R, uint8_t* codes4, float* rscale, float* cscale,
                          gm_stream_t stream) {
   GM_CHECK_ARG(shape_ok(B, m, n), "bad shape B=%d m=%d n=%d", B, m, n);
+  GM_CHECK_ARG(block == kGrid, "block=%d: only %d x %d grid blocks are built", block, kGrid, kGrid);
   GM_CHECK_ARG(X && codes4 && rscale && cscale, "NULL input or output pointer");
   GM_CHECK_ARG((P == nullptr) == (R == nullptr), "P and R must both be NULL or both set");
   GM_CHECK_ARG(!P || (k >= 1 && k <= kMaxK), "k=%d out of [1, %d]", k, kMaxK);
@@ -424,6 +425,8 @@ static gm_status step_checks(int B, int m, int n, const gm_grasp_params* prm, co
   GM_CHECK_ARG(prm->residual_from_codes == 0 || prm->residual_from_codes == 1,
                "residual_from_codes must be 0 or 1");
   GM_CHECK_ARG(al16(prm->matrix_ids), "matrix_ids must be 16-byte aligned");
+  GM_CHECK_ARG(prm->block == 0 || prm->block == kGrid, "block=%d: only %d x %d grid blocks are built",
+               prm->block, kGrid, kGrid);
   GM_CHECK_ARG(st->codes4 && st->rscale && st->cscale && st->P8 && st->Pscale && st->R8 &&
                    st->Rscale && st->step && st->dev_status,
                "NULL state pointer");
@@ -510,7 +513,7 @@ gm_status gm_grasp_state_update(int B, int m, int n, const gm_grasp_params* prm,
                                s));
   // worked step 5: residual -> 4-bit grid codes (tensor cores); P, R -> 8-bit codes
   // (state in place)
-  GM_CUDA(launch_residual_tc(B, m, n, k, M, P, R, PT, RT, st->codes4, st->rscale, st->cscale, PRmax,
+  GM_CUDA(launch_residual_ws(B, m, n, k, M, P, R, PT, RT, st->codes4, st->rscale, st->cscale, PRmax,
                              st->P8, st->Pscale, st->R8, st->Rscale, st->step, status, status, s));
   return GM_OK;
 }

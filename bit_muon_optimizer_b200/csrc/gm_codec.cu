@@ -1514,33 +1514,37 @@ __global__ void __launch_bounds__(kRT, 2) k_residual_quant4(
 }
 
 // ---------------------------------------------- S7 on the 5th-generation tensor cores
-// The step's residual pass with the rank-k product on tcgen05 (kind::tf32) and the
-// block held in tensor memory, one thread per row. Per 128 x 128 grid block:
-//   * TMA brings the block's P rows and R rows as tf32 hi / lo pairs (pre-split by
-//     the kernels that produce P and R; the k <= 32 factor columns zero-padded to
-//     32, one 128-byte swizzled row each: the K-major operand layout);
-//   * one thread issues the 3xTF32 product D = P_hi R_hi^T + P_hi R_lo^T +
-//     P_lo R_hi^T (M = N = 128, K = 8 per instruction) into 128 TMEM columns;
-//   * warp w owns the TMEM lanes (rows) 32 (w & 3) .. + 31 and the 64 columns of
-//     half w >> 2: it reads D in 16-column chunks, forms x = M - D from its rows of
-//     M (fp32 loads, one 64-byte row segment per chunk), keeps the row maxima in
-//     the thread, reduces the column maxima over its 32 rows with redux.sync and
-//     writes x back into TMEM; the two halves of a row and the four row quarters
-//     of a column meet in shared memory;
-//   * a second sweep over TMEM turns x into codes q = rint(fp32(x / s) * 7), s =
-//     min(row max, column max), with the same fl(7 / s) shortcut and IEEE fallback
-//     as k_residual_quant4, and stores each thread's 8 code bytes per chunk.
-// The 8-bit factor codes, scales and step count are written as in k_residual_quant4.
-// Every mbarrier wait is bounded; a wait that runs out records GM_E_TIMEOUT in
-// `status` and the CTA skips its outputs, always releasing its tensor memory.
-constexpr int kTcThreads = 256;
-constexpr int kTcTmemCols = 128;
-constexpr uint32_t kTcTileBytes = 128 * 32 * 4;               // 128 rows x 32 fp32
-constexpr uint32_t kTcSmemBytes = 4 * kTcTileBytes + 1024;    // P hi, lo, R hi, lo + alignment
-
-struct ResidualTcMaps {
-  CUtensorMap P, Plo, R, Rlo;   // [B][rows][32] fp32, {32, 128, 1} boxes, 128-byte swizzle
-};
+// The step's residual pass, one persistent CTA per SM walking a contiguous run of
+// 128 x 128 grid blocks (batch, block row, block column; columns fastest), with the
+// rank-k product on tcgen05 (kind::tf32) and the block held in tensor memory:
+//   warp 0      : TMA producer: the block's M tile (four 128 x 32 fp32 boxes,
+//                 128-byte swizzle) into a two-stage ring; the block's R operand
+//                 rows and, when the block row changes, its P rows, as tf32 hi / lo
+//                 pairs (pre-split by the kernels that produce P and R; the k <= 32
+//                 factor columns zero-padded to 32, one 128-byte swizzled row each:
+//                 the K-major operand layout);
+//   warp 1      : allocates 256 TMEM columns; lane 0 issues the 3xTF32 product
+//                 D = P_hi R_hi^T + P_hi R_lo^T + P_lo R_hi^T (M = N = 128, K = 8 per
+//                 instruction) into one of two 128-column accumulators;
+//   warps 2..17 : the block sweeps, while the next block's M streams in and its
+//                 product runs. Warp w owns the TMEM lanes (rows) 32 (w & 3) .. + 31
+//                 and a 32-column group of the block: it reads D in 16-column chunks,
+//                 forms x = M - D from its rows of the swizzled M stage, keeps the row
+//                 maxima in the thread, reduces the column maxima over its 32 rows
+//                 with redux.sync and writes x back into TMEM; the column groups of a
+//                 row and the four row quarters of a column meet in shared memory. A
+//                 second sweep over TMEM turns x into codes q = rint(fp32(x / s) * 7),
+//                 s = min(row max, column max), with the same fl(7 / s) shortcut and
+//                 IEEE fallback as k_residual_quant4, and stores each thread's 8 code
+//                 bytes per chunk. The 8-bit factor codes, scales and step count are
+//                 written as in k_residual_quant4.
+// Operand tiles are single-buffered: the next block's R (and P) rows load as soon as
+// the product that read them has completed. Every wait is bounded (~2 s of
+// %globaltimer) and gives up at once when another role has aborted; a timeout records
+// GM_E_TIMEOUT in `status`, every role leaves its loop, the producer and the MMA
+// issuer wait (bounded) for their copies and products still in flight, and the
+// tensor memory is freed.
+constexpr int kTcTmemCols = 128;   // one accumulator: 128 lanes x 128 fp32 columns
 
 __device__ __forceinline__ uint32_t tc_smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -1555,20 +1559,6 @@ __device__ __forceinline__ bool tc_try_wait(uint32_t bar, uint32_t parity) {
       : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
-}
-// Bounded wait on phase `parity` of an mbarrier: false after ~2 s.
-__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity) {
-  if (tc_try_wait(bar, parity)) return true;
-  uint64_t t0;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-  for (uint32_t it = 1;; ++it) {
-    if (tc_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      uint64_t t;
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-      if (t - t0 > 2000000000ull) return false;
-    }
-  }
 }
 // UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
 __device__ __forceinline__ uint64_t tc_sdesc(uint32_t saddr) {
@@ -1604,55 +1594,113 @@ __device__ __forceinline__ void tc_st16(uint32_t taddr, const float (&v)[16]) {
       : "memory");
 }
 
-__global__ void __launch_bounds__(kTcThreads, 3) k_residual_tc(
-    const __grid_constant__ ResidualTcMaps maps, int m, int n, int k,
-    const float* __restrict__ X, const float* __restrict__ P, const float* __restrict__ R,
-    uint8_t* __restrict__ codes4, float* __restrict__ rscale, float* __restrict__ cscale,
-    Quant8Out q8, const int32_t* skip, int32_t* status) {
-  if (skip && *skip) return;
-  const int bj = blockIdx.x, bi = blockIdx.y, b = blockIdx.z;
-  const int nb = gridDim.x, mb = gridDim.y;
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int quarter = warp & 3, half = warp >> 2;
-  const int rl = 32 * quarter + lane;                 // this thread's row of the block
-  const int r0 = bi * kGrid, c0 = bj * kGrid, gi = r0 + rl;
-  const int cbase = c0 + 64 * half;                   // first column of this thread's half
-  const bool row_ok = gi < m;
-  extern __shared__ __align__(1024) uint8_t tsm[];
-  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bars[2];           // operands landed, product done
-  __shared__ uint32_t tmem_slot;
-  __shared__ int bad;
-  __shared__ float RMX[2][kGrid];                     // row maxima of the two column halves
-  __shared__ uint32_t CMX[4][kGrid];                  // column maxima of the four row quarters
-  __shared__ float smax_c[kGrid], r7c[kGrid];
-  const uint32_t bar_ld = tc_smem_u32(&bars[0]), bar_mma = tc_smem_u32(&bars[1]);
+constexpr int kWsEpiWarps = 16;
+constexpr int kWsColGroups = kWsEpiWarps / 4;          // column groups of a block
+constexpr int kWsCols = kGrid / kWsColGroups;          // columns per epilogue warp
+constexpr int kWsChunks = kWsCols / 16;
+constexpr int kWsThreads = (2 + kWsEpiWarps) * 32;
+constexpr uint32_t kWsTile = 128 * 32 * 4;                        // one 128 x 32 fp32 box
+constexpr uint32_t kWsOps = 4 * kWsTile;                          // P hi, lo, R hi, lo
+constexpr uint32_t kWsStage = 4 * kWsTile;                        // M: four boxes
+constexpr uint32_t kWsSmemBytes = kWsOps + 2 * kWsStage + 1024;   // + alignment
 
-  if (t == 0) {
-    bad = 0;
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_ld) : "memory");
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    const uint32_t dst = tc_smem_u32(tiles);
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_ld),
-                 "r"(4 * kTcTileBytes)
-                 : "memory");
-    const CUtensorMap* mp[4] = {&maps.P, &maps.Plo, &maps.R, &maps.Rlo};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int row = q < 2 ? r0 : c0;
-      asm volatile(
-          "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-          " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst + q * kTcTileBytes),
-          "l"(reinterpret_cast<uint64_t>(mp[q])), "r"(bar_ld), "r"(0), "r"(row), "r"(b)
-          : "memory");
+struct ResidualWsMaps {
+  CUtensorMap P, Plo, R, Rlo;   // [B][rows][32] fp32 operand rows, {32, 128, 1} boxes, 128-byte swizzle
+  CUtensorMap M;                // [B][m][n] fp32, {32, 128, 1} boxes, 128-byte swizzle
+};
+
+__device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (tc_try_wait(bar, parity)) return true;
+  uint64_t t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (uint32_t it = 1;; ++it) {
+    if (tc_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort_flag) return false;
+      uint64_t t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (t - t0 > 2000000000ull) {
+        *abort_flag = 1;
+        return false;
+      }
     }
   }
-  if (warp == 0) {
+}
+__device__ __forceinline__ void ws_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void ws_expect(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void ws_tma3(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                        int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void ws_epi_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kWsEpiWarps * 32) : "memory");
+}
+// true in every epilogue thread when `pred` holds in any of them
+__device__ __forceinline__ bool ws_epi_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 2, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "n"(kWsEpiWarps * 32)
+      : "memory");
+  return r != 0;
+}
+
+__global__ void __launch_bounds__(kWsThreads, 1) k_residual_ws(
+    const __grid_constant__ ResidualWsMaps maps, int m, int n, int k, int nb, int mb, int total,
+    const float* __restrict__ P, const float* __restrict__ R, uint8_t* __restrict__ codes4,
+    float* __restrict__ rscale, float* __restrict__ cscale, Quant8Out q8, const int32_t* skip,
+    int32_t* status) {
+  if (skip && *skip) return;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  // this CTA's contiguous run of blocks (runs differ in length by at most one)
+  const int blk0 = (int)((long long)blockIdx.x * total / gridDim.x);
+  const int blk1 = (int)((long long)(blockIdx.x + 1) * total / gridDim.x);
+  extern __shared__ __align__(1024) uint8_t wsm[];
+  uint8_t* sbase = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(wsm) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bars[10];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_word;
+  __shared__ float RMX[kWsColGroups][kGrid];
+  __shared__ uint32_t CMX[4][kGrid];
+  __shared__ float smax_c[kGrid], r7c[kGrid];
+  volatile int* abort_flag = &abort_word;
+  const uint32_t ops_full = tc_smem_u32(&bars[0]), ops_empty = tc_smem_u32(&bars[1]);
+  auto m_full = [&](int s) { return tc_smem_u32(&bars[2 + s]); };
+  auto m_empty = [&](int s) { return tc_smem_u32(&bars[4 + s]); };
+  auto acc_full = [&](int a) { return tc_smem_u32(&bars[6 + a]); };
+  auto acc_empty = [&](int a) { return tc_smem_u32(&bars[8 + a]); };
+  const uint32_t sP = tc_smem_u32(sbase), sPlo = sP + kWsTile, sR = sP + 2 * kWsTile, sRlo = sP + 3 * kWsTile;
+  auto sM = [&](int s) { return tc_smem_u32(sbase + kWsOps + s * kWsStage); };
+
+  if (t == 0) {
+    abort_word = 0;
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(ops_full) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(ops_empty) : "memory");
+    for (int i = 0; i < 2; ++i) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(m_full(i)) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(m_empty(i)), "r"(kWsEpiWarps) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(acc_full(i)) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(acc_empty(i)), "r"(kWsEpiWarps) : "memory");
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      tc_smem_u32(&tmem_slot)),
-                 "r"(kTcTmemCols)
+                 "r"(2 * kTcTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -1660,160 +1708,218 @@ __global__ void __launch_bounds__(kTcThreads, 3) k_residual_tc(
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = tmem_slot;
-  const uint32_t tbase = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(64 * half);
-
-  // this thread's M row segment of the first chunk, in flight while the product runs
-  const float* Mrow = X + ((long long)b * m + gi) * n;
-  float4 mnext[4];
-  auto load_m = [&](int ch, float4 (&dst)[4]) {
-    const int c = cbase + 16 * ch;    // n % 16 == 0: a 16-column run is all in or all out
-    const bool ok = row_ok && c < n;
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      dst[u] = ok ? reinterpret_cast<const float4*>(Mrow + c)[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+  auto decode = [&](int blk, int& b, int& bi, int& bj) {
+    bj = blk % nb;
+    bi = (blk / nb) % mb;
+    b = blk / (nb * mb);
   };
-  load_m(0, mnext);
 
-  if (t == 0) {
-    if (!tc_wait(bar_ld, 0)) {
-      bad = 1;
-    } else {
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ producer
+      int pb = -1, pbi = -1;
+      int j = 0, last_ops = -1, m_issued = 0;
+      for (int blk = blk0; blk < blk1; ++blk, ++j) {
+        int b, bi, bj;
+        decode(blk, b, bi, bj);
+        const int s = j & 1;
+        if (j >= 2 && !ws_wait(m_empty(s), ((j >> 1) - 1) & 1, abort_flag)) break;
+        ws_expect(m_full(s), kWsStage);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) ws_tma3(sM(s) + q * kWsTile, &maps.M, m_full(s), bj * kGrid + 32 * q, bi * kGrid, b);
+        m_issued = j + 1;
+        if (j >= 1 && !ws_wait(ops_empty, (j - 1) & 1, abort_flag)) break;
+        const bool newrow = b != pb || bi != pbi;
+        ws_expect(ops_full, (newrow ? 4 : 2) * kWsTile);
+        ws_tma3(sR, &maps.R, ops_full, 0, bj * kGrid, b);
+        ws_tma3(sRlo, &maps.Rlo, ops_full, 0, bj * kGrid, b);
+        if (newrow) {
+          ws_tma3(sP, &maps.P, ops_full, 0, bi * kGrid, b);
+          ws_tma3(sPlo, &maps.Plo, ops_full, 0, bi * kGrid, b);
+          pb = b;
+          pbi = bi;
+        }
+        last_ops = j;
+      }
+      // the copies issued last have landed before the CTA may exit (these waits do not
+      // give up on an abort, only on their time limit)
+      volatile int no_abort = 0;
+      for (int jj = max(0, m_issued - 2); jj < m_issued; ++jj) ws_wait(m_full(jj & 1), (jj >> 1) & 1, &no_abort);
+      if (last_ops >= 0) ws_wait(ops_full, last_ops & 1, &no_abort);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      int j = 0, mma_issued = 0;
+      for (int blk = blk0; blk < blk1; ++blk, ++j) {
+        const int a = j & 1;
+        if (j >= 2 && !ws_wait(acc_empty(a), ((j >> 1) - 1) & 1, abort_flag)) break;
+        if (!ws_wait(ops_full, j & 1, abort_flag)) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t d = tmem + (uint32_t)(a * kTcTmemCols);
+        const uint32_t as[3] = {sP, sP, sPlo}, bs[3] = {sR, sRlo, sR};
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = tc_sdesc(as[term] + 32 * kk), bd = tc_sdesc(bs[term] + 32 * kk);
+            const uint32_t acc = (term | kk) ? 1u : 0u;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "setp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+                "l"(ad), "l"(bd), "r"(kTcIdesc), "r"(acc)
+                : "memory");
+          }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         ops_empty)
+                     : "memory");
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         acc_full(a))
+                     : "memory");
+        mma_issued = j + 1;
+      }
+      // every product issued above has completed before the tensor memory is freed
+      volatile int no_abort = 0;
+      if (mma_issued > 0) ws_wait(acc_full((mma_issued - 1) & 1), ((mma_issued - 1) >> 1) & 1, &no_abort);
+    }
+  } else {
+    // -------------------------------------------------- epilogue warps
+    const int ew = warp - 2;
+    const int quarter = warp & 3;          // TMEM lanes 32 (warp % 4) .. + 31
+    const int half = ew >> 2;              // column group of the block
+    const int rl = 32 * quarter + lane;    // this thread's row of the block
+    const int et = ew * 32 + lane;         // 0 .. 255
+    int j = 0;
+    for (int blk = blk0; blk < blk1; ++blk, ++j) {
+      int b, bi, bj;
+      decode(blk, b, bi, bj);
+      const int a = j & 1, s = j & 1;
+      const int r0 = bi * kGrid, c0 = bj * kGrid, gi = r0 + rl;
+      const int cbase = c0 + kWsCols * half;
+      const bool row_ok = gi < m;
+      bool ok = ws_wait(acc_full(a), (j >> 1) & 1, abort_flag);
+      ok = ok && ws_wait(m_full(s), (j >> 1) & 1, abort_flag);
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t sP = tc_smem_u32(tiles), sPlo = sP + kTcTileBytes;
-      const uint32_t sR = sP + 2 * kTcTileBytes, sRlo = sP + 3 * kTcTileBytes;
-      const uint32_t as[3] = {sP, sP, sPlo}, bs[3] = {sR, sRlo, sR};
-#pragma unroll
-      for (int term = 0; term < 3; ++term)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {   // K = 8 tf32 = 32 bytes per instruction
-          const uint64_t ad = tc_sdesc(as[term] + 32 * kk), bd = tc_sdesc(bs[term] + 32 * kk);
-          const uint32_t acc = (term | kk) ? 1u : 0u;
-          asm volatile(
-              "{\n\t.reg .pred p;\n\t"
-              "setp.ne.b32 p, %4, 0;\n\t"
-              "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-              "l"(ad), "l"(bd), "r"(kTcIdesc), "r"(acc)
-              : "memory");
-        }
-    }
-    // arrives once every MMA issued above has completed (at once when none was)
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     bar_mma)
-                 : "memory");
-  }
-  bool ok = tc_wait(bar_mma, 0);
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  __syncthreads();
-  ok = ok && !bad;
-
-  float rmax = 0.f;
-  if (ok) {
-    // sweep 1: x = M - P R^T, row and column maxima, x back into TMEM
+      if (ws_epi_any(!ok)) break;   // leave together: the epilogue warps share named barriers
+      const uint32_t tbase = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(a * kTcTmemCols + kWsCols * half);
+      const uint32_t mrow = sM(s) + (uint32_t)rl * 128u;   // this row in each of the four boxes
+      // sweep 1: x = M - P R^T, row and column maxima, x back into TMEM
+      float rmax = 0.f;
 #pragma unroll 1
-    for (int ch = 0; ch < 4; ++ch) {
-      __syncwarp();                       // TMEM loads, stores and redux are warp collectives
-      float4 mv[4];
+      for (int ch = 0; ch < kWsChunks; ++ch) {
+        __syncwarp();
+        const int cl0 = kWsCols * half + 16 * ch;            // first column (in the block) of the chunk
+        const uint32_t box = mrow + (uint32_t)(cl0 >> 5) * kWsTile;
+        float mv[16];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) mv[u] = mnext[u];
-      if (ch + 1 < 4) load_m(ch + 1, mnext);
-      float x[16];
-      tc_ld16(tbase + 16 * ch, x);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        x[4 * u] = __fsub_rn(mv[u].x, x[4 * u]);
-        x[4 * u + 1] = __fsub_rn(mv[u].y, x[4 * u + 1]);
-        x[4 * u + 2] = __fsub_rn(mv[u].z, x[4 * u + 2]);
-        x[4 * u + 3] = __fsub_rn(mv[u].w, x[4 * u + 3]);
-      }
-      if (!row_ok || cbase + 16 * ch >= n) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) x[e] = 0.f;   // rows and columns outside the matrix
-      }
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const uint32_t a = __float_as_uint(fabsf(x[e]));
-        rmax = fmaxf(rmax, fabsf(x[e]));
-        uint32_t cm;
-        asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(cm) : "r"(a));
-        if (lane == e) CMX[quarter][64 * half + 16 * ch + e] = cm;
-      }
-      tc_st16(tbase + 16 * ch, x);
-    }
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-    RMX[half][rl] = rmax;
-  }
-  __syncthreads();
-  if (ok && t < kGrid) {
-    const uint32_t v = max(max(CMX[0][t], CMX[1][t]), max(CMX[2][t], CMX[3][t]));
-    const float f = __uint_as_float(v);
-    smax_c[t] = f;
-    r7c[t] = f > 0.f ? __fdiv_rn(7.0f, f) : 0.f;
-    if (c0 + t < n) cscale[((long long)b * mb + bi) * n + c0 + t] = f;
-  }
-  __syncthreads();
-  if (ok) {
-    rmax = fmaxf(RMX[0][rl], RMX[1][rl]);
-    if (half == 0 && row_ok) rscale[((long long)b * m + gi) * nb + bj] = rmax;
-    const float rr7 = rmax > 0.f ? __fdiv_rn(7.0f, rmax) : 0.f;
-    // sweep 2: the codes
-#pragma unroll 1
-    for (int ch = 0; ch < 4; ++ch) {
-      const int c = cbase + 16 * ch;
-      float x[16];
-      __syncwarp();                       // the TMEM load is a collective of the whole warp
-      tc_ld16(tbase + 16 * ch, x);
-      if (!row_ok || c >= n) continue;    // rows (and 16-column runs) outside the matrix
-      uint32_t w[2] = {0u, 0u};
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int cl = 64 * half + 16 * ch + e;
-        const float z = __fmul_rn(x[e], fmaxf(rr7, r7c[cl]));
-        const float zr = rintf(z);
-        int q;
-        if (fabsf(__fsub_rn(z, zr)) < 0.49998474f) {   // 0.5 - 2^-16
-          q = (int)zr;
-        } else {
-          const float sv = fminf(rmax, smax_c[cl]);
-          q = sv > 0.f ? (int)rintf(__fmul_rn(__fdiv_rn(x[e], sv), 7.0f)) : 0;
+        for (int pcs = 0; pcs < 4; ++pcs) {             // four 16-byte pieces of the 128-byte row
+          const int piece = ((cl0 & 31) >> 2) + pcs;
+          const uint32_t addr = box + (uint32_t)(((piece ^ (rl & 7)) & 7) << 4);
+          float4 v;
+          asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                       : "r"(addr));
+          mv[4 * pcs] = v.x; mv[4 * pcs + 1] = v.y; mv[4 * pcs + 2] = v.z; mv[4 * pcs + 3] = v.w;
         }
-        q = max(-7, min(7, q));
-        w[e >> 3] |= (uint32_t)(q & 0xF) << (4 * (e & 7));
+        float x[16];
+        tc_ld16(tbase + 16 * ch, x);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e] = __fsub_rn(mv[e], x[e]);
+        if (!row_ok || cbase + 16 * ch >= n) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) x[e] = 0.f;   // rows and columns outside the matrix
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          rmax = fmaxf(rmax, fabsf(x[e]));
+          uint32_t cm;
+          asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(cm) : "r"(__float_as_uint(fabsf(x[e]))));
+          if (lane == e) CMX[quarter][cl0 + e] = cm;
+        }
+        __syncwarp();
+        tc_st16(tbase + 16 * ch, x);
       }
-      *reinterpret_cast<uint2*>(codes4 + ((long long)b * m + gi) * (n / 2) + c / 2) = make_uint2(w[0], w[1]);
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) ws_arrive(m_empty(s));     // this warp is done with the M stage
+      RMX[half][rl] = rmax;
+      ws_epi_bar();
+      if (et < kGrid) {
+        const uint32_t v = max(max(CMX[0][et], CMX[1][et]), max(CMX[2][et], CMX[3][et]));
+        const float f = __uint_as_float(v);
+        smax_c[et] = f;
+        r7c[et] = f > 0.f ? __fdiv_rn(7.0f, f) : 0.f;
+        if (c0 + et < n) cscale[((long long)b * mb + bi) * n + c0 + et] = f;
+      }
+      ws_epi_bar();
+      rmax = RMX[0][rl];
+#pragma unroll
+      for (int h = 1; h < kWsColGroups; ++h) rmax = fmaxf(rmax, RMX[h][rl]);
+      if (half == 0 && row_ok) rscale[((long long)b * m + gi) * nb + bj] = rmax;
+      const float rr7 = rmax > 0.f ? __fdiv_rn(7.0f, rmax) : 0.f;
+      // sweep 2: the codes
+#pragma unroll 1
+      for (int ch = 0; ch < kWsChunks; ++ch) {
+        const int c = cbase + 16 * ch;
+        float x[16];
+        __syncwarp();
+        tc_ld16(tbase + 16 * ch, x);
+        if (row_ok && c < n) {
+          uint32_t w[2] = {0u, 0u};
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int cl = kWsCols * half + 16 * ch + e;
+            const float z = __fmul_rn(x[e], fmaxf(rr7, r7c[cl]));
+            const float zr = rintf(z);
+            int q;
+            if (fabsf(__fsub_rn(z, zr)) < 0.49998474f) {   // 0.5 - 2^-16
+              q = (int)zr;
+            } else {
+              const float sv = fminf(rmax, smax_c[cl]);
+              q = sv > 0.f ? (int)rintf(__fmul_rn(__fdiv_rn(x[e], sv), 7.0f)) : 0;
+            }
+            q = max(-7, min(7, q));
+            w[e >> 3] |= (uint32_t)(q & 0xF) << (4 * (e & 7));
+          }
+          *reinterpret_cast<uint2*>(codes4 + ((long long)b * m + gi) * (n / 2) + c / 2) = make_uint2(w[0], w[1]);
+        }
+      }
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) ws_arrive(acc_empty(a));   // this warp is done with the accumulator
+      // 8-bit codes of P (block column 0) and R (block row 0), scales, step count
+      if (q8.Pmax && (bj == 0 || bi == 0)) {
+        const int nrows = min(kGrid, m - r0), ncols = min(kGrid, n - c0);
+        for (int which = 0; which < 2; ++which) {
+          const bool doit = which == 0 ? bj == 0 : bi == 0;
+          if (!doit) continue;
+          const unsigned* mx = which == 0 ? q8.Pmax : q8.Rmax;
+          const float* src = which == 0 ? P + ((long long)b * m + r0) * k : R + ((long long)b * n + c0) * k;
+          int8_t* dst = which == 0 ? q8.P8 + ((long long)b * m + r0) * k : q8.R8 + ((long long)b * n + c0) * k;
+          const int cnt = (which == 0 ? nrows : ncols) * k;
+          for (int e = et; e < cnt; e += kWsEpiWarps * 32) {
+            const int l = e % k;
+            const float sv = __uint_as_float(mx[b * k + l]);
+            const float r127 = sv > 0.f ? __fdiv_rn(127.0f, sv) : 0.f;
+            dst[e] = code8(src[e], sv, r127);
+          }
+        }
+        if (bi == 0 && bj == 0 && et < k) {
+          q8.Pscale[b * k + et] = __uint_as_float(q8.Pmax[b * k + et]);
+          q8.Rscale[b * k + et] = __uint_as_float(q8.Rmax[b * k + et]);
+        }
+      }
+      if (q8.step && b == 0 && bi == 0 && bj == 0 && et == 0) *q8.step += 1;
+      ws_epi_bar();   // RMX, smax_c and r7c are rewritten by the next block
     }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols)
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kTcTmemCols)
                  : "memory");
-  if (!ok) {
-    if (t == 0 && status) atomicExch(status, (int32_t)GM_E_TIMEOUT);
-    return;
-  }
-  // 8-bit codes of P (block column 0) and R (block row 0), scales, step count
-  const int nrows = min(kGrid, m - r0), ncols = min(kGrid, n - c0);
-  if (q8.Pmax && (bj == 0 || bi == 0)) {
-    for (int which = 0; which < 2; ++which) {
-      const bool doit = which == 0 ? bj == 0 : bi == 0;
-      if (!doit) continue;
-      const unsigned* mx = which == 0 ? q8.Pmax : q8.Rmax;
-      const float* src = which == 0 ? P + ((long long)b * m + r0) * k : R + ((long long)b * n + c0) * k;
-      int8_t* dst = which == 0 ? q8.P8 + ((long long)b * m + r0) * k : q8.R8 + ((long long)b * n + c0) * k;
-      const int cnt = (which == 0 ? nrows : ncols) * k;
-      for (int e = t; e < cnt; e += kTcThreads) {
-        const int l = e % k;
-        const float sv = __uint_as_float(mx[b * k + l]);
-        const float r127 = sv > 0.f ? __fdiv_rn(127.0f, sv) : 0.f;
-        dst[e] = code8(src[e], sv, r127);
-      }
-    }
-    if (bi == 0 && bj == 0 && t < k) {
-      q8.Pscale[b * k + t] = __uint_as_float(q8.Pmax[b * k + t]);
-      q8.Rscale[b * k + t] = __uint_as_float(q8.Rmax[b * k + t]);
-    }
-  }
-  if (q8.step && b == 0 && bi == 0 && bj == 0 && t == 0) *q8.step += 1;
+  if (t == 0 && *abort_flag && status) atomicExch(status, (int32_t)GM_E_TIMEOUT);
 }
 
 // ------------------------------------------------------------------ S6
@@ -2154,23 +2260,38 @@ static bool tc_operand_maps(CUtensorMap* hi, CUtensorMap* lo, const float* base,
   return true;
 }
 
-cudaError_t launch_residual_tc(int B, int m, int n, int k, const float* X, const float* P,
+cudaError_t launch_residual_ws(int B, int m, int n, int k, const float* X, const float* P,
                                const float* R, const float* PT, const float* RT, uint8_t* codes4,
                                float* rscale, float* cscale, const unsigned* PRmax, int8_t* P8,
                                float* Pscale, int8_t* R8, float* Rscale, int64_t* step,
                                const int32_t* skip, int32_t* status, cudaStream_t s) {
-  ResidualTcMaps maps;
+  ResidualWsMaps maps;
   if (!tc_operand_maps(&maps.P, &maps.Plo, PT, B, m) || !tc_operand_maps(&maps.R, &maps.Rlo, RT, B, n))
     return cudaErrorInvalidValue;
+  {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    const cuuint64_t dims[3] = {(cuuint64_t)n, (cuuint64_t)m, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)n * 4, (cuuint64_t)m * n * 4};
+    const cuuint32_t box[3] = {32, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(&maps.M, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(X), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   static DeviceOnce attr;
   {
-    const cudaError_t e = smem_attr_once(attr, k_residual_tc, kTcSmemBytes);
+    const cudaError_t e = smem_attr_once(attr, k_residual_ws, kWsSmemBytes);
     if (e != cudaSuccess) return e;
   }
   const Quant8Out q8{PRmax, PRmax ? PRmax + (size_t)B * k : nullptr, P8, Pscale, R8, Rscale, step};
-  dim3 grid(cdiv(n, kGrid), cdiv(m, kGrid), B);
-  k_residual_tc<<<grid, kTcThreads, kTcSmemBytes, s>>>(maps, m, n, k, X, P, R, codes4, rscale, cscale,
-                                                       q8, skip, status);
+  const int nb = cdiv(n, kGrid), mb = cdiv(m, kGrid);
+  const long long total = (long long)nb * mb * B;
+  if (total > (1LL << 30)) return cudaErrorInvalidValue;
+  const int grid = (int)min(total, (long long)num_sms());
+  k_residual_ws<<<grid, kWsThreads, kWsSmemBytes, s>>>(maps, m, n, k, nb, mb, (int)total, P, R, codes4,
+                                                       rscale, cscale, q8, skip, status);
   return cudaGetLastError();
 }
 

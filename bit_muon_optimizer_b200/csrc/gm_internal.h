@@ -10,6 +10,8 @@ namespace gm {
 
 // The driver's cuTensorMapEncodeTiled (NULL if the driver does not provide it).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
+// SM count of the current device.
+int num_sms();
 
 // Column / row split counts of the power-iteration reductions. They depend
 // only on the problem shape, so the workspace layout is a pure function of it.
@@ -73,10 +75,11 @@ cudaError_t launch_backproject(int B, int m, int n, int k, const float* M, const
                                float* R, uint32_t* RB, float* RT, unsigned* Rmax,
                                const int32_t* skip, cudaStream_t s);
 
-// The step's residual pass on the tensor cores (tcgen05, kind::tf32): the same
-// outputs as launch_residual_quant4 with ready-made operand rows PT, RT; status
-// gets GM_E_TIMEOUT when a bounded wait runs out.
-cudaError_t launch_residual_tc(int B, int m, int n, int k, const float* X, const float* P,
+// The step's residual pass on the tensor cores (tcgen05, kind::tf32), persistent and
+// warp-specialized (one CTA per SM streaming M through a TMA ring): the same outputs
+// as launch_residual_quant4 with ready-made operand rows PT, RT; status gets
+// GM_E_TIMEOUT when a bounded wait runs out.
+cudaError_t launch_residual_ws(int B, int m, int n, int k, const float* X, const float* P,
                                const float* R, const float* PT, const float* RT, uint8_t* codes4,
                                float* rscale, float* cscale, const unsigned* PRmax, int8_t* P8,
                                float* Pscale, int8_t* R8, float* Rscale, int64_t* step,

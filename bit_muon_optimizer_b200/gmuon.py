@@ -40,7 +40,7 @@ class GraspParams(ctypes.Structure):
                 ("ns", c_int), ("abc", ctypes.POINTER(c_float)),
                 ("restart_after", ctypes.POINTER(c_int)), ("n_restart", c_int),
                 ("eps", c_float), ("seed", c_uint64), ("power_steps", c_int),
-                ("residual_from_codes", c_int), ("matrix_ids", vp)]
+                ("residual_from_codes", c_int), ("matrix_ids", vp), ("block", c_int)]
 
 
 class GraspStateC(ctypes.Structure):
@@ -67,7 +67,7 @@ _sig("gm_workspace_bytes", c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int])
 _sig("gm_dequant_rebuild", c_int, [c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp])
 _sig("gm_momentum_powerit", c_int, [c_int, c_int, c_int, c_int, c_float, vp, vp, c_int, vp,
                                     c_uint64, vp, vp, vp, vp, c_size_t, vp])
-_sig("gm_grid_quant4", c_int, [c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, vp])
+_sig("gm_grid_quant4", c_int, [c_int, c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, vp])
 _sig("gm_quant8", c_int, [c_int, c_int, c_int, vp, vp, vp, vp])
 _sig("gm_group_quant4", c_int, [c_int, c_int, c_int, vp, vp, vp, vp])
 _sig("gm_group_dequant4", c_int, [c_int, c_int, c_int, vp, vp, vp, vp])
@@ -251,7 +251,7 @@ def grid_quant4(X, P=None, R=None, out=None):
         codes = torch.empty((B, m, n // 2), dtype=torch.uint8, device=dev)
         rs = torch.empty((B, m, -(-n // GRID_BLOCK)), dtype=torch.float32, device=dev)
         cs = torch.empty((B, -(-m // GRID_BLOCK), n), dtype=torch.float32, device=dev)
-    _check(lib.gm_grid_quant4(B, m, n, k, _ptr(X), _ptr(P), _ptr(R), _ptr(codes), _ptr(rs),
+    _check(lib.gm_grid_quant4(B, m, n, GRID_BLOCK, k, _ptr(X), _ptr(P), _ptr(R), _ptr(codes), _ptr(rs),
                               _ptr(cs), _stream()), "gm_grid_quant4")
     return codes, rs, cs
 

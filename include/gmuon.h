@@ -131,9 +131,11 @@ gm_status gm_momentum_powerit(int B, int m, int n, int k, float mu,
  * division, ties to even), s = 0 -> q = 0.
  *   X f32 [B][m][n]; P f32 [B][m][k] and R f32 [B][n][k] both NULL (quantize X)
  *   or both non-NULL (quantize the residual, fp32 FMA); codes4/rscale/cscale as
- *   in gm_dequant_rebuild (outputs).
+ *   in gm_dequant_rebuild (outputs). block is the grid block side: 128, the
+ *   size the method uses and the only one built (anything else: GM_E_INVALID);
+ *   k is ignored when P and R are NULL.
  */
-gm_status gm_grid_quant4(int B, int m, int n, int k, const float* X,
+gm_status gm_grid_quant4(int B, int m, int n, int block, int k, const float* X,
                          const float* P, const float* R,
                          uint8_t* codes4, float* rscale, float* cscale, gm_stream_t stream);
 
@@ -286,6 +288,8 @@ typedef struct {
                                 matrix its index in the whole parameter set makes the start
                                 vectors independent of how a set is split into calls (e.g.
                                 across ranks); ids lie in [0, 65536) */
+  int block;                 /* grid block side of the 4-bit residual: 0 or 128 (the only
+                                size built; anything else: GM_E_INVALID) */
 } gm_grasp_params;
 
 /* The quantized momentum state [GRASP, worked step, last paragraph];

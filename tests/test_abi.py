@@ -63,7 +63,7 @@ def test_argument_errors_are_reported_before_any_launch():
     assert r == gm.GM_E_ARG
     assert b"NULL" in gm.lib.gm_last_error()
     # bad shape
-    r = gm.lib.gm_grid_quant4(1, 250, 512, 0, ctypes.c_void_p(256), None, None, ctypes.c_void_p(256),
+    r = gm.lib.gm_grid_quant4(1, 250, 512, 128, 0, ctypes.c_void_p(256), None, None, ctypes.c_void_p(256),
                               ctypes.c_void_p(256), ctypes.c_void_p(256), None)
     assert r == gm.GM_E_ARG
     # k out of range
@@ -81,7 +81,7 @@ def test_argument_errors_are_reported_before_any_launch():
 def test_misaligned_arrays_are_rejected_before_any_launch():
     """Every device array must be 16-byte aligned (the kernels move 16-byte vectors)."""
     ok, bad = ctypes.c_void_p(4096), ctypes.c_void_p(4096 + 8)
-    r = gm.lib.gm_grid_quant4(1, 256, 512, 0, bad, None, None, ok, ok, ok, None)
+    r = gm.lib.gm_grid_quant4(1, 256, 512, 128, 0, bad, None, None, ok, ok, ok, None)
     assert r == gm.GM_E_ARG and b"aligned" in gm.lib.gm_last_error()
     prm = gm.GraspParams(0.95, 0.02, 0.0, 8, 5, 0, None, None, 0, 1e-7, 0)
     st = gm.GraspStateC(4096, 4096, 4096, 4096, 4096, 4096, 4096 + 4, 4096, 4096)   # Rscale off by 4
@@ -106,7 +106,7 @@ def test_empty_and_out_of_range_shapes_are_argument_errors(B, m, n):
         lambda: gm.lib.gm_grasp_step(B, m, n, ctypes.byref(prm), ctypes.byref(st), ok, ok, 1, ok,
                                      1 << 40, None),
         lambda: gm.lib.gm_newton_schulz(B, m, n, ok, 1, None, 5, 1e-7, ok, 0, ok, 1 << 40, None),
-        lambda: gm.lib.gm_grid_quant4(B, m, n, 0, ok, None, None, ok, ok, ok, None),
+        lambda: gm.lib.gm_grid_quant4(B, m, n, 128, 0, ok, None, None, ok, ok, ok, None),
         lambda: gm.lib.gm_dequant_rebuild(B, m, n, 0, ok, ok, ok, None, None, None, None, ok, None),
     ]
     for call in calls:
@@ -185,3 +185,17 @@ def test_new_entry_points_argument_errors():
     assert gm.lib.gm_test_wait_timeout(ok, ok, 10, None) == gm.GM_E_ARG
     assert gm.lib.gm_test_wait_timeout(ok, ok, 5_000_000_000, None) == gm.GM_E_ARG
     assert gm.lib.gm_test_wait_timeout(None, ok, 20_000_000, None) == gm.GM_E_ARG
+
+
+def test_grid_block_other_than_128_is_an_argument_error():
+    """The grid block side is an argument of gm_grid_quant4 and a field of the step's
+    parameters; 128 (or 0 in the parameters, the default) is the only size built."""
+    ok = ctypes.c_void_p(4096)
+    for block in (64, 256, 0):
+        r = gm.lib.gm_grid_quant4(1, 256, 512, block, 0, ok, None, None, ok, ok, ok, None)
+        assert r == gm.GM_E_ARG and b"block" in gm.lib.gm_last_error()
+    st = gm.GraspStateC(*([4096] * 9))
+    prm = gm.GraspParams(0.95, 0.02, 0.0, 8, 5, 0, None, None, 0, 1e-7, 0)
+    prm.block = 64
+    r = gm.lib.gm_grasp_step(1, 256, 512, ctypes.byref(prm), ctypes.byref(st), ok, ok, 1, ok, 1 << 40, None)
+    assert r == gm.GM_E_ARG and b"block" in gm.lib.gm_last_error()
