@@ -2289,7 +2289,7 @@ cudaError_t launch_residual_ws(int B, int m, int n, int k, const float* X, const
   const int nb = cdiv(n, kGrid), mb = cdiv(m, kGrid);
   const long long total = (long long)nb * mb * B;
   if (total > (1LL << 30)) return cudaErrorInvalidValue;
-  const int grid = (int)min(total, (long long)num_sms());
+  const int grid = (int)min(total, (long long)sm_count());
   k_residual_ws<<<grid, kWsThreads, kWsSmemBytes, s>>>(maps, m, n, k, nb, mb, (int)total, P, R, codes4,
                                                        rscale, cscale, q8, skip, status);
   return cudaGetLastError();

@@ -69,6 +69,20 @@ __host__ __device__ inline uint64_t splitmix64(uint64_t x) {
 // primary context), so every cache of them is keyed by the current device.
 constexpr int kMaxDevices = 64;
 
+// SM count of the current device (cached per device; 148 if the query fails).
+inline int sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      return 148;
+    cache[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
 // Runs `fn` once per device (the current one when called), thread-safe; a
 // failed `fn` is retried on the next call.
 class DeviceOnce {

@@ -910,8 +910,6 @@ bool map_mnmajor(CUtensorMap* m, const void* base, bool f16, int rows, int cols,
 constexpr int kShortK = 1024;
 int stage_kblocks(int K) { return K <= kShortK ? 1 : 2; }
 
-}  // namespace
-
 // SM count of the current device (cached per device).
 int num_sms() {
   static std::atomic<int> cache[kMaxDevices];
@@ -925,8 +923,6 @@ int num_sms() {
   }
   return n;
 }
-
-namespace {
 
 struct Maps {
   CUtensorMap A, B, D, Ds, D2, D2s;

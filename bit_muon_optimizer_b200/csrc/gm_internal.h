@@ -10,8 +10,6 @@ namespace gm {
 
 // The driver's cuTensorMapEncodeTiled (NULL if the driver does not provide it).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
-// SM count of the current device.
-int num_sms();
 
 // Column / row split counts of the power-iteration reductions. They depend
 // only on the problem shape, so the workspace layout is a pure function of it.
