@@ -160,7 +160,7 @@ def oracle_sample_seconds(w: WL.Workload, ns: str):
         G = WL.gradient(w, b, 1, g.m, g.n)
         t0 = time.perf_counter()
         O.grasp_step(O.zero_state(g.m, g.n, w.k), W, G, mu=w.mu, eta=w.eta, wd=w.wd, seed=w.seed,
-                     b=b, ns=ns, T=w.T)
+                     b=b, ns=ns_name(ns, g.m, g.n), T=w.T)
         per_shape.append((g, time.perf_counter() - t0))
     ms = 1e3 * sum(g.count * s for g, s in per_shape)
     sample = ("fp64 oracle, one step of one matrix per shape group ("
@@ -196,7 +196,7 @@ def run_reference(args, world, rank):
         G = WL.gradient(w, b, smp["t"], g.m, g.n)
         t0 = time.perf_counter()
         r = O.grasp_step(smp["st"], smp["W"], G, mu=w.mu, eta=w.eta, wd=w.wd, seed=w.seed, b=b,
-                         ns=args.ns, T=w.T)
+                         ns=ns_name(args.ns, g.m, g.n), T=w.T)
         smp["s"] = time.perf_counter() - t0
         smp["st"], smp["W"] = r.state, r.W.float()
 
@@ -264,12 +264,32 @@ def est_bytes(w: WL.Workload, pool: int) -> int:
     return elems * (22 + 2 * pool)
 
 
-def build_group(gm, w: WL.Workload, gi: int, ns_mode: int, pool: int, dev):
+def ns_name(ns: str, m: int, n: int) -> str:
+    """The NS form ("standard" or "gram") that --ns gives an m x n matrix."""
+    if ns == "auto":
+        return "gram" if m != n else "standard"
+    return ns
+
+
+def ns_chooser(gm, ns: str):
+    """The NS form of each shape: "standard" or "gram" everywhere, or "auto": the Gram
+    form for non-square matrices, the standard form for square ones (the Gram NS
+    page's FLOP comparison: (17 + 3 alpha) n^3 against 5 (3 alpha + 1) n^3 at T = 5,
+    fewer exactly when the aspect ratio alpha > 1)."""
+    std, gram = gm.GM_NS_STANDARD, gm.GM_NS_GRAM
+    if ns == "gram":
+        return lambda m, n: gram
+    if ns == "auto":
+        return lambda m, n: gram if m != n else std
+    return lambda m, n: std
+
+
+def build_group(gm, w: WL.Workload, gi: int, nsf, pool: int, dev):
     g = w.groups[gi]
     B, m, n = g.count, g.m, g.n
     base = w.group_base(gi)
     ids = list(range(base, base + B))
-    step = gm.GraspStep(B, m, n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=ns_mode,
+    step = gm.GraspStep(B, m, n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=nsf(m, n),
                         seed=w.seed, device=dev, matrix_ids=ids)
     st = gm.GraspState.zeros(B, m, n, w.k, dev)
     W = torch.empty((B, m, n), dtype=torch.float32, device=dev)
@@ -284,7 +304,7 @@ def build_group(gm, w: WL.Workload, gi: int, ns_mode: int, pool: int, dev):
     return dict(step=step, st=st, W=W, grads=grads, B=B, m=m, n=n)
 
 
-def our_launches(gm, w: WL.Workload, ns_mode: int, groups=None) -> int:
+def our_launches(gm, w: WL.Workload, nsf, groups=None) -> int:
     """Our kernels per step: per group 9 codec kernels (column norms, warm start
     with the factor fragments, rebuild + projection, three orthonormalisation
     kernels, back projection, its finalisation, the 4-bit quantisation with the
@@ -293,11 +313,11 @@ def our_launches(gm, w: WL.Workload, ns_mode: int, groups=None) -> int:
     launches = 0
     for (m, n) in (groups if groups is not None else [(g.m, g.n) for g in w.groups]):
         pad = int(min(m, n) % 64 != 0 or max(m, n) % 64 != 0)
-        launches += 9 + gm.ns_flops(ns_mode, m, n, w.T)[1] + pad
+        launches += 9 + gm.ns_flops(nsf(m, n), m, n, w.T)[1] + pad
     return launches
 
 
-def measure(gm, w, groups, ns_mode, args, world, local, do_e2e):
+def measure(gm, w, groups, nsf, args, world, local, do_e2e):
     """Times args.steps graph-replayed GRASP steps over `groups` (each group on
     its own stream); then the step's two halves with CUDA events around each
     (codec half: gm_grasp_state_update; NS half: gm_grasp_apply); the cuBLAS
@@ -373,8 +393,8 @@ def measure(gm, w, groups, ns_mode, args, world, local, do_e2e):
     torch.cuda.synchronize()
     cod_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in evs) / nb
     ns_ms = sum(e1.elapsed_time(e2) for _, e1, e2 in evs) / nb
-    ns_flops = sum(gm.ns_flops(ns_mode, g["m"], g["n"], w.T)[0] * g["B"] for g in groups)
-    ns_launches = sum(gm.ns_flops(ns_mode, g["m"], g["n"], w.T)[1] for g in groups)
+    ns_flops = sum(gm.ns_flops(nsf(g["m"], g["n"]), g["m"], g["n"], w.T)[0] * g["B"] for g in groups)
+    ns_launches = sum(gm.ns_flops(nsf(g["m"], g["n"]), g["m"], g["n"], w.T)[1] for g in groups)
 
     # ---- the standalone 4-bit codecs of the same entry points a user calls
     # (4bit-Muon-base group codec, MuonQ's mu-law codec), on the first group's
@@ -479,7 +499,7 @@ def codec_bytes(w: WL.Workload, groups) -> float:
     return sum(g["B"] * g["m"] * g["n"] for g in groups) * (gb + 2 * (0.5 + 0.0625) + 2)
 
 
-def run_single(gm, w, ns_mode, args, local):
+def run_single(gm, w, nsf, args, local):
     dev = torch.device("cuda", local)
     total_mem = torch.cuda.get_device_properties(dev).total_memory
     pool = min(GRAD_POOL, args.warmup + args.steps)
@@ -491,9 +511,9 @@ def run_single(gm, w, ns_mode, args, local):
     batches = [[gi] for gi in range(len(w.groups))] if per_group else [list(range(len(w.groups)))]
     res = []
     for i, gis in enumerate(batches):
-        groups = [build_group(gm, w, gi, ns_mode, pool, dev) for gi in gis]
+        groups = [build_group(gm, w, gi, nsf, pool, dev) for gi in gis]
         args.codecs = i == 0
-        r = measure(gm, w, groups, ns_mode, args, 1, local, not args.no_e2e)
+        r = measure(gm, w, groups, nsf, args, 1, local, not args.no_e2e)
         r["codec_bytes"] = codec_bytes(w, groups)
         res.append(r)
         del groups
@@ -518,22 +538,26 @@ def run_single(gm, w, ns_mode, args, local):
                        if per_group else ""))
     out["pool"] = pool
     out["codecs"] = res[0]["codecs"]
-    out["launches"] = our_launches(gm, w, ns_mode) * args.steps
+    out["launches"] = our_launches(gm, w, nsf) * args.steps
     return out
 
 
-def run_sharded(gm, w, ns_mode, args, world, rank, local):
+def run_sharded(gm, w, nsf, args, world, rank, local):
     """N > 1: the set split by ownership (sharding.ShardedStep: LPT owners, the
-    owners' GRASP steps, one NCCL all-gather of the updated fp32 weights per
-    shape group), one shape group at a time; eager launches (the exchange is
+    owners' GRASP steps up to O, one NCCL all-gather of the bf16 O and skip
+    flags per shape group, every rank's weight update; or, with --exchange
+    weights, the owners' whole steps and an all-gather of the updated fp32
+    weights), one shape group at a time; eager launches (the exchange is
     torch.distributed). Returns the max over ranks of the summed group times."""
     from bit_muon_optimizer_b200 import sharding as S
     dev = torch.device("cuda", local)
-    make = S.grasp_make_step(w.k, dev, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=ns_mode, seed=w.seed)
+    update = S.grasp_update(w.eta, w.wd) if args.exchange == "update" else None
     ms_total, clocks, launches, owned = 0.0, [], 0, []
     for gi, g in enumerate(w.groups):
         base = w.group_base(gi)
-        sh = S.ShardedStep([(g.m, g.n, g.count)], world, rank, make, first_index=base)
+        make = S.grasp_make_step(w.k, dev, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=nsf(g.m, g.n),
+                                 seed=w.seed)
+        sh = S.ShardedStep([(g.m, g.n, g.count)], world, rank, make, first_index=base, update=update)
         W = torch.empty((g.count, g.m, g.n), dtype=torch.float32, device=dev)
         grads = []
         for b in range(g.count):
@@ -563,7 +587,9 @@ def run_sharded(gm, w, ns_mode, args, world, rank, local):
         mine = len(sh.owned[0][rank])
         owned.append(mine)
         if mine:
-            launches += our_launches(gm, w, ns_mode, [(g.m, g.n)])
+            launches += our_launches(gm, w, nsf, [(g.m, g.n)])
+        if update is not None:
+            launches += 1                              # k_weight_update on every rank
         del sh, W, grads
         torch.cuda.empty_cache()
     clk = None
@@ -578,22 +604,29 @@ def run_sharded(gm, w, ns_mode, args, world, rank, local):
 def run_ours(args, world, rank, local):
     from bit_muon_optimizer_b200 import gmuon as gm
     w = WL.WORKLOADS[args.config]
-    ns_mode = gm.GM_NS_GRAM if args.ns == "gram" else gm.GM_NS_STANDARD
+    nsf = ns_chooser(gm, args.ns)
     hbm, bf16, bf16_sus, peak_kind = _peaks()
     elements = sum(g.count * g.m * g.n for g in w.groups)
-    step_flops = sum(gm.ns_flops(ns_mode, g.m, g.n, w.T)[0] * g.count for g in w.groups)
+    step_flops = sum(gm.ns_flops(nsf(g.m, g.n), g.m, g.n, w.T)[0] * g.count for g in w.groups)
     step_bytes = elements * FL.step_bytes_per_element(2 if w.gdtype != torch.float32 else 4)
     t_roof = max(step_flops / (bf16 * 1e12), step_bytes / (hbm * 1e9)) * 1e3
     config = {"workload": w.name, "ns": args.ns, "k": w.k,
               "shapes": [[g.m, g.n, g.count] for g in w.groups],
               "elements": elements, "grad_dtype": str(w.gdtype).replace("torch.", ""),
               "l2": "per-step working set (G, W, state, fp32 M) > L2; no flush"}
-    dtype = "bf16" if ns_mode == gm.GM_NS_STANDARD else "f16"
+    modes = {nsf(g.m, g.n) for g in w.groups}
+    dtype = "+".join(d for mode, d in ((gm.GM_NS_STANDARD, "bf16"), (gm.GM_NS_GRAM, "f16")) if mode in modes)
+    if args.ns == "auto":
+        config["ns_per_group"] = ["gram" if nsf(g.m, g.n) == gm.GM_NS_GRAM else "standard"
+                                  for g in w.groups]
     if world > 1:
-        ms_step, clocks, launches, owned = run_sharded(gm, w, ns_mode, args, world, rank, local)
+        ms_step, clocks, launches, owned = run_sharded(gm, w, nsf, args, world, rank, local)
         if rank == 0:
+            what = ("the owners' bf16 update directions O (2 B per element) and skip flags, "
+                    "then every rank's weight update" if args.exchange == "update"
+                    else "the owners' updated fp32 weights (4 B per element)")
             config.update(parallelism=f"ownership sharding x{world}: LPT owners per shape group, "
-                                      "one NCCL all-gather of the updated fp32 weights per group",
+                                      f"one NCCL all-gather per group of {what}",
                           graph="eager launches, shape groups one at a time, set time = sum",
                           owned_per_group_rank0=owned)
             line = {"metric": METRIC, "value": ms_step, "unit": UNIT, "n_gpus": world,
@@ -606,7 +639,7 @@ def run_ours(args, world, rank, local):
                     "gpu_launches": launches, "clocks": clocks, "e2e": None, "cpu_baseline": None}
             print(json.dumps(line), flush=True)
         return
-    r = run_single(gm, w, ns_mode, args, local)
+    r = run_single(gm, w, nsf, args, local)
     ns_tflops = r["ns_flops"] / (r["ns_ms"] * 1e-3) / 1e12
     codec_gbs = r["codec_bytes"] / (r["cod_ms"] * 1e-3) / 1e9
     long_step = r["ms_step"] > 50.0
@@ -663,14 +696,14 @@ def run_profile(args):
     and no JSON line; the device status is checked after every group."""
     from bit_muon_optimizer_b200 import gmuon as gm
     w = WL.WORKLOADS[args.config]
-    ns_mode = gm.GM_NS_GRAM if args.ns == "gram" else gm.GM_NS_STANDARD
+    nsf = ns_chooser(gm, args.ns)
     dev = torch.device("cuda", 0)
     gis = range(len(w.groups)) if args.group < 0 else [args.group]
     for gi in gis:
         g = w.groups[gi]
         B = args.batch or g.count
         base = w.group_base(gi)
-        step = gm.GraspStep(B, g.m, g.n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=ns_mode,
+        step = gm.GraspStep(B, g.m, g.n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=nsf(g.m, g.n),
                             seed=w.seed, device=dev, matrix_ids=list(range(base, base + B)))
         st = gm.GraspState.zeros(B, g.m, g.n, w.k, dev)
         W = torch.empty((B, g.m, g.n), dtype=torch.float32, device=dev)
@@ -694,7 +727,10 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", type=int, default=4)
-    ap.add_argument("--ns", choices=["standard", "gram"], default="standard")
+    ap.add_argument("--ns", choices=["standard", "gram", "auto"], default="standard",
+                    help="NS form; auto: Gram NS for non-square shapes, standard for square ones")
+    ap.add_argument("--exchange", choices=["update", "weights"], default="update",
+                    help="N > 1: all-gather the bf16 update direction (default) or the fp32 weights")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgmuon.so")
-SOURCES = ["gm_api.cu", "gm_codec.cu", "gm_gemm.cu", "gm_noalloc.cu", "gm_base4.cu"]
+SOURCES = ["gm_api.cu", "gm_codec.cu", "gm_gemm.cu", "gm_noalloc.cu", "gm_base4.cu", "gm_update.cu"]
 HEADERS = ["gm_common.cuh", "gm_internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -2,6 +2,7 @@
 // layout and the enqueueing of the step's kernels on the caller's stream.
 
 #include <stdarg.h>
+#include <cmath>
 #include <stdio.h>
 #include <string.h>
 
@@ -536,6 +537,45 @@ gm_status gm_grasp_apply(int B, int m, int n, const gm_grasp_params* prm, const 
                         w + L.ns, status, status, s));
   else
     GM_CUDA(run_ns_standard(B, m, n, X, tab, prm->T, out, w + L.ns, status, status, s));
+  return GM_OK;
+}
+
+gm_status gm_grasp_orth(int B, int m, int n, const gm_grasp_params* prm, const gm_grasp_state* st,
+                        void* O, gm_dtype odt, void* ws, size_t ws_bytes, gm_stream_t stream) {
+  GM_CHECK_ARG(odt == GM_F32 || odt == GM_BF16 || odt == GM_F16, "bad odt");
+  GM_CHECK_ARG(O, "NULL O");
+  GM_CHECK_ARG(al16(O), "device arrays must be 16-byte aligned");
+  StepLayout L;
+  const gm_status chk =
+      step_checks(B, m, n, prm, st, nullptr, false, nullptr, false, GM_F32, ws, ws_bytes, &L);
+  if (chk != GM_OK) return chk;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* X = reinterpret_cast<uint16_t*>(w + L.X);
+  int32_t* status = st->dev_status;
+  float tab[3 * GM_MAX_T];
+  expand_abc(prm->abc, prm->T, tab);
+  // worked step 6 up to O = NS(M_t)
+  NsOutput out{0, O, (int)odt, nullptr, 0.f, 0.f};
+  if (prm->ns == GM_NS_GRAM)
+    GM_CUDA(run_ns_gram(B, m, n, X, tab, prm->T, prm->restart_after, prm->n_restart, out,
+                        w + L.ns, status, status, s));
+  else
+    GM_CUDA(run_ns_standard(B, m, n, X, tab, prm->T, out, w + L.ns, status, status, s));
+  return GM_OK;
+}
+
+gm_status gm_weight_update(int B, int m, int n, float eta, float wd, const void* O, gm_dtype odt,
+                           float* W, const int32_t* skip, int skip_stride, gm_stream_t stream) {
+  GM_CHECK_ARG(shape_ok(B, m, n), "bad shape B=%d m=%d n=%d", B, m, n);
+  GM_CHECK_ARG(O && W, "NULL O or W");
+  GM_CHECK_ARG(odt == GM_F32 || odt == GM_BF16 || odt == GM_F16, "bad odt");
+  GM_CHECK_ARG(al16(O) && al16(W) && al16(skip), "device arrays must be 16-byte aligned");
+  GM_CHECK_ARG(skip_stride == 0 || skip_stride == 1, "skip_stride must be 0 or 1");
+  GM_CHECK_ARG(std::isfinite(eta) && std::isfinite(wd), "eta and wd must be finite");
+  GM_DEVICE();
+  GM_CUDA(launch_weight_update(B, m, n, eta, wd, O, (int)odt, W, skip, skip_stride,
+                               reinterpret_cast<cudaStream_t>(stream)));
   return GM_OK;
 }
 

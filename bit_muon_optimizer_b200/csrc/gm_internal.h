@@ -83,6 +83,11 @@ cudaError_t launch_residual_ws(int B, int m, int n, int k, const float* X, const
                                float* Pscale, int8_t* R8, float* Rscale, int64_t* step,
                                const int32_t* skip, int32_t* status, cudaStream_t s);
 
+// W <- W - eta (O + wd W) (O in odt: GM_F32, GM_BF16 or GM_F16); matrix b is
+// left alone when skip && skip[b * skip_stride].
+cudaError_t launch_weight_update(int B, int m, int n, float eta, float wd, const void* O, int odt,
+                                 float* W, const int32_t* skip, int skip_stride, cudaStream_t s);
+
 // PA, RB: ready-made fragments of -P and R (both or neither; NULL stages P, R).
 // PRmax (nullable): the P then R column maxima; with it the kernel also writes the
 // 8-bit state P8, Pscale, R8, Rscale and increments step.

@@ -85,6 +85,9 @@ _sig("gm_grasp_state_update", c_int, [c_int, c_int, c_int, ctypes.POINTER(GraspP
                                       ctypes.POINTER(GraspStateC), vp, c_int, vp, c_size_t, vp])
 _sig("gm_grasp_apply", c_int, [c_int, c_int, c_int, ctypes.POINTER(GraspParams),
                                ctypes.POINTER(GraspStateC), vp, vp, c_size_t, vp])
+_sig("gm_grasp_orth", c_int, [c_int, c_int, c_int, ctypes.POINTER(GraspParams),
+                              ctypes.POINTER(GraspStateC), vp, c_int, vp, c_size_t, vp])
+_sig("gm_weight_update", c_int, [c_int, c_int, c_int, c_float, c_float, vp, c_int, vp, vp, c_int, vp])
 _sig("gm_grasp_workspace_layout", c_int, [c_int, c_int, c_int, c_int, c_int,
                                           ctypes.POINTER(GraspWsLayout)])
 _sig("gm_ns_flops", c_int, [c_int, c_int, c_int, c_int, vp, c_int,
@@ -482,6 +485,26 @@ class GraspState:
         return GraspState(*[t.clone() for t in self.tensors()])
 
 
+def weight_update(W, O, eta, wd=0.0, skip=None):
+    """W <- W - eta (O + wd W) in place (gm_weight_update); O in float32, bfloat16 or
+    float16 of W's shape. ``skip`` (optional device int32): one flag for the batch
+    ([1]) or one per matrix ([B]); a flagged matrix keeps its weights."""
+    B, m, n = _bmn(W)
+    _expect(W, (B, m, n), (torch.float32,), "W")
+    _expect(O, (B, m, n), (torch.float32, torch.bfloat16, torch.float16), "O")
+    stride = 0
+    if skip is not None:
+        if skip.dtype != torch.int32 or not skip.is_contiguous() or skip.numel() not in (1, B):
+            raise ValueError("skip: a contiguous int32 tensor of 1 or B flags expected")
+        stride = 0 if skip.numel() == 1 else 1
+        _placed((W, O, skip), ("W", "O", "skip"))
+    else:
+        _placed((W, O), ("W", "O"))
+    _check(lib.gm_weight_update(B, m, n, float(eta), float(wd), _ptr(O), _DT[O.dtype], _ptr(W),
+                                _ptr(skip), stride, _stream()), "gm_weight_update")
+    return W
+
+
 class GraspStep:
     """Marshals one gm_grasp_step call for a fixed shape batch.
 
@@ -552,6 +575,28 @@ class GraspStep:
         st = state.c_struct()
         _check(lib.gm_grasp_apply(B, m, n, ctypes.byref(self.params), ctypes.byref(st), _ptr(W),
                                   _ptr(self.ws), self.ws_bytes, _stream()), "gm_grasp_apply")
+
+    def orth(self, state: GraspState, out=None, dtype=torch.bfloat16):
+        """Worked step 6 up to O = NS(M_t) (gm_grasp_orth) on the NS input the state
+        update left; O [B, m, n] in ``dtype`` (float32, bfloat16 or float16), not
+        written when the state update flagged a non-finite value."""
+        B, m, n = self.B, self.m, self.n
+        state.check(B, m, n, self.k)
+        if out is None:
+            out = torch.empty((B, m, n), dtype=dtype, device=self.ws.device)
+        _expect(out, (B, m, n), (torch.float32, torch.bfloat16, torch.float16), "O")
+        _placed((out,), ("O",))
+        _ws_fits(self.ws, self.ws_bytes)
+        st = state.c_struct()
+        _check(lib.gm_grasp_orth(B, m, n, ctypes.byref(self.params), ctypes.byref(st), _ptr(out),
+                                 _DT[out.dtype], _ptr(self.ws), self.ws_bytes, _stream()),
+               "gm_grasp_orth")
+        return out
+
+    def direction(self, state: GraspState, G, out=None, dtype=torch.bfloat16):
+        """Worked steps 1-5 and O = NS(M_t): the state update, then ``orth``."""
+        self.state_update(state, G)
+        return self.orth(state, out, dtype)
 
     # stage buffers inside the workspace (views; valid after the step ran)
     def _view(self, off, shape, dtype):

@@ -23,6 +23,15 @@ Rademacher start vectors) from them, so a matrix's results do not depend on
 the number of ranks or on which rank owns it. The exchange is one all-gather
 per shape group through ``torch.distributed`` (NCCL on GPUs), each rank
 sending its owned matrices padded to the largest owner's count.
+
+Two things can be exchanged. By default the owners update their weights and
+send the updated fp32 weights (4 B per element). Given an ``update`` callable,
+the owners instead send the orthogonalized update O of worked step 6 in 16
+bits (2 B per element, half the bytes) with one skip flag per matrix, and
+every rank, owners included, applies W <- W - eta (O + wd W) to its own copy
+through ``update(W, O, flags)``: all ranks apply the same O to the same W, so
+they keep identical weights. The step object then provides
+``direction(G) -> (O, flags)`` instead of updating W.
 """
 
 from __future__ import annotations
@@ -65,11 +74,13 @@ class ShardedStep:
 
     def __init__(self, shapes: Sequence[tuple[int, int, int]], world: int, rank: int,
                  make_step: Callable[[int, int, list], Callable], cost=ns_cost, group=None,
-                 first_index: int = 0):
+                 first_index: int = 0, update: Callable | None = None,
+                 update_dtype: torch.dtype = torch.bfloat16):
         if not 0 <= rank < world:
             raise ValueError(f"rank {rank} outside world {world}")
         self.shapes = [tuple(s) for s in shapes]
         self.world, self.rank, self.group = world, rank, group
+        self.update, self.update_dtype = update, update_dtype
         costs = [cost(m, n) for m, n, count in self.shapes for _ in range(count)]
         flat = lpt_owners(costs, world)
         self.owner: list[list[int]] = []          # owner of matrix i of group g
@@ -100,6 +111,9 @@ class ShardedStep:
             if tuple(W.shape) != (count, m, n) or tuple(G.shape) != (count, m, n):
                 raise ValueError(f"group {g}: expected [{count}, {m}, {n}] weights and gradients")
             mine = self.owned[g][self.rank]
+            if self.update is not None:
+                self._exchange_update(g, m, n, count, W, G)
+                continue
             Wb = None
             if mine:
                 idx = torch.tensor(mine, device=W.device)
@@ -120,6 +134,36 @@ class ShardedStep:
                     W.index_copy_(0, torch.tensor(own, device=W.device), recv[r][:len(own)])
 
 
+    def _exchange_update(self, g, m, n, count, W, G):
+        """Owners send (O, flags); every rank applies all of them to its W."""
+        mine = self.owned[g][self.rank]
+        O = flags = None
+        if mine:
+            idx = torch.tensor(mine, device=W.device)
+            O, flags = self.steps[g].direction(G.index_select(0, idx))
+        if self.world == 1:
+            self.update(W, O, flags)         # the one rank owns every matrix, in order
+            return
+        width = max(len(o) for o in self.owned[g])
+        send = torch.zeros((width, m, n), dtype=self.update_dtype, device=W.device)
+        sendf = torch.ones((width,), dtype=torch.int32, device=W.device)
+        if mine:
+            send[:len(mine)] = O
+            sendf[:len(mine)] = flags
+        recv = [torch.empty_like(send) for _ in range(self.world)]
+        recvf = [torch.empty_like(sendf) for _ in range(self.world)]
+        dist.all_gather(recv, send, group=self.group)
+        dist.all_gather(recvf, sendf, group=self.group)
+        O_all = torch.empty((count, m, n), dtype=self.update_dtype, device=W.device)
+        f_all = torch.empty((count,), dtype=torch.int32, device=W.device)
+        for r, own in enumerate(self.owned[g]):
+            if own:
+                t = torch.tensor(own, device=W.device)
+                O_all.index_copy_(0, t, recv[r][:len(own)])
+                f_all.index_copy_(0, t, recvf[r][:len(own)])
+        self.update(W, O_all, f_all)
+
+
 def grasp_make_step(k: int, device=None, **params) -> Callable[[int, int, list], Callable]:
     """``make_step`` for the library's GRASP step: each owner batch gets its own
     step object and zero state (its quantized momentum lives on this rank only),
@@ -134,7 +178,23 @@ def grasp_make_step(k: int, device=None, **params) -> Callable[[int, int, list],
         def run(W: torch.Tensor, G: torch.Tensor) -> None:
             step(state, W, G)
 
+        def direction(G: torch.Tensor):
+            O = step.direction(state, G)
+            return O, state.dev_status.expand(B).contiguous()
+
         run.state = state
+        run.direction = direction
         return run
 
     return make
+
+
+def grasp_update(eta: float, wd: float = 0.0) -> Callable:
+    """``update`` for ShardedStep: the library's weight update (gm_weight_update),
+    each matrix skipped when its owner's step flagged a non-finite value."""
+    from . import gmuon as gm
+
+    def update(W: torch.Tensor, O: torch.Tensor, flags: torch.Tensor) -> None:
+        gm.weight_update(W, O, eta, wd, skip=flags)
+
+    return update

@@ -343,6 +343,32 @@ gm_status gm_grasp_apply(int B, int m, int n, const gm_grasp_params* params,
                          const gm_grasp_state* state, float* W,
                          void* ws, size_t ws_bytes, gm_stream_t stream);
 
+/*
+ * Worked step 6 split at O, for callers that move O before applying it (a
+ * parameter set split across ranks by ownership exchanges the owners' 16-bit
+ * O: half the bytes of their fp32 weights):
+ *  - gm_grasp_orth: O = NS(X) on the X that gm_grasp_state_update left in
+ *    `ws` (the NS form, table and restarts of `params`), written to O
+ *    [B][m][n] in odt (GM_F32, GM_BF16 or GM_F16; device, 16-byte aligned,
+ *    owned by the caller). When *dev_status is non-zero nothing is written.
+ *    The NS chain overwrites X.
+ *  - gm_weight_update: W <- W - eta (O + wd W), elementwise in fp32 with O
+ *    widened from odt; W f32 [B][m][n] (device, 16-byte aligned, in place).
+ *    skip (device int32, nullable): matrix b keeps its weights when
+ *    skip[b * skip_stride] is non-zero (skip_stride 0: one flag for the whole
+ *    batch, e.g. a state's dev_status; 1: one flag per matrix).
+ * gm_grasp_state_update, gm_grasp_orth (O in GM_F32) and gm_weight_update
+ * give W within fp32 rounding of gm_grasp_step's (whose last NS product
+ * applies the same update to its fp32 accumulators); with O in 16 bits, within
+ * eta times O's rounding. Every rank that applies the same O to the same W gets
+ * the same bits.
+ */
+gm_status gm_grasp_orth(int B, int m, int n, const gm_grasp_params* params,
+                        const gm_grasp_state* state, void* O, gm_dtype odt,
+                        void* ws, size_t ws_bytes, gm_stream_t stream);
+gm_status gm_weight_update(int B, int m, int n, float eta, float wd, const void* O, gm_dtype odt,
+                           float* W, const int32_t* skip, int skip_stride, gm_stream_t stream);
+
 /* Byte offsets of the stage buffers inside the gm_grasp_step workspace, for
  * inspection by tests: M f32 [B][m][n]; Q f32 [B][n][k]; P, R f32; X the NS
  * input (bf16 or fp16, wide form); scale f32 [B] = 1/(|M|_F + eps). */

@@ -199,3 +199,23 @@ def test_grid_block_other_than_128_is_an_argument_error():
     prm.block = 64
     r = gm.lib.gm_grasp_step(1, 256, 512, ctypes.byref(prm), ctypes.byref(st), ok, ok, 1, ok, 1 << 40, None)
     assert r == gm.GM_E_ARG and b"block" in gm.lib.gm_last_error()
+
+
+def test_orth_and_weight_update_argument_errors():
+    """gm_grasp_orth and gm_weight_update reject bad arguments on the host."""
+    ok, bad = ctypes.c_void_p(4096), ctypes.c_void_p(4096 + 8)
+    st = gm.GraspStateC(*([4096] * 9))
+    prm = gm.GraspParams(0.95, 0.02, 0.0, 8, 5, 0, None, None, 0, 1e-7, 0)
+    orth = lambda O, odt, ws_bytes=1 << 40: gm.lib.gm_grasp_orth(  # noqa: E731
+        2, 256, 512, ctypes.byref(prm), ctypes.byref(st), O, odt, ok, ws_bytes, None)
+    assert orth(None, gm.GM_BF16) == gm.GM_E_ARG
+    assert orth(ok, 7) == gm.GM_E_ARG and b"odt" in gm.lib.gm_last_error()
+    assert orth(bad, gm.GM_BF16) == gm.GM_E_ARG and b"aligned" in gm.lib.gm_last_error()
+    assert orth(ok, gm.GM_BF16, 16) == gm.GM_E_WORKSPACE
+    upd = gm.lib.gm_weight_update
+    assert upd(2, 250, 512, 0.02, 0.0, ok, gm.GM_BF16, ok, None, 0, None) == gm.GM_E_ARG
+    assert upd(2, 256, 512, 0.02, 0.0, None, gm.GM_BF16, ok, None, 0, None) == gm.GM_E_ARG
+    assert upd(2, 256, 512, 0.02, 0.0, ok, 9, ok, None, 0, None) == gm.GM_E_ARG
+    assert upd(2, 256, 512, 0.02, 0.0, ok, gm.GM_BF16, bad, None, 0, None) == gm.GM_E_ARG
+    assert upd(2, 256, 512, 0.02, 0.0, ok, gm.GM_BF16, ok, ok, 2, None) == gm.GM_E_ARG
+    assert upd(2, 256, 512, float("nan"), 0.0, ok, gm.GM_BF16, ok, None, 0, None) == gm.GM_E_ARG

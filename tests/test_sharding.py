@@ -58,16 +58,41 @@ class _StandIn:
         W.sub_(0.1 * self.t * G)
 
 
+class _StandInDir:
+    """Per-batch state as _StandIn; the update direction O = 0.1 t G in bf16 (a
+    non-finite G flags its matrix)."""
+
+    def __init__(self, m, n, ids):
+        self.t = 0
+
+    def direction(self, G):
+        self.t += 1
+        flags = (~torch.isfinite(G).flatten(1).all(1)).to(torch.int32)
+        return (0.1 * self.t * G).to(torch.bfloat16), flags
+
+
+def _standin_update(W, Od, flags):
+    keep = flags.bool()
+    Wn = W - 0.5 * (Od.float() + 0.1 * W)
+    W.copy_(torch.where(keep[:, None, None], W, Wn))
+
+
 def _inputs(step):
     g = torch.Generator().manual_seed(100 + step)
     return [torch.randn((c, m, n), generator=g) for m, n, c in SHAPES]
 
 
-def _run(world, rank, steps=2):
-    sh = S.ShardedStep(SHAPES, world, rank, _StandIn)
+def _run(world, rank, steps=2, exchange="weights"):
+    if exchange == "weights":
+        sh = S.ShardedStep(SHAPES, world, rank, _StandIn)
+    else:
+        sh = S.ShardedStep(SHAPES, world, rank, _StandInDir, update=_standin_update)
     W = [x.clone() for x in _inputs(0)]
     for t in range(1, steps + 1):
-        sh(W, _inputs(t))
+        G = _inputs(t)
+        if exchange == "update" and t == 2:
+            G[0][3, 1, 1] = float("nan")      # matrix 3 of group 0 is skipped in step 2
+        sh(W, G)
     return sh, W
 
 
@@ -78,11 +103,13 @@ O_K, O_SEED = 2, 7
 
 class _OracleStep:
     """The oracle's GRASP step for an owner batch; the Rademacher counter index b
-    is each matrix's set index (``set_ids``) or its place in the batch."""
+    is each matrix's set index (``set_ids``) or its place in the batch.
+    ``direction`` returns the oracle's O in bf16 instead of updating W."""
 
     def __init__(self, m, n, ids, set_ids=True):
         import oracle as O
         self.O = O
+        self.m, self.n = m, n
         self.ids = list(ids) if set_ids else list(range(len(ids)))
         self.states = [O.zero_state(m, n, O_K) for _ in ids]
 
@@ -93,6 +120,19 @@ class _OracleStep:
             self.states[i] = r.state
             W[i] = r.W.float()
 
+    def direction(self, G):
+        Od = torch.empty((len(self.ids), self.m, self.n), dtype=torch.bfloat16)
+        for i, b in enumerate(self.ids):
+            r = self.O.grasp_step(self.states[i], torch.zeros(self.m, self.n), G[i], mu=0.95,
+                                  eta=0.02, seed=O_SEED, b=b, T=2)
+            self.states[i] = r.state
+            Od[i] = r.O.to(torch.bfloat16)
+        return Od, torch.zeros(len(self.ids), dtype=torch.int32)
+
+
+def _oracle_update(W, Od, flags):
+    W.sub_(0.02 * (Od.float() + 0.0 * W))
+
 
 def _oracle_inputs(step):
     g = torch.Generator().manual_seed(300 + step)
@@ -100,7 +140,7 @@ def _oracle_inputs(step):
             for m, n, c in O_SHAPES]
 
 
-def _run_oracle(world, rank, set_ids):
+def _run_oracle(world, rank, set_ids, exchange="weights"):
     steps = []
 
     def make(m, n, ids):
@@ -108,7 +148,8 @@ def _run_oracle(world, rank, set_ids):
         steps.append((m, n, ids, st))
         return st
 
-    sh = S.ShardedStep(O_SHAPES, world, rank, make)
+    sh = S.ShardedStep(O_SHAPES, world, rank, make,
+                       update=_oracle_update if exchange == "update" else None)
     W = [x.clone() * 20 for x in _oracle_inputs(0)]
     for t in (1, 2):
         sh(W, _oracle_inputs(t))
@@ -116,7 +157,7 @@ def _run_oracle(world, rank, set_ids):
     return W, codes
 
 
-def _rank_main(rank, world, port, q, kind="standin", set_ids=True):
+def _rank_main(rank, world, port, q, kind="standin", set_ids=True, exchange="weights"):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world))
     sys.path.insert(0, ROOT)
@@ -129,20 +170,20 @@ def _rank_main(rank, world, port, q, kind="standin", set_ids=True):
         # plain arrays, pickled by value: a tensor would be shared through a file
         # descriptor that dies with this process if it exits before the parent reads
         if kind == "standin":
-            sh, W = _run(world, rank)
+            sh, W = _run(world, rank, exchange=exchange)
             q.put((rank, sh.owner, [w.numpy() for w in W]))
         else:
-            W, codes = _run_oracle(world, rank, set_ids)
+            W, codes = _run_oracle(world, rank, set_ids, exchange)
             q.put((rank, [w.numpy() for w in W], {k: v.numpy() for k, v in codes.items()}))
     finally:
         dist.destroy_process_group()
 
 
-def _spawn(world, kind="standin", set_ids=True):
+def _spawn(world, kind="standin", set_ids=True, exchange="weights"):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q, kind, set_ids))
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q, kind, set_ids, exchange))
              for r in range(world)]
     for p in procs:
         p.start()
@@ -197,3 +238,29 @@ def test_oracle_step_results_do_not_depend_on_the_world_size():
             assert torch.equal(codes[key], codes1[key])
     local = _spawn(2, "oracle", set_ids=False)
     assert any(not torch.equal(a, b) for a, b in zip(local[0][1], W1))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_update_exchange_ranks_end_with_the_single_process_weights(world):
+    """Exchanging the 16-bit update direction (with a per-matrix skip flag)
+    instead of the weights: every rank ends with the weights one process
+    computes, bit for bit, and the matrix whose gradient was non-finite in step
+    2 kept its step-1 weights on every rank."""
+    _, W_ref = _run(1, 0, exchange="update")
+    _, W_one = _run(1, 0, steps=1, exchange="update")
+    assert torch.equal(W_ref[0][3], W_one[0][3])
+    assert not torch.equal(W_ref[0][2], W_one[0][2])
+    for _, _, W in _spawn(world, exchange="update"):
+        for a, b in zip(W, W_ref):
+            assert torch.equal(a, b)
+
+
+def test_update_exchange_oracle_results_do_not_depend_on_the_world_size():
+    """The oracle's GRASP step with the bf16 O exchanged: weights and quantized
+    states after two steps are the same on 1 and 2 ranks."""
+    ref = _spawn(1, "oracle", exchange="update")[0]
+    for _, W, c in _spawn(2, "oracle", exchange="update"):
+        for a, b in zip(W, ref[1]):
+            assert torch.equal(a, b)
+        for key in c:
+            assert torch.equal(c[key], ref[2][key])
