@@ -301,7 +301,7 @@ def build_group(gm, w: WL.Workload, gi: int, nsf, pool: int, dev):
         for b in range(B):
             WL.gradient(w, base + b, t, m, n, device=dev, out=G[b])
         grads.append(G)
-    return dict(step=step, st=st, W=W, grads=grads, B=B, m=m, n=n)
+    return dict(step=step, st=st, W=W, grads=grads, B=B, m=m, n=n, ids=ids, ns=nsf(m, n))
 
 
 def our_launches(gm, w: WL.Workload, nsf, groups=None) -> int:
@@ -462,30 +462,39 @@ def measure(gm, w, groups, nsf, args, world, local, do_e2e):
     for g in groups:
         del g["Xc"], g["Xw"]
 
-    # ---- end to end through host buffers: H2D W and G, the step, D2H W
+    # ---- end to end through host buffers: every step copies W and G in from
+    # pinned host memory and the updated W back out, through the library's
+    # host-streamed step (offload.HostStreamedStep: chunks of the batch, copies
+    # in and out overlapping the steps of neighbouring chunks)
     e2e = None
     if do_e2e:
-        host = []
+        from bit_muon_optimizer_b200.offload import HostStreamedStep
+        runs = []
         for g in groups:
-            host.append(dict(W=g["W"].cpu().pin_memory(), G=g["grads"][-1].cpu().pin_memory()))
-        h2d = sum(h["W"].numel() * 4 + h["G"].numel() * h["G"].element_size() for h in host)
-        d2h = sum(h["W"].numel() * 4 for h in host)
+            hs = HostStreamedStep(g["B"], g["m"], g["n"], w.k, gdtype=w.gdtype, device=dev,
+                                  matrix_ids=g["ids"], mu=w.mu, eta=w.eta, wd=w.wd, T=w.T,
+                                  ns=g["ns"], seed=w.seed)
+            runs.append((hs, g["W"].cpu().pin_memory(), g["grads"][-1].cpu().pin_memory()))
+        h2d = sum(hs.h2d_bytes() for hs, _, _ in runs)
+        d2h = sum(hs.d2h_bytes() for hs, _, _ in runs)
         e_steps = 3 if h2d < 4e9 else 2
+        for hs, Wh, Gh in runs:            # one untimed step (first use of the streams)
+            hs(Wh, Gh)
         torch.cuda.synchronize()
         barrier(world)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record()
         for _ in range(e_steps):
-            for g, h in zip(groups, host):
-                g["W"].copy_(h["W"], non_blocking=True)
-                g["grads"][-1].copy_(h["G"], non_blocking=True)
-                g["step"](g["st"], g["W"], g["grads"][-1])
-                h["W"].copy_(g["W"], non_blocking=True)
+            for hs, Wh, Gh in runs:
+                hs(Wh, Gh)
         s1.record()
         torch.cuda.synchronize()
         barrier(world)
+        bad = [hs.status() for hs, _, _ in runs]
+        if any(bad):
+            raise RuntimeError(f"device status {bad}")
         e2e = (max_over_ranks(s0.elapsed_time(s1) / e_steps, world), h2d, d2h)
-        del host
+        del runs
     return dict(ms_step=ms_step, clocks=clk.summary(), ns_ms=ns_ms, ns_flops=ns_flops,
                 ns_launches=ns_launches, cod_ms=cod_ms, e2e=e2e, cub_ms=cub_ms,
                 cub_flops_dense=cub_flops_dense, codecs=codecs)
@@ -532,7 +541,9 @@ def run_single(gm, w, nsf, args, local):
     if all(r["e2e"] is not None for r in res):
         out["e2e"] = {"value": sum(r["e2e"][0] for r in res), "unit": UNIT,
                       "h2d_bytes_per_step": int(sum(r["e2e"][1] for r in res)),
-                      "d2h_bytes_per_step": int(sum(r["e2e"][2] for r in res))}
+                      "d2h_bytes_per_step": int(sum(r["e2e"][2] for r in res)),
+                      "api": "offload.HostStreamedStep per shape group: pinned host W and G in, "
+                             "the step, W out, in chunks of B/8 matrices on three streams"}
     out["graph"] = ("one CUDA graph per gradient slot, one stream per shape group"
                     + ("; shape groups measured one at a time (device memory), set time = sum"
                        if per_group else ""))

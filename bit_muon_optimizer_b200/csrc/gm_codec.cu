@@ -1599,6 +1599,7 @@ constexpr int kWsColGroups = kWsEpiWarps / 4;          // column groups of a blo
 constexpr int kWsCols = kGrid / kWsColGroups;          // columns per epilogue warp
 constexpr int kWsChunks = kWsCols / 16;
 constexpr int kWsThreads = (2 + kWsEpiWarps) * 32;
+constexpr int kQ8Per = kGrid * kMaxK / (kWsEpiWarps * 32);   // 8-bit codes per thread and job
 constexpr uint32_t kWsTile = 128 * 32 * 4;                        // one 128 x 32 fp32 box
 constexpr uint32_t kWsOps = 4 * kWsTile;                          // P hi, lo, R hi, lo
 constexpr uint32_t kWsStage = 4 * kWsTile;                        // M: four boxes
@@ -1888,21 +1889,35 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_residual_ws(
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       __syncwarp();
       if (lane == 0) ws_arrive(acc_empty(a));   // this warp is done with the accumulator
-      // 8-bit codes of P (block column 0) and R (block row 0), scales, step count
-      if (q8.Pmax && (bj == 0 || bi == 0)) {
+      // 8-bit codes of P's 128 rows of block row bi (in the block whose column is
+      // bi mod nb) and of R's 128 rows of block column bj (in the block whose row is
+      // bj mod mb): one job per block row and per block column, spread over the
+      // grid instead of piling up in block row 0 of each matrix; scales, step count
+      const bool pjob = bj == bi % nb, rjob = bi == bj % mb;
+      if (q8.Pmax && (pjob || rjob)) {
         const int nrows = min(kGrid, m - r0), ncols = min(kGrid, n - c0);
         for (int which = 0; which < 2; ++which) {
-          const bool doit = which == 0 ? bj == 0 : bi == 0;
-          if (!doit) continue;
+          if (!(which == 0 ? pjob : rjob)) continue;
           const unsigned* mx = which == 0 ? q8.Pmax : q8.Rmax;
           const float* src = which == 0 ? P + ((long long)b * m + r0) * k : R + ((long long)b * n + c0) * k;
           int8_t* dst = which == 0 ? q8.P8 + ((long long)b * m + r0) * k : q8.R8 + ((long long)b * n + c0) * k;
           const int cnt = (which == 0 ? nrows : ncols) * k;
-          for (int e = et; e < cnt; e += kWsEpiWarps * 32) {
-            const int l = e % k;
-            const float sv = __uint_as_float(mx[b * k + l]);
-            const float r127 = sv > 0.f ? __fdiv_rn(127.0f, sv) : 0.f;
-            dst[e] = code8(src[e], sv, r127);
+          // all of this thread's loads first (at most kQ8Per), then the codes
+          float v[kQ8Per];
+#pragma unroll
+          for (int u = 0; u < kQ8Per; ++u) {
+            const int e = et + u * kWsEpiWarps * 32;
+            v[u] = e < cnt ? __ldg(src + e) : 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < kQ8Per; ++u) {
+            const int e = et + u * kWsEpiWarps * 32;
+            if (e < cnt) {
+              const int l = e % k;
+              const float sv = __uint_as_float(__ldg(mx + b * k + l));
+              const float r127 = sv > 0.f ? __fdiv_rn(127.0f, sv) : 0.f;
+              dst[e] = code8(v[u], sv, r127);
+            }
           }
         }
         if (bi == 0 && bj == 0 && et < k) {

@@ -14,6 +14,8 @@ import os
 import subprocess
 import sys
 
+import pytest
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PKG = os.path.join(ROOT, "bit_muon_optimizer_b200")
 ORACLE = os.path.join(ROOT, "oracle")
@@ -150,3 +152,19 @@ def test_entry_point_bindings_check_tensors_before_passing_pointers():
     for call, msg in cases:
         with pytest.raises(ValueError, match=msg):
             call()
+
+
+def test_offload_chunk_bounds():
+    """offload.chunk_bounds covers 0 .. B-1 in order with runs of at most `chunk`."""
+    from bit_muon_optimizer_b200.offload import chunk_bounds
+    assert chunk_bounds(5, 2) == [(0, 2), (2, 4), (4, 5)]
+    assert chunk_bounds(4, 4) == [(0, 4)]
+    assert chunk_bounds(1, 8) == [(0, 1)]
+    for B in range(1, 20):
+        for c in range(1, 7):
+            bounds = chunk_bounds(B, c)
+            assert bounds[0][0] == 0 and bounds[-1][1] == B
+            assert all(b1 == a2 for (_, b1), (a2, _) in zip(bounds, bounds[1:]))
+            assert all(0 < b - a <= c for a, b in bounds)
+    with pytest.raises(ValueError):
+        chunk_bounds(0, 2)
