@@ -1675,7 +1675,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_residual_ws(
   __shared__ int abort_word;
   __shared__ float RMX[kWsColGroups][kGrid];
   __shared__ uint32_t CMX[4][kGrid];
-  __shared__ float smax_c[kGrid], r7c[kGrid];
+  __shared__ float smax_c[kGrid];
+  __shared__ __align__(16) float r7c[kGrid];
   volatile int* abort_flag = &abort_word;
   const uint32_t ops_full = tc_smem_u32(&bars[0]), ops_empty = tc_smem_u32(&bars[1]);
   auto m_full = [&](int s) { return tc_smem_u32(&bars[2 + s]); };
@@ -1867,22 +1868,41 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_residual_ws(
         __syncwarp();
         tc_ld16(tbase + 16 * ch, x);
         if (row_ok && c < n) {
-          uint32_t w[2] = {0u, 0u};
+          // q = rint(x fl(7 / s)) away from rounding ties; |x| <= s (s is the smaller of
+          // x's row and column maxima), so |q| <= 7 there without a clamp. A tie
+          // candidate anywhere in the chunk sends the thread through the IEEE division
+          // for those elements (rare: one branch per chunk instead of one per element).
+          const int cl0 = kWsCols * half + 16 * ch;
+          float r7v[16];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 v = reinterpret_cast<const float4*>(r7c + cl0)[u];
+            r7v[4 * u] = v.x; r7v[4 * u + 1] = v.y; r7v[4 * u + 2] = v.z; r7v[4 * u + 3] = v.w;
+          }
+          int q[16];
+          bool tie = false;
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const int cl = kWsCols * half + 16 * ch + e;
-            const float z = __fmul_rn(x[e], fmaxf(rr7, r7c[cl]));
+            const float z = __fmul_rn(x[e], fmaxf(rr7, r7v[e]));
             const float zr = rintf(z);
-            int q;
-            if (fabsf(__fsub_rn(z, zr)) < 0.49998474f) {   // 0.5 - 2^-16
-              q = (int)zr;
-            } else {
-              const float sv = fminf(rmax, smax_c[cl]);
-              q = sv > 0.f ? (int)rintf(__fmul_rn(__fdiv_rn(x[e], sv), 7.0f)) : 0;
-            }
-            q = max(-7, min(7, q));
-            w[e >> 3] |= (uint32_t)(q & 0xF) << (4 * (e & 7));
+            q[e] = (int)zr;
+            tie |= !(fabsf(__fsub_rn(z, zr)) < 0.49998474f);   // 0.5 - 2^-16
           }
+          if (tie) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float z = __fmul_rn(x[e], fmaxf(rr7, r7v[e]));
+              if (!(fabsf(__fsub_rn(z, rintf(z))) < 0.49998474f)) {
+                const float sv = fminf(rmax, smax_c[cl0 + e]);
+                const int qq = sv > 0.f ? (int)rintf(__fmul_rn(__fdiv_rn(x[e], sv), 7.0f)) : 0;
+                q[e] = max(-7, min(7, qq));
+              }
+            }
+          }
+          uint32_t w[2] = {0u, 0u};
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            asm("bfi.b32 %0, %1, %0, %2, 4;" : "+r"(w[e >> 3]) : "r"((uint32_t)q[e]), "r"(4 * (e & 7)));
           *reinterpret_cast<uint2*>(codes4 + ((long long)b * m + gi) * (n / 2) + c / 2) = make_uint2(w[0], w[1]);
         }
       }
