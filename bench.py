@@ -317,11 +317,11 @@ def our_launches(gm, w: WL.Workload, nsf, groups=None) -> int:
     return launches
 
 
-def measure(gm, w, groups, nsf, args, world, local, do_e2e):
-    """Times args.steps graph-replayed GRASP steps over `groups` (each group on
-    its own stream); then the step's two halves with CUDA events around each
-    (codec half: gm_grasp_state_update; NS half: gm_grasp_apply); the cuBLAS
-    comparator; and (if asked) steps end to end through pinned host buffers."""
+def time_steps(groups, args, world, local):
+    """args.steps graph-replayed GRASP steps over `groups` (each group on its own
+    stream, one graph per gradient slot) after args.warmup untimed ones; returns
+    (ms per step, max over ranks; clocks sampled during the timed region; the
+    fork helper and streams for further work on the same groups)."""
     dev = groups[0]["W"].device
     streams = [torch.cuda.Stream(device=dev) for _ in groups]
     main = torch.cuda.Stream(device=dev)        # graphs are captured on a side stream
@@ -375,6 +375,17 @@ def measure(gm, w, groups, nsf, args, world, local, do_e2e):
     if any(status):
         raise RuntimeError(f"device status {status}")
     del graphs
+    return ms_step, clk.summary(), fork, main
+
+
+def measure(gm, w, groups, nsf, args, world, local, do_e2e):
+    """Times args.steps graph-replayed GRASP steps over `groups` (time_steps);
+    then the step's two halves with CUDA events around each (codec half:
+    gm_grasp_state_update; NS half: gm_grasp_apply); the cuBLAS comparator; and
+    (if asked) steps end to end through pinned host buffers."""
+    dev = groups[0]["W"].device
+    ms_step, clocks, fork, main = time_steps(groups, args, world, local)
+    npool = len(groups[0]["grads"])
 
     # ---- the step's two halves, each bracketed by CUDA events on the stream
     # that launches it; groups one after another (no overlap between groups)
@@ -495,7 +506,7 @@ def measure(gm, w, groups, nsf, args, world, local, do_e2e):
             raise RuntimeError(f"device status {bad}")
         e2e = (max_over_ranks(s0.elapsed_time(s1) / e_steps, world), h2d, d2h)
         del runs
-    return dict(ms_step=ms_step, clocks=clk.summary(), ns_ms=ns_ms, ns_flops=ns_flops,
+    return dict(ms_step=ms_step, clocks=clocks, ns_ms=ns_ms, ns_flops=ns_flops,
                 ns_launches=ns_launches, cod_ms=cod_ms, e2e=e2e, cub_ms=cub_ms,
                 cub_flops_dense=cub_flops_dense, codecs=codecs)
 
@@ -543,13 +554,40 @@ def run_single(gm, w, nsf, args, local):
                       "h2d_bytes_per_step": int(sum(r["e2e"][1] for r in res)),
                       "d2h_bytes_per_step": int(sum(r["e2e"][2] for r in res)),
                       "api": "offload.HostStreamedStep per shape group: pinned host W and G in, "
-                             "the step, W out, in chunks of B/8 matrices on three streams"}
+                             "the step, W out, in chunks of about 2^25 elements (at most B/8 "
+                             "matrices) on three streams"}
     out["graph"] = ("one CUDA graph per gradient slot, one stream per shape group"
                     + ("; shape groups measured one at a time (device memory), set time = sum"
                        if per_group else ""))
     out["pool"] = pool
     out["codecs"] = res[0]["codecs"]
     out["launches"] = our_launches(gm, w, nsf) * args.steps
+    # the same set with the Gram form on its non-square shapes (--ns auto), graph
+    # replay only; batches whose forms do not change keep the time measured above
+    out["ns_auto"] = None
+    if args.ns == "standard" and not args.no_auto:
+        auto = ns_chooser(gm, "auto")
+        ms, clk_a = 0.0, []
+        for gis, r in zip(batches, res):
+            if all(auto(w.groups[gi].m, w.groups[gi].n) == nsf(w.groups[gi].m, w.groups[gi].n)
+                   for gi in gis):
+                ms += r["ms_step"]
+                continue
+            groups = [build_group(gm, w, gi, auto, pool, dev) for gi in gis]
+            t, c, _, _ = time_steps(groups, args, 1, local)
+            ms += t
+            if c:
+                clk_a.append(c["sm_mhz"])
+            del groups
+            torch.cuda.empty_cache()
+        out["ns_auto"] = {
+            "value": ms, "unit": UNIT,
+            "ns_per_group": ["gram" if auto(g.m, g.n) == gm.GM_NS_GRAM else "standard"
+                             for g in w.groups],
+            "sm_mhz": statistics.median(clk_a) if clk_a else None,
+            "what": "the same step and set with the Gram NS form (fp16) on non-square shapes "
+                    "and the standard form on square ones (the Gram NS page's FLOP rule), "
+                    "graph-replayed like the headline; not the headline"}
     return out
 
 
@@ -692,6 +730,7 @@ def run_ours(args, world, rank, local):
                                   what="gm_group_quant4 / gm_group_dequant4 (4bit-Muon-base) and "
                                        "gm_mulaw_quant4 / gm_mulaw_dequant4 (MuonQ mu-law, mu = 255) "
                                        "on the first shape group's fp32 M_t; not part of the step"),
+        "ns_auto": r["ns_auto"],
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
         "e2e": r["e2e"],
@@ -745,6 +784,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-auto", action="store_true",
+                    help="skip the extra timing of the set with Gram NS on non-square shapes")
     ap.add_argument("--profile", type=int, default=0,
                     help="run this many eager steps per shape group for a profiler, then exit")
     ap.add_argument("--group", type=int, default=-1, help="--profile: this shape group only")

@@ -30,22 +30,30 @@ def chunk_bounds(B: int, chunk: int) -> list[tuple[int, int]]:
     return [(a, min(B, a + chunk)) for a in range(0, B, chunk)]
 
 
+def default_chunk(B: int, m: int, n: int) -> int:
+    """Matrices per chunk: about 2^25 elements, between 1 and B / 8 rounded up."""
+    return max(1, min(-(-B // 8), -(-(1 << 25) // (m * n))))
+
+
 class HostStreamedStep:
     """``step(W_host, G_host)``: one GRASP step of B same-shape matrices whose fp32
     weights ``W_host`` [B, m, n] (updated in place) and gradients ``G_host``
     [B, m, n] (fp32, bf16 or fp16) are pinned host tensors; the state lives on
-    ``device``. ``chunk`` matrices per library call (default: B / 8 rounded up),
-    ``nbuf`` device buffer slots. The call returns once the work is queued; the
-    caller's current stream is made to wait for the last copy out. Further
-    keyword arguments are GraspStep's (mu, eta, wd, T, ns, seed, ...)."""
+    ``device``. ``chunk`` matrices per library call (default: about 2^25 elements,
+    at least one matrix and at most B / 8 rounded up: the copies of one chunk are
+    the part that nothing overlaps at either end); ``nbuf`` device buffer slots
+    (three let chunk i + 1 come in while chunk i steps and chunk i - 1 goes out).
+    The call returns once the work is queued; the caller's current stream is made
+    to wait for the last copy out. Further keyword arguments are GraspStep's (mu,
+    eta, wd, T, ns, seed, ...)."""
 
     def __init__(self, B: int, m: int, n: int, k: int, gdtype=torch.bfloat16, chunk: int | None = None,
-                 device=None, matrix_ids=None, nbuf: int = 2, **params):
+                 device=None, matrix_ids=None, nbuf: int = 3, **params):
         dev = torch.device(device or "cuda")
         if nbuf < 2:
             raise ValueError("nbuf must be >= 2")
         self.B, self.m, self.n, self.k, self.gdtype, self.nbuf = B, m, n, k, gdtype, nbuf
-        self.bounds = chunk_bounds(B, chunk or max(1, -(-B // 8)))
+        self.bounds = chunk_bounds(B, chunk or default_chunk(B, m, n))
         ids = list(range(B)) if matrix_ids is None else [int(i) for i in matrix_ids]
         if len(ids) != B:
             raise ValueError("matrix_ids: B indices expected")

@@ -168,3 +168,6 @@ def test_offload_chunk_bounds():
             assert all(0 < b - a <= c for a, b in bounds)
     with pytest.raises(ValueError):
         chunk_bounds(0, 2)
+    from bit_muon_optimizer_b200.offload import default_chunk
+    assert default_chunk(56, 18944, 3584) == 1 and default_chunk(56, 3584, 3584) == 3
+    assert default_chunk(48, 768, 768) == 6 and default_chunk(1, 256, 512) == 1
