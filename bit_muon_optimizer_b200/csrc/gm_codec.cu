@@ -705,7 +705,6 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_pipe(
           }
           const float o = ok ? __fadd_rn(__fmul_rn(mu, mp), gv) : 0.f;
           acc[nt][2 * h + e] = o;
-          bad |= !(fabsf(o) <= 3.402823466e38f);
           nsq = fmaf(o, o, nsq);
         }
       }
@@ -716,6 +715,14 @@ __global__ void __launch_bounds__(kRBT, 2) k_rebuild_pipe(
           dst[u] = make_float4(acc[2 * u][2 * h], acc[2 * u][2 * h + 1], acc[2 * u + 1][2 * h],
                                acc[2 * u + 1][2 * h + 1]);
       }
+    }
+    // a non-finite M_t makes nsq non-finite; only then (or when the finite squares
+    // overflowed) are the thread's 32 values checked one by one
+    if (!(fabsf(nsq) <= 3.402823466e38f)) {
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) bad |= !(fabsf(acc[nt][r]) <= 3.402823466e38f);
     }
     // |M|^2 partial of this warp's 16 x 64 part of the tile (fixed shuffle tree)
     double wsq = (double)nsq;
