@@ -242,6 +242,30 @@ GEMM_TRAFFIC = [
 ]
 
 
+# Thread instructions per element of the codec half (the nine kernels of
+# gm_grasp_state_update, k = 32), from the committed ncu summary of the codec
+# passes (`smsp__inst_executed.sum` x 32 / elements on the 18944 x 3584 shape);
+# valid only for the gm_codec.cu source it was captured on.
+CODEC_INSTR = [
+    {"configs": [4], "thread_instr_per_element": 115.83,
+     "source_sha256": "d316fb877864d2875efcd4c54be536a042d9a13852e4f9dbf7a4700e39cf421f"},
+]
+
+
+def codec_instr(config: int):
+    import hashlib
+    path = os.path.join(ROOT, "bit_muon_optimizer_b200", "csrc", "gm_codec.cu")
+    try:
+        with open(path, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    for t in CODEC_INSTR:
+        if sha == t["source_sha256"] and config in t["configs"]:
+            return t["thread_instr_per_element"]
+    return None
+
+
 def gemm_traffic(config: int, ns: str):
     import hashlib
     path = os.path.join(ROOT, "bit_muon_optimizer_b200", "csrc", "gm_gemm.cu")
@@ -650,6 +674,21 @@ def run_sharded(gm, w, nsf, args, world, rank, local):
     return ms_total, clk, launches * args.steps, owned
 
 
+def codec_issue(config: int, elements: int, ms: float, clocks):
+    """The codec half against its instruction-issue bound: thread instructions per
+    element (ncu) x elements / time, against 148 SMs x 4 schedulers x 32 lanes at
+    the SM clock sampled during the timed region (the passes are issue-bound, not
+    DRAM-bound). None without a matching capture or clock record."""
+    ipe = codec_instr(config)
+    if ipe is None or not clocks or not clocks.get("sm_mhz"):
+        return None
+    achieved = ipe * elements / (ms * 1e-3)
+    peak = 148 * 4 * 32 * clocks["sm_mhz"] * 1e6
+    return {"bound": "issue", "thread_instr_per_element": ipe, "achieved_tinstr_s": achieved,
+            "peak_tinstr_s": peak, "frac": achieved / peak,
+            "peak_kind": "148 SMs x 4 schedulers x 32 lanes x median SM clock of the timed region"}
+
+
 def run_ours(args, world, rank, local):
     from bit_muon_optimizer_b200 import gmuon as gm
     w = WL.WORKLOADS[args.config]
@@ -723,7 +762,8 @@ def run_ours(args, world, rank, local):
                   "bytes": r["codec_bytes"],
                   "kernels": "the codec half of the step (gm_grasp_state_update: 9 kernels per "
                              "group), CUDA events around it; algorithmic bytes G + old and new "
-                             "codes and scales + the 16-bit NS input"},
+                             "codes and scales + the 16-bit NS input",
+                  "issue": codec_issue(args.config, elements, r["cod_ms"], r["clocks"])},
         "step_roofline": {"ms": t_roof, "frac": t_roof / r["ms_step"], "flops": step_flops,
                           "bytes": step_bytes},
         "standalone_codecs": dict(r["codecs"] or {}, peak_gbs=hbm,

@@ -839,42 +839,43 @@ __global__ void __launch_bounds__(kThreads) k_orth_gram(int m, int k, int csplit
 // shuffle from lane c), in ascending j as the textbook left-looking sums do.
 // Writes L below the diagonal and the reciprocal diagonal on it (0 for a dead
 // column) for the forward substitution in (c); NS scale 1 / (|M_t|_F + eps).
-__global__ void __launch_bounds__(32) k_orth_chol(int k, int rsplit, const double* __restrict__ gram_part,
+constexpr int kCholThreads = 256;
+__global__ void __launch_bounds__(kCholThreads) k_orth_chol(int k, int rsplit, const double* __restrict__ gram_part,
                                                    double* __restrict__ Lmat,
                                                    const double* __restrict__ norm2_part, int ntiles,
                                                    float eps, float* __restrict__ scale,
                                                    const int32_t* skip) {
   if (skip && *skip) return;
-  const int b = blockIdx.x, lane = threadIdx.x;
+  const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   constexpr unsigned kAll = 0xffffffffu;
-  // row `lane` of the Gram, summed over the row splits in order
+  __shared__ double Gs[kMaxK][kMaxK + 1];
+  __shared__ double wsum[kCholThreads / 32];
+  // the Gram, each entry summed over the row splits in order (all the block's
+  // threads, several splits' loads in flight: these sums are latency-bound)
+  for (int e = t; e < k * k; e += kCholThreads) {
+    const double* gp = gram_part + (long long)b * rsplit * k * k + e;
+    double acc = 0.0;
+#pragma unroll 8
+    for (int p = 0; p < rsplit; ++p) acc += gp[(long long)p * k * k];
+    Gs[e / k][e % k] = acc;
+  }
+  // |M_t|^2 from the rebuild's partials: 256 thread-strided chains, then a fixed tree
+  double nsq = 0.0;
+  const double* np = norm2_part + (long long)b * ntiles;
+#pragma unroll 8
+  for (int p = t; p < ntiles; p += kCholThreads) nsq += np[p];
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) nsq += __shfl_xor_sync(kAll, nsq, off);
+  if (lane == 0) wsum[warp] = nsq;
+  __syncthreads();
+  if (warp != 0) return;   // the factorisation is one warp's (no block barrier follows)
+  double ns2 = 0.0;
+#pragma unroll
+  for (int w = 0; w < kCholThreads / 32; ++w) ns2 += wsum[w];
+  // row `lane` of the Gram
   double g[kMaxK];
 #pragma unroll
-  for (int c = 0; c < kMaxK; ++c) g[c] = 0.0;
-  if (lane < k) {
-    const double* gp = gram_part + (long long)b * rsplit * k * k + (long long)lane * k;
-#pragma unroll 2
-    for (int p = 0; p < rsplit; ++p) {
-#pragma unroll
-      for (int c = 0; c < kMaxK; ++c)
-        if (c < k) g[c] += gp[(long long)p * k * k + c];
-    }
-  }
-  // |M_t|^2 from the rebuild's partials: eight lane-strided chains, then a fixed tree
-  double nsq[8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) nsq[u] = 0.0;
-  const double* np = norm2_part + (long long)b * ntiles;
-  for (int p0 = 0; p0 < ntiles; p0 += 256) {
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int p = p0 + 32 * u + lane;
-      if (p < ntiles) nsq[u] += np[p];
-    }
-  }
-  double ns2 = ((nsq[0] + nsq[1]) + (nsq[2] + nsq[3])) + ((nsq[4] + nsq[5]) + (nsq[6] + nsq[7]));
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) ns2 += __shfl_xor_sync(kAll, ns2, off);
+  for (int c = 0; c < kMaxK; ++c) g[c] = (lane < k && c < k) ? Gs[lane][c] : 0.0;
   // dead-column tolerance: (1e-6 * max column norm)^2
   double maxn2 = 0.0;
 #pragma unroll
@@ -2234,7 +2235,7 @@ cudaError_t launch_orth(int B, int m, int k, int csplit, const float* Ppart, dou
   k_orth_gram<<<dim3(rs, B), kThreads, 0, s>>>(m, k, csplit, rs, Ppart, Ptil, gram_part, skip);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_orth_chol<<<B, 32, 0, s>>>(k, rs, gram_part, Lmat, norm2_part, ntiles, eps, scale, skip);
+  k_orth_chol<<<B, kCholThreads, 0, s>>>(k, rs, gram_part, Lmat, norm2_part, ntiles, eps, scale, skip);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int kp = factor_width(k);

@@ -62,3 +62,23 @@ def test_peaks_come_from_the_measured_file_when_present():
         assert (hbm, bf16) == (d["hbm_gbs"], d["bf16_tflops"])
     else:
         assert kind == "fallback" and (hbm, bf16, bf16_sus) == (6650.0, 1590.0, 1400.0)
+
+
+def test_codec_issue_roofline_needs_a_matching_capture(monkeypatch):
+    """The codec half's issue figure uses the instructions per element of a capture
+    of the same gm_codec.cu source, and none otherwise."""
+    import hashlib
+    path = os.path.join(os.path.dirname(bench.__file__), "bit_muon_optimizer_b200", "csrc", "gm_codec.cu")
+    sha = hashlib.sha256(open(path, "rb").read()).hexdigest()
+    clocks = {"sm_mhz": 1500.0}
+    monkeypatch.setattr(bench, "CODEC_INSTR", [{"configs": [4], "source_sha256": "0" * 64,
+                                                "thread_instr_per_element": 100.0}])
+    assert bench.codec_issue(4, 10 ** 9, 50.0, clocks) is None
+    monkeypatch.setattr(bench, "CODEC_INSTR", [{"configs": [4], "source_sha256": sha,
+                                                "thread_instr_per_element": 100.0}])
+    r = bench.codec_issue(4, 10 ** 9, 50.0, clocks)
+    assert r["achieved_tinstr_s"] == 100.0 * 10 ** 9 / 0.05
+    assert r["peak_tinstr_s"] == 148 * 4 * 32 * 1500.0e6
+    assert abs(r["frac"] - r["achieved_tinstr_s"] / r["peak_tinstr_s"]) < 1e-12
+    assert bench.codec_issue(2, 10 ** 9, 50.0, clocks) is None        # another workload
+    assert bench.codec_issue(4, 10 ** 9, 50.0, None) is None          # no clock record
