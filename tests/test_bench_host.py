@@ -82,3 +82,13 @@ def test_codec_issue_roofline_needs_a_matching_capture(monkeypatch):
     assert abs(r["frac"] - r["achieved_tinstr_s"] / r["peak_tinstr_s"]) < 1e-12
     assert bench.codec_issue(2, 10 ** 9, 50.0, clocks) is None        # another workload
     assert bench.codec_issue(4, 10 ** 9, 50.0, None) is None          # no clock record
+
+
+def test_ns_auto_picks_gram_for_non_square_shapes():
+    """--ns auto: the Gram form exactly where the Gram NS page's FLOP rule favours it
+    (aspect ratio above 1), the standard form on square matrices."""
+    assert bench.ns_name("auto", 768, 768) == "standard"
+    assert bench.ns_name("auto", 2048, 768) == "gram"
+    assert bench.ns_name("auto", 3584, 18944) == "gram"
+    assert bench.ns_name("standard", 2048, 768) == "standard"
+    assert bench.ns_name("gram", 768, 768) == "gram"
