@@ -1002,12 +1002,24 @@ __global__ void __launch_bounds__(kThreads) k_orth_apply(int m, int k, const dou
 // g + 8 h of m-tile mt in the A fragment of M^T (tf32 mma.m16n8k8, 3xTF32
 // against P's precomputed fragments). fp32 sums over at most 1024 rows per
 // split, the four row warps added in order, fp64 across splits.
-template <int KP>
+// Two fp32 values rounded to a packed pair of 16-bit floats (a in the low half).
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_h16x2(float a, float b) {
+  if constexpr (F16) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  } else {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+}
+
+template <int KP, bool F16>   // F16: the NS input in fp16 (Gram NS), else bf16
 __global__ void __launch_bounds__(kThreads, 2) k_backproject(int m, int n, int k, int rsplit,
                                                               const float* __restrict__ M,
                                                               const uint32_t* __restrict__ PB,
                                                               const float* __restrict__ scale,
-                                                              uint16_t* __restrict__ X16, int f16,
+                                                              uint16_t* __restrict__ X16,
                                                               double* __restrict__ Rpart,
                                                               const int32_t* skip) {
   if (skip && *skip) return;
@@ -1109,8 +1121,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_backproject(int m, int n, int k
             if (gi < m && colok) {
               const float4 x = v[s][hh];
               uint2 w;
-              w.x = (uint32_t)float_to_h16(x.x * sc, f16) | ((uint32_t)float_to_h16(x.y * sc, f16) << 16);
-              w.y = (uint32_t)float_to_h16(x.z * sc, f16) | ((uint32_t)float_to_h16(x.w * sc, f16) << 16);
+              w.x = pack_h16x2<F16>(x.x * sc, x.y * sc);
+              w.y = pack_h16x2<F16>(x.z * sc, x.w * sc);
               *reinterpret_cast<uint2*>(Xb + (long long)gi * n + cq) = w;
             }
           }
@@ -1122,10 +1134,12 @@ __global__ void __launch_bounds__(kThreads, 2) k_backproject(int m, int n, int k
           for (int hh = 0; hh < 2; ++hh) {
             const int ii = 8 * s + tq + 4 * hh;
             const float4 x = v[s][hh];
-            Xt[warp][4 * g][ii] = float_to_h16(x.x * sc, f16);
-            Xt[warp][4 * g + 1][ii] = float_to_h16(x.y * sc, f16);
-            Xt[warp][4 * g + 2][ii] = float_to_h16(x.z * sc, f16);
-            Xt[warp][4 * g + 3][ii] = float_to_h16(x.w * sc, f16);
+            const uint32_t p01 = pack_h16x2<F16>(x.x * sc, x.y * sc);
+            const uint32_t p23 = pack_h16x2<F16>(x.z * sc, x.w * sc);
+            Xt[warp][4 * g][ii] = (uint16_t)(p01 & 0xFFFFu);
+            Xt[warp][4 * g + 1][ii] = (uint16_t)(p01 >> 16);
+            Xt[warp][4 * g + 2][ii] = (uint16_t)(p23 & 0xFFFFu);
+            Xt[warp][4 * g + 3][ii] = (uint16_t)(p23 >> 16);
           }
         __syncwarp();
         if (c0 + lane < n) {
@@ -2076,15 +2090,19 @@ cudaError_t launch_backproject_t(int B, int m, int n, int k, const float* M, con
                                  const int32_t* skip, cudaStream_t s) {
   const int rs = backproject_row_splits(B, m, n);
   const size_t smem = (size_t)2 * 8 * 8 * 32 * sizeof(float4);
-  static DeviceOnce attr;
+  static DeviceOnce attr_bf16, attr_f16;   // one latch per kernel instantiation
   {
-    const cudaError_t e = smem_attr_once(attr, k_backproject<KP>, smem);
+    const cudaError_t e = f16 ? smem_attr_once(attr_f16, k_backproject<KP, true>, smem)
+                              : smem_attr_once(attr_bf16, k_backproject<KP, false>, smem);
     if (e != cudaSuccess) return e;
   }
   dim3 grid(cdiv(n, 64), rs, B);
-  k_backproject<KP><<<grid, kThreads, smem, s>>>(m, n, k, rs, M, PB, scale,
-                                                 static_cast<uint16_t*>(X16), f16 ? 1 : 0, Rpart,
-                                                 skip);
+  if (f16)
+    k_backproject<KP, true><<<grid, kThreads, smem, s>>>(m, n, k, rs, M, PB, scale,
+                                                         static_cast<uint16_t*>(X16), Rpart, skip);
+  else
+    k_backproject<KP, false><<<grid, kThreads, smem, s>>>(m, n, k, rs, M, PB, scale,
+                                                          static_cast<uint16_t*>(X16), Rpart, skip);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g2((int)cdivll((long long)cdiv(n, 64) * 64 * KP, kThreads), B);
