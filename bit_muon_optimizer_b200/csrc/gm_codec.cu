@@ -1906,8 +1906,11 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_residual_ws(
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const float z = __fmul_rn(x[e], fmaxf(rr7, r7v[e]));
-            const float zr = rintf(z);
-            q[e] = (int)zr;
+            // rint(z) by adding and removing 1.5 * 2^23 (exact round-to-nearest-even
+            // for |z| < 2^22) on the FMA pipe; the integer is the sum's low bits
+            const float zm = __fadd_rn(z, 12582912.0f);
+            const float zr = __fsub_rn(zm, 12582912.0f);
+            q[e] = __float_as_int(zm) - 0x4B400000;
             tie |= !(fabsf(__fsub_rn(z, zr)) < 0.49998474f);   // 0.5 - 2^-16
           }
           if (tie) {
