@@ -247,8 +247,8 @@ GEMM_TRAFFIC = [
 # passes (`smsp__inst_executed.sum` x 32 / elements on the 18944 x 3584 shape);
 # valid only for the gm_codec.cu source it was captured on.
 CODEC_INSTR = [
-    {"configs": [4], "thread_instr_per_element": 115.83,
-     "source_sha256": "d316fb877864d2875efcd4c54be536a042d9a13852e4f9dbf7a4700e39cf421f"},
+    {"configs": [4], "thread_instr_per_element": 116.03,
+     "source_sha256": "fd2224401ae4389c160824c579386bf3e9a52b77da131c7e9f1587483b3d7a59"},
 ]
 
 
