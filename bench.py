@@ -237,8 +237,8 @@ GRAD_POOL = 6   # distinct gradient buffers per group, used cyclically step afte
 # k_gemm summaries under profiles/); reported only while gm_gemm.cu is the source
 # that capture measured.
 GEMM_TRAFFIC = [
-    {"config": 4, "ns": "standard", "bytes_per_launch": 10683.4e6,
-     "source_sha256": "6fba3398bf3fcb13a0d3d5b362e00bf5493841fc890ff6a46a3a55ae9781dae0"},
+    {"config": 4, "ns": "standard", "bytes_per_launch": 8868.3e6,
+     "source_sha256": "d8cac0d9bacf42c2a06c6af7b09cd89c2a32c210593a66093925bae5ae9b91a4"},
 ]
 
 
@@ -624,13 +624,15 @@ def run_sharded(gm, w, nsf, args, world, rank, local):
     torch.distributed). Returns the max over ranks of the summed group times."""
     from bit_muon_optimizer_b200 import sharding as S
     dev = torch.device("cuda", local)
-    update = S.grasp_update(w.eta, w.wd) if args.exchange == "update" else None
+    update = S.grasp_update(w.eta, w.wd) if args.exchange in ("update", "peer") else None
+    peer = args.exchange == "peer"
     ms_total, clocks, launches, owned = 0.0, [], 0, []
     for gi, g in enumerate(w.groups):
         base = w.group_base(gi)
         make = S.grasp_make_step(w.k, dev, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=nsf(g.m, g.n),
                                  seed=w.seed)
-        sh = S.ShardedStep([(g.m, g.n, g.count)], world, rank, make, first_index=base, update=update)
+        sh = S.ShardedStep([(g.m, g.n, g.count)], world, rank, make, first_index=base, update=update,
+                           peer=peer)
         W = torch.empty((g.count, g.m, g.n), dtype=torch.float32, device=dev)
         grads = []
         for b in range(g.count):
@@ -663,6 +665,10 @@ def run_sharded(gm, w, nsf, args, world, rank, local):
             launches += our_launches(gm, w, nsf, [(g.m, g.n)])
         if update is not None:
             launches += 1                              # k_weight_update on every rank
+        torch.cuda.synchronize()
+        barrier(world)
+        sh.close()           # unmap the other ranks' receive buffers before anyone frees them
+        barrier(world)
         del sh, W, grads
         torch.cuda.empty_cache()
     clk = None
@@ -710,11 +716,14 @@ def run_ours(args, world, rank, local):
     if world > 1:
         ms_step, clocks, launches, owned = run_sharded(gm, w, nsf, args, world, rank, local)
         if rank == 0:
-            what = ("the owners' bf16 update directions O (2 B per element) and skip flags, "
-                    "then every rank's weight update" if args.exchange == "update"
-                    else "the owners' updated fp32 weights (4 B per element)")
+            what = {"update": "the owners' bf16 update directions O (2 B per element) and skip "
+                              "flags, then every rank's weight update",
+                    "peer": "none: the owners' last NS product stores O (bf16) and the skip flags "
+                            "into every rank's receive buffers over NVLink (CUDA IPC), then every "
+                            "rank's weight update",
+                    "weights": "the owners' updated fp32 weights (4 B per element)"}[args.exchange]
             config.update(parallelism=f"ownership sharding x{world}: LPT owners per shape group, "
-                                      f"one NCCL all-gather per group of {what}",
+                                      f"exchange per group: {what}",
                           graph="eager launches, shape groups one at a time, set time = sum",
                           owned_per_group_rank0=owned)
             line = {"metric": METRIC, "value": ms_step, "unit": UNIT, "n_gpus": world,
@@ -819,8 +828,10 @@ def main():
     ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--ns", choices=["standard", "gram", "auto"], default="standard",
                     help="NS form; auto: Gram NS for non-square shapes, standard for square ones")
-    ap.add_argument("--exchange", choices=["update", "weights"], default="update",
-                    help="N > 1: all-gather the bf16 update direction (default) or the fp32 weights")
+    ap.add_argument("--exchange", choices=["update", "peer", "weights"], default="update",
+                    help="N > 1: all-gather the bf16 update direction (default), store it into "
+                         "every rank's buffers from the NS epilogue (peer), or all-gather the fp32 "
+                         "weights")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")

@@ -2,6 +2,7 @@
 // layout and the enqueueing of the step's kernels on the caller's stream.
 
 #include <stdarg.h>
+#include <atomic>
 #include <cmath>
 #include <stdio.h>
 #include <string.h>
@@ -562,6 +563,84 @@ gm_status gm_grasp_orth(int B, int m, int n, const gm_grasp_params* prm, const g
                         w + L.ns, status, status, s));
   else
     GM_CUDA(run_ns_standard(B, m, n, X, tab, prm->T, out, w + L.ns, status, status, s));
+  return GM_OK;
+}
+
+gm_status gm_grasp_orth_peers(int B, int m, int n, const gm_grasp_params* prm,
+                              const gm_grasp_state* st, void* const* peer_O,
+                              int32_t* const* peer_flags, int npeers, const int64_t* dst_index,
+                              gm_dtype odt, void* ws, size_t ws_bytes, gm_stream_t stream) {
+  GM_CHECK_ARG(odt == GM_F32 || odt == GM_BF16 || odt == GM_F16, "bad odt");
+  GM_CHECK_ARG(npeers >= 1 && npeers <= kMaxPeers, "npeers=%d out of [1, %d]", npeers, kMaxPeers);
+  GM_CHECK_ARG(peer_O && peer_flags, "NULL peer arrays");
+  for (int r = 0; r < npeers; ++r) {
+    GM_CHECK_ARG(peer_O[r] && peer_flags[r], "NULL receive buffer of peer %d", r);
+    GM_CHECK_ARG(al16(peer_O[r]) && al16(peer_flags[r]), "device arrays must be 16-byte aligned");
+  }
+  GM_CHECK_ARG(al16(dst_index), "device arrays must be 16-byte aligned");
+  StepLayout L;
+  const gm_status chk =
+      step_checks(B, m, n, prm, st, nullptr, false, nullptr, false, GM_F32, ws, ws_bytes, &L);
+  if (chk != GM_OK) return chk;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* X = reinterpret_cast<uint16_t*>(w + L.X);
+  int32_t* status = st->dev_status;
+  float tab[3 * GM_MAX_T];
+  expand_abc(prm->abc, prm->T, tab);
+  // worked step 6 up to O = NS(M_t), stored straight into every receive buffer
+  NsOutput out{0, nullptr, (int)odt, nullptr, 0.f, 0.f};
+  out.npeers = npeers;
+  for (int r = 0; r < npeers; ++r) out.peer[r] = peer_O[r];
+  out.dst_index = dst_index;
+  if (prm->ns == GM_NS_GRAM)
+    GM_CUDA(run_ns_gram(B, m, n, X, tab, prm->T, prm->restart_after, prm->n_restart, out,
+                        w + L.ns, status, status, s));
+  else
+    GM_CUDA(run_ns_standard(B, m, n, X, tab, prm->T, out, w + L.ns, status, status, s));
+  GM_CUDA(launch_put_status(B, npeers, peer_flags, dst_index, status, s));
+  return GM_OK;
+}
+
+static_assert(sizeof(gm_ipc_handle) >= sizeof(cudaIpcMemHandle_t), "IPC handle size");
+
+gm_status gm_ipc_export(const void* dev_ptr, gm_ipc_handle* handle, size_t* offset) {
+  GM_CHECK_ARG(dev_ptr && handle && offset, "NULL argument");
+  using AddrRange = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+  static std::atomic<AddrRange> fn{nullptr};
+  AddrRange f = fn.load(std::memory_order_acquire);
+  if (!f) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return set_error(GM_E_UNSUPPORTED, "cuMemGetAddressRange is not available");
+    f = reinterpret_cast<AddrRange>(p);
+    fn.store(f, std::memory_order_release);
+  }
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (f(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS)
+    return set_error(GM_E_ARG, "not a device allocation");
+  cudaIpcMemHandle_t h;
+  GM_CUDA(cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)));
+  memset(handle, 0, sizeof(*handle));
+  memcpy(handle->bytes, &h, sizeof(h));
+  *offset = (size_t)(reinterpret_cast<CUdeviceptr>(dev_ptr) - base);
+  return GM_OK;
+}
+
+gm_status gm_ipc_open(const gm_ipc_handle* handle, void** base) {
+  GM_CHECK_ARG(handle && base, "NULL argument");
+  cudaIpcMemHandle_t h;
+  memcpy(&h, handle->bytes, sizeof(h));
+  GM_CUDA(cudaIpcOpenMemHandle(base, h, cudaIpcMemLazyEnablePeerAccess));
+  return GM_OK;
+}
+
+gm_status gm_ipc_close(void* base) {
+  GM_CHECK_ARG(base, "NULL argument");
+  GM_CUDA(cudaIpcCloseMemHandle(base));
   return GM_OK;
 }
 

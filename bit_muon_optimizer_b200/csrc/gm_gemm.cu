@@ -91,6 +91,7 @@ struct GemmParams {
   int mode;
   int transpose_out;           // EPI_OUT / EPI_WUPDATE: natural = transpose of the tile
   void* O; int odt; long long o_bs; int ldo;
+  int npeers; void* peer[kMaxPeers]; const int64_t* dst_index;   // EPI_OUT to several destinations
   float* W; long long w_bs; int ldw; float eta, wd;
   const int32_t* skip;
   int32_t* err;
@@ -550,7 +551,14 @@ __device__ __forceinline__ void epilogue_out_slab(const GemmParams& p, uint8_t* 
       for (int u = 0; u < NB; ++u) {
         if (!okc[u]) continue;
         if (p.mode == EPI_OUT) {
-          store4_from_float(p.O, (long long)tc.bz * p.o_bs + off[u], p.odt, val[u]);
+          if (p.npeers == 0) {
+            store4_from_float(p.O, (long long)tc.bz * p.o_bs + off[u], p.odt, val[u]);
+          } else {   // every rank's receive buffer, peers' over NVLink (plain stores)
+            const long long mb = p.dst_index ? p.dst_index[tc.bz] : tc.bz;
+#pragma unroll
+            for (int r = 0; r < kMaxPeers; ++r)
+              if (r < p.npeers) store4_from_float(p.peer[r], mb * p.o_bs + off[u], p.odt, val[u]);
+          }
         } else {
           float4 w = wv[u];
           w.x -= p.eta * (val[u].x + p.wd * w.x);
@@ -1058,6 +1066,9 @@ cudaError_t leftmul(const Ns& c, const uint16_t* S, const uint16_t* X, float alp
     if (out->mode == 0) {
       p.mode = EPI_OUT;
       p.O = out->O; p.odt = out->odt; p.o_bs = (long long)c.vN * c.vMp; p.ldo = ld;
+      p.npeers = out->npeers;
+      for (int r = 0; r < kMaxPeers; ++r) p.peer[r] = r < out->npeers ? out->peer[r] : nullptr;
+      p.dst_index = out->dst_index;
     } else {
       p.mode = EPI_WUPDATE;
       p.W = out->W; p.w_bs = (long long)c.vN * c.vMp; p.ldw = ld;

@@ -83,6 +83,11 @@ cudaError_t launch_residual_ws(int B, int m, int n, int k, const float* X, const
                                float* Pscale, int8_t* R8, float* Rscale, int64_t* step,
                                const int32_t* skip, int32_t* status, cudaStream_t s);
 
+// flags[r][dst_index[b]] = *status for every destination r < npeers (<= kMaxPeers)
+// and matrix b < B (dst_index NULL: b).
+cudaError_t launch_put_status(int B, int npeers, int32_t* const* flags, const int64_t* dst_index,
+                              const int32_t* status, cudaStream_t s);
+
 // W <- W - eta (O + wd W) (O in odt: GM_F32, GM_BF16 or GM_F16); matrix b is
 // left alone when skip && skip[b * skip_stride].
 cudaError_t launch_weight_update(int B, int m, int n, float eta, float wd, const void* O, int odt,
@@ -130,12 +135,19 @@ cudaError_t launch_ns_prep(int B, int m, int n, const void* X, int xdt, float ep
 int ns_prep_parts(int m, int n);
 
 // ---- tensor-core Newton-Schulz chains (gm_gemm.cu) --------------------------
+constexpr int kMaxPeers = 8;   // destinations of one O store (ranks of a node)
 struct NsOutput {
   int mode;            // 0: write O (dtype odt), 1: W -= eta (O + wd W)
   void* O;
   int odt;
   float* W;
   float eta, wd;
+  // mode 0 only: with npeers > 0, O goes to every peer[r] (device pointers, other
+  // GPUs' memory included) instead of O, matrix b of the batch at index
+  // dst_index[b] (device int64) of each [.][m][n] destination
+  int npeers;
+  void* peer[kMaxPeers];
+  const int64_t* dst_index;
 };
 
 size_t ns_standard_ws_bytes(int B, int m, int n);

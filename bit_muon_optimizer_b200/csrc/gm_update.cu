@@ -7,6 +7,9 @@
 // the bytes of the fp32 weights, and every rank then applies the same update
 // to its copy of W).
 //
+// k_put_status hands a batch's device status (the step's skip flag) to the ranks
+// that receive its O, one int32 per matrix.
+//
 // HBM-bound: W read and written (8 B per element) and O read (2 or 4 B). Each
 // thread moves one float4 of W and the matching four values of O per trip; the
 // grid's y index is the matrix, so a matrix that its skip flag marks keeps its
@@ -67,7 +70,32 @@ __global__ void __launch_bounds__(kUpdThreads) k_weight_update(long long per4, f
   }
 }
 
+struct PeerFlags {
+  int32_t* flag[kMaxPeers];
+};
+
+// Every destination's flag of every matrix of the batch gets the batch's status.
+__global__ void k_put_status(int B, int npeers, const __grid_constant__ PeerFlags pf,
+                             const int64_t* __restrict__ dst_index, const int32_t* __restrict__ status) {
+  const int32_t v = *status;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    const long long at = dst_index ? dst_index[b] : b;
+#pragma unroll
+    for (int r = 0; r < kMaxPeers; ++r)
+      if (r < npeers) pf.flag[r][at] = v;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_put_status(int B, int npeers, int32_t* const* flags, const int64_t* dst_index,
+                              const int32_t* status, cudaStream_t s) {
+  if (npeers < 1 || npeers > kMaxPeers) return cudaErrorInvalidValue;
+  PeerFlags pf{};
+  for (int r = 0; r < npeers; ++r) pf.flag[r] = flags[r];
+  k_put_status<<<1, 256, 0, s>>>(B, npeers, pf, dst_index, status);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_weight_update(int B, int m, int n, float eta, float wd, const void* O, int odt,
                                  float* W, const int32_t* skip, int skip_stride, cudaStream_t s) {

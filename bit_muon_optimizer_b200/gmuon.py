@@ -88,6 +88,18 @@ _sig("gm_grasp_apply", c_int, [c_int, c_int, c_int, ctypes.POINTER(GraspParams),
 _sig("gm_grasp_orth", c_int, [c_int, c_int, c_int, ctypes.POINTER(GraspParams),
                               ctypes.POINTER(GraspStateC), vp, c_int, vp, c_size_t, vp])
 _sig("gm_weight_update", c_int, [c_int, c_int, c_int, c_float, c_float, vp, c_int, vp, vp, c_int, vp])
+_sig("gm_grasp_orth_peers", c_int, [c_int, c_int, c_int, ctypes.POINTER(GraspParams),
+                                    ctypes.POINTER(GraspStateC), ctypes.POINTER(vp),
+                                    ctypes.POINTER(vp), c_int, vp, c_int, vp, c_size_t, vp])
+
+
+class IpcHandle(ctypes.Structure):
+    _fields_ = [("bytes", ctypes.c_ubyte * 64)]
+
+
+_sig("gm_ipc_export", c_int, [vp, ctypes.POINTER(IpcHandle), ctypes.POINTER(c_size_t)])
+_sig("gm_ipc_open", c_int, [ctypes.POINTER(IpcHandle), ctypes.POINTER(vp)])
+_sig("gm_ipc_close", c_int, [vp])
 _sig("gm_grasp_workspace_layout", c_int, [c_int, c_int, c_int, c_int, c_int,
                                           ctypes.POINTER(GraspWsLayout)])
 _sig("gm_ns_flops", c_int, [c_int, c_int, c_int, c_int, vp, c_int,
@@ -485,6 +497,28 @@ class GraspState:
         return GraspState(*[t.clone() for t in self.tensors()])
 
 
+def ipc_export(t):
+    """(handle bytes, byte offset) of the device allocation holding tensor t (gm_ipc_export)."""
+    _placed((t,), ("t",))
+    h = IpcHandle()
+    off = c_size_t()
+    _check(lib.gm_ipc_export(_ptr(t), ctypes.byref(h), ctypes.byref(off)), "gm_ipc_export")
+    return bytes(h.bytes), off.value
+
+
+def ipc_open(handle: bytes) -> int:
+    """Device address of the start of another process's exported allocation (gm_ipc_open)."""
+    h = IpcHandle()
+    ctypes.memmove(h.bytes, handle, 64)
+    base = vp()
+    _check(lib.gm_ipc_open(ctypes.byref(h), ctypes.byref(base)), "gm_ipc_open")
+    return base.value
+
+
+def ipc_close(base: int) -> None:
+    _check(lib.gm_ipc_close(vp(base)), "gm_ipc_close")
+
+
 def weight_update(W, O, eta, wd=0.0, skip=None):
     """W <- W - eta (O + wd W) in place (gm_weight_update); O in float32, bfloat16 or
     float16 of W's shape. ``skip`` (optional device int32): one flag for the batch
@@ -592,6 +626,26 @@ class GraspStep:
                                  _DT[out.dtype], _ptr(self.ws), self.ws_bytes, _stream()),
                "gm_grasp_orth")
         return out
+
+    def orth_peers(self, state: GraspState, peer_O, peer_flags, dst_index, dtype=torch.bfloat16):
+        """O = NS(M_t) on the NS input the state update left, stored into every receive
+        buffer of ``peer_O`` (device addresses of [.][m][n] ``dtype`` buffers, this
+        process's or mapped from others) at matrix dst_index[b], with the step's status
+        in ``peer_flags`` (int32 buffers) at the same index (gm_grasp_orth_peers)."""
+        B, m, n = self.B, self.m, self.n
+        state.check(B, m, n, self.k)
+        if not 1 <= len(peer_O) == len(peer_flags) <= 8:
+            raise ValueError("1 to 8 receive buffers, one flag buffer each")
+        if dst_index.dtype != torch.int64 or tuple(dst_index.shape) != (B,):
+            raise ValueError("dst_index: int64 [B] expected")
+        _placed((dst_index,), ("dst_index",))
+        _ws_fits(self.ws, self.ws_bytes)
+        po = (vp * len(peer_O))(*[vp(int(a)) for a in peer_O])
+        pf = (vp * len(peer_flags))(*[vp(int(a)) for a in peer_flags])
+        st = state.c_struct()
+        _check(lib.gm_grasp_orth_peers(B, m, n, ctypes.byref(self.params), ctypes.byref(st), po, pf,
+                                       len(peer_O), _ptr(dst_index), _DT[dtype], _ptr(self.ws),
+                                       self.ws_bytes, _stream()), "gm_grasp_orth_peers")
 
     def direction(self, state: GraspState, G, out=None, dtype=torch.bfloat16):
         """Worked steps 1-5 and O = NS(M_t): the state update, then ``orth``."""

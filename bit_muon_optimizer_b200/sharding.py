@@ -32,6 +32,15 @@ every rank, owners included, applies W <- W - eta (O + wd W) to its own copy
 through ``update(W, O, flags)``: all ranks apply the same O to the same W, so
 they keep identical weights. The step object then provides
 ``direction(G) -> (O, flags)`` instead of updating W.
+
+With ``peer=True`` (and an ``update``) the exchange is fused into the step: each
+rank holds receive buffers for O and the flags of every shape group, mapped into
+every other rank's address space through CUDA IPC, and the owners' last NS
+product stores O straight into all of them (``orth_peers(G, peer_O, peer_flags,
+dst_index)`` of the step object: gm_grasp_orth_peers), peers' over NVLink; a
+stream synchronize and a barrier later every rank applies the update. Receive
+buffers alternate between two sets from one call to the next, so a rank that
+runs ahead never writes a buffer another rank may still be reading.
 """
 
 from __future__ import annotations
@@ -75,12 +84,18 @@ class ShardedStep:
     def __init__(self, shapes: Sequence[tuple[int, int, int]], world: int, rank: int,
                  make_step: Callable[[int, int, list], Callable], cost=ns_cost, group=None,
                  first_index: int = 0, update: Callable | None = None,
-                 update_dtype: torch.dtype = torch.bfloat16):
+                 update_dtype: torch.dtype = torch.bfloat16, peer: bool = False):
         if not 0 <= rank < world:
             raise ValueError(f"rank {rank} outside world {world}")
         self.shapes = [tuple(s) for s in shapes]
         self.world, self.rank, self.group = world, rank, group
         self.update, self.update_dtype = update, update_dtype
+        if peer and update is None:
+            raise ValueError("the fused peer exchange delivers the update direction: give update")
+        self.peer = peer
+        self._bufs: dict = {}      # group -> two (O, flags) PeerBuffers sets
+        self._idx: dict = {}       # group -> device int64 indices of this rank's matrices
+        self._calls = 0
         costs = [cost(m, n) for m, n, count in self.shapes for _ in range(count)]
         flat = lpt_owners(costs, world)
         self.owner: list[list[int]] = []          # owner of matrix i of group g
@@ -107,10 +122,17 @@ class ShardedStep:
     def __call__(self, Ws: Sequence[torch.Tensor], Gs: Sequence[torch.Tensor]) -> None:
         if len(Ws) != len(self.shapes) or len(Gs) != len(self.shapes):
             raise ValueError("one weight and one gradient tensor per shape group")
+        self._call(Ws, Gs)
+        self._calls += 1
+
+    def _call(self, Ws, Gs) -> None:
         for g, ((m, n, count), W, G) in enumerate(zip(self.shapes, Ws, Gs)):
             if tuple(W.shape) != (count, m, n) or tuple(G.shape) != (count, m, n):
                 raise ValueError(f"group {g}: expected [{count}, {m}, {n}] weights and gradients")
             mine = self.owned[g][self.rank]
+            if self.peer:
+                self._exchange_peer(g, m, n, count, W, G)
+                continue
             if self.update is not None:
                 self._exchange_update(g, m, n, count, W, G)
                 continue
@@ -133,6 +155,32 @@ class ShardedStep:
                 if own:
                     W.index_copy_(0, torch.tensor(own, device=W.device), recv[r][:len(own)])
 
+    def _exchange_peer(self, g, m, n, count, W, G):
+        """Owners' NS stores O and flags into every rank's receive buffers; after a
+        barrier every rank applies all of them to its W."""
+        if g not in self._bufs:
+            mk = lambda shape, dt: PeerBuffers(shape, dt, W.device, self.world, self.rank,  # noqa: E731
+                                                self.group)
+            self._bufs[g] = [(mk((count, m, n), self.update_dtype), mk((count,), torch.int32))
+                             for _ in range(2)]
+            self._idx[g] = torch.tensor(self.owned[g][self.rank], dtype=torch.int64, device=W.device)
+        Ob, Fb = self._bufs[g][self._calls & 1]
+        mine = self.owned[g][self.rank]
+        if mine:
+            idx = self._idx[g]
+            self.steps[g].orth_peers(G.index_select(0, idx), Ob.ptrs, Fb.ptrs, idx)
+        if self.world > 1:
+            torch.cuda.current_stream(W.device).synchronize()   # this rank's stores are done
+            dist.barrier(group=self.group)                        # and every other rank's
+        self.update(W, Ob.local, Fb.local)
+
+    def close(self) -> None:
+        """Unmaps the other ranks' receive buffers (every rank calls it)."""
+        for sets in self._bufs.values():
+            for Ob, Fb in sets:
+                Ob.close()
+                Fb.close()
+        self._bufs.clear()
 
     def _exchange_update(self, g, m, n, count, W, G):
         """Owners send (O, flags); every rank applies all of them to its W."""
@@ -164,6 +212,35 @@ class ShardedStep:
         self.update(W, O_all, f_all)
 
 
+class PeerBuffers:
+    """One zeroed device buffer per rank, and on every rank the addresses of all of
+    them: its own, and the other ranks' mapped through CUDA IPC (gm_ipc_export /
+    gm_ipc_open). Collective: every rank constructs it alike."""
+
+    def __init__(self, shape, dtype, device, world: int, rank: int, group=None):
+        from . import gmuon as gm
+        self.local = torch.zeros(shape, dtype=dtype, device=device)
+        self._opened: list[int] = []
+        self.ptrs = [self.local.data_ptr()]
+        if world > 1:
+            handles: list = [None] * world
+            dist.all_gather_object(handles, gm.ipc_export(self.local), group=group)
+            self.ptrs = []
+            for r, (h, off) in enumerate(handles):
+                if r == rank:
+                    self.ptrs.append(self.local.data_ptr())
+                else:
+                    base = gm.ipc_open(h)
+                    self._opened.append(base)
+                    self.ptrs.append(base + off)
+
+    def close(self) -> None:
+        from . import gmuon as gm
+        for base in self._opened:
+            gm.ipc_close(base)
+        self._opened = []
+
+
 def grasp_make_step(k: int, device=None, **params) -> Callable[[int, int, list], Callable]:
     """``make_step`` for the library's GRASP step: each owner batch gets its own
     step object and zero state (its quantized momentum lives on this rank only),
@@ -182,8 +259,13 @@ def grasp_make_step(k: int, device=None, **params) -> Callable[[int, int, list],
             O = step.direction(state, G)
             return O, state.dev_status.expand(B).contiguous()
 
+        def orth_peers(G: torch.Tensor, peer_O, peer_flags, dst_index) -> None:
+            step.state_update(state, G)
+            step.orth_peers(state, peer_O, peer_flags, dst_index)
+
         run.state = state
         run.direction = direction
+        run.orth_peers = orth_peers
         return run
 
     return make

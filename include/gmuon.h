@@ -369,6 +369,41 @@ gm_status gm_grasp_orth(int B, int m, int n, const gm_grasp_params* params,
 gm_status gm_weight_update(int B, int m, int n, float eta, float wd, const void* O, gm_dtype odt,
                            float* W, const int32_t* skip, int skip_stride, gm_stream_t stream);
 
+/*
+ * gm_grasp_orth with O delivered to several receive buffers at once, for a set
+ * split by ownership across the GPUs of a node: the last NS product's epilogue
+ * stores each element of O into every peer_O[r] (r < npeers <= 8: device
+ * pointers, other GPUs' memory mapped through gm_ipc_open included; plain
+ * stores, over NVLink for a peer) at matrix dst_index[b] (device int64 [B];
+ * NULL: b) of that [.][m][n] buffer in odt; then peer_flags[r][dst_index[b]]
+ * (int32) = *dev_status for every r and b. The compute step and the exchange
+ * are one pass: no separate all-gather. When *dev_status is non-zero no O is
+ * written, only the flags. The caller orders the receivers' reads after every
+ * sender's call has completed (e.g. a stream synchronize and a host barrier)
+ * and keeps a receive buffer alive while senders may write it.
+ */
+gm_status gm_grasp_orth_peers(int B, int m, int n, const gm_grasp_params* params,
+                              const gm_grasp_state* state, void* const* peer_O,
+                              int32_t* const* peer_flags, int npeers, const int64_t* dst_index,
+                              gm_dtype odt, void* ws, size_t ws_bytes, gm_stream_t stream);
+
+/*
+ * Device buffers shared between the processes of one node (CUDA IPC), for the
+ * receive buffers of gm_grasp_orth_peers.
+ *  - gm_ipc_export: the handle of the allocation that holds dev_ptr and the
+ *    offset of dev_ptr in it.
+ *  - gm_ipc_open (in another process): maps that allocation, *base its start
+ *    (add the exporter's offset); peer access is enabled on first use.
+ *  - gm_ipc_close: unmaps a base returned by gm_ipc_open.
+ * The exporter keeps the allocation alive until every importer has closed it.
+ */
+typedef struct {
+  unsigned char bytes[64];
+} gm_ipc_handle;
+gm_status gm_ipc_export(const void* dev_ptr, gm_ipc_handle* handle, size_t* offset);
+gm_status gm_ipc_open(const gm_ipc_handle* handle, void** base);
+gm_status gm_ipc_close(void* base);
+
 /* Byte offsets of the stage buffers inside the gm_grasp_step workspace, for
  * inspection by tests: M f32 [B][m][n]; Q f32 [B][n][k]; P, R f32; X the NS
  * input (bf16 or fp16, wide form); scale f32 [B] = 1/(|M|_F + eps). */

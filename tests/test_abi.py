@@ -219,3 +219,24 @@ def test_orth_and_weight_update_argument_errors():
     assert upd(2, 256, 512, 0.02, 0.0, ok, gm.GM_BF16, bad, None, 0, None) == gm.GM_E_ARG
     assert upd(2, 256, 512, 0.02, 0.0, ok, gm.GM_BF16, ok, ok, 2, None) == gm.GM_E_ARG
     assert upd(2, 256, 512, float("nan"), 0.0, ok, gm.GM_BF16, ok, None, 0, None) == gm.GM_E_ARG
+
+
+def test_orth_peers_and_ipc_argument_errors():
+    """gm_grasp_orth_peers and the IPC helpers reject bad arguments on the host."""
+    ok = ctypes.c_void_p(4096)
+    st = gm.GraspStateC(*([4096] * 9))
+    prm = gm.GraspParams(0.95, 0.02, 0.0, 8, 5, 0, None, None, 0, 1e-7, 0)
+    arr = lambda *v: (ctypes.c_void_p * len(v))(*[ctypes.c_void_p(x) for x in v])  # noqa: E731
+    call = lambda po, pf, npeers, odt=gm.GM_BF16, dst=ok: gm.lib.gm_grasp_orth_peers(  # noqa: E731
+        2, 256, 512, ctypes.byref(prm), ctypes.byref(st), po, pf, npeers, dst, odt, ok, 1 << 40, None)
+    assert call(arr(4096), arr(4096), 0) == gm.GM_E_ARG                         # no destination
+    assert call(arr(*[4096] * 9), arr(*[4096] * 9), 9) == gm.GM_E_ARG           # more than 8
+    assert call(arr(4096, 0), arr(4096, 4096), 2) == gm.GM_E_ARG                # a NULL buffer
+    assert call(arr(4096 + 8), arr(4096), 1) == gm.GM_E_ARG                     # misaligned
+    assert call(arr(4096), arr(4096), 1, odt=5) == gm.GM_E_ARG
+    assert call(arr(4096), arr(4096), 1, dst=ctypes.c_void_p(4096 + 4)) == gm.GM_E_ARG
+    h = gm.IpcHandle()
+    off = ctypes.c_size_t()
+    assert gm.lib.gm_ipc_export(None, ctypes.byref(h), ctypes.byref(off)) == gm.GM_E_ARG
+    assert gm.lib.gm_ipc_open(None, None) == gm.GM_E_ARG
+    assert gm.lib.gm_ipc_close(None) == gm.GM_E_ARG
