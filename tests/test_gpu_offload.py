@@ -14,18 +14,19 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-@pytest.mark.parametrize("ns", ["standard", "gram"])
+@pytest.mark.parametrize("ns,gdtype", [("standard", torch.bfloat16), ("gram", torch.bfloat16),
+                                       ("standard", torch.float32)])
 @pytest.mark.parametrize("B,m,n,chunk", [(5, 256, 384, 2), (3, 272, 144, 1), (4, 128, 256, 4)])
-def test_host_streamed_step_equals_the_resident_step(cuda_lib, ns, B, m, n, chunk):
+def test_host_streamed_step_equals_the_resident_step(cuda_lib, ns, gdtype, B, m, n, chunk):
     from bit_muon_optimizer_b200.offload import HostStreamedStep
     gm = cuda_lib
     k = 8
     mode = gm.GM_NS_GRAM if ns == "gram" else gm.GM_NS_STANDARD
     ids = [100 + 3 * b for b in range(B)]
     W0 = WL.random_matrix((B, m, n), 61, std=0.02)
-    grads = [WL.random_matrix((B, m, n), 62 + t, std=1e-3).to(torch.bfloat16) for t in (1, 2, 3)]
-    hs = HostStreamedStep(B, m, n, k, chunk=chunk, device=DEV, matrix_ids=ids, ns=mode, seed=9,
-                          wd=0.1)
+    grads = [WL.random_matrix((B, m, n), 62 + t, std=1e-3).to(gdtype) for t in (1, 2, 3)]
+    hs = HostStreamedStep(B, m, n, k, gdtype=gdtype, chunk=chunk, device=DEV, matrix_ids=ids,
+                          ns=mode, seed=9, wd=0.1)
     Wh = W0.clone().pin_memory()
     ref = gm.GraspStep(B, m, n, k, ns=mode, seed=9, wd=0.1, device=DEV, matrix_ids=ids)
     st = gm.GraspState.zeros(B, m, n, k, DEV)
