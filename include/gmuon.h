@@ -13,7 +13,8 @@
  *
  * Ownership: the caller allocates every buffer (typically torch tensors) and
  * keeps it alive until the stream work completes. The library never
- * allocates or frees device memory and keeps no per-call device state.
+ * allocates or frees device memory (gm_ipc_open only maps another process's
+ * allocation, which gm_ipc_close unmaps) and keeps no per-call device state.
  * Library-wide device state is limited to two file-scope arrays that every
  * GPU loading the library holds: one int32 error word (see
  * gm_device_errors) and the scratch of gm_newton_schulz_noalloc.
