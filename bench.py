@@ -248,7 +248,7 @@ GEMM_TRAFFIC = [
 # valid only for the gm_codec.cu source it was captured on.
 CODEC_INSTR = [
     {"configs": [4], "thread_instr_per_element": 116.03,
-     "source_sha256": "fd2224401ae4389c160824c579386bf3e9a52b77da131c7e9f1587483b3d7a59"},
+     "source_sha256": "c6f4a95d77a721cb4c1eb17c1c8e3a6895f5c6f61c190f4d9992a02fdf1467c7"},
 ]
 
 

@@ -1557,9 +1557,13 @@ __global__ void __launch_bounds__(kRT, 2) k_residual_quant4(
 //                 row and the four row quarters of a column meet in shared memory. A
 //                 second sweep over TMEM turns x into codes q = rint(fp32(x / s) * 7),
 //                 s = min(row max, column max), with the same fl(7 / s) shortcut and
-//                 IEEE fallback as k_residual_quant4, and stores each thread's 8 code
-//                 bytes per chunk. The 8-bit factor codes, scales and step count are
-//                 written as in k_residual_quant4.
+//                 IEEE fallback as k_residual_quant4 (one tie test per 16-element
+//                 run, the rounding on the FMA pipe), and stores each thread's 8 code
+//                 bytes per chunk. The 8-bit codes of P's rows of block row bi are
+//                 written by the block (bi, bi mod nb), those of R's rows of block
+//                 column bj by the block (bj mod mb, bj): one job per block row and
+//                 column, spread over the grid; block (0, 0) writes the scales and
+//                 the step count.
 // Operand tiles are single-buffered: the next block's R (and P) rows load as soon as
 // the product that read them has completed. Every wait is bounded (~2 s of
 // %globaltimer) and gives up at once when another role has aborted; a timeout records
