@@ -9,8 +9,8 @@ re-quantization, Newton-Schulz, weight update) over every matrix of the
 parameter set, with that step's synthetic gradients already resident in HBM.
 The default parameter set is the largest one that fits one GPU: the
 Qwen2.5-7B-shaped set (6.5e9 weight elements), measured one shape group at a
-time (each group batched in one gm_grasp_step call and replayed from CUDA
-graphs); the set's time is the sum over its groups. N > 1 (torchrun): the set
+time (each group batched in gm_grasp_step calls of at most about 1e9 elements,
+replayed from CUDA graphs); the set's time is the sum over its groups. N > 1 (torchrun): the set
 is split by ownership across the ranks (each matrix's step runs on one owner,
 then one NCCL all-gather per shape group gives every rank the updated set:
 strong scaling); the time is the max over ranks.
@@ -308,14 +308,42 @@ def ns_chooser(gm, ns: str):
     return lambda m, n: std
 
 
+# A shape group larger than this many elements is stepped as several library calls on
+# contiguous sub-batches (each matrix's step is independent of its batch, so the
+# results are the same bit for bit): on the 3.8e9-element 56 x 18944 x 3584 group, 4
+# calls of 14 matrices ran both halves of the step 4-6 % faster than one call of 56,
+# at a higher SM clock under the same power cap, with a quarter of the workspace;
+# groups of up to 0.7e9 elements gained nothing from splitting.
+SUB_BATCH_ELEMENTS = 1.0e9
+
+
+def sub_batches(B: int, m: int, n: int) -> int:
+    """Matrices per library call for a group of B m x n matrices."""
+    calls = max(1, -(-B * m * n // int(SUB_BATCH_ELEMENTS)))
+    return -(-B // calls)
+
+
 def build_group(gm, w: WL.Workload, gi: int, nsf, pool: int, dev):
+    from bit_muon_optimizer_b200.offload import chunk_bounds
     g = w.groups[gi]
     B, m, n = g.count, g.m, g.n
     base = w.group_base(gi)
     ids = list(range(base, base + B))
-    step = gm.GraspStep(B, m, n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=nsf(m, n),
-                        seed=w.seed, device=dev, matrix_ids=ids)
+    ns = nsf(m, n)
+    bounds = chunk_bounds(B, sub_batches(B, m, n))
+    sizes = sorted({b - a for a, b in bounds})
+    ws = torch.empty(max(gm.workspace_bytes(gm.GM_OP_GRASP_STEP, c, m, n, w.k, ns) for c in sizes),
+                     dtype=torch.uint8, device=dev)
+    steps = {c: gm.GraspStep(c, m, n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=ns, seed=w.seed,
+                             device=dev, ws=ws, matrix_ids=ids[:c]) for c in sizes}
     st = gm.GraspState.zeros(B, m, n, w.k, dev)
+    status = torch.zeros(len(bounds), dtype=torch.int32, device=dev)
+    subs = []
+    for i, (a, b) in enumerate(bounds):
+        sub_st = gm.GraspState(st.codes4[a:b], st.rscale[a:b], st.cscale[a:b], st.P8[a:b],
+                               st.Pscale[a:b], st.R8[a:b], st.Rscale[a:b],
+                               torch.zeros(1, dtype=torch.int64, device=dev), status[i:i + 1])
+        subs.append((a, b, steps[b - a], sub_st, torch.tensor(ids[a:b], dtype=torch.int64, device=dev)))
     W = torch.empty((B, m, n), dtype=torch.float32, device=dev)
     for b in range(B):
         W[b] = WL.initial_weight(w, base + b, m, n, device=dev)
@@ -325,7 +353,29 @@ def build_group(gm, w: WL.Workload, gi: int, nsf, pool: int, dev):
         for b in range(B):
             WL.gradient(w, base + b, t, m, n, device=dev, out=G[b])
         grads.append(G)
-    return dict(step=step, st=st, W=W, grads=grads, B=B, m=m, n=n, ids=ids, ns=nsf(m, n))
+    return dict(subs=subs, ws=ws, st=st, status=status, W=W, grads=grads, B=B, m=m, n=n, ids=ids,
+                ns=ns)
+
+
+def group_step(g, G) -> None:
+    """One GRASP step of the group (its sub-batches in order) on the current stream."""
+    for a, b, step, st, ids in g["subs"]:
+        step.ids.copy_(ids, non_blocking=True)
+        step(st, g["W"][a:b], G[a:b])
+
+
+def group_halves(g, G, events) -> None:
+    """The same step as its two halves per sub-batch, CUDA events (before the codec
+    half, between the halves, after the NS half) appended to `events`."""
+    for a, b, step, st, ids in g["subs"]:
+        step.ids.copy_(ids, non_blocking=True)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        step.state_update(st, G[a:b])
+        e[1].record()
+        step.apply(st, g["W"][a:b])
+        e[2].record()
+        events.append(e)
 
 
 def our_launches(gm, w: WL.Workload, nsf, groups=None) -> int:
@@ -335,9 +385,10 @@ def our_launches(gm, w: WL.Workload, nsf, groups=None) -> int:
     8-bit one folded in), the NS products, and the zero-padding copy when a
     dimension is not a multiple of 64."""
     launches = 0
-    for (m, n) in (groups if groups is not None else [(g.m, g.n) for g in w.groups]):
+    for (B, m, n) in (groups if groups is not None else [(g.count, g.m, g.n) for g in w.groups]):
         pad = int(min(m, n) % 64 != 0 or max(m, n) % 64 != 0)
-        launches += 9 + gm.ns_flops(nsf(m, n), m, n, w.T)[1] + pad
+        calls = -(-B // sub_batches(B, m, n))
+        launches += calls * (9 + gm.ns_flops(nsf(m, n), m, n, w.T)[1] + pad)
     return launches
 
 
@@ -367,13 +418,13 @@ def time_steps(groups, args, world, local):
     # eager warm-up (also sets kernel attributes), then one graph per gradient slot
     main.wait_stream(torch.cuda.current_stream(dev))
     npool = len(groups[0]["grads"])
-    fork(lambda g: g["step"](g["st"], g["W"], g["grads"][0]))
+    fork(lambda g: group_step(g, g["grads"][0]))
     torch.cuda.synchronize()
     graphs = []
     for t in range(npool):
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=main):
-            fork(lambda g, t=t: g["step"](g["st"], g["W"], g["grads"][t]))
+            fork(lambda g, t=t: group_step(g, g["grads"][t]))
         graphs.append(gr)
     torch.cuda.synchronize()
     with torch.cuda.stream(main):
@@ -395,7 +446,7 @@ def time_steps(groups, args, world, local):
         torch.cuda.synchronize()
         barrier(world)
     ms_step = max_over_ranks(start.elapsed_time(end) / args.steps, world)
-    status = [int(g["st"].dev_status.item()) for g in groups]
+    status = [int(g["status"].abs().max()) for g in groups]
     if any(status):
         raise RuntimeError(f"device status {status}")
     del graphs
@@ -414,17 +465,11 @@ def measure(gm, w, groups, nsf, args, world, local, do_e2e):
     # ---- the step's two halves, each bracketed by CUDA events on the stream
     # that launches it; groups one after another (no overlap between groups)
     nb = max(2, min(args.steps, 5))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nb * len(groups))]
+    evs = []
     with torch.cuda.stream(main):
         for i in range(nb):
-            for j, g in enumerate(groups):
-                e0, e1, e2 = evs[i * len(groups) + j]
-                G = g["grads"][(args.warmup + args.steps + i) % npool]
-                e0.record(main)
-                g["step"].state_update(g["st"], G)
-                e1.record(main)
-                g["step"].apply(g["st"], g["W"])
-                e2.record(main)
+            for g in groups:
+                group_halves(g, g["grads"][(args.warmup + args.steps + i) % npool], evs)
     torch.cuda.synchronize()
     cod_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in evs) / nb
     ns_ms = sum(e1.elapsed_time(e2) for _, e1, e2 in evs) / nb
@@ -437,7 +482,7 @@ def measure(gm, w, groups, nsf, args, world, local, do_e2e):
     codecs = None
     if args.codecs:
         g = groups[0]
-        M = g["step"].stage_M()
+        M = g["subs"][-1][2].stage_M()      # the group's last sub-batch
         codes = torch.empty((g["B"], g["m"], g["n"] // 2), dtype=torch.uint8, device=dev)
         gsc = torch.empty((g["B"], g["m"] * g["n"] // 128), dtype=torch.float32, device=dev)
         Xo = torch.empty_like(M)
@@ -463,8 +508,14 @@ def measure(gm, w, groups, nsf, args, world, local, do_e2e):
     # ---- comparator: the same standard NS chain written with torch.matmul
     # (cuBLAS, bf16, no symmetry) on the same normalised inputs, graph-replayed
     abc = [(3.4445, -4.7750, 2.0315)] * w.T
-    for g in groups:
-        g["Xc"] = g["step"].stage_X().to(torch.bfloat16).clone()
+    for g in groups:                        # one more codec half per sub-batch, untimed
+        g["Xc"] = torch.empty((g["B"], min(g["m"], g["n"]), max(g["m"], g["n"])), dtype=torch.bfloat16,
+                              device=dev)
+        G = g["grads"][0]
+        for a, b, step, st, ids in g["subs"]:
+            step.ids.copy_(ids)
+            step.state_update(st, G[a:b])
+            g["Xc"][a:b].copy_(step.stage_X())
         g["Xw"] = torch.empty_like(g["Xc"])
 
     def cublas_enqueue(g):
@@ -642,7 +693,8 @@ def run_single(gm, w, nsf, args, local):
             "api": "offload.HostStreamedStep per shape group with the weights in pinned host memory "
                    "too: W and G in, the step, W out, in chunks of about 2^25 elements (at most "
                    "B/8 matrices) on three streams; groups one after another, set time = sum"}
-    out["graph"] = ("one CUDA graph per gradient slot, one stream per shape group"
+    out["graph"] = ("one CUDA graph per gradient slot (each group's gm_grasp_step calls on "
+                    "sub-batches of at most about 1e9 elements), one stream per shape group"
                     + ("; shape groups measured one at a time (device memory), set time = sum"
                        if per_group else ""))
     out["pool"] = pool
@@ -724,7 +776,7 @@ def run_sharded(gm, w, nsf, args, world, rank, local):
         mine = len(sh.owned[0][rank])
         owned.append(mine)
         if mine:
-            launches += our_launches(gm, w, nsf, [(g.m, g.n)])
+            launches += our_launches(gm, w, nsf, [(1, g.m, g.n)])   # one call per owned batch
         if update is not None:
             launches += 1                              # k_weight_update on every rank
         torch.cuda.synchronize()

@@ -92,3 +92,18 @@ def test_ns_auto_picks_gram_for_non_square_shapes():
     assert bench.ns_name("auto", 3584, 18944) == "gram"
     assert bench.ns_name("standard", 2048, 768) == "standard"
     assert bench.ns_name("gram", 768, 768) == "gram"
+
+
+def test_sub_batches_split_only_the_largest_groups():
+    """Groups above about 1e9 elements are stepped as several calls of equal size
+    (at most one matrix apart); smaller groups as one call."""
+    import bench
+    assert bench.sub_batches(56, 18944, 3584) == 14      # 3.8e9 elements: 4 calls
+    assert bench.sub_batches(28, 3584, 18944) == 14      # 1.9e9: 2 calls
+    assert bench.sub_batches(56, 3584, 3584) == 56       # 0.72e9: one call
+    assert bench.sub_batches(44, 5632, 2048) == 44
+    assert bench.sub_batches(1, 65536, 65536) == 1       # one matrix above the limit: one call
+    for B, m, n in ((56, 18944, 3584), (57, 18944, 3584), (3, 40000, 40000)):
+        c = bench.sub_batches(B, m, n)
+        calls = -(-B // c)
+        assert 1 <= c <= B and (calls == 1 or c == 1 or c * m * n <= bench.SUB_BATCH_ELEMENTS * 1.5)
