@@ -917,21 +917,33 @@ def run_profile(args):
         g = w.groups[gi]
         B = args.batch or g.count
         base = w.group_base(gi)
-        step = gm.GraspStep(B, g.m, g.n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=nsf(g.m, g.n),
-                            seed=w.seed, device=dev, matrix_ids=list(range(base, base + B)))
+        # the bench's sub-batch calls, unless a batch size is given
+        c = B if args.batch else sub_batches(B, g.m, g.n)
+        step = gm.GraspStep(c, g.m, g.n, w.k, mu=w.mu, eta=w.eta, wd=w.wd, T=w.T, ns=nsf(g.m, g.n),
+                            seed=w.seed, device=dev, matrix_ids=list(range(base, base + c)))
         st = gm.GraspState.zeros(B, g.m, g.n, w.k, dev)
         W = torch.empty((B, g.m, g.n), dtype=torch.float32, device=dev)
         G = torch.empty((B, g.m, g.n), dtype=w.gdtype, device=dev)
         for b in range(B):
             W[b] = WL.initial_weight(w, base + b, g.m, g.n, device=dev)
             WL.gradient(w, base + b, 1, g.m, g.n, device=dev, out=G[b])
+        subs = [(a, min(B, a + c)) for a in range(0, B, c)]
+        sts = [gm.GraspState(st.codes4[a:e], st.rscale[a:e], st.cscale[a:e], st.P8[a:e], st.Pscale[a:e],
+                             st.R8[a:e], st.Rscale[a:e], torch.zeros(1, dtype=torch.int64, device=dev),
+                             torch.zeros(1, dtype=torch.int32, device=dev)) for a, e in subs]
+        if any(e - a != c for a, e in subs):
+            raise ValueError("--profile: the sub-batches must be of equal size")
+        ids = torch.arange(base, base + B, dtype=torch.int64, device=dev)
         for _ in range(args.profile):
-            step(st, W, G)
+            for (a, e), sst in zip(subs, sts):
+                step.ids.copy_(ids[a:e])
+                step(sst, W[a:e], G[a:e])
         torch.cuda.synchronize()
-        if int(st.dev_status.item()):
-            raise RuntimeError(f"device status {int(st.dev_status.item())}")
-        print(f"profile: group {gi} ({g.m} x {g.n} x {B}): {args.profile} steps", flush=True)
-        del step, st, W, G
+        bad = [int(s.dev_status.item()) for s in sts]
+        if any(bad):
+            raise RuntimeError(f"device status {bad}")
+        print(f"profile: group {gi} ({g.m} x {g.n} x {B}, calls of {c}): {args.profile} steps", flush=True)
+        del step, st, sts, W, G
         torch.cuda.empty_cache()
 
 
