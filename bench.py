@@ -474,7 +474,8 @@ def measure(gm, w, groups, nsf, args, world, local, do_e2e):
     cod_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in evs) / nb
     ns_ms = sum(e1.elapsed_time(e2) for _, e1, e2 in evs) / nb
     ns_flops = sum(gm.ns_flops(nsf(g["m"], g["n"]), g["m"], g["n"], w.T)[0] * g["B"] for g in groups)
-    ns_launches = sum(gm.ns_flops(nsf(g["m"], g["n"]), g["m"], g["n"], w.T)[1] for g in groups)
+    ns_launches = sum(gm.ns_flops(nsf(g["m"], g["n"]), g["m"], g["n"], w.T)[1] * len(g["subs"])
+                      for g in groups)
 
     # ---- the standalone 4-bit codecs of the same entry points a user calls
     # (4bit-Muon-base group codec, MuonQ's mu-law codec), on the first group's
@@ -884,8 +885,8 @@ def run_ours(args, world, rank, local):
         "codec": {"gbs": codec_gbs, "peak_gbs": hbm, "frac": codec_gbs / hbm, "ms": r["cod_ms"],
                   "bytes": r["codec_bytes"],
                   "kernels": "the codec half of the step (gm_grasp_state_update: 9 kernels per "
-                             "group), CUDA events around it; algorithmic bytes G + old and new "
-                             "codes and scales + the 16-bit NS input",
+                             "call), CUDA events around each call; algorithmic bytes G + old and "
+                             "new codes and scales + the 16-bit NS input",
                   "issue": codec_issue(args.config, elements, r["cod_ms"], r["clocks"])},
         "step_roofline": {"ms": t_roof, "frac": t_roof / r["ms_step"], "flops": step_flops,
                           "bytes": step_bytes},
