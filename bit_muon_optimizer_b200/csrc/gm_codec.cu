@@ -70,10 +70,13 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
 // of two such pairs summed as lo*hi + hi*lo + hi*hi reach fp32-level accuracy
 // (the 3xTF32 emulation); the small terms go first.
 __device__ __forceinline__ uint32_t tf32_hi(float x) { return __float_as_uint(x) & 0xFFFFE000u; }
+// The remainder's rounding to tf32 is round-to-nearest with ties away from zero on
+// the magnitude (the rna rounding of the tf32 conversion): adding half of the last
+// kept bit to the sign-magnitude pattern and clearing the 13 dropped bits gives it
+// for every finite value (a carry out of the mantissa rounds up into the next
+// binade), in two integer operations where the conversion instruction costs about four.
 __device__ __forceinline__ uint32_t tf32_lo(float x, uint32_t hi) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(__fsub_rn(x, __uint_as_float(hi))));
-  return r;
+  return (__float_as_uint(__fsub_rn(x, __uint_as_float(hi))) + 0x1000u) & 0xFFFFE000u;
 }
 
 // x = p0 + p1 + p2 with every part a bf16: exact for normal fp32 (3 x 8
