@@ -247,8 +247,8 @@ GEMM_TRAFFIC = [
 # passes (`smsp__inst_executed.sum` x 32 / elements on the 18944 x 3584 shape);
 # valid only for the gm_codec.cu source it was captured on.
 CODEC_INSTR = [
-    {"configs": [4], "thread_instr_per_element": 116.03,
-     "source_sha256": "c6f4a95d77a721cb4c1eb17c1c8e3a6895f5c6f61c190f4d9992a02fdf1467c7"},
+    {"configs": [4], "thread_instr_per_element": 112.69,
+     "source_sha256": "9b557427a1d8be3afa17d4d052f12ff82014a2ee157e45c90db2948a57d7daef"},
 ]
 
 
