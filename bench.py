@@ -312,8 +312,10 @@ def ns_chooser(gm, ns: str):
 # contiguous sub-batches (each matrix's step is independent of its batch, so the
 # results are the same bit for bit): on the 3.8e9-element 56 x 18944 x 3584 group, 4
 # calls of 14 matrices ran both halves of the step 4-6 % faster than one call of 56,
-# at a higher SM clock under the same power cap, with a quarter of the workspace;
-# groups of up to 0.7e9 elements gained nothing from splitting.
+# at a higher SM clock under the same power cap, with a quarter of the workspace; the
+# 0.72e9-element 56 x 3584^2 group gained 1-2 % from splitting and the 0.5e9-element
+# 44 x 5632 x 2048 group nothing (15 % less in graph replays), so splitting starts above
+# 1e9.
 SUB_BATCH_ELEMENTS = 1.0e9
 
 
