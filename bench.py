@@ -308,21 +308,11 @@ def ns_chooser(gm, ns: str):
     return lambda m, n: std
 
 
-# A shape group larger than this many elements is stepped as several library calls on
-# contiguous sub-batches (each matrix's step is independent of its batch, so the
-# results are the same bit for bit): on the 3.8e9-element 56 x 18944 x 3584 group, 4
-# calls of 14 matrices ran both halves of the step 4-6 % faster than one call of 56,
-# at a higher SM clock under the same power cap, with a quarter of the workspace; the
-# 0.72e9-element 56 x 3584^2 group gained 1-2 % from splitting and the 0.5e9-element
-# 44 x 5632 x 2048 group nothing (15 % less in graph replays), so splitting starts above
-# 1e9.
-SUB_BATCH_ELEMENTS = 1.0e9
-
-
 def sub_batches(B: int, m: int, n: int) -> int:
-    """Matrices per library call for a group of B m x n matrices."""
-    calls = max(1, -(-B * m * n // int(SUB_BATCH_ELEMENTS)))
-    return -(-B // calls)
+    """Matrices per library call for a group of B m x n matrices (offload.sub_batch_size:
+    calls of at most about 1e9 elements)."""
+    from bit_muon_optimizer_b200.offload import sub_batch_size
+    return sub_batch_size(B, m, n)
 
 
 def build_group(gm, w: WL.Workload, gi: int, nsf, pool: int, dev):
@@ -779,7 +769,7 @@ def run_sharded(gm, w, nsf, args, world, rank, local):
         mine = len(sh.owned[0][rank])
         owned.append(mine)
         if mine:
-            launches += our_launches(gm, w, nsf, [(1, g.m, g.n)])   # one call per owned batch
+            launches += our_launches(gm, w, nsf, [(mine, g.m, g.n)])   # the owner's sub-batch calls
         if update is not None:
             launches += 1                              # k_weight_update on every rank
         torch.cuda.synchronize()

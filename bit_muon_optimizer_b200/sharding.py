@@ -241,27 +241,79 @@ class PeerBuffers:
         self._opened = []
 
 
-def grasp_make_step(k: int, device=None, **params) -> Callable[[int, int, list], Callable]:
+def grasp_make_step(k: int, device=None, sub_batch_elements: float | None = None,
+                    **params) -> Callable[[int, int, list], Callable]:
     """``make_step`` for the library's GRASP step: each owner batch gets its own
     step object and zero state (its quantized momentum lives on this rank only),
-    with the batch's set indices as the step's matrix ids."""
+    with the batch's set indices as the step's matrix ids. A batch above
+    ``sub_batch_elements`` (default: offload.SUB_BATCH_ELEMENTS) is stepped as
+    several library calls on contiguous sub-batches sharing one workspace, the
+    same results bit for bit; ``state`` then carries the first sub-batch's step
+    count and the first non-zero sub-batch status after every call."""
     from . import gmuon as gm
+    from .offload import SUB_BATCH_ELEMENTS, chunk_bounds, sub_batch_size
+
+    limit = SUB_BATCH_ELEMENTS if sub_batch_elements is None else sub_batch_elements
 
     def make(m: int, n: int, ids: list):
         B = len(ids)
-        step = gm.GraspStep(B, m, n, k, device=device, matrix_ids=ids, **params)
         state = gm.GraspState.zeros(B, m, n, k, device)
+        bounds = chunk_bounds(B, sub_batch_size(B, m, n, limit))
+        if len(bounds) == 1:
+            step = gm.GraspStep(B, m, n, k, device=device, matrix_ids=ids, **params)
 
-        def run(W: torch.Tensor, G: torch.Tensor) -> None:
-            step(state, W, G)
+            def run(W: torch.Tensor, G: torch.Tensor) -> None:
+                step(state, W, G)
 
-        def direction(G: torch.Tensor):
-            O = step.direction(state, G)
-            return O, state.dev_status.expand(B).contiguous()
+            def direction(G: torch.Tensor):
+                O = step.direction(state, G)
+                return O, state.dev_status.expand(B).contiguous()
 
-        def orth_peers(G: torch.Tensor, peer_O, peer_flags, dst_index) -> None:
-            step.state_update(state, G)
-            step.orth_peers(state, peer_O, peer_flags, dst_index)
+            def orth_peers(G: torch.Tensor, peer_O, peer_flags, dst_index) -> None:
+                step.state_update(state, G)
+                step.orth_peers(state, peer_O, peer_flags, dst_index)
+        else:
+            sizes = sorted({e - a for a, e in bounds})
+            ns = params.get("ns", gm.GM_NS_STANDARD)
+            ws = torch.empty(max(gm.workspace_bytes(gm.GM_OP_GRASP_STEP, c, m, n, k, ns) for c in sizes),
+                             dtype=torch.uint8, device=device)
+            steps = {c: gm.GraspStep(c, m, n, k, device=device, ws=ws, matrix_ids=ids[:c], **params)
+                     for c in sizes}
+            status = torch.zeros(len(bounds), dtype=torch.int32, device=device)
+            subs = []
+            for i, (a, e) in enumerate(bounds):
+                st = gm.GraspState(state.codes4[a:e], state.rscale[a:e], state.cscale[a:e],
+                                   state.P8[a:e], state.Pscale[a:e], state.R8[a:e], state.Rscale[a:e],
+                                   torch.zeros(1, dtype=torch.int64, device=device), status[i:i + 1])
+                subs.append((a, e, steps[e - a], st,
+                             torch.tensor(ids[a:e], dtype=torch.int64, device=device)))
+            counts = torch.tensor([e - a for a, e in bounds], device=device)
+
+            def settle() -> None:
+                """The batch's step count and first non-zero status into ``state``."""
+                state.step.copy_(subs[0][3].step)
+                first = (status != 0).to(torch.int32).argmax()   # 0 when all are clean
+                state.dev_status.copy_(status.index_select(0, first.view(1)))
+
+            def each(fn) -> None:
+                for a, e, stp, st, sid in subs:
+                    stp.ids.copy_(sid, non_blocking=True)
+                    fn(a, e, stp, st)
+                settle()
+
+            def run(W: torch.Tensor, G: torch.Tensor) -> None:
+                each(lambda a, e, stp, st: stp(st, W[a:e], G[a:e]))
+
+            def direction(G: torch.Tensor):
+                O = torch.empty((B, m, n), dtype=torch.bfloat16, device=device)
+                each(lambda a, e, stp, st: stp.direction(st, G[a:e], out=O[a:e]))
+                return O, status.repeat_interleave(counts, output_size=B)
+
+            def orth_peers(G: torch.Tensor, peer_O, peer_flags, dst_index) -> None:
+                def one(a, e, stp, st):
+                    stp.state_update(st, G[a:e])
+                    stp.orth_peers(st, peer_O, peer_flags, dst_index[a:e])
+                each(one)
 
         run.state = state
         run.direction = direction

@@ -150,3 +150,51 @@ def test_sharded_step_with_update_exchange_on_one_rank(cuda_lib):
         for a, b in zip(mine.tensors(), st.tensors()):
             assert torch.equal(a, b)
         assert (Ws[g] - W).abs().max().item() <= 2 * 2 * eta * 2.0 ** -9 + 1e-6
+
+
+def test_sharded_owner_step_in_sub_batches_equals_one_call(cuda_lib):
+    """grasp_make_step with a small sub-batch limit steps an owner batch as several
+    library calls (here of 2, 2 and 1 matrices): the weights, the direction O with
+    its flags, the peer stores and the state are bit for bit those of the one-call
+    step, and the batch state carries the step count and a sub-batch's status."""
+    from bit_muon_optimizer_b200 import sharding as S
+    gm = cuda_lib
+    k, B, m, n = 8, 5, 256, 384
+    ids = [3, 4, 5, 6, 7]
+    one = S.grasp_make_step(k, torch.device(DEV), eta=0.02, wd=0.1, seed=5)(m, n, ids)
+    split = S.grasp_make_step(k, torch.device(DEV), sub_batch_elements=2 * m * n, eta=0.02, wd=0.1,
+                              seed=5)(m, n, ids)
+    W1 = WL.random_matrix((B, m, n), 31, std=0.02).to(DEV)
+    W2 = W1.clone()
+    for t in (1, 2):
+        G = _outlier(B, m, n, 60 + t, dtype=torch.bfloat16).to(DEV)
+        one(W1, G)
+        split(W2, G)
+    torch.cuda.synchronize()
+    assert torch.equal(W1, W2)
+    for a, b in zip(one.state.tensors(), split.state.tensors()):
+        assert torch.equal(a, b)
+    assert int(split.state.step.item()) == 2
+    G = _outlier(B, m, n, 63, dtype=torch.bfloat16).to(DEV)
+    O1, f1 = one.direction(G)
+    O2, f2 = split.direction(G)
+    torch.cuda.synchronize()
+    assert torch.equal(O1, O2) and torch.equal(f1, f2) and not f2.any()
+    dst = torch.tensor([9, 1, 6, 0, 4], dtype=torch.int64, device=DEV)
+    bufs = [torch.zeros((10, m, n), dtype=torch.bfloat16, device=DEV) for _ in range(2)]
+    flags = [torch.full((10,), -1, dtype=torch.int32, device=DEV) for _ in range(2)]
+    G = _outlier(B, m, n, 64, dtype=torch.bfloat16).to(DEV)
+    one.orth_peers(G, [bufs[0].data_ptr()], [flags[0].data_ptr()], dst)
+    split.orth_peers(G, [bufs[1].data_ptr()], [flags[1].data_ptr()], dst)
+    torch.cuda.synchronize()
+    assert torch.equal(bufs[0], bufs[1]) and torch.equal(flags[0], flags[1])
+    for a, b in zip(one.state.tensors(), split.state.tensors()):
+        assert torch.equal(a, b)
+    # a non-finite gradient in the second sub-batch: the batch status says so, and
+    # the direction's flags mark that sub-batch's matrices
+    G = _outlier(B, m, n, 65, dtype=torch.bfloat16).to(DEV)
+    G[2, 5, 7] = float("nan")
+    O2, f2 = split.direction(G)
+    torch.cuda.synchronize()
+    assert f2.tolist()[2:4] == [gm.GM_E_NONFINITE] * 2 and f2.tolist()[:2] == [0, 0] and f2.tolist()[4] == 0
+    assert int(split.state.dev_status.item()) == gm.GM_E_NONFINITE
