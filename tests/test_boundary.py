@@ -171,3 +171,19 @@ def test_offload_chunk_bounds():
     from bit_muon_optimizer_b200.offload import default_chunk
     assert default_chunk(56, 18944, 3584) == 1 and default_chunk(56, 3584, 3584) == 3
     assert default_chunk(48, 768, 768) == 6 and default_chunk(1, 256, 512) == 1
+
+
+def test_offload_sub_batch_size():
+    """offload.sub_batch_size: the fewest calls of at most `limit` elements (one
+    matrix per call at least), as equal as the count allows."""
+    from bit_muon_optimizer_b200.offload import sub_batch_size
+    assert sub_batch_size(56, 18944, 3584) == 14 and sub_batch_size(56, 3584, 3584) == 56
+    assert sub_batch_size(5, 256, 384, limit=2 * 256 * 384) == 2
+    assert sub_batch_size(3, 100, 100, limit=1) == 1
+    for B in range(1, 40):
+        for limit in (1, 3, 7, 10, 64):
+            c = sub_batch_size(B, 1, 1, limit=limit)
+            calls = -(-B // c)
+            assert c <= max(1, limit) and calls == -(-B // limit) or (limit >= B and c == B)
+    with pytest.raises(ValueError):
+        sub_batch_size(0, 16, 16)
