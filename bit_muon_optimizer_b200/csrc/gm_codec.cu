@@ -1026,8 +1026,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_backproject(int m, int n, int k
                                                               double* __restrict__ Rpart,
                                                               const int32_t* skip) {
   if (skip && *skip) return;
-  constexpr int NL = KP / 8, CH = 128, XS = 40;
-  __shared__ __align__(16) uint16_t Xt[8][32][XS];   // per-warp transpose tile [col][row]
+  // per-warp transpose tile [col][row]; rows of 36 halves (72 B): the 2-byte stores
+  // of a warp (8 columns 4 apart) fall on 2-way shared banks, the 8-byte row reads
+  // on distinct ones
+  constexpr int NL = KP / 8, CH = 128, XS = 36;
+  __shared__ __align__(16) uint16_t Xt[8][32][XS];
   __shared__ float redR[64][KP + 1];
   extern __shared__ __align__(16) float4 Ms[];       // [stage][warp][slot][lane]
   const int cbk = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
@@ -1149,10 +1152,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_backproject(int m, int n, int k
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             if (i0 + 16 * q < m) {   // m % 16 == 0: 16-row runs are all in or all out
-              const uint4* src = reinterpret_cast<const uint4*>(&Xt[warp][lane][16 * q]);
+              const uint2* src = reinterpret_cast<const uint2*>(&Xt[warp][lane][16 * q]);
               uint4* dst = reinterpret_cast<uint4*>(Xb + (long long)(c0 + lane) * m + i0 + 16 * q);
-              dst[0] = src[0];
-              dst[1] = src[1];
+              const uint2 a = src[0], b2 = src[1], c = src[2], d = src[3];
+              dst[0] = make_uint4(a.x, a.y, b2.x, b2.y);
+              dst[1] = make_uint4(c.x, c.y, d.x, d.y);
             }
           }
         }
