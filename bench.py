@@ -248,7 +248,7 @@ GEMM_TRAFFIC = [
 # valid only for the gm_codec.cu source it was captured on.
 CODEC_INSTR = [
     {"configs": [4], "thread_instr_per_element": 112.69,
-     "source_sha256": "9b557427a1d8be3afa17d4d052f12ff82014a2ee157e45c90db2948a57d7daef"},
+     "source_sha256": "214c383857469e9b96f3dcc4823d1632f9ee13bd46ff8f58043e62e9737de36d"},
 ]
 
 
